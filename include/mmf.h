@@ -1,0 +1,235 @@
+/*
+ * mmf.h -- C ABI of the B200 (sm_100a) HGRNBit block forward library (libmmf.so).
+ *
+ * What it computes. The MatMul-free language model replaces every dense projection with a
+ * FusedBitLinear and replaces attention with a gated linear recurrence:
+ *   - FusedBitLinear: RMSNorm (eps 1e-08), per-token absmax INT8 activation quantisation,
+ *     ternary {-1, 0, +1} weights by round-to-nearest of W / mean|W|, an exact integer product
+ *     and a rescale.  Sources: nightvoyager.top "MatMul-Free LLM" report, innovations table
+ *     (ternary weight_quant) and reusable-patterns list (RMSNorm fused with INT8 quantisation);
+ *     hysenlabs.com, "HGRNBitBlock structure" (i/f/g/o_proj, gate_proj, down_proj are each a
+ *     FusedBitLinear with an RMSNorm of eps=1e-08).
+ *   - HGRN recurrence h_t = f_t * h_{t-1} + i_t per channel, O(T*D) (nightvoyager.top, innovations
+ *     table), closed by g_norm = RMSNorm(h) * SiLU(g) (FusedRMSNormSwishGate, hysenlabs.com block
+ *     structure) and an MLP gate_proj -> SiLU gate -> down_proj whose gate_proj is twice as wide
+ *     as down_proj's input (11264 vs 5632 at hidden 2048, same section).
+ *
+ * Conventions shared by every call.
+ *   Memory:   every pointer argument is DEVICE memory unless its comment says host. The caller
+ *             owns all buffers and streams; the library allocates nothing. Calls that need
+ *             scratch take a caller buffer `ws` of at least mmf_workspace_bytes(...) bytes,
+ *             aligned to 256 bytes, which must not be used by anything else until the stream has
+ *             passed the call.
+ *   Streams:  every compute call only enqueues work on `stream` (0 = legacy default stream) and
+ *             returns before it runs.
+ *   Layouts:  activations are row-major [rows][features]; weights follow PyTorch's Linear layout
+ *             [out_features N][in_features K], y = x W^T.
+ *   Dtypes:   MMF_F32 or MMF_BF16 for activations; reductions, the recurrence and epilogues run in
+ *             float32 whatever the storage type; integer products are exact int32.
+ *   Errors:   arguments are validated on the host before anything is enqueued; a bad argument
+ *             returns MMF_ERR_INVALID_ARG (or MMF_ERR_UNSUPPORTED / MMF_ERR_WORKSPACE) and enqueues
+ *             nothing. A failed launch returns MMF_ERR_CUDA. Every wait inside a kernel is bounded:
+ *             when one runs out the kernel records MMF_ERR_TIMEOUT in a device flag, drains its own
+ *             in-flight copies, releases its tensor memory and returns; mmf_sync_status() reports
+ *             and clears that flag. There is no fallback path: an unsupported case is an error.
+ *             mmf_last_error() gives a one-line description of the last failure on this thread.
+ *   Alignment: device pointers must be 16-byte aligned.
+ *
+ * Packed ternary format (this library's own; the pages fix only "ternary codes plus a scale").
+ *   One weight matrix [N][K] is stored as u32 words codes[N][mmf_packed_row_words(K)] plus one
+ *   float32 scale s = max(mean|W|, 1e-5). A row holds 16 codes per word and is padded with zero
+ *   codes to a multiple of 64 codes, so every row starts on a 16-byte boundary. Column
+ *   k = 16*w + 4*quad + lane (quad, lane in 0..3) sits in word w at bit
+ *   16*(quad >> 1) + 2*(quad & 1) + 4*lane as a two's-complement 2-bit field: 00 = 0, 01 = +1,
+ *   11 = -1 (10 is never written). This puts the four codes of one quad in the low two bits of
+ *   the four nibbles of one 16-bit half, so a byte permute expands four codes to four int8 lanes.
+ */
+#ifndef MMF_H_
+#define MMF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* mmf_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  MMF_OK = 0,
+  MMF_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or dtype */
+  MMF_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve (e.g. no sm_100a device) */
+  MMF_ERR_WORKSPACE = 3,   /* ws smaller than mmf_workspace_bytes() or misaligned */
+  MMF_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
+  MMF_ERR_TIMEOUT = 5      /* a bounded in-kernel wait ran out (reported by mmf_sync_status) */
+} mmf_status;
+
+typedef enum { MMF_F32 = 0, MMF_BF16 = 1 } mmf_dtype;
+
+/* Workspace queries: which call the scratch is for. */
+typedef enum {
+  MMF_OP_PACK = 0,      /* mmf_pack_ternary: m = n*k elements                     */
+  MMF_OP_BITLINEAR = 1, /* mmf_bitlinear_fwd: m rows, d = K, inner = N            */
+  MMF_OP_BLOCK = 2,     /* mmf_block_fwd: m = b*t tokens, d, inner                */
+  MMF_OP_DECODE = 3,    /* mmf_decode_step: m = b, d, inner                       */
+  MMF_OP_STACK = 4      /* mmf_stack_fwd: m = b*t tokens, d, inner, n_layers      */
+} mmf_op;
+
+/* A packed ternary weight (device pointers). */
+typedef struct {
+  const uint32_t* codes; /* [n][mmf_packed_row_words(k)] u32, format above */
+  const float* scale;    /* 1 float: s = max(mean|W|, 1e-5)                   */
+  int32_t n;             /* out_features */
+  int32_t k;             /* in_features  */
+} mmf_ternary;
+
+/* One HGRNBit block (hysenlabs.com block structure). Gains are device float32 vectors:
+ * nw_i/f/g/o/gate have d entries, nw_down has `inner`, gnorm_w has d. The GLU reading:
+ * gate_proj rows [0, inner) are the SiLU gate, rows [inner, 2*inner) the linear "up" half. */
+typedef struct {
+  int32_t d;     /* hidden size */
+  int32_t inner; /* MLP inner size I; gate_proj is [2I][d], down_proj is [d][I] */
+  float eps;     /* RMSNorm eps of every norm in the block (1e-8) */
+  const float *nw_i, *nw_f, *nw_g, *nw_o, *nw_gate, *nw_down, *gnorm_w;
+  mmf_ternary i, f, g, o, gate, down;
+} mmf_block_weights;
+
+/* ---- sizes ---------------------------------------------------------------------------------- */
+
+/* u32 words in one packed row of k codes: 4 * ceil(k / 64). */
+int32_t mmf_packed_row_words(int32_t k);
+/* u32 words of a packed [n][k] matrix: n * mmf_packed_row_words(k). */
+size_t mmf_packed_words(int32_t n, int32_t k);
+/* Scratch bytes that `op` needs for the given sizes (0 if none). */
+size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32_t n_layers);
+
+/* ---- calls ---------------------------------------------------------------------------------- */
+
+/* Ternarise and pack one weight matrix (weight_quant, nightvoyager.top innovations table:
+ * round-to-nearest onto {-1, 0, +1}).
+ *   w          [n][k] MMF_F32 or MMF_BF16 latent weights.
+ *   codes_out  [n][mmf_packed_row_words(k)] u32, written entirely (padding codes are 0).
+ *   scale_out  1 float: s = max(mean|W|, 1e-5), with mean|W| summed in float64.
+ *   Codes are t = clamp(rint(w / s), -1, 1) with the division in float32 (IEEE, ties to even).
+ *   ws >= mmf_workspace_bytes(MMF_OP_PACK, n*k, 0, 0, 0). Deterministic. */
+mmf_status mmf_pack_ternary(const void* w, mmf_dtype w_dtype, int32_t n, int32_t k,
+                            uint32_t* codes_out, float* scale_out, void* ws, size_t ws_bytes,
+                            mmf_stream_t stream);
+
+/* One FusedBitLinear, y = BitLinear(x) (nightvoyager.top reusable patterns; hysenlabs.com block
+ * structure):
+ *   r = x / sqrt(mean(x^2) + eps) * norm_w              (eps = 1e-8)
+ *   a = max(max|r|, 1e-5);  q = clamp(rint(r * (127/a)), -127, 127)   (int8, float32 decision)
+ *   acc[m][n] = sum_k q[m][k] * t[n][k]                 (exact int32)
+ *   y[m][n] = acc * (a/127) * s
+ *   x       [m][w->k] x_dtype.    norm_w [w->k] float32, or NULL for a unit gain.
+ *   y       [m][w->n] y_dtype.
+ *   q_dbg   optional [m][w->k] int8: the activation codes.
+ *   deq_dbg optional [m] float32: a/127 per row.
+ *   acc_dbg optional [m][w->n] int32: the integer accumulators.
+ *   ws >= mmf_workspace_bytes(MMF_OP_BITLINEAR, m, w->k, w->n, 0).  m = 0 is a no-op. */
+mmf_status mmf_bitlinear_fwd(const void* x, mmf_dtype x_dtype, int64_t m, const float* norm_w,
+                             const mmf_ternary* w, void* y, mmf_dtype y_dtype, int8_t* q_dbg,
+                             float* deq_dbg, int32_t* acc_dbg, void* ws, size_t ws_bytes,
+                             mmf_stream_t stream);
+
+/* HGRN gated linear recurrence with its gates fused in (nightvoyager.top innovations table):
+ *   f = sigmoid(zf);  i = SiLU(zi) * (1 - f);  h_t = f_t * h_{t-1} + i_t,  h_{-1} = h0 or 0.
+ *   zf, zi  [b][t][z_stride] z_dtype, channels [0, d) of each row are used (z_stride >= d).
+ *   h0      optional [b][d] float32.
+ *   h_out   [b][t][d] h_dtype.   h_last optional [b][d] float32 (= h at the last step).
+ *   Channel-parallel over b*d, chunk-parallel over t with float32 carries. */
+mmf_status mmf_hgrn_scan(const void* zf, const void* zi, mmf_dtype z_dtype, int64_t z_stride,
+                         int32_t b, int64_t t, int32_t d, const float* h0, void* h_out,
+                         mmf_dtype h_dtype, float* h_last, mmf_stream_t stream);
+
+/* One HGRNBit block forward over b sequences of t tokens (hysenlabs.com block structure):
+ *   zi, zf, g = i/f/g_proj(x);  h = scan(f = sigmoid(zf), i = SiLU(zi)(1-f));
+ *   u = RMSNorm(h) * gnorm_w * SiLU(g);  x1 = x + o_proj(u);
+ *   [a | c] = gate_proj(x1);  y = x1 + down_proj(SiLU(a) * c).
+ *   x, y    [b][t][d] dtype (may not alias).   h0 optional [b][d] float32 initial state.
+ *   h_last  optional [b][d] float32 final state.
+ *   ws >= mmf_workspace_bytes(MMF_OP_BLOCK, b*t, d, inner, 1). */
+mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dtype, int32_t b,
+                         int64_t t, const float* h0, void* y, float* h_last, void* ws,
+                         size_t ws_bytes, mmf_stream_t stream);
+
+/* One autoregressive step through n_layers blocks: the block above with t = 1 and the
+ * recurrent state carried per layer.
+ *   layers  HOST array of n_layers block descriptors (device pointers inside).
+ *   x       [b][d] dtype: hidden state of the current token entering layer 0.
+ *   state   [n_layers][b][d] float32, read and overwritten in place.
+ *   y       [b][d] dtype: hidden state leaving the last layer (may not alias x).
+ *   ws >= mmf_workspace_bytes(MMF_OP_DECODE, b, d, inner, n_layers). */
+mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
+                           mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
+                           size_t ws_bytes, mmf_stream_t stream);
+
+/* Token embedding gather: out[r] = table[ids[r]] for r < m.
+ *   ids [m] int32. Ids live on the device and are not checked on the host; an id outside
+ *   [0, vocab) yields a zero row (never an out-of-bounds read).
+ *   table [vocab][d] dtype; out [m][d] dtype. */
+mmf_status mmf_embed_gather(const int32_t* ids, int64_t m, const void* table, mmf_dtype dtype,
+                            int32_t vocab, int32_t d, void* out, mmf_stream_t stream);
+
+/* Prefill forward of an HGRNBitModel block stack (hysenlabs.com: HGRNBitModel = embedding + a
+ * stack of HGRNBitBlock): embedding gather, then the n_layers blocks in order.
+ *   layers  HOST array of n_layers block descriptors.  ids [b][t] int32.
+ *   table   [vocab][d] dtype.   y [b][t][d] dtype.
+ *   h_last  optional [n_layers][b][d] float32 final recurrent state of every layer.
+ *   ws >= mmf_workspace_bytes(MMF_OP_STACK, b*t, d, inner, n_layers). */
+mmf_status mmf_stack_fwd(const mmf_block_weights* layers, int32_t n_layers, const int32_t* ids,
+                         int32_t b, int64_t t, const void* table, int32_t vocab, mmf_dtype dtype,
+                         void* y, float* h_last, void* ws, size_t ws_bytes, mmf_stream_t stream);
+
+/* ---- status, errors and tuning --------------------------------------------------------------- */
+
+/* Synchronise `stream`, then report and clear the device error flag: MMF_OK,
+ * MMF_ERR_TIMEOUT (an in-kernel wait ran out) or MMF_ERR_CUDA (the stream reported an error). */
+mmf_status mmf_sync_status(mmf_stream_t stream);
+/* Static description of a status code. */
+const char* mmf_status_string(mmf_status s);
+/* Description of the last failure on the calling thread ("" if none). */
+const char* mmf_last_error(void);
+
+/* Which integer-product engine the BitLinear calls use (process-wide, not thread-safe):
+ *   MMF_GEMM_AUTO   tensor-core kernel (tcgen05 int8 MMA, TMEM accumulators) for row counts
+ *                   where it pays, CUDA-core kernel otherwise (default);
+ *   MMF_GEMM_TENSOR always the tensor-core kernel;
+ *   MMF_GEMM_SIMT   always the CUDA-core kernel.
+ * Both produce identical int32 accumulators; tests use this to check each on every shape. */
+typedef enum { MMF_GEMM_AUTO = 0, MMF_GEMM_TENSOR = 1, MMF_GEMM_SIMT = 2 } mmf_gemm_path;
+mmf_status mmf_set_gemm_path(mmf_gemm_path path);
+
+/* Wall-clock cap, in microseconds, of every bounded in-kernel wait (default 2,000,000 = 2 s;
+ * 0 restores the default), measured on the GPU's global timer. Lowering it makes waits run out
+ * early, which the fault tests use to exercise the timeout path without hanging or faulting the
+ * GPU. Process-wide; read at launch. */
+mmf_status mmf_set_wait_limit(uint32_t microseconds);
+
+/* ---- instrumentation (benchmarks; no counterpart on the pages) ------------------------------ */
+
+typedef enum {
+  MMF_KERNEL_GEMM_TC = 0,    /* tensor-core ternary GEMM; work = integer ops 2*m*n*k          */
+  MMF_KERNEL_GEMM_SIMT = 1,  /* CUDA-core ternary GEMM; work = algorithmic HBM bytes            */
+  MMF_KERNEL_NORM_QUANT = 2, /* RMSNorm + int8 quant (+GLU / g_norm); work = HBM bytes          */
+  MMF_KERNEL_SCAN = 3,       /* HGRN scan; work = HBM bytes                                       */
+  MMF_KERNEL_OTHER = 4,      /* pack, embedding gather; work = HBM bytes                          */
+  MMF_KERNEL_CLASSES = 5
+} mmf_kernel_class;
+
+/* Kernels launched by this process through the library so far. */
+uint64_t mmf_launch_count(void);
+/* When on (process-wide), every launch is bracketed by two CUDA events recorded on the launch's
+ * own stream. Leave it off while a stream is being captured into a CUDA graph. */
+mmf_status mmf_timing_enable(int on);
+/* Synchronise on the recorded events and return, for kernel class `cls`, the launches, their
+ * total device milliseconds and their total algorithmic work (see mmf_kernel_class) recorded
+ * since the previous read of that class; the class's records are then cleared. */
+mmf_status mmf_timing_read(mmf_kernel_class cls, int64_t* launches, double* total_ms, double* work);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MMF_H_ */

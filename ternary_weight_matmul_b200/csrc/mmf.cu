@@ -1,0 +1,753 @@
+// mmf.cu -- C ABI of libmmf (declared in include/mmf.h): argument validation, workspace layout,
+// engine dispatch and launches. All kernels live in the headers included below (one translation
+// unit, so the device error flag is shared without relocatable device code).
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <atomic>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "common.cuh"
+#include "gemm_tc.cuh"
+#include "kernels.cuh"
+
+using namespace mmf;
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<int> g_gemm_path{MMF_GEMM_AUTO};
+constexpr uint32_t kDefaultWaitLimit = 2000000u;  // microseconds
+std::atomic<uint32_t> g_wait_limit{kDefaultWaitLimit};
+
+mmf_status fail(mmf_status s, const char* fmt, ...) __attribute__((format(printf, 2, 3)));
+mmf_status fail(mmf_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define MMF_CHECK_ARG(cond, ...)                                   \
+  do {                                                             \
+    if (!(cond)) return fail(MMF_ERR_INVALID_ARG, __VA_ARGS__);    \
+  } while (0)
+
+#define MMF_CUDA(call)                                                                       \
+  do {                                                                                       \
+    cudaError_t e_ = (call);                                                                 \
+    if (e_ != cudaSuccess) return fail(MMF_ERR_CUDA, "%s: %s", #call, cudaGetErrorString(e_)); \
+  } while (0)
+
+#define MMF_TRY(expr)                \
+  do {                               \
+    mmf_status s_ = (expr);          \
+    if (s_ != MMF_OK) return s_;     \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool valid_dtype(mmf_dtype d) { return d == MMF_F32 || d == MMF_BF16; }
+inline size_t dsize(mmf_dtype d) { return d == MMF_F32 ? 4 : 2; }
+inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int32_t row_words(int32_t k) { return 4 * ((k + 63) / 64); }
+inline int64_t row_q(int32_t k) { return 16 * (int64_t)row_words(k); }  // int8 codes per row
+
+// ---------------------------------------------------------------------------------------------
+// per-device state
+// ---------------------------------------------------------------------------------------------
+struct DevInfo {
+  bool init = false;
+  int sms = 0;
+  int major = 0, minor = 0;
+  bool tc_ready = false;
+};
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+mmf_status device_info(DevInfo** out) {
+  int dev = 0;
+  MMF_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MMF_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& di = g_dev[dev];
+  if (!di.init) {
+    MMF_CUDA(cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev));
+    MMF_CUDA(cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev));
+    MMF_CUDA(cudaDeviceGetAttribute(&di.minor, cudaDevAttrComputeCapabilityMinor, dev));
+    if (di.major == 10 && di.minor == 0) {
+      MMF_CUDA(cudaFuncSetAttribute(tc::ternary_gemm_tc_kernel,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+      MMF_CUDA(cudaFuncSetAttribute(simt_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    200 * 1024));
+      MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowPlain>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+      MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowGlu>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+      MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowGnorm>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+      di.tc_ready = true;
+    }
+    di.init = true;
+  }
+  if (!di.tc_ready)
+    return fail(MMF_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library runs on sm_100a (B200) only",
+                dev, di.major, di.minor);
+  *out = &di;
+  return MMF_OK;
+}
+
+mmf_status get_encoder() {
+  std::call_once(g_encode_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (!g_encode) return fail(MMF_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  return MMF_OK;
+}
+
+mmf_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t dim0,
+                     uint64_t dim1, uint64_t stride1_bytes, uint32_t box0, uint32_t box1,
+                     CUtensorMapSwizzle swz) {
+  MMF_TRY(get_encoder());
+  cuuint64_t dims[2] = {dim0, dim1};
+  cuuint64_t strides[1] = {stride1_bytes};
+  cuuint32_t box[2] = {box0, box1};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MMF_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MMF_OK;
+}
+
+mmf_status check_launch(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return MMF_OK;
+}
+
+// ---------------------------------------------------------------------------------------------
+// instrumentation: launch counter and optional per-class event timing
+// ---------------------------------------------------------------------------------------------
+std::atomic<uint64_t> g_launches{0};
+std::atomic<int> g_timing{0};
+struct TimedRec {
+  int cls;
+  cudaEvent_t a, b;
+  double work;
+};
+std::mutex g_tmu;
+std::vector<TimedRec> g_recs;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pooled_event() {
+  cudaEvent_t e = nullptr;
+  if (!g_event_pool.empty()) {
+    e = g_event_pool.back();
+    g_event_pool.pop_back();
+  } else if (cudaEventCreate(&e) != cudaSuccess) {
+    e = nullptr;
+  }
+  return e;
+}
+
+// Counts one launch and, when timing is on, brackets it with events on its stream.
+struct LaunchScope {
+  bool on = false;
+  TimedRec rec{};
+  cudaStream_t st;
+  LaunchScope(int cls, double work, cudaStream_t s) : st(s) {
+    g_launches.fetch_add(1);
+    if (g_timing.load()) {
+      std::lock_guard<std::mutex> lk(g_tmu);
+      rec.cls = cls;
+      rec.work = work;
+      rec.a = pooled_event();
+      rec.b = pooled_event();
+      on = rec.a && rec.b;
+    }
+    if (on) cudaEventRecord(rec.a, st);
+  }
+  ~LaunchScope() {
+    if (!on) return;
+    cudaEventRecord(rec.b, st);
+    std::lock_guard<std::mutex> lk(g_tmu);
+    g_recs.push_back(rec);
+  }
+};
+
+// ---------------------------------------------------------------------------------------------
+// internal launchers
+// ---------------------------------------------------------------------------------------------
+mmf_status launch_norm_quant(const NormQuantArgs& a, int mode, cudaStream_t st) {
+  if (a.m == 0) return MMF_OK;
+  const size_t smem = (size_t)a.k * sizeof(float);
+  const int threads = a.k >= 2048 ? 256 : 128;
+  dim3 grid((unsigned)a.m);
+  const double es = a.xdt == MMF_F32 ? 4.0 : 2.0;
+  double in_row = (mode == kRowGlu ? 2.0 : 1.0) * a.k * es;
+  if (mode == kRowGnorm) in_row += a.k * (a.gdt == MMF_F32 ? 4.0 : 2.0);
+  LaunchScope ls(MMF_KERNEL_NORM_QUANT, (double)a.m * (in_row + a.ngain * ((double)a.ldq + 4.0)), st);
+  if (mode == kRowPlain) norm_quant_kernel<kRowPlain><<<grid, threads, smem, st>>>(a);
+  else if (mode == kRowGlu) norm_quant_kernel<kRowGlu><<<grid, threads, smem, st>>>(a);
+  else norm_quant_kernel<kRowGnorm><<<grid, threads, smem, st>>>(a);
+  return check_launch("norm_quant_kernel");
+}
+
+bool use_tensor_path(int64_t m) {
+  const int p = g_gemm_path.load();
+  if (p == MMF_GEMM_TENSOR) return true;
+  if (p == MMF_GEMM_SIMT) return false;
+  return m > kSimtMT;
+}
+
+mmf_status launch_gemm(const GemmArgs& g, const DevInfo& di, cudaStream_t st) {
+  if (g.m == 0) return MMF_OK;
+  if (!use_tensor_path(g.m)) {
+    int maxn = 0;
+    for (int s = 0; s < g.nseg; ++s) maxn = std::max(maxn, g.seg[s].n);
+    const int nchunk = g.kw / 4;
+    const size_t smem = (size_t)kSimtMT * nchunk * 4 * sizeof(uint4);
+    if (smem > 200 * 1024) return fail(MMF_ERR_UNSUPPORTED, "K=%d too large for the CUDA-core engine", g.k);
+    const int gx = std::min((maxn + 31) / 32, di.sms * 8);
+    dim3 grid((unsigned)std::max(gx, 1), (unsigned)((g.m + kSimtMT - 1) / kSimtMT), (unsigned)g.nseg);
+    double bytes = 0;
+    const double yes = g.ydt == MMF_F32 ? 4.0 : 2.0;
+    for (int s = 0; s < g.nseg; ++s)
+      bytes += (double)g.seg[s].n * g.kw * 4.0 + (double)g.m * g.ldq + (double)g.m * g.seg[s].n * yes *
+               (g.seg[s].res ? 2.0 : 1.0);
+    LaunchScope ls(MMF_KERNEL_GEMM_SIMT, bytes, st);
+    simt_gemm_kernel<<<grid, 256, smem, st>>>(g);
+    return check_launch("simt_gemm_kernel");
+  }
+  tc::Params P;
+  memset(&P, 0, sizeof(P));
+  P.g = g;
+  P.m_tiles = (int32_t)((g.m + tc::BN - 1) / tc::BN);
+  int32_t tiles = 0;
+  for (int s = 0; s < g.nseg; ++s) {
+    const GemmSeg& S = g.seg[s];
+    P.tile_start[s] = tiles;
+    tiles += ((S.n + tc::BM - 1) / tc::BM) * P.m_tiles;
+    MMF_TRY(encode_2d(&P.act_map[s], CU_TENSOR_MAP_DATA_TYPE_UINT8, S.q, (uint64_t)g.ldq,
+                      (uint64_t)g.m, (uint64_t)g.ldq, tc::BK, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B));
+    MMF_TRY(encode_2d(&P.w_map[s], CU_TENSOR_MAP_DATA_TYPE_UINT32, S.codes, (uint64_t)g.kw,
+                      (uint64_t)S.n, (uint64_t)g.kw * 4, tc::W_WORDS_PER_ROW, tc::BM,
+                      CU_TENSOR_MAP_SWIZZLE_NONE));
+  }
+  P.tile_start[g.nseg] = tiles;
+  P.num_kb = (int32_t)((g.ldq + tc::BK - 1) / tc::BK);
+  P.wait_limit_us = g_wait_limit.load();
+  const int grid = std::min(tiles, di.sms);
+  double ops = 0;
+  for (int s = 0; s < g.nseg; ++s) ops += 2.0 * (double)g.m * g.seg[s].n * g.k;
+  LaunchScope ls(MMF_KERNEL_GEMM_TC, ops, st);
+  tc::ternary_gemm_tc_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(P);
+  return check_launch("ternary_gemm_tc_kernel");
+}
+
+mmf_status launch_scan(const ScanArgs& a, cudaStream_t st) {
+  if ((int64_t)a.b * a.d == 0) return MMF_OK;
+  const int64_t chans = (int64_t)a.b * a.d;
+  dim3 grid((unsigned)((chans + 31) / 32));
+  if (a.t == 0) {
+    // no steps: the final state is the initial one
+    if (a.h_last) {
+      if (a.h0) {
+        cudaError_t e = cudaMemcpyAsync(a.h_last, a.h0, chans * sizeof(float), cudaMemcpyDeviceToDevice, st);
+        if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
+      } else {
+        cudaError_t e = cudaMemsetAsync(a.h_last, 0, chans * sizeof(float), st);
+        if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+      }
+    }
+    return MMF_OK;
+  }
+  const double zes = a.zdt == MMF_F32 ? 4.0 : 2.0, hes = a.hdt == MMF_F32 ? 4.0 : 2.0;
+  LaunchScope ls(MMF_KERNEL_SCAN, (double)chans * a.t * (2.0 * zes + hes) + (double)chans * 4.0 *
+                 ((a.h0 ? 1.0 : 0.0) + (a.h_last ? 1.0 : 0.0)), st);
+  hgrn_scan_kernel<<<grid, kScanWarps * 32, 0, st>>>(a);
+  return check_launch("hgrn_scan_kernel");
+}
+
+mmf_status check_ternary(const mmf_ternary* w, int32_t n, int32_t k, const char* name) {
+  MMF_CHECK_ARG(w != nullptr, "%s: null weight descriptor", name);
+  MMF_CHECK_ARG(w->codes && w->scale, "%s: null codes or scale", name);
+  MMF_CHECK_ARG(aligned16(w->codes), "%s: codes not 16-byte aligned", name);
+  MMF_CHECK_ARG(w->n == n && w->k == k, "%s: shape [%d][%d], expected [%d][%d]", name, w->n, w->k, n, k);
+  return MMF_OK;
+}
+
+// Workspace carve-up of one block forward over m tokens.
+struct BlockWs {
+  int8_t* q3;  // [3][m][ldq_d]
+  float* deq;  // [6][m]
+  void* z;     // [m][3d]
+  void* h;     // [m][d]
+  int8_t* qo;  // [m][ldq_d]
+  void* x1;    // [m][d]
+  int8_t* qg;  // [m][ldq_d]
+  void* gu;    // [m][2I]
+  int8_t* qd;  // [m][ldq_I]
+  size_t bytes;
+};
+
+BlockWs block_ws(void* base, int64_t m, int32_t d, int32_t inner, mmf_dtype dt) {
+  BlockWs w;
+  uint8_t* p = reinterpret_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* r = p ? p + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  const size_t es = dsize(dt);
+  w.q3 = reinterpret_cast<int8_t*>(take(3 * m * row_q(d)));
+  w.deq = reinterpret_cast<float*>(take(6 * m * sizeof(float)));
+  w.z = take(m * 3 * (size_t)d * es);
+  w.h = take(m * (size_t)d * es);
+  w.qo = reinterpret_cast<int8_t*>(take(m * row_q(d)));
+  w.x1 = take(m * (size_t)d * es);
+  w.qg = reinterpret_cast<int8_t*>(take(m * row_q(d)));
+  w.gu = take(m * 2 * (size_t)inner * es);
+  w.qd = reinterpret_cast<int8_t*>(take(m * row_q(inner)));
+  w.bytes = off;
+  return w;
+}
+
+GemmSeg make_seg(const int8_t* q, const float* deq, const mmf_ternary& w, void* y, int64_t ldy,
+                 int32_t ycol, const void* res, int64_t ldres, int32_t* acc, int64_t ldacc) {
+  GemmSeg s;
+  memset(&s, 0, sizeof(s));
+  s.q = q;
+  s.deq = deq;
+  s.codes = w.codes;
+  s.sw = w.scale;
+  s.n = w.n;
+  s.y = y;
+  s.ldy = ldy;
+  s.ycol = ycol;
+  s.res = res;
+  s.ldres = ldres;
+  s.rescol = 0;
+  s.acc = acc;
+  s.ldacc = ldacc;
+  return s;
+}
+
+mmf_status check_block(const mmf_block_weights* w) {
+  MMF_CHECK_ARG(w != nullptr, "null block weights");
+  MMF_CHECK_ARG(w->d > 0 && w->inner > 0, "bad block sizes d=%d inner=%d", w->d, w->inner);
+  MMF_CHECK_ARG(w->d <= 32768 && w->inner <= 32768, "block sizes above 32768 are not supported");
+  MMF_CHECK_ARG(w->eps >= 0.0f, "negative eps");
+  MMF_TRY(check_ternary(&w->i, w->d, w->d, "i_proj"));
+  MMF_TRY(check_ternary(&w->f, w->d, w->d, "f_proj"));
+  MMF_TRY(check_ternary(&w->g, w->d, w->d, "g_proj"));
+  MMF_TRY(check_ternary(&w->o, w->d, w->d, "o_proj"));
+  MMF_TRY(check_ternary(&w->gate, 2 * w->inner, w->d, "gate_proj"));
+  MMF_TRY(check_ternary(&w->down, w->d, w->inner, "down_proj"));
+  return MMF_OK;
+}
+
+// The block forward on m = b*t tokens; ws already validated.
+mmf_status run_block(const mmf_block_weights* w, const void* x, mmf_dtype dt, int32_t b, int64_t t,
+                     const float* h0, void* y, float* h_last, const BlockWs& W, const DevInfo& di,
+                     cudaStream_t st) {
+  const int64_t m = (int64_t)b * t;
+  const int32_t d = w->d, inner = w->inner;
+  const int64_t ldq_d = row_q(d), ldq_i = row_q(inner);
+  const size_t es = dsize(dt);
+  float* deq = W.deq;
+  // 1. RMSNorm + int8 quant of x with the three gains of i/f/g_proj (one shared rms)
+  NormQuantArgs nq;
+  memset(&nq, 0, sizeof(nq));
+  nq.x = x; nq.ldx = d; nq.xdt = dt; nq.m = m; nq.k = d; nq.eps = w->eps; nq.ngain = 3;
+  nq.gain[0] = w->nw_i; nq.gain[1] = w->nw_f; nq.gain[2] = w->nw_g;
+  for (int j = 0; j < 3; ++j) {
+    nq.q[j] = W.q3 + j * m * ldq_d;
+    nq.deq[j] = deq + j * m;
+  }
+  nq.ldq = ldq_d;
+  MMF_TRY(launch_norm_quant(nq, kRowPlain, st));
+  // 2. i/f/g projections in one grouped GEMM: z = [zi | zf | g]
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.m = m; g.k = d; g.kw = row_words(d); g.ldq = ldq_d; g.ydt = dt; g.nseg = 3;
+  g.seg[0] = make_seg(W.q3, deq, w->i, W.z, 3 * d, 0, nullptr, 0, nullptr, 0);
+  g.seg[1] = make_seg(W.q3 + m * ldq_d, deq + m, w->f, W.z, 3 * d, d, nullptr, 0, nullptr, 0);
+  g.seg[2] = make_seg(W.q3 + 2 * m * ldq_d, deq + 2 * m, w->g, W.z, 3 * d, 2 * d, nullptr, 0, nullptr, 0);
+  MMF_TRY(launch_gemm(g, di, st));
+  // 3. HGRN scan with gates
+  ScanArgs sa;
+  memset(&sa, 0, sizeof(sa));
+  sa.zf = reinterpret_cast<const uint8_t*>(W.z) + d * es;
+  sa.zi = W.z;
+  sa.zdt = dt; sa.zstride = 3 * d; sa.b = b; sa.t = t; sa.d = d;
+  sa.h0 = h0; sa.h = W.h; sa.hdt = dt; sa.h_last = h_last;
+  MMF_TRY(launch_scan(sa, st));
+  // 4. g_norm (RMSNorm(h) * gnorm_w * SiLU(g)) fused with o_proj's RMSNorm + quant
+  memset(&nq, 0, sizeof(nq));
+  nq.x = W.h; nq.ldx = d; nq.xdt = dt;
+  nq.g = reinterpret_cast<const uint8_t*>(W.z) + 2 * d * es; nq.ldg = 3 * d; nq.gdt = dt;
+  nq.gw = w->gnorm_w; nq.m = m; nq.k = d; nq.eps = w->eps; nq.ngain = 1; nq.gain[0] = w->nw_o;
+  nq.q[0] = W.qo; nq.deq[0] = deq + 3 * m; nq.ldq = ldq_d;
+  MMF_TRY(launch_norm_quant(nq, kRowGnorm, st));
+  // 5. o_proj + residual: x1 = x + o_proj(u)
+  memset(&g, 0, sizeof(g));
+  g.m = m; g.k = d; g.kw = row_words(d); g.ldq = ldq_d; g.ydt = dt; g.nseg = 1;
+  g.seg[0] = make_seg(W.qo, deq + 3 * m, w->o, W.x1, d, 0, x, d, nullptr, 0);
+  MMF_TRY(launch_gemm(g, di, st));
+  // 6. gate_proj input norm + quant
+  memset(&nq, 0, sizeof(nq));
+  nq.x = W.x1; nq.ldx = d; nq.xdt = dt; nq.m = m; nq.k = d; nq.eps = w->eps; nq.ngain = 1;
+  nq.gain[0] = w->nw_gate; nq.q[0] = W.qg; nq.deq[0] = deq + 4 * m; nq.ldq = ldq_d;
+  MMF_TRY(launch_norm_quant(nq, kRowPlain, st));
+  // 7. gate_proj: gu = [a | c]
+  memset(&g, 0, sizeof(g));
+  g.m = m; g.k = d; g.kw = row_words(d); g.ldq = ldq_d; g.ydt = dt; g.nseg = 1;
+  g.seg[0] = make_seg(W.qg, deq + 4 * m, w->gate, W.gu, 2 * inner, 0, nullptr, 0, nullptr, 0);
+  MMF_TRY(launch_gemm(g, di, st));
+  // 8. v = SiLU(a) * c fused with down_proj's RMSNorm + quant
+  memset(&nq, 0, sizeof(nq));
+  nq.x = W.gu; nq.ldx = 2 * inner; nq.xdt = dt; nq.m = m; nq.k = inner; nq.eps = w->eps;
+  nq.ngain = 1; nq.gain[0] = w->nw_down; nq.q[0] = W.qd; nq.deq[0] = deq + 5 * m; nq.ldq = ldq_i;
+  MMF_TRY(launch_norm_quant(nq, kRowGlu, st));
+  // 9. down_proj + residual: y = x1 + down_proj(v)
+  memset(&g, 0, sizeof(g));
+  g.m = m; g.k = inner; g.kw = row_words(inner); g.ldq = ldq_i; g.ydt = dt; g.nseg = 1;
+  g.seg[0] = make_seg(W.qd, deq + 5 * m, w->down, y, d, 0, W.x1, d, nullptr, 0);
+  return launch_gemm(g, di, st);
+}
+
+mmf_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+  if (need == 0) return MMF_OK;
+  if (ws == nullptr || ws_bytes < need)
+    return fail(MMF_ERR_WORKSPACE, "workspace of %zu bytes given, %zu needed", ws ? ws_bytes : (size_t)0, need);
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0)
+    return fail(MMF_ERR_WORKSPACE, "workspace not 256-byte aligned");
+  return MMF_OK;
+}
+
+}  // namespace
+
+// =============================================================================================
+// exported C ABI
+// =============================================================================================
+extern "C" {
+
+int32_t mmf_packed_row_words(int32_t k) { return k <= 0 ? 0 : row_words(k); }
+
+size_t mmf_packed_words(int32_t n, int32_t k) {
+  return (n <= 0 || k <= 0) ? 0 : (size_t)n * (size_t)row_words(k);
+}
+
+size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32_t n_layers) {
+  if (m < 0 || d < 0 || inner < 0) return 0;
+  switch (op) {
+    case MMF_OP_PACK:
+      return align256(kPackSumBlocks * sizeof(double));
+    case MMF_OP_BITLINEAR:
+      return d > 0 ? align256((size_t)m * row_q(d)) + align256((size_t)m * sizeof(float)) : 0;
+    case MMF_OP_BLOCK:
+      return block_ws(nullptr, m, d, inner, MMF_F32).bytes;
+    case MMF_OP_DECODE:
+    case MMF_OP_STACK:
+      return block_ws(nullptr, m, d, inner, MMF_F32).bytes + 2 * align256((size_t)m * d * 4);
+  }
+  return 0;
+}
+
+mmf_status mmf_pack_ternary(const void* w, mmf_dtype w_dtype, int32_t n, int32_t k,
+                            uint32_t* codes_out, float* scale_out, void* ws, size_t ws_bytes,
+                            mmf_stream_t stream) {
+  MMF_CHECK_ARG(n > 0 && k > 0, "pack: bad shape [%d][%d]", n, k);
+  MMF_CHECK_ARG(valid_dtype(w_dtype), "pack: bad dtype %d", (int)w_dtype);
+  MMF_CHECK_ARG(w && codes_out && scale_out, "pack: null pointer");
+  MMF_CHECK_ARG(aligned16(codes_out), "pack: codes_out not 16-byte aligned");
+  MMF_TRY(check_ws(ws, ws_bytes, mmf_workspace_bytes(MMF_OP_PACK, (int64_t)n * k, 0, 0, 0)));
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  double* partial = reinterpret_cast<double*>(ws);
+  const int64_t count = (int64_t)n * k;
+  const int32_t kw = row_words(k);
+  const int64_t words = (int64_t)n * kw;
+  const unsigned pgrid = (unsigned)std::min<int64_t>((words + 255) / 256, (int64_t)di->sms * 16);
+  LaunchScope ls(MMF_KERNEL_OTHER, (double)count * 2.0 * dsize(w_dtype) + (double)words * 4.0, st);
+  g_launches.fetch_add(2);  // three kernels under one timing scope
+  if (w_dtype == MMF_F32) {
+    pack_abssum_kernel<MMF_F32><<<kPackSumBlocks, 256, 0, st>>>(reinterpret_cast<const float*>(w), count, partial);
+    MMF_TRY(check_launch("pack_abssum_kernel"));
+    pack_scale_kernel<<<1, 32, 0, st>>>(partial, kPackSumBlocks, count, scale_out);
+    MMF_TRY(check_launch("pack_scale_kernel"));
+    pack_codes_kernel<MMF_F32><<<pgrid, 256, 0, st>>>(reinterpret_cast<const float*>(w), n, k, kw, scale_out, codes_out);
+  } else {
+    pack_abssum_kernel<MMF_BF16><<<kPackSumBlocks, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(w), count, partial);
+    MMF_TRY(check_launch("pack_abssum_kernel"));
+    pack_scale_kernel<<<1, 32, 0, st>>>(partial, kPackSumBlocks, count, scale_out);
+    MMF_TRY(check_launch("pack_scale_kernel"));
+    pack_codes_kernel<MMF_BF16><<<pgrid, 256, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(w), n, k, kw, scale_out, codes_out);
+  }
+  return check_launch("pack_codes_kernel");
+}
+
+mmf_status mmf_bitlinear_fwd(const void* x, mmf_dtype x_dtype, int64_t m, const float* norm_w,
+                             const mmf_ternary* w, void* y, mmf_dtype y_dtype, int8_t* q_dbg,
+                             float* deq_dbg, int32_t* acc_dbg, void* ws, size_t ws_bytes,
+                             mmf_stream_t stream) {
+  MMF_CHECK_ARG(m >= 0, "bitlinear: negative m");
+  MMF_CHECK_ARG(valid_dtype(x_dtype) && valid_dtype(y_dtype), "bitlinear: bad dtype");
+  MMF_CHECK_ARG(w != nullptr && w->n > 0 && w->k > 0 && w->k <= 32768, "bitlinear: bad weight descriptor");
+  MMF_TRY(check_ternary(w, w->n, w->k, "bitlinear"));
+  if (m == 0) return MMF_OK;
+  MMF_CHECK_ARG(x && y, "bitlinear: null x or y");
+  MMF_CHECK_ARG(aligned16(x) && aligned16(y), "bitlinear: x / y not 16-byte aligned");
+  MMF_TRY(check_ws(ws, ws_bytes, mmf_workspace_bytes(MMF_OP_BITLINEAR, m, w->k, w->n, 0)));
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t ldq = row_q(w->k);
+  int8_t* q = reinterpret_cast<int8_t*>(ws);
+  float* deq = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + align256((size_t)m * ldq));
+  NormQuantArgs nq;
+  memset(&nq, 0, sizeof(nq));
+  nq.x = x; nq.ldx = w->k; nq.xdt = x_dtype; nq.m = m; nq.k = w->k; nq.eps = 1e-8f; nq.ngain = 1;
+  nq.gain[0] = norm_w; nq.q[0] = q; nq.deq[0] = deq; nq.ldq = ldq;
+  MMF_TRY(launch_norm_quant(nq, kRowPlain, st));
+  GemmArgs g;
+  memset(&g, 0, sizeof(g));
+  g.m = m; g.k = w->k; g.kw = row_words(w->k); g.ldq = ldq; g.ydt = y_dtype; g.nseg = 1;
+  g.seg[0] = make_seg(q, deq, *w, y, w->n, 0, nullptr, 0, acc_dbg, w->n);
+  MMF_TRY(launch_gemm(g, *di, st));
+  if (q_dbg) {
+    cudaError_t e = cudaMemcpy2DAsync(q_dbg, w->k, q, ldq, w->k, m, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemcpy2DAsync: %s", cudaGetErrorString(e));
+  }
+  if (deq_dbg) {
+    cudaError_t e = cudaMemcpyAsync(deq_dbg, deq, m * sizeof(float), cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
+  }
+  return MMF_OK;
+}
+
+mmf_status mmf_hgrn_scan(const void* zf, const void* zi, mmf_dtype z_dtype, int64_t z_stride,
+                         int32_t b, int64_t t, int32_t d, const float* h0, void* h_out,
+                         mmf_dtype h_dtype, float* h_last, mmf_stream_t stream) {
+  MMF_CHECK_ARG(b >= 0 && t >= 0 && d >= 0, "scan: negative size");
+  MMF_CHECK_ARG(valid_dtype(z_dtype) && valid_dtype(h_dtype), "scan: bad dtype");
+  MMF_CHECK_ARG(z_stride >= d, "scan: z_stride %lld < d %d", (long long)z_stride, d);
+  if ((int64_t)b * d == 0) return MMF_OK;
+  MMF_CHECK_ARG(t == 0 || (zf && zi && h_out), "scan: null pointer");
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  ScanArgs a;
+  memset(&a, 0, sizeof(a));
+  a.zf = zf; a.zi = zi; a.zdt = z_dtype; a.zstride = z_stride; a.b = b; a.t = t; a.d = d;
+  a.h0 = h0; a.h = h_out; a.hdt = h_dtype; a.h_last = h_last;
+  return launch_scan(a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dtype, int32_t b,
+                         int64_t t, const float* h0, void* y, float* h_last, void* ws,
+                         size_t ws_bytes, mmf_stream_t stream) {
+  MMF_TRY(check_block(w));
+  MMF_CHECK_ARG(valid_dtype(dtype), "block: bad dtype");
+  MMF_CHECK_ARG(b >= 0 && t >= 0, "block: negative size");
+  const int64_t m = (int64_t)b * t;
+  if (m == 0) {
+    if (b > 0 && h_last) {
+      DevInfo* di;
+      MMF_TRY(device_info(&di));
+      ScanArgs a;
+      memset(&a, 0, sizeof(a));
+      a.b = b; a.t = 0; a.d = w->d; a.h0 = h0; a.h_last = h_last;
+      return launch_scan(a, reinterpret_cast<cudaStream_t>(stream));
+    }
+    return MMF_OK;
+  }
+  MMF_CHECK_ARG(x && y && x != y, "block: null or aliased x / y");
+  MMF_CHECK_ARG(aligned16(x) && aligned16(y), "block: x / y not 16-byte aligned");
+  MMF_TRY(check_ws(ws, ws_bytes, mmf_workspace_bytes(MMF_OP_BLOCK, m, w->d, w->inner, 1)));
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  const BlockWs W = block_ws(ws, m, w->d, w->inner, dtype);
+  return run_block(w, x, dtype, b, t, h0, y, h_last, W, *di, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
+                           mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
+                           size_t ws_bytes, mmf_stream_t stream) {
+  MMF_CHECK_ARG(layers != nullptr && n_layers > 0, "decode: no layers");
+  MMF_CHECK_ARG(valid_dtype(dtype), "decode: bad dtype");
+  MMF_CHECK_ARG(b >= 0, "decode: negative batch");
+  for (int l = 0; l < n_layers; ++l) {
+    MMF_TRY(check_block(&layers[l]));
+    MMF_CHECK_ARG(layers[l].d == layers[0].d && layers[l].inner == layers[0].inner,
+                  "decode: layer %d has a different shape", l);
+  }
+  if (b == 0) return MMF_OK;
+  MMF_CHECK_ARG(x && y && state && x != y, "decode: null or aliased pointer");
+  MMF_CHECK_ARG(aligned16(x) && aligned16(y), "decode: x / y not 16-byte aligned");
+  const int32_t d = layers[0].d, inner = layers[0].inner;
+  MMF_TRY(check_ws(ws, ws_bytes, mmf_workspace_bytes(MMF_OP_DECODE, b, d, inner, n_layers)));
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const BlockWs W = block_ws(ws, b, d, inner, dtype);
+  uint8_t* pp = reinterpret_cast<uint8_t*>(ws) + W.bytes;
+  void* buf[2] = {pp, pp + align256((size_t)b * d * 4)};
+  const void* cur = x;
+  for (int l = 0; l < n_layers; ++l) {
+    void* out = (l == n_layers - 1) ? y : buf[l & 1];
+    float* st_l = state + (int64_t)l * b * d;
+    MMF_TRY(run_block(&layers[l], cur, dtype, b, 1, st_l, out, st_l, W, *di, st));
+    cur = out;
+  }
+  return MMF_OK;
+}
+
+mmf_status mmf_embed_gather(const int32_t* ids, int64_t m, const void* table, mmf_dtype dtype,
+                            int32_t vocab, int32_t d, void* out, mmf_stream_t stream) {
+  MMF_CHECK_ARG(m >= 0 && vocab > 0 && d > 0, "embed: bad sizes");
+  MMF_CHECK_ARG(valid_dtype(dtype), "embed: bad dtype");
+  if (m == 0) return MMF_OK;
+  MMF_CHECK_ARG(ids && table && out, "embed: null pointer");
+  MMF_CHECK_ARG(aligned16(table) && aligned16(out), "embed: table / out not 16-byte aligned");
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  {
+    LaunchScope ls(MMF_KERNEL_OTHER, (double)m * d * 2.0 * dsize(dtype) + m * 4.0, reinterpret_cast<cudaStream_t>(stream));
+    embed_gather_kernel<<<(unsigned)m, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ids, m, table, dtype, vocab, d, out);
+  }
+  return check_launch("embed_gather_kernel");
+}
+
+mmf_status mmf_stack_fwd(const mmf_block_weights* layers, int32_t n_layers, const int32_t* ids,
+                         int32_t b, int64_t t, const void* table, int32_t vocab, mmf_dtype dtype,
+                         void* y, float* h_last, void* ws, size_t ws_bytes, mmf_stream_t stream) {
+  MMF_CHECK_ARG(layers != nullptr && n_layers > 0, "stack: no layers");
+  MMF_CHECK_ARG(valid_dtype(dtype), "stack: bad dtype");
+  MMF_CHECK_ARG(b >= 0 && t >= 0 && vocab > 0, "stack: bad sizes");
+  for (int l = 0; l < n_layers; ++l) {
+    MMF_TRY(check_block(&layers[l]));
+    MMF_CHECK_ARG(layers[l].d == layers[0].d && layers[l].inner == layers[0].inner,
+                  "stack: layer %d has a different shape", l);
+  }
+  const int64_t m = (int64_t)b * t;
+  if (m == 0) return MMF_OK;
+  MMF_CHECK_ARG(ids && table && y, "stack: null pointer");
+  MMF_CHECK_ARG(aligned16(table) && aligned16(y), "stack: table / y not 16-byte aligned");
+  const int32_t d = layers[0].d, inner = layers[0].inner;
+  MMF_TRY(check_ws(ws, ws_bytes, mmf_workspace_bytes(MMF_OP_STACK, m, d, inner, n_layers)));
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const BlockWs W = block_ws(ws, m, d, inner, dtype);
+  uint8_t* pp = reinterpret_cast<uint8_t*>(ws) + W.bytes;
+  void* buf[2] = {pp, pp + align256((size_t)m * d * 4)};
+  {
+    LaunchScope ls(MMF_KERNEL_OTHER, (double)m * d * 2.0 * dsize(dtype) + m * 4.0, st);
+    embed_gather_kernel<<<(unsigned)m, 128, 0, st>>>(ids, m, table, dtype, vocab, d, buf[0]);
+  }
+  MMF_TRY(check_launch("embed_gather_kernel"));
+  const void* cur = buf[0];
+  for (int l = 0; l < n_layers; ++l) {
+    void* out = (l == n_layers - 1) ? y : buf[(l + 1) & 1];
+    float* hl = h_last ? h_last + (int64_t)l * b * d : nullptr;
+    MMF_TRY(run_block(&layers[l], cur, dtype, b, t, nullptr, out, hl, W, *di, st));
+    cur = out;
+  }
+  return MMF_OK;
+}
+
+mmf_status mmf_sync_status(mmf_stream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  unsigned flag = 0;
+  e = cudaMemcpyFromSymbol(&flag, g_device_error, sizeof(flag));
+  if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "reading the device error flag: %s", cudaGetErrorString(e));
+  if (flag != 0) {
+    const unsigned zero = 0;
+    e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "clearing the device error flag: %s", cudaGetErrorString(e));
+    return fail(MMF_ERR_TIMEOUT, "an in-kernel wait ran out (device flag 0x%x)", flag);
+  }
+  return MMF_OK;
+}
+
+const char* mmf_status_string(mmf_status s) {
+  switch (s) {
+    case MMF_OK: return "ok";
+    case MMF_ERR_INVALID_ARG: return "invalid argument";
+    case MMF_ERR_UNSUPPORTED: return "unsupported";
+    case MMF_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case MMF_ERR_CUDA: return "CUDA error";
+    case MMF_ERR_TIMEOUT: return "in-kernel wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* mmf_last_error(void) { return g_last_error.c_str(); }
+
+mmf_status mmf_set_gemm_path(mmf_gemm_path path) {
+  if (path != MMF_GEMM_AUTO && path != MMF_GEMM_TENSOR && path != MMF_GEMM_SIMT)
+    return fail(MMF_ERR_INVALID_ARG, "bad gemm path %d", (int)path);
+  g_gemm_path.store(path);
+  return MMF_OK;
+}
+
+uint64_t mmf_launch_count(void) { return g_launches.load(); }
+
+mmf_status mmf_timing_enable(int on) {
+  g_timing.store(on ? 1 : 0);
+  return MMF_OK;
+}
+
+mmf_status mmf_timing_read(mmf_kernel_class cls, int64_t* launches, double* total_ms, double* work) {
+  if ((int)cls < 0 || (int)cls >= MMF_KERNEL_CLASSES) return fail(MMF_ERR_INVALID_ARG, "bad kernel class %d", (int)cls);
+  std::lock_guard<std::mutex> lk(g_tmu);
+  int64_t n = 0;
+  double ms = 0.0, wk = 0.0;
+  std::vector<TimedRec> keep;
+  mmf_status st = MMF_OK;
+  for (const TimedRec& r : g_recs) {
+    if (r.cls != (int)cls) {
+      keep.push_back(r);
+      continue;
+    }
+    float e = 0.0f;
+    if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&e, r.a, r.b) != cudaSuccess)
+      st = fail(MMF_ERR_CUDA, "timing events failed");
+    ms += e;
+    wk += r.work;
+    ++n;
+    g_event_pool.push_back(r.a);
+    g_event_pool.push_back(r.b);
+  }
+  g_recs.swap(keep);
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = ms;
+  if (work) *work = wk;
+  return st;
+}
+
+mmf_status mmf_set_wait_limit(uint32_t microseconds) {
+  g_wait_limit.store(microseconds == 0 ? kDefaultWaitLimit : microseconds);
+  return MMF_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,96 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports every symbol
+include/mmf.h declares, reports sizes, and rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import ternary_weight_matmul_b200 as mmf
+from ternary_weight_matmul_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mmf.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    mbuild.build()
+    return mmf.lib()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mmf_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declarations_exported(L):
+    names = _declared()
+    assert len(names) >= 15
+    out = subprocess.run(["nm", "-D", "--defined-only", mbuild.OUT], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (mmf_[a-z_0-9]+)", out))
+    assert set(names) <= exported, set(names) - exported
+    assert set(names) == set(mmf.EXPORTED)
+    for n in names:
+        assert getattr(L, n) is not None
+
+
+def test_sizes(L):
+    for k, w in [(1, 4), (16, 4), (63, 4), (64, 4), (65, 8), (256, 16), (704, 44), (7040, 440)]:
+        assert L.mmf_packed_row_words(k) == w
+    assert L.mmf_packed_words(3, 65) == 24
+    assert L.mmf_packed_words(0, 65) == 0
+    assert L.mmf_workspace_bytes(mmf.MMF_OP_PACK, 10, 0, 0, 0) >= 296 * 8
+    b1 = L.mmf_workspace_bytes(mmf.MMF_OP_BLOCK, 256, 256, 704, 1)
+    b2 = L.mmf_workspace_bytes(mmf.MMF_OP_BLOCK, 512, 256, 704, 1)
+    assert 0 < b1 < b2
+    assert L.mmf_workspace_bytes(mmf.MMF_OP_STACK, 256, 256, 704, 2) > b1
+    assert L.mmf_workspace_bytes(mmf.MMF_OP_BITLINEAR, 5, 100, 7, 0) >= 5 * 128 + 5 * 4
+
+
+def test_status_strings(L):
+    for s in range(6):
+        assert L.mmf_status_string(s)
+    assert L.mmf_status_string(99) == b"unknown status"
+
+
+def test_invalid_arguments_rejected_on_host(L):
+    # every one of these fails validation before any CUDA call
+    assert L.mmf_pack_ternary(None, 0, 4, 4, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_pack_ternary(None, 7, 4, 4, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_pack_ternary(None, 0, 0, 4, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert b"pack" in L.mmf_last_error()
+    t = mmf.Ternary(None, None, 8, 16)
+    assert L.mmf_bitlinear_fwd(None, 0, 4, None, ctypes.byref(t), None, 0, None, None, None, None, 0,
+                               None) == mmf.MMF_ERR_INVALID_ARG
+    t = mmf.Ternary(16, 32, 8, 16)  # misaligned codes pointer (16 is aligned; 20 is not)
+    t.codes = 20
+    assert L.mmf_bitlinear_fwd(None, 0, 4, None, ctypes.byref(t), None, 0, None, None, None, None, 0,
+                               None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_hgrn_scan(None, None, 0, 2, 1, 4, 4, None, None, 0, None, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_hgrn_scan(None, None, 5, 4, 1, 4, 4, None, None, 0, None, None) == mmf.MMF_ERR_INVALID_ARG
+    bw = mmf.BlockWeightsC(d=0, inner=4)
+    assert L.mmf_block_fwd(ctypes.byref(bw), None, 0, 1, 1, None, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_decode_step(None, 0, None, 0, 1, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_stack_fwd(None, 0, None, 1, 1, None, 10, 0, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_embed_gather(None, 4, None, 0, 0, 4, None, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_set_gemm_path(9) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_set_gemm_path(mmf.MMF_GEMM_AUTO) == mmf.MMF_OK
+    assert L.mmf_set_wait_limit(0) == mmf.MMF_OK
+
+
+def test_block_shape_mismatch_rejected(L):
+    z = mmf.Ternary(256, 256, 64, 64)
+    bw = mmf.BlockWeightsC(d=64, inner=32, eps=1e-8, i=z, f=z, g=z, o=z,
+                           gate=mmf.Ternary(256, 256, 64, 64),  # should be [64][64] -> [2*32][64] ok
+                           down=mmf.Ternary(256, 256, 64, 64))  # should be [64][32]: wrong
+    assert L.mmf_block_fwd(ctypes.byref(bw), None, 0, 1, 1, None, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert b"down_proj" in L.mmf_last_error()
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    with pytest.raises(ValueError):
+        mmf.pack_ternary(torch.zeros(4, 4))

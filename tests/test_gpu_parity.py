@@ -1,0 +1,308 @@
+"""GPU parity of every kernel path against the CPU oracle, through the C ABI.
+
+Tolerances (stated by the build target): integer accumulations bit-exact; float32 outputs within
+1e-5 absolute + 1e-3 relative per element; bfloat16 outputs within 2e-2 relative. Quantisation
+decisions: the first activation quantisation of a BitLinear sees a correctly rounded float32 r on
+both sides, so its codes must match exactly except where the oracle's pre-rounding value lies
+within 1e-4 of a half-integer (none are expected); in chained stages a code can flip by one at
+such near-ties, which the block-level checks bound instead of forbidding (see the block tests).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+
+pytestmark = pytest.mark.gpu
+
+RTOL32, ATOL32 = 1e-3, 1e-5
+RTOL16 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def mmf():
+    import ternary_weight_matmul_b200 as m
+    from ternary_weight_matmul_b200 import build
+    build.build()
+    m.lib()
+    torch.cuda.set_device(0)
+    yield m
+    m.set_gemm_path(m.MMF_GEMM_AUTO)
+
+
+DEV = "cuda:0"
+
+
+def _to(x, dtype=torch.float32):
+    return torch.from_numpy(np.ascontiguousarray(x)).to(DEV, dtype)
+
+
+def _bf16_round(a):
+    return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).to(torch.bfloat16).float().numpy()
+
+
+def _ok(mmf):
+    assert mmf.sync_status(DEV) == 0
+
+
+# ---------------------------------------------------------------------------------------------
+# K0 pack
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("n,k", [(256, 256), (1408, 256), (256, 704), (37, 100), (3, 1), (5, 64), (7, 65)])
+@pytest.mark.parametrize("wdt", ["f32", "bf16"])
+def test_pack_parity(mmf, n, k, wdt):
+    W = synth.weight(100 + n + k, n, k)
+    if wdt == "bf16":
+        W = _bf16_round(W)
+    wt = _to(W, torch.float32 if wdt == "f32" else torch.bfloat16)
+    pt = mmf.pack_ternary(wt)
+    _ok(mmf)
+    t_ref, s_ref = O.ternarize(W)
+    assert pt.scale.item() == float(s_ref)
+    words = pt.codes.cpu().numpy().view(np.uint32)
+    assert np.array_equal(words, O.pack_codes(t_ref))
+
+
+def test_pack_degenerate_zero_matrix(mmf):
+    pt = mmf.pack_ternary(torch.zeros(4, 70, device=DEV))
+    _ok(mmf)
+    assert pt.scale.item() == np.float32(1e-5)
+    assert int(pt.codes.abs().sum()) == 0
+
+
+# ---------------------------------------------------------------------------------------------
+# BitLinear (both integer-product engines)
+# ---------------------------------------------------------------------------------------------
+def _near_tie(v, margin=1e-4):
+    a = np.abs(v.astype(np.float64))
+    return np.abs(a - np.floor(a) - 0.5) < margin
+
+
+BITLINEAR_SHAPES = [(1, 256, 256), (3, 768, 256), (8, 1408, 256), (127, 256, 704), (256, 256, 256),
+                    (300, 200, 100), (130, 384, 1024), (9, 64, 2560)]
+
+
+@pytest.mark.parametrize("engine", ["tensor", "simt"])
+@pytest.mark.parametrize("m,n,k", BITLINEAR_SHAPES)
+@pytest.mark.parametrize("xdt", ["f32", "bf16"])
+def test_bitlinear_parity(mmf, engine, m, n, k, xdt):
+    mmf.set_gemm_path(mmf.MMF_GEMM_TENSOR if engine == "tensor" else mmf.MMF_GEMM_SIMT)
+    try:
+        seed = m * 7 + n * 3 + k
+        x = synth.activations(seed, (m, k))
+        if xdt == "bf16":
+            x = _bf16_round(x)
+        nw = synth.norm_weight(seed + 1, k, random=True)
+        W = synth.weight(seed + 2, n, k)
+        pt = mmf.pack_ternary(_to(W))
+        y, q, deq, acc = mmf.bitlinear_fwd(_to(x, torch.float32 if xdt == "f32" else torch.bfloat16), _to(nw), pt,
+                                            y_dtype=torch.float32, debug=True)
+        _ok(mmf)
+    finally:
+        mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
+    t, s = O.ternarize(W)
+    y_ref, taps = O.bitlinear(x.astype(np.float64), nw, t, s)
+    q_g, acc_g, deq_g, y_g = q.cpu().numpy(), acc.cpu().numpy(), deq.cpu().numpy(), y.cpu().numpy()
+    # activation codes: identical except at near-ties of the oracle's float32 value
+    mism = q_g != taps["q"]
+    assert np.all(np.abs(q_g.astype(int) - taps["q"].astype(int)) <= 1)
+    assert np.all(_near_tie(taps["v"])[mism])
+    # integer accumulation: bit-exact given the kernel's own codes
+    assert np.array_equal(acc_g.astype(np.int64), O.int_matmul(q_g, t))
+    np.testing.assert_allclose(deq_g, taps["deq"], rtol=1e-6)
+    # epilogue arithmetic on the kernel's own accumulators
+    y_from_acc = acc_g.astype(np.float64) * deq_g.astype(np.float64)[:, None] * float(s)
+    np.testing.assert_allclose(y_g, y_from_acc, rtol=RTOL32, atol=ATOL32)
+    # end to end against the oracle: elementwise where no code flipped
+    rows_ok = ~mism.any(axis=1)
+    np.testing.assert_allclose(y_g[rows_ok], y_ref[rows_ok], rtol=RTOL32, atol=ATOL32)
+
+
+def test_bitlinear_zero_rows_and_bf16_output(mmf):
+    k, n = 256, 512
+    x = synth.activations(5, (20, k))
+    x[3] = 0.0
+    x[17] = 0.0
+    W = synth.weight(6, n, k)
+    pt = mmf.pack_ternary(_to(W))
+    y = mmf.bitlinear_fwd(_to(x), None, pt, y_dtype=torch.bfloat16)
+    _ok(mmf)
+    t, s = O.ternarize(W)
+    y_ref, _ = O.bitlinear(x.astype(np.float64), None, t, s)
+    yg = y.float().cpu().numpy()
+    assert np.all(yg[3] == 0) and np.all(yg[17] == 0)
+    np.testing.assert_allclose(yg, y_ref, rtol=RTOL16, atol=1e-2 * np.abs(y_ref).max())
+
+
+@pytest.mark.parametrize("m", [1, 64, 1000])
+def test_bitlinear_engines_bit_identical(mmf, m):
+    k, n = 1024, 640
+    x = _to(synth.activations(40 + m, (m, k)))
+    pt = mmf.pack_ternary(_to(synth.weight(41, n, k)))
+    outs = []
+    for path in (mmf.MMF_GEMM_TENSOR, mmf.MMF_GEMM_SIMT):
+        mmf.set_gemm_path(path)
+        outs.append(mmf.bitlinear_fwd(x, None, pt, debug=True))
+    mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
+    _ok(mmf)
+    assert torch.equal(outs[0][3], outs[1][3])   # accumulators
+    assert torch.equal(outs[0][0], outs[1][0])   # rescaled outputs
+
+
+# ---------------------------------------------------------------------------------------------
+# HGRN scan
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("b,t,d", [(1, 1, 32), (2, 7, 96), (3, 128, 100), (1, 129, 64), (2, 1000, 32), (1, 300, 2048)])
+@pytest.mark.parametrize("long_memory", [False, True])
+@pytest.mark.parametrize("with_h0", [False, True])
+def test_scan_parity_f32(mmf, b, t, d, long_memory, with_h0):
+    zf, zi = synth.scan_inputs(b * t + d, b, t, d, long_memory)
+    h0 = synth.activations(9, (b, d)) if with_h0 else None
+    h, hl = mmf.hgrn_scan(_to(zf), _to(zi), _to(h0) if with_h0 else None)
+    _ok(mmf)
+    f, i = O.hgrn_gates(zf, zi)
+    h_ref = O.hgrn_scan(f, i, h0)
+    np.testing.assert_allclose(h.cpu().numpy(), h_ref, rtol=RTOL32, atol=ATOL32)
+    np.testing.assert_allclose(hl.cpu().numpy(), h_ref[:, -1], rtol=RTOL32, atol=ATOL32)
+
+
+def test_scan_parity_bf16_strided(mmf):
+    b, t, d = 2, 333, 256
+    z = synth.activations(11, (b, t, 3 * d))
+    z = _bf16_round(z)
+    zt = _to(z, torch.bfloat16)
+    zi_v, zf_v = zt[:, :, :d], zt[:, :, d:2 * d]
+    h, hl = mmf.hgrn_scan(zf_v, zi_v, None, h_dtype=torch.bfloat16)
+    _ok(mmf)
+    f, i = O.hgrn_gates(z[:, :, d:2 * d], z[:, :, :d])
+    h_ref = O.hgrn_scan(f, i)
+    np.testing.assert_allclose(h.float().cpu().numpy(), h_ref, rtol=RTOL16, atol=RTOL16 * 0.1)
+
+
+def test_scan_long_sequence_closed_form(mmf):
+    # constant gates: h_t = SiLU(zi) (1 - f^t); T = 65536 with f = sigmoid(4) checks carry drift
+    b, t, d = 1, 65536, 64
+    zf = np.full((b, t, d), 4.0, np.float32)
+    zi = np.tile(np.linspace(-2, 2, d, dtype=np.float32), (b, t, 1))
+    h, hl = mmf.hgrn_scan(_to(zf), _to(zi))
+    _ok(mmf)
+    f = 1 / (1 + np.exp(-4.0))
+    silu = zi[0, 0].astype(np.float64) / (1 + np.exp(-zi[0, 0].astype(np.float64)))
+    ts = np.array([1, 2, 10, 100, 1000, 30000, 65536])
+    want = silu[None, :] * (1 - f ** ts[:, None])
+    np.testing.assert_allclose(h[0, ts - 1].cpu().numpy(), want, rtol=RTOL32, atol=ATOL32)
+
+
+def test_scan_empty_sequence_returns_h0(mmf):
+    h0 = _to(synth.activations(3, (2, 64)))
+    zf = torch.zeros(2, 0, 64, device=DEV)
+    h, hl = mmf.hgrn_scan(zf, zf, h0)
+    _ok(mmf)
+    assert h.numel() == 0 and torch.equal(hl, h0)
+
+
+# ---------------------------------------------------------------------------------------------
+# block, decode, stack
+# ---------------------------------------------------------------------------------------------
+def _block_case(mmf, seed, d, inner, random_norms=True):
+    shape = synth.BlockShape("case", d, inner, 1)
+    params = synth.block_params(seed, shape, random_norms)
+    return params, O.quantize_block(params), mmf.make_block(params, DEV)
+
+
+def _assert_block_close(y_g, y_ref, bf16):
+    """Relative L2 error of the whole output, plus elementwise agreement on all but the few
+    elements downstream of a near-tie quantisation flip."""
+    err = np.abs(y_g - y_ref)
+    rel = np.linalg.norm(y_g - y_ref) / np.linalg.norm(y_ref)
+    if bf16:
+        assert rel < RTOL16, rel
+        frac_bad = np.mean(err > RTOL16 * np.abs(y_ref) + 1e-2 * np.sqrt(np.mean(y_ref ** 2)))
+    else:
+        assert rel < 1e-4, rel
+        frac_bad = np.mean(err > ATOL32 + RTOL32 * np.abs(y_ref))
+    assert frac_bad < 2e-3, frac_bad
+    return rel
+
+
+@pytest.mark.parametrize("engine", ["auto", "tensor", "simt"])
+def test_block_parity_tiny_config_f32(mmf, engine):
+    # one HGRNBit block, fp32, d=256, I=704, x ~ N(0,1) [2, 128, 256]
+    mmf.set_gemm_path({"auto": 0, "tensor": 1, "simt": 2}[engine])
+    try:
+        params, qp, blk = _block_case(mmf, 1, 256, 704, random_norms=False)
+        x = synth.activations(2, (2, 128, 256))
+        y, hl = mmf.block_fwd(blk, _to(x))
+        _ok(mmf)
+    finally:
+        mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
+    y_ref, h_ref, _ = O.block_forward(x.astype(np.float64), qp)
+    _assert_block_close(y.cpu().numpy(), y_ref, bf16=False)
+    np.testing.assert_allclose(hl.cpu().numpy(), h_ref, rtol=RTOL32, atol=ATOL32 * 10)
+
+
+def test_block_parity_bf16_ragged_with_state(mmf):
+    params, qp, blk = _block_case(mmf, 3, 256, 704)
+    x = _bf16_round(synth.activations(4, (3, 37, 256)))
+    h0 = synth.activations(5, (3, 256))
+    y, hl = mmf.block_fwd(blk, _to(x, torch.bfloat16), _to(h0))
+    _ok(mmf)
+    y_ref, h_ref, _ = O.block_forward(x.astype(np.float64), qp, h0)
+    _assert_block_close(y.float().cpu().numpy(), y_ref, bf16=True)
+    assert np.linalg.norm(hl.cpu().numpy() - h_ref) / np.linalg.norm(h_ref) < RTOL16
+
+
+def test_block_prefill_equals_stepwise_decode_on_gpu(mmf):
+    params, qp, blk = _block_case(mmf, 6, 256, 704)
+    params2, qp2, blk2 = _block_case(mmf, 7, 256, 704)
+    x = synth.activations(8, (2, 12, 256))
+    xt = _to(x)
+    y1, h1 = mmf.block_fwd(blk, xt)
+    y2, h2 = mmf.block_fwd(blk2, y1)
+    state = torch.zeros(2, 2, 256, device=DEV)
+    outs = []
+    for t in range(12):
+        outs.append(mmf.decode_step([blk, blk2], xt[:, t].contiguous(), state))
+    _ok(mmf)
+    yd = torch.stack(outs, 1).cpu().numpy()
+    _assert_block_close(yd, y2.cpu().numpy(), bf16=False)
+    np.testing.assert_allclose(state[0].cpu().numpy(), h1.cpu().numpy(), rtol=1e-4, atol=1e-4)
+    np.testing.assert_allclose(state[1].cpu().numpy(), h2.cpu().numpy(), rtol=1e-4, atol=1e-4)
+
+
+@pytest.mark.parametrize("b", [1, 3, 8, 64])
+def test_decode_step_parity(mmf, b):
+    layers = [_block_case(mmf, 20 + l, 256, 704) for l in range(2)]
+    x = synth.activations(30 + b, (b, 256))
+    state0 = synth.activations(31 + b, (2, b, 256)) * 0.5
+    st = _to(state0)
+    y = mmf.decode_step([c[2] for c in layers], _to(x), st)
+    _ok(mmf)
+    y_ref, st_ref = O.decode_step(x.astype(np.float64), [c[1] for c in layers], state0.astype(np.float64))
+    _assert_block_close(y.cpu().numpy(), y_ref, bf16=False)
+    np.testing.assert_allclose(st.cpu().numpy(), st_ref, rtol=1e-3, atol=1e-4)
+
+
+def test_embed_gather(mmf):
+    table = synth.embedding(50, 1000, 256)
+    ids = synth.token_ids(51, (3, 17), vocab=1000)
+    ids[0, 0] = -1
+    ids[2, 5] = 1000
+    out = mmf.embed_gather(_to(ids, torch.int32), _to(table))
+    _ok(mmf)
+    o = out.cpu().numpy()
+    ok = (ids >= 0) & (ids < 1000)
+    assert np.array_equal(o[ok], table[ids[ok]])
+    assert np.all(o[~ok] == 0)
+
+
+def test_stack_parity_two_layers(mmf):
+    layers = [_block_case(mmf, 60 + l, 256, 704) for l in range(2)]
+    table = synth.embedding(62, 500, 256)
+    ids = synth.token_ids(63, (2, 50), vocab=500)
+    y, hl = mmf.stack_fwd([c[2] for c in layers], _to(ids, torch.int32), _to(table), want_state=True)
+    _ok(mmf)
+    y_ref, st_ref = O.stack_forward(ids, table, [c[1] for c in layers])
+    _assert_block_close(y.cpu().numpy(), y_ref, bf16=False)
+    np.testing.assert_allclose(hl.cpu().numpy(), st_ref, rtol=1e-3, atol=1e-4)
