@@ -155,6 +155,34 @@ mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dt
                          int64_t t, const float* h0, void* y, float* h_last, void* ws,
                          size_t ws_bytes, mmf_stream_t stream);
 
+/* Debug taps of one block forward: every non-NULL pointer receives a copy of that intermediate,
+ * taken after the forward from the very buffers its kernels used (m = b*t tokens, es = dtype):
+ *   q_ifg [3][m][d] int8 and deq_ifg [3][m] float: activation codes / a/127 of the i, f, g inputs
+ *   z [m][3d] dtype = [zi | zf | g];  h [m][d] dtype;  q_o [m][d], deq_o [m]: o_proj input codes
+ *   x1 [m][d] dtype;  q_gate [m][d], deq_gate [m];  gu [m][2I] dtype = [gate | up]
+ *   q_down [m][I], deq_down [m]. */
+typedef struct {
+  int8_t* q_ifg;
+  float* deq_ifg;
+  void* z;
+  void* h;
+  int8_t* q_o;
+  float* deq_o;
+  void* x1;
+  int8_t* q_gate;
+  float* deq_gate;
+  void* gu;
+  int8_t* q_down;
+  float* deq_down;
+} mmf_block_taps;
+
+/* mmf_block_fwd followed by copies of its intermediates into `taps` (same kernels, same
+ * workspace). For tests and debugging; the copies add traffic. */
+mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dtype dtype, int32_t b,
+                              int64_t t, const float* h0, void* y, float* h_last,
+                              const mmf_block_taps* taps, void* ws, size_t ws_bytes,
+                              mmf_stream_t stream);
+
 /* One autoregressive step through n_layers blocks: the block above with t = 1 and the
  * recurrent state carried per layer.
  *   layers  HOST array of n_layers block descriptors (device pointers inside).

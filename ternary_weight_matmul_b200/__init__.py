@@ -26,7 +26,8 @@ MMF_GEMM_AUTO, MMF_GEMM_TENSOR, MMF_GEMM_SIMT = range(3)
 
 EXPORTED = (
     "mmf_packed_row_words", "mmf_packed_words", "mmf_workspace_bytes", "mmf_pack_ternary",
-    "mmf_bitlinear_fwd", "mmf_hgrn_scan", "mmf_block_fwd", "mmf_decode_step", "mmf_embed_gather",
+    "mmf_bitlinear_fwd", "mmf_hgrn_scan", "mmf_block_fwd", "mmf_block_fwd_taps", "mmf_decode_step",
+    "mmf_embed_gather",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
 )
@@ -48,6 +49,11 @@ class BlockWeightsC(ctypes.Structure):
         [(f"nw_{p}", ctypes.c_void_p) for p in ("i", "f", "g", "o", "gate", "down")] + \
         [("gnorm_w", ctypes.c_void_p)] + \
         [(p, Ternary) for p in ("i", "f", "g", "o", "gate", "down")]
+
+
+class BlockTapsC(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in (
+        "q_ifg", "deq_ifg", "z", "h", "q_o", "deq_o", "x1", "q_gate", "deq_gate", "gu", "q_down", "deq_down")]
 
 
 _lib = None
@@ -73,6 +79,8 @@ def lib() -> ctypes.CDLL:
         "mmf_hgrn_scan": (ctypes.c_int, [vp, vp, ctypes.c_int, i64, i32, i64, i32, vp, vp, ctypes.c_int, vp, st]),
         "mmf_block_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), vp, ctypes.c_int, i32, i64, vp, vp, vp,
                                          vp, sz, st]),
+        "mmf_block_fwd_taps": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), vp, ctypes.c_int, i32, i64, vp, vp,
+                                              vp, ctypes.POINTER(BlockTapsC), vp, sz, st]),
         "mmf_decode_step": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, ctypes.c_int, i32, vp, vp,
                                            vp, sz, st]),
         "mmf_embed_gather": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, i32, i32, vp, st]),
@@ -272,6 +280,37 @@ def block_fwd(block: Block, x: torch.Tensor, h0: torch.Tensor | None = None):
     _check(lib().mmf_block_fwd(ctypes.byref(bw), x.data_ptr(), _dt(x.dtype), b, t, _ptr(h0), y.data_ptr(),
                                h_last.data_ptr(), ws.data_ptr(), ws.numel(), _stream(x.device)), "mmf_block_fwd")
     return y, h_last
+
+
+def block_fwd_taps(block: Block, x: torch.Tensor, h0: torch.Tensor | None = None):
+    """mmf_block_fwd_taps: the block forward plus every intermediate (see mmf_block_taps).
+    Returns (y, h_last, taps) with taps a dict of tensors."""
+    _dev(x)
+    b, t, d = x.shape
+    m, inner, dev, dt = b * t, block.inner, x.device, x.dtype
+    y = torch.empty_like(x)
+    h_last = torch.empty(b, d, dtype=torch.float32, device=dev)
+    taps = {
+        "q_ifg": torch.empty(3, m, d, dtype=torch.int8, device=dev),
+        "deq_ifg": torch.empty(3, m, dtype=torch.float32, device=dev),
+        "z": torch.empty(m, 3 * d, dtype=dt, device=dev),
+        "h": torch.empty(m, d, dtype=dt, device=dev),
+        "q_o": torch.empty(m, d, dtype=torch.int8, device=dev),
+        "deq_o": torch.empty(m, dtype=torch.float32, device=dev),
+        "x1": torch.empty(m, d, dtype=dt, device=dev),
+        "q_gate": torch.empty(m, d, dtype=torch.int8, device=dev),
+        "deq_gate": torch.empty(m, dtype=torch.float32, device=dev),
+        "gu": torch.empty(m, 2 * inner, dtype=dt, device=dev),
+        "q_down": torch.empty(m, inner, dtype=torch.int8, device=dev),
+        "deq_down": torch.empty(m, dtype=torch.float32, device=dev),
+    }
+    tc = BlockTapsC(**{k: v.data_ptr() for k, v in taps.items()})
+    ws = workspace(MMF_OP_BLOCK, m, block.d, inner, 1, dev)
+    bw = block.c()
+    _check(lib().mmf_block_fwd_taps(ctypes.byref(bw), x.data_ptr(), _dt(dt), b, t, _ptr(h0), y.data_ptr(),
+                                    h_last.data_ptr(), ctypes.byref(tc), ws.data_ptr(), ws.numel(), _stream(dev)),
+           "mmf_block_fwd_taps")
+    return y, h_last, taps
 
 
 def decode_step(blocks: list[Block], x: torch.Tensor, state: torch.Tensor, out: torch.Tensor | None = None):

@@ -133,20 +133,27 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Bounded wait for the phase with the given parity. Gives up once `limit_us` microseconds of
-// wall time have passed (measured on the global timer) or as soon as another role of the CTA has
-// set *abort; on giving up it raises the timeout flag, sets *abort and returns false.
+// SM cycles per microsecond used to turn the wait cap into a cycle budget. The SM clock never
+// exceeds 1.965 GHz on B200, so the real cap is at least the requested time.
+constexpr int64_t kCyclesPerUs = 2000;
+
+// Bounded wait for the phase with the given parity. Gives up after `limit_us` microseconds
+// (counted in SM cycles, checked every 16 polls) or as soon as another role of the CTA has set
+// *abort; on giving up it raises the timeout flag, sets *abort and returns false.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, uint32_t limit_us,
                                                   volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  const uint64_t lim = (uint64_t)limit_us * 1000ull;
+  const int64_t t0 = clock64();
+  const int64_t lim = (int64_t)limit_us * kCyclesPerUs;
+  uint32_t polls = 0;
   while (!mbar_try_wait(bar, parity)) {
-    if (*abort) return false;
-    if (globaltimer_ns() - t0 >= lim) {
-      raise_device_error(kErrTimeout);
-      *abort = 1;
-      return false;
+    if ((++polls & 15u) == 0u) {
+      if (*abort) return false;
+      if (clock64() - t0 >= lim) {
+        raise_device_error(kErrTimeout);
+        *abort = 1;
+        return false;
+      }
     }
   }
   return true;

@@ -79,14 +79,16 @@ __device__ __forceinline__ void decode_tile(const Params& P, int tile, int& seg,
 // Wait without an abort check, used only while draining after an abort. Its own cap (1 s) does
 // not follow the (possibly lowered) wait limit: copies and MMAs already issued complete within
 // microseconds, and the CTA must not release shared or tensor memory before they have.
-constexpr uint64_t kDrainNs = 1000000000ull;
+constexpr int64_t kDrainCycles = 1000000ll * kCyclesPerUs;
 __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const uint64_t t0 = globaltimer_ns();
-  while (!mbar_try_wait(bar, parity) && globaltimer_ns() - t0 < kDrainNs) {
+  const int64_t t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 < kDrainCycles) {
   }
 }
 
+template <mmf_dtype YT>
 __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const __grid_constant__ Params P) {
+  using OutT = typename Elem<YT>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* act_s = smem;
@@ -221,6 +223,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     }
   } else {
     // ------------------------------------------------------------------ epilogue
+    // Thread = one weight row n (its TMEM lane); for each token column j of a 32-column chunk it
+    // writes y[m0 + j][n]: the 32 lanes of a warp store 32 consecutive features of one token.
+    // The per-token factor a/127 is loaded once per chunk (lane j holds token j) and broadcast.
     const uint32_t sub = (uint32_t)(warp & 3);
     const int row = (int)sub * 32 + lane;
     const uint32_t lane_addr = (sub * 32u) << 16;
@@ -231,20 +236,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
       tc_fence_after();
       int seg, nt, mt;
       decode_tile(P, tile, seg, nt, mt);
-      const GemmSeg& S = P.g.seg[seg];
+      const GemmSeg* S = seg == 0 ? &P.g.seg[0] : (seg == 1 ? &P.g.seg[1] : &P.g.seg[2]);
       const int n = nt * BM + row;
-      const bool nvalid = n < S.n;
-      const float sw = S.sw[0];
+      const bool nvalid = n < S->n;
+      const float sw = S->sw[0];
+      const float* deq = S->deq;
+      OutT* y = reinterpret_cast<OutT*>(S->y);
+      const int64_t ldy = S->ldy;
+      const OutT* res = reinterpret_cast<const OutT*>(S->res);
+      const int64_t ldres = S->ldres;
+      int32_t* accp = S->acc;
+      const int64_t ldacc = S->ldacc;
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + lane_addr + ACC_COL + b * BN + c0, v);
         tmem_wait_ld();
-        const int64_t m_first = (int64_t)mt * BN + c0;
-        if (nvalid) {
-#pragma unroll 4
-          for (int j = 0; j < 32; ++j) {
-            const int64_t m = m_first + j;
-            if (m < P.g.m) bitlinear_epilogue(S, P.g.ydt, m, n, (int32_t)v[j], sw);
+        const int64_t m0 = (int64_t)mt * BN + c0;
+        const int64_t rem = P.g.m - m0;
+        const int jmax = rem < 32 ? (int)rem : 32;
+        const float dq = lane < jmax ? deq[m0 + lane] * sw : 0.0f;
+        OutT* yp = y + m0 * ldy + S->ycol + n;
+        const OutT* rp = res ? res + m0 * ldres + S->rescol + n : nullptr;
+        int32_t* ap = accp ? accp + m0 * ldacc + n : nullptr;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          const float dj = __shfl_sync(0xffffffffu, dq, j);
+          if (j < jmax && nvalid) {
+            float z = (float)(int32_t)v[j] * dj;
+            if (ap) ap[j * ldacc] = (int32_t)v[j];
+            if (rp) z += Elem<YT>::load(rp + j * ldres);
+            Elem<YT>::store(yp + j * ldy, z);
           }
         }
       }

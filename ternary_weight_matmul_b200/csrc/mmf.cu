@@ -86,7 +86,9 @@ mmf_status device_info(DevInfo** out) {
     MMF_CUDA(cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev));
     MMF_CUDA(cudaDeviceGetAttribute(&di.minor, cudaDevAttrComputeCapabilityMinor, dev));
     if (di.major == 10 && di.minor == 0) {
-      MMF_CUDA(cudaFuncSetAttribute(tc::ternary_gemm_tc_kernel,
+      MMF_CUDA(cudaFuncSetAttribute(tc::ternary_gemm_tc_kernel<MMF_F32>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
+      MMF_CUDA(cudaFuncSetAttribute(tc::ternary_gemm_tc_kernel<MMF_BF16>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
       MMF_CUDA(cudaFuncSetAttribute(simt_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     200 * 1024));
@@ -256,7 +258,10 @@ mmf_status launch_gemm(const GemmArgs& g, const DevInfo& di, cudaStream_t st) {
   double ops = 0;
   for (int s = 0; s < g.nseg; ++s) ops += 2.0 * (double)g.m * g.seg[s].n * g.k;
   LaunchScope ls(MMF_KERNEL_GEMM_TC, ops, st);
-  tc::ternary_gemm_tc_kernel<<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(P);
+  if (g.ydt == MMF_F32)
+    tc::ternary_gemm_tc_kernel<MMF_F32><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(P);
+  else
+    tc::ternary_gemm_tc_kernel<MMF_BF16><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(P);
   return check_launch("ternary_gemm_tc_kernel");
 }
 
@@ -586,6 +591,39 @@ mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dt
   MMF_TRY(device_info(&di));
   const BlockWs W = block_ws(ws, m, w->d, w->inner, dtype);
   return run_block(w, x, dtype, b, t, h0, y, h_last, W, *di, reinterpret_cast<cudaStream_t>(stream));
+}
+
+mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dtype dtype, int32_t b,
+                              int64_t t, const float* h0, void* y, float* h_last,
+                              const mmf_block_taps* taps, void* ws, size_t ws_bytes,
+                              mmf_stream_t stream) {
+  MMF_CHECK_ARG(taps != nullptr, "block taps: null taps");
+  MMF_TRY(mmf_block_fwd(w, x, dtype, b, t, h0, y, h_last, ws, ws_bytes, stream));
+  const int64_t m = (int64_t)b * t;
+  if (m == 0) return MMF_OK;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const BlockWs W = block_ws(ws, m, w->d, w->inner, dtype);
+  const int32_t d = w->d, inner = w->inner;
+  const size_t es = dsize(dtype);
+  auto copy2d = [&](void* dst, size_t dpitch, const void* src, size_t spitch, size_t width, size_t rows) -> mmf_status {
+    if (!dst) return MMF_OK;
+    cudaError_t e = cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, rows, cudaMemcpyDeviceToDevice, st);
+    if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "taps copy: %s", cudaGetErrorString(e));
+    return MMF_OK;
+  };
+  MMF_TRY(copy2d(taps->q_ifg, d, W.q3, row_q(d), d, 3 * m));
+  MMF_TRY(copy2d(taps->deq_ifg, 3 * m * 4, W.deq, 3 * m * 4, 3 * m * 4, 1));
+  MMF_TRY(copy2d(taps->z, 3 * d * es, W.z, 3 * d * es, 3 * d * es, m));
+  MMF_TRY(copy2d(taps->h, d * es, W.h, d * es, d * es, m));
+  MMF_TRY(copy2d(taps->q_o, d, W.qo, row_q(d), d, m));
+  MMF_TRY(copy2d(taps->deq_o, m * 4, W.deq + 3 * m, m * 4, m * 4, 1));
+  MMF_TRY(copy2d(taps->x1, d * es, W.x1, d * es, d * es, m));
+  MMF_TRY(copy2d(taps->q_gate, d, W.qg, row_q(d), d, m));
+  MMF_TRY(copy2d(taps->deq_gate, m * 4, W.deq + 4 * m, m * 4, m * 4, 1));
+  MMF_TRY(copy2d(taps->gu, 2 * inner * es, W.gu, 2 * inner * es, 2 * inner * es, m));
+  MMF_TRY(copy2d(taps->q_down, inner, W.qd, row_q(inner), inner, m));
+  MMF_TRY(copy2d(taps->deq_down, m * 4, W.deq + 5 * m, m * 4, m * 4, 1));
+  return MMF_OK;
 }
 
 mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,

@@ -211,18 +211,94 @@ def _block_case(mmf, seed, d, inner, random_norms=True):
     return params, O.quantize_block(params), mmf.make_block(params, DEV)
 
 
-def _assert_block_close(y_g, y_ref, bf16):
-    """Relative L2 error of the whole output, plus elementwise agreement on all but the few
-    elements downstream of a near-tie quantisation flip."""
-    err = np.abs(y_g - y_ref)
+def _np(t):
+    return t.float().cpu().numpy() if t.dtype in (torch.bfloat16, torch.float32) else t.cpu().numpy()
+
+
+def _codes_match(q_gpu, v_oracle, q_oracle, margin):
+    """Activation codes equal the oracle's except by one step where the oracle's float32 value
+    lies within `margin` of a half-integer."""
+    mism = q_gpu != q_oracle
+    assert np.all(np.abs(q_gpu.astype(int) - q_oracle.astype(int)) <= 1)
+    assert np.all(_near_tie(v_oracle, margin)[mism]), int(mism.sum())
+    return mism
+
+
+def _close(got, want, bf16):
+    if bf16:
+        np.testing.assert_allclose(got, want, rtol=RTOL16, atol=1e-6 * max(1.0, np.abs(want).max()))
+    else:
+        np.testing.assert_allclose(got, want, rtol=RTOL32, atol=ATOL32)
+
+
+def check_block_stages(x, qp, taps, y_g, hl_g, h0, bf16):
+    """Stage-wise parity: each stage of the kernel's block forward against the oracle's definition
+    of that stage applied to the kernel's own inputs to it. Integer accumulations are exact; codes
+    of the first quantisation match exactly, chained ones up to near-ties; floats elementwise."""
+    m, d = x.shape[0] * x.shape[1], x.shape[2]
+    B, T = x.shape[:2]
+    x2 = x.reshape(m, d).astype(np.float64)
+    q_ifg, deq_ifg = _np(taps["q_ifg"]), _np(taps["deq_ifg"])
+    z = _np(taps["z"]).astype(np.float64)
+    # 1. i/f/g input codes (first quantisation: exact) and 2. the three products
+    for j, p in enumerate(("i", "f", "g")):
+        r = O.rmsnorm(x2, qp[f"nw_{p}"])
+        qo, deqo, vo = O.act_quant(r)
+        _codes_match(q_ifg[j], vo, qo, 1e-4)
+        np.testing.assert_allclose(deq_ifg[j], deqo, rtol=1e-6)
+        acc = O.int_matmul(q_ifg[j], qp[f"t_{p}"])
+        _close(z[:, j * d:(j + 1) * d], acc * deq_ifg[j].astype(np.float64)[:, None] * float(qp[f"s_{p}"]), bf16)
+    # 3. scan on the kernel's gate pre-activations
+    zi, zf, g = z[:, :d], z[:, d:2 * d], z[:, 2 * d:]
+    f, i = O.hgrn_gates(zf.reshape(B, T, d), zi.reshape(B, T, d))
+    h_ref = O.hgrn_scan(f, i, h0)
+    h = _np(taps["h"]).astype(np.float64)
+    _close(h, h_ref.reshape(m, d), bf16)
+    np.testing.assert_allclose(hl_g, h_ref[:, -1], rtol=1e-3 if not bf16 else RTOL16, atol=1e-5)
+    # 4. g_norm + o_proj codes, 5. o_proj + residual
+    u = O.rmsnorm(h, qp["gnorm_w"]) * O.silu(g)
+    qo, _, vo = O.act_quant(O.rmsnorm(u, qp["nw_o"]))
+    q_o = _np(taps["q_o"])
+    _codes_match(q_o, vo, qo, 1e-3)
+    x1_ref = x2 + O.int_matmul(q_o, qp["t_o"]) * _np(taps["deq_o"]).astype(np.float64)[:, None] * float(qp["s_o"])
+    x1 = _np(taps["x1"]).astype(np.float64)
+    _close(x1, x1_ref, bf16)
+    # 6. gate_proj codes and product
+    qg, _, vg = O.act_quant(O.rmsnorm(x1, qp["nw_gate"]))
+    q_gate = _np(taps["q_gate"])
+    _codes_match(q_gate, vg, qg, 1e-3)
+    gu_ref = O.int_matmul(q_gate, qp["t_gate"]) * _np(taps["deq_gate"]).astype(np.float64)[:, None] * float(qp["s_gate"])
+    gu = _np(taps["gu"]).astype(np.float64)
+    _close(gu, gu_ref, bf16)
+    # 7. GLU + down_proj codes, 8. down_proj + residual
+    inner = gu.shape[1] // 2
+    qd, _, vd = O.act_quant(O.rmsnorm(O.silu(gu[:, :inner]) * gu[:, inner:], qp["nw_down"]))
+    q_down = _np(taps["q_down"])
+    _codes_match(q_down, vd, qd, 1e-3)
+    y_ref = x1 + O.int_matmul(q_down, qp["t_down"]) * _np(taps["deq_down"]).astype(np.float64)[:, None] * float(qp["s_down"])
+    _close(y_g.reshape(m, d), y_ref, bf16)
+
+
+def check_block_end_to_end(y_g, y_ref, inter, qp, bf16):
+    """Against the oracle's own forward: relative L2 error of the block output; in float32 also
+    elementwise tolerance on every row whose chained quantisations have no value within 1e-4 of a
+    half-integer (a code there may legitimately differ by one)."""
     rel = np.linalg.norm(y_g - y_ref) / np.linalg.norm(y_ref)
     if bf16:
         assert rel < RTOL16, rel
-        frac_bad = np.mean(err > RTOL16 * np.abs(y_ref) + 1e-2 * np.sqrt(np.mean(y_ref ** 2)))
-    else:
-        assert rel < 1e-4, rel
-        frac_bad = np.mean(err > ATOL32 + RTOL32 * np.abs(y_ref))
-    assert frac_bad < 2e-3, frac_bad
+        return rel
+    assert rel < 1e-3, rel
+    d = y_ref.shape[-1]
+    m = y_ref.size // d
+    flag = np.zeros(m, bool)
+    _, _, vo = O.act_quant(O.rmsnorm(inter["u"].reshape(m, d), qp["nw_o"]))
+    _, _, vg = O.act_quant(O.rmsnorm(inter["x1"].reshape(m, d), qp["nw_gate"]))
+    _, _, vd = O.act_quant(O.rmsnorm(inter["v"].reshape(m, -1), qp["nw_down"]))
+    for v in (vo, vg, vd):
+        flag |= _near_tie(v, 1e-4).any(axis=1)
+    assert flag.mean() < 0.5
+    yg, yr = y_g.reshape(m, d), y_ref.reshape(m, d)
+    np.testing.assert_allclose(yg[~flag], yr[~flag], rtol=RTOL32, atol=ATOL32)
     return rel
 
 
@@ -233,24 +309,32 @@ def test_block_parity_tiny_config_f32(mmf, engine):
     try:
         params, qp, blk = _block_case(mmf, 1, 256, 704, random_norms=False)
         x = synth.activations(2, (2, 128, 256))
-        y, hl = mmf.block_fwd(blk, _to(x))
+        y, hl, taps = mmf.block_fwd_taps(blk, _to(x))
+        y2, hl2 = mmf.block_fwd(blk, _to(x))
         _ok(mmf)
     finally:
         mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
-    y_ref, h_ref, _ = O.block_forward(x.astype(np.float64), qp)
-    _assert_block_close(y.cpu().numpy(), y_ref, bf16=False)
+    assert torch.equal(y, y2) and torch.equal(hl, hl2)   # taps variant runs the same path
+    check_block_stages(x, qp, taps, y.cpu().numpy(), hl.cpu().numpy(), None, bf16=False)
+    y_ref, h_ref, inter = O.block_forward(x.astype(np.float64), qp)
+    check_block_end_to_end(y.cpu().numpy(), y_ref, inter, qp, bf16=False)
     np.testing.assert_allclose(hl.cpu().numpy(), h_ref, rtol=RTOL32, atol=ATOL32 * 10)
 
 
-def test_block_parity_bf16_ragged_with_state(mmf):
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_block_parity_ragged_with_state(mmf, dtype):
+    bf16 = dtype == "bf16"
     params, qp, blk = _block_case(mmf, 3, 256, 704)
-    x = _bf16_round(synth.activations(4, (3, 37, 256)))
+    x = synth.activations(4, (3, 37, 256))
+    if bf16:
+        x = _bf16_round(x)
     h0 = synth.activations(5, (3, 256))
-    y, hl = mmf.block_fwd(blk, _to(x, torch.bfloat16), _to(h0))
+    y, hl, taps = mmf.block_fwd_taps(blk, _to(x, torch.bfloat16 if bf16 else torch.float32), _to(h0))
     _ok(mmf)
-    y_ref, h_ref, _ = O.block_forward(x.astype(np.float64), qp, h0)
-    _assert_block_close(y.float().cpu().numpy(), y_ref, bf16=True)
-    assert np.linalg.norm(hl.cpu().numpy() - h_ref) / np.linalg.norm(h_ref) < RTOL16
+    yg = _np(y)
+    check_block_stages(x, qp, taps, yg, hl.cpu().numpy(), h0, bf16=bf16)
+    y_ref, h_ref, inter = O.block_forward(x.astype(np.float64), qp, h0)
+    check_block_end_to_end(yg, y_ref, inter, qp, bf16=bf16)
 
 
 def test_block_prefill_equals_stepwise_decode_on_gpu(mmf):
@@ -266,7 +350,8 @@ def test_block_prefill_equals_stepwise_decode_on_gpu(mmf):
         outs.append(mmf.decode_step([blk, blk2], xt[:, t].contiguous(), state))
     _ok(mmf)
     yd = torch.stack(outs, 1).cpu().numpy()
-    _assert_block_close(yd, y2.cpu().numpy(), bf16=False)
+    rel = np.linalg.norm(yd - y2.cpu().numpy()) / np.linalg.norm(y2.cpu().numpy())
+    assert rel < 1e-3, rel
     np.testing.assert_allclose(state[0].cpu().numpy(), h1.cpu().numpy(), rtol=1e-4, atol=1e-4)
     np.testing.assert_allclose(state[1].cpu().numpy(), h2.cpu().numpy(), rtol=1e-4, atol=1e-4)
 
@@ -280,8 +365,11 @@ def test_decode_step_parity(mmf, b):
     y = mmf.decode_step([c[2] for c in layers], _to(x), st)
     _ok(mmf)
     y_ref, st_ref = O.decode_step(x.astype(np.float64), [c[1] for c in layers], state0.astype(np.float64))
-    _assert_block_close(y.cpu().numpy(), y_ref, bf16=False)
-    np.testing.assert_allclose(st.cpu().numpy(), st_ref, rtol=1e-3, atol=1e-4)
+    rel = np.linalg.norm(y.cpu().numpy() - y_ref) / np.linalg.norm(y_ref)
+    assert rel < 1e-3, rel
+    # the first layer's state depends only on exactly quantised inputs: elementwise
+    np.testing.assert_allclose(st.cpu().numpy()[0], st_ref[0], rtol=RTOL32, atol=ATOL32)
+    np.testing.assert_allclose(st.cpu().numpy(), st_ref, rtol=1e-2, atol=1e-3)
 
 
 def test_embed_gather(mmf):
@@ -303,6 +391,16 @@ def test_stack_parity_two_layers(mmf):
     ids = synth.token_ids(63, (2, 50), vocab=500)
     y, hl = mmf.stack_fwd([c[2] for c in layers], _to(ids, torch.int32), _to(table), want_state=True)
     _ok(mmf)
+    # the stack is the embedding gather followed by the block forward of each layer: same kernels,
+    # same inputs, so it reproduces the per-layer calls bit for bit (each block is checked against
+    # the oracle stage by stage above)
+    x0 = mmf.embed_gather(_to(ids, torch.int32), _to(table))
+    y1, h1 = mmf.block_fwd(layers[0][2], x0)
+    y2, h2 = mmf.block_fwd(layers[1][2], y1)
+    _ok(mmf)
+    assert torch.equal(y, y2) and torch.equal(hl[0], h1) and torch.equal(hl[1], h2)
     y_ref, st_ref = O.stack_forward(ids, table, [c[1] for c in layers])
-    _assert_block_close(y.cpu().numpy(), y_ref, bf16=False)
-    np.testing.assert_allclose(hl.cpu().numpy(), st_ref, rtol=1e-3, atol=1e-4)
+    rel = np.linalg.norm(y.cpu().numpy() - y_ref) / np.linalg.norm(y_ref)
+    assert rel < 1e-2, rel
+    # first layer: exactly quantised inputs, so its state matches elementwise
+    np.testing.assert_allclose(hl.cpu().numpy()[0], st_ref[0], rtol=RTOL32, atol=ATOL32)
