@@ -40,9 +40,15 @@ constexpr uint32_t ACC_COL = 0;          // accumulators at columns [0, 128) and
 constexpr uint32_t A_COL = 2 * BN;       // A stages at 256 + 32 * s (32 columns = 128 int8 per lane)
 static_assert(A_COL + STAGES * (BK / 4) <= TMEM_COLS, "TMEM budget");
 
-constexpr int SMEM_BAR_OFF = STAGES * (ACT_BYTES + W_BYTES);
+// Epilogue staging: the raw int32 accumulators of a 32-token chunk, [32 tokens][128 rows],
+// double-buffered (2 x 16 KB).
+constexpr int EPI_CHUNK = 32;
+constexpr int EPI_BUF_BYTES = EPI_CHUNK * BM * 4;
+constexpr int SMEM_EPI_OFF = STAGES * (ACT_BYTES + W_BYTES);
+constexpr int SMEM_BAR_OFF = SMEM_EPI_OFF + 2 * EPI_BUF_BYTES;
 constexpr int NUM_BARS = 3 * STAGES + 5;
 constexpr int SMEM_BYTES = SMEM_BAR_OFF + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
+static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
 
 // Instruction descriptor, kind::i8: D = s32 (bits 4-5 = 2), A and B signed int8 (bits 7-9 and
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
@@ -86,6 +92,20 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
+// OR of `pred` over the 128 epilogue threads (named barrier 1); every caller gets the result.
+__device__ __forceinline__ bool epi_any(bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred)
+      : "memory");
+  return r != 0u;
+}
+
 template <mmf_dtype YT>
 __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const __grid_constant__ Params P) {
   using OutT = typename Elem<YT>::T;
@@ -93,6 +113,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* act_s = smem;
   uint32_t* w_s = reinterpret_cast<uint32_t*>(smem + STAGES * ACT_BYTES);
+  int32_t* epi_s = reinterpret_cast<int32_t*>(smem + SMEM_EPI_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
   uint64_t* full = bars;                   // TMA -> expanders      (count 1 + tx bytes)
   uint64_t* afull = bars + STAGES;         // expanders -> MMA      (count 4)
@@ -223,55 +244,105 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    // Thread = one weight row n (its TMEM lane); for each token column j of a 32-column chunk it
-    // writes y[m0 + j][n]: the 32 lanes of a warp store 32 consecutive features of one token.
-    // The per-token factor a/127 is loaded once per chunk (lane j holds token j) and broadcast.
+    // Two phases per 32-token chunk. Phase 1: each warp loads its 32 weight rows x 32 tokens of
+    // int32 accumulators from TMEM (thread = row) and stores them to shared memory transposed,
+    // as [token][row] (one conflict-free 32-bit store per element). Phase 2: the 128 epilogue
+    // threads walk the chunk token-major in 16-byte pieces (4 rows each), rescale by
+    // (a/127) * s of the token, add the residual and write 8- or 16-byte vectors, so every
+    // global access covers whole row segments of the output.
     const uint32_t sub = (uint32_t)(warp & 3);
     const int row = (int)sub * 32 + lane;
     const uint32_t lane_addr = (sub * 32u) << 16;
-    uint32_t tl = 0;
+    const int etid = threadIdx.x - 6 * 32;  // 0..127
+    uint32_t tl = 0, chunk_ctr = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tl) {
       const uint32_t b = tl & 1u;
-      if (!mbar_wait_bounded(&accfull[b], (tl >> 1) & 1u, limit, abort_flag)) break;
+      const bool got = mbar_wait_bounded(&accfull[b], (tl >> 1) & 1u, limit, abort_flag);
+      // The four epilogue warps meet at named barrier 1 below, so they must agree on leaving:
+      // if any of them gave up waiting, all of them leave (barrier reduction over 128 threads).
+      if (epi_any(!got)) break;
       tc_fence_after();
       int seg, nt, mt;
       decode_tile(P, tile, seg, nt, mt);
       const GemmSeg* S = seg == 0 ? &P.g.seg[0] : (seg == 1 ? &P.g.seg[1] : &P.g.seg[2]);
-      const int n = nt * BM + row;
-      const bool nvalid = n < S->n;
+      const int n0 = nt * BM;
+      const int nrows = S->n - n0 < BM ? S->n - n0 : BM;
       const float sw = S->sw[0];
       const float* deq = S->deq;
-      OutT* y = reinterpret_cast<OutT*>(S->y);
+      OutT* y = reinterpret_cast<OutT*>(S->y) + S->ycol + n0;
       const int64_t ldy = S->ldy;
-      const OutT* res = reinterpret_cast<const OutT*>(S->res);
+      const OutT* res = S->res ? reinterpret_cast<const OutT*>(S->res) + S->rescol + n0 : nullptr;
       const int64_t ldres = S->ldres;
-      int32_t* accp = S->acc;
+      int32_t* accp = S->acc ? S->acc + n0 : nullptr;
       const int64_t ldacc = S->ldacc;
-      for (int c0 = 0; c0 < BN; c0 += 32) {
+      // vectorised phase 2 needs every row segment 16-byte aligned and complete
+      const bool vec_ok = nrows == BM &&
+          ((reinterpret_cast<uintptr_t>(y) | (uintptr_t)(ldy * sizeof(OutT))) & 15u) == 0 &&
+          (!res || ((reinterpret_cast<uintptr_t>(res) | (uintptr_t)(ldres * sizeof(OutT))) & 15u) == 0) &&
+          (!accp || ((reinterpret_cast<uintptr_t>(accp) | (uintptr_t)(ldacc * 4)) & 15u) == 0);
+      for (int c0 = 0; c0 < BN; c0 += EPI_CHUNK, ++chunk_ctr) {
+        int32_t* buf = epi_s + (chunk_ctr & 1u) * (EPI_CHUNK * BM);
         uint32_t v[32];
         tmem_ld_32x32b_x32(tmem_base + lane_addr + ACC_COL + b * BN + c0, v);
         tmem_wait_ld();
+        if (c0 + EPI_CHUNK >= BN) {
+          // the accumulator buffer is drained: hand it back to the MMA issuer
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&accempty[b]);
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) buf[j * BM + row] = (int32_t)v[j];
+        asm volatile("bar.sync 1, 128;" ::: "memory");
         const int64_t m0 = (int64_t)mt * BN + c0;
         const int64_t rem = P.g.m - m0;
-        const int jmax = rem < 32 ? (int)rem : 32;
-        const float dq = lane < jmax ? deq[m0 + lane] * sw : 0.0f;
-        OutT* yp = y + m0 * ldy + S->ycol + n;
-        const OutT* rp = res ? res + m0 * ldres + S->rescol + n : nullptr;
-        int32_t* ap = accp ? accp + m0 * ldacc + n : nullptr;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const float dj = __shfl_sync(0xffffffffu, dq, j);
-          if (j < jmax && nvalid) {
-            float z = (float)(int32_t)v[j] * dj;
-            if (ap) ap[j * ldacc] = (int32_t)v[j];
-            if (rp) z += Elem<YT>::load(rp + j * ldres);
-            Elem<YT>::store(yp + j * ldy, z);
+        const int jmax = rem < EPI_CHUNK ? (int)rem : EPI_CHUNK;
+        if (vec_ok) {
+          // 32 tokens x 32 pieces of 4 rows = 1024 pieces, 8 per thread
+#pragma unroll 2
+          for (int pidx = etid; pidx < EPI_CHUNK * (BM / 4); pidx += 128) {
+            const int j = pidx >> 5, q4 = (pidx & 31) * 4;
+            if (j >= jmax) break;
+            const int64_t m = m0 + j;
+            const int4 a = *reinterpret_cast<const int4*>(buf + j * BM + q4);
+            const float dj = deq[m] * sw;
+            float z0 = (float)a.x * dj, z1 = (float)a.y * dj, z2 = (float)a.z * dj, z3 = (float)a.w * dj;
+            if (accp) *reinterpret_cast<int4*>(accp + m * ldacc + q4) = a;
+            if (YT == MMF_F32) {
+              if (res) {
+                const float4 r = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(res) + m * ldres + q4);
+                z0 += r.x; z1 += r.y; z2 += r.z; z3 += r.w;
+              }
+              *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + m * ldy + q4) = make_float4(z0, z1, z2, z3);
+            } else {
+              if (res) {
+                const uint2 r = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(res) + m * ldres + q4);
+                const float2 r01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
+                const float2 r23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
+                z0 += r01.x; z1 += r01.y; z2 += r23.x; z3 += r23.y;
+              }
+              const __nv_bfloat162 o01 = __floats2bfloat162_rn(z0, z1), o23 = __floats2bfloat162_rn(z2, z3);
+              uint2 o;
+              o.x = *reinterpret_cast<const uint32_t*>(&o01);
+              o.y = *reinterpret_cast<const uint32_t*>(&o23);
+              *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(y) + m * ldy + q4) = o;
+            }
+          }
+        } else {
+          // ragged tile or unaligned output: one element per step, still token-major
+          for (int e = etid; e < EPI_CHUNK * BM; e += 128) {
+            const int j = e / BM, r = e - j * BM;
+            if (j >= jmax) break;
+            if (r >= nrows) continue;
+            const int64_t m = m0 + j;
+            const int32_t a = buf[j * BM + r];
+            float z = (float)a * (deq[m] * sw);
+            if (accp) accp[m * ldacc + r] = a;
+            if (res) z += Elem<YT>::load(res + m * ldres + r);
+            Elem<YT>::store(y + m * ldy + r, z);
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&accempty[b]);
     }
   }
 

@@ -209,7 +209,7 @@ struct GemmArgs {
 __device__ __forceinline__ void bitlinear_epilogue(const GemmSeg& s, mmf_dtype ydt, int64_t row,
                                                    int32_t col, int32_t acc, float sw) {
   if (s.acc) s.acc[row * s.ldacc + col] = acc;
-  float z = (float)acc * s.deq[row] * sw;
+  float z = (float)acc * (s.deq[row] * sw);  // same rounding order as the tensor-core epilogue
   if (s.res) z += load_as_float(s.res, row * s.ldres + s.rescol + col, ydt);
   store_from_float(s.y, row * s.ldy + s.ycol + col, ydt, z);
 }
