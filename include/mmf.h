@@ -211,6 +211,31 @@ mmf_status mmf_stack_fwd(const mmf_block_weights* layers, int32_t n_layers, cons
                          int32_t b, int64_t t, const void* table, int32_t vocab, mmf_dtype dtype,
                          void* y, float* h_last, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
+/* ---- allocation-free variant (no counterpart on the pages) ---------------------------------- */
+
+/* Bytes of the library's static scratch array used by mmf_bitlinear_fwd_noalloc (8 MiB). */
+#define MMF_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* mmf_bitlinear_fwd for callers that cannot allocate device memory and have no workspace to pass:
+ * a plug-in or custom-op interface that hands an operation only its input and output buffers,
+ * a host runtime that has reserved all device memory for its own pool, or a latency-critical
+ * loop where cudaMalloc / cudaFree (which can synchronise the device) are not allowed. It computes
+ * exactly what mmf_bitlinear_fwd computes (same kernels; no debug taps) and calls no cudaMalloc,
+ * cudaFree or other allocating routine.
+ *   Scratch: the int8 activation codes and per-row factors live in one file-scope device array of
+ *   MMF_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the library holds until the
+ *   process exits. A call needs mmf_workspace_bytes(MMF_OP_BITLINEAR, m, w->k, w->n, 0) bytes of
+ *   it; larger requests return MMF_ERR_WORKSPACE before anything is enqueued.
+ *   Set-up: the first call on each device looks up the array's device address on that device
+ *   (the device must be current); make that first call before any stream capture begins.
+ *   Sharing: every call on a device uses the same array and leaves its contents behind; the
+ *   kernels overwrite every byte they read, so nothing needs clearing between calls. Calls whose
+ *   execution overlaps on the GPU (other streams, other host threads) race on the array: order
+ *   them on one stream or synchronise between them. */
+mmf_status mmf_bitlinear_fwd_noalloc(const void* x, mmf_dtype x_dtype, int64_t m, const float* norm_w,
+                                     const mmf_ternary* w, void* y, mmf_dtype y_dtype,
+                                     mmf_stream_t stream);
+
 /* ---- status, errors and tuning --------------------------------------------------------------- */
 
 /* Synchronise `stream`, then report and clear the device error flag: MMF_OK,

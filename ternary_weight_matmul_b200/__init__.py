@@ -30,7 +30,9 @@ EXPORTED = (
     "mmf_embed_gather",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
+    "mmf_bitlinear_fwd_noalloc",
 )
+NOALLOC_SCRATCH_BYTES = 8 << 20
 
 
 class MmfError(RuntimeError):
@@ -76,6 +78,8 @@ def lib() -> ctypes.CDLL:
         "mmf_pack_ternary": (ctypes.c_int, [vp, ctypes.c_int, i32, i32, vp, vp, vp, sz, st]),
         "mmf_bitlinear_fwd": (ctypes.c_int, [vp, ctypes.c_int, i64, vp, ctypes.POINTER(Ternary), vp,
                                              ctypes.c_int, vp, vp, vp, vp, sz, st]),
+        "mmf_bitlinear_fwd_noalloc": (ctypes.c_int, [vp, ctypes.c_int, i64, vp, ctypes.POINTER(Ternary), vp,
+                                                     ctypes.c_int, st]),
         "mmf_hgrn_scan": (ctypes.c_int, [vp, vp, ctypes.c_int, i64, i32, i64, i32, vp, vp, ctypes.c_int, vp, st]),
         "mmf_block_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), vp, ctypes.c_int, i32, i64, vp, vp, vp,
                                          vp, sz, st]),

@@ -447,6 +447,31 @@ mmf_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   return MMF_OK;
 }
 
+// ---------------------------------------------------------------------------------------------
+// static scratch of the allocation-free BitLinear entry point
+// ---------------------------------------------------------------------------------------------
+// Device-side storage; in host code `g_noalloc_scratch` only names the symbol, so its device
+// address is looked up once per device with cudaGetSymbolAddress and passed to the kernels.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MMF_NOALLOC_SCRATCH_BYTES];
+void* g_noalloc_ptr[64] = {};
+std::mutex g_noalloc_mu;
+
+mmf_status noalloc_scratch(void** out) {
+  int dev = 0;
+  MMF_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(MMF_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(MMF_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return MMF_OK;
+}
+
 }  // namespace
 
 // =============================================================================================
@@ -547,6 +572,24 @@ mmf_status mmf_bitlinear_fwd(const void* x, mmf_dtype x_dtype, int64_t m, const 
     if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemcpyAsync: %s", cudaGetErrorString(e));
   }
   return MMF_OK;
+}
+
+mmf_status mmf_bitlinear_fwd_noalloc(const void* x, mmf_dtype x_dtype, int64_t m, const float* norm_w,
+                                     const mmf_ternary* w, void* y, mmf_dtype y_dtype,
+                                     mmf_stream_t stream) {
+  MMF_CHECK_ARG(m >= 0, "bitlinear_noalloc: negative m");
+  MMF_CHECK_ARG(w != nullptr && w->n > 0 && w->k > 0, "bitlinear_noalloc: bad weight descriptor");
+  if (m == 0) return MMF_OK;
+  const size_t need = mmf_workspace_bytes(MMF_OP_BITLINEAR, m, w->k, w->n, 0);
+  if (need > (size_t)MMF_NOALLOC_SCRATCH_BYTES)
+    return fail(MMF_ERR_WORKSPACE,
+                "bitlinear_noalloc: m=%lld rows of K=%d need %zu bytes of scratch; the static array "
+                "holds %u bytes (use mmf_bitlinear_fwd with a workspace, or fewer rows per call)",
+                (long long)m, w->k, need, (unsigned)MMF_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  MMF_TRY(noalloc_scratch(&scratch));
+  return mmf_bitlinear_fwd(x, x_dtype, m, norm_w, w, y, y_dtype, nullptr, nullptr, nullptr, scratch,
+                           (size_t)MMF_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 mmf_status mmf_hgrn_scan(const void* zf, const void* zi, mmf_dtype z_dtype, int64_t z_stride,
