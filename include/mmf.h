@@ -73,7 +73,8 @@ typedef enum {
   MMF_OP_BITLINEAR = 1, /* mmf_bitlinear_fwd: m rows, d = K, inner = N            */
   MMF_OP_BLOCK = 2,     /* mmf_block_fwd: m = b*t tokens, d, inner                */
   MMF_OP_DECODE = 3,    /* mmf_decode_step: m = b, d, inner                       */
-  MMF_OP_STACK = 4      /* mmf_stack_fwd: m = b*t tokens, d, inner, n_layers      */
+  MMF_OP_STACK = 4,     /* mmf_stack_fwd: m = b*t tokens, d, inner, n_layers      */
+  MMF_OP_SCAN = 5       /* mmf_hgrn_scan: m = b*t tokens, d channels              */
 } mmf_op;
 
 /* A packed ternary weight (device pointers). */
@@ -137,12 +138,15 @@ mmf_status mmf_bitlinear_fwd(const void* x, mmf_dtype x_dtype, int64_t m, const 
 /* HGRN gated linear recurrence with its gates fused in (nightvoyager.top innovations table):
  *   f = sigmoid(zf);  i = SiLU(zi) * (1 - f);  h_t = f_t * h_{t-1} + i_t,  h_{-1} = h0 or 0.
  *   zf, zi  [b][t][z_stride] z_dtype, channels [0, d) of each row are used (z_stride >= d).
- *   h0      optional [b][d] float32.
+ *   h0      optional [b][d] float32 (may alias h_last: read before it is written).
  *   h_out   [b][t][d] h_dtype.   h_last optional [b][d] float32 (= h at the last step).
- *   Channel-parallel over b*d, chunk-parallel over t with float32 carries. */
+ *   ws >= mmf_workspace_bytes(MMF_OP_SCAN, b*t, d, 0, 0) when t > 16 (unused otherwise).
+ *   Chunked: per (channel, chunk of steps) affine aggregates, a carry pass per channel, then a
+ *   replay that stores h; float32 carries throughout. */
 mmf_status mmf_hgrn_scan(const void* zf, const void* zi, mmf_dtype z_dtype, int64_t z_stride,
                          int32_t b, int64_t t, int32_t d, const float* h0, void* h_out,
-                         mmf_dtype h_dtype, float* h_last, mmf_stream_t stream);
+                         mmf_dtype h_dtype, float* h_last, void* ws, size_t ws_bytes,
+                         mmf_stream_t stream);
 
 /* One HGRNBit block forward over b sequences of t tokens (hysenlabs.com block structure):
  *   zi, zf, g = i/f/g_proj(x);  h = scan(f = sigmoid(zf), i = SiLU(zi)(1-f));

@@ -21,7 +21,7 @@ LIB_PATH = os.path.join(_HERE, "libmmf.so")
 
 MMF_OK, MMF_ERR_INVALID_ARG, MMF_ERR_UNSUPPORTED, MMF_ERR_WORKSPACE, MMF_ERR_CUDA, MMF_ERR_TIMEOUT = range(6)
 MMF_F32, MMF_BF16 = 0, 1
-MMF_OP_PACK, MMF_OP_BITLINEAR, MMF_OP_BLOCK, MMF_OP_DECODE, MMF_OP_STACK = range(5)
+MMF_OP_PACK, MMF_OP_BITLINEAR, MMF_OP_BLOCK, MMF_OP_DECODE, MMF_OP_STACK, MMF_OP_SCAN = range(6)
 MMF_GEMM_AUTO, MMF_GEMM_TENSOR, MMF_GEMM_SIMT = range(3)
 
 EXPORTED = (
@@ -80,7 +80,8 @@ def lib() -> ctypes.CDLL:
                                              ctypes.c_int, vp, vp, vp, vp, sz, st]),
         "mmf_bitlinear_fwd_noalloc": (ctypes.c_int, [vp, ctypes.c_int, i64, vp, ctypes.POINTER(Ternary), vp,
                                                      ctypes.c_int, st]),
-        "mmf_hgrn_scan": (ctypes.c_int, [vp, vp, ctypes.c_int, i64, i32, i64, i32, vp, vp, ctypes.c_int, vp, st]),
+        "mmf_hgrn_scan": (ctypes.c_int, [vp, vp, ctypes.c_int, i64, i32, i64, i32, vp, vp, ctypes.c_int, vp, vp, sz,
+                                         st]),
         "mmf_block_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), vp, ctypes.c_int, i32, i64, vp, vp, vp,
                                          vp, sz, st]),
         "mmf_block_fwd_taps": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), vp, ctypes.c_int, i32, i64, vp, vp,
@@ -268,8 +269,10 @@ def hgrn_scan(zf: torch.Tensor, zi: torch.Tensor, h0: torch.Tensor | None = None
     h = torch.empty(b, t, d, dtype=h_dtype, device=zf.device)
     h_last = torch.empty(b, d, dtype=torch.float32, device=zf.device)
     zstride = zf.stride(1) if t > 1 else max(d, zf.stride(0) if b > 1 else d)
+    ws = workspace(MMF_OP_SCAN, b * t, d, 0, 0, zf.device)
     _check(lib().mmf_hgrn_scan(zf.data_ptr(), zi.data_ptr(), _dt(zf.dtype), zstride, b, t, d, _ptr(h0),
-                               h.data_ptr(), _dt(h_dtype), h_last.data_ptr(), _stream(zf.device)), "mmf_hgrn_scan")
+                               h.data_ptr(), _dt(h_dtype), h_last.data_ptr(), ws.data_ptr(), ws.numel(),
+                               _stream(zf.device)), "mmf_hgrn_scan")
     return h, h_last
 
 

@@ -43,9 +43,18 @@ __device__ __forceinline__ void store_from_float(void* base, int64_t idx, mmf_dt
   else reinterpret_cast<__nv_bfloat16*>(base)[idx] = __float2bfloat16_rn(v);
 }
 
-// sigmoid and SiLU from their definitions (1 / (1 + e^-z), z * sigmoid(z)) with the CUDA expf.
-__device__ __forceinline__ float sigmoidf_(float z) { return 1.0f / (1.0f + expf(-z)); }
+// sigmoid and SiLU from their definitions, 1 / (1 + e^-z) and z * sigmoid(z), with the CUDA
+// fast-math intrinsics __expf and __fdividef (a few ulp; e^-z overflowing to +inf gives 0).
+__device__ __forceinline__ float sigmoidf_(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
 __device__ __forceinline__ float siluf_(float z) { return z * sigmoidf_(z); }
+// HGRN gates: f = sigmoid(zf) and 1 - f = sigmoid(-zf) = e^-zf * f, formed from one exponential so
+// 1 - f keeps full relative accuracy when f is close to 1; zf is clamped at -80 (e^80 is finite,
+// and sigmoid(-80) is below 2e-35) so the product never meets inf * 0.
+__device__ __forceinline__ void hgrn_forget(float zf, float& f, float& one_minus_f) {
+  const float e = __expf(-fmaxf(zf, -80.0f));
+  f = __fdividef(1.0f, 1.0f + e);
+  one_minus_f = e * f;
+}
 
 // ---------------------------------------------------------------------------------------------
 // reductions
@@ -238,6 +247,19 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&v)
       : "memory");
 }
 #undef MMF_W32
+#define MMF_W16(i) "=r"(v[i])
+// 32 lanes x 16 consecutive 32-bit columns.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, "
+      "%11, %12, %13, %14, %15}, [%16];"
+      : MMF_W16(0), MMF_W16(1), MMF_W16(2), MMF_W16(3), MMF_W16(4), MMF_W16(5), MMF_W16(6),
+        MMF_W16(7), MMF_W16(8), MMF_W16(9), MMF_W16(10), MMF_W16(11), MMF_W16(12), MMF_W16(13),
+        MMF_W16(14), MMF_W16(15)
+      : "r"(taddr)
+      : "memory");
+}
+#undef MMF_W16
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }

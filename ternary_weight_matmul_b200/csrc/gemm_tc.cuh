@@ -11,12 +11,13 @@
 //     into tensor memory (tcgen05.st), one weight row per TMEM lane: no unpacked copy ever touches
 //     shared memory, so the MMA reads only the activation tile from shared memory.
 //   * One thread issues tcgen05.mma.kind::i8 (A from TMEM, B from shared memory, D in TMEM).
-//   * Four epilogue warps read the int32 accumulators back with tcgen05.ld, rescale and store.
+//   * Eight epilogue warps (two per TMEM sub-partition) read the int32 accumulators back with
+//     tcgen05.ld, rescale and store.
 //   * The kernel is persistent (one CTA per SM) with a 6-stage operand ring and a double-buffered
 //     accumulator, so the epilogue of one tile overlaps the MMAs of the next.
 //
-// Warp roles (320 threads): 0 = TMA producer, 1 = TMEM allocator + MMA issuer, 2..5 = expanders,
-// 6..9 = epilogue. Every mbarrier wait is bounded; on a timeout the CTA drains its in-flight TMA
+// Warp roles (448 threads): 0 = TMA producer, 1 = TMEM allocator + MMA issuer, 2..5 = expanders,
+// 6..13 = epilogue. Every mbarrier wait is bounded; on a timeout the CTA drains its in-flight TMA
 // copies and MMAs, releases its tensor memory and exits with the device timeout flag raised.
 #pragma once
 
@@ -34,7 +35,9 @@ constexpr int STAGES = 6;
 constexpr int ACT_BYTES = BN * BK;       // 16 KB
 constexpr int W_BYTES = BM * BK / 4;     // 4 KB (2 bits per code)
 constexpr int W_WORDS_PER_ROW = BK / 16; // 8
-constexpr int NUM_THREADS = 320;
+constexpr int NUM_THREADS = 448;
+constexpr int EPI_WARPS = 8;
+constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;          // accumulators at columns [0, 128) and [128, 256)
 constexpr uint32_t A_COL = 2 * BN;       // A stages at 256 + 32 * s (32 columns = 128 int8 per lane)
@@ -92,13 +95,13 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) 
   }
 }
 
-// OR of `pred` over the 128 epilogue threads (named barrier 1); every caller gets the result.
+// OR of `pred` over the 256 epilogue threads (named barrier 1); every caller gets the result.
 __device__ __forceinline__ bool epi_any(bool pred) {
   uint32_t r;
   asm volatile(
       "{\n\t.reg .pred p, q;\n\t"
       "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, 1, 128, p;\n\t"
+      "bar.red.or.pred q, 1, 256, p;\n\t"
       "selp.u32 %0, 1, 0, q;\n\t}"
       : "=r"(r)
       : "r"((uint32_t)pred)
@@ -119,7 +122,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
   uint64_t* afull = bars + STAGES;         // expanders -> MMA      (count 4)
   uint64_t* empty = bars + 2 * STAGES;     // MMA commit -> producer (count 1)
   uint64_t* accfull = bars + 3 * STAGES;   // MMA commit -> epilogue (count 1), 2 buffers
-  uint64_t* accempty = accfull + 2;        // epilogue -> MMA        (count 4), 2 buffers
+  uint64_t* accempty = accfull + 2;        // epilogue -> MMA        (count 8), 2 buffers
   uint64_t* drain = accempty + 2;          // MMA drain after abort  (count 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + NUM_BARS);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -137,7 +140,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&accfull[b], 1);
-      mbar_init(&accempty[b], 4);
+      mbar_init(&accempty[b], EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -244,22 +247,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    // Two phases per 32-token chunk. Phase 1: each warp loads its 32 weight rows x 32 tokens of
-    // int32 accumulators from TMEM (thread = row) and stores them to shared memory transposed,
-    // as [token][row] (one conflict-free 32-bit store per element). Phase 2: the 128 epilogue
-    // threads walk the chunk token-major in 16-byte pieces (4 rows each), rescale by
-    // (a/127) * s of the token, add the residual and write 8- or 16-byte vectors, so every
-    // global access covers whole row segments of the output.
+    // Two phases per 32-token chunk. Phase 1: each warp loads its sub-partition's 32 weight rows
+    // x 16 tokens (its half of the chunk) of int32 accumulators from TMEM (thread = row) and
+    // stores them to shared memory transposed, as [token][row] (one conflict-free 32-bit store
+    // per element). Phase 2: the 256 epilogue threads walk the chunk token-major in 16-byte
+    // pieces (4 rows each), rescale by (a/127) * s of the token, add the residual and write 8- or
+    // 16-byte vectors, so every global access covers whole row segments of the output.
     const uint32_t sub = (uint32_t)(warp & 3);
+    const int half = (warp - 6) >> 2;        // which 16 tokens of a chunk this warp loads
     const int row = (int)sub * 32 + lane;
     const uint32_t lane_addr = (sub * 32u) << 16;
-    const int etid = threadIdx.x - 6 * 32;  // 0..127
+    const int etid = threadIdx.x - 6 * 32;  // 0..255
     uint32_t tl = 0, chunk_ctr = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tl) {
       const uint32_t b = tl & 1u;
       const bool got = mbar_wait_bounded(&accfull[b], (tl >> 1) & 1u, limit, abort_flag);
-      // The four epilogue warps meet at named barrier 1 below, so they must agree on leaving:
-      // if any of them gave up waiting, all of them leave (barrier reduction over 128 threads).
+      // The eight epilogue warps meet at named barrier 1 below, so they must agree on leaving:
+      // if any of them gave up waiting, all of them leave (barrier reduction over 256 threads).
       if (epi_any(!got)) break;
       tc_fence_after();
       int seg, nt, mt;
@@ -275,6 +279,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
       const int64_t ldres = S->ldres;
       int32_t* accp = S->acc ? S->acc + n0 : nullptr;
       const int64_t ldacc = S->ldacc;
+      const int32_t act = S->act;
+      const int act_rows = S->act_cols - n0;  // rows of this tile (from 0) that take the activation
       // vectorised phase 2 needs every row segment 16-byte aligned and complete
       const bool vec_ok = nrows == BM &&
           ((reinterpret_cast<uintptr_t>(y) | (uintptr_t)(ldy * sizeof(OutT))) & 15u) == 0 &&
@@ -282,8 +288,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
           (!accp || ((reinterpret_cast<uintptr_t>(accp) | (uintptr_t)(ldacc * 4)) & 15u) == 0);
       for (int c0 = 0; c0 < BN; c0 += EPI_CHUNK, ++chunk_ctr) {
         int32_t* buf = epi_s + (chunk_ctr & 1u) * (EPI_CHUNK * BM);
-        uint32_t v[32];
-        tmem_ld_32x32b_x32(tmem_base + lane_addr + ACC_COL + b * BN + c0, v);
+        uint32_t v[16];
+        tmem_ld_32x32b_x16(tmem_base + lane_addr + ACC_COL + b * BN + c0 + 16 * half, v);
         tmem_wait_ld();
         if (c0 + EPI_CHUNK >= BN) {
           // the accumulator buffer is drained: hand it back to the MMA issuer
@@ -292,15 +298,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
           if (lane == 0) mbar_arrive(&accempty[b]);
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) buf[j * BM + row] = (int32_t)v[j];
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        for (int j = 0; j < 16; ++j) buf[(16 * half + j) * BM + row] = (int32_t)v[j];
+        asm volatile("bar.sync 1, 256;" ::: "memory");
         const int64_t m0 = (int64_t)mt * BN + c0;
         const int64_t rem = P.g.m - m0;
         const int jmax = rem < EPI_CHUNK ? (int)rem : EPI_CHUNK;
         if (vec_ok) {
-          // 32 tokens x 32 pieces of 4 rows = 1024 pieces, 8 per thread
+          // 32 tokens x 32 pieces of 4 rows = 1024 pieces, 4 per thread
 #pragma unroll 2
-          for (int pidx = etid; pidx < EPI_CHUNK * (BM / 4); pidx += 128) {
+          for (int pidx = etid; pidx < EPI_CHUNK * (BM / 4); pidx += EPI_THREADS) {
             const int j = pidx >> 5, q4 = (pidx & 31) * 4;
             if (j >= jmax) break;
             const int64_t m = m0 + j;
@@ -308,6 +314,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
             const float dj = deq[m] * sw;
             float z0 = (float)a.x * dj, z1 = (float)a.y * dj, z2 = (float)a.z * dj, z3 = (float)a.w * dj;
             if (accp) *reinterpret_cast<int4*>(accp + m * ldacc + q4) = a;
+            if (act != kActNone) {
+              if (q4 + 0 < act_rows) z0 = apply_act(act, z0);
+              if (q4 + 1 < act_rows) z1 = apply_act(act, z1);
+              if (q4 + 2 < act_rows) z2 = apply_act(act, z2);
+              if (q4 + 3 < act_rows) z3 = apply_act(act, z3);
+            }
             if (YT == MMF_F32) {
               if (res) {
                 const float4 r = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(res) + m * ldres + q4);
@@ -330,7 +342,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
           }
         } else {
           // ragged tile or unaligned output: one element per step, still token-major
-          for (int e = etid; e < EPI_CHUNK * BM; e += 128) {
+          for (int e = etid; e < EPI_CHUNK * BM; e += EPI_THREADS) {
             const int j = e / BM, r = e - j * BM;
             if (j >= jmax) break;
             if (r >= nrows) continue;
@@ -339,6 +351,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
             float z = (float)a * (deq[m] * sw);
             if (accp) accp[m * ldacc + r] = a;
             if (res) z += Elem<YT>::load(res + m * ldres + r);
+            if (r < act_rows) z = apply_act(act, z);
             Elem<YT>::store(y + m * ldy + r, z);
           }
         }

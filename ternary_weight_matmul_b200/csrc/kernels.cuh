@@ -103,6 +103,7 @@ struct NormQuantArgs {
   int8_t* q[3];    // [m][ldq] (columns [k, ldq) are written as 0)
   int64_t ldq;
   float* deq[3];   // [m]
+  int32_t pre_act; // 1: the SiLU of the gate input (g for g_norm, the gate half for GLU) is precomputed
 };
 
 __device__ __forceinline__ double block_sum_d(double v, double* red) {
@@ -143,11 +144,11 @@ __global__ void __launch_bounds__(256) norm_quant_kernel(const NormQuantArgs a) 
     } else if (MODE == kRowGlu) {
       const float gate = load_as_float(a.x, row * a.ldx + c, a.xdt);
       const float up = load_as_float(a.x, row * a.ldx + k + c, a.xdt);
-      v = siluf_(gate) * up;
+      v = (a.pre_act ? gate : siluf_(gate)) * up;
     } else {
       const double hv = load_as_float(a.x, row * a.ldx + c, a.xdt);
       const float gv = load_as_float(a.g, row * a.ldg + c, a.gdt);
-      v = (float)(hv * rinv_h * (double)(a.gw ? a.gw[c] : 1.0f)) * siluf_(gv);
+      v = (float)(hv * rinv_h * (double)(a.gw ? a.gw[c] : 1.0f)) * (a.pre_act ? gv : siluf_(gv));
     }
     vrow[c] = v;
     ss += (double)v * (double)v;
@@ -176,6 +177,208 @@ __global__ void __launch_bounds__(256) norm_quant_kernel(const NormQuantArgs a) 
   }
 }
 
+// Vectorised variant for K % 8 == 0 and 16-byte aligned rows (K <= 8192): a row group of W
+// warps owns one row and keeps it in registers (at most 4 chunks of 8 values per thread), loads
+// and stores whole 16-/8-byte pieces and reduces with shuffles (plus one double-buffered shared
+// exchange per reduction when W > 1). Arithmetic is that of norm_quant_kernel.
+constexpr int kNqThreads = 256;
+constexpr int kNqMaxChunks = 4;
+
+template <int W>
+__device__ __forceinline__ double nq_group_sum(double v, double (*red)[8], int& ph) {
+  v = warp_sum_d(v);
+  if (W == 1) return v;
+  const int wid = threadIdx.x >> 5, g0 = (wid / W) * W;
+  double* r = red[ph & 1];
+  ++ph;
+  if ((threadIdx.x & 31) == 0) r[wid] = v;
+  __syncthreads();
+  double s = 0.0;
+#pragma unroll
+  for (int k = 0; k < W; ++k) s += r[g0 + k];
+  return s;
+}
+// Maxima of three values over the row group (one exchange for all gains).
+template <int W>
+__device__ __forceinline__ void nq_group_max3(float (&v)[3], float (*red)[8][3], int& ph) {
+#pragma unroll
+  for (int j = 0; j < 3; ++j) v[j] = warp_max(v[j]);
+  if (W == 1) return;
+  const int wid = threadIdx.x >> 5, g0 = (wid / W) * W;
+  float(*r)[3] = red[ph & 1];
+  ++ph;
+  if ((threadIdx.x & 31) == 0) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j) r[wid][j] = v[j];
+  }
+  __syncthreads();
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    float m = 0.0f;
+#pragma unroll
+    for (int k = 0; k < W; ++k) m = fmaxf(m, r[g0 + k][j]);
+    v[j] = m;
+  }
+}
+
+template <mmf_dtype DT>
+__device__ __forceinline__ void load8(const void* base, int64_t idx, float (&o)[8]) {
+  if (DT == MMF_BF16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w[q]));
+      o[2 * q] = f.x;
+      o[2 * q + 1] = f.y;
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(base) + idx + 4);
+    o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+    o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+  }
+}
+__device__ __forceinline__ void load8_gain(const float* g, int64_t idx, float (&o)[8]) {
+  if (!g) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) o[e] = 1.0f;
+    return;
+  }
+  const float4 a = __ldg(reinterpret_cast<const float4*>(g + idx));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(g + idx + 4));
+  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
+  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
+}
+// r = float32(v * g * rinv) with rinv = 1/rms given as a float64 split rh + rl (rl = rinv - rh).
+// Double-float arithmetic: v*g and (v*g)*rh are formed exactly as hi + lo pairs with FMA, the
+// remaining terms are added, and the sum is rounded once, so r is the float32 rounding of the
+// product to within ~2^-44 relative, the same value a float64 evaluation rounds to (barring a
+// product that lies that close to a float32 rounding boundary).
+__device__ __forceinline__ float nq_r(float v, float g, float rh, float rl) {
+  const float p = __fmul_rn(v, g);
+  const float pe = fmaf(v, g, -p);
+  const float q = __fmul_rn(p, rh);
+  const float qe = fmaf(p, rh, -q);
+  return __fadd_rn(q, fmaf(p, rl, fmaf(pe, rh, qe)));
+}
+__device__ __forceinline__ void nq_split(double rinv, float& rh, float& rl) {
+  rh = (float)rinv;
+  rl = (float)(rinv - (double)rh);
+}
+
+// Row group of W warps per row, NCH chunks of 8 values per thread (K <= 256 * W * NCH).
+template <mmf_dtype XT, int MODE, int W, int NCH>
+__global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQuantArgs a) {
+  constexpr int GT = 32 * W;
+  __shared__ double redd[2][8];
+  __shared__ float redf[2][8][3];
+  int phd = 0, phf = 0;
+  const int grp = (threadIdx.x >> 5) / W;
+  const int gl = threadIdx.x - grp * GT;
+  const int64_t row = (int64_t)blockIdx.x * (8 / W) + grp;
+  const bool active = row < a.m;
+  const int k = a.k, nck = k >> 3;
+  float v[NCH][8];
+  double ss = 0.0;
+  if (MODE == kRowGnorm) {
+    float g[NCH][8];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = gl + i * GT;
+      if (active && c < nck) {
+        load8<XT>(a.x, row * a.ldx + 8 * c, v[i]);
+        load8<XT>(a.g, row * a.ldg + 8 * c, g[i]);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss += (double)v[i][e] * (double)v[i][e];
+      }
+    }
+    const double rinv_h = 1.0 / sqrt(nq_group_sum<W>(ss, redd, phd) / (double)k + (double)a.eps);
+    float rhh, rlh;
+    nq_split(rinv_h, rhh, rlh);
+    ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = gl + i * GT;
+      if (active && c < nck) {
+        float gw[8];
+        load8_gain(a.gw, 8 * c, gw);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          v[i][e] = nq_r(v[i][e], gw[e], rhh, rlh) * (a.pre_act ? g[i][e] : siluf_(g[i][e]));
+          ss += (double)v[i][e] * (double)v[i][e];
+        }
+      }
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = gl + i * GT;
+      if (active && c < nck) {
+        if (MODE == kRowPlain) {
+          load8<XT>(a.x, row * a.ldx + 8 * c, v[i]);
+        } else {
+          float up[8];
+          load8<XT>(a.x, row * a.ldx + 8 * c, v[i]);
+          load8<XT>(a.x, row * a.ldx + k + 8 * c, up);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[i][e] = (a.pre_act ? v[i][e] : siluf_(v[i][e])) * up[e];
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss += (double)v[i][e] * (double)v[i][e];
+      }
+    }
+  }
+  const double rinv = 1.0 / sqrt(nq_group_sum<W>(ss, redd, phd) / (double)k + (double)a.eps);
+  float rh, rl;
+  nq_split(rinv, rh, rl);
+  // maxima of |r| for every gain in one pass and one exchange
+  float amax[3] = {0.0f, 0.0f, 0.0f};
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    if (j < a.ngain) {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int c = gl + i * GT;
+        if (active && c < nck) {
+          float gg[8];
+          load8_gain(a.gain[j], 8 * c, gg);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) amax[j] = fmaxf(amax[j], fabsf(nq_r(v[i][e], gg[e], rh, rl)));
+        }
+      }
+    }
+  }
+  nq_group_max3<W>(amax, redf, phf);
+  if (!active) return;
+#pragma unroll
+  for (int j = 0; j < 3; ++j) {
+    if (j < a.ngain) {
+      const float* gn = a.gain[j];
+      const float am = fmaxf(amax[j], 1e-5f);
+      const float sx = __fdiv_rn(127.0f, am);
+      int8_t* qrow = a.q[j] + row * a.ldq;
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+        const int c = gl + i * GT;
+        if (c < nck) {
+          float gg[8];
+          load8_gain(gn, 8 * c, gg);
+          uint32_t w[2] = {0u, 0u};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int qv = (int)fminf(fmaxf(rintf(__fmul_rn(nq_r(v[i][e], gg[e], rh, rl), sx)), -127.0f), 127.0f);
+            w[e >> 2] |= ((uint32_t)qv & 0xFFu) << (8 * (e & 3));
+          }
+          *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(w[0], w[1]);
+        }
+      }
+      for (int c = nck + gl; c < (int)(a.ldq >> 3); c += GT) *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(0u, 0u);
+      if (gl == 0) a.deq[j][row] = __fdiv_rn(am, 127.0f);
+    }
+  }
+}
+
 // =============================================================================================
 // BitLinear segments (shared by both integer-product engines)
 // =============================================================================================
@@ -193,6 +396,8 @@ struct GemmSeg {
   int32_t rescol;
   int32_t* acc;          // optional raw accumulators acc[row * ldacc + col]
   int64_t ldacc;
+  int32_t act;           // activation applied to output columns [0, act_cols): kActNone/Silu/SigmoidNeg
+  int32_t act_cols;
 };
 
 struct GemmArgs {
@@ -205,12 +410,26 @@ struct GemmArgs {
   mmf_dtype ydt;
 };
 
-// y = acc * deq[row] * s (+ residual), plus the optional raw accumulator.
+// Element-wise activations a BitLinear epilogue can apply to its output (the gates that follow
+// the projections in the block, evaluated once where the value is produced).
+enum ActKind : int32_t {
+  kActNone = 0,
+  kActSilu = 1,        // SiLU(z) = z * sigmoid(z)
+  kActSigmoidNeg = 2   // sigmoid(-z) = 1 - sigmoid(z), the forget gate's complement
+};
+__device__ __forceinline__ float apply_act(int32_t act, float z) {
+  if (act == kActSilu) return siluf_(z);
+  if (act == kActSigmoidNeg) return __fdividef(1.0f, 1.0f + __expf(z));
+  return z;
+}
+
+// y = act(acc * deq[row] * s (+ residual)), plus the optional raw accumulator.
 __device__ __forceinline__ void bitlinear_epilogue(const GemmSeg& s, mmf_dtype ydt, int64_t row,
                                                    int32_t col, int32_t acc, float sw) {
   if (s.acc) s.acc[row * s.ldacc + col] = acc;
   float z = (float)acc * (s.deq[row] * sw);  // same rounding order as the tensor-core epilogue
   if (s.res) z += load_as_float(s.res, row * s.ldres + s.rescol + col, ydt);
+  if (col < s.act_cols) z = apply_act(s.act, z);
   store_from_float(s.y, row * s.ldy + s.ycol + col, ydt, z);
 }
 
@@ -285,16 +504,15 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const GemmArgs a) {
 }
 
 // =============================================================================================
-// K4: HGRN scan with fused gates
+// K4: HGRN scan with fused gates (chunked: aggregate -> carry -> replay)
 // =============================================================================================
-// CTA = 32 channels (lanes) x kScanWarps warps. The sequence is processed in segments of
-// kScanWarps * kScanL steps; warp w owns steps [w*L, (w+1)*L) of a segment. Each warp folds its
-// steps into an affine map (A, B) (h -> A h + B), the maps are published in shared memory, each
-// warp composes the maps of the warps before it onto the segment's carry, then replays its own
-// steps sequentially from that carry and stores h.
-constexpr int kScanWarps = 16;
-constexpr int kScanL = 8;
-
+// The step h -> f h + i is affine, so a run of steps composes to h -> A h + B. The sequence is
+// cut into chunks of `chunk` steps. Phase 1 folds every (channel, chunk) into its (A, B);
+// phase 2 walks the chunks of each channel in order and records the state entering each chunk
+// (and the final state); phase 3 replays every chunk from its entry state and stores h. Each
+// thread owns VEC adjacent channels (paired 4- or 8-byte loads), lanes cover consecutive channel
+// pairs, so every access is a coalesced row segment. Sequences no longer than one chunk (decode)
+// take the single-pass kernel instead.
 struct ScanArgs {
   const void* zf;
   const void* zi;
@@ -307,59 +525,284 @@ struct ScanArgs {
   void* h;          // [b][t][d]
   mmf_dtype hdt;
   float* h_last;
+  int32_t chunk;    // steps per chunk
+  int32_t nchunk;
+  float* agg_a;     // [b][nchunk][d]
+  float* agg_b;     // [b][nchunk][d]
+  float* cin;       // [b][nchunk][d] state entering each chunk
+  int32_t gated;    // 0: zf, zi are gate pre-activations; 1: zf holds 1 - f, zi holds SiLU(zi)
 };
+constexpr int kScanThreads = 128;
 
-__global__ void __launch_bounds__(kScanWarps * 32) hgrn_scan_kernel(const ScanArgs a) {
-  __shared__ float sA[kScanWarps][32];
-  __shared__ float sB[kScanWarps][32];
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int64_t ch = (int64_t)blockIdx.x * 32 + lane;
-  const bool valid = ch < (int64_t)a.b * a.d;
-  const int64_t bi = valid ? ch / a.d : 0;
-  const int64_t c = valid ? ch - bi * a.d : 0;
-  const int64_t zbase = bi * a.t * a.zstride + c;
-  const int64_t hbase = bi * a.t * a.d + c;
-  float carry = (valid && a.h0) ? a.h0[bi * a.d + c] : 0.0f;
-  for (int64_t seg0 = 0; seg0 < a.t; seg0 += kScanWarps * kScanL) {
-    const int64_t t0 = seg0 + (int64_t)warp * kScanL;
-    float f[kScanL], in[kScanL];
+template <mmf_dtype DT, int VEC>
+__device__ __forceinline__ void load_vec(const void* base, int64_t idx, float (&o)[VEC]) {
+  if (VEC == 2) {
+    if (DT == MMF_F32) {
+      const float2 v = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(base) + idx);
+      o[0] = v.x;
+      o[VEC - 1] = v.y;
+    } else {
+      const float2 v = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(
+          reinterpret_cast<const __nv_bfloat16*>(base) + idx));
+      o[0] = v.x;
+      o[VEC - 1] = v.y;
+    }
+  } else {
+    o[0] = Elem<DT>::load(reinterpret_cast<const typename Elem<DT>::T*>(base) + idx);
+  }
+}
+template <mmf_dtype DT, int VEC>
+__device__ __forceinline__ void store_vec(void* base, int64_t idx, const float (&v)[VEC]) {
+  if (VEC == 2) {
+    if (DT == MMF_F32)
+      *reinterpret_cast<float2*>(reinterpret_cast<float*>(base) + idx) = make_float2(v[0], v[VEC - 1]);
+    else
+      *reinterpret_cast<__nv_bfloat162*>(reinterpret_cast<__nv_bfloat16*>(base) + idx) =
+          __floats2bfloat162_rn(v[0], v[VEC - 1]);
+  } else {
+    Elem<DT>::store(reinterpret_cast<typename Elem<DT>::T*>(base) + idx, v[0]);
+  }
+}
+
+// f = sigmoid(zf), i = SiLU(zi) * (1 - f); with GATED the inputs already are (1 - f, SiLU(zi)).
+template <bool GATED>
+__device__ __forceinline__ void hgrn_gate(float zf, float zi, float& f, float& i) {
+  if (GATED) {
+    f = 1.0f - zf;
+    i = zi * zf;
+  } else {
+    float omf;
+    hgrn_forget(zf, f, omf);
+    i = siluf_(zi) * omf;
+  }
+}
+
+// Steps loaded ahead into registers before the dependent recurrence runs over them.
+constexpr int kScanPrefetch = 16;  // = the chunk length for sequences up to 2048 steps
+
+template <mmf_dtype ZT, int VEC>
+__device__ __forceinline__ void scan_load_block(const ScanArgs& a, int64_t zb, int64_t t, int64_t t1,
+                                                float (&zf)[kScanPrefetch][VEC], float (&zi)[kScanPrefetch][VEC]) {
 #pragma unroll
-    for (int s = 0; s < kScanL; ++s) {
-      const int64_t t = t0 + s;
-      if (valid && t < a.t) {
-        const float zf = load_as_float(a.zf, zbase + t * a.zstride, a.zdt);
-        const float zi = load_as_float(a.zi, zbase + t * a.zstride, a.zdt);
-        const float fg = sigmoidf_(zf);
-        f[s] = fg;
-        in[s] = siluf_(zi) * (1.0f - fg);
-      } else {
-        f[s] = 1.0f;  // identity step
-        in[s] = 0.0f;
+  for (int u = 0; u < kScanPrefetch; ++u) {
+    if (t + u < t1) {
+      load_vec<ZT, VEC>(a.zf, zb + (t + u) * a.zstride, zf[u]);
+      load_vec<ZT, VEC>(a.zi, zb + (t + u) * a.zstride, zi[u]);
+    }
+  }
+}
+
+template <mmf_dtype ZT, int VEC, bool GATED>
+__global__ void __launch_bounds__(kScanThreads) scan_aggregate_kernel(const ScanArgs a) {
+  const int64_t ch = ((int64_t)blockIdx.x * kScanThreads + threadIdx.x) * VEC;
+  if (ch >= a.d) return;
+  const int c = blockIdx.y, bi = blockIdx.z;
+  const int64_t t0 = (int64_t)c * a.chunk;
+  const int64_t t1 = t0 + a.chunk < a.t ? t0 + a.chunk : a.t;
+  const int64_t zb = (int64_t)bi * a.t * a.zstride + ch;
+  float A[VEC], B[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) { A[v] = 1.0f; B[v] = 0.0f; }
+  for (int64_t t = t0; t < t1; t += kScanPrefetch) {
+    float zf[kScanPrefetch][VEC], zi[kScanPrefetch][VEC];
+    scan_load_block<ZT, VEC>(a, zb, t, t1, zf, zi);
+#pragma unroll
+    for (int u = 0; u < kScanPrefetch; ++u) {
+      if (t + u < t1) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          float f, i;
+          hgrn_gate<GATED>(zf[u][v], zi[u][v], f, i);
+          A[v] = f * A[v];
+          B[v] = f * B[v] + i;
+        }
       }
     }
-    float A = 1.0f, B = 0.0f;
-#pragma unroll
-    for (int s = 0; s < kScanL; ++s) {
-      A = f[s] * A;
-      B = f[s] * B + in[s];
-    }
-    sA[warp][lane] = A;
-    sB[warp][lane] = B;
-    __syncthreads();
-    float h = carry;
-    for (int w = 0; w < warp; ++w) h = sA[w][lane] * h + sB[w][lane];
-#pragma unroll
-    for (int s = 0; s < kScanL; ++s) {
-      h = f[s] * h + in[s];
-      const int64_t t = t0 + s;
-      if (valid && t < a.t) store_from_float(a.h, hbase + t * a.d, a.hdt, h);
-    }
-    float cnext = carry;
-    for (int w = 0; w < kScanWarps; ++w) cnext = sA[w][lane] * cnext + sB[w][lane];
-    carry = cnext;
-    __syncthreads();
   }
-  if (valid && warp == 0 && a.h_last) a.h_last[bi * a.d + c] = carry;
+  const int64_t o = ((int64_t)bi * a.nchunk + c) * a.d + ch;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    a.agg_a[o + v] = A[v];
+    a.agg_b[o + v] = B[v];
+  }
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_carry_kernel(const ScanArgs a) {
+  const int64_t ch = (int64_t)blockIdx.x * kScanThreads + threadIdx.x;
+  if (ch >= a.d) return;
+  const int bi = blockIdx.y;
+  const float* __restrict__ A = a.agg_a;
+  const float* __restrict__ B = a.agg_b;
+  float* __restrict__ cin = a.cin;
+  float carry = a.h0 ? a.h0[(int64_t)bi * a.d + ch] : 0.0f;
+  const int64_t base = (int64_t)bi * a.nchunk * a.d + ch;
+  constexpr int PF = 32;
+  for (int c0 = 0; c0 < a.nchunk; c0 += PF) {
+    float av[PF], bv[PF];
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      if (c0 + u < a.nchunk) {
+        av[u] = A[base + (int64_t)(c0 + u) * a.d];
+        bv[u] = B[base + (int64_t)(c0 + u) * a.d];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      if (c0 + u < a.nchunk) {
+        cin[base + (int64_t)(c0 + u) * a.d] = carry;
+        carry = av[u] * carry + bv[u];
+      }
+    }
+  }
+  if (a.h_last) a.h_last[(int64_t)bi * a.d + ch] = carry;
+}
+
+// Replays chunk c from its entry state (phase 3); with SINGLE the whole sequence is one chunk
+// entered from h0 and the final state is written too.
+template <mmf_dtype ZT, mmf_dtype HT, int VEC, bool SINGLE, bool GATED>
+__global__ void __launch_bounds__(kScanThreads) scan_apply_kernel(const ScanArgs a) {
+  const int64_t ch = ((int64_t)blockIdx.x * kScanThreads + threadIdx.x) * VEC;
+  if (ch >= a.d) return;
+  const int c = blockIdx.y, bi = blockIdx.z;
+  const int64_t t0 = (int64_t)c * a.chunk;
+  const int64_t t1 = t0 + a.chunk < a.t ? t0 + a.chunk : a.t;
+  const int64_t zb = (int64_t)bi * a.t * a.zstride + ch;
+  const int64_t hb = (int64_t)bi * a.t * a.d + ch;
+  float h[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    if (SINGLE) h[v] = a.h0 ? a.h0[(int64_t)bi * a.d + ch + v] : 0.0f;
+    else h[v] = a.cin[((int64_t)bi * a.nchunk + c) * a.d + ch + v];
+  }
+  for (int64_t t = t0; t < t1; t += kScanPrefetch) {
+    float zf[kScanPrefetch][VEC], zi[kScanPrefetch][VEC];
+    scan_load_block<ZT, VEC>(a, zb, t, t1, zf, zi);
+#pragma unroll
+    for (int u = 0; u < kScanPrefetch; ++u) {
+      if (t + u < t1) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          float f, i;
+          hgrn_gate<GATED>(zf[u][v], zi[u][v], f, i);
+          h[v] = f * h[v] + i;
+        }
+        store_vec<HT, VEC>(a.h, hb + (t + u) * a.d, h);
+      }
+    }
+  }
+  if (SINGLE && a.h_last) {
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) a.h_last[(int64_t)bi * a.d + ch + v] = h[v];
+  }
+}
+
+// Tiled variant of the aggregate / apply / single-pass phases for 16-byte aligned rows: a CTA of
+// kScanThreads threads owns kScanTileCh channels (two per thread) and streams its chunk through
+// shared memory in tiles of kScanTileSteps steps with double-buffered cp.async copies, so many
+// KB per SM are in flight without holding them in registers.
+constexpr int kScanTileCh = 2 * kScanThreads;  // 256 channels per CTA
+constexpr int kScanTileSteps = 16;
+
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+template <mmf_dtype ZT>
+constexpr int scan_tile_bytes() {
+  return 2 /*stages*/ * 2 /*zf, zi*/ * kScanTileSteps * kScanTileCh * (ZT == MMF_F32 ? 4 : 2);
+}
+
+// PHASE 0: aggregates; 1: replay from the chunk's entry state; 2: single chunk from h0 (+ h_last).
+template <mmf_dtype ZT, mmf_dtype HT, bool GATED, int PHASE>
+__global__ void __launch_bounds__(kScanThreads) scan_tile_kernel(const ScanArgs a) {
+  constexpr int ES = ZT == MMF_F32 ? 4 : 2;
+  constexpr int ROWB = kScanTileCh * ES;                    // bytes of one step row of one array
+  constexpr int PIECES = 2 * kScanTileSteps * ROWB / 16;    // 16-byte copies per stage
+  extern __shared__ __align__(16) uint8_t scan_sm[];
+  const int tid = threadIdx.x;
+  const int64_t ch0 = (int64_t)blockIdx.x * kScanTileCh;
+  const int c = blockIdx.y, bi = blockIdx.z;
+  const int64_t t0 = (int64_t)c * a.chunk;
+  const int64_t t1 = t0 + a.chunk < a.t ? t0 + a.chunk : a.t;
+  const int nblk = (int)((t1 - t0 + kScanTileSteps - 1) / kScanTileSteps);
+  const int64_t row_bytes_valid = (a.d - ch0) * ES < ROWB ? (a.d - ch0) * ES : ROWB;
+  const uint8_t* zfb = reinterpret_cast<const uint8_t*>(a.zf);
+  const uint8_t* zib = reinterpret_cast<const uint8_t*>(a.zi);
+
+  auto issue = [&](int stage, int blk) {
+    uint8_t* dst0 = scan_sm + stage * (2 * kScanTileSteps * ROWB);
+    for (int p = tid; p < PIECES; p += kScanThreads) {
+      const int arr = p / (PIECES / 2);
+      const int rem = p - arr * (PIECES / 2);
+      const int u = rem / (ROWB / 16), col = (rem - u * (ROWB / 16)) * 16;
+      const int64_t t = t0 + (int64_t)blk * kScanTileSteps + u;
+      if (t < t1 && col < row_bytes_valid) {
+        const uint8_t* src = (arr ? zib : zfb) + (((int64_t)bi * a.t + t) * a.zstride + ch0) * ES + col;
+        cp_async16(dst0 + (arr * kScanTileSteps + u) * ROWB + col, src);
+      }
+    }
+    cp_async_commit();
+  };
+
+  const int64_t ch = ch0 + 2 * tid;
+  const bool valid = ch < a.d;  // d is even on this path
+  float A0 = 1.0f, A1 = 1.0f, B0 = 0.0f, B1 = 0.0f, h0v = 0.0f, h1v = 0.0f;
+  if (valid) {
+    if (PHASE == 1) {
+      const int64_t o = ((int64_t)bi * a.nchunk + c) * a.d + ch;
+      h0v = a.cin[o];
+      h1v = a.cin[o + 1];
+    } else if (PHASE == 2 && a.h0) {
+      h0v = a.h0[(int64_t)bi * a.d + ch];
+      h1v = a.h0[(int64_t)bi * a.d + ch + 1];
+    }
+  }
+  issue(0, 0);
+  for (int blk = 0; blk < nblk; ++blk) {
+    if (blk + 1 < nblk) {
+      issue((blk + 1) & 1, blk + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
+    }
+    __syncthreads();
+    const uint8_t* st = scan_sm + (blk & 1) * (2 * kScanTileSteps * ROWB);
+    const int64_t tb = t0 + (int64_t)blk * kScanTileSteps;
+    const int steps = t1 - tb < kScanTileSteps ? (int)(t1 - tb) : kScanTileSteps;
+    if (valid) {
+#pragma unroll 4
+      for (int u = 0; u < steps; ++u) {
+        float zf[2], zi[2];
+        load_vec<ZT, 2>(st + (0 * kScanTileSteps + u) * ROWB, 2 * tid, zf);
+        load_vec<ZT, 2>(st + (1 * kScanTileSteps + u) * ROWB, 2 * tid, zi);
+        float f0, i0, f1, i1;
+        hgrn_gate<GATED>(zf[0], zi[0], f0, i0);
+        hgrn_gate<GATED>(zf[1], zi[1], f1, i1);
+        if (PHASE == 0) {
+          A0 *= f0; B0 = f0 * B0 + i0;
+          A1 *= f1; B1 = f1 * B1 + i1;
+        } else {
+          h0v = f0 * h0v + i0;
+          h1v = f1 * h1v + i1;
+          const float hv[2] = {h0v, h1v};
+          store_vec<HT, 2>(a.h, ((int64_t)bi * a.t + tb + u) * a.d + ch, hv);
+        }
+      }
+    }
+    __syncthreads();  // the stage is refilled by the next iteration's copies
+  }
+  if (!valid) return;
+  if (PHASE == 0) {
+    const int64_t o = ((int64_t)bi * a.nchunk + c) * a.d + ch;
+    a.agg_a[o] = A0; a.agg_a[o + 1] = A1;
+    a.agg_b[o] = B0; a.agg_b[o + 1] = B1;
+  } else if (PHASE == 2 && a.h_last) {
+    a.h_last[(int64_t)bi * a.d + ch] = h0v;
+    a.h_last[(int64_t)bi * a.d + ch + 1] = h1v;
+  }
 }
 
 // =============================================================================================

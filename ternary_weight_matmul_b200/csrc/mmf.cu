@@ -72,6 +72,22 @@ struct DevInfo {
 DevInfo g_dev[64];
 std::mutex g_dev_mu;
 
+template <mmf_dtype ZT, mmf_dtype HT>
+cudaError_t scan_tile_attrs() {
+  cudaError_t e = cudaSuccess;
+  const int smem = scan_tile_bytes<ZT>();
+  auto set = [&](const void* f) {
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  };
+  set((const void*)scan_tile_kernel<ZT, HT, false, 0>);
+  set((const void*)scan_tile_kernel<ZT, HT, false, 1>);
+  set((const void*)scan_tile_kernel<ZT, HT, false, 2>);
+  set((const void*)scan_tile_kernel<ZT, HT, true, 0>);
+  set((const void*)scan_tile_kernel<ZT, HT, true, 1>);
+  set((const void*)scan_tile_kernel<ZT, HT, true, 2>);
+  return e;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -98,6 +114,10 @@ mmf_status device_info(DevInfo** out) {
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
       MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowGnorm>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
+      MMF_CUDA((scan_tile_attrs<MMF_F32, MMF_F32>()));
+      MMF_CUDA((scan_tile_attrs<MMF_F32, MMF_BF16>()));
+      MMF_CUDA((scan_tile_attrs<MMF_BF16, MMF_F32>()));
+      MMF_CUDA((scan_tile_attrs<MMF_BF16, MMF_BF16>()));
       di.tc_ready = true;
     }
     di.init = true;
@@ -195,15 +215,50 @@ struct LaunchScope {
 // ---------------------------------------------------------------------------------------------
 // internal launchers
 // ---------------------------------------------------------------------------------------------
+template <mmf_dtype XT, int MODE>
+void nq_vec_launch(const NormQuantArgs& a, int w, int nch, cudaStream_t st) {
+  const unsigned rows_per_cta = 8u / (unsigned)w;
+  const dim3 grid((unsigned)((a.m + rows_per_cta - 1) / rows_per_cta));
+  if (w == 1) norm_quant_vec_kernel<XT, MODE, 1, 2><<<grid, kNqThreads, 0, st>>>(a);
+  else if (w == 2) norm_quant_vec_kernel<XT, MODE, 2, 2><<<grid, kNqThreads, 0, st>>>(a);
+  else if (w == 4) norm_quant_vec_kernel<XT, MODE, 4, 2><<<grid, kNqThreads, 0, st>>>(a);
+  else if (nch <= 2) norm_quant_vec_kernel<XT, MODE, 8, 2><<<grid, kNqThreads, 0, st>>>(a);
+  else norm_quant_vec_kernel<XT, MODE, 8, 4><<<grid, kNqThreads, 0, st>>>(a);
+}
+
+template <mmf_dtype XT>
+void nq_vec_dispatch(const NormQuantArgs& a, int mode, int w, int nch, cudaStream_t st) {
+  if (mode == kRowPlain) nq_vec_launch<XT, kRowPlain>(a, w, nch, st);
+  else if (mode == kRowGlu) nq_vec_launch<XT, kRowGlu>(a, w, nch, st);
+  else nq_vec_launch<XT, kRowGnorm>(a, w, nch, st);
+}
+
+inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 mmf_status launch_norm_quant(const NormQuantArgs& a, int mode, cudaStream_t st) {
   if (a.m == 0) return MMF_OK;
-  const size_t smem = (size_t)a.k * sizeof(float);
-  const int threads = a.k >= 2048 ? 256 : 128;
-  dim3 grid((unsigned)a.m);
   const double es = a.xdt == MMF_F32 ? 4.0 : 2.0;
   double in_row = (mode == kRowGlu ? 2.0 : 1.0) * a.k * es;
   if (mode == kRowGnorm) in_row += a.k * (a.gdt == MMF_F32 ? 4.0 : 2.0);
   LaunchScope ls(MMF_KERNEL_NORM_QUANT, (double)a.m * (in_row + a.ngain * ((double)a.ldq + 4.0)), st);
+  // row-group-in-registers variant when sizes and alignment allow it
+  const size_t xes = dsize(a.xdt);
+  bool vec = a.k % 8 == 0 && a.k <= 8 * 32 * 8 * kNqMaxChunks && al16(a.x) && (a.ldx * xes) % 16 == 0;
+  if (mode == kRowGnorm)
+    vec = vec && a.gdt == a.xdt && al16(a.g) && (a.ldg * xes) % 16 == 0 && al16(a.gw);
+  for (int j = 0; j < a.ngain; ++j) vec = vec && al16(a.gain[j]) && al16(a.q[j]);
+  if (vec) {
+    // smallest row group holding the row at two 8-value chunks per thread (four beyond 4096)
+    const int nck = a.k / 8;
+    const int w = nck <= 64 ? 1 : nck <= 128 ? 2 : nck <= 256 ? 4 : 8;
+    const int nch = (nck + 32 * w - 1) / (32 * w);
+    if (a.xdt == MMF_F32) nq_vec_dispatch<MMF_F32>(a, mode, w, nch, st);
+    else nq_vec_dispatch<MMF_BF16>(a, mode, w, nch, st);
+    return check_launch("norm_quant_vec_kernel");
+  }
+  const size_t smem = (size_t)a.k * sizeof(float);
+  const int threads = a.k >= 2048 ? 256 : 128;
+  dim3 grid((unsigned)a.m);
   if (mode == kRowPlain) norm_quant_kernel<kRowPlain><<<grid, threads, smem, st>>>(a);
   else if (mode == kRowGlu) norm_quant_kernel<kRowGlu><<<grid, threads, smem, st>>>(a);
   else norm_quant_kernel<kRowGnorm><<<grid, threads, smem, st>>>(a);
@@ -265,10 +320,69 @@ mmf_status launch_gemm(const GemmArgs& g, const DevInfo& di, cudaStream_t st) {
   return check_launch("ternary_gemm_tc_kernel");
 }
 
-mmf_status launch_scan(const ScanArgs& a, cudaStream_t st) {
+// Steps per chunk of the chunked scan: 16 (one register prefetch block per thread) up to 2048
+// steps, then a multiple of 16 giving at most 128 chunks.
+inline int32_t scan_chunk(int64_t t) {
+  if (t <= 2048) return 16;
+  const int64_t c = (t + 127) / 128;
+  return (int32_t)((c + 15) / 16 * 16);
+}
+// Scratch of the chunked scan for m = b*t tokens of d channels: three [b][nchunk][d] float
+// arrays. b * nchunk <= ceil(m / 8) whenever t > 16 (shorter sequences need no scratch):
+// t <= 2048 gives nchunk = ceil(t/16) < t/8, longer ones nchunk <= 128 < t/16.
+inline size_t scan_ws_bytes(int64_t m, int32_t d) {
+  return 3 * align256((size_t)d * 4 * (size_t)((m + 7) / 8));
+}
+
+template <mmf_dtype ZT, mmf_dtype HT, int VEC, bool GATED>
+void scan_launch_gated(const ScanArgs& a, cudaStream_t st) {
+  const unsigned gx = (unsigned)((a.d / VEC + kScanThreads - 1) / kScanThreads);
+  if (a.nchunk == 1) {
+    scan_apply_kernel<ZT, HT, VEC, true, GATED><<<dim3(gx, 1, a.b), kScanThreads, 0, st>>>(a);
+    return;
+  }
+  scan_aggregate_kernel<ZT, VEC, GATED><<<dim3(gx, a.nchunk, a.b), kScanThreads, 0, st>>>(a);
+  scan_carry_kernel<<<dim3((unsigned)((a.d + kScanThreads - 1) / kScanThreads), a.b), kScanThreads, 0, st>>>(a);
+  scan_apply_kernel<ZT, HT, VEC, false, GATED><<<dim3(gx, a.nchunk, a.b), kScanThreads, 0, st>>>(a);
+}
+
+template <mmf_dtype ZT, mmf_dtype HT, int VEC>
+void scan_launch_typed(const ScanArgs& a, cudaStream_t st) {
+  if (a.gated) scan_launch_gated<ZT, HT, VEC, true>(a, st);
+  else scan_launch_gated<ZT, HT, VEC, false>(a, st);
+}
+
+// Tiled (shared-memory staged) phases; needs 16-byte aligned rows and an even channel count.
+template <mmf_dtype ZT, mmf_dtype HT, bool GATED>
+void scan_tiled_gated(const ScanArgs& a, cudaStream_t st) {
+  constexpr int smem = scan_tile_bytes<ZT>();
+  const unsigned gx = (unsigned)((a.d + kScanTileCh - 1) / kScanTileCh);
+  if (a.nchunk == 1) {
+    scan_tile_kernel<ZT, HT, GATED, 2><<<dim3(gx, 1, a.b), kScanThreads, smem, st>>>(a);
+    return;
+  }
+  scan_tile_kernel<ZT, HT, GATED, 0><<<dim3(gx, a.nchunk, a.b), kScanThreads, smem, st>>>(a);
+  scan_carry_kernel<<<dim3((unsigned)((a.d + kScanThreads - 1) / kScanThreads), a.b), kScanThreads, 0, st>>>(a);
+  scan_tile_kernel<ZT, HT, GATED, 1><<<dim3(gx, a.nchunk, a.b), kScanThreads, smem, st>>>(a);
+}
+template <mmf_dtype ZT, mmf_dtype HT>
+void scan_tiled_typed(const ScanArgs& a, cudaStream_t st) {
+  if (a.gated) scan_tiled_gated<ZT, HT, true>(a, st);
+  else scan_tiled_gated<ZT, HT, false>(a, st);
+}
+
+template <int VEC>
+void scan_launch_vec(const ScanArgs& a, cudaStream_t st) {
+  if (a.zdt == MMF_F32 && a.hdt == MMF_F32) scan_launch_typed<MMF_F32, MMF_F32, VEC>(a, st);
+  else if (a.zdt == MMF_F32) scan_launch_typed<MMF_F32, MMF_BF16, VEC>(a, st);
+  else if (a.hdt == MMF_F32) scan_launch_typed<MMF_BF16, MMF_F32, VEC>(a, st);
+  else scan_launch_typed<MMF_BF16, MMF_BF16, VEC>(a, st);
+}
+
+// ws: scan_ws_bytes(b*t, d) bytes (unused when t <= 16).
+mmf_status launch_scan(ScanArgs a, void* ws, cudaStream_t st) {
   if ((int64_t)a.b * a.d == 0) return MMF_OK;
   const int64_t chans = (int64_t)a.b * a.d;
-  dim3 grid((unsigned)((chans + 31) / 32));
   if (a.t == 0) {
     // no steps: the final state is the initial one
     if (a.h_last) {
@@ -282,11 +396,40 @@ mmf_status launch_scan(const ScanArgs& a, cudaStream_t st) {
     }
     return MMF_OK;
   }
-  const double zes = a.zdt == MMF_F32 ? 4.0 : 2.0, hes = a.hdt == MMF_F32 ? 4.0 : 2.0;
-  LaunchScope ls(MMF_KERNEL_SCAN, (double)chans * a.t * (2.0 * zes + hes) + (double)chans * 4.0 *
+  if (a.t <= 16) {
+    a.chunk = (int32_t)a.t;
+    a.nchunk = 1;
+  } else {
+    a.chunk = scan_chunk(a.t);
+    a.nchunk = (int32_t)((a.t + a.chunk - 1) / a.chunk);
+    const size_t arr = align256((size_t)a.d * 4 * (size_t)(((int64_t)a.b * a.t + 7) / 8));
+    uint8_t* p = reinterpret_cast<uint8_t*>(ws);
+    a.agg_a = reinterpret_cast<float*>(p);
+    a.agg_b = reinterpret_cast<float*>(p + arr);
+    a.cin = reinterpret_cast<float*>(p + 2 * arr);
+  }
+  const size_t zes = dsize(a.zdt), hes = dsize(a.hdt);
+  const bool pair = (a.d % 2 == 0) && (a.zstride % 2 == 0) &&
+                    (reinterpret_cast<uintptr_t>(a.zf) % (2 * zes) == 0) &&
+                    (reinterpret_cast<uintptr_t>(a.zi) % (2 * zes) == 0) &&
+                    (reinterpret_cast<uintptr_t>(a.h) % (2 * hes) == 0);
+  const double zb = (double)zes, hb = (double)hes;
+  LaunchScope ls(MMF_KERNEL_SCAN, (double)chans * a.t * (2.0 * zb + hb) + (double)chans * 4.0 *
                  ((a.h0 ? 1.0 : 0.0) + (a.h_last ? 1.0 : 0.0)), st);
-  hgrn_scan_kernel<<<grid, kScanWarps * 32, 0, st>>>(a);
-  return check_launch("hgrn_scan_kernel");
+  if (a.nchunk > 1) g_launches.fetch_add(2);  // three kernels under one timing scope
+  const bool tiled = pair && (a.zstride * zes) % 16 == 0 && (a.d * zes) % 16 == 0 &&
+                     (reinterpret_cast<uintptr_t>(a.zf) & 15u) == 0 && (reinterpret_cast<uintptr_t>(a.zi) & 15u) == 0;
+  if (tiled) {
+    if (a.zdt == MMF_F32 && a.hdt == MMF_F32) scan_tiled_typed<MMF_F32, MMF_F32>(a, st);
+    else if (a.zdt == MMF_F32) scan_tiled_typed<MMF_F32, MMF_BF16>(a, st);
+    else if (a.hdt == MMF_F32) scan_tiled_typed<MMF_BF16, MMF_F32>(a, st);
+    else scan_tiled_typed<MMF_BF16, MMF_BF16>(a, st);
+  } else if (pair) {
+    scan_launch_vec<2>(a, st);
+  } else {
+    scan_launch_vec<1>(a, st);
+  }
+  return check_launch("hgrn scan kernels");
 }
 
 mmf_status check_ternary(const mmf_ternary* w, int32_t n, int32_t k, const char* name) {
@@ -308,6 +451,7 @@ struct BlockWs {
   int8_t* qg;  // [m][ldq_d]
   void* gu;    // [m][2I]
   int8_t* qd;  // [m][ldq_I]
+  void* scan;  // chunked-scan scratch
   size_t bytes;
 };
 
@@ -330,6 +474,7 @@ BlockWs block_ws(void* base, int64_t m, int32_t d, int32_t inner, mmf_dtype dt) 
   w.qg = reinterpret_cast<int8_t*>(take(m * row_q(d)));
   w.gu = take(m * 2 * (size_t)inner * es);
   w.qd = reinterpret_cast<int8_t*>(take(m * row_q(inner)));
+  w.scan = take(scan_ws_bytes(m, d));
   w.bytes = off;
   return w;
 }
@@ -403,7 +548,7 @@ mmf_status run_block(const mmf_block_weights* w, const void* x, mmf_dtype dt, in
   sa.zi = W.z;
   sa.zdt = dt; sa.zstride = 3 * d; sa.b = b; sa.t = t; sa.d = d;
   sa.h0 = h0; sa.h = W.h; sa.hdt = dt; sa.h_last = h_last;
-  MMF_TRY(launch_scan(sa, st));
+  MMF_TRY(launch_scan(sa, W.scan, st));
   // 4. g_norm (RMSNorm(h) * gnorm_w * SiLU(g)) fused with o_proj's RMSNorm + quant
   memset(&nq, 0, sizeof(nq));
   nq.x = W.h; nq.ldx = d; nq.xdt = dt;
@@ -494,6 +639,8 @@ size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32
       return d > 0 ? align256((size_t)m * row_q(d)) + align256((size_t)m * sizeof(float)) : 0;
     case MMF_OP_BLOCK:
       return block_ws(nullptr, m, d, inner, MMF_F32).bytes;
+    case MMF_OP_SCAN:
+      return d > 0 ? scan_ws_bytes(m, d) : 0;
     case MMF_OP_DECODE:
     case MMF_OP_STACK:
       return block_ws(nullptr, m, d, inner, MMF_F32).bytes + 2 * align256((size_t)m * d * 4);
@@ -594,19 +741,21 @@ mmf_status mmf_bitlinear_fwd_noalloc(const void* x, mmf_dtype x_dtype, int64_t m
 
 mmf_status mmf_hgrn_scan(const void* zf, const void* zi, mmf_dtype z_dtype, int64_t z_stride,
                          int32_t b, int64_t t, int32_t d, const float* h0, void* h_out,
-                         mmf_dtype h_dtype, float* h_last, mmf_stream_t stream) {
+                         mmf_dtype h_dtype, float* h_last, void* ws, size_t ws_bytes,
+                         mmf_stream_t stream) {
   MMF_CHECK_ARG(b >= 0 && t >= 0 && d >= 0, "scan: negative size");
   MMF_CHECK_ARG(valid_dtype(z_dtype) && valid_dtype(h_dtype), "scan: bad dtype");
   MMF_CHECK_ARG(z_stride >= d, "scan: z_stride %lld < d %d", (long long)z_stride, d);
   if ((int64_t)b * d == 0) return MMF_OK;
   MMF_CHECK_ARG(t == 0 || (zf && zi && h_out), "scan: null pointer");
+  if (t > 16) MMF_TRY(check_ws(ws, ws_bytes, scan_ws_bytes((int64_t)b * t, d)));
   DevInfo* di;
   MMF_TRY(device_info(&di));
   ScanArgs a;
   memset(&a, 0, sizeof(a));
   a.zf = zf; a.zi = zi; a.zdt = z_dtype; a.zstride = z_stride; a.b = b; a.t = t; a.d = d;
   a.h0 = h0; a.h = h_out; a.hdt = h_dtype; a.h_last = h_last;
-  return launch_scan(a, reinterpret_cast<cudaStream_t>(stream));
+  return launch_scan(a, ws, reinterpret_cast<cudaStream_t>(stream));
 }
 
 mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dtype, int32_t b,
@@ -623,7 +772,7 @@ mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dt
       ScanArgs a;
       memset(&a, 0, sizeof(a));
       a.b = b; a.t = 0; a.d = w->d; a.h0 = h0; a.h_last = h_last;
-      return launch_scan(a, reinterpret_cast<cudaStream_t>(stream));
+      return launch_scan(a, nullptr, reinterpret_cast<cudaStream_t>(stream));
     }
     return MMF_OK;
   }

@@ -48,6 +48,8 @@ def test_sizes(L):
     assert 0 < b1 < b2
     assert L.mmf_workspace_bytes(mmf.MMF_OP_STACK, 256, 256, 704, 2) > b1
     assert L.mmf_workspace_bytes(mmf.MMF_OP_BITLINEAR, 5, 100, 7, 0) >= 5 * 128 + 5 * 4
+    # chunked scan: three float arrays of b * nchunk * d with b * nchunk <= ceil(m / 8)
+    assert L.mmf_workspace_bytes(mmf.MMF_OP_SCAN, 8 * 2048, 1024, 0, 0) >= 3 * 1024 * 4 * 8 * 128
 
 
 def test_status_strings(L):
@@ -69,8 +71,10 @@ def test_invalid_arguments_rejected_on_host(L):
     t.codes = 20
     assert L.mmf_bitlinear_fwd(None, 0, 4, None, ctypes.byref(t), None, 0, None, None, None, None, 0,
                                None) == mmf.MMF_ERR_INVALID_ARG
-    assert L.mmf_hgrn_scan(None, None, 0, 2, 1, 4, 4, None, None, 0, None, None) == mmf.MMF_ERR_INVALID_ARG
-    assert L.mmf_hgrn_scan(None, None, 5, 4, 1, 4, 4, None, None, 0, None, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_hgrn_scan(None, None, 0, 2, 1, 4, 4, None, None, 0, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_hgrn_scan(None, None, 5, 4, 1, 4, 4, None, None, 0, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    # a long sequence needs scratch: too little is reported before anything runs
+    assert L.mmf_hgrn_scan(16, 16, 0, 4, 1, 1000, 4, None, 16, 0, None, None, 0, None) == mmf.MMF_ERR_WORKSPACE
     bw = mmf.BlockWeightsC(d=0, inner=4)
     assert L.mmf_block_fwd(ctypes.byref(bw), None, 0, 1, 1, None, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
     assert L.mmf_decode_step(None, 0, None, 0, 1, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG

@@ -80,7 +80,7 @@ def _near_tie(v, margin=1e-4):
 
 
 BITLINEAR_SHAPES = [(1, 256, 256), (3, 768, 256), (8, 1408, 256), (127, 256, 704), (256, 256, 256),
-                    (300, 200, 100), (130, 384, 1024), (9, 64, 2560)]
+                    (300, 200, 100), (130, 384, 1024), (9, 64, 2560), (40, 128, 2048), (5, 96, 7040)]
 
 
 @pytest.mark.parametrize("engine", ["tensor", "simt"])
@@ -240,7 +240,7 @@ def check_block_stages(x, qp, taps, y_g, hl_g, h0, bf16):
     x2 = x.reshape(m, d).astype(np.float64)
     q_ifg, deq_ifg = _np(taps["q_ifg"]), _np(taps["deq_ifg"])
     z = _np(taps["z"]).astype(np.float64)
-    # 1. i/f/g input codes (first quantisation: exact) and 2. the three products
+    # 1. i/f/g input codes (first quantisation: exact) and 2. the three products z = [zi | zf | g]
     for j, p in enumerate(("i", "f", "g")):
         r = O.rmsnorm(x2, qp[f"nw_{p}"])
         qo, deqo, vo = O.act_quant(r)
@@ -248,7 +248,7 @@ def check_block_stages(x, qp, taps, y_g, hl_g, h0, bf16):
         np.testing.assert_allclose(deq_ifg[j], deqo, rtol=1e-6)
         acc = O.int_matmul(q_ifg[j], qp[f"t_{p}"])
         _close(z[:, j * d:(j + 1) * d], acc * deq_ifg[j].astype(np.float64)[:, None] * float(qp[f"s_{p}"]), bf16)
-    # 3. scan on the kernel's gate pre-activations
+    # 3. gates and scan on the kernel's pre-activations
     zi, zf, g = z[:, :d], z[:, d:2 * d], z[:, 2 * d:]
     f, i = O.hgrn_gates(zf.reshape(B, T, d), zi.reshape(B, T, d))
     h_ref = O.hgrn_scan(f, i, h0)
