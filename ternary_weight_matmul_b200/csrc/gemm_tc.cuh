@@ -48,7 +48,8 @@ static_assert(A_COL + STAGES * (BK / 4) <= TMEM_COLS, "TMEM budget");
 constexpr int EPI_CHUNK = 32;
 constexpr int EPI_BUF_BYTES = EPI_CHUNK * BM * 4;
 constexpr int SMEM_EPI_OFF = STAGES * (ACT_BYTES + W_BYTES);
-constexpr int SMEM_BAR_OFF = SMEM_EPI_OFF + 2 * EPI_BUF_BYTES;
+constexpr int SMEM_DQ_OFF = SMEM_EPI_OFF + 2 * EPI_BUF_BYTES;  // per-token (a/127)*s, 2 x BN floats
+constexpr int SMEM_BAR_OFF = SMEM_DQ_OFF + 2 * BN * 4;
 constexpr int NUM_BARS = 3 * STAGES + 5;
 constexpr int SMEM_BYTES = SMEM_BAR_OFF + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -117,6 +118,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
   uint8_t* act_s = smem;
   uint32_t* w_s = reinterpret_cast<uint32_t*>(smem + STAGES * ACT_BYTES);
   int32_t* epi_s = reinterpret_cast<int32_t*>(smem + SMEM_EPI_OFF);
+  float* dq_s = reinterpret_cast<float*>(smem + SMEM_DQ_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
   uint64_t* full = bars;                   // TMA -> expanders      (count 1 + tx bytes)
   uint64_t* afull = bars + STAGES;         // expanders -> MMA      (count 4)
@@ -282,6 +284,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
       const int32_t act = S->act;
       const int act_rows = S->act_cols - n0;  // rows of this tile (from 0) that take the activation
       // vectorised phase 2 needs every row segment 16-byte aligned and complete
+      // per-token factors of this tile, staged once (buffer by tile parity; published to all
+      // epilogue threads by the named barrier of the first chunk)
+      float* dq = dq_s + (tl & 1u) * BN;
+      if (etid < BN) {
+        const int64_t m = (int64_t)mt * BN + etid;
+        dq[etid] = m < P.g.m ? deq[m] * sw : 0.0f;
+      }
       const bool vec_ok = nrows == BM &&
           ((reinterpret_cast<uintptr_t>(y) | (uintptr_t)(ldy * sizeof(OutT))) & 15u) == 0 &&
           (!res || ((reinterpret_cast<uintptr_t>(res) | (uintptr_t)(ldres * sizeof(OutT))) & 15u) == 0) &&
@@ -304,40 +313,62 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
         const int64_t rem = P.g.m - m0;
         const int jmax = rem < EPI_CHUNK ? (int)rem : EPI_CHUNK;
         if (vec_ok) {
-          // 32 tokens x 32 pieces of 4 rows = 1024 pieces, 4 per thread
-#pragma unroll 2
-          for (int pidx = etid; pidx < EPI_CHUNK * (BM / 4); pidx += EPI_THREADS) {
-            const int j = pidx >> 5, q4 = (pidx & 31) * 4;
-            if (j >= jmax) break;
-            const int64_t m = m0 + j;
-            const int4 a = *reinterpret_cast<const int4*>(buf + j * BM + q4);
-            const float dj = deq[m] * sw;
-            float z0 = (float)a.x * dj, z1 = (float)a.y * dj, z2 = (float)a.z * dj, z3 = (float)a.w * dj;
-            if (accp) *reinterpret_cast<int4*>(accp + m * ldacc + q4) = a;
-            if (act != kActNone) {
-              if (q4 + 0 < act_rows) z0 = apply_act(act, z0);
-              if (q4 + 1 < act_rows) z1 = apply_act(act, z1);
-              if (q4 + 2 < act_rows) z2 = apply_act(act, z2);
-              if (q4 + 3 < act_rows) z3 = apply_act(act, z3);
-            }
-            if (YT == MMF_F32) {
-              if (res) {
-                const float4 r = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(res) + m * ldres + q4);
-                z0 += r.x; z1 += r.y; z2 += r.z; z3 += r.w;
+          // 32 tokens x 16 pieces of 8 rows = 512 pieces, 2 per thread; a warp writes two whole
+          // 128-row segments (256 B in bf16, 512 B in fp32)
+#pragma unroll
+          for (int it = 0; it < 2; ++it) {
+            const int pidx = etid + it * EPI_THREADS;
+            const int j = pidx >> 4, r8 = (pidx & 15) * 8;
+            if (j < jmax) {
+              const int64_t m = m0 + j;
+              const int4 a0 = *reinterpret_cast<const int4*>(buf + j * BM + r8);
+              const int4 a1 = *reinterpret_cast<const int4*>(buf + j * BM + r8 + 4);
+              const float dj = dq[c0 + j];
+              float z[8] = {(float)a0.x * dj, (float)a0.y * dj, (float)a0.z * dj, (float)a0.w * dj,
+                            (float)a1.x * dj, (float)a1.y * dj, (float)a1.z * dj, (float)a1.w * dj};
+              if (accp) {
+                *reinterpret_cast<int4*>(accp + m * ldacc + r8) = a0;
+                *reinterpret_cast<int4*>(accp + m * ldacc + r8 + 4) = a1;
               }
-              *reinterpret_cast<float4*>(reinterpret_cast<float*>(y) + m * ldy + q4) = make_float4(z0, z1, z2, z3);
-            } else {
-              if (res) {
-                const uint2 r = *reinterpret_cast<const uint2*>(reinterpret_cast<const __nv_bfloat16*>(res) + m * ldres + q4);
-                const float2 r01 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.x));
-                const float2 r23 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&r.y));
-                z0 += r01.x; z1 += r01.y; z2 += r23.x; z3 += r23.y;
+              if (YT == MMF_F32) {
+                if (res) {
+                  const float4 ra = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(res) + m * ldres + r8);
+                  const float4 rb = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(res) + m * ldres + r8 + 4);
+                  z[0] += ra.x; z[1] += ra.y; z[2] += ra.z; z[3] += ra.w;
+                  z[4] += rb.x; z[5] += rb.y; z[6] += rb.z; z[7] += rb.w;
+                }
+                if (act != kActNone) {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e)
+                    if (r8 + e < act_rows) z[e] = apply_act(act, z[e]);
+                }
+                float* yp = reinterpret_cast<float*>(y) + m * ldy + r8;
+                *reinterpret_cast<float4*>(yp) = make_float4(z[0], z[1], z[2], z[3]);
+                *reinterpret_cast<float4*>(yp + 4) = make_float4(z[4], z[5], z[6], z[7]);
+              } else {
+                if (res) {
+                  const uint4 r = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(res) + m * ldres + r8);
+                  const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+                  for (int q = 0; q < 4; ++q) {
+                    const float2 rf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[q]));
+                    z[2 * q] += rf.x;
+                    z[2 * q + 1] += rf.y;
+                  }
+                }
+                if (act != kActNone) {
+#pragma unroll
+                  for (int e = 0; e < 8; ++e)
+                    if (r8 + e < act_rows) z[e] = apply_act(act, z[e]);
+                }
+                uint32_t o[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  const __nv_bfloat162 h2 = __floats2bfloat162_rn(z[2 * q], z[2 * q + 1]);
+                  o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+                }
+                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(y) + m * ldy + r8) = make_uint4(o[0], o[1], o[2], o[3]);
               }
-              const __nv_bfloat162 o01 = __floats2bfloat162_rn(z0, z1), o23 = __floats2bfloat162_rn(z2, z3);
-              uint2 o;
-              o.x = *reinterpret_cast<const uint32_t*>(&o01);
-              o.y = *reinterpret_cast<const uint32_t*>(&o23);
-              *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(y) + m * ldy + q4) = o;
             }
           }
         } else {
@@ -348,7 +379,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
             if (r >= nrows) continue;
             const int64_t m = m0 + j;
             const int32_t a = buf[j * BM + r];
-            float z = (float)a * (deq[m] * sw);
+            float z = (float)a * dq[c0 + j];
             if (accp) accp[m * ldacc + r] = a;
             if (res) z += Elem<YT>::load(res + m * ldres + r);
             if (r < act_rows) z = apply_act(act, z);
