@@ -163,7 +163,11 @@ mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dt
  * taken after the forward from the very buffers its kernels used (m = b*t tokens, es = dtype):
  *   q_ifg [3][m][d] int8 and deq_ifg [3][m] float: activation codes / a/127 of the i, f, g inputs
  *   z [m][3d] dtype = [zi | zf | g];  h [m][d] dtype;  q_o [m][d], deq_o [m]: o_proj input codes
- *   x1 [m][d] dtype;  q_gate [m][d], deq_gate [m];  gu [m][2I] dtype = [gate | up]
+ *   x1 [m][d] dtype;  q_gate [m][d], deq_gate [m]
+ *   gu [m][2I] dtype = [gate | up], written when gate_proj stores both halves;
+ *   v [m][I] dtype = SiLU(gate) * up, written instead when gate_proj's epilogue forms the GLU
+ *     product itself: on the tensor-core engine (more than 8 rows under MMF_GEMM_AUTO, or
+ *     MMF_GEMM_TENSOR) with I % 64 == 0
  *   q_down [m][I], deq_down [m]. */
 typedef struct {
   int8_t* q_ifg;
@@ -178,6 +182,7 @@ typedef struct {
   void* gu;
   int8_t* q_down;
   float* deq_down;
+  void* v;
 } mmf_block_taps;
 
 /* mmf_block_fwd followed by copies of its intermediates into `taps` (same kernels, same

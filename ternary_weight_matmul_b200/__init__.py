@@ -55,7 +55,8 @@ class BlockWeightsC(ctypes.Structure):
 
 class BlockTapsC(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in (
-        "q_ifg", "deq_ifg", "z", "h", "q_o", "deq_o", "x1", "q_gate", "deq_gate", "gu", "q_down", "deq_down")]
+        "q_ifg", "deq_ifg", "z", "h", "q_o", "deq_o", "x1", "q_gate", "deq_gate", "gu", "q_down", "deq_down",
+        "v")]
 
 
 _lib = None
@@ -310,6 +311,7 @@ def block_fwd_taps(block: Block, x: torch.Tensor, h0: torch.Tensor | None = None
         "gu": torch.empty(m, 2 * inner, dtype=dt, device=dev),
         "q_down": torch.empty(m, inner, dtype=torch.int8, device=dev),
         "deq_down": torch.empty(m, dtype=torch.float32, device=dev),
+        "v": torch.empty(m, inner, dtype=dt, device=dev),
     }
     tc = BlockTapsC(**{k: v.data_ptr() for k, v in taps.items()})
     ws = workspace(MMF_OP_BLOCK, m, block.d, inner, 1, dev)
@@ -366,8 +368,20 @@ def sync_status(device: torch.device | str | None = None) -> int:
     return int(lib().mmf_sync_status(_stream(dev)))
 
 
+_gemm_path = MMF_GEMM_AUTO
+
+
 def set_gemm_path(path: int) -> None:
+    global _gemm_path
     _check(lib().mmf_set_gemm_path(path), "mmf_set_gemm_path")
+    _gemm_path = path
+
+
+def glu_fused(m: int, inner: int) -> bool:
+    """Whether a block forward on m tokens forms SiLU(gate) * up in gate_proj's epilogue (taps
+    then carry ``v`` instead of ``gu``): the tensor-core engine with inner % 64 == 0."""
+    tensor = _gemm_path == MMF_GEMM_TENSOR or (_gemm_path == MMF_GEMM_AUTO and m > 8)
+    return tensor and inner % 64 == 0
 
 
 KERNEL_CLASSES = {"gemm_tc": 0, "gemm_simt": 1, "norm_quant": 2, "scan": 3, "other": 4}

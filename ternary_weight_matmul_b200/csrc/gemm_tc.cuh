@@ -5,15 +5,18 @@
 // (M = 128 weight rows per tile) and the activation codes are the B operand (N = 128 tokens per
 // tile), so the D accumulator is [weight row][token] in tensor memory.
 //
-//   * TMA stages the packed 2-bit weight tile (128 rows x 8 words = 4 KB) and the int8 activation
-//     tile (128 tokens x 128 bytes, 128-byte swizzle = 16 KB) of every k-block into shared memory.
+//   * TMA stages, per 256-wide k-block, the packed 2-bit weight tile (128 rows x 16 words = 8 KB,
+//     64-byte swizzle) and the int8 activation tile (128 tokens x 256 bytes as two 128-byte-
+//     swizzled boxes = 32 KB) into shared memory.
 //   * Four expander warps turn the packed tile into int8 with byte permutes and write it straight
 //     into tensor memory (tcgen05.st), one weight row per TMEM lane: no unpacked copy ever touches
 //     shared memory, so the MMA reads only the activation tile from shared memory.
-//   * One thread issues tcgen05.mma.kind::i8 (A from TMEM, B from shared memory, D in TMEM).
+//   * One thread issues tcgen05.mma.kind::i8 (A from TMEM, B from shared memory, D in TMEM),
+//     eight instructions per k-block between two barrier waits.
 //   * Eight epilogue warps (two per TMEM sub-partition) read the int32 accumulators back with
-//     tcgen05.ld, rescale and store.
-//   * The kernel is persistent (one CTA per SM) with a 6-stage operand ring and a double-buffered
+//     tcgen05.ld, stage them transposed in shared memory, rescale, optionally add the residual or
+//     form the SiLU-gated product of paired gate/up rows (GLU), and store whole row segments.
+//   * The kernel is persistent (one CTA per SM) with a 4-stage operand ring and a double-buffered
 //     accumulator, so the epilogue of one tile overlaps the MMAs of the next.
 //
 // Warp roles (448 threads): 0 = TMA producer, 1 = TMEM allocator + MMA issuer, 2..5 = expanders,
@@ -29,30 +32,41 @@ namespace tc {
 
 constexpr int BM = 128;      // weight rows per tile (MMA M)
 constexpr int BN = 128;      // tokens per tile (MMA N)
-constexpr int BK = 128;      // K per stage: one 128-byte swizzle atom of int8
+constexpr int BK = 256;      // K per stage
 constexpr int UK = 32;       // K per kind::i8 MMA instruction
-constexpr int STAGES = 6;
-constexpr int ACT_BYTES = BN * BK;       // 16 KB
-constexpr int W_BYTES = BM * BK / 4;     // 4 KB (2 bits per code)
-constexpr int W_WORDS_PER_ROW = BK / 16; // 8
+constexpr int STAGES = 4;
+constexpr int ACT_BOX = 128;                  // K bytes per activation box (one 128-byte swizzle atom)
+constexpr int ACT_BOX_BYTES = BN * ACT_BOX;   // 16 KB
+constexpr int ACT_BYTES = BN * BK;            // 32 KB per stage (two boxes)
+constexpr int W_WORDS_PER_ROW = BK / 16;      // 16 words = 64 bytes per weight row per stage
+constexpr int W_BYTES = BM * BK / 4;          // 8 KB (2 bits per code)
+constexpr int GLU_ROWS = BM / 2;              // GLU tiles pair 64 gate rows with 64 up rows
 constexpr int NUM_THREADS = 448;
 constexpr int EPI_WARPS = 8;
 constexpr int EPI_THREADS = 32 * EPI_WARPS;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t ACC_COL = 0;          // accumulators at columns [0, 128) and [128, 256)
-constexpr uint32_t A_COL = 2 * BN;       // A stages at 256 + 32 * s (32 columns = 128 int8 per lane)
-static_assert(A_COL + STAGES * (BK / 4) <= TMEM_COLS, "TMEM budget");
+constexpr uint32_t A_COLS = BK / 4;      // TMEM columns of one expanded A stage (256 int8 per lane)
+constexpr uint32_t A_COL = 2 * BN;       // A stages at 256 + 64 * s
+static_assert(A_COL + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
 
 // Epilogue staging: the raw int32 accumulators of a 32-token chunk, [32 tokens][128 rows],
-// double-buffered (2 x 16 KB).
+// double-buffered (2 x 16 KB). Within a token's 512-byte row the 16-byte chunk c sits at
+// c ^ ((c >> 3) & 1), which keeps both the row-wise writes and the 32-byte piece reads free of
+// bank conflicts.
 constexpr int EPI_CHUNK = 32;
 constexpr int EPI_BUF_BYTES = EPI_CHUNK * BM * 4;
-constexpr int SMEM_EPI_OFF = STAGES * (ACT_BYTES + W_BYTES);
+constexpr int SMEM_W_OFF = STAGES * ACT_BYTES;
+constexpr int SMEM_EPI_OFF = SMEM_W_OFF + STAGES * W_BYTES;
 constexpr int SMEM_DQ_OFF = SMEM_EPI_OFF + 2 * EPI_BUF_BYTES;  // per-token (a/127)*s, 2 x BN floats
 constexpr int SMEM_BAR_OFF = SMEM_DQ_OFF + 2 * BN * 4;
 constexpr int NUM_BARS = 3 * STAGES + 5;
 constexpr int SMEM_BYTES = SMEM_BAR_OFF + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
+
+__device__ __forceinline__ int epi_word(int r) {  // staged position of row r within a token row
+  return r ^ (((r >> 5) & 1) << 2);
+}
 
 // Instruction descriptor, kind::i8: D = s32 (bits 4-5 = 2), A and B signed int8 (bits 7-9 and
 // 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at bits 24-28.
@@ -68,13 +82,31 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
          ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
+// float(a) for |a| < 2^22 without a conversion instruction: a + 1.5 * 2^23 laid into the
+// mantissa of a float whose spacing is 1, minus that constant again (both steps exact).
+__device__ __forceinline__ float acc_to_float(int32_t a) {
+  return __fsub_rn(__int_as_float(a + 0x4B400000), 12582912.0f);
+}
+
+// z = float(a) * dj for eight accumulators (the branch is uniform across the launch).
+__device__ __forceinline__ void scale8(const int32_t (&a)[8], float dj, bool small_acc, float (&z)[8]) {
+  if (small_acc) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = __fmul_rn(acc_to_float(a[e]), dj);
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = __fmul_rn((float)a[e], dj);
+  }
+}
+
 struct Params {
   CUtensorMap act_map[3];  // int8 activation codes [m][ldq], box 128 x 128, swizzle 128B
-  CUtensorMap w_map[3];    // u32 packed weights [n][kw], box 8 x 128
+  CUtensorMap w_map[3];    // u32 packed weights [n][kw], box 16 x 128 (GLU: 16 x 64), swizzle 64B
   GemmArgs g;
   int32_t m_tiles;
   int32_t tile_start[4];   // first tile of each segment; tile_start[nseg] = total
   int32_t num_kb;
+  int32_t small_acc;       // every |acc| < 2^22 (127 * k), so acc_to_float is exact
   uint32_t wait_limit_us;
 };
 
@@ -110,13 +142,49 @@ __device__ __forceinline__ bool epi_any(bool pred) {
   return r != 0u;
 }
 
+// Eight values of one output row segment, bf16 or float32, 16- or 32-byte store.
+template <mmf_dtype YT>
+__device__ __forceinline__ void store8(typename Elem<YT>::T* p, const float (&z)[8]) {
+  if (YT == MMF_F32) {
+    float* f = reinterpret_cast<float*>(p);
+    *reinterpret_cast<float4*>(f) = make_float4(z[0], z[1], z[2], z[3]);
+    *reinterpret_cast<float4*>(f + 4) = make_float4(z[4], z[5], z[6], z[7]);
+  } else {
+    uint32_t o[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __nv_bfloat162 h2 = __floats2bfloat162_rn(z[2 * q], z[2 * q + 1]);
+      o[q] = *reinterpret_cast<const uint32_t*>(&h2);
+    }
+    *reinterpret_cast<uint4*>(p) = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+template <mmf_dtype YT>
+__device__ __forceinline__ void add8(const typename Elem<YT>::T* p, float (&z)[8]) {
+  if (YT == MMF_F32) {
+    const float4 ra = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p));
+    const float4 rb = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(p) + 4);
+    z[0] += ra.x; z[1] += ra.y; z[2] += ra.z; z[3] += ra.w;
+    z[4] += rb.x; z[5] += rb.y; z[6] += rb.z; z[7] += rb.w;
+  } else {
+    const uint4 r = *reinterpret_cast<const uint4*>(p);
+    const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 rf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[q]));
+      z[2 * q] += rf.x;
+      z[2 * q + 1] += rf.y;
+    }
+  }
+}
+
 template <mmf_dtype YT>
 __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const __grid_constant__ Params P) {
   using OutT = typename Elem<YT>::T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* act_s = smem;
-  uint32_t* w_s = reinterpret_cast<uint32_t*>(smem + STAGES * ACT_BYTES);
+  uint32_t* w_s = reinterpret_cast<uint32_t*>(smem + SMEM_W_OFF);
   int32_t* epi_s = reinterpret_cast<int32_t*>(smem + SMEM_EPI_OFF);
   float* dq_s = reinterpret_cast<float*>(smem + SMEM_DQ_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
@@ -168,13 +236,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         int seg, nt, mt;
         decode_tile(P, tile, seg, nt, mt);
+        const GemmSeg& S = P.g.seg[seg];
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
           if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&full[s], ACT_BYTES + W_BYTES);
-          tma_load_2d(act_s + s * ACT_BYTES, &P.act_map[seg], kb * BK, mt * BN, &full[s]);
-          tma_load_2d(w_s + s * (W_BYTES / 4), &P.w_map[seg], kb * W_WORDS_PER_ROW, nt * BM, &full[s]);
+          uint8_t* ad = act_s + s * ACT_BYTES;
+          tma_load_2d(ad, &P.act_map[seg], kb * BK, mt * BN, &full[s]);
+          tma_load_2d(ad + ACT_BOX_BYTES, &P.act_map[seg], kb * BK + ACT_BOX, mt * BN, &full[s]);
+          uint32_t* wd = w_s + s * (W_BYTES / 4);
+          if (S.glu) {
+            // rows [0, 64) of the tile: gate rows 64 nt..; rows [64, 128): the paired up rows
+            tma_load_2d(wd, &P.w_map[seg], kb * W_WORDS_PER_ROW, nt * GLU_ROWS, &full[s]);
+            tma_load_2d(wd + GLU_ROWS * W_WORDS_PER_ROW, &P.w_map[seg], kb * W_WORDS_PER_ROW,
+                        S.glu_inner + nt * GLU_ROWS, &full[s]);
+          } else {
+            tma_load_2d(wd, &P.w_map[seg], kb * W_WORDS_PER_ROW, nt * BM, &full[s]);
+          }
         }
       }
       if (!ok || *abort_flag) {
@@ -198,13 +277,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
         for (int kb = 0; kb < num_kb; ++kb, ++it) {
           const int s = it % STAGES;
           const uint32_t ph = (it / STAGES) & 1u;
+          // afull implies the stage's TMA landed: the expanders waited on full[s] first
           if (!mbar_wait_bounded(&afull[s], ph, limit, abort_flag)) { ok = false; break; }
           tc_fence_after();
-          const uint32_t a_tmem = tmem_base + A_COL + s * (BK / 4);
+          const uint32_t a_tmem = tmem_base + A_COL + s * A_COLS;
           const uint32_t b_addr = smem_u32(act_s + s * ACT_BYTES);
 #pragma unroll
           for (int kk = 0; kk < BK / UK; ++kk)
-            tc_mma_i8_ts(d_tmem, a_tmem + kk * (UK / 4), sw128_desc(b_addr + kk * UK), IDESC,
+            tc_mma_i8_ts(d_tmem, a_tmem + kk * (UK / 4),
+                         sw128_desc(b_addr + (kk >> 2) * ACT_BOX_BYTES + (kk & 3) * UK), IDESC,
                          (kb | kk) != 0 ? 1u : 0u);
           tc_commit(&empty[s]);
         }
@@ -222,6 +303,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     const uint32_t sub = (uint32_t)(warp & 3);          // TMEM sub-partition of this warp
     const int row = (int)sub * 32 + lane;               // weight row within the tile = TMEM lane
     const uint32_t lane_addr = (sub * 32u) << 16;
+    // the weight tile arrives with the 64-byte swizzle: 16-byte chunk c of row r sits at
+    // c ^ ((r >> 1) & 3), so the 32 rows a warp reads at once fall in distinct banks
+    const uint32_t swz = (uint32_t)((row >> 1) & 3);
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
@@ -230,17 +314,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
         const uint32_t ph = (it / STAGES) & 1u;
         if (!mbar_wait_bounded(&full[s], ph, limit, abort_flag)) { ok = false; break; }
         const uint4* src = reinterpret_cast<const uint4*>(w_s + s * (W_BYTES / 4) + row * W_WORDS_PER_ROW);
-        const uint4 p0 = src[0], p1 = src[1];
-        uint32_t v[32];
-        expand_word(p0.x, v + 0);
-        expand_word(p0.y, v + 4);
-        expand_word(p0.z, v + 8);
-        expand_word(p0.w, v + 12);
-        expand_word(p1.x, v + 16);
-        expand_word(p1.y, v + 20);
-        expand_word(p1.z, v + 24);
-        expand_word(p1.w, v + 28);
-        tmem_st_32x32b_x32(tmem_base + lane_addr + A_COL + s * (BK / 4), v);
+        const uint32_t ta = tmem_base + lane_addr + A_COL + s * A_COLS;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const uint4 p0 = src[(2 * h) ^ swz], p1 = src[(2 * h + 1) ^ swz];
+          uint32_t v[32];
+          expand_word(p0.x, v + 0);
+          expand_word(p0.y, v + 4);
+          expand_word(p0.z, v + 8);
+          expand_word(p0.w, v + 12);
+          expand_word(p1.x, v + 16);
+          expand_word(p1.y, v + 20);
+          expand_word(p1.z, v + 24);
+          expand_word(p1.w, v + 28);
+          tmem_st_32x32b_x32(ta + 32 * h, v);
+        }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
@@ -252,14 +340,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     // Two phases per 32-token chunk. Phase 1: each warp loads its sub-partition's 32 weight rows
     // x 16 tokens (its half of the chunk) of int32 accumulators from TMEM (thread = row) and
     // stores them to shared memory transposed, as [token][row] (one conflict-free 32-bit store
-    // per element). Phase 2: the 256 epilogue threads walk the chunk token-major in 16-byte
-    // pieces (4 rows each), rescale by (a/127) * s of the token, add the residual and write 8- or
-    // 16-byte vectors, so every global access covers whole row segments of the output.
+    // per element). Phase 2: the 256 epilogue threads walk the chunk token-major in pieces of
+    // 8 output columns, rescale by (a/127) * s of the token, add the residual (or, for a GLU
+    // tile, form SiLU(gate) * up from rows r and 64 + r) and write 16- or 32-byte vectors, so
+    // every global access covers whole row segments of the output.
     const uint32_t sub = (uint32_t)(warp & 3);
     const int half = (warp - 6) >> 2;        // which 16 tokens of a chunk this warp loads
     const int row = (int)sub * 32 + lane;
+    const int srow = epi_word(row);
     const uint32_t lane_addr = (sub * 32u) << 16;
     const int etid = threadIdx.x - 6 * 32;  // 0..255
+    const bool small_acc = P.small_acc != 0;
     uint32_t tl = 0, chunk_ctr = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tl) {
       const uint32_t b = tl & 1u;
@@ -271,8 +362,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
       int seg, nt, mt;
       decode_tile(P, tile, seg, nt, mt);
       const GemmSeg* S = seg == 0 ? &P.g.seg[0] : (seg == 1 ? &P.g.seg[1] : &P.g.seg[2]);
-      const int n0 = nt * BM;
-      const int nrows = S->n - n0 < BM ? S->n - n0 : BM;
+      const bool glu = S->glu != 0;
+      const int n0 = nt * (glu ? GLU_ROWS : BM);           // first output column of the tile
+      const int nrows = glu ? GLU_ROWS : (S->n - n0 < BM ? S->n - n0 : BM);
       const float sw = S->sw[0];
       const float* deq = S->deq;
       OutT* y = reinterpret_cast<OutT*>(S->y) + S->ycol + n0;
@@ -283,7 +375,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
       const int64_t ldacc = S->ldacc;
       const int32_t act = S->act;
       const int act_rows = S->act_cols - n0;  // rows of this tile (from 0) that take the activation
-      // vectorised phase 2 needs every row segment 16-byte aligned and complete
       // per-token factors of this tile, staged once (buffer by tile parity; published to all
       // epilogue threads by the named barrier of the first chunk)
       float* dq = dq_s + (tl & 1u) * BN;
@@ -291,7 +382,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
         const int64_t m = (int64_t)mt * BN + etid;
         dq[etid] = m < P.g.m ? deq[m] * sw : 0.0f;
       }
-      const bool vec_ok = nrows == BM &&
+      // vectorised phase 2 needs every row segment 16-byte aligned and complete
+      const bool vec_ok = nrows == (glu ? GLU_ROWS : BM) &&
           ((reinterpret_cast<uintptr_t>(y) | (uintptr_t)(ldy * sizeof(OutT))) & 15u) == 0 &&
           (!res || ((reinterpret_cast<uintptr_t>(res) | (uintptr_t)(ldres * sizeof(OutT))) & 15u) == 0) &&
           (!accp || ((reinterpret_cast<uintptr_t>(accp) | (uintptr_t)(ldacc * 4)) & 15u) == 0);
@@ -307,69 +399,68 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
           if (lane == 0) mbar_arrive(&accempty[b]);
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) buf[(16 * half + j) * BM + row] = (int32_t)v[j];
+        for (int j = 0; j < 16; ++j) buf[(16 * half + j) * BM + srow] = (int32_t)v[j];
         asm volatile("bar.sync 1, 256;" ::: "memory");
         const int64_t m0 = (int64_t)mt * BN + c0;
         const int64_t rem = P.g.m - m0;
         const int jmax = rem < EPI_CHUNK ? (int)rem : EPI_CHUNK;
-        if (vec_ok) {
+        if (vec_ok && glu) {
+          // 32 tokens x 8 pieces of 8 output columns = 256 pieces, one per thread
+          const int j = etid >> 3, r8 = (etid & 7) * 8;
+          if (j < jmax) {
+            const int32_t* bj = buf + j * BM;
+            const int4 g0 = *reinterpret_cast<const int4*>(bj + epi_word(r8));
+            const int4 g1 = *reinterpret_cast<const int4*>(bj + epi_word(r8 + 4));
+            const int4 u0 = *reinterpret_cast<const int4*>(bj + epi_word(GLU_ROWS + r8));
+            const int4 u1 = *reinterpret_cast<const int4*>(bj + epi_word(GLU_ROWS + r8 + 4));
+            const int32_t ga[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+            const int32_t ua[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
+            const float dj = dq[c0 + j];
+            float gv[8], z[8];
+            scale8(ga, dj, small_acc, gv);
+            scale8(ua, dj, small_acc, z);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) z[e] = siluf_(gv[e]) * z[e];
+            store8<YT>(y + (m0 + j) * ldy + r8, z);
+          }
+        } else if (vec_ok) {
           // 32 tokens x 16 pieces of 8 rows = 512 pieces, 2 per thread; a warp writes two whole
           // 128-row segments (256 B in bf16, 512 B in fp32)
 #pragma unroll
-          for (int it = 0; it < 2; ++it) {
-            const int pidx = etid + it * EPI_THREADS;
+          for (int itp = 0; itp < 2; ++itp) {
+            const int pidx = etid + itp * EPI_THREADS;
             const int j = pidx >> 4, r8 = (pidx & 15) * 8;
             if (j < jmax) {
               const int64_t m = m0 + j;
-              const int4 a0 = *reinterpret_cast<const int4*>(buf + j * BM + r8);
-              const int4 a1 = *reinterpret_cast<const int4*>(buf + j * BM + r8 + 4);
+              const int32_t* bj = buf + j * BM;
+              const int4 a0 = *reinterpret_cast<const int4*>(bj + epi_word(r8));
+              const int4 a1 = *reinterpret_cast<const int4*>(bj + epi_word(r8 + 4));
+              const int32_t aa[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
               const float dj = dq[c0 + j];
-              float z[8] = {(float)a0.x * dj, (float)a0.y * dj, (float)a0.z * dj, (float)a0.w * dj,
-                            (float)a1.x * dj, (float)a1.y * dj, (float)a1.z * dj, (float)a1.w * dj};
+              float z[8];
+              scale8(aa, dj, small_acc, z);
               if (accp) {
                 *reinterpret_cast<int4*>(accp + m * ldacc + r8) = a0;
                 *reinterpret_cast<int4*>(accp + m * ldacc + r8 + 4) = a1;
               }
-              if (YT == MMF_F32) {
-                if (res) {
-                  const float4 ra = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(res) + m * ldres + r8);
-                  const float4 rb = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(res) + m * ldres + r8 + 4);
-                  z[0] += ra.x; z[1] += ra.y; z[2] += ra.z; z[3] += ra.w;
-                  z[4] += rb.x; z[5] += rb.y; z[6] += rb.z; z[7] += rb.w;
-                }
-                if (act != kActNone) {
+              if (res) add8<YT>(res + m * ldres + r8, z);
+              if (act != kActNone) {
 #pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    if (r8 + e < act_rows) z[e] = apply_act(act, z[e]);
-                }
-                float* yp = reinterpret_cast<float*>(y) + m * ldy + r8;
-                *reinterpret_cast<float4*>(yp) = make_float4(z[0], z[1], z[2], z[3]);
-                *reinterpret_cast<float4*>(yp + 4) = make_float4(z[4], z[5], z[6], z[7]);
-              } else {
-                if (res) {
-                  const uint4 r = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(res) + m * ldres + r8);
-                  const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-                  for (int q = 0; q < 4; ++q) {
-                    const float2 rf = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&rw[q]));
-                    z[2 * q] += rf.x;
-                    z[2 * q + 1] += rf.y;
-                  }
-                }
-                if (act != kActNone) {
-#pragma unroll
-                  for (int e = 0; e < 8; ++e)
-                    if (r8 + e < act_rows) z[e] = apply_act(act, z[e]);
-                }
-                uint32_t o[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  const __nv_bfloat162 h2 = __floats2bfloat162_rn(z[2 * q], z[2 * q + 1]);
-                  o[q] = *reinterpret_cast<const uint32_t*>(&h2);
-                }
-                *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(y) + m * ldy + r8) = make_uint4(o[0], o[1], o[2], o[3]);
+                for (int e = 0; e < 8; ++e)
+                  if (r8 + e < act_rows) z[e] = apply_act(act, z[e]);
               }
+              store8<YT>(y + m * ldy + r8, z);
             }
+          }
+        } else if (glu) {
+          // unaligned GLU output: one output column per step
+          for (int e = etid; e < EPI_CHUNK * GLU_ROWS; e += EPI_THREADS) {
+            const int j = e / GLU_ROWS, r = e - j * GLU_ROWS;
+            if (j >= jmax) break;
+            const float dj = dq[c0 + j];
+            const float gv = __fmul_rn((float)buf[j * BM + epi_word(r)], dj);
+            const float uv = __fmul_rn((float)buf[j * BM + epi_word(GLU_ROWS + r)], dj);
+            Elem<YT>::store(y + (m0 + j) * ldy + r, siluf_(gv) * uv);
           }
         } else {
           // ragged tile or unaligned output: one element per step, still token-major
@@ -378,8 +469,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
             if (j >= jmax) break;
             if (r >= nrows) continue;
             const int64_t m = m0 + j;
-            const int32_t a = buf[j * BM + r];
-            float z = (float)a * dq[c0 + j];
+            const int32_t a = buf[j * BM + epi_word(r)];
+            float z = __fmul_rn((float)a, dq[c0 + j]);
             if (accp) accp[m * ldacc + r] = a;
             if (res) z += Elem<YT>::load(res + m * ldres + r);
             if (r < act_rows) z = apply_act(act, z);

@@ -180,20 +180,26 @@ __global__ void __launch_bounds__(256) norm_quant_kernel(const NormQuantArgs a) 
 // Vectorised variant for K % 8 == 0 and 16-byte aligned rows (K <= 8192): a row group of W
 // warps owns one row and keeps it in registers (at most 4 chunks of 8 values per thread), loads
 // and stores whole 16-/8-byte pieces and reduces with shuffles (plus one double-buffered shared
-// exchange per reduction when W > 1). Arithmetic is that of norm_quant_kernel.
+// exchange per reduction when W > 1).
+//
+// Arithmetic: r = (v * (1/rms)) * gain in float32, a = max|r|, code = rint(r * (127/a)). The
+// factor 1/rms cancels between r and a, so the codes depend on the mean square only through the
+// float32 rounding of r (a relative perturbation of the mean square moves r * 127/a by a few
+// ulp at most); the sum of squares therefore runs in float32 and only the final 1/sqrt is formed
+// in float64. The dequantisation factor a/127 carries the mean square's own rounding (~1e-7).
 constexpr int kNqThreads = 256;
 constexpr int kNqMaxChunks = 4;
 
 template <int W>
-__device__ __forceinline__ double nq_group_sum(double v, double (*red)[8], int& ph) {
-  v = warp_sum_d(v);
+__device__ __forceinline__ float nq_group_sum(float v, float (*red)[8], int& ph) {
+  v = warp_sum(v);
   if (W == 1) return v;
   const int wid = threadIdx.x >> 5, g0 = (wid / W) * W;
-  double* r = red[ph & 1];
+  float* r = red[ph & 1];
   ++ph;
   if ((threadIdx.x & 31) == 0) r[wid] = v;
   __syncthreads();
-  double s = 0.0;
+  float s = 0.0f;
 #pragma unroll
   for (int k = 0; k < W; ++k) s += r[g0 + k];
   return s;
@@ -250,37 +256,36 @@ __device__ __forceinline__ void load8_gain(const float* g, int64_t idx, float (&
   o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
   o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
 }
-// r = float32(v * g * rinv) with rinv = 1/rms given as a float64 split rh + rl (rl = rinv - rh).
-// Double-float arithmetic: v*g and (v*g)*rh are formed exactly as hi + lo pairs with FMA, the
-// remaining terms are added, and the sum is rounded once, so r is the float32 rounding of the
-// product to within ~2^-44 relative, the same value a float64 evaluation rounds to (barring a
-// product that lies that close to a float32 rounding boundary).
-__device__ __forceinline__ float nq_r(float v, float g, float rh, float rl) {
-  const float p = __fmul_rn(v, g);
-  const float pe = fmaf(v, g, -p);
-  const float q = __fmul_rn(p, rh);
-  const float qe = fmaf(p, rh, -q);
-  return __fadd_rn(q, fmaf(p, rl, fmaf(pe, rh, qe)));
+// 1 / sqrt(ss / k + eps), formed in float64 from the float32 sum and rounded once.
+__device__ __forceinline__ float nq_rinv(float ss, int k, float eps) {
+  return (float)(1.0 / sqrt((double)ss / (double)k + (double)eps));
 }
-__device__ __forceinline__ void nq_split(double rinv, float& rh, float& rl) {
-  rh = (float)rinv;
-  rl = (float)(rinv - (double)rh);
+// int8 code of x: clamp to [-127, 127], then round half to even by adding 1.5 * 2^23 (where the
+// float32 spacing is exactly 1, so the IEEE round-to-nearest-even addition does the rounding)
+// and reading the integer back from the low mantissa bits.
+__device__ __forceinline__ uint32_t q8_code(float x) {
+  const float c = fminf(fmaxf(x, -127.0f), 127.0f);
+  return (uint32_t)(__float_as_int(__fadd_rn(c, 12582912.0f)) - 0x4B400000);
+}
+// Low bytes of four words packed into one word, a in byte 0.
+__device__ __forceinline__ uint32_t pack4_lo_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
 }
 
 // Row group of W warps per row, NCH chunks of 8 values per thread (K <= 256 * W * NCH).
 template <mmf_dtype XT, int MODE, int W, int NCH>
 __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQuantArgs a) {
   constexpr int GT = 32 * W;
-  __shared__ double redd[2][8];
-  __shared__ float redf[2][8][3];
-  int phd = 0, phf = 0;
+  __shared__ float reds[2][8];
+  __shared__ float redm[2][8][3];
+  int phs = 0, phm = 0;
   const int grp = (threadIdx.x >> 5) / W;
   const int gl = threadIdx.x - grp * GT;
   const int64_t row = (int64_t)blockIdx.x * (8 / W) + grp;
   const bool active = row < a.m;
   const int k = a.k, nck = k >> 3;
   float v[NCH][8];
-  double ss = 0.0;
+  float ss = 0.0f;
   if (MODE == kRowGnorm) {
     float g[NCH][8];
 #pragma unroll
@@ -290,13 +295,11 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
         load8<XT>(a.x, row * a.ldx + 8 * c, v[i]);
         load8<XT>(a.g, row * a.ldg + 8 * c, g[i]);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss += (double)v[i][e] * (double)v[i][e];
+        for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
       }
     }
-    const double rinv_h = 1.0 / sqrt(nq_group_sum<W>(ss, redd, phd) / (double)k + (double)a.eps);
-    float rhh, rlh;
-    nq_split(rinv_h, rhh, rlh);
-    ss = 0.0;
+    const float rfh = nq_rinv(nq_group_sum<W>(ss, reds, phs), k, a.eps);
+    ss = 0.0f;
 #pragma unroll
     for (int i = 0; i < NCH; ++i) {
       const int c = gl + i * GT;
@@ -305,8 +308,8 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
         load8_gain(a.gw, 8 * c, gw);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          v[i][e] = nq_r(v[i][e], gw[e], rhh, rlh) * (a.pre_act ? g[i][e] : siluf_(g[i][e]));
-          ss += (double)v[i][e] * (double)v[i][e];
+          v[i][e] = __fmul_rn(__fmul_rn(v[i][e], rfh), gw[e]) * (a.pre_act ? g[i][e] : siluf_(g[i][e]));
+          ss = fmaf(v[i][e], v[i][e], ss);
         }
       }
     }
@@ -325,31 +328,31 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
           for (int e = 0; e < 8; ++e) v[i][e] = (a.pre_act ? v[i][e] : siluf_(v[i][e])) * up[e];
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss += (double)v[i][e] * (double)v[i][e];
+        for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
       }
     }
   }
-  const double rinv = 1.0 / sqrt(nq_group_sum<W>(ss, redd, phd) / (double)k + (double)a.eps);
-  float rh, rl;
-  nq_split(rinv, rh, rl);
-  // maxima of |r| for every gain in one pass and one exchange
+  const float rf = nq_rinv(nq_group_sum<W>(ss, reds, phs), k, a.eps);
+  // v <- v / rms (shared by every gain), then the maxima of |r| = |v * gain| in one exchange
   float amax[3] = {0.0f, 0.0f, 0.0f};
 #pragma unroll
-  for (int j = 0; j < 3; ++j) {
-    if (j < a.ngain) {
+  for (int i = 0; i < NCH; ++i) {
+    const int c = gl + i * GT;
+    if (active && c < nck) {
 #pragma unroll
-      for (int i = 0; i < NCH; ++i) {
-        const int c = gl + i * GT;
-        if (active && c < nck) {
+      for (int e = 0; e < 8; ++e) v[i][e] = __fmul_rn(v[i][e], rf);
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        if (j < a.ngain) {
           float gg[8];
           load8_gain(a.gain[j], 8 * c, gg);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) amax[j] = fmaxf(amax[j], fabsf(nq_r(v[i][e], gg[e], rh, rl)));
+          for (int e = 0; e < 8; ++e) amax[j] = fmaxf(amax[j], fabsf(__fmul_rn(v[i][e], gg[e])));
         }
       }
     }
   }
-  nq_group_max3<W>(amax, redf, phf);
+  nq_group_max3<W>(amax, redm, phm);
   if (!active) return;
 #pragma unroll
   for (int j = 0; j < 3; ++j) {
@@ -364,13 +367,11 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
         if (c < nck) {
           float gg[8];
           load8_gain(gn, 8 * c, gg);
-          uint32_t w[2] = {0u, 0u};
+          uint32_t q[8];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int qv = (int)fminf(fmaxf(rintf(__fmul_rn(nq_r(v[i][e], gg[e], rh, rl), sx)), -127.0f), 127.0f);
-            w[e >> 2] |= ((uint32_t)qv & 0xFFu) << (8 * (e & 3));
-          }
-          *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(w[0], w[1]);
+          for (int e = 0; e < 8; ++e) q[e] = q8_code(__fmul_rn(__fmul_rn(v[i][e], gg[e]), sx));
+          *reinterpret_cast<uint2*>(qrow + 8 * c) =
+              make_uint2(pack4_lo_bytes(q[0], q[1], q[2], q[3]), pack4_lo_bytes(q[4], q[5], q[6], q[7]));
         }
       }
       for (int c = nck + gl; c < (int)(a.ldq >> 3); c += GT) *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(0u, 0u);
@@ -398,6 +399,8 @@ struct GemmSeg {
   int64_t ldacc;
   int32_t act;           // activation applied to output columns [0, act_cols): kActNone/Silu/SigmoidNeg
   int32_t act_cols;
+  int32_t glu;           // 1: codes are [2 * glu_inner][kw] (gate rows, then up rows) and the output
+  int32_t glu_inner;     //    is v[row][col] = SiLU(gate col) * up col, col < glu_inner (tensor engine)
 };
 
 struct GemmArgs {

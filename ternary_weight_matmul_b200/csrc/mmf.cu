@@ -272,11 +272,17 @@ bool use_tensor_path(int64_t m) {
   return m > kSimtMT;
 }
 
+// gate_proj forms the GLU product in its epilogue when the tensor engine runs it and the inner
+// size splits into 64-row gate/up tile halves.
+bool glu_fused(int64_t m, int32_t inner) { return use_tensor_path(m) && inner % tc::GLU_ROWS == 0; }
+
 mmf_status launch_gemm(const GemmArgs& g, const DevInfo& di, cudaStream_t st) {
   if (g.m == 0) return MMF_OK;
   if (!use_tensor_path(g.m)) {
     int maxn = 0;
     for (int s = 0; s < g.nseg; ++s) maxn = std::max(maxn, g.seg[s].n);
+    for (int s = 0; s < g.nseg; ++s)
+      if (g.seg[s].glu) return fail(MMF_ERR_UNSUPPORTED, "GLU segments run on the tensor engine only");
     const int nchunk = g.kw / 4;
     const size_t smem = (size_t)kSimtMT * nchunk * 4 * sizeof(uint4);
     if (smem > 200 * 1024) return fail(MMF_ERR_UNSUPPORTED, "K=%d too large for the CUDA-core engine", g.k);
@@ -298,16 +304,19 @@ mmf_status launch_gemm(const GemmArgs& g, const DevInfo& di, cudaStream_t st) {
   int32_t tiles = 0;
   for (int s = 0; s < g.nseg; ++s) {
     const GemmSeg& S = g.seg[s];
+    if (S.glu && (S.glu_inner % tc::GLU_ROWS != 0 || S.n != 2 * S.glu_inner || S.acc != nullptr || S.res != nullptr))
+      return fail(MMF_ERR_INVALID_ARG, "GLU segment needs inner %% 64 == 0, n == 2 * inner, no taps, no residual");
     P.tile_start[s] = tiles;
-    tiles += ((S.n + tc::BM - 1) / tc::BM) * P.m_tiles;
+    tiles += (S.glu ? S.glu_inner / tc::GLU_ROWS : (S.n + tc::BM - 1) / tc::BM) * P.m_tiles;
     MMF_TRY(encode_2d(&P.act_map[s], CU_TENSOR_MAP_DATA_TYPE_UINT8, S.q, (uint64_t)g.ldq,
-                      (uint64_t)g.m, (uint64_t)g.ldq, tc::BK, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B));
+                      (uint64_t)g.m, (uint64_t)g.ldq, tc::ACT_BOX, tc::BN, CU_TENSOR_MAP_SWIZZLE_128B));
     MMF_TRY(encode_2d(&P.w_map[s], CU_TENSOR_MAP_DATA_TYPE_UINT32, S.codes, (uint64_t)g.kw,
-                      (uint64_t)S.n, (uint64_t)g.kw * 4, tc::W_WORDS_PER_ROW, tc::BM,
-                      CU_TENSOR_MAP_SWIZZLE_NONE));
+                      (uint64_t)S.n, (uint64_t)g.kw * 4, tc::W_WORDS_PER_ROW,
+                      S.glu ? tc::GLU_ROWS : tc::BM, CU_TENSOR_MAP_SWIZZLE_64B));
   }
   P.tile_start[g.nseg] = tiles;
   P.num_kb = (int32_t)((g.ldq + tc::BK - 1) / tc::BK);
+  P.small_acc = (int64_t)127 * g.k < ((int64_t)1 << 22) ? 1 : 0;
   P.wait_limit_us = g_wait_limit.load();
   const int grid = std::min(tiles, di.sms);
   double ops = 0;
@@ -566,16 +575,22 @@ mmf_status run_block(const mmf_block_weights* w, const void* x, mmf_dtype dt, in
   nq.x = W.x1; nq.ldx = d; nq.xdt = dt; nq.m = m; nq.k = d; nq.eps = w->eps; nq.ngain = 1;
   nq.gain[0] = w->nw_gate; nq.q[0] = W.qg; nq.deq[0] = deq + 4 * m; nq.ldq = ldq_d;
   MMF_TRY(launch_norm_quant(nq, kRowPlain, st));
-  // 7. gate_proj: gu = [a | c]
+  // 7. gate_proj. The tensor engine pairs gate and up rows in one tile and writes
+  //    v = SiLU(gate) * up directly ([m][inner] in the gu buffer); otherwise gu = [gate | up].
+  const bool fuse_glu = glu_fused(m, inner);
   memset(&g, 0, sizeof(g));
   g.m = m; g.k = d; g.kw = row_words(d); g.ldq = ldq_d; g.ydt = dt; g.nseg = 1;
-  g.seg[0] = make_seg(W.qg, deq + 4 * m, w->gate, W.gu, 2 * inner, 0, nullptr, 0, nullptr, 0);
+  g.seg[0] = make_seg(W.qg, deq + 4 * m, w->gate, W.gu, fuse_glu ? inner : 2 * inner, 0, nullptr, 0, nullptr, 0);
+  if (fuse_glu) {
+    g.seg[0].glu = 1;
+    g.seg[0].glu_inner = inner;
+  }
   MMF_TRY(launch_gemm(g, di, st));
-  // 8. v = SiLU(a) * c fused with down_proj's RMSNorm + quant
+  // 8. down_proj's RMSNorm + quant of v (formed here from [gate | up] when not fused above)
   memset(&nq, 0, sizeof(nq));
-  nq.x = W.gu; nq.ldx = 2 * inner; nq.xdt = dt; nq.m = m; nq.k = inner; nq.eps = w->eps;
+  nq.x = W.gu; nq.ldx = fuse_glu ? inner : 2 * inner; nq.xdt = dt; nq.m = m; nq.k = inner; nq.eps = w->eps;
   nq.ngain = 1; nq.gain[0] = w->nw_down; nq.q[0] = W.qd; nq.deq[0] = deq + 5 * m; nq.ldq = ldq_i;
-  MMF_TRY(launch_norm_quant(nq, kRowGlu, st));
+  MMF_TRY(launch_norm_quant(nq, fuse_glu ? kRowPlain : kRowGlu, st));
   // 9. down_proj + residual: y = x1 + down_proj(v)
   memset(&g, 0, sizeof(g));
   g.m = m; g.k = inner; g.kw = row_words(inner); g.ldq = ldq_i; g.ydt = dt; g.nseg = 1;
@@ -812,7 +827,8 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
   MMF_TRY(copy2d(taps->x1, d * es, W.x1, d * es, d * es, m));
   MMF_TRY(copy2d(taps->q_gate, d, W.qg, row_q(d), d, m));
   MMF_TRY(copy2d(taps->deq_gate, m * 4, W.deq + 4 * m, m * 4, m * 4, 1));
-  MMF_TRY(copy2d(taps->gu, 2 * inner * es, W.gu, 2 * inner * es, 2 * inner * es, m));
+  if (glu_fused(m, inner)) MMF_TRY(copy2d(taps->v, inner * es, W.gu, inner * es, inner * es, m));
+  else MMF_TRY(copy2d(taps->gu, 2 * inner * es, W.gu, 2 * inner * es, 2 * inner * es, m));
   MMF_TRY(copy2d(taps->q_down, inner, W.qd, row_q(inner), inner, m));
   MMF_TRY(copy2d(taps->deq_down, m * 4, W.deq + 5 * m, m * 4, m * 4, 1));
   return MMF_OK;

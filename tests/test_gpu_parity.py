@@ -150,6 +150,32 @@ def test_bitlinear_engines_bit_identical(mmf, m):
     assert torch.equal(outs[0][0], outs[1][0])   # rescaled outputs
 
 
+@pytest.mark.parametrize("m,n,k", [(4096, 9472, 1024), (4096, 2048, 2816)])
+def test_bitlinear_large_sampled_rows(mmf, m, n, k):
+    # enough weight tiles that the tensor-core engine groups several of them per resident
+    # activation block (K <= 1024) or streams (K > 1024); checked on sampled rows
+    mmf.set_gemm_path(mmf.MMF_GEMM_TENSOR)
+    try:
+        x = synth.activations(70 + k, (m, k))
+        W = synth.weight(71 + k, n, k)
+        pt = mmf.pack_ternary(_to(W))
+        y, q, deq, acc = mmf.bitlinear_fwd(_to(x), None, pt, debug=True)
+        _ok(mmf)
+    finally:
+        mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
+    rows = np.random.default_rng(72).choice(m, 48, replace=False)
+    rows = np.concatenate([rows, [0, 127, 128, m - 1]])
+    t, s = O.ternarize(W)
+    q_g = q[rows].cpu().numpy()
+    acc_g = acc[rows].cpu().numpy()
+    assert np.array_equal(acc_g.astype(np.int64), O.int_matmul(q_g, t))
+    y_ref, taps = O.bitlinear(x[rows].astype(np.float64), None, t, s)
+    mism = q_g != taps["q"]
+    assert np.all(_near_tie(taps["v"])[mism])
+    ok = ~mism.any(axis=1)
+    np.testing.assert_allclose(y[rows].cpu().numpy()[ok], y_ref[ok], rtol=RTOL32, atol=ATOL32)
+
+
 # ---------------------------------------------------------------------------------------------
 # HGRN scan
 # ---------------------------------------------------------------------------------------------
@@ -231,7 +257,7 @@ def _close(got, want, bf16):
         np.testing.assert_allclose(got, want, rtol=RTOL32, atol=ATOL32)
 
 
-def check_block_stages(x, qp, taps, y_g, hl_g, h0, bf16):
+def check_block_stages(x, qp, taps, y_g, hl_g, h0, bf16, glu_fused=False):
     """Stage-wise parity: each stage of the kernel's block forward against the oracle's definition
     of that stage applied to the kernel's own inputs to it. Integer accumulations are exact; codes
     of the first quantisation match exactly, chained ones up to near-ties; floats elementwise."""
@@ -268,11 +294,17 @@ def check_block_stages(x, qp, taps, y_g, hl_g, h0, bf16):
     q_gate = _np(taps["q_gate"])
     _codes_match(q_gate, vg, qg, 1e-3)
     gu_ref = O.int_matmul(q_gate, qp["t_gate"]) * _np(taps["deq_gate"]).astype(np.float64)[:, None] * float(qp["s_gate"])
-    gu = _np(taps["gu"]).astype(np.float64)
-    _close(gu, gu_ref, bf16)
-    # 7. GLU + down_proj codes, 8. down_proj + residual
-    inner = gu.shape[1] // 2
-    qd, _, vd = O.act_quant(O.rmsnorm(O.silu(gu[:, :inner]) * gu[:, inner:], qp["nw_down"]))
+    inner = gu_ref.shape[1] // 2
+    # 7. GLU: v = SiLU(gate) * up, formed by gate_proj's epilogue or from the stored halves
+    if glu_fused:
+        v = _np(taps["v"]).astype(np.float64)
+        _close(v, O.silu(gu_ref[:, :inner]) * gu_ref[:, inner:], bf16)
+    else:
+        gu = _np(taps["gu"]).astype(np.float64)
+        _close(gu, gu_ref, bf16)
+        v = O.silu(gu[:, :inner]) * gu[:, inner:]
+    #    + down_proj codes, 8. down_proj + residual
+    qd, _, vd = O.act_quant(O.rmsnorm(v, qp["nw_down"]))
     q_down = _np(taps["q_down"])
     _codes_match(q_down, vd, qd, 1e-3)
     y_ref = x1 + O.int_matmul(q_down, qp["t_down"]) * _np(taps["deq_down"]).astype(np.float64)[:, None] * float(qp["s_down"])
@@ -312,10 +344,12 @@ def test_block_parity_tiny_config_f32(mmf, engine):
         y, hl, taps = mmf.block_fwd_taps(blk, _to(x))
         y2, hl2 = mmf.block_fwd(blk, _to(x))
         _ok(mmf)
+        fused = mmf.glu_fused(2 * 128, 704)
     finally:
         mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
+    assert fused == (engine != "simt")
     assert torch.equal(y, y2) and torch.equal(hl, hl2)   # taps variant runs the same path
-    check_block_stages(x, qp, taps, y.cpu().numpy(), hl.cpu().numpy(), None, bf16=False)
+    check_block_stages(x, qp, taps, y.cpu().numpy(), hl.cpu().numpy(), None, bf16=False, glu_fused=fused)
     y_ref, h_ref, inter = O.block_forward(x.astype(np.float64), qp)
     check_block_end_to_end(y.cpu().numpy(), y_ref, inter, qp, bf16=False)
     np.testing.assert_allclose(hl.cpu().numpy(), h_ref, rtol=RTOL32, atol=ATOL32 * 10)
@@ -332,8 +366,26 @@ def test_block_parity_ragged_with_state(mmf, dtype):
     y, hl, taps = mmf.block_fwd_taps(blk, _to(x, torch.bfloat16 if bf16 else torch.float32), _to(h0))
     _ok(mmf)
     yg = _np(y)
-    check_block_stages(x, qp, taps, yg, hl.cpu().numpy(), h0, bf16=bf16)
+    check_block_stages(x, qp, taps, yg, hl.cpu().numpy(), h0, bf16=bf16, glu_fused=mmf.glu_fused(3 * 37, 704))
     y_ref, h_ref, inter = O.block_forward(x.astype(np.float64), qp, h0)
+    check_block_end_to_end(yg, y_ref, inter, qp, bf16=bf16)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_block_parity_inner_not_multiple_of_64(mmf, dtype):
+    # I = 720 does not split into 64-row gate/up halves: gate_proj stores [gate | up] and the
+    # GLU is formed by down_proj's norm kernel, on the tensor-core engine as well
+    bf16 = dtype == "bf16"
+    params, qp, blk = _block_case(mmf, 13, 256, 720)
+    x = synth.activations(14, (2, 50, 256))
+    if bf16:
+        x = _bf16_round(x)
+    assert not mmf.glu_fused(100, 720)
+    y, hl, taps = mmf.block_fwd_taps(blk, _to(x, torch.bfloat16 if bf16 else torch.float32))
+    _ok(mmf)
+    yg = _np(y)
+    check_block_stages(x, qp, taps, yg, hl.cpu().numpy(), None, bf16=bf16, glu_fused=False)
+    y_ref, h_ref, inter = O.block_forward(x.astype(np.float64), qp)
     check_block_end_to_end(yg, y_ref, inter, qp, bf16=bf16)
 
 
