@@ -178,17 +178,16 @@ __global__ void __launch_bounds__(256) norm_quant_kernel(const NormQuantArgs a) 
 }
 
 // Vectorised variant for K % 8 == 0 and 16-byte aligned rows (K <= 8192): a row group of W
-// warps owns one row and keeps it in registers (at most 4 chunks of 8 values per thread), loads
-// and stores whole 16-/8-byte pieces and reduces with shuffles (plus one double-buffered shared
-// exchange per reduction when W > 1).
+// warps owns one row and keeps it in registers (NCH chunks of 8 values per thread), loads and
+// stores whole 16-/8-byte pieces and reduces with shuffles (plus one double-buffered shared
+// exchange per reduction when W > 1). NG is 1 or 3 norm gains sharing the row's rms.
 //
 // Arithmetic: r = (v * (1/rms)) * gain in float32, a = max|r|, code = rint(r * (127/a)). The
 // factor 1/rms cancels between r and a, so the codes depend on the mean square only through the
 // float32 rounding of r (a relative perturbation of the mean square moves r * 127/a by a few
-// ulp at most); the sum of squares therefore runs in float32 and only the final 1/sqrt is formed
-// in float64. The dequantisation factor a/127 carries the mean square's own rounding (~1e-7).
+// ulp at most); the sum of squares and 1/sqrt therefore run in float32 (each step IEEE-rounded).
+// The dequantisation factor a/127 carries the mean square's own rounding (~1e-7 relative).
 constexpr int kNqThreads = 256;
-constexpr int kNqMaxChunks = 4;
 
 template <int W>
 __device__ __forceinline__ float nq_group_sum(float v, float (*red)[8], int& ph) {
@@ -204,22 +203,22 @@ __device__ __forceinline__ float nq_group_sum(float v, float (*red)[8], int& ph)
   for (int k = 0; k < W; ++k) s += r[g0 + k];
   return s;
 }
-// Maxima of three values over the row group (one exchange for all gains).
-template <int W>
-__device__ __forceinline__ void nq_group_max3(float (&v)[3], float (*red)[8][3], int& ph) {
+// Maxima of NG values over the row group (one exchange for all gains).
+template <int W, int NG>
+__device__ __forceinline__ void nq_group_max(float (&v)[NG], float (*red)[8][3], int& ph) {
 #pragma unroll
-  for (int j = 0; j < 3; ++j) v[j] = warp_max(v[j]);
+  for (int j = 0; j < NG; ++j) v[j] = warp_max(v[j]);
   if (W == 1) return;
   const int wid = threadIdx.x >> 5, g0 = (wid / W) * W;
   float(*r)[3] = red[ph & 1];
   ++ph;
   if ((threadIdx.x & 31) == 0) {
 #pragma unroll
-    for (int j = 0; j < 3; ++j) r[wid][j] = v[j];
+    for (int j = 0; j < NG; ++j) r[wid][j] = v[j];
   }
   __syncthreads();
 #pragma unroll
-  for (int j = 0; j < 3; ++j) {
+  for (int j = 0; j < NG; ++j) {
     float m = 0.0f;
 #pragma unroll
     for (int k = 0; k < W; ++k) m = fmaxf(m, r[g0 + k][j]);
@@ -256,16 +255,15 @@ __device__ __forceinline__ void load8_gain(const float* g, int64_t idx, float (&
   o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
   o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
 }
-// 1 / sqrt(ss / k + eps), formed in float64 from the float32 sum and rounded once.
+// 1 / sqrt(ss / k + eps) in float32 (IEEE division and square root).
 __device__ __forceinline__ float nq_rinv(float ss, int k, float eps) {
-  return (float)(1.0 / sqrt((double)ss / (double)k + (double)eps));
+  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)k), eps)));
 }
-// int8 code of x: clamp to [-127, 127], then round half to even by adding 1.5 * 2^23 (where the
-// float32 spacing is exactly 1, so the IEEE round-to-nearest-even addition does the rounding)
-// and reading the integer back from the low mantissa bits.
-__device__ __forceinline__ uint32_t q8_code(float x) {
-  const float c = fminf(fmaxf(x, -127.0f), 127.0f);
-  return (uint32_t)(__float_as_int(__fadd_rn(c, 12582912.0f)) - 0x4B400000);
+// Bits of clamp(x, -127, 127) + 1.5 * 2^23: the addition (where the float32 spacing is exactly
+// 1) rounds half to even, and the low byte of the result is the int8 code rint(x) itself
+// (0x4B400000 has a zero low byte, and the code lies in [-127, 127]).
+__device__ __forceinline__ uint32_t q8_bits(float x) {
+  return __float_as_uint(__fadd_rn(fminf(fmaxf(x, -127.0f), 127.0f), 12582912.0f));
 }
 // Low bytes of four words packed into one word, a in byte 0.
 __device__ __forceinline__ uint32_t pack4_lo_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -273,7 +271,7 @@ __device__ __forceinline__ uint32_t pack4_lo_bytes(uint32_t a, uint32_t b, uint3
 }
 
 // Row group of W warps per row, NCH chunks of 8 values per thread (K <= 256 * W * NCH).
-template <mmf_dtype XT, int MODE, int W, int NCH>
+template <mmf_dtype XT, int MODE, int W, int NCH, int NG>
 __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQuantArgs a) {
   constexpr int GT = 32 * W;
   __shared__ float reds[2][8];
@@ -333,31 +331,42 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
     }
   }
   const float rf = nq_rinv(nq_group_sum<W>(ss, reds, phs), k, a.eps);
-  // v <- v / rms (shared by every gain), then the maxima of |r| = |v * gain| in one exchange
-  float amax[3] = {0.0f, 0.0f, 0.0f};
+  // v <- v / rms (and, with one gain, <- r = v / rms * gain); maxima of |r| per gain
+  float amax[NG];
+#pragma unroll
+  for (int j = 0; j < NG; ++j) amax[j] = 0.0f;
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int c = gl + i * GT;
     if (active && c < nck) {
+      if (NG == 1) {
+        float gg[8];
+        load8_gain(a.gain[0], 8 * c, gg);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) v[i][e] = __fmul_rn(v[i][e], rf);
+        for (int e = 0; e < 8; ++e) {
+          v[i][e] = __fmul_rn(__fmul_rn(v[i][e], rf), gg[e]);
+          amax[0] = fmaxf(amax[0], fabsf(v[i][e]));
+        }
+      } else {
 #pragma unroll
-      for (int j = 0; j < 3; ++j) {
-        if (j < a.ngain) {
-          float gg[8];
-          load8_gain(a.gain[j], 8 * c, gg);
+        for (int e = 0; e < 8; ++e) v[i][e] = __fmul_rn(v[i][e], rf);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) amax[j] = fmaxf(amax[j], fabsf(__fmul_rn(v[i][e], gg[e])));
+        for (int j = 0; j < NG; ++j) {
+          if (j < a.ngain) {
+            float gg[8];
+            load8_gain(a.gain[j], 8 * c, gg);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) amax[j] = fmaxf(amax[j], fabsf(__fmul_rn(v[i][e], gg[e])));
+          }
         }
       }
     }
   }
-  nq_group_max3<W>(amax, redm, phm);
+  nq_group_max<W, NG>(amax, redm, phm);
   if (!active) return;
 #pragma unroll
-  for (int j = 0; j < 3; ++j) {
+  for (int j = 0; j < NG; ++j) {
     if (j < a.ngain) {
-      const float* gn = a.gain[j];
       const float am = fmaxf(amax[j], 1e-5f);
       const float sx = __fdiv_rn(127.0f, am);
       int8_t* qrow = a.q[j] + row * a.ldq;
@@ -365,11 +374,16 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
       for (int i = 0; i < NCH; ++i) {
         const int c = gl + i * GT;
         if (c < nck) {
-          float gg[8];
-          load8_gain(gn, 8 * c, gg);
           uint32_t q[8];
+          if (NG == 1) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) q[e] = q8_code(__fmul_rn(__fmul_rn(v[i][e], gg[e]), sx));
+            for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(v[i][e], sx));
+          } else {
+            float gg[8];
+            load8_gain(a.gain[j], 8 * c, gg);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(__fmul_rn(v[i][e], gg[e]), sx));
+          }
           *reinterpret_cast<uint2*>(qrow + 8 * c) =
               make_uint2(pack4_lo_bytes(q[0], q[1], q[2], q[3]), pack4_lo_bytes(q[4], q[5], q[6], q[7]));
         }

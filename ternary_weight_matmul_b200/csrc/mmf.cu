@@ -215,22 +215,30 @@ struct LaunchScope {
 // ---------------------------------------------------------------------------------------------
 // internal launchers
 // ---------------------------------------------------------------------------------------------
-template <mmf_dtype XT, int MODE>
+template <mmf_dtype XT, int MODE, int NG>
 void nq_vec_launch(const NormQuantArgs& a, int w, int nch, cudaStream_t st) {
   const unsigned rows_per_cta = 8u / (unsigned)w;
   const dim3 grid((unsigned)((a.m + rows_per_cta - 1) / rows_per_cta));
-  if (w == 1) norm_quant_vec_kernel<XT, MODE, 1, 2><<<grid, kNqThreads, 0, st>>>(a);
-  else if (w == 2) norm_quant_vec_kernel<XT, MODE, 2, 2><<<grid, kNqThreads, 0, st>>>(a);
-  else if (w == 4) norm_quant_vec_kernel<XT, MODE, 4, 2><<<grid, kNqThreads, 0, st>>>(a);
-  else if (nch <= 2) norm_quant_vec_kernel<XT, MODE, 8, 2><<<grid, kNqThreads, 0, st>>>(a);
-  else norm_quant_vec_kernel<XT, MODE, 8, 4><<<grid, kNqThreads, 0, st>>>(a);
+#define MMF_NQ(W_, C_) norm_quant_vec_kernel<XT, MODE, W_, C_, NG><<<grid, kNqThreads, 0, st>>>(a)
+#define MMF_NQ_W(W_) \
+  do { if (nch <= 2) MMF_NQ(W_, 2); else if (nch <= 4) MMF_NQ(W_, 4); else if (nch <= 6) MMF_NQ(W_, 6); else MMF_NQ(W_, 8); } while (0)
+  if (w == 1) MMF_NQ_W(1);
+  else if (w == 2) MMF_NQ_W(2);
+  else MMF_NQ_W(4);
+#undef MMF_NQ_W
+#undef MMF_NQ
 }
 
 template <mmf_dtype XT>
 void nq_vec_dispatch(const NormQuantArgs& a, int mode, int w, int nch, cudaStream_t st) {
-  if (mode == kRowPlain) nq_vec_launch<XT, kRowPlain>(a, w, nch, st);
-  else if (mode == kRowGlu) nq_vec_launch<XT, kRowGlu>(a, w, nch, st);
-  else nq_vec_launch<XT, kRowGnorm>(a, w, nch, st);
+  if (mode == kRowPlain) {
+    if (a.ngain == 1) nq_vec_launch<XT, kRowPlain, 1>(a, w, nch, st);
+    else nq_vec_launch<XT, kRowPlain, 3>(a, w, nch, st);
+  } else if (mode == kRowGlu) {
+    nq_vec_launch<XT, kRowGlu, 1>(a, w, nch, st);
+  } else {
+    nq_vec_launch<XT, kRowGnorm, 1>(a, w, nch, st);
+  }
 }
 
 inline bool al16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -243,14 +251,16 @@ mmf_status launch_norm_quant(const NormQuantArgs& a, int mode, cudaStream_t st) 
   LaunchScope ls(MMF_KERNEL_NORM_QUANT, (double)a.m * (in_row + a.ngain * ((double)a.ldq + 4.0)), st);
   // row-group-in-registers variant when sizes and alignment allow it
   const size_t xes = dsize(a.xdt);
-  bool vec = a.k % 8 == 0 && a.k <= 8 * 32 * 8 * kNqMaxChunks && al16(a.x) && (a.ldx * xes) % 16 == 0;
+  bool vec = a.k % 8 == 0 && a.k <= 8 * 32 * 4 * 8 && al16(a.x) && (a.ldx * xes) % 16 == 0 &&
+             (mode == kRowPlain || a.ngain == 1);
   if (mode == kRowGnorm)
     vec = vec && a.gdt == a.xdt && al16(a.g) && (a.ldg * xes) % 16 == 0 && al16(a.gw);
   for (int j = 0; j < a.ngain; ++j) vec = vec && al16(a.gain[j]) && al16(a.q[j]);
   if (vec) {
-    // smallest row group holding the row at two 8-value chunks per thread (four beyond 4096)
+    // smallest row group (1, 2 or 4 warps) holding the row at up to eight 8-value chunks per
+    // thread, so the per-row reductions are amortised over many values
     const int nck = a.k / 8;
-    const int w = nck <= 64 ? 1 : nck <= 128 ? 2 : nck <= 256 ? 4 : 8;
+    const int w = nck <= 256 ? 1 : nck <= 512 ? 2 : 4;
     const int nch = (nck + 32 * w - 1) / (32 * w);
     if (a.xdt == MMF_F32) nq_vec_dispatch<MMF_F32>(a, mode, w, nch, st);
     else nq_vec_dispatch<MMF_BF16>(a, mode, w, nch, st);
