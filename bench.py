@@ -30,6 +30,9 @@ WORKLOADS = {
     "prefill-370M": dict(d=1024, inner=2816, layers=24, vocab=32000, batch=8, seq=2048),
     "prefill-1.3B": dict(d=2048, inner=5632, layers=24, vocab=32000, batch=16, seq=2048),
 }
+# Autoregressive decode of the 2.7B-shape stack: a 512-token prompt (prefill, untimed) then
+# decode steps with the recurrent state carried per layer, at three batch sizes.
+DECODE = dict(name="decode-2.7B", d=2560, inner=7040, layers=32, vocab=32000, prompt=512, batches=(1, 8, 64))
 
 
 def parse():
@@ -41,6 +44,8 @@ def parse():
     ap.add_argument("--workload", default="prefill-370M", choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-steps", type=int, default=64)
     return ap.parse_args()
 
 
@@ -202,6 +207,75 @@ def build_model(wl, device, seed=1234):
     return blocks, table
 
 
+def run_decode(args, device, hbm_peak):
+    """Decode-step throughput of the 2.7B-shape stack for each batch size: prompt prefill through
+    mmf_stack_fwd (untimed, gives every layer's recurrent state), then `--decode-steps` steps of
+    embedding gather + mmf_decode_step replayed from a CUDA graph (one graph per step, captured
+    after warm-up), timed with CUDA events on the replay stream. Token ids are pre-drawn (the LM
+    head is outside the block stack). HBM roofline: every step streams all packed weights."""
+    import torch
+
+    import ternary_weight_matmul_b200 as mmf
+
+    dw = DECODE
+    blocks, table = build_model(dw, device, seed=2718)
+    weight_bytes = 0
+    for blk in blocks:
+        for p in blk.packed.values():
+            weight_bytes += p.codes.numel() * 4 + 4
+        weight_bytes += sum(t.numel() * 4 for t in blk.norms.values())
+    out = {"workload": dw["name"], "layers": dw["layers"], "hidden": dw["d"], "inner": dw["inner"],
+           "prompt": dw["prompt"], "steps": args.decode_steps, "unit": "tokens/s",
+           "bytes_per_step_weights": weight_bytes, "batches": {}}
+    for B in dw["batches"]:
+        g = torch.Generator(device="cpu")
+        g.manual_seed(99 + B)
+        prompt = torch.randint(0, dw["vocab"], (B, dw["prompt"]), generator=g, dtype=torch.int32).to(device)
+        steps_ids = torch.randint(0, dw["vocab"], (args.decode_steps + 8, B), generator=g, dtype=torch.int32).to(device)
+        _, state = mmf.stack_fwd(blocks, prompt, table, want_state=True)
+        x = torch.empty(B, dw["d"], dtype=torch.bfloat16, device=device)
+        y = torch.empty_like(x)
+        cur = torch.zeros(B, dtype=torch.int32, device=device)
+        s = torch.cuda.Stream(device)
+
+        def step():
+            xx = mmf.embed_gather(cur, table)
+            x.copy_(xx)
+            mmf.decode_step(blocks, x, state, out=y)
+
+        with torch.cuda.stream(s):
+            for i in range(3):
+                cur.copy_(steps_ids[i])
+                step()
+        torch.cuda.synchronize(device)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=s):
+            step()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(s):
+            for i in range(3):
+                cur.copy_(steps_ids[3 + i])
+                graph.replay()
+            torch.cuda.synchronize(device)
+            ev0.record(s)
+            for i in range(args.decode_steps):
+                cur.copy_(steps_ids[i % steps_ids.shape[0]])
+                graph.replay()
+            ev1.record(s)
+        torch.cuda.synchronize(device)
+        st = mmf.sync_status(device)
+        if st != 0:
+            raise RuntimeError(f"device status {st} in decode")
+        ms = ev0.elapsed_time(ev1) / args.decode_steps
+        gbs = weight_bytes / (ms / 1e3) / 1e9
+        out["batches"][str(B)] = {"value": B / (ms / 1e3), "ms_per_step": ms, "GB/s_weights": gbs,
+                                  "frac_hbm": gbs / hbm_peak}
+        del graph
+    del blocks, table
+    torch.cuda.empty_cache()
+    return out
+
+
 def run_gpu(args, wl):
     import torch
     import torch.distributed as dist
@@ -301,6 +375,12 @@ def run_gpu(args, wl):
         e2e = {"value": tokens / (float(e_t.item()) / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": ids_host.numel() * 4, "d2h_bytes_per_step": y_host.numel() * 2}
 
+    decode = None
+    if not args.no_decode and rank == 0:
+        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        hbm = json.load(open(pp)).get("hbm_gbs", 6650.0) if os.path.exists(pp) else 6650.0
+        decode = run_decode(args, device, hbm)
+
     line = None
     if rank == 0:
         peaks = {}
@@ -347,6 +427,7 @@ def run_gpu(args, wl):
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
             "gpu_launches_per_step": gpu_launches / args.steps, "clocks": clk,
             "step_ms_all": [round(v, 4) for v in step_ms],
+            "decode": decode,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
