@@ -1,0 +1,338 @@
+// decode.cuh -- K8: fused decode projections for up to 8 token rows (one autoregressive step).
+//
+// One decode step of a block is four launches of dec_proj_kernel, one per projection group, each
+// with its producer and consumer steps fused in:
+//   kIFG   RMSNorm + int8 quantisation of x with the i/f/g gains (prologue), the i, f and g
+//          products, and the HGRN gates + one recurrence step h = f h_prev + i on the carried
+//          state (epilogue; writes h and g in float32);
+//   kO     g_norm u = RMSNorm(h) * w_g * SiLU(g) and o_proj's RMSNorm + quantisation (prologue),
+//          o_proj and the residual x1 = x + o (epilogue);
+//   kGate  gate_proj's RMSNorm + quantisation of x1, gate and up rows of the same channels, and
+//          v = SiLU(gate) * up (epilogue);
+//   kDown  down_proj's RMSNorm + quantisation of v, down_proj and y = x1 + down (epilogue).
+// Each CTA owns a contiguous range of output channels. Its first thread starts bulk copies of
+// the input's norm gains and of the CTA's packed weight rows into shared memory (two barriers);
+// while the weights stream in, the CTA quantises the input rows itself -- every CTA computes the
+// same codes, in the arithmetic of norm_quant_vec_kernel -- and each warp then forms whole
+// output channels: lanes stride over 64-code chunks of the weight row (expanded with byte
+// permutes), dp4a against the codes, and a warp reduction per (matrix, row).
+#pragma once
+
+#include "common.cuh"
+#include "kernels.cuh"
+
+namespace mmf {
+namespace dec {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxRows = 8;            // token rows per launch
+constexpr int kMaxSmem = 200 * 1024;   // dynamic shared memory budget per CTA
+
+enum Mode : int32_t { kIFG = 0, kO = 1, kGate = 2, kDown = 3 };
+
+struct Args {
+  int32_t mode;
+  int32_t b;              // token rows (1..8)
+  int32_t k;              // input features
+  int32_t kw;             // packed words per weight row (4 * ceil(k / 64))
+  int32_t nout;           // output channels
+  int32_t chan_per_cta;
+  int32_t nmat;           // weight rows per channel: kIFG 3 (i, f, g), kGate 2 (gate, up), else 1
+  int32_t ngain;          // quantisations of the input: kIFG 3 (one per gain), else 1
+  float eps;
+  const uint32_t* w[3];   // weight row c of matrix j: w[j] + (row_off[j] + c) * kw
+  int32_t row_off[3];
+  const float* sw[3];     // weight scales
+  const float* gain[3];   // RMSNorm gains of the input (kIFG: i, f, g; else the projection's)
+  const void* x;          // input rows [b][k]: x (kIFG), x1 (kGate), v (kDown), dtype xdt
+  mmf_dtype xdt;
+  const float* h;         // kO: h [b][k] float32
+  const float* gin;       // kO: g [b][k] float32
+  const float* gnorm_w;   // kO: g_norm gain (nullable = 1)
+  const void* res;        // kO / kDown: residual [b][nout], dtype ydt
+  void* y;                // kIFG: h float32; kO: x1; kGate: v; kDown: y -- [b][nout]
+  mmf_dtype ydt;
+  float* g_out;           // kIFG: g [b][nout] float32
+  float* state;           // kIFG: recurrent state [b][nout] float32, read and overwritten
+  uint32_t wait_limit_us;
+};
+
+// Shared-memory layout of one CTA: weight rows, norm gains (ngain vectors of k floats; kO also
+// the g_norm gain), the g_norm output u (kO only, [b][k] float32), the codes, factors, scratch.
+struct Smem {
+  size_t w_bytes, gain_off, u_off, q_off, q_bytes, deq_off, red_off, bar_off, total;
+};
+__host__ __device__ inline Smem smem_layout(int mode, int nmat, int chan_per_cta, int kw, int k, int ngain, int b) {
+  Smem s;
+  s.w_bytes = (size_t)nmat * chan_per_cta * kw * 4;
+  s.gain_off = (s.w_bytes + 127) & ~(size_t)127;
+  const int ngv = ngain + (mode == kO ? 1 : 0);
+  s.u_off = (s.gain_off + (size_t)ngv * k * 4 + 127) & ~(size_t)127;
+  const size_t u_bytes = mode == kO ? (size_t)b * k * 4 : 0;
+  s.q_off = (s.u_off + u_bytes + 127) & ~(size_t)127;
+  s.q_bytes = (size_t)ngain * b * kw * 16;   // codes of the padded K, [gain][row][piece][chunk]
+  s.deq_off = (s.q_off + s.q_bytes + 15) & ~(size_t)15;
+  s.red_off = s.deq_off + 3 * kMaxRows * sizeof(float);
+  s.bar_off = (s.red_off + (kWarps * 3 + 4) * kMaxRows * sizeof(float) + 7) & ~(size_t)7;
+  s.total = s.bar_off + 16;   // two mbarriers: gains, weights
+  return s;
+}
+
+// Untiled bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Input value k of token row r as the projection's RMSNorm sees it: the row itself, or for kO
+// the g_norm output u staged in shared memory.
+template <mmf_dtype XT>
+__device__ __forceinline__ void in8(const Args& a, const float* us, int r, int kk, float (&o)[8]) {
+  if (a.mode == kO) {
+    const float4 p = *reinterpret_cast<const float4*>(us + (size_t)r * a.k + kk);
+    const float4 q = *reinterpret_cast<const float4*>(us + (size_t)r * a.k + kk + 4);
+    o[0] = p.x; o[1] = p.y; o[2] = p.z; o[3] = p.w;
+    o[4] = q.x; o[5] = q.y; o[6] = q.z; o[7] = q.w;
+  } else {
+    load8<XT>(a.x, (int64_t)r * a.k + kk, o);
+  }
+}
+__device__ __forceinline__ void sm8(const float* p, float (&o)[8]) {
+  const float4 x = *reinterpret_cast<const float4*>(p);
+  const float4 y = *reinterpret_cast<const float4*>(p + 4);
+  o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+  o[4] = y.x; o[5] = y.y; o[6] = y.z; o[7] = y.w;
+}
+
+// The kernel runs once per SM for a few microseconds, so its instructions are fetched cold:
+// the code is kept compact (runtime loops over rows, gains and matrices; per-row statistics in
+// shared memory) rather than unrolled.
+template <mmf_dtype XT>
+__global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const Smem L = smem_layout(a.mode, a.nmat, a.chan_per_cta, a.kw, a.k, a.ngain, a.b);
+  uint32_t* wsm = reinterpret_cast<uint32_t*>(sm);
+  float* gains = reinterpret_cast<float*>(sm + L.gain_off);   // [ngain (+1)][k]
+  float* us = reinterpret_cast<float*>(sm + L.u_off);
+  int8_t* qs = reinterpret_cast<int8_t*>(sm + L.q_off);
+  float* deqs = reinterpret_cast<float*>(sm + L.deq_off);   // [gain][row] a/127
+  float* red = reinterpret_cast<float*>(sm + L.red_off);    // [warp][gain][row] partials, then stats
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar_off);
+  const int c0 = blockIdx.x * a.chan_per_cta;
+  const int nc = a.nout - c0 < a.chan_per_cta ? a.nout - c0 : a.chan_per_cta;
+  const uint32_t row_bytes = (uint32_t)a.kw * 4u;
+  const uint32_t gbytes = (uint32_t)a.k * 4u;
+  const bool has_gw = a.mode == kO && a.gnorm_w != nullptr;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int ng = a.ngain;
+
+  // 1. this CTA's weight rows and the norm gains into shared memory (absent gains are ones)
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+    uint32_t tx = 0;
+    for (int j = 0; j < ng; ++j) tx += a.gain[j] ? gbytes : 0u;
+    if (has_gw) tx += gbytes;
+    mbar_arrive_expect_tx(&bar[0], tx);
+    for (int j = 0; j < ng; ++j)
+      if (a.gain[j]) bulk_load(gains + (size_t)j * a.k, a.gain[j], gbytes, &bar[0]);
+    if (has_gw) bulk_load(gains + (size_t)ng * a.k, a.gnorm_w, gbytes, &bar[0]);
+    mbar_arrive_expect_tx(&bar[1], (uint32_t)a.nmat * (uint32_t)nc * row_bytes);
+    for (int j = 0; j < a.nmat; ++j)
+      bulk_load(wsm + (size_t)j * a.chan_per_cta * a.kw, a.w[j] + ((int64_t)a.row_off[j] + c0) * a.kw,
+                (uint32_t)nc * row_bytes, &bar[1]);
+  }
+  for (int j = 0; j < ng + (a.mode == kO ? 1 : 0); ++j) {
+    const bool absent = j < ng ? a.gain[j] == nullptr : !has_gw;
+    if (absent)
+      for (int t = threadIdx.x; t < a.k; t += kThreads) gains[(size_t)j * a.k + t] = 1.0f;
+  }
+  // (a timed-out wait drains both copies before the CTA leaves: shared memory must outlive them)
+  volatile int abort_flag = 0;
+  auto wait_or_leave = [&](int i) {
+    if (mbar_wait_bounded(&bar[i], 0u, a.wait_limit_us, &abort_flag)) return true;
+    for (int q = 0; q < 2; ++q) {
+      const int64_t t0 = clock64();
+      while (!mbar_try_wait(&bar[q], 0u) && clock64() - t0 < 1000000ll * kCyclesPerUs) {
+      }
+    }
+    return false;
+  };
+  if (!wait_or_leave(0)) return;
+
+  // 2. prologue: the codes of every input row (the same in every CTA).
+  const int nck = a.k >> 3;
+  const int kq = a.kw * 16;
+  float* rfs = red + kWarps * 3 * kMaxRows;          // [row] 1/rms
+  float* sxs = rfs + kMaxRows;                       // [gain][row] 127/a
+  // 2a. mean squares of every row (kO: of h, then u = h / rms(h) * w_g * SiLU(g) into shared
+  //     memory and its mean squares)
+  for (int pass = 0; pass < (a.mode == kO ? 2 : 1); ++pass) {
+    for (int r = 0; r < a.b; ++r) {
+      float ss = 0.0f;
+      for (int c = threadIdx.x; c < nck; c += kThreads) {
+        float v[8];
+        if (a.mode == kO && pass == 0) {
+          load8<MMF_F32>(a.h, (int64_t)r * a.k + 8 * c, v);
+        } else if (a.mode == kO) {
+          float g[8], w8[8];
+          load8<MMF_F32>(a.h, (int64_t)r * a.k + 8 * c, v);
+          load8<MMF_F32>(a.gin, (int64_t)r * a.k + 8 * c, g);
+          sm8(gains + (size_t)ng * a.k + 8 * c, w8);
+          const float rfh = rfs[r];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(__fmul_rn(v[e], rfh), w8[e]) * siluf_(g[e]);
+          float* up = us + (size_t)r * a.k + 8 * c;
+          *reinterpret_cast<float4*>(up) = make_float4(v[0], v[1], v[2], v[3]);
+          *reinterpret_cast<float4*>(up + 4) = make_float4(v[4], v[5], v[6], v[7]);
+        } else {
+          load8<XT>(a.x, (int64_t)r * a.k + 8 * c, v);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+      }
+      ss = warp_sum(ss);
+      if (lane == 0) red[warp * kMaxRows + r] = ss;
+    }
+    __syncthreads();
+    if (threadIdx.x < a.b) {
+      float t = 0.0f;
+      for (int w = 0; w < kWarps; ++w) t += red[w * kMaxRows + threadIdx.x];
+      rfs[threadIdx.x] = nq_rinv(t, a.k, a.eps);
+    }
+    __syncthreads();
+  }
+  // 2b. maxima of |r| = |v / rms * gain| per (gain, row)
+  for (int r = 0; r < a.b; ++r) {
+    const float rf = rfs[r];
+    for (int j = 0; j < ng; ++j) {
+      float am = 0.0f;
+      for (int c = threadIdx.x; c < nck; c += kThreads) {
+        float v[8], gg[8];
+        in8<XT>(a, us, r, 8 * c, v);
+        sm8(gains + (size_t)j * a.k + 8 * c, gg);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(__fmul_rn(__fmul_rn(v[e], rf), gg[e])));
+      }
+      am = warp_max(am);
+      if (lane == 0) red[(warp * 3 + j) * kMaxRows + r] = am;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < ng * kMaxRows) {
+    const int j = threadIdx.x / kMaxRows, r = threadIdx.x - j * kMaxRows;
+    if (r < a.b) {
+      float t = 0.0f;
+      for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[(w * 3 + j) * kMaxRows + r]);
+      t = fmaxf(t, 1e-5f);
+      sxs[j * kMaxRows + r] = __fdiv_rn(127.0f, t);
+      deqs[j * kMaxRows + r] = __fdiv_rn(t, 127.0f);
+    }
+  }
+  __syncthreads();
+  // 2c. codes, piece-major: code k of (gain j, row r) at
+  //     qs + (j * b + r) * kq + ((k % 64) / 16) * (kq / 4) + (k / 64) * 16 + k % 16
+  for (int r = 0; r < a.b; ++r) {
+    const float rf = rfs[r];
+    for (int j = 0; j < ng; ++j) {
+      const float sx = sxs[j * kMaxRows + r];
+      int8_t* qrow = qs + (size_t)(j * a.b + r) * kq;
+      for (int c = threadIdx.x; c < nck; c += kThreads) {
+        float v[8], gg[8];
+        in8<XT>(a, us, r, 8 * c, v);
+        sm8(gains + (size_t)j * a.k + 8 * c, gg);
+        uint32_t q[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(__fmul_rn(__fmul_rn(v[e], rf), gg[e]), sx));
+        const int kk = 8 * c;
+        *reinterpret_cast<uint2*>(qrow + ((kk & 63) >> 4) * (kq >> 2) + (kk >> 6) * 16 + (kk & 15)) =
+            make_uint2(pack4_lo_bytes(q[0], q[1], q[2], q[3]), pack4_lo_bytes(q[4], q[5], q[6], q[7]));
+      }
+    }
+  }
+  __syncthreads();
+
+  if (!wait_or_leave(1)) return;
+
+  // 3. one warp per output channel: each weight row against all token rows; lane r keeps the
+  //    total of token row r
+  const int nchunk = a.kw >> 2;           // 16-byte chunks (64 codes) per weight row
+  for (int cl = warp; cl < nc; cl += kWarps) {
+    int tot0 = 0, tot1 = 0, tot2 = 0;
+    for (int m = 0; m < a.nmat; ++m) {
+      const int gsel = ng == 3 ? m : 0;
+      int acc[kMaxRows];
+#pragma unroll
+      for (int r = 0; r < kMaxRows; ++r) acc[r] = 0;
+      const uint4* wrow = reinterpret_cast<const uint4*>(wsm + ((size_t)m * a.chan_per_cta + cl) * a.kw);
+      const int8_t* qg = qs + (size_t)gsel * a.b * kq;
+      for (int ch = lane; ch < nchunk; ch += 32) {
+        const uint4 wv = wrow[ch];
+        uint32_t e[16];
+        expand_word(wv.x, e + 0);
+        expand_word(wv.y, e + 4);
+        expand_word(wv.z, e + 8);
+        expand_word(wv.w, e + 12);
+#pragma unroll
+        for (int r = 0; r < kMaxRows; ++r) {
+          if (r < a.b) {
+            const int8_t* qr = qg + (size_t)r * kq + ch * 16;
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const uint4 av = *reinterpret_cast<const uint4*>(qr + p * (kq >> 2));
+              acc[r] = __dp4a((int)e[4 * p + 0], (int)av.x, acc[r]);
+              acc[r] = __dp4a((int)e[4 * p + 1], (int)av.y, acc[r]);
+              acc[r] = __dp4a((int)e[4 * p + 2], (int)av.z, acc[r]);
+              acc[r] = __dp4a((int)e[4 * p + 3], (int)av.w, acc[r]);
+            }
+          }
+        }
+      }
+      int mine = 0;
+#pragma unroll
+      for (int r = 0; r < kMaxRows; ++r) {
+        if (r < a.b) {
+          int s = acc[r];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (lane == r) mine = s;
+        }
+      }
+      if (m == 0) tot0 = mine;
+      else if (m == 1) tot1 = mine;
+      else tot2 = mine;
+    }
+    if (lane < a.b) {
+      const int r = lane;
+      const int c = c0 + cl;
+      const int64_t o = (int64_t)r * a.nout + c;
+      auto zof = [&](int m, int tot) {
+        const int gsel = ng == 3 ? m : 0;
+        return __fmul_rn((float)tot, __fmul_rn(deqs[gsel * kMaxRows + r], a.sw[m][0]));
+      };
+      if (a.mode == kIFG) {
+        // f = sigmoid(zf), i = SiLU(zi) * (1 - f), h = f * h_prev + i
+        const float zi = zof(0, tot0), zf = zof(1, tot1), zg = zof(2, tot2);
+        float f, omf;
+        hgrn_forget(zf, f, omf);
+        const float iv = siluf_(zi) * omf;
+        const float hv = f * a.state[o] + iv;
+        a.state[o] = hv;
+        reinterpret_cast<float*>(a.y)[o] = hv;
+        a.g_out[o] = zg;
+      } else if (a.mode == kGate) {
+        store_from_float(a.y, o, a.ydt, siluf_(zof(0, tot0)) * zof(1, tot1));
+      } else {
+        store_from_float(a.y, o, a.ydt, zof(0, tot0) + load_as_float(a.res, o, a.ydt));
+      }
+    }
+  }
+}
+
+}  // namespace dec
+}  // namespace mmf

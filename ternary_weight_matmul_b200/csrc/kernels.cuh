@@ -464,6 +464,21 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const GemmArgs a) {
   const int64_t m0 = (int64_t)blockIdx.y * kSimtMT;
   const int mt = (int)(a.m - m0 < kSimtMT ? a.m - m0 : kSimtMT);
   const int nchunk = a.kw >> 2;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int grp = lane >> 3, l8 = lane & 7;
+  // The first PF chunks of this lane's first weight row are loaded before the activations are
+  // staged, so the weight stream is in flight while the block copies and synchronises.
+  constexpr int PF = 8;
+  uint4 wpf[PF];
+  {
+    const int n = blockIdx.x * 32 + warp * 4 + grp;
+    const uint4* wrow = reinterpret_cast<const uint4*>(s.codes + (int64_t)(n < s.n ? n : 0) * a.kw);
+#pragma unroll
+    for (int p = 0; p < PF; ++p) {
+      const int c = l8 + 8 * p;
+      wpf[p] = (n < s.n && c < nchunk) ? __ldg(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+    }
+  }
   // stage activations
   for (int idx = threadIdx.x; idx < mt * nchunk * 4; idx += blockDim.x) {
     const int j = idx / (nchunk * 4);
@@ -473,9 +488,8 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const GemmArgs a) {
         *reinterpret_cast<const uint4*>(s.q + (m0 + j) * a.ldq + c * 64 + p * 16);
   }
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int grp = lane >> 3, l8 = lane & 7;
   const float sw = s.sw[0];
+  bool first = true;
   for (int base = blockIdx.x * 32 + warp * 4; base < s.n; base += gridDim.x * 32) {
     const int n = base + grp;
     const bool valid = n < s.n;
@@ -483,9 +497,7 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const GemmArgs a) {
 #pragma unroll
     for (int j = 0; j < kSimtMT; ++j) acc[j] = 0;
     const uint4* wrow = reinterpret_cast<const uint4*>(s.codes + (int64_t)(valid ? n : 0) * a.kw);
-    for (int c = l8; c < nchunk; c += 8) {
-      uint4 wv = make_uint4(0u, 0u, 0u, 0u);
-      if (valid) wv = __ldg(wrow + c);
+    auto consume = [&](const uint4& wv, int c) {
       uint32_t e[16];
       expand_word(wv.x, e + 0);
       expand_word(wv.y, e + 4);
@@ -505,6 +517,18 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const GemmArgs a) {
           }
         }
       }
+    };
+    int c0 = l8;
+    if (first) {
+#pragma unroll
+      for (int p = 0; p < PF; ++p)
+        if (l8 + 8 * p < nchunk) consume(wpf[p], l8 + 8 * p);
+      c0 = l8 + 8 * PF;
+      first = false;
+    }
+    for (int c = c0; c < nchunk; c += 8) {
+      const uint4 wv = valid ? __ldg(wrow + c) : make_uint4(0u, 0u, 0u, 0u);
+      consume(wv, c);
     }
 #pragma unroll
     for (int j = 0; j < kSimtMT; ++j) {

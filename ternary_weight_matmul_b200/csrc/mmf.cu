@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <utility>
 #include <cstdarg>
 #include <atomic>
 #include <cstdio>
@@ -13,6 +14,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "decode.cuh"
 #include "gemm_tc.cuh"
 #include "kernels.cuh"
 
@@ -108,6 +110,8 @@ mmf_status device_info(DevInfo** out) {
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
       MMF_CUDA(cudaFuncSetAttribute(simt_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     200 * 1024));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
       MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowPlain>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
       MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowGlu>,
@@ -154,6 +158,18 @@ mmf_status encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(MMF_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
   return MMF_OK;
+}
+
+// Launches a kernel (cudaLaunchKernelEx; errors surface through check_launch).
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 mmf_status check_launch(const char* what) {
@@ -219,7 +235,7 @@ template <mmf_dtype XT, int MODE, int NG>
 void nq_vec_launch(const NormQuantArgs& a, int w, int nch, cudaStream_t st) {
   const unsigned rows_per_cta = 8u / (unsigned)w;
   const dim3 grid((unsigned)((a.m + rows_per_cta - 1) / rows_per_cta));
-#define MMF_NQ(W_, C_) norm_quant_vec_kernel<XT, MODE, W_, C_, NG><<<grid, kNqThreads, 0, st>>>(a)
+#define MMF_NQ(W_, C_) launch_k(norm_quant_vec_kernel<XT, MODE, W_, C_, NG>, grid, dim3(kNqThreads), 0, st, a)
 #define MMF_NQ_W(W_) \
   do { if (nch <= 2) MMF_NQ(W_, 2); else if (nch <= 4) MMF_NQ(W_, 4); else if (nch <= 6) MMF_NQ(W_, 6); else MMF_NQ(W_, 8); } while (0)
   if (w == 1) MMF_NQ_W(1);
@@ -269,9 +285,9 @@ mmf_status launch_norm_quant(const NormQuantArgs& a, int mode, cudaStream_t st) 
   const size_t smem = (size_t)a.k * sizeof(float);
   const int threads = a.k >= 2048 ? 256 : 128;
   dim3 grid((unsigned)a.m);
-  if (mode == kRowPlain) norm_quant_kernel<kRowPlain><<<grid, threads, smem, st>>>(a);
-  else if (mode == kRowGlu) norm_quant_kernel<kRowGlu><<<grid, threads, smem, st>>>(a);
-  else norm_quant_kernel<kRowGnorm><<<grid, threads, smem, st>>>(a);
+  if (mode == kRowPlain) launch_k(norm_quant_kernel<kRowPlain>, grid, dim3(threads), smem, st, a);
+  else if (mode == kRowGlu) launch_k(norm_quant_kernel<kRowGlu>, grid, dim3(threads), smem, st, a);
+  else launch_k(norm_quant_kernel<kRowGnorm>, grid, dim3(threads), smem, st, a);
   return check_launch("norm_quant_kernel");
 }
 
@@ -304,7 +320,7 @@ mmf_status launch_gemm(const GemmArgs& g, const DevInfo& di, cudaStream_t st) {
       bytes += (double)g.seg[s].n * g.kw * 4.0 + (double)g.m * g.ldq + (double)g.m * g.seg[s].n * yes *
                (g.seg[s].res ? 2.0 : 1.0);
     LaunchScope ls(MMF_KERNEL_GEMM_SIMT, bytes, st);
-    simt_gemm_kernel<<<grid, 256, smem, st>>>(g);
+    launch_k(simt_gemm_kernel, grid, dim3(256), smem, st, g);
     return check_launch("simt_gemm_kernel");
   }
   tc::Params P;
@@ -333,9 +349,9 @@ mmf_status launch_gemm(const GemmArgs& g, const DevInfo& di, cudaStream_t st) {
   for (int s = 0; s < g.nseg; ++s) ops += 2.0 * (double)g.m * g.seg[s].n * g.k;
   LaunchScope ls(MMF_KERNEL_GEMM_TC, ops, st);
   if (g.ydt == MMF_F32)
-    tc::ternary_gemm_tc_kernel<MMF_F32><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(P);
+    launch_k(tc::ternary_gemm_tc_kernel<MMF_F32>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, st, P);
   else
-    tc::ternary_gemm_tc_kernel<MMF_BF16><<<grid, tc::NUM_THREADS, tc::SMEM_BYTES, st>>>(P);
+    launch_k(tc::ternary_gemm_tc_kernel<MMF_BF16>, dim3(grid), dim3(tc::NUM_THREADS), tc::SMEM_BYTES, st, P);
   return check_launch("ternary_gemm_tc_kernel");
 }
 
@@ -357,12 +373,12 @@ template <mmf_dtype ZT, mmf_dtype HT, int VEC, bool GATED>
 void scan_launch_gated(const ScanArgs& a, cudaStream_t st) {
   const unsigned gx = (unsigned)((a.d / VEC + kScanThreads - 1) / kScanThreads);
   if (a.nchunk == 1) {
-    scan_apply_kernel<ZT, HT, VEC, true, GATED><<<dim3(gx, 1, a.b), kScanThreads, 0, st>>>(a);
+    launch_k(scan_apply_kernel<ZT, HT, VEC, true, GATED>, dim3(gx, 1, a.b), dim3(kScanThreads), 0, st, a);
     return;
   }
-  scan_aggregate_kernel<ZT, VEC, GATED><<<dim3(gx, a.nchunk, a.b), kScanThreads, 0, st>>>(a);
-  scan_carry_kernel<<<dim3((unsigned)((a.d + kScanThreads - 1) / kScanThreads), a.b), kScanThreads, 0, st>>>(a);
-  scan_apply_kernel<ZT, HT, VEC, false, GATED><<<dim3(gx, a.nchunk, a.b), kScanThreads, 0, st>>>(a);
+  launch_k(scan_aggregate_kernel<ZT, VEC, GATED>, dim3(gx, a.nchunk, a.b), dim3(kScanThreads), 0, st, a);
+  launch_k(scan_carry_kernel, dim3((unsigned)((a.d + kScanThreads - 1) / kScanThreads), a.b), dim3(kScanThreads), 0, st, a);
+  launch_k(scan_apply_kernel<ZT, HT, VEC, false, GATED>, dim3(gx, a.nchunk, a.b), dim3(kScanThreads), 0, st, a);
 }
 
 template <mmf_dtype ZT, mmf_dtype HT, int VEC>
@@ -377,12 +393,12 @@ void scan_tiled_gated(const ScanArgs& a, cudaStream_t st) {
   constexpr int smem = scan_tile_bytes<ZT>();
   const unsigned gx = (unsigned)((a.d + kScanTileCh - 1) / kScanTileCh);
   if (a.nchunk == 1) {
-    scan_tile_kernel<ZT, HT, GATED, 2><<<dim3(gx, 1, a.b), kScanThreads, smem, st>>>(a);
+    launch_k(scan_tile_kernel<ZT, HT, GATED, 2>, dim3(gx, 1, a.b), dim3(kScanThreads), smem, st, a);
     return;
   }
-  scan_tile_kernel<ZT, HT, GATED, 0><<<dim3(gx, a.nchunk, a.b), kScanThreads, smem, st>>>(a);
-  scan_carry_kernel<<<dim3((unsigned)((a.d + kScanThreads - 1) / kScanThreads), a.b), kScanThreads, 0, st>>>(a);
-  scan_tile_kernel<ZT, HT, GATED, 1><<<dim3(gx, a.nchunk, a.b), kScanThreads, smem, st>>>(a);
+  launch_k(scan_tile_kernel<ZT, HT, GATED, 0>, dim3(gx, a.nchunk, a.b), dim3(kScanThreads), smem, st, a);
+  launch_k(scan_carry_kernel, dim3((unsigned)((a.d + kScanThreads - 1) / kScanThreads), a.b), dim3(kScanThreads), 0, st, a);
+  launch_k(scan_tile_kernel<ZT, HT, GATED, 1>, dim3(gx, a.nchunk, a.b), dim3(kScanThreads), smem, st, a);
 }
 template <mmf_dtype ZT, mmf_dtype HT>
 void scan_tiled_typed(const ScanArgs& a, cudaStream_t st) {
@@ -844,6 +860,81 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
   return MMF_OK;
 }
 
+// ---------------------------------------------------------------------------------------------
+// fused decode (up to 8 token rows on the CUDA-core engine): four launches per block
+// ---------------------------------------------------------------------------------------------
+// (One or two rows: with more, the per-CTA quantisation of every input row costs more than the
+// separate norm-quant launches it replaces.)
+bool decode_fused(int32_t b, int32_t d, int32_t inner) {
+  if (b < 1 || b > 2 || use_tensor_path(b)) return false;
+  if (d % 8 || inner % 8) return false;
+  return true;
+}
+
+// Channels per CTA: about one CTA per SM, fewer channels when the weight slice would not fit.
+int dec_chan_per_cta(int mode, int nout, int nmat, int kw, int k, int ngain, int b, int sms) {
+  int cpc = std::max(1, (nout + sms - 1) / sms);
+  while (cpc > 1 && dec::smem_layout(mode, nmat, cpc, kw, k, ngain, b).total > (size_t)dec::kMaxSmem) cpc = (cpc + 1) / 2;
+  return cpc;
+}
+
+mmf_status launch_dec(dec::Args& a, const DevInfo& di, cudaStream_t st) {
+  a.chan_per_cta = dec_chan_per_cta(a.mode, a.nout, a.nmat, a.kw, a.k, a.ngain, a.b, di.sms);
+  const dec::Smem L = dec::smem_layout(a.mode, a.nmat, a.chan_per_cta, a.kw, a.k, a.ngain, a.b);
+  if (L.total > (size_t)dec::kMaxSmem) return fail(MMF_ERR_UNSUPPORTED, "decode: K=%d too large for one CTA", a.k);
+  a.wait_limit_us = g_wait_limit.load();
+  const dim3 grid((unsigned)((a.nout + a.chan_per_cta - 1) / a.chan_per_cta));
+  double bytes = 0;
+  for (int j = 0; j < a.nmat; ++j) bytes += (double)a.nout * a.kw * 4.0;
+  LaunchScope ls(MMF_KERNEL_GEMM_SIMT, bytes, st);
+  if (a.xdt == MMF_F32) launch_k(dec::dec_proj_kernel<MMF_F32>, grid, dim3(dec::kThreads), L.total, st, a);
+  else launch_k(dec::dec_proj_kernel<MMF_BF16>, grid, dim3(dec::kThreads), L.total, st, a);
+  return check_launch("dec_proj_kernel");
+}
+
+// One block, one token per row: x [b][d] -> y [b][d], state [b][d] updated in place. Scratch:
+// h and g (float32, [b][d]), x1 [b][d] and v [b][inner] (dtype).
+mmf_status run_block_decode(const mmf_block_weights* w, const void* x, mmf_dtype dt, int32_t b, float* state,
+                            void* y, uint8_t* scratch, const DevInfo& di, cudaStream_t st) {
+  const int32_t d = w->d, inner = w->inner;
+  float* h32 = reinterpret_cast<float*>(scratch);
+  float* g32 = reinterpret_cast<float*>(scratch + align256((size_t)b * d * 4));
+  void* x1 = scratch + 2 * align256((size_t)b * d * 4);
+  void* v = scratch + 3 * align256((size_t)b * d * 4);
+  dec::Args a;
+  memset(&a, 0, sizeof(a));
+  a.b = b; a.eps = w->eps; a.xdt = dt; a.ydt = dt;
+  // i/f/g + gates + recurrence step
+  a.mode = dec::kIFG; a.k = d; a.kw = row_words(d); a.nout = d; a.nmat = 3; a.ngain = 3;
+  a.w[0] = w->i.codes; a.w[1] = w->f.codes; a.w[2] = w->g.codes;
+  a.sw[0] = w->i.scale; a.sw[1] = w->f.scale; a.sw[2] = w->g.scale;
+  a.gain[0] = w->nw_i; a.gain[1] = w->nw_f; a.gain[2] = w->nw_g;
+  a.x = x; a.y = h32; a.g_out = g32; a.state = state;
+  MMF_TRY(launch_dec(a, di, st));
+  // g_norm + o_proj + residual
+  memset(&a, 0, sizeof(a));
+  a.b = b; a.eps = w->eps; a.xdt = dt; a.ydt = dt;
+  a.mode = dec::kO; a.k = d; a.kw = row_words(d); a.nout = d; a.nmat = 1; a.ngain = 1;
+  a.w[0] = w->o.codes; a.sw[0] = w->o.scale; a.gain[0] = w->nw_o;
+  a.h = h32; a.gin = g32; a.gnorm_w = w->gnorm_w; a.res = x; a.y = x1;
+  MMF_TRY(launch_dec(a, di, st));
+  // gate_proj: v = SiLU(gate) * up
+  memset(&a, 0, sizeof(a));
+  a.b = b; a.eps = w->eps; a.xdt = dt; a.ydt = dt;
+  a.mode = dec::kGate; a.k = d; a.kw = row_words(d); a.nout = inner; a.nmat = 2; a.ngain = 1;
+  a.w[0] = w->gate.codes; a.w[1] = w->gate.codes; a.row_off[1] = inner;
+  a.sw[0] = w->gate.scale; a.sw[1] = w->gate.scale; a.gain[0] = w->nw_gate;
+  a.x = x1; a.y = v;
+  MMF_TRY(launch_dec(a, di, st));
+  // down_proj + residual
+  memset(&a, 0, sizeof(a));
+  a.b = b; a.eps = w->eps; a.xdt = dt; a.ydt = dt;
+  a.mode = dec::kDown; a.k = inner; a.kw = row_words(inner); a.nout = d; a.nmat = 1; a.ngain = 1;
+  a.w[0] = w->down.codes; a.sw[0] = w->down.scale; a.gain[0] = w->nw_down;
+  a.x = v; a.res = x1; a.y = y;
+  return launch_dec(a, di, st);
+}
+
 mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
                            mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
                            size_t ws_bytes, mmf_stream_t stream) {
@@ -867,10 +958,12 @@ mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, co
   uint8_t* pp = reinterpret_cast<uint8_t*>(ws) + W.bytes;
   void* buf[2] = {pp, pp + align256((size_t)b * d * 4)};
   const void* cur = x;
+  const bool fused = decode_fused(b, d, inner);
   for (int l = 0; l < n_layers; ++l) {
     void* out = (l == n_layers - 1) ? y : buf[l & 1];
     float* st_l = state + (int64_t)l * b * d;
-    MMF_TRY(run_block(&layers[l], cur, dtype, b, 1, st_l, out, st_l, W, *di, st));
+    if (fused) MMF_TRY(run_block_decode(&layers[l], cur, dtype, b, st_l, out, reinterpret_cast<uint8_t*>(ws), *di, st));
+    else MMF_TRY(run_block(&layers[l], cur, dtype, b, 1, st_l, out, st_l, W, *di, st));
     cur = out;
   }
   return MMF_OK;
@@ -887,7 +980,7 @@ mmf_status mmf_embed_gather(const int32_t* ids, int64_t m, const void* table, mm
   MMF_TRY(device_info(&di));
   {
     LaunchScope ls(MMF_KERNEL_OTHER, (double)m * d * 2.0 * dsize(dtype) + m * 4.0, reinterpret_cast<cudaStream_t>(stream));
-    embed_gather_kernel<<<(unsigned)m, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ids, m, table, dtype, vocab, d, out);
+    launch_k(embed_gather_kernel, dim3((unsigned)m), dim3(128), 0, reinterpret_cast<cudaStream_t>(stream), ids, m, table, dtype, vocab, d, out);
   }
   return check_launch("embed_gather_kernel");
 }
@@ -917,7 +1010,7 @@ mmf_status mmf_stack_fwd(const mmf_block_weights* layers, int32_t n_layers, cons
   void* buf[2] = {pp, pp + align256((size_t)m * d * 4)};
   {
     LaunchScope ls(MMF_KERNEL_OTHER, (double)m * d * 2.0 * dsize(dtype) + m * 4.0, st);
-    embed_gather_kernel<<<(unsigned)m, 128, 0, st>>>(ids, m, table, dtype, vocab, d, buf[0]);
+    launch_k(embed_gather_kernel, dim3((unsigned)m), dim3(128), 0, st, ids, m, table, dtype, vocab, d, buf[0]);
   }
   MMF_TRY(check_launch("embed_gather_kernel"));
   const void* cur = buf[0];

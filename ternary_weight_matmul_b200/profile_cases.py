@@ -3,6 +3,7 @@
     python -m ternary_weight_matmul_b200.profile_cases gemm --m 16384 --n 5632 --k 1024
     python -m ternary_weight_matmul_b200.profile_cases scan --b 4 --t 8192 --d 2048
     python -m ternary_weight_matmul_b200.profile_cases block --m 16384 --d 1024 --inner 2816
+    python -m ternary_weight_matmul_b200.profile_cases decode --b 1 --d 2560 --inner 7040 --layers 4
 
 Inputs are seeded and synthetic (weights N(0, 0.02), activations N(0, 1)); prints the mean device
 time per iteration measured with CUDA events.
@@ -18,7 +19,8 @@ import ternary_weight_matmul_b200 as mmf
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["gemm", "scan", "block", "norm"])
+    ap.add_argument("case", choices=["gemm", "scan", "block", "norm", "decode"])
+    ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--m", type=int, default=16384)
     ap.add_argument("--n", type=int, default=5632)
     ap.add_argument("--k", type=int, default=1024)
@@ -62,6 +64,23 @@ def main() -> None:
         def run():
             return mmf.bitlinear_fwd(x, None, w, y_dtype=dt)
         work, unit = float(a.m * a.k * (x.element_size() + 1)), "GB/s (norm part only)"
+    elif a.case == "decode":
+        d, inner = a.d, a.inner
+        shapes = {"i": (d, d), "f": (d, d), "g": (d, d), "o": (d, d), "gate": (2 * inner, d), "down": (d, inner)}
+        blocks = []
+        for _ in range(a.layers):
+            packed = {p: mmf.pack_ternary(torch.randn(n, k, generator=g, device=dev) * 0.02) for p, (n, k) in shapes.items()}
+            norms = {f"nw_{p}": torch.ones(k, device=dev) for p, (n, k) in shapes.items()}
+            norms["gnorm_w"] = torch.ones(d, device=dev)
+            blocks.append(mmf.Block(d, inner, packed, norms))
+        x = torch.randn(a.b, d, generator=g, device=dev).to(dt)
+        state = torch.zeros(a.layers, a.b, d, device=dev)
+        y = torch.empty_like(x)
+
+        def run():
+            return mmf.decode_step(blocks, x, state, out=y)
+        wbytes = sum(p.codes.numel() * 4 for blk in blocks for p in blk.packed.values())
+        work, unit = float(wbytes), "GB/s (packed weights)"
     else:
         d, inner = a.d, a.inner
         shapes = {"i": (d, d), "f": (d, d), "g": (d, d), "o": (d, d), "gate": (2 * inner, d), "down": (d, inner)}

@@ -408,7 +408,7 @@ def test_block_prefill_equals_stepwise_decode_on_gpu(mmf):
     np.testing.assert_allclose(state[1].cpu().numpy(), h2.cpu().numpy(), rtol=1e-4, atol=1e-4)
 
 
-@pytest.mark.parametrize("b", [1, 3, 8, 64])
+@pytest.mark.parametrize("b", [1, 2, 3, 8, 64])
 def test_decode_step_parity(mmf, b):
     layers = [_block_case(mmf, 20 + l, 256, 704) for l in range(2)]
     x = synth.activations(30 + b, (b, 256))
@@ -422,6 +422,27 @@ def test_decode_step_parity(mmf, b):
     # the first layer's state depends only on exactly quantised inputs: elementwise
     np.testing.assert_allclose(st.cpu().numpy()[0], st_ref[0], rtol=RTOL32, atol=ATOL32)
     np.testing.assert_allclose(st.cpu().numpy(), st_ref, rtol=1e-2, atol=1e-3)
+
+
+@pytest.mark.parametrize("b", [1, 2])
+def test_decode_fused_matches_unfused(mmf, b):
+    # one or two rows take the fused four-launch decode; forcing the tensor-core engine takes the
+    # nine-launch block path instead. Same quantisation arithmetic: states agree closely and the
+    # outputs within the chained-quantisation tolerance.
+    layers = [_block_case(mmf, 40 + l, 256, 704) for l in range(2)]
+    x = _to(synth.activations(41 + b, (b, 256)))
+    state0 = _to(synth.activations(42 + b, (2, b, 256)) * 0.5)
+    st_f, st_u = state0.clone(), state0.clone()
+    y_f = mmf.decode_step([c[2] for c in layers], x, st_f)
+    mmf.set_gemm_path(mmf.MMF_GEMM_TENSOR)
+    try:
+        y_u = mmf.decode_step([c[2] for c in layers], x, st_u)
+        _ok(mmf)
+    finally:
+        mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
+    np.testing.assert_allclose(st_f[0].cpu().numpy(), st_u[0].cpu().numpy(), rtol=RTOL32, atol=ATOL32)
+    rel = float(torch.linalg.norm(y_f - y_u) / torch.linalg.norm(y_u))
+    assert rel < 1e-3, rel
 
 
 def test_embed_gather(mmf):
