@@ -49,6 +49,22 @@ def parse():
     return ap.parse_args()
 
 
+def max_over_ranks(ms: float, device, world: int) -> float:
+    """The slowest rank's time: replicas finish a step when the last one does."""
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replicas_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
+    """Whole-job tokens/s of `world` independent replicas, each processing its own batch."""
+    return tokens_per_rank * world / (ms_max / 1e3)
+
+
 def dist_env():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -337,12 +353,9 @@ def run_gpu(args, wl):
         raise RuntimeError(f"device status {st} in the timed region")
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
-    ms_t = torch.tensor([ms], device=device)
-    if world > 1:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
+    ms_max = max_over_ranks(ms, device, world)
     tokens = B * T * world
-    value = tokens / (ms_max / 1e3)
+    value = replicas_throughput(B * T, world, ms_max)
 
     kern = {}
     for cls in ("gemm_tc", "gemm_simt", "norm_quant", "scan", "other"):
@@ -369,10 +382,7 @@ def run_gpu(args, wl):
             e_e[i].record(stream)
         torch.cuda.synchronize(device)
         e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / args.steps
-        e_t = torch.tensor([e_ms], device=device)
-        if world > 1:
-            dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
-        e2e = {"value": tokens / (float(e_t.item()) / 1e3), "unit": "tokens/s",
+        e2e = {"value": replicas_throughput(B * T, world, max_over_ranks(e_ms, device, world)), "unit": "tokens/s",
                "h2d_bytes_per_step": ids_host.numel() * 4, "d2h_bytes_per_step": y_host.numel() * 2}
 
     decode = None

@@ -1,0 +1,58 @@
+"""Replica timing across ranks (bench.py, `--gpus N`): two gloo ranks on the CPU.
+
+The block stack shards by independent sequences, so N GPUs run N replicas with no collective on
+the data path; the only cross-rank steps are the barrier and the maximum of the step time. These
+tests run that host logic with world_size 2 over gloo (127.0.0.1)."""
+import os
+import socket
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out) -> None:
+    sys.path.insert(0, ROOT)
+    import bench
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        dist.barrier()
+        local_ms = 10.0 + 2.0 * rank            # rank 1 is the slow one
+        ms_max = bench.max_over_ranks(local_ms, torch.device("cpu"), world)
+        value = bench.replicas_throughput(16384, world, ms_max)
+        out[rank] = (ms_max, value)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_replicas_time_is_the_slowest_rank_and_throughput_sums_batches():
+    port = _free_port()
+    mgr = mp.get_context("spawn").Manager()
+    out = mgr.dict()
+    mp.start_processes(_rank_main, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+    assert set(out.keys()) == {0, 1}
+    for r in (0, 1):
+        ms_max, value = out[r]
+        assert ms_max == pytest.approx(12.0)
+        assert value == pytest.approx(2 * 16384 / 0.012)
+
+
+def test_single_rank_needs_no_process_group():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.max_over_ranks(7.5, torch.device("cpu"), 1) == 7.5
+    assert bench.replicas_throughput(1000, 1, 2.0) == pytest.approx(500000.0)
