@@ -32,6 +32,11 @@ WORKLOADS = {
 }
 # Autoregressive decode of the 2.7B-shape stack: a 512-token prompt (prefill, untimed) then
 # decode steps with the recurrent state carried per layer, at three batch sizes.
+# DRAM traffic of one ternary_gemm_tc_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum,
+# averaged over the 96 GEMM launches of one step) from an ncu capture of this bench's own workload;
+# valid only while the kernel source is the one captured (SHA-256 prefix), else reported as null.
+GEMM_TRAFFIC = {"prefill-370M": dict(bytes=78.6e6, algorithmic=115.2e6, sha256="555ae3df1a5fa605",
+                                     profile="profiles/ternary_gemm_tc_kernel_prefill-370M_traffic.md")}
 DECODE = dict(name="decode-2.7B", d=2560, inner=7040, layers=32, vocab=32000, prompt=512, batches=(1, 8, 64))
 
 
@@ -47,6 +52,21 @@ def parse():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-steps", type=int, default=64)
     return ap.parse_args()
+
+
+def gemm_traffic(workload: str):
+    """Measured DRAM bytes per GEMM launch for this workload, or None when no capture matches the
+    current kernel source."""
+    import hashlib
+
+    t = GEMM_TRAFFIC.get(workload)
+    if t is None:
+        return None
+    src = os.path.join(ROOT, "ternary_weight_matmul_b200", "csrc", "gemm_tc.cuh")
+    with open(src, "rb") as fh:
+        if hashlib.sha256(fh.read()).hexdigest()[:16] != t["sha256"]:
+            return None
+    return t["bytes"]
 
 
 def max_over_ranks(ms: float, device, world: int) -> float:
@@ -409,7 +429,9 @@ def run_gpu(args, wl):
         achieved = (tc["work"] / (tc["ms"] / 1e3) / 1e12) if tc["ms"] > 0 else 0.0
         roofline = {"bound": "tensor", "kernel": "ternary_gemm_tc_kernel", "achieved": achieved,
                     "peak": int8_peak, "unit": "TOPS (int8)", "frac": achieved / int8_peak,
-                    "peak_source": peak_src, "traffic": None,
+                    "peak_source": peak_src, "traffic": gemm_traffic(args.workload),
+                    "traffic_source": GEMM_TRAFFIC.get(args.workload, {}).get("profile"),
+                    "algorithmic_bytes_per_launch": GEMM_TRAFFIC.get(args.workload, {}).get("algorithmic"),
                     "launches": tc["launches"], "avg_launch_us": tc["ms"] / max(tc["launches"], 1) * 1e3,
                     "share_of_step": tc["ms"] / (ms * args.steps)}
         hbm_kernels = {}

@@ -56,3 +56,14 @@ def test_single_rank_needs_no_process_group():
 
     assert bench.max_over_ranks(7.5, torch.device("cpu"), 1) == 7.5
     assert bench.replicas_throughput(1000, 1, 2.0) == pytest.approx(500000.0)
+
+
+def test_gemm_traffic_tracks_kernel_source():
+    """The traffic figure is reported only for the captured workload and kernel source, and the
+    profile it cites is committed."""
+    import bench
+
+    t = bench.gemm_traffic("prefill-370M")
+    assert t is not None and 0 < t < bench.GEMM_TRAFFIC["prefill-370M"]["algorithmic"]
+    assert bench.gemm_traffic("prefill-1.3B") is None
+    assert os.path.exists(os.path.join(bench.ROOT, bench.GEMM_TRAFFIC["prefill-370M"]["profile"]))
