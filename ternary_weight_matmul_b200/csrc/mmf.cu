@@ -362,9 +362,17 @@ inline int32_t scan_chunk(int64_t t) {
   const int64_t c = (t + 127) / 128;
   return (int32_t)((c + 15) / 16 * 16);
 }
+// Steps per chunk of the shared-memory staged scan: 64 (four double-buffered tiles) up to 8192
+// steps, then a multiple of 16 giving at most 128 chunks.
+inline int32_t scan_tile_chunk(int64_t t) {
+  if (t <= 8192) return 64;
+  const int64_t c = (t + 127) / 128;
+  return (int32_t)((c + 15) / 16 * 16);
+}
 // Scratch of the chunked scan for m = b*t tokens of d channels: three [b][nchunk][d] float
 // arrays. b * nchunk <= ceil(m / 8) whenever t > 16 (shorter sequences need no scratch):
-// t <= 2048 gives nchunk = ceil(t/16) < t/8, longer ones nchunk <= 128 < t/16.
+// chunks are at least 16 steps, so nchunk = ceil(t/16) <= t/8, and past 2048 (register path) or
+// 8192 (staged path) steps nchunk <= 128 < t/16.
 inline size_t scan_ws_bytes(int64_t m, int32_t d) {
   return 3 * align256((size_t)d * 4 * (size_t)((m + 7) / 8));
 }
@@ -414,7 +422,7 @@ void scan_launch_vec(const ScanArgs& a, cudaStream_t st) {
   else scan_launch_typed<MMF_BF16, MMF_BF16, VEC>(a, st);
 }
 
-// ws: scan_ws_bytes(b*t, d) bytes (unused when t <= 16).
+// ws: scan_ws_bytes(b*t, d) bytes (unused when t <= 16, or while the sequence is one chunk).
 mmf_status launch_scan(ScanArgs a, void* ws, cudaStream_t st) {
   if ((int64_t)a.b * a.d == 0) return MMF_OK;
   const int64_t chans = (int64_t)a.b * a.d;
@@ -431,11 +439,18 @@ mmf_status launch_scan(ScanArgs a, void* ws, cudaStream_t st) {
     }
     return MMF_OK;
   }
-  if (a.t <= 16) {
+  const size_t zes = dsize(a.zdt), hes = dsize(a.hdt);
+  const auto aligned = [](const void* q, size_t n) { return (reinterpret_cast<uintptr_t>(q) % n) == 0; };
+  const bool pair = (a.d % 2 == 0) && (a.zstride % 2 == 0) && aligned(a.zf, 2 * zes) && aligned(a.zi, 2 * zes) &&
+                    aligned(a.h, 2 * hes);
+  const bool tiled = pair && (a.zstride * zes) % 16 == 0 && (a.d * zes) % 16 == 0 && aligned(a.zf, 16) &&
+                     aligned(a.zi, 16) && aligned(a.h0, 8) && aligned(a.h_last, 8);
+  const int32_t chunk = tiled ? scan_tile_chunk(a.t) : (a.t <= 16 ? (int32_t)a.t : scan_chunk(a.t));
+  if (a.t <= chunk) {
     a.chunk = (int32_t)a.t;
     a.nchunk = 1;
   } else {
-    a.chunk = scan_chunk(a.t);
+    a.chunk = chunk;
     a.nchunk = (int32_t)((a.t + a.chunk - 1) / a.chunk);
     const size_t arr = align256((size_t)a.d * 4 * (size_t)(((int64_t)a.b * a.t + 7) / 8));
     uint8_t* p = reinterpret_cast<uint8_t*>(ws);
@@ -443,17 +458,10 @@ mmf_status launch_scan(ScanArgs a, void* ws, cudaStream_t st) {
     a.agg_b = reinterpret_cast<float*>(p + arr);
     a.cin = reinterpret_cast<float*>(p + 2 * arr);
   }
-  const size_t zes = dsize(a.zdt), hes = dsize(a.hdt);
-  const bool pair = (a.d % 2 == 0) && (a.zstride % 2 == 0) &&
-                    (reinterpret_cast<uintptr_t>(a.zf) % (2 * zes) == 0) &&
-                    (reinterpret_cast<uintptr_t>(a.zi) % (2 * zes) == 0) &&
-                    (reinterpret_cast<uintptr_t>(a.h) % (2 * hes) == 0);
   const double zb = (double)zes, hb = (double)hes;
   LaunchScope ls(MMF_KERNEL_SCAN, (double)chans * a.t * (2.0 * zb + hb) + (double)chans * 4.0 *
                  ((a.h0 ? 1.0 : 0.0) + (a.h_last ? 1.0 : 0.0)), st);
   if (a.nchunk > 1) g_launches.fetch_add(2);  // three kernels under one timing scope
-  const bool tiled = pair && (a.zstride * zes) % 16 == 0 && (a.d * zes) % 16 == 0 &&
-                     (reinterpret_cast<uintptr_t>(a.zf) & 15u) == 0 && (reinterpret_cast<uintptr_t>(a.zi) & 15u) == 0;
   if (tiled) {
     if (a.zdt == MMF_F32 && a.hdt == MMF_F32) scan_tiled_typed<MMF_F32, MMF_F32>(a, st);
     else if (a.zdt == MMF_F32) scan_tiled_typed<MMF_F32, MMF_BF16>(a, st);

@@ -206,6 +206,34 @@ def test_scan_parity_bf16_strided(mmf):
     np.testing.assert_allclose(h.float().cpu().numpy(), h_ref, rtol=RTOL16, atol=RTOL16 * 0.1)
 
 
+@pytest.mark.parametrize("b,t,d", [(2, 50, 33), (1, 300, 31), (2, 70, 34), (3, 129, 6)])
+def test_scan_parity_unaligned_channels(mmf, b, t, d):
+    # rows that are not 16-byte multiples take the three-pass kernels (paired for even d)
+    zf, zi = synth.scan_inputs(b * t + d, b, t, d, False)
+    h0 = synth.activations(5, (b, d))
+    h, hl = mmf.hgrn_scan(_to(zf), _to(zi), _to(h0))
+    _ok(mmf)
+    h_ref = O.hgrn_scan(*O.hgrn_gates(zf, zi), h0)
+    np.testing.assert_allclose(h.cpu().numpy(), h_ref, rtol=RTOL32, atol=ATOL32)
+    np.testing.assert_allclose(hl.cpu().numpy(), h_ref[:, -1], rtol=RTOL32, atol=ATOL32)
+
+
+def test_scan_parity_bf16_full_size(mmf):
+    # the prefill step's scan: 8 sequences of 2048 steps, 1024 channels, gates read in place from
+    # the [i | f | g] projection output (row stride 3d), float32 states; every element checked
+    b, t, d = 8, 2048, 1024
+    z = _bf16_round(synth.activations(17, (b, t, 3 * d)))
+    z[:, :, d:2 * d] += 3.0  # forget gates near 0.95: long memory across chunks
+    z = _bf16_round(z)
+    zt = _to(z, torch.bfloat16)
+    h0 = synth.activations(19, (b, d))
+    h, hl = mmf.hgrn_scan(zt[:, :, d:2 * d], zt[:, :, :d], _to(h0), h_dtype=torch.float32)
+    _ok(mmf)
+    h_ref = O.hgrn_scan(*O.hgrn_gates(z[:, :, d:2 * d], z[:, :, :d]), h0)
+    np.testing.assert_allclose(h.cpu().numpy(), h_ref, rtol=RTOL32, atol=ATOL32)
+    np.testing.assert_allclose(hl.cpu().numpy(), h_ref[:, -1], rtol=RTOL32, atol=ATOL32)
+
+
 def test_scan_long_sequence_closed_form(mmf):
     # constant gates: h_t = SiLU(zi) (1 - f^t); T = 65536 with f = sigmoid(4) checks carry drift
     b, t, d = 1, 65536, 64
