@@ -187,7 +187,7 @@ __global__ void __launch_bounds__(256) norm_quant_kernel(const NormQuantArgs a) 
 // float32 rounding of r (a relative perturbation of the mean square moves r * 127/a by a few
 // ulp at most); the sum of squares and 1/sqrt therefore run in float32 (each step IEEE-rounded).
 // The dequantisation factor a/127 carries the mean square's own rounding (~1e-7 relative).
-constexpr int kNqThreads = 256;
+constexpr int kNqThreads = 128;
 
 template <int W>
 __device__ __forceinline__ float nq_group_sum(float v, float (*red)[8], int& ph) {
@@ -259,137 +259,218 @@ __device__ __forceinline__ void load8_gain(const float* g, int64_t idx, float (&
 __device__ __forceinline__ float nq_rinv(float ss, int k, float eps) {
   return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)k), eps)));
 }
-// Bits of clamp(x, -127, 127) + 1.5 * 2^23: the addition (where the float32 spacing is exactly
-// 1) rounds half to even, and the low byte of the result is the int8 code rint(x) itself
-// (0x4B400000 has a zero low byte, and the code lies in [-127, 127]).
-__device__ __forceinline__ uint32_t q8_bits(float x) {
-  return __float_as_uint(__fadd_rn(fminf(fmaxf(x, -127.0f), 127.0f), 12582912.0f));
+// Bits of x + 1.5 * 2^23 for |x| <= 127.5: the addition (where the float32 spacing is exactly 1)
+// rounds half to even, and the low byte of the result is the int8 code rint(x) itself
+// (0x4B400000 has a zero low byte). No clamp is needed: x = r * fl(127 / a) with a the maximum of
+// the very |r| values, so |x| <= 127 (1 + 2^-24)^2 < 127.5 and the code lies in [-127, 127].
+__device__ __forceinline__ uint32_t q8_bits(float x) { return __float_as_uint(__fadd_rn(x, 12582912.0f)); }
+__device__ __forceinline__ float2 q8_add2(float2 x) {
+  return __fadd2_rn(x, make_float2(12582912.0f, 12582912.0f));
 }
 // Low bytes of four words packed into one word, a in byte 0.
 __device__ __forceinline__ uint32_t pack4_lo_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   return __byte_perm(__byte_perm(a, b, 0x0040u), __byte_perm(c, d, 0x0040u), 0x5410u);
 }
+// Eight codes (four float2 of x + 1.5 * 2^23) as two words.
+__device__ __forceinline__ uint2 pack8_codes(const float2 (&b)[4]) {
+  return make_uint2(pack4_lo_bytes(__float_as_uint(b[0].x), __float_as_uint(b[0].y), __float_as_uint(b[1].x),
+                                   __float_as_uint(b[1].y)),
+                    pack4_lo_bytes(__float_as_uint(b[2].x), __float_as_uint(b[2].y), __float_as_uint(b[3].x),
+                                   __float_as_uint(b[3].y)));
+}
 
-// Row group of W warps per row, NCH chunks of 8 values per thread (K <= 256 * W * NCH).
+// Raw 8-value chunks (one 16-byte word for bf16, two for float32), loaded a row ahead of use.
+template <mmf_dtype XT> struct Raw8 { uint4 w[XT == MMF_F32 ? 2 : 1]; };
+template <mmf_dtype XT>
+__device__ __forceinline__ void raw8_load(const void* base, int64_t idx, Raw8<XT>& r) {
+  const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const uint8_t*>(base) + idx * (XT == MMF_F32 ? 4 : 2));
+  r.w[0] = __ldcs(p);
+  if (XT == MMF_F32) r.w[XT == MMF_F32 ? 1 : 0] = __ldcs(p + 1);
+}
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t w) {
+  return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+template <mmf_dtype XT>
+__device__ __forceinline__ void raw8_unpack(const Raw8<XT>& r, float2 (&o)[4]) {
+  if (XT == MMF_F32) {
+    o[0] = make_float2(__uint_as_float(r.w[0].x), __uint_as_float(r.w[0].y));
+    o[1] = make_float2(__uint_as_float(r.w[0].z), __uint_as_float(r.w[0].w));
+    o[2] = make_float2(__uint_as_float(r.w[XT == MMF_F32 ? 1 : 0].x), __uint_as_float(r.w[XT == MMF_F32 ? 1 : 0].y));
+    o[3] = make_float2(__uint_as_float(r.w[XT == MMF_F32 ? 1 : 0].z), __uint_as_float(r.w[XT == MMF_F32 ? 1 : 0].w));
+  } else {
+    o[0] = bf2_to_f2(r.w[0].x);
+    o[1] = bf2_to_f2(r.w[0].y);
+    o[2] = bf2_to_f2(r.w[0].z);
+    o[3] = bf2_to_f2(r.w[0].w);
+  }
+}
+__device__ __forceinline__ void gain8(const float* g, int64_t idx, float2 (&o)[4]) {
+  if (!g) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] = make_float2(1.0f, 1.0f);
+    return;
+  }
+  const float4 a = __ldg(reinterpret_cast<const float4*>(g + idx));
+  const float4 b = __ldg(reinterpret_cast<const float4*>(g + idx + 4));
+  o[0] = make_float2(a.x, a.y); o[1] = make_float2(a.z, a.w);
+  o[2] = make_float2(b.x, b.y); o[3] = make_float2(b.z, b.w);
+}
+__device__ __forceinline__ float2 silu2(float2 z) { return make_float2(siluf_(z.x), siluf_(z.y)); }
+__device__ __forceinline__ float amax2(float m, float2 r) { return fmaxf(m, fmaxf(fabsf(r.x), fabsf(r.y))); }
+
+// Row group of W warps per row, NCH chunks of 8 values per thread (K <= 256 * W * NCH). The CTAs
+// are persistent: each row group walks rows gridDim.x * (4 / W) apart. A thread sees the same
+// columns in every row, so it holds their norm gains in registers for the whole launch, and it
+// loads the next row's inputs into registers before it works on the current one, so a row's HBM
+// latency overlaps the previous row's reductions and arithmetic. Element-wise products use packed
+// f32x2 arithmetic (each lane rounds exactly as the scalar operation would).
 template <mmf_dtype XT, int MODE, int W, int NCH, int NG>
 __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQuantArgs a) {
   constexpr int GT = 32 * W;
+  constexpr int RPC = (kNqThreads / 32) / W;  // rows per CTA step
+  constexpr bool TWO = MODE != kRowPlain;      // a second input: the up half (GLU) or g (g_norm)
+  constexpr bool GN = MODE == kRowGnorm;
   __shared__ float reds[2][8];
   __shared__ float redm[2][8][3];
   int phs = 0, phm = 0;
   const int grp = (threadIdx.x >> 5) / W;
   const int gl = threadIdx.x - grp * GT;
-  const int64_t row = (int64_t)blockIdx.x * (8 / W) + grp;
-  const bool active = row < a.m;
   const int k = a.k, nck = k >> 3;
-  float v[NCH][8];
-  float ss = 0.0f;
-  if (MODE == kRowGnorm) {
-    float g[NCH][8];
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int c = gl + i * GT;
-      if (active && c < nck) {
-        load8<XT>(a.x, row * a.ldx + 8 * c, v[i]);
-        load8<XT>(a.g, row * a.ldg + 8 * c, g[i]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
-      }
-    }
-    const float rfh = nq_rinv(nq_group_sum<W>(ss, reds, phs), k, a.eps);
-    ss = 0.0f;
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int c = gl + i * GT;
-      if (active && c < nck) {
-        float gw[8];
-        load8_gain(a.gw, 8 * c, gw);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          v[i][e] = __fmul_rn(__fmul_rn(v[i][e], rfh), gw[e]) * (a.pre_act ? g[i][e] : siluf_(g[i][e]));
-          ss = fmaf(v[i][e], v[i][e], ss);
-        }
-      }
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      const int c = gl + i * GT;
-      if (active && c < nck) {
-        if (MODE == kRowPlain) {
-          load8<XT>(a.x, row * a.ldx + 8 * c, v[i]);
-        } else {
-          float up[8];
-          load8<XT>(a.x, row * a.ldx + 8 * c, v[i]);
-          load8<XT>(a.x, row * a.ldx + k + 8 * c, up);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[i][e] = (a.pre_act ? v[i][e] : siluf_(v[i][e])) * up[e];
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(v[i][e], v[i][e], ss);
-      }
-    }
-  }
-  const float rf = nq_rinv(nq_group_sum<W>(ss, reds, phs), k, a.eps);
-  // v <- v / rms (and, with one gain, <- r = v / rms * gain); maxima of |r| per gain
-  float amax[NG];
-#pragma unroll
-  for (int j = 0; j < NG; ++j) amax[j] = 0.0f;
+  const int64_t nrb = (a.m + RPC - 1) / RPC;
+  Raw8<XT> rx[NCH], ry[TWO ? NCH : 1];
+  float2 gr[NG][NCH][4], gwr[GN ? NCH : 1][4];
 #pragma unroll
   for (int i = 0; i < NCH; ++i) {
     const int c = gl + i * GT;
-    if (active && c < nck) {
-      if (NG == 1) {
-        float gg[8];
-        load8_gain(a.gain[0], 8 * c, gg);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          v[i][e] = __fmul_rn(__fmul_rn(v[i][e], rf), gg[e]);
-          amax[0] = fmaxf(amax[0], fabsf(v[i][e]));
-        }
-      } else {
+    for (int j = 0; j < NG; ++j) {
+      if (c < nck && j < a.ngain) gain8(a.gain[j], 8 * c, gr[j][i]);
+      else
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[i][e] = __fmul_rn(v[i][e], rf);
+        for (int e = 0; e < 4; ++e) gr[j][i][e] = make_float2(0.0f, 0.0f);
+    }
+    if (GN) {
+      if (c < nck) gain8(a.gw, 8 * c, gwr[GN ? i : 0]);
+      else
 #pragma unroll
-        for (int j = 0; j < NG; ++j) {
-          if (j < a.ngain) {
-            float gg[8];
-            load8_gain(a.gain[j], 8 * c, gg);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) amax[j] = fmaxf(amax[j], fabsf(__fmul_rn(v[i][e], gg[e])));
-          }
-        }
-      }
+        for (int e = 0; e < 4; ++e) gwr[GN ? i : 0][e] = make_float2(0.0f, 0.0f);
     }
   }
-  nq_group_max<W, NG>(amax, redm, phm);
-  if (!active) return;
-#pragma unroll
-  for (int j = 0; j < NG; ++j) {
-    if (j < a.ngain) {
-      const float am = fmaxf(amax[j], 1e-5f);
-      const float sx = __fdiv_rn(127.0f, am);
-      int8_t* qrow = a.q[j] + row * a.ldq;
+
+  auto fetch = [&](int64_t rb) {
+    const int64_t row = rb * RPC + grp;
+    if (rb < nrb && row < a.m) {
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
         const int c = gl + i * GT;
         if (c < nck) {
-          uint32_t q[8];
-          if (NG == 1) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(v[i][e], sx));
-          } else {
-            float gg[8];
-            load8_gain(a.gain[j], 8 * c, gg);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(__fmul_rn(v[i][e], gg[e]), sx));
-          }
-          *reinterpret_cast<uint2*>(qrow + 8 * c) =
-              make_uint2(pack4_lo_bytes(q[0], q[1], q[2], q[3]), pack4_lo_bytes(q[4], q[5], q[6], q[7]));
+          raw8_load<XT>(a.x, row * a.ldx + 8 * c, rx[i]);
+          if (MODE == kRowGlu) raw8_load<XT>(a.x, row * a.ldx + k + 8 * c, ry[TWO ? i : 0]);
+          if (MODE == kRowGnorm) raw8_load<XT>(a.g, row * a.ldg + 8 * c, ry[TWO ? i : 0]);
         }
       }
-      for (int c = nck + gl; c < (int)(a.ldq >> 3); c += GT) *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(0u, 0u);
-      if (gl == 0) a.deq[j][row] = __fdiv_rn(am, 127.0f);
+    }
+  };
+
+  int64_t rb = blockIdx.x;
+  fetch(rb);
+  for (; rb < nrb; rb += gridDim.x) {
+    const int64_t row = rb * RPC + grp;
+    const bool active = row < a.m;
+    float2 v[NCH][4], y[TWO ? NCH : 1][4];
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      const int c = gl + i * GT;
+      if (active && c < nck) {
+        raw8_unpack<XT>(rx[i], v[i]);
+        if (TWO) raw8_unpack<XT>(ry[TWO ? i : 0], y[TWO ? i : 0]);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[i][e] = make_float2(0.0f, 0.0f);
+          if (TWO) y[TWO ? i : 0][e] = make_float2(0.0f, 0.0f);
+        }
+      }
+    }
+    fetch(rb + gridDim.x);  // the next row's loads are in flight during the work below
+
+    float2 ss2 = make_float2(0.0f, 0.0f);
+    if (MODE == kRowGlu) {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[i][e] = __fmul2_rn(a.pre_act ? v[i][e] : silu2(v[i][e]), y[TWO ? i : 0][e]);
+          ss2 = __ffma2_rn(v[i][e], v[i][e], ss2);
+        }
+    } else {
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) ss2 = __ffma2_rn(v[i][e], v[i][e], ss2);
+    }
+    if (GN) {
+      // u = h / rms(h) * w_g * SiLU(g), then the BitLinear norm of u
+      const float rfh = nq_rinv(nq_group_sum<W>(ss2.x + ss2.y, reds, phs), k, a.eps);
+      const float2 rfh2 = make_float2(rfh, rfh);
+      ss2 = make_float2(0.0f, 0.0f);
+#pragma unroll
+      for (int i = 0; i < NCH; ++i) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 sg = a.pre_act ? y[TWO ? i : 0][e] : silu2(y[TWO ? i : 0][e]);
+          v[i][e] = __fmul2_rn(__fmul2_rn(__fmul2_rn(v[i][e], rfh2), gwr[GN ? i : 0][e]), sg);
+          ss2 = __ffma2_rn(v[i][e], v[i][e], ss2);
+        }
+      }
+    }
+    const float rf = nq_rinv(nq_group_sum<W>(ss2.x + ss2.y, reds, phs), k, a.eps);
+    const float2 rf2 = make_float2(rf, rf);
+    // v <- v / rms (and, with one gain, <- r = v / rms * gain); maxima of |r| per gain
+    float amax[NG];
+#pragma unroll
+    for (int j = 0; j < NG; ++j) amax[j] = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NCH; ++i) {
+      if (NG == 1) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[i][e] = __fmul2_rn(__fmul2_rn(v[i][e], rf2), gr[0][i][e]);
+          amax[0] = amax2(amax[0], v[i][e]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) v[i][e] = __fmul2_rn(v[i][e], rf2);
+#pragma unroll
+        for (int j = 0; j < NG; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) amax[j] = amax2(amax[j], __fmul2_rn(v[i][e], gr[j][i][e]));
+      }
+    }
+    nq_group_max<W, NG>(amax, redm, phm);
+    if (active) {
+#pragma unroll
+      for (int j = 0; j < NG; ++j) {
+        if (j < a.ngain) {
+          const float am = fmaxf(amax[j], 1e-5f);
+          const float sx = __fdiv_rn(127.0f, am);
+          const float2 sx2 = make_float2(sx, sx);
+          int8_t* qrow = a.q[j] + row * a.ldq;
+#pragma unroll
+          for (int i = 0; i < NCH; ++i) {
+            const int c = gl + i * GT;
+            if (c < nck) {
+              float2 b[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e)
+                b[e] = q8_add2(__fmul2_rn(NG == 1 ? v[i][e] : __fmul2_rn(v[i][e], gr[j][i][e]), sx2));
+              *reinterpret_cast<uint2*>(qrow + 8 * c) = pack8_codes(b);
+            }
+          }
+          for (int c = nck + gl; c < (int)(a.ldq >> 3); c += GT) *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(0u, 0u);
+          if (gl == 0) a.deq[j][row] = __fdiv_rn(am, 127.0f);
+        }
+      }
     }
   }
 }

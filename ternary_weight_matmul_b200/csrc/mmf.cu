@@ -9,6 +9,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
 #include <string>
 #include <vector>
@@ -233,11 +234,43 @@ struct LaunchScope {
 // ---------------------------------------------------------------------------------------------
 template <mmf_dtype XT, int MODE, int NG>
 void nq_vec_launch(const NormQuantArgs& a, int w, int nch, cudaStream_t st) {
-  const unsigned rows_per_cta = 8u / (unsigned)w;
-  const dim3 grid((unsigned)((a.m + rows_per_cta - 1) / rows_per_cta));
-#define MMF_NQ(W_, C_) launch_k(norm_quant_vec_kernel<XT, MODE, W_, C_, NG>, grid, dim3(kNqThreads), 0, st, a)
+  const int64_t rows_per_cta = (kNqThreads / 32) / w;
+  const int64_t blocks = (a.m + rows_per_cta - 1) / rows_per_cta;
+  int sms = 148;
+  {
+    DevInfo* di = nullptr;
+    if (device_info(&di) == MMF_OK) sms = di->sms;
+  }
+  // persistent CTAs: as many as are resident at once (occupancy of this instantiation), each
+  // walking row blocks gridDim.x apart
+  const auto grid_for = [&](const void* fn) {
+    static std::mutex mu;
+    static std::map<const void*, int> per_sm;
+    int n = 0;
+    {
+      std::lock_guard<std::mutex> lk(mu);
+      auto it = per_sm.find(fn);
+      if (it == per_sm.end()) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, fn, kNqThreads, 0) != cudaSuccess || n < 1) n = 1;
+        per_sm[fn] = n;
+      } else {
+        n = it->second;
+      }
+    }
+    return dim3((unsigned)std::min<int64_t>(blocks, (int64_t)sms * n));
+  };
+#define MMF_NQ(W_, C_)                                                                    \
+  launch_k(norm_quant_vec_kernel<XT, MODE, W_, C_, NG>,                                   \
+           grid_for((const void*)norm_quant_vec_kernel<XT, MODE, W_, C_, NG>), dim3(kNqThreads), 0, st, a)
 #define MMF_NQ_W(W_) \
-  do { if (nch <= 2) MMF_NQ(W_, 2); else if (nch <= 4) MMF_NQ(W_, 4); else if (nch <= 6) MMF_NQ(W_, 6); else MMF_NQ(W_, 8); } while (0)
+  do {                                                                                    \
+    if (nch <= 1) MMF_NQ(W_, 1);                                                          \
+    else if (nch <= 2) MMF_NQ(W_, 2);                                                     \
+    else if (nch <= 3) MMF_NQ(W_, 3);                                                     \
+    else if (nch <= 4) MMF_NQ(W_, 4);                                                     \
+    else if (nch <= 6) MMF_NQ(W_, 6);                                                     \
+    else MMF_NQ(W_, 8);                                                                   \
+  } while (0)
   if (w == 1) MMF_NQ_W(1);
   else if (w == 2) MMF_NQ_W(2);
   else MMF_NQ_W(4);
@@ -273,10 +306,13 @@ mmf_status launch_norm_quant(const NormQuantArgs& a, int mode, cudaStream_t st) 
     vec = vec && a.gdt == a.xdt && al16(a.g) && (a.ldg * xes) % 16 == 0 && al16(a.gw);
   for (int j = 0; j < a.ngain; ++j) vec = vec && al16(a.gain[j]) && al16(a.q[j]);
   if (vec) {
-    // smallest row group (1, 2 or 4 warps) holding the row at up to eight 8-value chunks per
-    // thread, so the per-row reductions are amortised over many values
+    // smallest row group (1, 2 or 4 warps) whose threads hold at most `cap` 8-value chunks: the
+    // row, its prefetched successor and the register-resident gains of those columns then fit
+    // in about 100 registers (more warps per row only when the row needs it)
     const int nck = a.k / 8;
-    const int w = nck <= 256 ? 1 : nck <= 512 ? 2 : 4;
+    const int cap = (mode == kRowPlain && a.ngain == 1) ? 4 : 2;
+    int w = 1;
+    while (w < 4 && (nck + 32 * w - 1) / (32 * w) > cap) w *= 2;
     const int nch = (nck + 32 * w - 1) / (32 * w);
     if (a.xdt == MMF_F32) nq_vec_dispatch<MMF_F32>(a, mode, w, nch, st);
     else nq_vec_dispatch<MMF_BF16>(a, mode, w, nch, st);
