@@ -230,8 +230,8 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
       float t = 0.0f;
       for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[(w * 3 + j) * kMaxRows + r]);
       t = fmaxf(t, 1e-5f);
-      sxs[j * kMaxRows + r] = __fdiv_rn(127.0f, t);
-      deqs[j * kMaxRows + r] = __fdiv_rn(t, 127.0f);
+      sxs[j * kMaxRows + r] = q127_over(t);
+      deqs[j * kMaxRows + r] = over_127(t);
     }
   }
   __syncthreads();

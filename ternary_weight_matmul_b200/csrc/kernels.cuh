@@ -106,6 +106,16 @@ struct NormQuantArgs {
   int32_t pre_act; // 1: the SiLU of the gate input (g for g_norm, the gate half for GLU) is precomputed
 };
 
+// 1 / sqrt(ss / k + eps) in float32 (approximate reciprocal square root: 1/rms is a common
+// factor of a row's values and of their maximum, so it reaches a code only through rounding).
+__device__ __forceinline__ float nq_rinv(float ss, int k, float eps) {
+  return rsqrtf(__fdividef(ss, (float)k) + eps);
+}
+// 127 / a (correctly rounded: it sets every code of the row) and a / 127 (the dequantisation
+// factor, within 1.5 ulp), for a >= 1e-5.
+__device__ __forceinline__ float q127_over(float a) { return __fdiv_rn(127.0f, a); }
+__device__ __forceinline__ float over_127(float a) { return a * (1.0f / 127.0f); }
+
 __device__ __forceinline__ double block_sum_d(double v, double* red) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5, nw = (blockDim.x + 31) >> 5;
   v = warp_sum_d(v);
@@ -163,7 +173,7 @@ __global__ void __launch_bounds__(256) norm_quant_kernel(const NormQuantArgs a) 
       amax = fmaxf(amax, fabsf(r));
     }
     amax = fmaxf(block_max(amax, red), 1e-5f);
-    const float sx = __fdiv_rn(127.0f, amax);
+    const float sx = q127_over(amax);
     int8_t* qrow = a.q[j] + row * a.ldq;
     for (int c = threadIdx.x; c < a.ldq; c += blockDim.x) {
       int8_t code = 0;
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(256) norm_quant_kernel(const NormQuantArgs a) 
       }
       qrow[c] = code;
     }
-    if (threadIdx.x == 0) a.deq[j][row] = __fdiv_rn(amax, 127.0f);
+    if (threadIdx.x == 0) a.deq[j][row] = over_127(amax);
   }
 }
 
@@ -255,10 +265,6 @@ __device__ __forceinline__ void load8_gain(const float* g, int64_t idx, float (&
   o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
   o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
 }
-// 1 / sqrt(ss / k + eps) in float32 (IEEE division and square root).
-__device__ __forceinline__ float nq_rinv(float ss, int k, float eps) {
-  return __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(__fdiv_rn(ss, (float)k), eps)));
-}
 // Bits of x + 1.5 * 2^23 for |x| <= 127.5: the addition (where the float32 spacing is exactly 1)
 // rounds half to even, and the low byte of the result is the int8 code rint(x) itself
 // (0x4B400000 has a zero low byte). No clamp is needed: x = r * fl(127 / a) with a the maximum of
@@ -316,7 +322,24 @@ __device__ __forceinline__ void gain8(const float* g, int64_t idx, float2 (&o)[4
   o[2] = make_float2(b.x, b.y); o[3] = make_float2(b.z, b.w);
 }
 __device__ __forceinline__ float2 silu2(float2 z) { return make_float2(siluf_(z.x), siluf_(z.y)); }
-__device__ __forceinline__ float amax2(float m, float2 r) { return fmaxf(m, fmaxf(fabsf(r.x), fabsf(r.y))); }
+
+// Sum of squares of a thread's chunks: one packed accumulator per chunk, then a pairwise tree, so
+// the dependent chains are four products long instead of 4 * NCH.
+template <int NCH>
+__device__ __forceinline__ float2 sumsq_tree(const float2 (&v)[NCH][4]) {
+  float2 p[NCH];
+#pragma unroll
+  for (int i = 0; i < NCH; ++i) {
+    p[i] = __fmul2_rn(v[i][0], v[i][0]);
+#pragma unroll
+    for (int e = 1; e < 4; ++e) p[i] = __ffma2_rn(v[i][e], v[i][e], p[i]);
+  }
+#pragma unroll
+  for (int h = 1; h < NCH; h *= 2)
+#pragma unroll
+    for (int i = 0; i + h < NCH; i += 2 * h) p[i] = __fadd2_rn(p[i], p[i + h]);
+  return p[0];
+}
 
 // Row group of W warps per row, NCH chunks of 8 values per thread (K <= 256 * W * NCH). The CTAs
 // are persistent: each row group walks rows gridDim.x * (4 / W) apart. A thread sees the same
@@ -394,57 +417,60 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
     }
     fetch(rb + gridDim.x);  // the next row's loads are in flight during the work below
 
-    float2 ss2 = make_float2(0.0f, 0.0f);
     if (MODE == kRowGlu) {
 #pragma unroll
       for (int i = 0; i < NCH; ++i)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[i][e] = __fmul2_rn(a.pre_act ? v[i][e] : silu2(v[i][e]), y[TWO ? i : 0][e]);
-          ss2 = __ffma2_rn(v[i][e], v[i][e], ss2);
-        }
-    } else {
-#pragma unroll
-      for (int i = 0; i < NCH; ++i)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) ss2 = __ffma2_rn(v[i][e], v[i][e], ss2);
+        for (int e = 0; e < 4; ++e) v[i][e] = __fmul2_rn(a.pre_act ? v[i][e] : silu2(v[i][e]), y[TWO ? i : 0][e]);
     }
+    float2 ss2 = sumsq_tree<NCH>(v);
     if (GN) {
       // u = h / rms(h) * w_g * SiLU(g), then the BitLinear norm of u
       const float rfh = nq_rinv(nq_group_sum<W>(ss2.x + ss2.y, reds, phs), k, a.eps);
       const float2 rfh2 = make_float2(rfh, rfh);
-      ss2 = make_float2(0.0f, 0.0f);
 #pragma unroll
       for (int i = 0; i < NCH; ++i) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const float2 sg = a.pre_act ? y[TWO ? i : 0][e] : silu2(y[TWO ? i : 0][e]);
           v[i][e] = __fmul2_rn(__fmul2_rn(__fmul2_rn(v[i][e], rfh2), gwr[GN ? i : 0][e]), sg);
-          ss2 = __ffma2_rn(v[i][e], v[i][e], ss2);
         }
       }
+      ss2 = sumsq_tree<NCH>(v);
     }
     const float rf = nq_rinv(nq_group_sum<W>(ss2.x + ss2.y, reds, phs), k, a.eps);
     const float2 rf2 = make_float2(rf, rf);
     // v <- v / rms (and, with one gain, <- r = v / rms * gain); maxima of |r| per gain
     float amax[NG];
+    {
+      float am[NG][NCH];  // per-chunk maxima, combined as a tree (max is exact in any order)
 #pragma unroll
-    for (int j = 0; j < NG; ++j) amax[j] = 0.0f;
+      for (int i = 0; i < NCH; ++i) {
+        if (NG == 1) {
 #pragma unroll
-    for (int i = 0; i < NCH; ++i) {
-      if (NG == 1) {
+          for (int e = 0; e < 4; ++e) v[i][e] = __fmul2_rn(__fmul2_rn(v[i][e], rf2), gr[0][i][e]);
+          am[0][i] = fmaxf(fmaxf(fabsf(v[i][0].x), fabsf(v[i][0].y)), fmaxf(fabsf(v[i][1].x), fabsf(v[i][1].y)));
+          am[0][i] = fmaxf(am[0][i], fmaxf(fmaxf(fabsf(v[i][2].x), fabsf(v[i][2].y)), fmaxf(fabsf(v[i][3].x), fabsf(v[i][3].y))));
+        } else {
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          v[i][e] = __fmul2_rn(__fmul2_rn(v[i][e], rf2), gr[0][i][e]);
-          amax[0] = amax2(amax[0], v[i][e]);
+          for (int e = 0; e < 4; ++e) v[i][e] = __fmul2_rn(v[i][e], rf2);
+#pragma unroll
+          for (int j = 0; j < NG; ++j) {
+            float2 r[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) r[e] = __fmul2_rn(v[i][e], gr[j][i][e]);
+            am[j][i] = fmaxf(fmaxf(fmaxf(fabsf(r[0].x), fabsf(r[0].y)), fmaxf(fabsf(r[1].x), fabsf(r[1].y))),
+                             fmaxf(fmaxf(fabsf(r[2].x), fabsf(r[2].y)), fmaxf(fabsf(r[3].x), fabsf(r[3].y))));
+          }
         }
-      } else {
+      }
 #pragma unroll
-        for (int e = 0; e < 4; ++e) v[i][e] = __fmul2_rn(v[i][e], rf2);
+      for (int j = 0; j < NG; ++j) {
 #pragma unroll
-        for (int j = 0; j < NG; ++j)
+        for (int h = 1; h < NCH; h *= 2)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) amax[j] = amax2(amax[j], __fmul2_rn(v[i][e], gr[j][i][e]));
+          for (int i = 0; i + h < NCH; i += 2 * h) am[j][i] = fmaxf(am[j][i], am[j][i + h]);
+        amax[j] = am[j][0];
       }
     }
     nq_group_max<W, NG>(amax, redm, phm);
@@ -453,7 +479,7 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
       for (int j = 0; j < NG; ++j) {
         if (j < a.ngain) {
           const float am = fmaxf(amax[j], 1e-5f);
-          const float sx = __fdiv_rn(127.0f, am);
+          const float sx = q127_over(am);
           const float2 sx2 = make_float2(sx, sx);
           int8_t* qrow = a.q[j] + row * a.ldq;
 #pragma unroll
@@ -468,7 +494,7 @@ __global__ void __launch_bounds__(kNqThreads) norm_quant_vec_kernel(const NormQu
             }
           }
           for (int c = nck + gl; c < (int)(a.ldq >> 3); c += GT) *reinterpret_cast<uint2*>(qrow + 8 * c) = make_uint2(0u, 0u);
-          if (gl == 0) a.deq[j][row] = __fdiv_rn(am, 127.0f);
+          if (gl == 0) a.deq[j][row] = over_127(am);
         }
       }
     }
