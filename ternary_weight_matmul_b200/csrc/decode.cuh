@@ -11,7 +11,8 @@
 //          v = SiLU(gate) * up (epilogue);
 //   kDown  down_proj's RMSNorm + quantisation of v, down_proj and y = x1 + down (epilogue).
 // Each CTA owns a contiguous range of output channels. Its first thread starts bulk copies of
-// the input's norm gains and of the CTA's packed weight rows into shared memory (two barriers);
+// the input rows and their norm gains, and of the CTA's packed weight rows, into shared memory
+// (two barriers);
 // while the weights stream in, the CTA quantises the input rows itself -- every CTA computes the
 // same codes, in the arithmetic of norm_quant_vec_kernel -- and each warp then forms whole
 // output channels: lanes stride over 64-code chunks of the weight row (expanded with byte
@@ -61,7 +62,7 @@ struct Args {
 // Shared-memory layout of one CTA: weight rows, norm gains (ngain vectors of k floats; kO also
 // the g_norm gain), the g_norm output u (kO only, [b][k] float32), the codes, factors, scratch.
 struct Smem {
-  size_t w_bytes, gain_off, u_off, q_off, q_bytes, deq_off, red_off, bar_off, total;
+  size_t w_bytes, gain_off, u_off, x_off, q_off, q_bytes, deq_off, red_off, bar_off, total;
 };
 __host__ __device__ inline Smem smem_layout(int mode, int nmat, int chan_per_cta, int kw, int k, int ngain, int b) {
   Smem s;
@@ -70,7 +71,10 @@ __host__ __device__ inline Smem smem_layout(int mode, int nmat, int chan_per_cta
   const int ngv = ngain + (mode == kO ? 1 : 0);
   s.u_off = (s.gain_off + (size_t)ngv * k * 4 + 127) & ~(size_t)127;
   const size_t u_bytes = mode == kO ? (size_t)b * k * 4 : 0;
-  s.q_off = (s.u_off + u_bytes + 127) & ~(size_t)127;
+  // the input rows, copied in with the gains: x, x1 or v (<= 4 bytes per value); kO: h and g
+  s.x_off = (s.u_off + u_bytes + 127) & ~(size_t)127;
+  const size_t x_bytes = (size_t)(mode == kO ? 2 : 1) * b * k * 4;
+  s.q_off = (s.x_off + x_bytes + 127) & ~(size_t)127;
   s.q_bytes = (size_t)ngain * b * kw * 16;   // codes of the padded K, [gain][row][piece][chunk]
   s.deq_off = (s.q_off + s.q_bytes + 15) & ~(size_t)15;
   s.red_off = s.deq_off + 3 * kMaxRows * sizeof(float);
@@ -88,17 +92,17 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
-// Input value k of token row r as the projection's RMSNorm sees it: the row itself, or for kO
-// the g_norm output u staged in shared memory.
+// Input value k of token row r as the projection's RMSNorm sees it: the staged row itself, or for
+// kO the g_norm output u; both in shared memory.
 template <mmf_dtype XT>
-__device__ __forceinline__ void in8(const Args& a, const float* us, int r, int kk, float (&o)[8]) {
+__device__ __forceinline__ void in8(const Args& a, const float* us, const void* xs, int r, int kk, float (&o)[8]) {
   if (a.mode == kO) {
     const float4 p = *reinterpret_cast<const float4*>(us + (size_t)r * a.k + kk);
     const float4 q = *reinterpret_cast<const float4*>(us + (size_t)r * a.k + kk + 4);
     o[0] = p.x; o[1] = p.y; o[2] = p.z; o[3] = p.w;
     o[4] = q.x; o[5] = q.y; o[6] = q.z; o[7] = q.w;
   } else {
-    load8<XT>(a.x, (int64_t)r * a.k + kk, o);
+    load8<XT>(xs, (int64_t)r * a.k + kk, o);
   }
 }
 __device__ __forceinline__ void sm8(const float* p, float (&o)[8]) {
@@ -111,13 +115,16 @@ __device__ __forceinline__ void sm8(const float* p, float (&o)[8]) {
 // The kernel runs once per SM for a few microseconds, so its instructions are fetched cold:
 // the code is kept compact (runtime loops over rows, gains and matrices; per-row statistics in
 // shared memory) rather than unrolled.
-template <mmf_dtype XT>
+template <mmf_dtype XT, int NB>
 __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constant__ Args a) {
   extern __shared__ __align__(128) uint8_t sm[];
   const Smem L = smem_layout(a.mode, a.nmat, a.chan_per_cta, a.kw, a.k, a.ngain, a.b);
   uint32_t* wsm = reinterpret_cast<uint32_t*>(sm);
   float* gains = reinterpret_cast<float*>(sm + L.gain_off);   // [ngain (+1)][k]
   float* us = reinterpret_cast<float*>(sm + L.u_off);
+  uint8_t* xs = sm + L.x_off;                                 // staged input rows (kO: h, then g)
+  const float* hs = reinterpret_cast<const float*>(xs);
+  const float* gs = hs + (size_t)a.b * a.k;
   int8_t* qs = reinterpret_cast<int8_t*>(sm + L.q_off);
   float* deqs = reinterpret_cast<float*>(sm + L.deq_off);   // [gain][row] a/127
   float* red = reinterpret_cast<float*>(sm + L.red_off);    // [warp][gain][row] partials, then stats
@@ -135,10 +142,17 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
     mbar_fence_init();
-    uint32_t tx = 0;
+    const uint32_t xbytes = (uint32_t)a.b * (uint32_t)a.k * (a.mode == kO ? 4u : (XT == MMF_F32 ? 4u : 2u));
+    uint32_t tx = (a.mode == kO ? 2u : 1u) * xbytes;
     for (int j = 0; j < ng; ++j) tx += a.gain[j] ? gbytes : 0u;
     if (has_gw) tx += gbytes;
     mbar_arrive_expect_tx(&bar[0], tx);
+    if (a.mode == kO) {
+      bulk_load(xs, a.h, xbytes, &bar[0]);
+      bulk_load(xs + xbytes, a.gin, xbytes, &bar[0]);
+    } else {
+      bulk_load(xs, a.x, xbytes, &bar[0]);
+    }
     for (int j = 0; j < ng; ++j)
       if (a.gain[j]) bulk_load(gains + (size_t)j * a.k, a.gain[j], gbytes, &bar[0]);
     if (has_gw) bulk_load(gains + (size_t)ng * a.k, a.gnorm_w, gbytes, &bar[0]);
@@ -178,11 +192,11 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
       for (int c = threadIdx.x; c < nck; c += kThreads) {
         float v[8];
         if (a.mode == kO && pass == 0) {
-          load8<MMF_F32>(a.h, (int64_t)r * a.k + 8 * c, v);
+          load8<MMF_F32>(hs, (int64_t)r * a.k + 8 * c, v);
         } else if (a.mode == kO) {
           float g[8], w8[8];
-          load8<MMF_F32>(a.h, (int64_t)r * a.k + 8 * c, v);
-          load8<MMF_F32>(a.gin, (int64_t)r * a.k + 8 * c, g);
+          load8<MMF_F32>(hs, (int64_t)r * a.k + 8 * c, v);
+          load8<MMF_F32>(gs, (int64_t)r * a.k + 8 * c, g);
           sm8(gains + (size_t)ng * a.k + 8 * c, w8);
           const float rfh = rfs[r];
 #pragma unroll
@@ -191,7 +205,7 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
           *reinterpret_cast<float4*>(up) = make_float4(v[0], v[1], v[2], v[3]);
           *reinterpret_cast<float4*>(up + 4) = make_float4(v[4], v[5], v[6], v[7]);
         } else {
-          load8<XT>(a.x, (int64_t)r * a.k + 8 * c, v);
+          load8<XT>(xs, (int64_t)r * a.k + 8 * c, v);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
@@ -214,7 +228,7 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
       float am = 0.0f;
       for (int c = threadIdx.x; c < nck; c += kThreads) {
         float v[8], gg[8];
-        in8<XT>(a, us, r, 8 * c, v);
+        in8<XT>(a, us, xs, r, 8 * c, v);
         sm8(gains + (size_t)j * a.k + 8 * c, gg);
 #pragma unroll
         for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(__fmul_rn(__fmul_rn(v[e], rf), gg[e])));
@@ -244,7 +258,7 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
       int8_t* qrow = qs + (size_t)(j * a.b + r) * kq;
       for (int c = threadIdx.x; c < nck; c += kThreads) {
         float v[8], gg[8];
-        in8<XT>(a, us, r, 8 * c, v);
+        in8<XT>(a, us, xs, r, 8 * c, v);
         sm8(gains + (size_t)j * a.k + 8 * c, gg);
         uint32_t q[8];
 #pragma unroll
@@ -259,49 +273,44 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
 
   if (!wait_or_leave(1)) return;
 
-  // 3. one warp per output channel: each weight row against all token rows; lane r keeps the
-  //    total of token row r
-  const int nchunk = a.kw >> 2;           // 16-byte chunks (64 codes) per weight row
+  // 3. one warp per output channel: lanes stride over 32-code (8-byte) pieces of each weight row
+  //    of the channel, dp4a against the codes of the NB token rows (NB = b, a compile-time count
+  //    so no work is issued for absent rows); lane r keeps the total of token row r
+  const int npc = a.kw >> 1;              // 8-byte pieces per weight row
   for (int cl = warp; cl < nc; cl += kWarps) {
     int tot0 = 0, tot1 = 0, tot2 = 0;
     for (int m = 0; m < a.nmat; ++m) {
       const int gsel = ng == 3 ? m : 0;
-      int acc[kMaxRows];
+      int acc[NB];
 #pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) acc[r] = 0;
-      const uint4* wrow = reinterpret_cast<const uint4*>(wsm + ((size_t)m * a.chan_per_cta + cl) * a.kw);
-      const int8_t* qg = qs + (size_t)gsel * a.b * kq;
-      for (int ch = lane; ch < nchunk; ch += 32) {
-        const uint4 wv = wrow[ch];
-        uint32_t e[16];
+      for (int r = 0; r < NB; ++r) acc[r] = 0;
+      const uint2* wrow = reinterpret_cast<const uint2*>(wsm + ((size_t)m * a.chan_per_cta + cl) * a.kw);
+      const int8_t* qg = qs + (size_t)gsel * NB * kq;
+      for (int pc = lane; pc < npc; pc += 32) {
+        const uint2 wv = wrow[pc];
+        uint32_t e[8];
         expand_word(wv.x, e + 0);
         expand_word(wv.y, e + 4);
-        expand_word(wv.z, e + 8);
-        expand_word(wv.w, e + 12);
+        const int8_t* qc = qg + (pc >> 1) * 16 + (pc & 1) * 2 * (kq >> 2);  // 64-code chunk, piece pair
 #pragma unroll
-        for (int r = 0; r < kMaxRows; ++r) {
-          if (r < a.b) {
-            const int8_t* qr = qg + (size_t)r * kq + ch * 16;
+        for (int r = 0; r < NB; ++r) {
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const uint4 av = *reinterpret_cast<const uint4*>(qr + p * (kq >> 2));
-              acc[r] = __dp4a((int)e[4 * p + 0], (int)av.x, acc[r]);
-              acc[r] = __dp4a((int)e[4 * p + 1], (int)av.y, acc[r]);
-              acc[r] = __dp4a((int)e[4 * p + 2], (int)av.z, acc[r]);
-              acc[r] = __dp4a((int)e[4 * p + 3], (int)av.w, acc[r]);
-            }
+          for (int pp = 0; pp < 2; ++pp) {
+            const uint4 av = *reinterpret_cast<const uint4*>(qc + (size_t)r * kq + pp * (kq >> 2));
+            acc[r] = __dp4a((int)e[4 * pp + 0], (int)av.x, acc[r]);
+            acc[r] = __dp4a((int)e[4 * pp + 1], (int)av.y, acc[r]);
+            acc[r] = __dp4a((int)e[4 * pp + 2], (int)av.z, acc[r]);
+            acc[r] = __dp4a((int)e[4 * pp + 3], (int)av.w, acc[r]);
           }
         }
       }
       int mine = 0;
 #pragma unroll
-      for (int r = 0; r < kMaxRows; ++r) {
-        if (r < a.b) {
-          int s = acc[r];
+      for (int r = 0; r < NB; ++r) {
+        int s = acc[r];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-          if (lane == r) mine = s;
-        }
+        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+        if (lane == r) mine = s;
       }
       if (m == 0) tot0 = mine;
       else if (m == 1) tot1 = mine;

@@ -111,8 +111,10 @@ mmf_status device_info(DevInfo** out) {
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, tc::SMEM_BYTES));
       MMF_CUDA(cudaFuncSetAttribute(simt_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     200 * 1024));
-      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_F32>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
-      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_F32, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_F32, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
       MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowPlain>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
       MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowGlu>,
@@ -931,8 +933,14 @@ mmf_status launch_dec(dec::Args& a, const DevInfo& di, cudaStream_t st) {
   double bytes = 0;
   for (int j = 0; j < a.nmat; ++j) bytes += (double)a.nout * a.kw * 4.0;
   LaunchScope ls(MMF_KERNEL_GEMM_SIMT, bytes, st);
-  if (a.xdt == MMF_F32) launch_k(dec::dec_proj_kernel<MMF_F32>, grid, dim3(dec::kThreads), L.total, st, a);
-  else launch_k(dec::dec_proj_kernel<MMF_BF16>, grid, dim3(dec::kThreads), L.total, st, a);
+  if (a.b != 1 && a.b != 2) return fail(MMF_ERR_UNSUPPORTED, "fused decode takes 1 or 2 token rows, got %d", a.b);
+  if (a.xdt == MMF_F32) {
+    if (a.b == 1) launch_k(dec::dec_proj_kernel<MMF_F32, 1>, grid, dim3(dec::kThreads), L.total, st, a);
+    else launch_k(dec::dec_proj_kernel<MMF_F32, 2>, grid, dim3(dec::kThreads), L.total, st, a);
+  } else {
+    if (a.b == 1) launch_k(dec::dec_proj_kernel<MMF_BF16, 1>, grid, dim3(dec::kThreads), L.total, st, a);
+    else launch_k(dec::dec_proj_kernel<MMF_BF16, 2>, grid, dim3(dec::kThreads), L.total, st, a);
+  }
   return check_launch("dec_proj_kernel");
 }
 
@@ -1002,7 +1010,7 @@ mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, co
   uint8_t* pp = reinterpret_cast<uint8_t*>(ws) + W.bytes;
   void* buf[2] = {pp, pp + align256((size_t)b * d * 4)};
   const void* cur = x;
-  const bool fused = decode_fused(b, d, inner);
+  const bool fused = decode_fused(b, d, inner) && al16(x);  // the input rows are bulk-copied
   for (int l = 0; l < n_layers; ++l) {
     void* out = (l == n_layers - 1) ? y : buf[l & 1];
     float* st_l = state + (int64_t)l * b * d;
