@@ -28,6 +28,7 @@ namespace dec {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxRows = 8;            // token rows per launch
+constexpr int kStageRows = 2;          // input rows staged in shared memory up to this count
 constexpr int kMaxSmem = 200 * 1024;   // dynamic shared memory budget per CTA
 
 enum Mode : int32_t { kIFG = 0, kO = 1, kGate = 2, kDown = 3 };
@@ -71,9 +72,10 @@ __host__ __device__ inline Smem smem_layout(int mode, int nmat, int chan_per_cta
   const int ngv = ngain + (mode == kO ? 1 : 0);
   s.u_off = (s.gain_off + (size_t)ngv * k * 4 + 127) & ~(size_t)127;
   const size_t u_bytes = mode == kO ? (size_t)b * k * 4 : 0;
-  // the input rows, copied in with the gains: x, x1 or v (<= 4 bytes per value); kO: h and g
+  // the input rows, copied in with the gains when there are at most kStageRows of them: x, x1
+  // or v (<= 4 bytes per value); kO: h and g. More rows are read from global memory.
   s.x_off = (s.u_off + u_bytes + 127) & ~(size_t)127;
-  const size_t x_bytes = (size_t)(mode == kO ? 2 : 1) * b * k * 4;
+  const size_t x_bytes = b <= kStageRows ? (size_t)(mode == kO ? 2 : 1) * b * k * 4 : 0;
   s.q_off = (s.x_off + x_bytes + 127) & ~(size_t)127;
   s.q_bytes = (size_t)ngain * b * kw * 16;   // codes of the padded K, [gain][row][piece][chunk]
   s.deq_off = (s.q_off + s.q_bytes + 15) & ~(size_t)15;
@@ -122,9 +124,12 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
   uint32_t* wsm = reinterpret_cast<uint32_t*>(sm);
   float* gains = reinterpret_cast<float*>(sm + L.gain_off);   // [ngain (+1)][k]
   float* us = reinterpret_cast<float*>(sm + L.u_off);
-  uint8_t* xs = sm + L.x_off;                                 // staged input rows (kO: h, then g)
-  const float* hs = reinterpret_cast<const float*>(xs);
-  const float* gs = hs + (size_t)a.b * a.k;
+  // input rows: staged in shared memory (kO: h, then g) or read in place
+  constexpr bool kStage = NB <= kStageRows;
+  uint8_t* xsm = sm + L.x_off;
+  const void* xs = kStage ? static_cast<const void*>(xsm) : a.x;
+  const float* hs = kStage ? reinterpret_cast<const float*>(xsm) : a.h;
+  const float* gs = kStage ? hs + (size_t)a.b * a.k : a.gin;
   int8_t* qs = reinterpret_cast<int8_t*>(sm + L.q_off);
   float* deqs = reinterpret_cast<float*>(sm + L.deq_off);   // [gain][row] a/127
   float* red = reinterpret_cast<float*>(sm + L.red_off);    // [warp][gain][row] partials, then stats
@@ -142,16 +147,16 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
     mbar_fence_init();
-    const uint32_t xbytes = (uint32_t)a.b * (uint32_t)a.k * (a.mode == kO ? 4u : (XT == MMF_F32 ? 4u : 2u));
+    const uint32_t xbytes = kStage ? (uint32_t)a.b * (uint32_t)a.k * (a.mode == kO ? 4u : (XT == MMF_F32 ? 4u : 2u)) : 0u;
     uint32_t tx = (a.mode == kO ? 2u : 1u) * xbytes;
     for (int j = 0; j < ng; ++j) tx += a.gain[j] ? gbytes : 0u;
     if (has_gw) tx += gbytes;
     mbar_arrive_expect_tx(&bar[0], tx);
-    if (a.mode == kO) {
-      bulk_load(xs, a.h, xbytes, &bar[0]);
-      bulk_load(xs + xbytes, a.gin, xbytes, &bar[0]);
-    } else {
-      bulk_load(xs, a.x, xbytes, &bar[0]);
+    if (kStage && a.mode == kO) {
+      bulk_load(xsm, a.h, xbytes, &bar[0]);
+      bulk_load(xsm + xbytes, a.gin, xbytes, &bar[0]);
+    } else if (kStage) {
+      bulk_load(xsm, a.x, xbytes, &bar[0]);
     }
     for (int j = 0; j < ng; ++j)
       if (a.gain[j]) bulk_load(gains + (size_t)j * a.k, a.gain[j], gbytes, &bar[0]);
@@ -179,7 +184,9 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
   };
   if (!wait_or_leave(0)) return;
 
-  // 2. prologue: the codes of every input row (the same in every CTA).
+  // 2. prologue: the codes of every input row (the same in every CTA). The row loops run over
+  //    the compile-time count NB inside the chunk loops, so the loads of all rows are in flight
+  //    together (the rows are read in place when there are more than kStageRows of them).
   const int nck = a.k >> 3;
   const int kq = a.kw * 16;
   float* rfs = red + kWarps * 3 * kMaxRows;          // [row] 1/rms
@@ -187,34 +194,47 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
   // 2a. mean squares of every row (kO: of h, then u = h / rms(h) * w_g * SiLU(g) into shared
   //     memory and its mean squares)
   for (int pass = 0; pass < (a.mode == kO ? 2 : 1); ++pass) {
-    for (int r = 0; r < a.b; ++r) {
-      float ss = 0.0f;
-      for (int c = threadIdx.x; c < nck; c += kThreads) {
-        float v[8];
-        if (a.mode == kO && pass == 0) {
-          load8<MMF_F32>(hs, (int64_t)r * a.k + 8 * c, v);
-        } else if (a.mode == kO) {
-          float g[8], w8[8];
+    float ss[NB];
+#pragma unroll
+    for (int r = 0; r < NB; ++r) ss[r] = 0.0f;
+    for (int c = threadIdx.x; c < nck; c += kThreads) {
+      if (a.mode == kO && pass == 1) {
+        float w8[8];
+        sm8(gains + (size_t)ng * a.k + 8 * c, w8);
+#pragma unroll
+        for (int r = 0; r < NB; ++r) {
+          float v[8], g[8];
           load8<MMF_F32>(hs, (int64_t)r * a.k + 8 * c, v);
           load8<MMF_F32>(gs, (int64_t)r * a.k + 8 * c, g);
-          sm8(gains + (size_t)ng * a.k + 8 * c, w8);
           const float rfh = rfs[r];
 #pragma unroll
           for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(__fmul_rn(v[e], rfh), w8[e]) * siluf_(g[e]);
           float* up = us + (size_t)r * a.k + 8 * c;
           *reinterpret_cast<float4*>(up) = make_float4(v[0], v[1], v[2], v[3]);
           *reinterpret_cast<float4*>(up + 4) = make_float4(v[4], v[5], v[6], v[7]);
-        } else {
-          load8<XT>(xs, (int64_t)r * a.k + 8 * c, v);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss[r] = fmaf(v[e], v[e], ss[r]);
+        }
+      } else {
+        float v[NB][8];
+#pragma unroll
+        for (int r = 0; r < NB; ++r) {
+          if (a.mode == kO) load8<MMF_F32>(hs, (int64_t)r * a.k + 8 * c, v[r]);
+          else load8<XT>(xs, (int64_t)r * a.k + 8 * c, v[r]);
         }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+        for (int r = 0; r < NB; ++r)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ss[r] = fmaf(v[r][e], v[r][e], ss[r]);
       }
-      ss = warp_sum(ss);
-      if (lane == 0) red[warp * kMaxRows + r] = ss;
+    }
+#pragma unroll
+    for (int r = 0; r < NB; ++r) {
+      const float t = warp_sum(ss[r]);
+      if (lane == 0) red[warp * kMaxRows + r] = t;
     }
     __syncthreads();
-    if (threadIdx.x < a.b) {
+    if (threadIdx.x < NB) {
       float t = 0.0f;
       for (int w = 0; w < kWarps; ++w) t += red[w * kMaxRows + threadIdx.x];
       rfs[threadIdx.x] = nq_rinv(t, a.k, a.eps);
@@ -222,25 +242,33 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
     __syncthreads();
   }
   // 2b. maxima of |r| = |v / rms * gain| per (gain, row)
-  for (int r = 0; r < a.b; ++r) {
-    const float rf = rfs[r];
-    for (int j = 0; j < ng; ++j) {
-      float am = 0.0f;
-      for (int c = threadIdx.x; c < nck; c += kThreads) {
-        float v[8], gg[8];
-        in8<XT>(a, us, xs, r, 8 * c, v);
-        sm8(gains + (size_t)j * a.k + 8 * c, gg);
+  for (int j = 0; j < ng; ++j) {
+    float am[NB];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(__fmul_rn(__fmul_rn(v[e], rf), gg[e])));
+    for (int r = 0; r < NB; ++r) am[r] = 0.0f;
+    for (int c = threadIdx.x; c < nck; c += kThreads) {
+      float gg[8];
+      sm8(gains + (size_t)j * a.k + 8 * c, gg);
+      float v[NB][8];
+#pragma unroll
+      for (int r = 0; r < NB; ++r) in8<XT>(a, us, xs, r, 8 * c, v[r]);
+#pragma unroll
+      for (int r = 0; r < NB; ++r) {
+        const float rf = rfs[r];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) am[r] = fmaxf(am[r], fabsf(__fmul_rn(__fmul_rn(v[r][e], rf), gg[e])));
       }
-      am = warp_max(am);
-      if (lane == 0) red[(warp * 3 + j) * kMaxRows + r] = am;
+    }
+#pragma unroll
+    for (int r = 0; r < NB; ++r) {
+      const float t = warp_max(am[r]);
+      if (lane == 0) red[(warp * 3 + j) * kMaxRows + r] = t;
     }
   }
   __syncthreads();
   if (threadIdx.x < ng * kMaxRows) {
     const int j = threadIdx.x / kMaxRows, r = threadIdx.x - j * kMaxRows;
-    if (r < a.b) {
+    if (r < NB) {
       float t = 0.0f;
       for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[(w * 3 + j) * kMaxRows + r]);
       t = fmaxf(t, 1e-5f);
@@ -251,19 +279,21 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
   __syncthreads();
   // 2c. codes, piece-major: code k of (gain j, row r) at
   //     qs + (j * b + r) * kq + ((k % 64) / 16) * (kq / 4) + (k / 64) * 16 + k % 16
-  for (int r = 0; r < a.b; ++r) {
-    const float rf = rfs[r];
-    for (int j = 0; j < ng; ++j) {
-      const float sx = sxs[j * kMaxRows + r];
-      int8_t* qrow = qs + (size_t)(j * a.b + r) * kq;
-      for (int c = threadIdx.x; c < nck; c += kThreads) {
-        float v[8], gg[8];
-        in8<XT>(a, us, xs, r, 8 * c, v);
-        sm8(gains + (size_t)j * a.k + 8 * c, gg);
+  for (int j = 0; j < ng; ++j) {
+    for (int c = threadIdx.x; c < nck; c += kThreads) {
+      float gg[8];
+      sm8(gains + (size_t)j * a.k + 8 * c, gg);
+      float v[NB][8];
+#pragma unroll
+      for (int r = 0; r < NB; ++r) in8<XT>(a, us, xs, r, 8 * c, v[r]);
+      const int kk = 8 * c;
+#pragma unroll
+      for (int r = 0; r < NB; ++r) {
+        const float rf = rfs[r], sx = sxs[j * kMaxRows + r];
         uint32_t q[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(__fmul_rn(__fmul_rn(v[e], rf), gg[e]), sx));
-        const int kk = 8 * c;
+        for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(__fmul_rn(__fmul_rn(v[r][e], rf), gg[e]), sx));
+        int8_t* qrow = qs + (size_t)(j * NB + r) * kq;
         *reinterpret_cast<uint2*>(qrow + ((kk & 63) >> 4) * (kq >> 2) + (kk >> 6) * 16 + (kk & 15)) =
             make_uint2(pack4_lo_bytes(q[0], q[1], q[2], q[3]), pack4_lo_bytes(q[4], q[5], q[6], q[7]));
       }
@@ -273,60 +303,77 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
 
   if (!wait_or_leave(1)) return;
 
-  // 3. one warp per output channel: lanes stride over 32-code (8-byte) pieces of each weight row
-  //    of the channel, dp4a against the codes of the NB token rows (NB = b, a compile-time count
-  //    so no work is issued for absent rows); lane r keeps the total of token row r
+  // 3. each warp forms kCpw output channels at once: lanes stride over 32-code (8-byte) pieces
+  //    of the channels' weight rows, load the codes of the NB token rows for a piece once and
+  //    dp4a them against all kCpw rows (NB = b is a compile-time count, so no work is issued for
+  //    absent rows); lane r keeps the totals of token row r
+  constexpr int kCpw = NB >= 4 ? 4 : 1;
   const int npc = a.kw >> 1;              // 8-byte pieces per weight row
-  for (int cl = warp; cl < nc; cl += kWarps) {
-    int tot0 = 0, tot1 = 0, tot2 = 0;
+  for (int cg = warp * kCpw; cg < nc; cg += kWarps * kCpw) {
+    int tot0[kCpw], tot1[kCpw], tot2[kCpw];
     for (int m = 0; m < a.nmat; ++m) {
       const int gsel = ng == 3 ? m : 0;
-      int acc[NB];
+      int acc[kCpw][NB];
 #pragma unroll
-      for (int r = 0; r < NB; ++r) acc[r] = 0;
-      const uint2* wrow = reinterpret_cast<const uint2*>(wsm + ((size_t)m * a.chan_per_cta + cl) * a.kw);
+      for (int c = 0; c < kCpw; ++c)
+#pragma unroll
+        for (int r = 0; r < NB; ++r) acc[c][r] = 0;
+      const uint2* wrow = reinterpret_cast<const uint2*>(wsm + ((size_t)m * a.chan_per_cta + cg) * a.kw);
       const int8_t* qg = qs + (size_t)gsel * NB * kq;
       for (int pc = lane; pc < npc; pc += 32) {
-        const uint2 wv = wrow[pc];
-        uint32_t e[8];
-        expand_word(wv.x, e + 0);
-        expand_word(wv.y, e + 4);
         const int8_t* qc = qg + (pc >> 1) * 16 + (pc & 1) * 2 * (kq >> 2);  // 64-code chunk, piece pair
+        uint4 av[NB][2];
 #pragma unroll
-        for (int r = 0; r < NB; ++r) {
+        for (int r = 0; r < NB; ++r)
 #pragma unroll
-          for (int pp = 0; pp < 2; ++pp) {
-            const uint4 av = *reinterpret_cast<const uint4*>(qc + (size_t)r * kq + pp * (kq >> 2));
-            acc[r] = __dp4a((int)e[4 * pp + 0], (int)av.x, acc[r]);
-            acc[r] = __dp4a((int)e[4 * pp + 1], (int)av.y, acc[r]);
-            acc[r] = __dp4a((int)e[4 * pp + 2], (int)av.z, acc[r]);
-            acc[r] = __dp4a((int)e[4 * pp + 3], (int)av.w, acc[r]);
+          for (int pp = 0; pp < 2; ++pp) av[r][pp] = *reinterpret_cast<const uint4*>(qc + (size_t)r * kq + pp * (kq >> 2));
+#pragma unroll
+        for (int c = 0; c < kCpw; ++c) {
+          if (cg + c < nc) {
+            const uint2 wv = wrow[(size_t)c * (a.kw >> 1) + pc];
+            uint32_t e[8];
+            expand_word(wv.x, e + 0);
+            expand_word(wv.y, e + 4);
+#pragma unroll
+            for (int r = 0; r < NB; ++r)
+#pragma unroll
+              for (int pp = 0; pp < 2; ++pp) {
+                acc[c][r] = __dp4a((int)e[4 * pp + 0], (int)av[r][pp].x, acc[c][r]);
+                acc[c][r] = __dp4a((int)e[4 * pp + 1], (int)av[r][pp].y, acc[c][r]);
+                acc[c][r] = __dp4a((int)e[4 * pp + 2], (int)av[r][pp].z, acc[c][r]);
+                acc[c][r] = __dp4a((int)e[4 * pp + 3], (int)av[r][pp].w, acc[c][r]);
+              }
           }
         }
       }
-      int mine = 0;
 #pragma unroll
-      for (int r = 0; r < NB; ++r) {
-        int s = acc[r];
+      for (int c = 0; c < kCpw; ++c) {
+        int mine = 0;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-        if (lane == r) mine = s;
+        for (int r = 0; r < NB; ++r) {
+          int s = acc[c][r];
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (lane == r) mine = s;
+        }
+        if (m == 0) tot0[c] = mine;
+        else if (m == 1) tot1[c] = mine;
+        else tot2[c] = mine;
       }
-      if (m == 0) tot0 = mine;
-      else if (m == 1) tot1 = mine;
-      else tot2 = mine;
     }
-    if (lane < a.b) {
+#pragma unroll
+    for (int cc = 0; cc < kCpw; ++cc) {
+      if (cg + cc >= nc || lane >= a.b) continue;
       const int r = lane;
-      const int c = c0 + cl;
-      const int64_t o = (int64_t)r * a.nout + c;
+      const int64_t o = (int64_t)r * a.nout + c0 + cg + cc;
+      const int t0 = tot0[cc], t1 = a.nmat > 1 ? tot1[cc] : 0, t2 = a.nmat > 2 ? tot2[cc] : 0;
       auto zof = [&](int m, int tot) {
         const int gsel = ng == 3 ? m : 0;
         return __fmul_rn((float)tot, __fmul_rn(deqs[gsel * kMaxRows + r], a.sw[m][0]));
       };
       if (a.mode == kIFG) {
         // f = sigmoid(zf), i = SiLU(zi) * (1 - f), h = f * h_prev + i
-        const float zi = zof(0, tot0), zf = zof(1, tot1), zg = zof(2, tot2);
+        const float zi = zof(0, t0), zf = zof(1, t1), zg = zof(2, t2);
         float f, omf;
         hgrn_forget(zf, f, omf);
         const float iv = siluf_(zi) * omf;
@@ -335,9 +382,9 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
         reinterpret_cast<float*>(a.y)[o] = hv;
         a.g_out[o] = zg;
       } else if (a.mode == kGate) {
-        store_from_float(a.y, o, a.ydt, siluf_(zof(0, tot0)) * zof(1, tot1));
+        store_from_float(a.y, o, a.ydt, siluf_(zof(0, t0)) * zof(1, t1));
       } else {
-        store_from_float(a.y, o, a.ydt, zof(0, tot0) + load_as_float(a.res, o, a.ydt));
+        store_from_float(a.y, o, a.ydt, zof(0, t0) + load_as_float(a.res, o, a.ydt));
       }
     }
   }

@@ -115,6 +115,10 @@ mmf_status device_info(DevInfo** out) {
       MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_F32, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
       MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
       MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_F32, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_F32, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
+      MMF_CUDA(cudaFuncSetAttribute(dec::dec_proj_kernel<MMF_BF16, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, dec::kMaxSmem));
       MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowPlain>,
                                     cudaFuncAttributeMaxDynamicSharedMemorySize, 160 * 1024));
       MMF_CUDA(cudaFuncSetAttribute(norm_quant_kernel<kRowGlu>,
@@ -912,7 +916,8 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
 // (One or two rows: with more, the per-CTA quantisation of every input row costs more than the
 // separate norm-quant launches it replaces.)
 bool decode_fused(int32_t b, int32_t d, int32_t inner) {
-  if (b < 1 || b > 2 || use_tensor_path(b)) return false;
+  // 1, 2, 4 or 8 token rows (the kernel's compile-time row count must equal b)
+  if ((b != 1 && b != 2 && b != 4 && b != 8) || use_tensor_path(b)) return false;
   if (d % 8 || inner % 8) return false;
   return true;
 }
@@ -933,14 +938,22 @@ mmf_status launch_dec(dec::Args& a, const DevInfo& di, cudaStream_t st) {
   double bytes = 0;
   for (int j = 0; j < a.nmat; ++j) bytes += (double)a.nout * a.kw * 4.0;
   LaunchScope ls(MMF_KERNEL_GEMM_SIMT, bytes, st);
-  if (a.b != 1 && a.b != 2) return fail(MMF_ERR_UNSUPPORTED, "fused decode takes 1 or 2 token rows, got %d", a.b);
+  if (a.b != 1 && a.b != 2 && a.b != 4 && a.b != 8)
+    return fail(MMF_ERR_UNSUPPORTED, "fused decode takes 1, 2, 4 or 8 token rows, got %d", a.b);
+  // token rows as a compile-time count: 1, 2, 4 or 8 (decode_fused admits no other count)
+#define MMF_DEC(XT_, NB_) launch_k(dec::dec_proj_kernel<XT_, NB_>, grid, dim3(dec::kThreads), L.total, st, a)
   if (a.xdt == MMF_F32) {
-    if (a.b == 1) launch_k(dec::dec_proj_kernel<MMF_F32, 1>, grid, dim3(dec::kThreads), L.total, st, a);
-    else launch_k(dec::dec_proj_kernel<MMF_F32, 2>, grid, dim3(dec::kThreads), L.total, st, a);
+    if (a.b == 1) MMF_DEC(MMF_F32, 1);
+    else if (a.b == 2) MMF_DEC(MMF_F32, 2);
+    else if (a.b == 4) MMF_DEC(MMF_F32, 4);
+    else MMF_DEC(MMF_F32, 8);
   } else {
-    if (a.b == 1) launch_k(dec::dec_proj_kernel<MMF_BF16, 1>, grid, dim3(dec::kThreads), L.total, st, a);
-    else launch_k(dec::dec_proj_kernel<MMF_BF16, 2>, grid, dim3(dec::kThreads), L.total, st, a);
+    if (a.b == 1) MMF_DEC(MMF_BF16, 1);
+    else if (a.b == 2) MMF_DEC(MMF_BF16, 2);
+    else if (a.b == 4) MMF_DEC(MMF_BF16, 4);
+    else MMF_DEC(MMF_BF16, 8);
   }
+#undef MMF_DEC
   return check_launch("dec_proj_kernel");
 }
 

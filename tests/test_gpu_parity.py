@@ -436,7 +436,7 @@ def test_block_prefill_equals_stepwise_decode_on_gpu(mmf):
     np.testing.assert_allclose(state[1].cpu().numpy(), h2.cpu().numpy(), rtol=1e-4, atol=1e-4)
 
 
-@pytest.mark.parametrize("b", [1, 2, 3, 8, 64])
+@pytest.mark.parametrize("b", [1, 2, 3, 4, 8, 64])
 def test_decode_step_parity(mmf, b):
     layers = [_block_case(mmf, 20 + l, 256, 704) for l in range(2)]
     x = synth.activations(30 + b, (b, 256))
@@ -452,10 +452,11 @@ def test_decode_step_parity(mmf, b):
     np.testing.assert_allclose(st.cpu().numpy(), st_ref, rtol=1e-2, atol=1e-3)
 
 
-@pytest.mark.parametrize("b", [1, 2])
+@pytest.mark.parametrize("b", [1, 2, 4, 8])
 def test_decode_fused_matches_unfused(mmf, b):
-    # one or two rows take the fused four-launch decode; forcing the tensor-core engine takes the
-    # nine-launch block path instead. Same quantisation arithmetic: states agree closely and the
+    # 1, 2, 4 or 8 rows take the fused four-launch decode (inputs staged in shared memory up to
+    # two rows, read in place beyond); forcing the tensor-core engine takes the nine-launch block
+    # path instead. Same quantisation arithmetic: states agree closely and the
     # outputs within the chained-quantisation tolerance.
     layers = [_block_case(mmf, 40 + l, 256, 704) for l in range(2)]
     x = _to(synth.activations(41 + b, (b, 256)))
