@@ -25,7 +25,7 @@
 namespace mmf {
 namespace dec {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxRows = 8;            // token rows per launch
 constexpr int kStageRows = 2;          // input rows staged in shared memory up to this count
@@ -114,75 +114,103 @@ __device__ __forceinline__ void sm8(const float* p, float (&o)[8]) {
   o[4] = y.x; o[5] = y.y; o[6] = y.z; o[7] = y.w;
 }
 
-// The kernel runs once per SM for a few microseconds, so its instructions are fetched cold:
-// the code is kept compact (runtime loops over rows, gains and matrices; per-row statistics in
-// shared memory) rather than unrolled.
+// The residual, read through L2 (it was written by an earlier launch on other SMs).
+__device__ __forceinline__ float res_as_float(const void* base, int64_t idx, mmf_dtype dt) {
+  if (dt == MMF_F32) return __ldcg(reinterpret_cast<const float*>(base) + idx);
+  const unsigned short u = __ldcg(reinterpret_cast<const unsigned short*>(base) + idx);
+  return __uint_as_float((uint32_t)u << 16);
+}
+
+// Shared-memory pieces of one CTA for one projection group: the weight rows (requested before the
+// phase, possibly during the previous one), the gains, u, the staged input rows, the codes, the
+// factors and scratch, and the two barriers with the parity each completes next.
+struct Bufs {
+  uint32_t* wsm;
+  float* gains;
+  float* us;
+  uint8_t* xsm;
+  int8_t* qs;
+  float* deqs;
+  float* red;
+  uint64_t* bar_in;   // input rows + gains
+  uint64_t* bar_w;    // weight rows
+  uint32_t par_in, par_w;
+};
+
+// Thread 0: request this CTA's weight rows of the group (channels cta * chan_per_cta ...).
+__device__ __forceinline__ void dec_issue_weights(const Args& a, uint32_t* wsm, uint64_t* bar_w, int cta) {
+  const int c0 = cta * a.chan_per_cta;
+  int nc = a.nout - c0 < a.chan_per_cta ? a.nout - c0 : a.chan_per_cta;
+  if (nc < 0) nc = 0;  // (defensive: the grid never has a CTA past the last channel)
+  const uint32_t row_bytes = (uint32_t)a.kw * 4u;
+  mbar_arrive_expect_tx(bar_w, (uint32_t)a.nmat * (uint32_t)nc * row_bytes);
+  if (nc > 0)
+    for (int j = 0; j < a.nmat; ++j)
+      bulk_load(wsm + (size_t)j * a.chan_per_cta * a.kw, a.w[j] + ((int64_t)a.row_off[j] + c0) * a.kw,
+                (uint32_t)nc * row_bytes, bar_w);
+}
+
+// One projection group on one CTA (its weight rows already requested on B.bar_w): input rows and
+// gains into shared memory, the codes of every input row, the products and the fused epilogue.
+// Returns false when a bounded wait gave up (the copies in flight are drained first).
 template <mmf_dtype XT, int NB>
-__global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constant__ Args a) {
-  extern __shared__ __align__(128) uint8_t sm[];
-  const Smem L = smem_layout(a.mode, a.nmat, a.chan_per_cta, a.kw, a.k, a.ngain, a.b);
-  uint32_t* wsm = reinterpret_cast<uint32_t*>(sm);
-  float* gains = reinterpret_cast<float*>(sm + L.gain_off);   // [ngain (+1)][k]
-  float* us = reinterpret_cast<float*>(sm + L.u_off);
+__device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta) {
+  float* gains = B.gains;
+  float* us = B.us;
   // input rows: staged in shared memory (kO: h, then g) or read in place
   constexpr bool kStage = NB <= kStageRows;
-  uint8_t* xsm = sm + L.x_off;
+  uint8_t* xsm = B.xsm;
   const void* xs = kStage ? static_cast<const void*>(xsm) : a.x;
   const float* hs = kStage ? reinterpret_cast<const float*>(xsm) : a.h;
   const float* gs = kStage ? hs + (size_t)a.b * a.k : a.gin;
-  int8_t* qs = reinterpret_cast<int8_t*>(sm + L.q_off);
-  float* deqs = reinterpret_cast<float*>(sm + L.deq_off);   // [gain][row] a/127
-  float* red = reinterpret_cast<float*>(sm + L.red_off);    // [warp][gain][row] partials, then stats
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar_off);
-  const int c0 = blockIdx.x * a.chan_per_cta;
+  int8_t* qs = B.qs;
+  float* deqs = B.deqs;
+  float* red = B.red;
+  uint32_t* wsm = B.wsm;
+  const int c0 = cta * a.chan_per_cta;
   const int nc = a.nout - c0 < a.chan_per_cta ? a.nout - c0 : a.chan_per_cta;
-  const uint32_t row_bytes = (uint32_t)a.kw * 4u;
   const uint32_t gbytes = (uint32_t)a.k * 4u;
   const bool has_gw = a.mode == kO && a.gnorm_w != nullptr;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int ng = a.ngain;
 
-  // 1. this CTA's weight rows and the norm gains into shared memory (absent gains are ones)
+  // 1. the input rows and their norm gains into shared memory (absent gains are ones)
   if (threadIdx.x == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
-    mbar_fence_init();
     const uint32_t xbytes = kStage ? (uint32_t)a.b * (uint32_t)a.k * (a.mode == kO ? 4u : (XT == MMF_F32 ? 4u : 2u)) : 0u;
     uint32_t tx = (a.mode == kO ? 2u : 1u) * xbytes;
     for (int j = 0; j < ng; ++j) tx += a.gain[j] ? gbytes : 0u;
     if (has_gw) tx += gbytes;
-    mbar_arrive_expect_tx(&bar[0], tx);
+    mbar_arrive_expect_tx(B.bar_in, tx);
     if (kStage && a.mode == kO) {
-      bulk_load(xsm, a.h, xbytes, &bar[0]);
-      bulk_load(xsm + xbytes, a.gin, xbytes, &bar[0]);
+      bulk_load(xsm, a.h, xbytes, B.bar_in);
+      bulk_load(xsm + xbytes, a.gin, xbytes, B.bar_in);
     } else if (kStage) {
-      bulk_load(xsm, a.x, xbytes, &bar[0]);
+      bulk_load(xsm, a.x, xbytes, B.bar_in);
     }
     for (int j = 0; j < ng; ++j)
-      if (a.gain[j]) bulk_load(gains + (size_t)j * a.k, a.gain[j], gbytes, &bar[0]);
-    if (has_gw) bulk_load(gains + (size_t)ng * a.k, a.gnorm_w, gbytes, &bar[0]);
-    mbar_arrive_expect_tx(&bar[1], (uint32_t)a.nmat * (uint32_t)nc * row_bytes);
-    for (int j = 0; j < a.nmat; ++j)
-      bulk_load(wsm + (size_t)j * a.chan_per_cta * a.kw, a.w[j] + ((int64_t)a.row_off[j] + c0) * a.kw,
-                (uint32_t)nc * row_bytes, &bar[1]);
+      if (a.gain[j]) bulk_load(gains + (size_t)j * a.k, a.gain[j], gbytes, B.bar_in);
+    if (has_gw) bulk_load(gains + (size_t)ng * a.k, a.gnorm_w, gbytes, B.bar_in);
   }
   for (int j = 0; j < ng + (a.mode == kO ? 1 : 0); ++j) {
     const bool absent = j < ng ? a.gain[j] == nullptr : !has_gw;
     if (absent)
       for (int t = threadIdx.x; t < a.k; t += kThreads) gains[(size_t)j * a.k + t] = 1.0f;
   }
-  // (a timed-out wait drains both copies before the CTA leaves: shared memory must outlive them)
+  // (the decision is CTA-uniform, so every thread takes the same barriers afterwards; a
+  //  timed-out wait drains both copies before the CTA leaves: shared memory must outlive them)
   volatile int abort_flag = 0;
-  auto wait_or_leave = [&](int i) {
-    if (mbar_wait_bounded(&bar[i], 0u, a.wait_limit_us, &abort_flag)) return true;
-    for (int q = 0; q < 2; ++q) {
-      const int64_t t0 = clock64();
-      while (!mbar_try_wait(&bar[q], 0u) && clock64() - t0 < 1000000ll * kCyclesPerUs) {
-      }
+  auto wait_or_leave = [&](uint64_t* bar, uint32_t par) {
+    const bool mine = mbar_wait_bounded(bar, par, a.wait_limit_us, &abort_flag);
+    if (!__syncthreads_or(mine ? 0 : 1)) return true;
+    const int64_t t0 = clock64();
+    while (!mbar_try_wait(B.bar_in, B.par_in) && clock64() - t0 < 1000000ll * kCyclesPerUs) {
+    }
+    const int64_t t1 = clock64();
+    while (!mbar_try_wait(B.bar_w, B.par_w) && clock64() - t1 < 1000000ll * kCyclesPerUs) {
     }
     return false;
   };
-  if (!wait_or_leave(0)) return;
+  if (!wait_or_leave(B.bar_in, B.par_in)) return false;
 
   // 2. prologue: the codes of every input row (the same in every CTA). The row loops run over
   //    the compile-time count NB inside the chunk loops, so the loads of all rows are in flight
@@ -301,15 +329,18 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
   }
   __syncthreads();
 
-  if (!wait_or_leave(1)) return;
+  if (!wait_or_leave(B.bar_w, B.par_w)) return false;
 
-  // 3. each warp forms kCpw output channels at once: lanes stride over 32-code (8-byte) pieces
-  //    of the channels' weight rows, load the codes of the NB token rows for a piece once and
-  //    dp4a them against all kCpw rows (NB = b is a compile-time count, so no work is issued for
-  //    absent rows); lane r keeps the totals of token row r
+  // 3. each half-warp forms kCpw output channels at once (two channel groups per warp): its 16
+  //    lanes stride over 32-code (8-byte) pieces of the channels' weight rows, load the codes of
+  //    the NB token rows for a piece once and dp4a them against all kCpw rows (NB = b is a
+  //    compile-time count, so no work is issued for absent rows); lane r of the half keeps the
+  //    totals of token row r. Both halves run the same trip counts, so the shuffles stay uniform.
   constexpr int kCpw = NB >= 4 ? 4 : 1;
   const int npc = a.kw >> 1;              // 8-byte pieces per weight row
-  for (int cg = warp * kCpw; cg < nc; cg += kWarps * kCpw) {
+  const int hw = lane >> 4, hl = lane & 15;
+  for (int cb = warp * 2 * kCpw; cb < nc; cb += kWarps * 2 * kCpw) {
+    const int cg = cb + hw * kCpw;        // this half-warp's first channel
     int tot0[kCpw], tot1[kCpw], tot2[kCpw];
     for (int m = 0; m < a.nmat; ++m) {
       const int gsel = ng == 3 ? m : 0;
@@ -320,7 +351,7 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
         for (int r = 0; r < NB; ++r) acc[c][r] = 0;
       const uint2* wrow = reinterpret_cast<const uint2*>(wsm + ((size_t)m * a.chan_per_cta + cg) * a.kw);
       const int8_t* qg = qs + (size_t)gsel * NB * kq;
-      for (int pc = lane; pc < npc; pc += 32) {
+      for (int pc = hl; pc < npc; pc += 16) {
         const int8_t* qc = qg + (pc >> 1) * 16 + (pc & 1) * 2 * (kq >> 2);  // 64-code chunk, piece pair
         uint4 av[NB][2];
 #pragma unroll
@@ -353,8 +384,8 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
         for (int r = 0; r < NB; ++r) {
           int s = acc[c][r];
 #pragma unroll
-          for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-          if (lane == r) mine = s;
+          for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+          if (hl == r) mine = s;
         }
         if (m == 0) tot0[c] = mine;
         else if (m == 1) tot1[c] = mine;
@@ -363,8 +394,8 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
     }
 #pragma unroll
     for (int cc = 0; cc < kCpw; ++cc) {
-      if (cg + cc >= nc || lane >= a.b) continue;
-      const int r = lane;
+      if (cg + cc >= nc || hl >= a.b) continue;
+      const int r = hl;
       const int64_t o = (int64_t)r * a.nout + c0 + cg + cc;
       const int t0 = tot0[cc], t1 = a.nmat > 1 ? tot1[cc] : 0, t2 = a.nmat > 2 ? tot2[cc] : 0;
       auto zof = [&](int m, int tot) {
@@ -384,10 +415,41 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
       } else if (a.mode == kGate) {
         store_from_float(a.y, o, a.ydt, siluf_(zof(0, t0)) * zof(1, t1));
       } else {
-        store_from_float(a.y, o, a.ydt, zof(0, t0) + load_as_float(a.res, o, a.ydt));
+        store_from_float(a.y, o, a.ydt, zof(0, t0) + res_as_float(a.res, o, a.ydt));
       }
     }
   }
+  return true;
+}
+
+// One projection group per launch. The kernel runs once per SM for a few microseconds, so its
+// instructions are fetched cold: the code is kept compact (runtime loops over gains and
+// matrices; per-row statistics in shared memory) rather than unrolled.
+template <mmf_dtype XT, int NB>
+__global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constant__ Args a) {
+  extern __shared__ __align__(128) uint8_t sm[];
+  const Smem L = smem_layout(a.mode, a.nmat, a.chan_per_cta, a.kw, a.k, a.ngain, a.b);
+  Bufs B;
+  B.wsm = reinterpret_cast<uint32_t*>(sm);
+  B.gains = reinterpret_cast<float*>(sm + L.gain_off);
+  B.us = reinterpret_cast<float*>(sm + L.u_off);
+  B.xsm = sm + L.x_off;
+  B.qs = reinterpret_cast<int8_t*>(sm + L.q_off);
+  B.deqs = reinterpret_cast<float*>(sm + L.deq_off);
+  B.red = reinterpret_cast<float*>(sm + L.red_off);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar_off);
+  B.bar_in = &bar[0];
+  B.bar_w = &bar[1];
+  B.par_in = 0u;
+  B.par_w = 0u;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    mbar_fence_init();
+    dec_issue_weights(a, B.wsm, B.bar_w, blockIdx.x);
+  }
+  __syncthreads();
+  dec_phase<XT, NB>(a, B, blockIdx.x);
 }
 
 }  // namespace dec

@@ -1000,6 +1000,17 @@ mmf_status run_block_decode(const mmf_block_weights* w, const void* x, mmf_dtype
   return launch_dec(a, di, st);
 }
 
+// The fused decode paths bulk-copy the norm gains: every gain vector must start on 16 bytes.
+bool gains_aligned(const mmf_block_weights* layers, int32_t n_layers) {
+  for (int l = 0; l < n_layers; ++l) {
+    const float* g[7] = {layers[l].nw_i, layers[l].nw_f, layers[l].nw_g, layers[l].nw_o,
+                         layers[l].nw_gate, layers[l].nw_down, layers[l].gnorm_w};
+    for (const float* p : g)
+      if (p && (reinterpret_cast<uintptr_t>(p) & 15u)) return false;
+  }
+  return true;
+}
+
 mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
                            mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
                            size_t ws_bytes, mmf_stream_t stream) {
@@ -1023,7 +1034,8 @@ mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, co
   uint8_t* pp = reinterpret_cast<uint8_t*>(ws) + W.bytes;
   void* buf[2] = {pp, pp + align256((size_t)b * d * 4)};
   const void* cur = x;
-  const bool fused = decode_fused(b, d, inner) && al16(x);  // the input rows are bulk-copied
+  // the input rows and the gains are bulk-copied
+  const bool fused = decode_fused(b, d, inner) && al16(x) && gains_aligned(layers, n_layers);
   for (int l = 0; l < n_layers; ++l) {
     void* out = (l == n_layers - 1) ? y : buf[l & 1];
     float* st_l = state + (int64_t)l * b * d;

@@ -474,6 +474,33 @@ def test_decode_fused_matches_unfused(mmf, b):
     assert rel < 1e-3, rel
 
 
+def test_decode_wait_cap_ends_and_recovers(mmf):
+    # with a 1 us cap on every in-kernel wait the fused decode's waits for its bulk copies run
+    # out: every launch must still end (the CTA drains its copies and leaves as a whole), report
+    # MMF_ERR_TIMEOUT (or, if no wait ran out, be right), and leave the context usable for the
+    # next step at the default cap
+    layers = [_block_case(mmf, 70 + l, 256, 704) for l in range(2)]
+    blocks = [c[2] for c in layers]
+    x = _to(synth.activations(71, (1, 256)))
+    state0 = _to(synth.activations(72, (2, 1, 256)) * 0.5)
+    y_ref, st_ref = O.decode_step(_np(x).astype(np.float64), [c[1] for c in layers], _np(state0).astype(np.float64))
+    st = state0.clone()
+    mmf.set_wait_limit(1)
+    try:
+        y = mmf.decode_step(blocks, x, st)
+        status = mmf.sync_status(DEV)
+    finally:
+        mmf.set_wait_limit(0)
+    assert status in (mmf.MMF_OK, mmf.MMF_ERR_TIMEOUT)
+    if status == mmf.MMF_OK:
+        assert np.linalg.norm(_np(y) - y_ref) / np.linalg.norm(y_ref) < 1e-3
+    st = state0.clone()
+    y = mmf.decode_step(blocks, x, st)
+    _ok(mmf)
+    assert np.linalg.norm(_np(y) - y_ref) / np.linalg.norm(y_ref) < 1e-3
+    np.testing.assert_allclose(_np(st)[0], st_ref[0], rtol=RTOL32, atol=ATOL32)
+
+
 def test_embed_gather(mmf):
     table = synth.embedding(50, 1000, 256)
     ids = synth.token_ids(51, (3, 17), vocab=1000)
