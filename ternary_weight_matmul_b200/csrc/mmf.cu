@@ -529,7 +529,7 @@ mmf_status check_ternary(const mmf_ternary* w, int32_t n, int32_t k, const char*
 struct BlockWs {
   int8_t* q3;  // [3][m][ldq_d]
   float* deq;  // [6][m]
-  void* z;     // [m][3d]
+  void* z;     // [3][m][d]: the i, f, g planes
   void* h;     // [m][d]
   int8_t* qo;  // [m][ldq_d]
   void* x1;    // [m][d]
@@ -622,22 +622,25 @@ mmf_status run_block(const mmf_block_weights* w, const void* x, mmf_dtype dt, in
   GemmArgs g;
   memset(&g, 0, sizeof(g));
   g.m = m; g.k = d; g.kw = row_words(d); g.ldq = ldq_d; g.ydt = dt; g.nseg = 3;
-  g.seg[0] = make_seg(W.q3, deq, w->i, W.z, 3 * d, 0, nullptr, 0, nullptr, 0);
-  g.seg[1] = make_seg(W.q3 + m * ldq_d, deq + m, w->f, W.z, 3 * d, d, nullptr, 0, nullptr, 0);
-  g.seg[2] = make_seg(W.q3 + 2 * m * ldq_d, deq + 2 * m, w->g, W.z, 3 * d, 2 * d, nullptr, 0, nullptr, 0);
+  // z is three planes [i | f | g] of [m][d], so the scan and g_norm read contiguous rows
+  uint8_t* zp = reinterpret_cast<uint8_t*>(W.z);
+  const size_t plane = (size_t)m * d * es;
+  g.seg[0] = make_seg(W.q3, deq, w->i, zp, d, 0, nullptr, 0, nullptr, 0);
+  g.seg[1] = make_seg(W.q3 + m * ldq_d, deq + m, w->f, zp + plane, d, 0, nullptr, 0, nullptr, 0);
+  g.seg[2] = make_seg(W.q3 + 2 * m * ldq_d, deq + 2 * m, w->g, zp + 2 * plane, d, 0, nullptr, 0, nullptr, 0);
   MMF_TRY(launch_gemm(g, di, st));
   // 3. HGRN scan with gates
   ScanArgs sa;
   memset(&sa, 0, sizeof(sa));
-  sa.zf = reinterpret_cast<const uint8_t*>(W.z) + d * es;
-  sa.zi = W.z;
-  sa.zdt = dt; sa.zstride = 3 * d; sa.b = b; sa.t = t; sa.d = d;
+  sa.zf = zp + plane;
+  sa.zi = zp;
+  sa.zdt = dt; sa.zstride = d; sa.b = b; sa.t = t; sa.d = d;
   sa.h0 = h0; sa.h = W.h; sa.hdt = dt; sa.h_last = h_last;
   MMF_TRY(launch_scan(sa, W.scan, st));
   // 4. g_norm (RMSNorm(h) * gnorm_w * SiLU(g)) fused with o_proj's RMSNorm + quant
   memset(&nq, 0, sizeof(nq));
   nq.x = W.h; nq.ldx = d; nq.xdt = dt;
-  nq.g = reinterpret_cast<const uint8_t*>(W.z) + 2 * d * es; nq.ldg = 3 * d; nq.gdt = dt;
+  nq.g = zp + 2 * plane; nq.ldg = d; nq.gdt = dt;
   nq.gw = w->gnorm_w; nq.m = m; nq.k = d; nq.eps = w->eps; nq.ngain = 1; nq.gain[0] = w->nw_o;
   nq.q[0] = W.qo; nq.deq[0] = deq + 3 * m; nq.ldq = ldq_d;
   MMF_TRY(launch_norm_quant(nq, kRowGnorm, st));
@@ -896,7 +899,9 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
   };
   MMF_TRY(copy2d(taps->q_ifg, d, W.q3, row_q(d), d, 3 * m));
   MMF_TRY(copy2d(taps->deq_ifg, 3 * m * 4, W.deq, 3 * m * 4, 3 * m * 4, 1));
-  MMF_TRY(copy2d(taps->z, 3 * d * es, W.z, 3 * d * es, 3 * d * es, m));
+  for (int p = 0; p < 3; ++p)  // the [i | f | g] planes into the [m][3d] tap
+    MMF_TRY(copy2d(taps->z ? reinterpret_cast<uint8_t*>(taps->z) + p * d * es : nullptr, 3 * d * es,
+                   reinterpret_cast<const uint8_t*>(W.z) + p * (size_t)m * d * es, d * es, d * es, m));
   MMF_TRY(copy2d(taps->h, d * es, W.h, d * es, d * es, m));
   MMF_TRY(copy2d(taps->q_o, d, W.qo, row_q(d), d, m));
   MMF_TRY(copy2d(taps->deq_o, m * 4, W.deq + 3 * m, m * 4, m * 4, 1));
