@@ -63,7 +63,7 @@ struct Args {
 // Shared-memory layout of one CTA: weight rows, norm gains (ngain vectors of k floats; kO also
 // the g_norm gain), the g_norm output u (kO only, [b][k] float32), the codes, factors, scratch.
 struct Smem {
-  size_t w_bytes, gain_off, u_off, x_off, q_off, q_bytes, deq_off, red_off, bar_off, total;
+  size_t w_bytes, gain_off, u_off, x_off, q_off, q_bytes, deq_off, red_off, tot_off, bar_off, total;
 };
 __host__ __device__ inline Smem smem_layout(int mode, int nmat, int chan_per_cta, int kw, int k, int ngain, int b) {
   Smem s;
@@ -80,7 +80,8 @@ __host__ __device__ inline Smem smem_layout(int mode, int nmat, int chan_per_cta
   s.q_bytes = (size_t)ngain * b * kw * 16;   // codes of the padded K, [gain][row][piece][chunk]
   s.deq_off = (s.q_off + s.q_bytes + 15) & ~(size_t)15;
   s.red_off = s.deq_off + 3 * kMaxRows * sizeof(float);
-  s.bar_off = (s.red_off + (kWarps * 3 + 4) * kMaxRows * sizeof(float) + 7) & ~(size_t)7;
+  s.tot_off = s.red_off + (kWarps * 3 + 4) * kMaxRows * sizeof(float);  // [matrix][channel][row] int32
+  s.bar_off = (s.tot_off + (size_t)nmat * chan_per_cta * b * 4 + 7) & ~(size_t)7;
   s.total = s.bar_off + 16;   // two mbarriers: gains, weights
   return s;
 }
@@ -132,6 +133,7 @@ struct Bufs {
   int8_t* qs;
   float* deqs;
   float* red;
+  int32_t* tots;      // [matrix][channel][row] integer products of the CTA's channels
   uint64_t* bar_in;   // input rows + gains
   uint64_t* bar_w;    // weight rows
   uint32_t par_in, par_w;
@@ -331,92 +333,97 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
 
   if (!wait_or_leave(B.bar_w, B.par_w)) return false;
 
-  // 3. each half-warp forms kCpw output channels at once (two channel groups per warp): its 16
-  //    lanes stride over 32-code (8-byte) pieces of the channels' weight rows, load the codes of
-  //    the NB token rows for a piece once and dp4a them against all kCpw rows (NB = b is a
-  //    compile-time count, so no work is issued for absent rows); lane r of the half keeps the
-  //    totals of token row r. Both halves run the same trip counts, so the shuffles stay uniform.
+  // 3. products: work items are (group of kCpw channels, matrix) pairs, spread evenly over the
+  //    half-warps; a half-warp's 16 lanes stride over 32-code (8-byte) pieces of the channels'
+  //    weight rows, load the codes of the NB token rows for a piece once and dp4a them against
+  //    all kCpw rows in two independent chains (NB = b is a compile-time count, so no work is
+  //    issued for absent rows). Lane r of the half leaves the total of token row r in shared
+  //    memory. Both halves of a warp run the same trip counts, so the shuffles stay uniform.
   constexpr int kCpw = NB >= 4 ? 4 : 1;
   const int npc = a.kw >> 1;              // 8-byte pieces per weight row
   const int hw = lane >> 4, hl = lane & 15;
-  for (int cb = warp * 2 * kCpw; cb < nc; cb += kWarps * 2 * kCpw) {
-    const int cg = cb + hw * kCpw;        // this half-warp's first channel
-    int tot0[kCpw], tot1[kCpw], tot2[kCpw];
-    for (int m = 0; m < a.nmat; ++m) {
-      const int gsel = ng == 3 ? m : 0;
-      int acc[kCpw][NB];
+  const int ngroups = (nc + kCpw - 1) / kCpw;
+  const int nitems = ngroups * a.nmat;
+  int32_t* tots = B.tots;                 // [matrix][channel][row]
+  for (int ib = warp * 2; ib < nitems; ib += kWarps * 2) {
+    const int it = ib + hw;
+    const bool live = it < nitems;
+    const int m = live ? it / ngroups : 0;
+    const int cg = live ? (it - m * ngroups) * kCpw : nc;  // first channel of the group
+    const int gsel = ng == 3 ? m : 0;
+    int acc0[kCpw][NB], acc1[kCpw][NB];
+    auto& acc1r = NB <= 2 ? acc1 : acc0;  // two chains only where the registers allow it
 #pragma unroll
-      for (int c = 0; c < kCpw; ++c)
+    for (int c = 0; c < kCpw; ++c)
 #pragma unroll
-        for (int r = 0; r < NB; ++r) acc[c][r] = 0;
-      const uint2* wrow = reinterpret_cast<const uint2*>(wsm + ((size_t)m * a.chan_per_cta + cg) * a.kw);
-      const int8_t* qg = qs + (size_t)gsel * NB * kq;
-      for (int pc = hl; pc < npc; pc += 16) {
-        const int8_t* qc = qg + (pc >> 1) * 16 + (pc & 1) * 2 * (kq >> 2);  // 64-code chunk, piece pair
-        uint4 av[NB][2];
+      for (int r = 0; r < NB; ++r) acc0[c][r] = acc1[c][r] = 0;
+    const uint2* wrow = reinterpret_cast<const uint2*>(wsm + ((size_t)m * a.chan_per_cta + cg) * a.kw);
+    const int8_t* qg = qs + (size_t)gsel * NB * kq;
+#pragma unroll 2
+    for (int pc = hl; pc < npc; pc += 16) {
+      const int8_t* qc = qg + (pc >> 1) * 16 + (pc & 1) * 2 * (kq >> 2);  // 64-code chunk, piece pair
+      uint4 av[NB][2];
 #pragma unroll
-        for (int r = 0; r < NB; ++r)
+      for (int r = 0; r < NB; ++r)
 #pragma unroll
-          for (int pp = 0; pp < 2; ++pp) av[r][pp] = *reinterpret_cast<const uint4*>(qc + (size_t)r * kq + pp * (kq >> 2));
+        for (int pp = 0; pp < 2; ++pp) av[r][pp] = *reinterpret_cast<const uint4*>(qc + (size_t)r * kq + pp * (kq >> 2));
 #pragma unroll
-        for (int c = 0; c < kCpw; ++c) {
-          if (cg + c < nc) {
-            const uint2 wv = wrow[(size_t)c * (a.kw >> 1) + pc];
-            uint32_t e[8];
-            expand_word(wv.x, e + 0);
-            expand_word(wv.y, e + 4);
+      for (int c = 0; c < kCpw; ++c) {
+        if (cg + c < nc) {
+          const uint2 wv = wrow[(size_t)c * (a.kw >> 1) + pc];
+          uint32_t e[8];
+          expand_word(wv.x, e + 0);
+          expand_word(wv.y, e + 4);
 #pragma unroll
-            for (int r = 0; r < NB; ++r)
-#pragma unroll
-              for (int pp = 0; pp < 2; ++pp) {
-                acc[c][r] = __dp4a((int)e[4 * pp + 0], (int)av[r][pp].x, acc[c][r]);
-                acc[c][r] = __dp4a((int)e[4 * pp + 1], (int)av[r][pp].y, acc[c][r]);
-                acc[c][r] = __dp4a((int)e[4 * pp + 2], (int)av[r][pp].z, acc[c][r]);
-                acc[c][r] = __dp4a((int)e[4 * pp + 3], (int)av[r][pp].w, acc[c][r]);
-              }
+          for (int r = 0; r < NB; ++r) {
+            acc0[c][r] = __dp4a((int)e[0], (int)av[r][0].x, acc0[c][r]);
+            acc1r[c][r] = __dp4a((int)e[4], (int)av[r][1].x, acc1r[c][r]);
+            acc0[c][r] = __dp4a((int)e[1], (int)av[r][0].y, acc0[c][r]);
+            acc1r[c][r] = __dp4a((int)e[5], (int)av[r][1].y, acc1r[c][r]);
+            acc0[c][r] = __dp4a((int)e[2], (int)av[r][0].z, acc0[c][r]);
+            acc1r[c][r] = __dp4a((int)e[6], (int)av[r][1].z, acc1r[c][r]);
+            acc0[c][r] = __dp4a((int)e[3], (int)av[r][0].w, acc0[c][r]);
+            acc1r[c][r] = __dp4a((int)e[7], (int)av[r][1].w, acc1r[c][r]);
           }
         }
       }
-#pragma unroll
-      for (int c = 0; c < kCpw; ++c) {
-        int mine = 0;
-#pragma unroll
-        for (int r = 0; r < NB; ++r) {
-          int s = acc[c][r];
-#pragma unroll
-          for (int o = 8; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-          if (hl == r) mine = s;
-        }
-        if (m == 0) tot0[c] = mine;
-        else if (m == 1) tot1[c] = mine;
-        else tot2[c] = mine;
-      }
     }
 #pragma unroll
-    for (int cc = 0; cc < kCpw; ++cc) {
-      if (cg + cc >= nc || hl >= a.b) continue;
-      const int r = hl;
-      const int64_t o = (int64_t)r * a.nout + c0 + cg + cc;
-      const int t0 = tot0[cc], t1 = a.nmat > 1 ? tot1[cc] : 0, t2 = a.nmat > 2 ? tot2[cc] : 0;
-      auto zof = [&](int m, int tot) {
-        const int gsel = ng == 3 ? m : 0;
-        return __fmul_rn((float)tot, __fmul_rn(deqs[gsel * kMaxRows + r], a.sw[m][0]));
-      };
-      if (a.mode == kIFG) {
-        // f = sigmoid(zf), i = SiLU(zi) * (1 - f), h = f * h_prev + i
-        const float zi = zof(0, t0), zf = zof(1, t1), zg = zof(2, t2);
-        float f, omf;
-        hgrn_forget(zf, f, omf);
-        const float iv = siluf_(zi) * omf;
-        const float hv = f * a.state[o] + iv;
-        a.state[o] = hv;
-        reinterpret_cast<float*>(a.y)[o] = hv;
-        a.g_out[o] = zg;
-      } else if (a.mode == kGate) {
-        store_from_float(a.y, o, a.ydt, siluf_(zof(0, t0)) * zof(1, t1));
-      } else {
-        store_from_float(a.y, o, a.ydt, zof(0, t0) + res_as_float(a.res, o, a.ydt));
+    for (int c = 0; c < kCpw; ++c) {
+#pragma unroll
+      for (int r = 0; r < NB; ++r) {
+        int sum = NB <= 2 ? acc0[c][r] + acc1[c][r] : acc0[c][r];
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (hl == r && cg + c < nc) tots[((size_t)m * a.chan_per_cta + cg + c) * NB + r] = sum;
       }
+    }
+  }
+  __syncthreads();
+
+  // 4. epilogue: one thread per (channel, token row) of the CTA
+  for (int idx = threadIdx.x; idx < nc * NB; idx += kThreads) {
+    const int cl = idx / NB, r = idx - cl * NB;
+    const int64_t o = (int64_t)r * a.nout + c0 + cl;
+    auto zof = [&](int m) {
+      const int gsel = ng == 3 ? m : 0;
+      const int tot = tots[((size_t)m * a.chan_per_cta + cl) * NB + r];
+      return __fmul_rn((float)tot, __fmul_rn(deqs[gsel * kMaxRows + r], a.sw[m][0]));
+    };
+    if (a.mode == kIFG) {
+      // f = sigmoid(zf), i = SiLU(zi) * (1 - f), h = f * h_prev + i
+      const float zi = zof(0), zf = zof(1), zg = zof(2);
+      float f, omf;
+      hgrn_forget(zf, f, omf);
+      const float iv = siluf_(zi) * omf;
+      const float hv = f * a.state[o] + iv;
+      a.state[o] = hv;
+      reinterpret_cast<float*>(a.y)[o] = hv;
+      a.g_out[o] = zg;
+    } else if (a.mode == kGate) {
+      store_from_float(a.y, o, a.ydt, siluf_(zof(0)) * zof(1));
+    } else {
+      store_from_float(a.y, o, a.ydt, zof(0) + res_as_float(a.res, o, a.ydt));
     }
   }
   return true;
@@ -437,6 +444,7 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
   B.qs = reinterpret_cast<int8_t*>(sm + L.q_off);
   B.deqs = reinterpret_cast<float*>(sm + L.deq_off);
   B.red = reinterpret_cast<float*>(sm + L.red_off);
+  B.tots = reinterpret_cast<int32_t*>(sm + L.tot_off);
   uint64_t* bar = reinterpret_cast<uint64_t*>(sm + L.bar_off);
   B.bar_in = &bar[0];
   B.bar_w = &bar[1];
