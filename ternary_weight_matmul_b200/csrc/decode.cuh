@@ -29,6 +29,9 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kMaxRows = 8;            // token rows per launch
 constexpr int kStageRows = 2;          // input rows staged in shared memory up to this count
+// per-row reduction scratch: two rounds of sum-of-squares partials [round][warp][row], maxima
+// partials [warp][gain][row]
+constexpr int kRedFloats = (2 * kWarps + 3 * kWarps) * kMaxRows;
 constexpr int kMaxSmem = 200 * 1024;   // dynamic shared memory budget per CTA
 
 enum Mode : int32_t { kIFG = 0, kO = 1, kGate = 2, kDown = 3 };
@@ -80,7 +83,7 @@ __host__ __device__ inline Smem smem_layout(int mode, int nmat, int chan_per_cta
   s.q_bytes = (size_t)ngain * b * kw * 16;   // codes of the padded K, [gain][row][piece][chunk]
   s.deq_off = (s.q_off + s.q_bytes + 15) & ~(size_t)15;
   s.red_off = s.deq_off + 3 * kMaxRows * sizeof(float);
-  s.tot_off = s.red_off + (kWarps * 3 + 4) * kMaxRows * sizeof(float);  // [matrix][channel][row] int32
+  s.tot_off = s.red_off + kRedFloats * sizeof(float);  // [matrix][channel][row] int32
   s.bar_off = (s.tot_off + (size_t)nmat * chan_per_cta * b * 4 + 7) & ~(size_t)7;
   s.total = s.bar_off + 16;   // two mbarriers: gains, weights
   return s;
@@ -219,8 +222,11 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
   //    together (the rows are read in place when there are more than kStageRows of them).
   const int nck = a.k >> 3;
   const int kq = a.kw * 16;
-  float* rfs = red + kWarps * 3 * kMaxRows;          // [row] 1/rms
-  float* sxs = rfs + kMaxRows;                       // [gain][row] 127/a
+  // every round leaves one partial per warp and row; after one barrier each thread combines
+  // them itself (same order everywhere), so no second barrier is needed
+  float* ssp = red;                                   // [round][warp][row]
+  float* amp = red + 2 * kWarps * kMaxRows;           // [warp][gain][row]
+  float rf[NB], rfh[NB];
   // 2a. mean squares of every row (kO: of h, then u = h / rms(h) * w_g * SiLU(g) into shared
   //     memory and its mean squares)
   for (int pass = 0; pass < (a.mode == kO ? 2 : 1); ++pass) {
@@ -236,9 +242,8 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
           float v[8], g[8];
           load8<MMF_F32>(hs, (int64_t)r * a.k + 8 * c, v);
           load8<MMF_F32>(gs, (int64_t)r * a.k + 8 * c, g);
-          const float rfh = rfs[r];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(__fmul_rn(v[e], rfh), w8[e]) * siluf_(g[e]);
+          for (int e = 0; e < 8; ++e) v[e] = __fmul_rn(__fmul_rn(v[e], rfh[r]), w8[e]) * siluf_(g[e]);
           float* up = us + (size_t)r * a.k + 8 * c;
           *reinterpret_cast<float4*>(up) = make_float4(v[0], v[1], v[2], v[3]);
           *reinterpret_cast<float4*>(up + 4) = make_float4(v[4], v[5], v[6], v[7]);
@@ -258,18 +263,20 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
           for (int e = 0; e < 8; ++e) ss[r] = fmaf(v[r][e], v[r][e], ss[r]);
       }
     }
+    float* part = ssp + pass * kWarps * kMaxRows;
 #pragma unroll
     for (int r = 0; r < NB; ++r) {
       const float t = warp_sum(ss[r]);
-      if (lane == 0) red[warp * kMaxRows + r] = t;
+      if (lane == 0) part[warp * kMaxRows + r] = t;
     }
     __syncthreads();
-    if (threadIdx.x < NB) {
+#pragma unroll
+    for (int r = 0; r < NB; ++r) {
       float t = 0.0f;
-      for (int w = 0; w < kWarps; ++w) t += red[w * kMaxRows + threadIdx.x];
-      rfs[threadIdx.x] = nq_rinv(t, a.k, a.eps);
+      for (int w = 0; w < kWarps; ++w) t += part[w * kMaxRows + r];
+      if (a.mode == kO && pass == 0) rfh[r] = nq_rinv(t, a.k, a.eps);
+      else rf[r] = nq_rinv(t, a.k, a.eps);
     }
-    __syncthreads();
   }
   // 2b. maxima of |r| = |v / rms * gain| per (gain, row)
   for (int j = 0; j < ng; ++j) {
@@ -284,29 +291,32 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
       for (int r = 0; r < NB; ++r) in8<XT>(a, us, xs, r, 8 * c, v[r]);
 #pragma unroll
       for (int r = 0; r < NB; ++r) {
-        const float rf = rfs[r];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) am[r] = fmaxf(am[r], fabsf(__fmul_rn(__fmul_rn(v[r][e], rf), gg[e])));
+        for (int e = 0; e < 8; ++e) am[r] = fmaxf(am[r], fabsf(__fmul_rn(__fmul_rn(v[r][e], rf[r]), gg[e])));
       }
     }
 #pragma unroll
     for (int r = 0; r < NB; ++r) {
       const float t = warp_max(am[r]);
-      if (lane == 0) red[(warp * 3 + j) * kMaxRows + r] = t;
+      if (lane == 0) amp[(warp * 3 + j) * kMaxRows + r] = t;
     }
   }
   __syncthreads();
-  if (threadIdx.x < ng * kMaxRows) {
-    const int j = threadIdx.x / kMaxRows, r = threadIdx.x - j * kMaxRows;
-    if (r < NB) {
+  // 127/a per (gain, row), formed by every thread; the factors a/127 for the epilogue
+  float sx[3][NB];
+  for (int j = 0; j < ng; ++j) {
+#pragma unroll
+    for (int r = 0; r < NB; ++r) {
       float t = 0.0f;
-      for (int w = 0; w < kWarps; ++w) t = fmaxf(t, red[(w * 3 + j) * kMaxRows + r]);
+      for (int w = 0; w < kWarps; ++w) t = fmaxf(t, amp[(w * 3 + j) * kMaxRows + r]);
       t = fmaxf(t, 1e-5f);
-      sxs[j * kMaxRows + r] = q127_over(t);
-      deqs[j * kMaxRows + r] = over_127(t);
+      const float q = q127_over(t);
+      if (j == 0) sx[0][r] = q;
+      else if (j == 1) sx[1][r] = q;
+      else sx[2][r] = q;
+      if (threadIdx.x == 0) deqs[j * kMaxRows + r] = over_127(t);
     }
   }
-  __syncthreads();
   // 2c. codes, piece-major: code k of (gain j, row r) at
   //     qs + (j * b + r) * kq + ((k % 64) / 16) * (kq / 4) + (k / 64) * 16 + k % 16
   for (int j = 0; j < ng; ++j) {
@@ -319,10 +329,10 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
       const int kk = 8 * c;
 #pragma unroll
       for (int r = 0; r < NB; ++r) {
-        const float rf = rfs[r], sx = sxs[j * kMaxRows + r];
+        const float sxr = j == 0 ? sx[0][r] : (j == 1 ? sx[1][r] : sx[2][r]);
         uint32_t q[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(__fmul_rn(__fmul_rn(v[r][e], rf), gg[e]), sx));
+        for (int e = 0; e < 8; ++e) q[e] = q8_bits(__fmul_rn(__fmul_rn(__fmul_rn(v[r][e], rf[r]), gg[e]), sxr));
         int8_t* qrow = qs + (size_t)(j * NB + r) * kq;
         *reinterpret_cast<uint2*>(qrow + ((kk & 63) >> 4) * (kq >> 2) + (kk >> 6) * 16 + (kk & 15)) =
             make_uint2(pack4_lo_bytes(q[0], q[1], q[2], q[3]), pack4_lo_bytes(q[4], q[5], q[6], q[7]));
