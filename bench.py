@@ -35,7 +35,7 @@ WORKLOADS = {
 # DRAM traffic of one ternary_gemm_tc_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum,
 # averaged over the 96 GEMM launches of one step) from an ncu capture of this bench's own workload;
 # valid only while the kernel source is the one captured (SHA-256 prefix), else reported as null.
-GEMM_TRAFFIC = {"prefill-370M": dict(bytes=78.6e6, algorithmic=115.2e6, sha256="555ae3df1a5fa605",
+GEMM_TRAFFIC = {"prefill-370M": dict(bytes=78.3e6, algorithmic=115.2e6, sha256="1e40409415946f20",
                                      profile="profiles/ternary_gemm_tc_kernel_prefill-370M_traffic.md")}
 DECODE = dict(name="decode-2.7B", d=2560, inner=7040, layers=32, vocab=32000, prompt=512, batches=(1, 8, 64))
 

@@ -59,7 +59,11 @@ constexpr int EPI_BUF_BYTES = EPI_CHUNK * BM * 4;
 constexpr int SMEM_W_OFF = STAGES * ACT_BYTES;
 constexpr int SMEM_EPI_OFF = SMEM_W_OFF + STAGES * W_BYTES;
 constexpr int SMEM_DQ_OFF = SMEM_EPI_OFF + 2 * EPI_BUF_BYTES;  // per-token (a/127)*s, 2 x BN floats
-constexpr int SMEM_BAR_OFF = SMEM_DQ_OFF + 2 * BN * 4;
+// residual tile (bf16 outputs), prefetched by the epilogue threads with cp.async before they wait
+// for the tile's accumulators: [chunk][piece][8 values], each thread reading back what it copied
+constexpr int RES_BYTES = BN * BM * 2;
+constexpr int SMEM_RES_OFF = SMEM_DQ_OFF + 2 * BN * 4;
+constexpr int SMEM_BAR_OFF = SMEM_RES_OFF + RES_BYTES;
 constexpr int NUM_BARS = 3 * STAGES + 5;
 constexpr int SMEM_BYTES = SMEM_BAR_OFF + NUM_BARS * 8 + 16 + 1024;  // + alignment slack
 static_assert(SMEM_BYTES <= 227 * 1024, "shared memory budget");
@@ -116,6 +120,15 @@ __device__ __forceinline__ void decode_tile(const Params& P, int tile, int& seg,
   const int local = tile - P.tile_start[seg];
   nt = local / P.m_tiles;
   mt = local - nt * P.m_tiles;
+}
+
+// Whether the epilogue prefetches tile (segment S, weight tile nt)'s residual into shared memory:
+// bf16 output, a residual, a full 128-row non-GLU tile, 16-byte aligned row segments.
+template <mmf_dtype YT>
+__device__ __forceinline__ bool res_prefetch(const GemmSeg* S, int nt) {
+  if (YT != MMF_BF16 || !S->res || S->glu || S->n - nt * BM < BM) return false;
+  const uintptr_t base = reinterpret_cast<uintptr_t>(S->res) + (uintptr_t)(S->rescol + nt * BM) * 2u;
+  return ((base | (uintptr_t)(S->ldres * 2)) & 15u) == 0;
 }
 
 // Wait without an abort check, used only while draining after an abort. Its own cap (1 s) does
@@ -187,6 +200,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
   uint32_t* w_s = reinterpret_cast<uint32_t*>(smem + SMEM_W_OFF);
   int32_t* epi_s = reinterpret_cast<int32_t*>(smem + SMEM_EPI_OFF);
   float* dq_s = reinterpret_cast<float*>(smem + SMEM_DQ_OFF);
+  OutT* res_s = reinterpret_cast<OutT*>(smem + SMEM_RES_OFF);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + SMEM_BAR_OFF);
   uint64_t* full = bars;                   // TMA -> expanders      (count 1 + tx bytes)
   uint64_t* afull = bars + STAGES;         // expanders -> MMA      (count 4)
@@ -354,13 +368,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     uint32_t tl = 0, chunk_ctr = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tl) {
       const uint32_t b = tl & 1u;
+      int seg, nt, mt;
+      decode_tile(P, tile, seg, nt, mt);
+      {
+        // bf16 residual of the whole tile into shared memory while the tile's MMAs may still
+        // run: one cp.async group per chunk, each thread copying exactly the pieces it adds in
+        // phase 2
+        const GemmSeg* S = seg == 0 ? &P.g.seg[0] : (seg == 1 ? &P.g.seg[1] : &P.g.seg[2]);
+        cp_async_wait<0>();  // (nothing in flight from the previous tile may land on the new copies)
+        if (res_prefetch<YT>(S, nt)) {
+          const OutT* rsrc = reinterpret_cast<const OutT*>(S->res) + S->rescol + nt * BM;
+#pragma unroll
+          for (int ci = 0; ci < BN / EPI_CHUNK; ++ci) {
+#pragma unroll
+            for (int itp = 0; itp < 2; ++itp) {
+              const int pidx = etid + itp * EPI_THREADS;
+              const int64_t m = (int64_t)mt * BN + ci * EPI_CHUNK + (pidx >> 4);
+              if (m < P.g.m) cp_async16(res_s + (ci * 2 * EPI_THREADS + pidx) * 8, rsrc + m * S->ldres + (pidx & 15) * 8);
+            }
+            cp_async_commit();
+          }
+        }
+      }
       const bool got = mbar_wait_bounded(&accfull[b], (tl >> 1) & 1u, limit, abort_flag);
       // The eight epilogue warps meet at named barrier 1 below, so they must agree on leaving:
       // if any of them gave up waiting, all of them leave (barrier reduction over 256 threads).
       if (epi_any(!got)) break;
       tc_fence_after();
-      int seg, nt, mt;
-      decode_tile(P, tile, seg, nt, mt);
       const GemmSeg* S = seg == 0 ? &P.g.seg[0] : (seg == 1 ? &P.g.seg[1] : &P.g.seg[2]);
       const bool glu = S->glu != 0;
       const int n0 = nt * (glu ? GLU_ROWS : BM);           // first output column of the tile
@@ -387,6 +421,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
           ((reinterpret_cast<uintptr_t>(y) | (uintptr_t)(ldy * sizeof(OutT))) & 15u) == 0 &&
           (!res || ((reinterpret_cast<uintptr_t>(res) | (uintptr_t)(ldres * sizeof(OutT))) & 15u) == 0) &&
           (!accp || ((reinterpret_cast<uintptr_t>(accp) | (uintptr_t)(ldacc * 4)) & 15u) == 0);
+      const bool res_pf = res_prefetch<YT>(S, nt);  // the residual is in shared memory
       for (int c0 = 0; c0 < BN; c0 += EPI_CHUNK, ++chunk_ctr) {
         int32_t* buf = epi_s + (chunk_ctr & 1u) * (EPI_CHUNK * BM);
         uint32_t v[16];
@@ -443,7 +478,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
                 *reinterpret_cast<int4*>(accp + m * ldacc + r8) = a0;
                 *reinterpret_cast<int4*>(accp + m * ldacc + r8 + 4) = a1;
               }
-              if (res) add8<YT>(res + m * ldres + r8, z);
+              if (res_pf) {
+                // this chunk's cp.async group (and the earlier ones) have landed
+                const int ci = c0 / EPI_CHUNK;
+                if (ci == 0) cp_async_wait<3>();
+                else if (ci == 1) cp_async_wait<2>();
+                else if (ci == 2) cp_async_wait<1>();
+                else cp_async_wait<0>();
+                add8<YT>(res_s + (ci * 2 * EPI_THREADS + pidx) * 8, z);
+              } else if (res) {
+                add8<YT>(res + m * ldres + r8, z);
+              }
               if (act != kActNone) {
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
@@ -481,6 +526,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     }
   }
 
+  cp_async_wait<0>();  // epilogue threads: residual copies of an abandoned tile
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();

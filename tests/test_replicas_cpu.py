@@ -58,12 +58,21 @@ def test_single_rank_needs_no_process_group():
     assert bench.replicas_throughput(1000, 1, 2.0) == pytest.approx(500000.0)
 
 
-def test_gemm_traffic_tracks_kernel_source():
-    """The traffic figure is reported only for the captured workload and kernel source, and the
-    profile it cites is committed."""
+def test_gemm_traffic_tracks_kernel_source(monkeypatch):
+    """The traffic figure is reported only for the captured workload and only while the kernel
+    source matches the captured one; the profile it cites is committed."""
+    import hashlib
+
     import bench
 
-    t = bench.gemm_traffic("prefill-370M")
-    assert t is not None and 0 < t < bench.GEMM_TRAFFIC["prefill-370M"]["algorithmic"]
+    src = os.path.join(bench.ROOT, "ternary_weight_matmul_b200", "csrc", "gemm_tc.cuh")
+    with open(src, "rb") as fh:
+        cur = hashlib.sha256(fh.read()).hexdigest()[:16]
+    entry = dict(bench.GEMM_TRAFFIC["prefill-370M"])
+    assert os.path.exists(os.path.join(bench.ROOT, entry["profile"]))
+    assert 0 < entry["bytes"] < entry["algorithmic"]
+    monkeypatch.setitem(bench.GEMM_TRAFFIC, "prefill-370M", dict(entry, sha256=cur))
+    assert bench.gemm_traffic("prefill-370M") == entry["bytes"]
+    monkeypatch.setitem(bench.GEMM_TRAFFIC, "prefill-370M", dict(entry, sha256="0" * 16))
+    assert bench.gemm_traffic("prefill-370M") is None
     assert bench.gemm_traffic("prefill-1.3B") is None
-    assert os.path.exists(os.path.join(bench.ROOT, bench.GEMM_TRAFFIC["prefill-370M"]["profile"]))
