@@ -198,7 +198,11 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
  *   x       [b][d] dtype: hidden state of the current token entering layer 0.
  *   state   [n_layers][b][d] float32, read and overwritten in place.
  *   y       [b][d] dtype: hidden state leaving the last layer (may not alias x).
- *   ws >= mmf_workspace_bytes(MMF_OP_DECODE, b, d, inner, n_layers). */
+ *   ws >= mmf_workspace_bytes(MMF_OP_DECODE, b, d, inner, n_layers).
+ * With b in {1, 2, 4, 8} rows (CUDA-core engine or MMF_GEMM_AUTO), d and inner multiples of 8
+ * and 16-byte aligned norm gains, each block runs as four fused launches (norm + quantisation
+ * of the input inside each, the products, and the gates / recurrence step / residual / GLU in
+ * their epilogues); otherwise as the block path with t = 1. Same arithmetic either way. */
 mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
                            mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
                            size_t ws_bytes, mmf_stream_t stream);
