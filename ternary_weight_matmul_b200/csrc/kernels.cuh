@@ -254,17 +254,6 @@ __device__ __forceinline__ void load8(const void* base, int64_t idx, float (&o)[
     o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
   }
 }
-__device__ __forceinline__ void load8_gain(const float* g, int64_t idx, float (&o)[8]) {
-  if (!g) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) o[e] = 1.0f;
-    return;
-  }
-  const float4 a = __ldg(reinterpret_cast<const float4*>(g + idx));
-  const float4 b = __ldg(reinterpret_cast<const float4*>(g + idx + 4));
-  o[0] = a.x; o[1] = a.y; o[2] = a.z; o[3] = a.w;
-  o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
-}
 // Bits of x + 1.5 * 2^23 for |x| <= 127.5: the addition (where the float32 spacing is exactly 1)
 // rounds half to even, and the low byte of the result is the int8 code rint(x) itself
 // (0x4B400000 has a zero low byte). No clamp is needed: x = r * fl(127 / a) with a the maximum of
