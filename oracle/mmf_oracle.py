@@ -328,6 +328,25 @@ def stack_forward(ids: np.ndarray, table: np.ndarray, layers: list[dict],
 
 
 # ----------------------------------------------------------------------------------------------
+# language-model head and greedy generation
+# ----------------------------------------------------------------------------------------------
+def lm_head_logits(x: np.ndarray, norm_w: np.ndarray | None, table: np.ndarray,
+                   eps: float = EPS_NORM) -> np.ndarray:
+    """Logits of the tied language-model head: the final RMSNorm of the last block's output,
+    then the product with the embedding table [vocab, d], which the input embedding and the
+    head share (hysenlabs.com, install and model-table sections: 32000-word vocabulary, the
+    causal-LM generation example). x [..., d] -> [..., vocab] float64."""
+    r = rmsnorm(np.asarray(x, dtype=np.float64), norm_w, eps)
+    return r @ np.asarray(table, dtype=np.float64).T
+
+
+def greedy_next(logits: np.ndarray) -> np.ndarray:
+    """Greedy decoding: the index of the largest logit of each row, the lowest index among
+    equal maxima (argmax returns the first)."""
+    return np.argmax(np.asarray(logits), axis=-1).astype(np.int64)
+
+
+# ----------------------------------------------------------------------------------------------
 # model-size bookkeeping
 # ----------------------------------------------------------------------------------------------
 def block_param_count(d: int, inner: int) -> int:

@@ -354,3 +354,41 @@ def test_parameter_counts_match_size_names(shape, name_params):
     assert O.block_param_count(shape.d, shape.inner) == per_block
     # both readings (tied or separate head) land within 10% of the published size name
     assert abs(tied / name_params - 1) < 0.10 and abs(untied / name_params - 1) < 0.10
+
+
+# ---------------------------------------------------------------------------------------------
+# language-model head and greedy generation
+# ---------------------------------------------------------------------------------------------
+def test_lm_head_hand_worked():
+    # x = [3, 4]: mean square 12.5, r = x / sqrt(12.5 + eps); rows [1,0], [0,1], [1,1], [-1,0]
+    x = np.array([[3.0, 4.0]])
+    table = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0], [-1.0, 0.0]])
+    logits = O.lm_head_logits(x, None, table)
+    r = np.array([3.0, 4.0]) / np.sqrt(12.5 + 1e-8)
+    np.testing.assert_allclose(logits[0], [r[0], r[1], r[0] + r[1], -r[0]], rtol=1e-12)
+    np.testing.assert_allclose(logits[0], [0.848528137, 1.131370850, 1.979898987, -0.848528137], rtol=1e-8)
+    assert O.greedy_next(logits)[0] == 2
+
+
+def test_lm_head_identity_table_and_gain():
+    # one-hot table rows: the logits are the normalised input itself, times the gain
+    rng = np.random.default_rng(3)
+    x = rng.standard_normal((3, 16))
+    w = 1.0 + 0.1 * rng.standard_normal(16)
+    logits = O.lm_head_logits(x, w, np.eye(16))
+    rms = np.sqrt((x ** 2).mean(axis=1, keepdims=True) + 1e-8)
+    np.testing.assert_allclose(logits, x / rms * w, rtol=1e-12)
+    assert np.array_equal(O.greedy_next(logits), np.argmax(x / rms * w, axis=1))
+
+
+def test_lm_head_scale_invariance_and_ties():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((2, 32))
+    table = rng.standard_normal((50, 32))
+    a = O.lm_head_logits(x, None, table)
+    b = O.lm_head_logits(1000.0 * x, None, table)   # RMSNorm removes a positive scale
+    np.testing.assert_allclose(a, b, rtol=1e-7)
+    # duplicated best row: the lowest index wins
+    best = int(O.greedy_next(a[:1])[0])
+    table2 = np.concatenate([table[:best], table[best:best + 1], table[best:]], axis=0)
+    assert int(O.greedy_next(O.lm_head_logits(x[:1], None, table2))[0]) == best
