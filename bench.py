@@ -244,11 +244,13 @@ def build_model(wl, device, seed=1234):
 
 
 def run_decode(args, device, hbm_peak):
-    """Decode-step throughput of the 2.7B-shape stack for each batch size: prompt prefill through
-    mmf_stack_fwd (untimed, gives every layer's recurrent state), then `--decode-steps` steps of
-    embedding gather + mmf_decode_step replayed from a CUDA graph (one graph per step, captured
-    after warm-up), timed with CUDA events on the replay stream. Token ids are pre-drawn (the LM
-    head is outside the block stack). HBM roofline: every step streams all packed weights."""
+    """Greedy autoregressive decode throughput of the 2.7B-shape stack for each batch size: prompt
+    prefill through mmf_stack_fwd (untimed; gives every layer's recurrent state and, through the
+    final norm and the tied head, the first generated token), then `--decode-steps` generated
+    tokens, each step = embedding gather of the current ids + mmf_decode_step + final RMSNorm,
+    tied head and argmax (mmf_lm_head_argmax writes the next ids in place), replayed from a CUDA
+    graph (captured after warm-up) and timed with CUDA events on the replay stream. HBM roofline:
+    every step streams all packed weights and the bf16 head table (once per 8 sequences)."""
     import torch
 
     import ternary_weight_matmul_b200 as mmf
@@ -260,28 +262,31 @@ def run_decode(args, device, hbm_peak):
         for p in blk.packed.values():
             weight_bytes += p.codes.numel() * 4 + 4
         weight_bytes += sum(t.numel() * 4 for t in blk.norms.values())
+    fnorm = torch.ones(dw["d"], dtype=torch.float32, device=device)  # final RMSNorm gain
+    head_bytes = table.numel() * table.element_size()
     out = {"workload": dw["name"], "layers": dw["layers"], "hidden": dw["d"], "inner": dw["inner"],
            "prompt": dw["prompt"], "steps": args.decode_steps, "unit": "tokens/s",
-           "bytes_per_step_weights": weight_bytes, "batches": {}}
+           "generation": "greedy (final RMSNorm + tied head + argmax on the GPU, ids fed back)",
+           "bytes_per_step_weights": weight_bytes, "bytes_head_table": head_bytes, "batches": {}}
     for B in dw["batches"]:
         g = torch.Generator(device="cpu")
         g.manual_seed(99 + B)
         prompt = torch.randint(0, dw["vocab"], (B, dw["prompt"]), generator=g, dtype=torch.int32).to(device)
-        steps_ids = torch.randint(0, dw["vocab"], (args.decode_steps + 8, B), generator=g, dtype=torch.int32).to(device)
-        _, state = mmf.stack_fwd(blocks, prompt, table, want_state=True)
+        yp, state = mmf.stack_fwd(blocks, prompt, table, want_state=True)
         x = torch.empty(B, dw["d"], dtype=torch.bfloat16, device=device)
         y = torch.empty_like(x)
-        cur = torch.zeros(B, dtype=torch.int32, device=device)
+        cur = torch.empty(B, dtype=torch.int32, device=device)
+        mmf.lm_head_argmax(yp[:, -1, :].contiguous(), fnorm, table, ids_out=cur)  # first generated token
         s = torch.cuda.Stream(device)
 
         def step():
             xx = mmf.embed_gather(cur, table)
             x.copy_(xx)
             mmf.decode_step(blocks, x, state, out=y)
+            mmf.lm_head_argmax(y, fnorm, table, ids_out=cur)
 
         with torch.cuda.stream(s):
             for i in range(3):
-                cur.copy_(steps_ids[i])
                 step()
         torch.cuda.synchronize(device)
         graph = torch.cuda.CUDAGraph()
@@ -290,12 +295,10 @@ def run_decode(args, device, hbm_peak):
         ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         with torch.cuda.stream(s):
             for i in range(3):
-                cur.copy_(steps_ids[3 + i])
                 graph.replay()
             torch.cuda.synchronize(device)
             ev0.record(s)
             for i in range(args.decode_steps):
-                cur.copy_(steps_ids[i % steps_ids.shape[0]])
                 graph.replay()
             ev1.record(s)
         torch.cuda.synchronize(device)
@@ -303,9 +306,12 @@ def run_decode(args, device, hbm_peak):
         if st != 0:
             raise RuntimeError(f"device status {st} in decode")
         ms = ev0.elapsed_time(ev1) / args.decode_steps
-        gbs = weight_bytes / (ms / 1e3) / 1e9
-        out["batches"][str(B)] = {"value": B / (ms / 1e3), "ms_per_step": ms, "GB/s_weights": gbs,
-                                  "frac_hbm": gbs / hbm_peak}
+        step_bytes = weight_bytes + head_bytes * ((B + 7) // 8)
+        gbs = step_bytes / (ms / 1e3) / 1e9
+        ids_end = cur.cpu()
+        assert int(ids_end.min()) >= 0 and int(ids_end.max()) < dw["vocab"]
+        out["batches"][str(B)] = {"value": B / (ms / 1e3), "ms_per_step": ms, "bytes_per_step": step_bytes,
+                                  "GB/s": gbs, "frac_hbm": gbs / hbm_peak}
         del graph
     del blocks, table
     torch.cuda.empty_cache()

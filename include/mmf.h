@@ -74,7 +74,8 @@ typedef enum {
   MMF_OP_BLOCK = 2,     /* mmf_block_fwd: m = b*t tokens, d, inner                */
   MMF_OP_DECODE = 3,    /* mmf_decode_step: m = b, d, inner                       */
   MMF_OP_STACK = 4,     /* mmf_stack_fwd: m = b*t tokens, d, inner, n_layers      */
-  MMF_OP_SCAN = 5       /* mmf_hgrn_scan: m = b*t tokens, d channels              */
+  MMF_OP_SCAN = 5,      /* mmf_hgrn_scan: m = b*t tokens, d channels              */
+  MMF_OP_HEAD = 6       /* mmf_lm_head_argmax: inner = vocabulary size            */
 } mmf_op;
 
 /* A packed ternary weight (device pointers). */
@@ -213,6 +214,24 @@ mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, co
  *   table [vocab][d] dtype; out [m][d] dtype. */
 mmf_status mmf_embed_gather(const int32_t* ids, int64_t m, const void* table, mmf_dtype dtype,
                             int32_t vocab, int32_t d, void* out, mmf_stream_t stream);
+
+/* Tied language-model head and greedy next token, for generation: only the last position of
+ * each sequence is needed, so x holds one row per sequence.
+ *   logits[r][v] = sum_k RMSNorm(x[r])[k] * table[v][k], RMSNorm(x) = x / sqrt(mean(x^2) + eps)
+ *   * norm_w (the final norm after the last block); ids[r] = argmax_v logits[r][v], the lowest
+ *   index among equal maxima (greedy decoding).
+ * Readings: the head shares the embedding table (tied); the final norm has the blocks' eps
+ * (hysenlabs.com "MatMul-Free LM", install and model-table sections: 32000-word vocabulary,
+ * causal-LM generation example).
+ *   x       [b][d] x_dtype, 16-byte aligned; d a multiple of 8, d * 4 <= 200 KB.
+ *   norm_w  [d] float32 or NULL (= 1).
+ *   table   [vocab][d] table_dtype (the embedding table), 16-byte aligned.
+ *   ids     [b] int32 out.   logits [b][vocab] float32 out or NULL (a test tap).
+ *   ws >= mmf_workspace_bytes(MMF_OP_HEAD, 0, 0, vocab, 0).
+ * Float32 accumulation over bf16 / float32 table rows; the table is streamed once per 8 rows. */
+mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32_t d, const float* norm_w,
+                              float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
+                              int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
 /* Prefill forward of an HGRNBitModel block stack (hysenlabs.com: HGRNBitModel = embedding + a
  * stack of HGRNBitBlock): embedding gather, then the n_layers blocks in order.

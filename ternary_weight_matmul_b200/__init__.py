@@ -21,13 +21,13 @@ LIB_PATH = os.path.join(_HERE, "libmmf.so")
 
 MMF_OK, MMF_ERR_INVALID_ARG, MMF_ERR_UNSUPPORTED, MMF_ERR_WORKSPACE, MMF_ERR_CUDA, MMF_ERR_TIMEOUT = range(6)
 MMF_F32, MMF_BF16 = 0, 1
-MMF_OP_PACK, MMF_OP_BITLINEAR, MMF_OP_BLOCK, MMF_OP_DECODE, MMF_OP_STACK, MMF_OP_SCAN = range(6)
+MMF_OP_PACK, MMF_OP_BITLINEAR, MMF_OP_BLOCK, MMF_OP_DECODE, MMF_OP_STACK, MMF_OP_SCAN, MMF_OP_HEAD = range(7)
 MMF_GEMM_AUTO, MMF_GEMM_TENSOR, MMF_GEMM_SIMT = range(3)
 
 EXPORTED = (
     "mmf_packed_row_words", "mmf_packed_words", "mmf_workspace_bytes", "mmf_pack_ternary",
     "mmf_bitlinear_fwd", "mmf_hgrn_scan", "mmf_block_fwd", "mmf_block_fwd_taps", "mmf_decode_step",
-    "mmf_embed_gather",
+    "mmf_embed_gather", "mmf_lm_head_argmax",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
     "mmf_bitlinear_fwd_noalloc",
@@ -90,6 +90,8 @@ def lib() -> ctypes.CDLL:
         "mmf_decode_step": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, ctypes.c_int, i32, vp, vp,
                                            vp, sz, st]),
         "mmf_embed_gather": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, i32, i32, vp, st]),
+        "mmf_lm_head_argmax": (ctypes.c_int, [vp, ctypes.c_int, i32, i32, vp, ctypes.c_float, vp, ctypes.c_int, i32,
+                                              vp, vp, vp, sz, st]),
         "mmf_stack_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, i32, i64, vp, i32,
                                          ctypes.c_int, vp, vp, vp, sz, st]),
         "mmf_sync_status": (ctypes.c_int, [st]),
@@ -343,6 +345,24 @@ def embed_gather(ids: torch.Tensor, table: torch.Tensor) -> torch.Tensor:
     _check(lib().mmf_embed_gather(ids.data_ptr(), ids.numel(), table.data_ptr(), _dt(table.dtype), table.shape[0],
                                   table.shape[1], out.data_ptr(), _stream(table.device)), "mmf_embed_gather")
     return out
+
+
+def lm_head_argmax(x: torch.Tensor, norm_w: torch.Tensor | None, table: torch.Tensor, eps: float = 1e-8,
+                   want_logits: bool = False, ids_out: torch.Tensor | None = None):
+    """mmf_lm_head_argmax: greedy next token ids [b] (int32) of x [b, d] through the final
+    RMSNorm and the tied head `table` [vocab, d]; with want_logits also the logits [b, vocab]."""
+    _dev(x)
+    _dev(table)
+    b, d = x.shape
+    vocab = table.shape[0]
+    ids = ids_out if ids_out is not None else torch.empty(b, dtype=torch.int32, device=x.device)
+    logits = torch.empty(b, vocab, dtype=torch.float32, device=x.device) if want_logits else None
+    ws = workspace(MMF_OP_HEAD, 0, 0, vocab, 0, x.device)
+    _check(lib().mmf_lm_head_argmax(x.data_ptr(), _dt(x.dtype), b, d, norm_w.data_ptr() if norm_w is not None else None,
+                                    eps, table.data_ptr(), _dt(table.dtype), vocab, ids.data_ptr(),
+                                    logits.data_ptr() if logits is not None else None, ws.data_ptr(), ws.numel(),
+                                    _stream(x.device)), "mmf_lm_head_argmax")
+    return (ids, logits) if want_logits else ids
 
 
 def stack_fwd(blocks: list[Block], ids: torch.Tensor, table: torch.Tensor, want_state: bool = False,

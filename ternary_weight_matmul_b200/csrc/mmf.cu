@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "gemm_tc.cuh"
+#include "head.cuh"
 #include "kernels.cuh"
 
 using namespace mmf;
@@ -711,6 +712,36 @@ mmf_status noalloc_scratch(void** out) {
   return MMF_OK;
 }
 
+// Partial maxima of the head: one (logit, index) per CTA and token row of a pass; CTAs cover at
+// least head::kMinRowsPerCta vocabulary rows each.
+size_t head_ws_bytes(int32_t vocab) {
+  const size_t parts = (size_t)((vocab + head::kMinRowsPerCta - 1) / head::kMinRowsPerCta);
+  return 2 * align256(parts * head::kRows * 4);
+}
+
+template <mmf_dtype XT, mmf_dtype TT>
+void head_launch(head::Args a, int nb, int nparts, int32_t* ids, cudaStream_t st) {
+  const size_t smem = (size_t)nb * a.d * 4;
+#define MMF_HEAD(NB_) launch_k(head::head_logits_kernel<XT, TT, NB_>, dim3((unsigned)nparts), dim3(head::kThreads), smem, st, a)
+  if (nb == 8) MMF_HEAD(8);
+  else if (nb == 4) MMF_HEAD(4);
+  else if (nb == 2) MMF_HEAD(2);
+  else MMF_HEAD(1);
+#undef MMF_HEAD
+  launch_k(head::head_argmax_kernel, dim3((unsigned)((nb + head::kWarps - 1) / head::kWarps)), dim3(head::kThreads), 0, st,
+           (const float*)a.pmax, (const int32_t*)a.pidx, nparts, nb, ids);
+}
+
+template <mmf_dtype XT, mmf_dtype TT>
+cudaError_t head_attrs() {
+  const int smem = 200 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
+}
+
 }  // namespace
 
 // =============================================================================================
@@ -724,6 +755,7 @@ size_t mmf_packed_words(int32_t n, int32_t k) {
   return (n <= 0 || k <= 0) ? 0 : (size_t)n * (size_t)row_words(k);
 }
 
+
 size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32_t n_layers) {
   if (m < 0 || d < 0 || inner < 0) return 0;
   switch (op) {
@@ -735,6 +767,8 @@ size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32
       return block_ws(nullptr, m, d, inner, MMF_F32).bytes;
     case MMF_OP_SCAN:
       return d > 0 ? scan_ws_bytes(m, d) : 0;
+    case MMF_OP_HEAD:
+      return inner > 0 ? head_ws_bytes(inner) : 0;
     case MMF_OP_DECODE:
     case MMF_OP_STACK:
       return block_ws(nullptr, m, d, inner, MMF_F32).bytes + 2 * align256((size_t)m * d * 4);
@@ -1065,6 +1099,68 @@ mmf_status mmf_embed_gather(const int32_t* ids, int64_t m, const void* table, mm
     launch_k(embed_gather_kernel, dim3((unsigned)m), dim3(128), 0, reinterpret_cast<cudaStream_t>(stream), ids, m, table, dtype, vocab, d, out);
   }
   return check_launch("embed_gather_kernel");
+}
+
+// ---------------------------------------------------------------------------------------------
+// language-model head + greedy next token
+// ---------------------------------------------------------------------------------------------
+mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32_t d, const float* norm_w,
+                              float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
+                              int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream) {
+  MMF_CHECK_ARG(b >= 0 && d > 0 && vocab > 0, "head: bad sizes");
+  MMF_CHECK_ARG(d % 8 == 0, "head: d = %d is not a multiple of 8", d);
+  MMF_CHECK_ARG(valid_dtype(x_dtype) && valid_dtype(table_dtype), "head: bad dtype");
+  MMF_CHECK_ARG((size_t)d * 4 <= 200 * 1024, "head: d = %d too large", d);
+  if (b == 0) return MMF_OK;
+  MMF_CHECK_ARG(x && table && ids, "head: null pointer");
+  MMF_CHECK_ARG(aligned16(x) && aligned16(table) && (!norm_w || aligned16(norm_w)),
+                "head: x / table / norm_w not 16-byte aligned");
+  MMF_TRY(check_ws(ws, ws_bytes, head_ws_bytes(vocab)));
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  {
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+      cudaError_t e = head_attrs<MMF_F32, MMF_F32>();
+      if (e == cudaSuccess) e = head_attrs<MMF_F32, MMF_BF16>();
+      if (e == cudaSuccess) e = head_attrs<MMF_BF16, MMF_F32>();
+      if (e == cudaSuccess) e = head_attrs<MMF_BF16, MMF_BF16>();
+      attr_err = e;
+    });
+    if (attr_err != cudaSuccess) return fail(MMF_ERR_CUDA, "head attributes: %s", cudaGetErrorString(attr_err));
+  }
+  // vocabulary split: a few CTAs per SM, at least kMinRowsPerCta rows each
+  int nparts = std::min((vocab + head::kMinRowsPerCta - 1) / head::kMinRowsPerCta, di->sms * 4);
+  const int rows_per_cta = (vocab + nparts - 1) / nparts;
+  nparts = (vocab + rows_per_cta - 1) / rows_per_cta;
+  const size_t parr = align256((size_t)((vocab + head::kMinRowsPerCta - 1) / head::kMinRowsPerCta) * head::kRows * 4);
+  head::Args a;
+  memset(&a, 0, sizeof(a));
+  a.xdt = x_dtype; a.d = d; a.norm_w = norm_w; a.eps = eps; a.table = table; a.tdt = table_dtype;
+  a.vocab = vocab; a.rows_per_cta = rows_per_cta; a.ld_logits = vocab;
+  a.pmax = reinterpret_cast<float*>(ws);
+  a.pidx = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) + parr);
+  const size_t xes = dsize(x_dtype);
+  LaunchScope ls(MMF_KERNEL_OTHER, (double)vocab * d * dsize(table_dtype) * ((b + head::kRows - 1) / head::kRows) +
+                 (double)b * vocab * (logits ? 4.0 : 0.0), st);
+  // passes of 8, 4, 2, 1 rows (each kernel handles exactly its row count)
+  for (int r0 = 0; r0 < b;) {
+    const int left = b - r0;
+    const int nb = left >= 8 ? 8 : left >= 4 ? 4 : left >= 2 ? 2 : 1;
+    a.x = reinterpret_cast<const uint8_t*>(x) + (size_t)r0 * d * xes;
+    a.b = nb;
+    a.logits = logits ? logits + (int64_t)r0 * vocab : nullptr;
+    if (x_dtype == MMF_F32 && table_dtype == MMF_F32) head_launch<MMF_F32, MMF_F32>(a, nb, nparts, ids + r0, st);
+    else if (x_dtype == MMF_F32) head_launch<MMF_F32, MMF_BF16>(a, nb, nparts, ids + r0, st);
+    else if (table_dtype == MMF_F32) head_launch<MMF_BF16, MMF_F32>(a, nb, nparts, ids + r0, st);
+    else head_launch<MMF_BF16, MMF_BF16>(a, nb, nparts, ids + r0, st);
+    r0 += nb;
+    g_launches.fetch_add(2);
+  }
+  g_launches.fetch_sub(1);  // the timing scope counted one launch itself
+  return check_launch("head kernels");
 }
 
 mmf_status mmf_stack_fwd(const mmf_block_weights* layers, int32_t n_layers, const int32_t* ids,

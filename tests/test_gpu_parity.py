@@ -501,6 +501,32 @@ def test_decode_wait_cap_ends_and_recovers(mmf):
     np.testing.assert_allclose(_np(st)[0], st_ref[0], rtol=RTOL32, atol=ATOL32)
 
 
+@pytest.mark.parametrize("b,d,vocab,xdt,tdt", [(1, 256, 1000, "f32", "f32"), (3, 256, 777, "bf16", "bf16"),
+                                                (11, 264, 1200, "f32", "bf16"), (8, 2560, 32000, "bf16", "bf16"),
+                                                (64, 2560, 32000, "bf16", "bf16")])
+def test_lm_head_argmax_parity(mmf, b, d, vocab, xdt, tdt):
+    # final RMSNorm + tied head + greedy next token against the oracle on the same (dtype-
+    # rounded) inputs: logits within 1e-4 (float32 accumulation of d products); the ids are the
+    # first argmax of the kernel's own logits, and the oracle's argmax except at near-ties
+    dts = {"f32": torch.float32, "bf16": torch.bfloat16}
+    x = _to(synth.activations(80 + b, (b, d)), dts[xdt])
+    w = synth.norm_weight(81, d, random=True)
+    table = _to(synth.embedding(82, vocab, d), dts[tdt])
+    ids, logits = mmf.lm_head_argmax(x, _to(w), table, want_logits=True)
+    ids2 = mmf.lm_head_argmax(x, _to(w), table)
+    _ok(mmf)
+    lg = logits.cpu().numpy()
+    ref = O.lm_head_logits(_np(x).astype(np.float64), w, _np(table).astype(np.float64))
+    scale = np.abs(ref).max()
+    np.testing.assert_allclose(lg, ref, rtol=1e-4, atol=1e-4 * scale)
+    got = ids.cpu().numpy().astype(np.int64)
+    assert np.array_equal(got, ids2.cpu().numpy())
+    assert np.array_equal(got, np.argmax(lg, axis=1))
+    want = O.greedy_next(ref)
+    for r in np.nonzero(got != want)[0]:
+        assert ref[r, got[r]] >= ref[r].max() - 2e-4 * scale  # a near-tie
+
+
 def test_embed_gather(mmf):
     table = synth.embedding(50, 1000, 256)
     ids = synth.token_ids(51, (3, 17), vocab=1000)
