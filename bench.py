@@ -35,7 +35,7 @@ WORKLOADS = {
 # DRAM traffic of one ternary_gemm_tc_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum,
 # averaged over the 96 GEMM launches of one step) from an ncu capture of this bench's own workload;
 # valid only while the kernel source is the one captured (SHA-256 prefix), else reported as null.
-GEMM_TRAFFIC = {"prefill-370M": dict(bytes=78.3e6, algorithmic=115.2e6, sha256="1e40409415946f20",
+GEMM_TRAFFIC = {"prefill-370M": dict(bytes=78.3e6, algorithmic=115.2e6, sha256="14a6d8df0242cadf",
                                      profile="profiles/ternary_gemm_tc_kernel_prefill-370M_traffic.md")}
 DECODE = dict(name="decode-2.7B", d=2560, inner=7040, layers=32, vocab=32000, prompt=512, batches=(1, 8, 64))
 
@@ -250,7 +250,8 @@ def run_decode(args, device, hbm_peak):
     tokens, each step = embedding gather of the current ids + mmf_decode_step + final RMSNorm,
     tied head and argmax (mmf_lm_head_argmax writes the next ids in place), replayed from a CUDA
     graph (captured after warm-up) and timed with CUDA events on the replay stream. HBM roofline:
-    every step streams all packed weights and the bf16 head table (once per 8 sequences)."""
+    every step streams all packed weights and the bf16 head table (once per pass of the head: one
+    row on the CUDA cores, up to 128 rows on the tensor cores)."""
     import torch
 
     import ternary_weight_matmul_b200 as mmf
@@ -306,7 +307,7 @@ def run_decode(args, device, hbm_peak):
         if st != 0:
             raise RuntimeError(f"device status {st} in decode")
         ms = ev0.elapsed_time(ev1) / args.decode_steps
-        step_bytes = weight_bytes + head_bytes * ((B + 7) // 8)
+        step_bytes = weight_bytes + head_bytes * ((B + 127) // 128)
         gbs = step_bytes / (ms / 1e3) / 1e9
         ids_end = cur.cpu()
         assert int(ids_end.min()) >= 0 and int(ids_end.max()) < dw["vocab"]

@@ -167,7 +167,7 @@ mmf_status mmf_block_fwd(const mmf_block_weights* w, const void* x, mmf_dtype dt
  *   x1 [m][d] dtype;  q_gate [m][d], deq_gate [m]
  *   gu [m][2I] dtype = [gate | up], written when gate_proj stores both halves;
  *   v [m][I] dtype = SiLU(gate) * up, written instead when gate_proj's epilogue forms the GLU
- *     product itself: on the tensor-core engine (more than 8 rows under MMF_GEMM_AUTO, or
+ *     product itself: on the tensor-core engine (8 or more rows under MMF_GEMM_AUTO, or
  *     MMF_GEMM_TENSOR) with I % 64 == 0
  *   q_down [m][I], deq_down [m]. */
 typedef struct {
@@ -200,7 +200,8 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
  *   state   [n_layers][b][d] float32, read and overwritten in place.
  *   y       [b][d] dtype: hidden state leaving the last layer (may not alias x).
  *   ws >= mmf_workspace_bytes(MMF_OP_DECODE, b, d, inner, n_layers).
- * With b in {1, 2, 4, 8} rows (CUDA-core engine or MMF_GEMM_AUTO), d and inner multiples of 8
+ * With b in {1, 2, 4} rows (CUDA-core engine or MMF_GEMM_AUTO) or 8 rows (CUDA-core engine
+ * only; MMF_GEMM_AUTO gives 8 rows to the tensor-core engine), d and inner multiples of 8
  * and 16-byte aligned norm gains, each block runs as four fused launches (norm + quantisation
  * of the input inside each, the products, and the gates / recurrence step / residual / GLU in
  * their epilogues); otherwise as the block path with t = 1. Same arithmetic either way. */
@@ -227,8 +228,10 @@ mmf_status mmf_embed_gather(const int32_t* ids, int64_t m, const void* table, mm
  *   norm_w  [d] float32 or NULL (= 1).
  *   table   [vocab][d] table_dtype (the embedding table), 16-byte aligned.
  *   ids     [b] int32 out.   logits [b][vocab] float32 out or NULL (a test tap).
- *   ws >= mmf_workspace_bytes(MMF_OP_HEAD, 0, 0, vocab, 0).
- * Float32 accumulation over bf16 / float32 table rows; the table is streamed once per 8 rows. */
+ *   ws >= mmf_workspace_bytes(MMF_OP_HEAD, 0, d, vocab, 0); a smaller ws is an error.
+ * bf16 table and b >= 2: tensor cores (tcgen05, bf16 operands, float32 accumulation); each
+ * normalised row enters as a bf16 pair hi + lo (16 significant bits), the table streams once per
+ * 128 rows. Otherwise CUDA cores, float32 accumulation, the table streamed once per 8 rows. */
 mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32_t d, const float* norm_w,
                               float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
                               int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream);

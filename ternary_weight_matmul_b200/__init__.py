@@ -357,7 +357,7 @@ def lm_head_argmax(x: torch.Tensor, norm_w: torch.Tensor | None, table: torch.Te
     vocab = table.shape[0]
     ids = ids_out if ids_out is not None else torch.empty(b, dtype=torch.int32, device=x.device)
     logits = torch.empty(b, vocab, dtype=torch.float32, device=x.device) if want_logits else None
-    ws = workspace(MMF_OP_HEAD, 0, 0, vocab, 0, x.device)
+    ws = workspace(MMF_OP_HEAD, 0, d, vocab, 0, x.device)
     _check(lib().mmf_lm_head_argmax(x.data_ptr(), _dt(x.dtype), b, d, norm_w.data_ptr() if norm_w is not None else None,
                                     eps, table.data_ptr(), _dt(table.dtype), vocab, ids.data_ptr(),
                                     logits.data_ptr() if logits is not None else None, ws.data_ptr(), ws.numel(),
@@ -400,7 +400,7 @@ def set_gemm_path(path: int) -> None:
 def glu_fused(m: int, inner: int) -> bool:
     """Whether a block forward on m tokens forms SiLU(gate) * up in gate_proj's epilogue (taps
     then carry ``v`` instead of ``gu``): the tensor-core engine with inner % 64 == 0."""
-    tensor = _gemm_path == MMF_GEMM_TENSOR or (_gemm_path == MMF_GEMM_AUTO and m > 8)
+    tensor = _gemm_path == MMF_GEMM_TENSOR or (_gemm_path == MMF_GEMM_AUTO and m >= 8)
     return tensor and inner % 64 == 0
 
 

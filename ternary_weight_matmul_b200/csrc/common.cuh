@@ -168,6 +168,16 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
   return true;
 }
 
+// Wait without an abort check, used only while draining after an abort. Its own cap (1 s) does
+// not follow the (possibly lowered) wait limit: copies and MMAs already issued complete within
+// microseconds, and the CTA must not release shared or tensor memory before they have.
+constexpr int64_t kDrainCycles = 1000000ll * kCyclesPerUs;
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
+  const int64_t t0 = clock64();
+  while (!mbar_try_wait(bar, parity) && clock64() - t0 < kDrainCycles) {
+  }
+}
+
 // 2-D tiled TMA load global -> shared, completion counted on `bar` (no multicast).
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t c0,
                                             int32_t c1, uint64_t* bar) {
@@ -215,6 +225,26 @@ __device__ __forceinline__ void tc_mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, u
       "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// D(tmem) (+)= A(smem) x B(smem), bf16 x bf16 -> float32 (kind::f16, both operands by descriptor).
+__device__ __forceinline__ void tc_mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                               uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled operand tile: start address
+// >> 4 (bits 0-13), leading byte offset 16 B (unused for this layout, bits 16-29), stride byte
+// offset 1024 B = 8 rows x 128 B (bits 32-45), descriptor version 1 (bits 46-47), layout type
+// SWIZZLE_128B = 2 (bits 61-63). The tile starts on a 1024-byte boundary; K steps inside the
+// 128-byte atom advance the start address.
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
+  return (uint64_t)((smem_addr & 0x3FFFFu) >> 4) | ((uint64_t)1u << 16) | ((uint64_t)64u << 32) |
+         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
 }
 
 #define MMF_R32(i) "r"(v[i])

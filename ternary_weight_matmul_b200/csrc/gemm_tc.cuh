@@ -77,15 +77,6 @@ __device__ __forceinline__ int epi_word(int r) {  // staged position of row r wi
 constexpr uint32_t IDESC = (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                            ((uint32_t)(BM >> 4) << 24);
 
-// Shared-memory matrix descriptor of a K-major, 128-byte-swizzled operand tile: start address
-// >> 4 (bits 0-13), leading byte offset 16 B (unused for this layout, bits 16-29), stride byte
-// offset 1024 B = 8 rows x 128 B (bits 32-45), descriptor version 1 (bits 46-47), layout type
-// SWIZZLE_128B = 2 (bits 61-63).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t smem_addr) {
-  return (uint64_t)((smem_addr & 0x3FFFFu) >> 4) | ((uint64_t)1u << 16) | ((uint64_t)64u << 32) |
-         ((uint64_t)1u << 46) | ((uint64_t)2u << 61);
-}
-
 // float(a) for |a| < 2^22 without a conversion instruction: a + 1.5 * 2^23 laid into the
 // mantissa of a float whose spacing is 1, minus that constant again (both steps exact).
 __device__ __forceinline__ float acc_to_float(int32_t a) {
@@ -129,16 +120,6 @@ __device__ __forceinline__ bool res_prefetch(const GemmSeg* S, int nt) {
   if (YT != MMF_BF16 || !S->res || S->glu || S->n - nt * BM < BM) return false;
   const uintptr_t base = reinterpret_cast<uintptr_t>(S->res) + (uintptr_t)(S->rescol + nt * BM) * 2u;
   return ((base | (uintptr_t)(S->ldres * 2)) & 15u) == 0;
-}
-
-// Wait without an abort check, used only while draining after an abort. Its own cap (1 s) does
-// not follow the (possibly lowered) wait limit: copies and MMAs already issued complete within
-// microseconds, and the CTA must not release shared or tensor memory before they have.
-constexpr int64_t kDrainCycles = 1000000ll * kCyclesPerUs;
-__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity) {
-  const int64_t t0 = clock64();
-  while (!mbar_try_wait(bar, parity) && clock64() - t0 < kDrainCycles) {
-  }
 }
 
 // OR of `pred` over the 256 epilogue threads (named barrier 1); every caller gets the result.

@@ -3,11 +3,16 @@
 // logits = RMSNorm(x) . E^T with E the embedding table [vocab][d] that the input embedding
 // shares, then next = argmax (lowest index among equal maxima). Only the last position of each
 // sequence is needed to generate, so this runs on a handful of token rows and streams the table
-// once per call: an HBM-bound product, done on the CUDA cores. Every CTA normalises the (up to
-// kRows) token rows into shared memory in float32; each warp then forms the logits of its
-// vocabulary rows from 16-byte table loads with float32 accumulation and keeps a running
-// (maximum, lowest index) per token row; the CTA's best per row goes to a partial array that a
-// one-warp-per-row kernel reduces to the ids.
+// once per pass: an HBM-bound product. Two forms:
+//   * CUDA cores (any table dtype, up to kRows token rows a pass): every CTA normalises the rows
+//     into shared memory in float32; each warp forms the logits of its vocabulary rows from
+//     16-byte table loads with float32 accumulation and keeps a running (maximum, lowest index)
+//     per token row.
+//   * Tensor cores (bf16 table, up to kTcRowsMax token rows a pass): a small kernel writes the
+//     normalised rows as bf16 hi / lo pairs, then tcgen05.mma.kind::f16 forms 128 vocabulary rows
+//     of logits per CTA from TMA-staged table tiles (below).
+// Either way the CTA's best per token row goes to a partial array that a one-warp-per-row kernel
+// reduces to the ids.
 #pragma once
 
 #include "common.cuh"
@@ -223,17 +228,17 @@ __global__ void __launch_bounds__(kThreads, 2) head_logits_kernel(const Args a) 
   }
 }
 
-// One warp per token row: the best of the CTAs' candidates.
+// One warp per token row: the best of the CTAs' candidates (`ld` entries per CTA).
 __global__ void __launch_bounds__(kThreads) head_argmax_kernel(const float* __restrict__ pmax,
                                                                const int32_t* __restrict__ pidx,
-                                                               int nparts, int b, int32_t* __restrict__ ids) {
+                                                               int nparts, int ld, int b, int32_t* __restrict__ ids) {
   const int r = blockIdx.x * kWarps + (threadIdx.x >> 5), lane = threadIdx.x & 31;
   if (r >= b) return;
   float bv = -INFINITY;
   int bi = 0x7fffffff;
   for (int p = lane; p < nparts; p += 32) {
-    const float v = pmax[(int64_t)p * kRows + r];
-    const int i = pidx[(int64_t)p * kRows + r];
+    const float v = pmax[(int64_t)p * ld + r];
+    const int i = pidx[(int64_t)p * ld + r];
     if (head_better(v, i, bv, bi)) { bv = v; bi = i; }
   }
 #pragma unroll
@@ -243,6 +248,236 @@ __global__ void __launch_bounds__(kThreads) head_argmax_kernel(const float* __re
     if (head_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
   }
   if (lane == 0) ids[r] = bi;
+}
+
+// ---------------------------------------------------------------------------------------------
+// tensor-core form (bf16 table)
+// ---------------------------------------------------------------------------------------------
+// logits[v][j] = sum_k E[v][k] r[j][k] is a skinny GEMM: the table is the A operand (M = 128
+// vocabulary rows per CTA, K-major), the normalised token rows the B operand, D float32 in tensor
+// memory. The MMA takes bf16 operands, so each float32 row r enters as two bf16 rows, hi = bf16(r)
+// and lo = bf16(r - hi), which together carry 16 significant bits; the two halves of D add up in
+// the epilogue to the product with r up to ~2^-17 relative, the size of float32 accumulation error
+// over d terms. One CTA = one vocabulary tile over all of K: a producer thread streams 64-wide
+// k-blocks of the table tile and of the token rows into a 4-stage ring with TMA (128-byte swizzle),
+// one thread issues four MMAs (K = 16 each) per k-block, then all four warps read D back (warp w
+// owns TMEM lanes 32w..32w+31, i.e. one vocabulary row per thread), write the logits and reduce
+// the (maximum, lowest index) per token row. Every wait is bounded.
+constexpr int kTcRowsMax = 128;   // token rows per pass: N = 2 x 128 = 256, the MMA maximum
+constexpr int kTcMinRows = 2;     // calls with fewer token rows take the CUDA-core form
+constexpr int kTcBM = 128;        // vocabulary rows per CTA (MMA M)
+constexpr int kTcBK = 64;         // bf16 per k-block: one 128-byte swizzle atom
+constexpr int kTcUK = 16;         // K per kind::f16 instruction
+constexpr int kTcStages = 4;
+constexpr int kTcThreads = 128;
+constexpr int kTcABytes = kTcBM * kTcBK * 2;   // 16 KB table tile per stage
+constexpr int kTcBars = 2 * kTcStages + 2;
+
+__host__ __device__ constexpr int tc_stage_bytes(int h) { return kTcABytes + 2 * h * kTcBK * 2; }
+__host__ __device__ constexpr int tc_smem_bytes(int h) {
+  return 1024 + kTcStages * tc_stage_bytes(h) + kTcBars * 8 + 16;
+}
+
+struct TcParams {
+  CUtensorMap tmap;     // table [vocab][d] bf16, box 64 x 128, 128-byte swizzle
+  CUtensorMap xmap;     // hi / lo rows [2h][d] bf16, box 64 x 2h, 128-byte swizzle
+  int32_t nb;           // token rows of the pass
+  int32_t h;            // hi rows at [0, h), lo rows at [h, 2h); nb <= h, h % 16 == 0
+  int32_t num_kb;       // ceil(d / 64); the tail k-block reads zeros past d on both operands
+  int32_t vocab;
+  float* logits;        // nullable [nb][ld_logits]
+  int64_t ld_logits;
+  float* pmax;          // [gridDim][kTcRowsMax]
+  int32_t* pidx;
+  uint32_t tmem_cols;   // power of two >= max(32, 2h)
+  uint32_t wait_limit_us;
+};
+
+// r = x / rms(x) * w for token row j = blockIdx.x of the pass, stored as bf16 rows hi (row j) and
+// lo (row h + j); slots j >= nb get zero rows.
+template <mmf_dtype XT>
+__global__ void __launch_bounds__(kThreads) head_pack_kernel(const void* __restrict__ x, int d,
+                                                             const float* __restrict__ norm_w, float eps,
+                                                             int nb, int h, __nv_bfloat16* __restrict__ xs) {
+  __shared__ float red[32];
+  const int j = blockIdx.x, nck = d >> 3;
+  uint4* hi = reinterpret_cast<uint4*>(xs + (size_t)j * d);
+  uint4* lo = reinterpret_cast<uint4*>(xs + (size_t)(h + j) * d);
+  if (j >= nb) {
+    for (int c = threadIdx.x; c < nck; c += kThreads) { hi[c] = make_uint4(0, 0, 0, 0); lo[c] = make_uint4(0, 0, 0, 0); }
+    return;
+  }
+  float ss = 0.0f;
+  for (int c = threadIdx.x; c < nck; c += kThreads) {
+    float v[8];
+    row8<XT>(x, (int64_t)j * d + 8 * c, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+  }
+  const float rinv = rsqrtf(__fdividef(block_sum(ss, red), (float)d) + eps);
+  for (int c = threadIdx.x; c < nck; c += kThreads) {
+    float v[8], g[8];
+    row8<XT>(x, (int64_t)j * d + 8 * c, v);
+    if (norm_w) {
+      row8<MMF_F32>(norm_w, 8 * c, g);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) g[e] = 1.0f;
+    }
+    uint32_t wh[4], wl[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float r0 = v[2 * q] * rinv * g[2 * q], r1 = v[2 * q + 1] * rinv * g[2 * q + 1];
+      const __nv_bfloat162 ph = __floats2bfloat162_rn(r0, r1);
+      const float2 hf = __bfloat1622float2(ph);
+      const __nv_bfloat162 pl = __floats2bfloat162_rn(r0 - hf.x, r1 - hf.y);
+      wh[q] = *reinterpret_cast<const uint32_t*>(&ph);
+      wl[q] = *reinterpret_cast<const uint32_t*>(&pl);
+    }
+    hi[c] = make_uint4(wh[0], wh[1], wh[2], wh[3]);
+    lo[c] = make_uint4(wl[0], wl[1], wl[2], wl[3]);
+  }
+}
+
+__global__ void __launch_bounds__(kTcThreads) head_tc_kernel(const __grid_constant__ TcParams P) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ float wbv[kTcThreads / 32][kTcRowsMax];
+  __shared__ int wbi[kTcThreads / 32][kTcRowsMax];
+  const int h = P.h, nb = P.nb, num_kb = P.num_kb;
+  const int stage_bytes = tc_stage_bytes(h);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kTcStages * stage_bytes);
+  uint64_t* full = bars;                     // TMA -> MMA          (count 1 + tx bytes)
+  uint64_t* empty = bars + kTcStages;        // MMA commit -> TMA   (count 1)
+  uint64_t* accfull = bars + 2 * kTcStages;  // MMA commit -> epilogue
+  uint64_t* drain = accfull + 1;             // MMA drain after an abort
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + kTcBars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int v0 = blockIdx.x * kTcBM;
+  const uint32_t limit = P.wait_limit_us;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accfull, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&P.tmap);
+    tma_prefetch_desc(&P.xmap);
+  }
+  if (warp == 1) tmem_alloc(tmem_slot, P.tmem_cols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int kb = 0;
+      for (; kb < num_kb; ++kb) {
+        const int s = kb % kTcStages;
+        const uint32_t ph = (uint32_t)(kb / kTcStages) & 1u;
+        if (!mbar_wait_bounded(&empty[s], ph ^ 1u, limit, abort_flag)) break;
+        uint8_t* st = smem + s * stage_bytes;
+        mbar_arrive_expect_tx(&full[s], (uint32_t)stage_bytes);
+        tma_load_2d(st, &P.tmap, kb * kTcBK, v0, &full[s]);
+        tma_load_2d(st + kTcABytes, &P.xmap, kb * kTcBK, 0, &full[s]);
+      }
+      if (kb < num_kb) {
+        // drain: the stages armed in the last kTcStages iterations must see their copies land
+        for (int j = kb > kTcStages ? kb - kTcStages : 0; j < kb; ++j)
+          mbar_wait_drain(&full[j % kTcStages], (uint32_t)(j / kTcStages) & 1u);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      // kind::f16: D float32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12 = 1), both K-major,
+      // N >> 3 at bits 17-22, M >> 4 at bits 24-28
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(2 * h) >> 3 << 17) |
+                             ((uint32_t)(kTcBM >> 4) << 24);
+      int kb = 0;
+      for (; kb < num_kb; ++kb) {
+        const int s = kb % kTcStages;
+        const uint32_t ph = (uint32_t)(kb / kTcStages) & 1u;
+        if (!mbar_wait_bounded(&full[s], ph, limit, abort_flag)) break;
+        tc_fence_after();
+        const uint32_t a_addr = smem_u32(smem + s * stage_bytes);
+        const uint32_t b_addr = a_addr + kTcABytes;
+#pragma unroll
+        for (int kk = 0; kk < kTcBK / kTcUK; ++kk)
+          tc_mma_bf16_ss(tmem, sw128_desc(a_addr + kk * kTcUK * 2), sw128_desc(b_addr + kk * kTcUK * 2), idesc,
+                         (kb | kk) != 0 ? 1u : 0u);
+        tc_commit(&empty[s]);
+      }
+      if (kb == num_kb) {
+        tc_commit(accfull);
+        // the accumulator is complete before this thread reaches the teardown barrier, whatever
+        // happens to the epilogue's waits
+        mbar_wait_drain(accfull, 0u);
+      } else {
+        tc_commit(drain);
+        mbar_wait_drain(drain, 0u);
+      }
+    }
+    __syncwarp();
+  }
+
+  // ------------------------------------------------------------------ epilogue (all four warps)
+  bool have = mbar_wait_bounded(accfull, 0u, limit, abort_flag);
+  have = __all_sync(0xffffffffu, have);
+  if (have) {
+    tc_fence_after();
+    const int v = v0 + warp * 32 + lane;
+    const bool valid = v < P.vocab;
+    const uint32_t taddr = tmem + ((uint32_t)(warp * 32) << 16);
+    for (int c0 = 0; c0 < nb; c0 += 16) {
+      uint32_t hv[16], lv[16];
+      tmem_ld_32x32b_x16(taddr + (uint32_t)c0, hv);
+      tmem_ld_32x32b_x16(taddr + (uint32_t)(h + c0), lv);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        const int j = c0 + e;
+        if (j < nb) {  // uniform across the warp
+          const float val = __uint_as_float(hv[e]) + __uint_as_float(lv[e]);
+          if (valid && P.logits) P.logits[(int64_t)j * P.ld_logits + v] = val;
+          float bv = valid ? val : -INFINITY;
+          int bi = valid ? v : 0x7fffffff;
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) {
+            const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+            const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+            if (head_better(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+          }
+          if (lane == 0) { wbv[warp][j] = bv; wbi[warp][j] = bi; }
+        }
+      }
+    }
+  } else if (lane == 0) {
+    for (int j = 0; j < nb; ++j) { wbv[warp][j] = -INFINITY; wbi[warp][j] = 0x7fffffff; }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) tmem_dealloc(tmem, P.tmem_cols);
+  if (threadIdx.x < nb) {
+    const int j = threadIdx.x;
+    float bv = -INFINITY;
+    int bi = 0x7fffffff;
+#pragma unroll
+    for (int w = 0; w < kTcThreads / 32; ++w)
+      if (head_better(wbv[w][j], wbi[w][j], bv, bi)) { bv = wbv[w][j]; bi = wbi[w][j]; }
+    P.pmax[(int64_t)blockIdx.x * kTcRowsMax + j] = bv;
+    P.pidx[(int64_t)blockIdx.x * kTcRowsMax + j] = bi;
+  }
 }
 
 }  // namespace head

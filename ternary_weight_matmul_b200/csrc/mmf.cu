@@ -338,7 +338,7 @@ bool use_tensor_path(int64_t m) {
   const int p = g_gemm_path.load();
   if (p == MMF_GEMM_TENSOR) return true;
   if (p == MMF_GEMM_SIMT) return false;
-  return m > kSimtMT;
+  return m >= kSimtMT;  // 8 rows and up: the tensor-core kernel's cost barely depends on m
 }
 
 // gate_proj forms the GLU product in its epilogue when the tensor engine runs it and the inner
@@ -712,11 +712,17 @@ mmf_status noalloc_scratch(void** out) {
   return MMF_OK;
 }
 
-// Partial maxima of the head: one (logit, index) per CTA and token row of a pass; CTAs cover at
-// least head::kMinRowsPerCta vocabulary rows each.
-size_t head_ws_bytes(int32_t vocab) {
-  const size_t parts = (size_t)((vocab + head::kMinRowsPerCta - 1) / head::kMinRowsPerCta);
-  return 2 * align256(parts * head::kRows * 4);
+// Scratch of the head: the partial maxima, one (logit, index) per CTA and token row of a pass
+// (CUDA-core form: CTAs of at least head::kMinRowsPerCta vocabulary rows, head::kRows rows a pass;
+// tensor-core form: CTAs of head::kTcBM rows, head::kTcRowsMax rows a pass), then the bf16 hi / lo
+// token rows of a tensor-core pass ([2 * kTcRowsMax][d]).
+size_t head_parts_bytes(int32_t vocab) {
+  const size_t simt = (size_t)((vocab + head::kMinRowsPerCta - 1) / head::kMinRowsPerCta) * head::kRows;
+  const size_t tc = (size_t)((vocab + head::kTcBM - 1) / head::kTcBM) * head::kTcRowsMax;
+  return align256(std::max(simt, tc) * 4);
+}
+size_t head_ws_bytes(int32_t vocab, int32_t d) {
+  return 2 * head_parts_bytes(vocab) + align256((size_t)2 * head::kTcRowsMax * std::max(d, 0) * 2);
 }
 
 template <mmf_dtype XT, mmf_dtype TT>
@@ -729,7 +735,37 @@ void head_launch(head::Args a, int nb, int nparts, int32_t* ids, cudaStream_t st
   else MMF_HEAD(1);
 #undef MMF_HEAD
   launch_k(head::head_argmax_kernel, dim3((unsigned)((nb + head::kWarps - 1) / head::kWarps)), dim3(head::kThreads), 0, st,
-           (const float*)a.pmax, (const int32_t*)a.pidx, nparts, nb, ids);
+           (const float*)a.pmax, (const int32_t*)a.pidx, nparts, (int)head::kRows, nb, ids);
+}
+
+// One tensor-core pass of nb <= kTcRowsMax token rows: hi / lo rows, logits tiles, argmax.
+mmf_status head_tc_pass(const void* x, mmf_dtype xdt, int nb, int d, const float* norm_w, float eps, const void* table,
+                        int32_t vocab, float* logits, float* pmax, int32_t* pidx, __nv_bfloat16* xs, int32_t* ids,
+                        cudaStream_t st) {
+  const int h = (nb + 15) / 16 * 16;
+  head::TcParams P;
+  memset(&P, 0, sizeof(P));
+  MMF_TRY(encode_2d(&P.tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, table, (uint64_t)d, (uint64_t)vocab, (uint64_t)d * 2,
+                    head::kTcBK, head::kTcBM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MMF_TRY(encode_2d(&P.xmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, xs, (uint64_t)d, (uint64_t)(2 * h), (uint64_t)d * 2,
+                    head::kTcBK, (uint32_t)(2 * h), CU_TENSOR_MAP_SWIZZLE_128B));
+  P.nb = nb; P.h = h;
+  P.num_kb = (d + head::kTcBK - 1) / head::kTcBK;
+  P.vocab = vocab; P.logits = logits; P.ld_logits = vocab;
+  P.pmax = pmax; P.pidx = pidx;
+  uint32_t cols = 32;
+  while (cols < (uint32_t)(2 * h)) cols <<= 1;
+  P.tmem_cols = cols;
+  P.wait_limit_us = g_wait_limit.load();
+  const int tiles = (vocab + head::kTcBM - 1) / head::kTcBM;
+  if (xdt == MMF_F32)
+    launch_k(head::head_pack_kernel<MMF_F32>, dim3((unsigned)h), dim3(head::kThreads), 0, st, x, d, norm_w, eps, nb, h, xs);
+  else
+    launch_k(head::head_pack_kernel<MMF_BF16>, dim3((unsigned)h), dim3(head::kThreads), 0, st, x, d, norm_w, eps, nb, h, xs);
+  launch_k(head::head_tc_kernel, dim3((unsigned)tiles), dim3(head::kTcThreads), (size_t)head::tc_smem_bytes(h), st, P);
+  launch_k(head::head_argmax_kernel, dim3((unsigned)((nb + head::kWarps - 1) / head::kWarps)), dim3(head::kThreads), 0, st,
+           (const float*)pmax, (const int32_t*)pidx, tiles, (int)head::kTcRowsMax, nb, ids);
+  return MMF_OK;
 }
 
 template <mmf_dtype XT, mmf_dtype TT>
@@ -740,6 +776,10 @@ cudaError_t head_attrs() {
   if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   return e;
+}
+cudaError_t head_tc_attrs() {
+  return cudaFuncSetAttribute(head::head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              head::tc_smem_bytes(head::kTcRowsMax));
 }
 
 }  // namespace
@@ -768,7 +808,7 @@ size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32
     case MMF_OP_SCAN:
       return d > 0 ? scan_ws_bytes(m, d) : 0;
     case MMF_OP_HEAD:
-      return inner > 0 ? head_ws_bytes(inner) : 0;
+      return inner > 0 ? head_ws_bytes(inner, d) : 0;
     case MMF_OP_DECODE:
     case MMF_OP_STACK:
       return block_ws(nullptr, m, d, inner, MMF_F32).bytes + 2 * align256((size_t)m * d * 4);
@@ -1115,7 +1155,7 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
   MMF_CHECK_ARG(x && table && ids, "head: null pointer");
   MMF_CHECK_ARG(aligned16(x) && aligned16(table) && (!norm_w || aligned16(norm_w)),
                 "head: x / table / norm_w not 16-byte aligned");
-  MMF_TRY(check_ws(ws, ws_bytes, head_ws_bytes(vocab)));
+  MMF_TRY(check_ws(ws, ws_bytes, head_ws_bytes(vocab, d)));
   DevInfo* di;
   MMF_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1127,22 +1167,39 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
       if (e == cudaSuccess) e = head_attrs<MMF_F32, MMF_BF16>();
       if (e == cudaSuccess) e = head_attrs<MMF_BF16, MMF_F32>();
       if (e == cudaSuccess) e = head_attrs<MMF_BF16, MMF_BF16>();
+      if (e == cudaSuccess) e = head_tc_attrs();
       attr_err = e;
     });
     if (attr_err != cudaSuccess) return fail(MMF_ERR_CUDA, "head attributes: %s", cudaGetErrorString(attr_err));
+  }
+  const size_t parr = head_parts_bytes(vocab);
+  float* pmax = reinterpret_cast<float*>(ws);
+  int32_t* pidx = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) + parr);
+  const size_t xes = dsize(x_dtype);
+  if (table_dtype == MMF_BF16 && b >= head::kTcMinRows) {
+    // tensor cores: the table streams once per kTcRowsMax token rows
+    __nv_bfloat16* xs = reinterpret_cast<__nv_bfloat16*>(reinterpret_cast<uint8_t*>(ws) + 2 * parr);
+    const int passes = (b + head::kTcRowsMax - 1) / head::kTcRowsMax;
+    LaunchScope ls(MMF_KERNEL_OTHER, (double)vocab * d * 2.0 * passes + (double)b * vocab * (logits ? 4.0 : 0.0), st);
+    for (int r0 = 0; r0 < b; r0 += head::kTcRowsMax) {
+      const int nb = std::min(b - r0, head::kTcRowsMax);
+      MMF_TRY(head_tc_pass(reinterpret_cast<const uint8_t*>(x) + (size_t)r0 * d * xes, x_dtype, nb, d, norm_w, eps,
+                           table, vocab, logits ? logits + (int64_t)r0 * vocab : nullptr, pmax, pidx, xs, ids + r0, st));
+      g_launches.fetch_add(3);
+    }
+    g_launches.fetch_sub(1);  // the timing scope counted one launch itself
+    return check_launch("head tensor-core kernels");
   }
   // vocabulary split: a few CTAs per SM, at least kMinRowsPerCta rows each
   int nparts = std::min((vocab + head::kMinRowsPerCta - 1) / head::kMinRowsPerCta, di->sms * 4);
   const int rows_per_cta = (vocab + nparts - 1) / nparts;
   nparts = (vocab + rows_per_cta - 1) / rows_per_cta;
-  const size_t parr = align256((size_t)((vocab + head::kMinRowsPerCta - 1) / head::kMinRowsPerCta) * head::kRows * 4);
   head::Args a;
   memset(&a, 0, sizeof(a));
   a.xdt = x_dtype; a.d = d; a.norm_w = norm_w; a.eps = eps; a.table = table; a.tdt = table_dtype;
   a.vocab = vocab; a.rows_per_cta = rows_per_cta; a.ld_logits = vocab;
-  a.pmax = reinterpret_cast<float*>(ws);
-  a.pidx = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) + parr);
-  const size_t xes = dsize(x_dtype);
+  a.pmax = pmax;
+  a.pidx = pidx;
   LaunchScope ls(MMF_KERNEL_OTHER, (double)vocab * d * dsize(table_dtype) * ((b + head::kRows - 1) / head::kRows) +
                  (double)b * vocab * (logits ? 4.0 : 0.0), st);
   // passes of 8, 4, 2, 1 rows (each kernel handles exactly its row count)

@@ -4,6 +4,7 @@
     python -m ternary_weight_matmul_b200.profile_cases scan --b 4 --t 8192 --d 2048
     python -m ternary_weight_matmul_b200.profile_cases block --m 16384 --d 1024 --inner 2816
     python -m ternary_weight_matmul_b200.profile_cases decode --b 1 --d 2560 --inner 7040 --layers 4
+    python -m ternary_weight_matmul_b200.profile_cases head --b 8 --d 2560 --vocab 32000 --iters 1
 
 Inputs are seeded and synthetic (weights N(0, 0.02), activations N(0, 1)); prints the mean device
 time per iteration measured with CUDA events.
@@ -19,7 +20,7 @@ import ternary_weight_matmul_b200 as mmf
 
 def main() -> None:
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["gemm", "scan", "block", "norm", "decode"])
+    ap.add_argument("case", choices=["gemm", "scan", "block", "norm", "decode", "head"])
     ap.add_argument("--layers", type=int, default=4)
     ap.add_argument("--m", type=int, default=16384)
     ap.add_argument("--n", type=int, default=5632)
@@ -28,6 +29,7 @@ def main() -> None:
     ap.add_argument("--t", type=int, default=8192)
     ap.add_argument("--d", type=int, default=1024)
     ap.add_argument("--inner", type=int, default=2816)
+    ap.add_argument("--vocab", type=int, default=32000)
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=2)
@@ -81,6 +83,15 @@ def main() -> None:
             return mmf.decode_step(blocks, x, state, out=y)
         wbytes = sum(p.codes.numel() * 4 for blk in blocks for p in blk.packed.values())
         work, unit = float(wbytes), "GB/s (packed weights)"
+    elif a.case == "head":
+        table = (torch.randn(a.vocab, a.d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        nw = torch.ones(a.d, device=dev)
+        x = torch.randn(a.b, a.d, generator=g, device=dev).to(dt)
+        ids = torch.empty(a.b, dtype=torch.int32, device=dev)
+
+        def run():
+            return mmf.lm_head_argmax(x, nw, table, ids_out=ids)
+        work, unit = float(table.numel() * 2 * ((a.b + 127) // 128 if a.b >= 2 else 1)), "GB/s (table)"
     else:
         d, inner = a.d, a.inner
         shapes = {"i": (d, d), "f": (d, d), "g": (d, d), "o": (d, d), "gate": (2 * inner, d), "down": (d, inner)}

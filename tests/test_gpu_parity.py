@@ -454,17 +454,19 @@ def test_decode_step_parity(mmf, b):
 
 @pytest.mark.parametrize("b", [1, 2, 4, 8])
 def test_decode_fused_matches_unfused(mmf, b):
-    # 1, 2, 4 or 8 rows take the fused four-launch decode (inputs staged in shared memory up to
-    # two rows, read in place beyond); forcing the tensor-core engine takes the nine-launch block
-    # path instead. Same quantisation arithmetic: states agree closely and the
-    # outputs within the chained-quantisation tolerance.
+    # on the CUDA-core engine 1, 2, 4 or 8 rows take the fused four-launch decode (inputs staged
+    # in shared memory up to two rows, read in place beyond; the automatic choice takes it for 1,
+    # 2 and 4 rows); forcing the tensor-core engine takes the nine-launch block path instead. Same
+    # quantisation arithmetic: states agree closely and the outputs within the chained-
+    # quantisation tolerance.
     layers = [_block_case(mmf, 40 + l, 256, 704) for l in range(2)]
     x = _to(synth.activations(41 + b, (b, 256)))
     state0 = _to(synth.activations(42 + b, (2, b, 256)) * 0.5)
     st_f, st_u = state0.clone(), state0.clone()
-    y_f = mmf.decode_step([c[2] for c in layers], x, st_f)
-    mmf.set_gemm_path(mmf.MMF_GEMM_TENSOR)
     try:
+        mmf.set_gemm_path(mmf.MMF_GEMM_SIMT)
+        y_f = mmf.decode_step([c[2] for c in layers], x, st_f)
+        mmf.set_gemm_path(mmf.MMF_GEMM_TENSOR)
         y_u = mmf.decode_step([c[2] for c in layers], x, st_u)
         _ok(mmf)
     finally:
@@ -501,12 +503,16 @@ def test_decode_wait_cap_ends_and_recovers(mmf):
     np.testing.assert_allclose(_np(st)[0], st_ref[0], rtol=RTOL32, atol=ATOL32)
 
 
-@pytest.mark.parametrize("b,d,vocab,xdt,tdt", [(1, 256, 1000, "f32", "f32"), (3, 256, 777, "bf16", "bf16"),
+# CUDA-core form: float32 table, or one row; tensor-core form: bf16 table and b >= 2 (ragged d and
+# vocabulary tails, two passes at b = 130)
+@pytest.mark.parametrize("b,d,vocab,xdt,tdt", [(1, 256, 1000, "f32", "f32"), (5, 264, 900, "bf16", "f32"),
+                                                (1, 2560, 32000, "bf16", "bf16"), (2, 256, 777, "bf16", "bf16"),
                                                 (11, 264, 1200, "f32", "bf16"), (8, 2560, 32000, "bf16", "bf16"),
-                                                (64, 2560, 32000, "bf16", "bf16")])
+                                                (64, 2560, 32000, "bf16", "bf16"), (130, 200, 1000, "bf16", "bf16")])
 def test_lm_head_argmax_parity(mmf, b, d, vocab, xdt, tdt):
     # final RMSNorm + tied head + greedy next token against the oracle on the same (dtype-
-    # rounded) inputs: logits within 1e-4 (float32 accumulation of d products); the ids are the
+    # rounded) inputs: logits within 1e-4 (float32 accumulation of d products; the tensor-core
+    # form's bf16 hi + lo split of the normalised rows adds ~2^-17 relative); the ids are the
     # first argmax of the kernel's own logits, and the oracle's argmax except at near-ties
     dts = {"f32": torch.float32, "bf16": torch.bfloat16}
     x = _to(synth.activations(80 + b, (b, d)), dts[xdt])
