@@ -30,6 +30,10 @@ Where floating point decides an integer code, this oracle takes the decision in 
 precision of the CUDA path: the weight code is rint(float32(W) / float32(s)) and the activation
 code is rint(float32(r) * float32(127 / absmax)). Everything else stays in float64.
 
+``hgrn2_recurrence`` (HGRN2's state expansion, a next step beyond the HGRN block) takes the one
+step the pages leave entirely open: they name HGRN2 but print no equations, so it restates the
+published HGRN2 recurrence (see its docstring).
+
 Parity is pinned for every function here by tests/test_oracle_pins.py (closed forms, hand-worked
 recurrences, brute force on tiny shapes, statistical and structural invariants).
 """
@@ -233,6 +237,40 @@ def hgrn_scan(f: np.ndarray, i: np.ndarray, h0: np.ndarray | None = None) -> np.
         prev = f[:, s, :] * prev + i[:, s, :]
         h[:, s, :] = prev
     return h
+
+
+# ----------------------------------------------------------------------------------------------
+# HGRN2: the recurrence with state expansion
+# ----------------------------------------------------------------------------------------------
+def hgrn2_recurrence(q: np.ndarray, f: np.ndarray, i: np.ndarray,
+                     S0: np.ndarray | None = None) -> tuple[np.ndarray, np.ndarray]:
+    """Gated linear recurrence with an outer-product state, per head:
+
+        S_t = diag(f_t) S_{t-1} + (1 - f_t)^T i_t      (S_t: dk x dv)
+        o_t = q_t S_t                                 (o_t: dv)
+
+    q, f [B, T, H, dk]; i [B, T, H, dv]; S0 [B, H, dk, dv] or None (zeros). Returns
+    (o [B, T, H, dv], S_T [B, H, dk, dv]) in float64, stepping t in order.
+
+    nightvoyager.top (MatMul-Free LLM report, innovations table and "if you study it" section)
+    names HGRN2 and its module with fused-recurrent and chunked kernel forms, but prints no
+    state-expansion equations. Reading: the published HGRN2 recurrence (Qin et al., 2024, "HGRN2:
+    Gated Linear RNNs with State Expansion"): HGRN's element-wise forget gate becomes a per-row
+    decay of a dk x dv state, the complement 1 - f of the forget gate the key, the input the value
+    and the output gate the query. With dk = 1 and q = 1 it is the element-wise recurrence
+    h_t = f_t h_{t-1} + (1 - f_t) i_t."""
+    q = np.asarray(q, dtype=np.float64)
+    f = np.asarray(f, dtype=np.float64)
+    i = np.asarray(i, dtype=np.float64)
+    b, t, h, dk = f.shape
+    dv = i.shape[-1]
+    S = np.zeros((b, h, dk, dv)) if S0 is None else np.asarray(S0, dtype=np.float64).copy()
+    o = np.zeros((b, t, h, dv))
+    for s in range(t):
+        key = 1.0 - f[:, s]                                   # [B, H, dk]
+        S = f[:, s][..., :, None] * S + key[..., :, None] * i[:, s][..., None, :]
+        o[:, s] = np.einsum("bhk,bhkv->bhv", q[:, s], S)
+    return o, S
 
 
 # ----------------------------------------------------------------------------------------------

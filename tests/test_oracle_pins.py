@@ -392,3 +392,94 @@ def test_lm_head_scale_invariance_and_ties():
     best = int(O.greedy_next(a[:1])[0])
     table2 = np.concatenate([table[:best], table[best:best + 1], table[best:]], axis=0)
     assert int(O.greedy_next(O.lm_head_logits(x[:1], None, table2))[0]) == best
+
+
+# ---------------------------------------------------------------------------------------------
+# HGRN2 recurrence (state expansion)
+# ---------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("case", _golden("hgrn2_recurrence_handworked.json")["cases"], ids=lambda c: c["name"])
+def test_hgrn2_handworked(case):
+    q = np.array(case["q"])[None, :, None, :]
+    f = np.array(case["f"])[None, :, None, :]
+    i = np.array(case["i"])[None, :, None, :]
+    S0 = np.array(case["S0"])[None, None]
+    o, S = O.hgrn2_recurrence(q, f, i, S0)
+    assert np.array_equal(o[0, :, 0], np.array(case["o"]))
+    assert np.array_equal(S[0, 0], np.array(case["S"]))
+
+
+def test_hgrn2_one_key_dimension_is_the_elementwise_recurrence():
+    # dk = 1, q = 1: the state is one row and S_t = f_t S_{t-1} + (1 - f_t) i_t channel by
+    # channel, which is the pinned element-wise scan with input (1 - f) i
+    g = np.random.default_rng(21)
+    B, T, H, dv = 2, 13, 3, 4
+    f = g.uniform(0, 1, (B, T, H, 1))
+    i = g.standard_normal((B, T, H, dv))
+    S0 = g.standard_normal((B, H, 1, dv))
+    o, S = O.hgrn2_recurrence(np.ones((B, T, H, 1)), f, i, S0)
+    fb = np.broadcast_to(f, (B, T, H, dv)).reshape(B, T, H * dv)
+    h = O.hgrn_scan(fb, ((1.0 - f) * i).reshape(B, T, H * dv), S0.reshape(B, H * dv))
+    np.testing.assert_allclose(o.reshape(B, T, H * dv), h, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S.reshape(B, H * dv), h[:, -1], rtol=1e-12, atol=1e-12)
+
+
+def test_hgrn2_bruteforce_attention_form():
+    # unrolled: o_t[v] = sum_k q_t[k] (prod_{r<=t} f_r[k]) S0[k, v]
+    #                  + sum_{s<=t} sum_k q_t[k] (prod_{s<r<=t} f_r[k]) (1 - f_s[k]) i_s[v]
+    g = np.random.default_rng(22)
+    B, T, H, dk, dv = 1, 6, 2, 3, 2
+    q = g.standard_normal((B, T, H, dk))
+    f = g.uniform(0, 1, (B, T, H, dk))
+    i = g.standard_normal((B, T, H, dv))
+    S0 = g.standard_normal((B, H, dk, dv))
+    want = np.zeros((B, T, H, dv))
+    for hh in range(H):
+        for t in range(T):
+            for v in range(dv):
+                acc = 0.0
+                for k in range(dk):
+                    decay0 = 1.0
+                    for r in range(t + 1):
+                        decay0 *= f[0, r, hh, k]
+                    acc += q[0, t, hh, k] * decay0 * S0[0, hh, k, v]
+                    for s in range(t + 1):
+                        w = 1.0 - f[0, s, hh, k]
+                        for r in range(s + 1, t + 1):
+                            w *= f[0, r, hh, k]
+                        acc += q[0, t, hh, k] * w * i[0, s, hh, v]
+                want[0, t, hh, v] = acc
+    o, _ = O.hgrn2_recurrence(q, f, i, S0)
+    np.testing.assert_allclose(o, want, rtol=1e-12, atol=1e-12)
+
+
+def test_hgrn2_zero_forget_closed_form():
+    # f = 0: the state is replaced every step by 1^T i_t, so o_t = (sum_k q_t[k]) i_t
+    g = np.random.default_rng(23)
+    B, T, H, dk, dv = 2, 5, 2, 4, 3
+    q = g.standard_normal((B, T, H, dk))
+    i = g.standard_normal((B, T, H, dv))
+    o, S = O.hgrn2_recurrence(q, np.zeros((B, T, H, dk)), i, g.standard_normal((B, H, dk, dv)))
+    np.testing.assert_allclose(o, q.sum(-1, keepdims=True) * i, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S, np.broadcast_to(i[:, -1, :, None, :], (B, H, dk, dv)), rtol=0, atol=0)
+
+
+def test_hgrn2_state_passing_and_causality():
+    g = np.random.default_rng(24)
+    B, T, H, dk, dv = 2, 24, 2, 4, 5
+    q = g.standard_normal((B, T, H, dk))
+    f = g.uniform(0.3, 1.0, (B, T, H, dk))
+    i = g.standard_normal((B, T, H, dv))
+    o, S = O.hgrn2_recurrence(q, f, i)
+    # two halves with the state carried between them give the same outputs and final state
+    o1, S1 = O.hgrn2_recurrence(q[:, :10], f[:, :10], i[:, :10])
+    o2, S2 = O.hgrn2_recurrence(q[:, 10:], f[:, 10:], i[:, 10:], S1)
+    np.testing.assert_allclose(np.concatenate([o1, o2], axis=1), o, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(S2, S, rtol=1e-12, atol=1e-12)
+    # a change at step 15 leaves every earlier output as it was and reaches step 15 itself
+    i2 = i.copy()
+    i2[1, 15, 0, 2] += 1.0
+    o3, _ = O.hgrn2_recurrence(q, f, i2)
+    assert np.array_equal(o3[:, :15], o[:, :15])
+    assert not np.array_equal(o3[1, 15, 0], o[1, 15, 0])
+    # heads and sequences are independent
+    assert np.array_equal(o3[0], o[0]) and np.array_equal(o3[1, :, 1], o[1, :, 1])
