@@ -85,6 +85,22 @@ def test_invalid_arguments_rejected_on_host(L):
     assert L.mmf_set_wait_limit(0) == mmf.MMF_OK
 
 
+def test_head_arguments_and_workspace_on_host(L):
+    # mmf_lm_head_argmax(x, x_dtype, b, d, norm_w, eps, table, table_dtype, vocab, ids, logits, ws,
+    # ws_bytes, stream): validation, alignment and workspace size are checked before any CUDA call
+    head = L.mmf_lm_head_argmax
+    assert head(16, 0, 2, 12, None, 1e-8, 16, 1, 100, 16, None, 16, 1 << 30, None) == mmf.MMF_ERR_INVALID_ARG  # d % 8
+    assert head(16, 0, 2, 16, None, 1e-8, 16, 1, 0, 16, None, 16, 1 << 30, None) == mmf.MMF_ERR_INVALID_ARG  # vocab
+    assert head(None, 0, 2, 16, None, 1e-8, 16, 1, 100, 16, None, 16, 1 << 30, None) == mmf.MMF_ERR_INVALID_ARG
+    assert head(24, 0, 2, 16, None, 1e-8, 16, 1, 100, 16, None, 16, 1 << 30, None) == mmf.MMF_ERR_INVALID_ARG  # x align
+    assert head(16, 0, 0, 16, None, 1e-8, None, 1, 100, None, None, None, 0, None) == mmf.MMF_OK  # b = 0: nothing
+    need = L.mmf_workspace_bytes(mmf.MMF_OP_HEAD, 0, 2560, 32000, 0)
+    assert head(16, 1, 8, 2560, None, 1e-8, 16, 1, 32000, 16, None, 16, need - 1, None) == mmf.MMF_ERR_WORKSPACE
+    # the tensor-core form keeps 2 x 128 bf16 token rows of d values in the workspace
+    assert need - L.mmf_workspace_bytes(mmf.MMF_OP_HEAD, 0, 0, 32000, 0) == 2 * 128 * 2560 * 2
+    assert L.mmf_workspace_bytes(mmf.MMF_OP_HEAD, 0, 2560, 0, 0) == 0
+
+
 def test_block_shape_mismatch_rejected(L):
     z = mmf.Ternary(256, 256, 64, 64)
     bw = mmf.BlockWeightsC(d=64, inner=32, eps=1e-8, i=z, f=z, g=z, o=z,
