@@ -32,7 +32,8 @@ code is rint(float32(r) * float32(127 / absmax)). Everything else stays in float
 
 ``hgrn2_recurrence`` (HGRN2's state expansion, a next step beyond the HGRN block) takes the one
 step the pages leave entirely open: they name HGRN2 but print no equations, so it restates the
-published HGRN2 recurrence (see its docstring).
+published HGRN2 recurrence (see its docstring). The ``*_backward`` functions give the gradients
+of a training step, exact for the smooth parts and straight-through for the two quantisers.
 
 Parity is pinned for every function here by tests/test_oracle_pins.py (closed forms, hand-worked
 recurrences, brute force on tiny shapes, statistical and structural invariants).
@@ -237,6 +238,85 @@ def hgrn_scan(f: np.ndarray, i: np.ndarray, h0: np.ndarray | None = None) -> np.
         prev = f[:, s, :] * prev + i[:, s, :]
         h[:, s, :] = prev
     return h
+
+
+# ----------------------------------------------------------------------------------------------
+# backward: the gradients of a training step (straight-through estimator through the quantisers)
+# ----------------------------------------------------------------------------------------------
+def hgrn_scan_backward(f: np.ndarray, i: np.ndarray, dh: np.ndarray,
+                       h0: np.ndarray | None = None) -> tuple[np.ndarray, np.ndarray, np.ndarray]:
+    """Gradients through h_t = f_t h_{t-1} + i_t given dL/dh_t = dh_t for every step ([B, T, D]).
+
+    The total gradient reaching h_t is G_t = dh_t + f_{t+1} G_{t+1} (nothing past the last step),
+    taken backwards in time; then dL/di_t = G_t, dL/df_t = G_t h_{t-1} and dL/dh0 = f_0 G_0.
+    Returns (df, di, dh0) in float64."""
+    f = np.asarray(f, dtype=np.float64)
+    dh = np.asarray(dh, dtype=np.float64)
+    b, t, d = f.shape
+    h = hgrn_scan(f, i, h0)
+    first = np.zeros((b, d)) if h0 is None else np.asarray(h0, dtype=np.float64)
+    hprev = np.concatenate([first[:, None, :], h[:, :-1, :]], axis=1)
+    df = np.zeros((b, t, d))
+    di = np.zeros((b, t, d))
+    G = np.zeros((b, d))
+    for s in reversed(range(t)):
+        G = dh[:, s] + (f[:, s + 1] * G if s + 1 < t else 0.0)
+        di[:, s] = G
+        df[:, s] = G * hprev[:, s]
+    return df, di, f[:, 0] * G
+
+
+def hgrn_gates_backward(zf: np.ndarray, zi: np.ndarray, df: np.ndarray,
+                        di: np.ndarray) -> tuple[np.ndarray, np.ndarray]:
+    """Gradients through f = sigmoid(zf), i = SiLU(zi) (1 - f): with sigma' = f (1 - f) and
+    SiLU'(z) = sigmoid(z) (1 + z (1 - sigmoid(z))),
+    dzf = (df - di SiLU(zi)) f (1 - f) and dzi = di (1 - f) SiLU'(zi). Returns (dzf, dzi)."""
+    zf = np.asarray(zf, dtype=np.float64)
+    zi = np.asarray(zi, dtype=np.float64)
+    f = sigmoid(zf)
+    sz = sigmoid(zi)
+    dzf = (np.asarray(df, dtype=np.float64) - np.asarray(di, dtype=np.float64) * silu(zi)) * f * (1.0 - f)
+    dzi = np.asarray(di, dtype=np.float64) * (1.0 - f) * sz * (1.0 + zi * (1.0 - sz))
+    return dzf, dzi
+
+
+def rmsnorm_backward(x: np.ndarray, w: np.ndarray | None, dr: np.ndarray,
+                     eps: float = EPS_NORM) -> tuple[np.ndarray, np.ndarray | None]:
+    """Gradients through r = x rho w with rho = (mean(x^2) + eps)^(-1/2) over the last axis of n:
+    with u = dr w, dx = rho u - rho^3 x mean(u x); dw = sum over rows of dr x rho (None without a
+    gain). Returns (dx, dw)."""
+    x = np.asarray(x, dtype=np.float64)
+    dr = np.asarray(dr, dtype=np.float64)
+    rho = 1.0 / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps)
+    u = dr * (np.asarray(w, dtype=np.float64) if w is not None else 1.0)
+    dx = rho * u - rho ** 3 * x * np.mean(u * x, axis=-1, keepdims=True)
+    dw = None if w is None else (dr * x * rho).reshape(-1, x.shape[-1]).sum(axis=0)
+    return dx, dw
+
+
+def bitlinear_backward(x: np.ndarray, norm_w: np.ndarray | None, W: np.ndarray, dy: np.ndarray,
+                       eps: float = EPS_NORM) -> tuple[np.ndarray, np.ndarray | None, np.ndarray]:
+    """Training gradients of FusedBitLinear with the latent float weight W [N, K], given dL/dy.
+
+    The forward uses the dequantised operands rq = q (a/127) and Wq = t s (``act_quant`` and
+    ``ternarize``); the straight-through estimator passes the gradient through both quantisers
+    unchanged (nightvoyager.top, innovations table: weight_quant quantises in the forward pass
+    and keeps the gradient in the backward pass; the activation quantiser is read the same way).
+    So dL/dr = dy Wq, then the RMSNorm backward gives dx and the gain's gradient, and the latent
+    weight receives dL/dW = dy^T rq. Returns (dx, dnorm_w, dW) in float64."""
+    x = np.asarray(x, dtype=np.float64)
+    k = x.shape[-1]
+    x2 = x.reshape(-1, k)
+    dy2 = np.asarray(dy, dtype=np.float64).reshape(x2.shape[0], -1)
+    t, s_w = ternarize(W)
+    Wq = t.astype(np.float64) * float(s_w)
+    r = rmsnorm(x2, norm_w, eps)
+    q, deq, _ = act_quant(r)
+    rq = q.astype(np.float64) * deq[:, None]
+    dr = dy2 @ Wq
+    dx, dnw = rmsnorm_backward(x2, norm_w, dr, eps)
+    dW = dy2.T @ rq
+    return dx.reshape(x.shape), dnw, dW
 
 
 # ----------------------------------------------------------------------------------------------

@@ -483,3 +483,92 @@ def test_hgrn2_state_passing_and_causality():
     assert not np.array_equal(o3[1, 15, 0], o[1, 15, 0])
     # heads and sequences are independent
     assert np.array_equal(o3[0], o[0]) and np.array_equal(o3[1, :, 1], o[1, :, 1])
+
+
+# ---------------------------------------------------------------------------------------------
+# backward: every gradient against central finite differences of the forward it differentiates
+# ---------------------------------------------------------------------------------------------
+def _fd(fun, arr, eps=1e-6):
+    """Central differences of the scalar fun() with respect to every element of arr (in place)."""
+    grad = np.zeros_like(arr)
+    it = np.nditer(arr, flags=["multi_index"])
+    for _ in it:
+        idx = it.multi_index
+        old = arr[idx]
+        arr[idx] = old + eps
+        up = fun()
+        arr[idx] = old - eps
+        dn = fun()
+        arr[idx] = old
+        grad[idx] = (up - dn) / (2 * eps)
+    return grad
+
+
+def test_scan_backward_finite_differences():
+    g = np.random.default_rng(31)
+    B, T, D = 2, 7, 3
+    f = g.uniform(0.1, 0.95, (B, T, D))
+    i = g.standard_normal((B, T, D))
+    h0 = g.standard_normal((B, D))
+    c = g.standard_normal((B, T, D))        # L = sum c * h, so dL/dh_t = c_t
+    loss = lambda: float(np.sum(c * O.hgrn_scan(f, i, h0)))
+    df, di, dh0 = O.hgrn_scan_backward(f, i, c, h0)
+    np.testing.assert_allclose(df, _fd(loss, f), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(di, _fd(loss, i), rtol=1e-6, atol=1e-8)
+    np.testing.assert_allclose(dh0, _fd(loss, h0), rtol=1e-6, atol=1e-8)
+
+
+def test_gates_backward_finite_differences():
+    g = np.random.default_rng(32)
+    zf = g.standard_normal((3, 5)) * 2
+    zi = g.standard_normal((3, 5)) * 2
+    a, b = g.standard_normal((3, 5)), g.standard_normal((3, 5))
+
+    def loss():
+        f, i = O.hgrn_gates(zf, zi)
+        return float(np.sum(a * f + b * i))
+    dzf, dzi = O.hgrn_gates_backward(zf, zi, a, b)
+    np.testing.assert_allclose(dzf, _fd(loss, zf), rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(dzi, _fd(loss, zi), rtol=1e-6, atol=1e-9)
+
+
+def test_rmsnorm_backward_finite_differences():
+    g = np.random.default_rng(33)
+    x = g.standard_normal((4, 9))
+    w = g.uniform(0.5, 1.5, 9)
+    c = g.standard_normal((4, 9))
+    loss = lambda: float(np.sum(c * O.rmsnorm(x, w)))
+    dx, dw = O.rmsnorm_backward(x, w, c)
+    np.testing.assert_allclose(dx, _fd(loss, x), rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(dw, _fd(loss, w), rtol=1e-6, atol=1e-9)
+    dx1, dw1 = O.rmsnorm_backward(x, None, c)
+    loss1 = lambda: float(np.sum(c * O.rmsnorm(x, None)))
+    np.testing.assert_allclose(dx1, _fd(loss1, x), rtol=1e-6, atol=1e-9)
+    assert dw1 is None
+
+
+def test_bitlinear_backward_is_straight_through():
+    # straight-through: the forward keeps each quantiser's rounding offset (Q(v) - v) frozen and
+    # differentiates v itself; finite differences of that surrogate give the gradients
+    g = np.random.default_rng(34)
+    M, K, N = 3, 16, 5
+    x = g.standard_normal((M, K))
+    nw = g.uniform(0.5, 1.5, K)
+    W = g.standard_normal((N, K)) * 0.05
+    dy = g.standard_normal((M, N))
+    dx, dnw, dW = O.bitlinear_backward(x, nw, W, dy)
+    t, s = O.ternarize(W)
+    Wq = t * float(s)
+    r0 = O.rmsnorm(x, nw)
+    q, deq, _ = O.act_quant(r0)
+    off_r = q * deq[:, None] - r0            # frozen activation rounding offset
+    x_v, nw_v, W_v = x.copy(), nw.copy(), W.copy()
+    loss_act = lambda: float(np.sum(dy * ((O.rmsnorm(x_v, nw_v) + off_r) @ Wq.T)))
+    np.testing.assert_allclose(dx, _fd(loss_act, x_v), rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(dnw, _fd(loss_act, nw_v), rtol=1e-6, atol=1e-9)
+    off_w = Wq - W                           # frozen weight rounding offset
+    loss_w = lambda: float(np.sum(dy * ((r0 + off_r) @ (W_v + off_w).T)))
+    np.testing.assert_allclose(dW, _fd(loss_w, W_v), rtol=1e-6, atol=1e-9)
+    # the forward values themselves are the quantised product (the offsets reproduce it)
+    y, _ = O.bitlinear(x, nw, t, s)
+    np.testing.assert_allclose((r0 + off_r) @ (W + off_w).T, y, rtol=1e-12, atol=1e-12)
