@@ -572,3 +572,30 @@ def test_bitlinear_backward_is_straight_through():
     # the forward values themselves are the quantised product (the offsets reproduce it)
     y, _ = O.bitlinear(x, nw, t, s)
     np.testing.assert_allclose((r0 + off_r) @ (W + off_w).T, y, rtol=1e-12, atol=1e-12)
+
+
+def test_hgrn2_chunked_form_matches_recurrence():
+    # the chunk-parallel form a tensor-core kernel evaluates: within a chunk, with
+    # B_t = prod_{c0 <= r <= t} f_r (per key row) and the key k_s = 1 - f_s,
+    #   o_t = (q_t * B_t) S_start + sum_{c0 <= s <= t} [(q_t * B_t) . (k_s / B_s)] i_s
+    #   S_end = diag(B_end) S_start + sum_s (k_s * B_end / B_s)^T i_s
+    # i.e. three small matrix products per chunk instead of a step-by-step state update
+    g = np.random.default_rng(25)
+    B, T, H, dk, dv, C = 2, 32, 2, 4, 3, 8
+    q = g.standard_normal((B, T, H, dk))
+    f = g.uniform(0.4, 1.0, (B, T, H, dk))
+    i = g.standard_normal((B, T, H, dv))
+    S0 = g.standard_normal((B, H, dk, dv))
+    o_ref, S_ref = O.hgrn2_recurrence(q, f, i, S0)
+    o = np.zeros_like(o_ref)
+    S = S0.copy()
+    for c0 in range(0, T, C):
+        qc, fc, ic = q[:, c0:c0 + C], f[:, c0:c0 + C], i[:, c0:c0 + C]
+        Bc = np.cumprod(fc, axis=1)                              # [B, C, H, dk]
+        qb = qc * Bc
+        kb = (1.0 - fc) / Bc
+        A = np.einsum("bthk,bshk->bhts", qb, kb) * np.tril(np.ones((C, C)))
+        o[:, c0:c0 + C] = np.einsum("bthk,bhkv->bthv", qb, S) + np.einsum("bhts,bshv->bthv", A, ic)
+        S = Bc[:, -1][..., :, None] * S + np.einsum("bshk,bshv->bhkv", kb * Bc[:, -1][:, None], ic)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-10, atol=1e-10)
+    np.testing.assert_allclose(S, S_ref, rtol=1e-10, atol=1e-10)
