@@ -80,6 +80,16 @@ def max_over_ranks(ms: float, device, world: int) -> float:
     return float(t.item())
 
 
+def decode_entry(batch: int, ms_local: float, step_bytes: float, device, world: int, hbm_peak: float) -> dict:
+    """One decode batch size across `world` replicas: each rank generates for its own `batch`
+    sequences; the step time is the slowest rank's, the throughput the tokens of all replicas, and
+    the bandwidth is per GPU (every replica streams its own copy of the weights)."""
+    ms = max_over_ranks(ms_local, device, world)
+    gbs = step_bytes / (ms / 1e3) / 1e9
+    return {"value": batch * world / (ms / 1e3), "ms_per_step": ms, "replicas": world,
+            "bytes_per_step": step_bytes, "GB/s": gbs, "frac_hbm": gbs / hbm_peak}
+
+
 def replicas_throughput(tokens_per_rank: int, world: int, ms_max: float) -> float:
     """Whole-job tokens/s of `world` independent replicas, each processing its own batch."""
     return tokens_per_rank * world / (ms_max / 1e3)
@@ -243,7 +253,7 @@ def build_model(wl, device, seed=1234):
     return blocks, table
 
 
-def run_decode(args, device, hbm_peak):
+def run_decode(args, device, hbm_peak, world=1):
     """Greedy autoregressive decode throughput of the 2.7B-shape stack for each batch size: prompt
     prefill through mmf_stack_fwd (untimed; gives every layer's recurrent state and, through the
     final norm and the tied head, the first generated token), then `--decode-steps` generated
@@ -251,8 +261,11 @@ def run_decode(args, device, hbm_peak):
     tied head and argmax (mmf_lm_head_argmax writes the next ids in place), replayed from a CUDA
     graph (captured after warm-up) and timed with CUDA events on the replay stream. HBM roofline:
     every step streams all packed weights and the bf16 head table (once per pass of the head: one
-    row on the CUDA cores, up to 128 rows on the tensor cores)."""
+    row on the CUDA cores, up to 128 rows on the tensor cores). With several ranks every rank is
+    a replica generating for its own sequences; the ranks meet at a barrier before each timed
+    region and the step time is the slowest rank's."""
     import torch
+    import torch.distributed as dist
 
     import ternary_weight_matmul_b200 as mmf
 
@@ -298,6 +311,8 @@ def run_decode(args, device, hbm_peak):
             for i in range(3):
                 graph.replay()
             torch.cuda.synchronize(device)
+            if world > 1:
+                dist.barrier()
             ev0.record(s)
             for i in range(args.decode_steps):
                 graph.replay()
@@ -308,11 +323,9 @@ def run_decode(args, device, hbm_peak):
             raise RuntimeError(f"device status {st} in decode")
         ms = ev0.elapsed_time(ev1) / args.decode_steps
         step_bytes = weight_bytes + head_bytes * ((B + 127) // 128)
-        gbs = step_bytes / (ms / 1e3) / 1e9
         ids_end = cur.cpu()
         assert int(ids_end.min()) >= 0 and int(ids_end.max()) < dw["vocab"]
-        out["batches"][str(B)] = {"value": B / (ms / 1e3), "ms_per_step": ms, "bytes_per_step": step_bytes,
-                                  "GB/s": gbs, "frac_hbm": gbs / hbm_peak}
+        out["batches"][str(B)] = decode_entry(B, ms, step_bytes, device, world, hbm_peak)
         del graph
     del blocks, table
     torch.cuda.empty_cache()
@@ -413,10 +426,10 @@ def run_gpu(args, wl):
                "h2d_bytes_per_step": ids_host.numel() * 4, "d2h_bytes_per_step": y_host.numel() * 2}
 
     decode = None
-    if not args.no_decode and rank == 0:
+    if not args.no_decode:  # every rank: decode replicas, timed as the slowest rank
         pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
         hbm = json.load(open(pp)).get("hbm_gbs", 6650.0) if os.path.exists(pp) else 6650.0
-        decode = run_decode(args, device, hbm)
+        decode = run_decode(args, device, hbm, world)
 
     line = None
     if rank == 0:

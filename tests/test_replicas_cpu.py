@@ -32,7 +32,9 @@ def _rank_main(rank: int, world: int, port: int, out) -> None:
         local_ms = 10.0 + 2.0 * rank            # rank 1 is the slow one
         ms_max = bench.max_over_ranks(local_ms, torch.device("cpu"), world)
         value = bench.replicas_throughput(16384, world, ms_max)
-        out[rank] = (ms_max, value)
+        # decode replicas: 8 sequences per rank, rank 1 slower, 0.9 GB streamed per step
+        dec = bench.decode_entry(8, 2.0 + rank, 0.9e9, torch.device("cpu"), world, 6525.0)
+        out[rank] = (ms_max, value, dec)
         dist.barrier()
     finally:
         dist.destroy_process_group()
@@ -45,9 +47,13 @@ def test_two_replicas_time_is_the_slowest_rank_and_throughput_sums_batches():
     mp.start_processes(_rank_main, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
     assert set(out.keys()) == {0, 1}
     for r in (0, 1):
-        ms_max, value = out[r]
+        ms_max, value, dec = out[r]
         assert ms_max == pytest.approx(12.0)
         assert value == pytest.approx(2 * 16384 / 0.012)
+        assert dec["ms_per_step"] == pytest.approx(3.0) and dec["replicas"] == 2
+        assert dec["value"] == pytest.approx(2 * 8 / 0.003)       # tokens of both replicas
+        assert dec["GB/s"] == pytest.approx(0.9e9 / 0.003 / 1e9)  # per GPU
+        assert dec["frac_hbm"] == pytest.approx(dec["GB/s"] / 6525.0)
 
 
 def test_single_rank_needs_no_process_group():
@@ -56,6 +62,8 @@ def test_single_rank_needs_no_process_group():
 
     assert bench.max_over_ranks(7.5, torch.device("cpu"), 1) == 7.5
     assert bench.replicas_throughput(1000, 1, 2.0) == pytest.approx(500000.0)
+    dec = bench.decode_entry(64, 2.5, 1e9, torch.device("cpu"), 1, 6525.0)
+    assert dec["value"] == pytest.approx(64 / 0.0025) and dec["replicas"] == 1
 
 
 def test_gemm_traffic_tracks_kernel_source(monkeypatch):
