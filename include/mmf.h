@@ -236,6 +236,21 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
                               float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
                               int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
+/* HGRN2 recurrence with state expansion, per sequence and head (nightvoyager.top, innovations
+ * table, names HGRN2 and its fused-recurrent and chunked kernels; the recurrence is HGRN2's
+ * published one, the pages print no equations):
+ *   S_t = diag(f_t) S_{t-1} + (1 - f_t)^T i_t   (S_t: dk x dv, S_{-1} = s0 or 0)
+ *   o_t = q_t S_t
+ *   q, f  [b][t][heads][dk] dtype, contiguous; f are forget gates in [0, 1] (gating applied by
+ *         the caller).   i [b][t][heads][dv] dtype.   o [b][t][heads][dv] dtype out.
+ *   s0    [b][heads][dk][dv] float32 or NULL (zeros).   s_out same shape float32 out, or NULL.
+ *   1 <= dk <= 128; b, heads <= 65535. t = 0 writes only s_out.
+ * CUDA cores, float32 state and accumulation: one thread per (sequence, head, value column),
+ * steps in order. No workspace. */
+mmf_status mmf_hgrn2_recurrence(const void* q, const void* f, const void* i, mmf_dtype dtype, int32_t b, int64_t t,
+                                int32_t heads, int32_t dk, int32_t dv, const float* s0, float* s_out, void* o,
+                                mmf_stream_t stream);
+
 /* Prefill forward of an HGRNBitModel block stack (hysenlabs.com: HGRNBitModel = embedding + a
  * stack of HGRNBitBlock): embedding gather, then the n_layers blocks in order.
  *   layers  HOST array of n_layers block descriptors.  ids [b][t] int32.

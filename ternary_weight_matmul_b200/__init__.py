@@ -27,7 +27,7 @@ MMF_GEMM_AUTO, MMF_GEMM_TENSOR, MMF_GEMM_SIMT = range(3)
 EXPORTED = (
     "mmf_packed_row_words", "mmf_packed_words", "mmf_workspace_bytes", "mmf_pack_ternary",
     "mmf_bitlinear_fwd", "mmf_hgrn_scan", "mmf_block_fwd", "mmf_block_fwd_taps", "mmf_decode_step",
-    "mmf_embed_gather", "mmf_lm_head_argmax",
+    "mmf_embed_gather", "mmf_lm_head_argmax", "mmf_hgrn2_recurrence",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
     "mmf_bitlinear_fwd_noalloc",
@@ -92,6 +92,7 @@ def lib() -> ctypes.CDLL:
         "mmf_embed_gather": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, i32, i32, vp, st]),
         "mmf_lm_head_argmax": (ctypes.c_int, [vp, ctypes.c_int, i32, i32, vp, ctypes.c_float, vp, ctypes.c_int, i32,
                                               vp, vp, vp, sz, st]),
+        "mmf_hgrn2_recurrence": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, i32, i64, i32, i32, i32, vp, vp, vp, st]),
         "mmf_stack_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, i32, i64, vp, i32,
                                          ctypes.c_int, vp, vp, vp, sz, st]),
         "mmf_sync_status": (ctypes.c_int, [st]),
@@ -277,6 +278,30 @@ def hgrn_scan(zf: torch.Tensor, zi: torch.Tensor, h0: torch.Tensor | None = None
                                h.data_ptr(), _dt(h_dtype), h_last.data_ptr(), ws.data_ptr(), ws.numel(),
                                _stream(zf.device)), "mmf_hgrn_scan")
     return h, h_last
+
+
+def hgrn2_recurrence(q: torch.Tensor, f: torch.Tensor, i: torch.Tensor, s0: torch.Tensor | None = None,
+                     want_state: bool = False):
+    """mmf_hgrn2_recurrence on q, f [b, t, heads, dk] and i [b, t, heads, dv] (one dtype,
+    contiguous): o [b, t, heads, dv] and, with want_state, the final state [b, heads, dk, dv]
+    float32."""
+    for a in (q, f, i):
+        _dev(a)
+        if not a.is_contiguous() or a.dtype != q.dtype:
+            raise ValueError("q, f and i need one dtype and contiguous storage")
+    b, t, heads, dk = q.shape
+    dv = i.shape[-1]
+    if tuple(f.shape) != (b, t, heads, dk) or tuple(i.shape[:3]) != (b, t, heads):
+        raise ValueError("shapes: q, f [b, t, heads, dk] and i [b, t, heads, dv]")
+    if s0 is not None and (tuple(s0.shape) != (b, heads, dk, dv) or s0.dtype != torch.float32
+                           or not s0.is_contiguous()):
+        raise ValueError("s0 must be a contiguous float32 [b, heads, dk, dv]")
+    o = torch.empty(b, t, heads, dv, dtype=q.dtype, device=q.device)
+    s_out = torch.empty(b, heads, dk, dv, dtype=torch.float32, device=q.device) if want_state else None
+    _check(lib().mmf_hgrn2_recurrence(q.data_ptr(), f.data_ptr(), i.data_ptr(), _dt(q.dtype), b, t, heads, dk, dv,
+                                      _ptr(s0), _ptr(s_out), o.data_ptr(), _stream(q.device)),
+           "mmf_hgrn2_recurrence")
+    return (o, s_out) if want_state else o
 
 
 def block_fwd(block: Block, x: torch.Tensor, h0: torch.Tensor | None = None):

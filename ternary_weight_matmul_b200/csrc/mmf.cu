@@ -18,6 +18,7 @@
 #include "decode.cuh"
 #include "gemm_tc.cuh"
 #include "head.cuh"
+#include "hgrn2.cuh"
 #include "kernels.cuh"
 
 using namespace mmf;
@@ -1220,6 +1221,44 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
   }
   g_launches.fetch_sub(1);  // the timing scope counted one launch itself
   return check_launch("head kernels");
+}
+
+// ---------------------------------------------------------------------------------------------
+// HGRN2 recurrence (state expansion)
+// ---------------------------------------------------------------------------------------------
+mmf_status mmf_hgrn2_recurrence(const void* q, const void* f, const void* i, mmf_dtype dtype, int32_t b, int64_t t,
+                                int32_t heads, int32_t dk, int32_t dv, const float* s0, float* s_out, void* o,
+                                mmf_stream_t stream) {
+  MMF_CHECK_ARG(b >= 0 && t >= 0 && heads >= 0 && dv >= 0, "hgrn2: negative size");
+  MMF_CHECK_ARG(dk >= 1 && dk <= 128, "hgrn2: dk = %d outside [1, 128]", dk);
+  MMF_CHECK_ARG(valid_dtype(dtype), "hgrn2: bad dtype");
+  MMF_CHECK_ARG(b <= 65535 && heads <= 65535, "hgrn2: b = %d or heads = %d above 65535", b, heads);
+  if ((int64_t)b * heads * dv == 0) return MMF_OK;
+  MMF_CHECK_ARG(t == 0 || (q && f && i && o), "hgrn2: null pointer");
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  hgrn2::Args a;
+  memset(&a, 0, sizeof(a));
+  a.q = q; a.f = f; a.i = i; a.dt = dtype; a.b = b; a.t = t; a.heads = heads; a.dk = dk; a.dv = dv;
+  a.s0 = s0; a.s_out = s_out; a.o = o;
+  const dim3 grid((unsigned)((dv + hgrn2::kThreads - 1) / hgrn2::kThreads), (unsigned)heads, (unsigned)b);
+  const double es = (double)dsize(dtype);
+  LaunchScope ls(MMF_KERNEL_OTHER, (double)b * t * heads * (2.0 * dk + 2.0 * dv) * es, st);
+#define MMF_HGRN2(DT_, DK_) launch_k(hgrn2::hgrn2_recurrent_kernel<DT_, DK_>, grid, dim3(hgrn2::kThreads), 0, st, a)
+  if (dtype == MMF_F32) {
+    if (dk <= 16) MMF_HGRN2(MMF_F32, 16);
+    else if (dk <= 32) MMF_HGRN2(MMF_F32, 32);
+    else if (dk <= 64) MMF_HGRN2(MMF_F32, 64);
+    else MMF_HGRN2(MMF_F32, 128);
+  } else {
+    if (dk <= 16) MMF_HGRN2(MMF_BF16, 16);
+    else if (dk <= 32) MMF_HGRN2(MMF_BF16, 32);
+    else if (dk <= 64) MMF_HGRN2(MMF_BF16, 64);
+    else MMF_HGRN2(MMF_BF16, 128);
+  }
+#undef MMF_HGRN2
+  return check_launch("hgrn2_recurrent_kernel");
 }
 
 mmf_status mmf_stack_fwd(const mmf_block_weights* layers, int32_t n_layers, const int32_t* ids,

@@ -101,6 +101,18 @@ def test_head_arguments_and_workspace_on_host(L):
     assert L.mmf_workspace_bytes(mmf.MMF_OP_HEAD, 0, 2560, 0, 0) == 0
 
 
+def test_hgrn2_arguments_on_host(L):
+    # mmf_hgrn2_recurrence(q, f, i, dtype, b, t, heads, dk, dv, s0, s_out, o, stream)
+    h2 = L.mmf_hgrn2_recurrence
+    assert h2(16, 16, 16, 0, 1, 4, 1, 0, 4, None, None, 16, None) == mmf.MMF_ERR_INVALID_ARG    # dk = 0
+    assert h2(16, 16, 16, 0, 1, 4, 1, 129, 4, None, None, 16, None) == mmf.MMF_ERR_INVALID_ARG  # dk > 128
+    assert h2(16, 16, 16, 5, 1, 4, 1, 8, 4, None, None, 16, None) == mmf.MMF_ERR_INVALID_ARG    # dtype
+    assert h2(None, 16, 16, 0, 1, 4, 1, 8, 4, None, None, 16, None) == mmf.MMF_ERR_INVALID_ARG  # null q
+    assert h2(16, 16, 16, 0, -1, 4, 1, 8, 4, None, None, 16, None) == mmf.MMF_ERR_INVALID_ARG   # b < 0
+    assert h2(16, 16, 16, 0, 70000, 4, 1, 8, 4, None, None, 16, None) == mmf.MMF_ERR_INVALID_ARG
+    assert h2(None, None, None, 0, 0, 4, 1, 8, 4, None, None, None, None) == mmf.MMF_OK          # b = 0
+
+
 def test_block_shape_mismatch_rejected(L):
     z = mmf.Ternary(256, 256, 64, 64)
     bw = mmf.BlockWeightsC(d=64, inner=32, eps=1e-8, i=z, f=z, g=z, o=z,
