@@ -236,6 +236,18 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
                               float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
                               int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
+/* Gradients of mmf_hgrn_scan for a training step (the recurrence and its gates are smooth, so
+ * these are exact derivatives; nightvoyager.top, innovations table, names the training method):
+ *   forward  f = sigmoid(zf), i = SiLU(zi) (1 - f), h_t = f_t h_{t-1} + i_t, h_{-1} = h0 or 0;
+ *   G_t = dh_t + f_{t+1} G_{t+1} (backwards in time), di_t = G_t, df_t = G_t h_{t-1};
+ *   dzf = (df - di SiLU(zi)) f (1 - f);  dzi = di (1 - f) SiLU'(zi);  dh0 = f_0 G_0.
+ *   zf, zi, h (the forward's states), dh (dL/dh) [b][t][d] dtype, contiguous.
+ *   h0 [b][d] float32 or NULL.   dzf, dzi [b][t][d] dtype out.   dh0 [b][d] float32 out or NULL.
+ * CUDA cores, float32 arithmetic: one thread per (sequence, channel), steps in reverse. */
+mmf_status mmf_hgrn_scan_backward(const void* zf, const void* zi, const void* h, const void* dh, mmf_dtype dtype,
+                                  int32_t b, int64_t t, int32_t d, const float* h0, void* dzf, void* dzi,
+                                  float* dh0, mmf_stream_t stream);
+
 /* HGRN2 recurrence with state expansion, per sequence and head (nightvoyager.top, innovations
  * table, names HGRN2 and its fused-recurrent and chunked kernels; the recurrence is HGRN2's
  * published one, the pages print no equations):

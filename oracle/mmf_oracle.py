@@ -263,7 +263,8 @@ def hgrn_scan_backward(f: np.ndarray, i: np.ndarray, dh: np.ndarray,
         G = dh[:, s] + (f[:, s + 1] * G if s + 1 < t else 0.0)
         di[:, s] = G
         df[:, s] = G * hprev[:, s]
-    return df, di, f[:, 0] * G
+    dh0 = f[:, 0] * G if t else np.zeros((b, d))  # no step: the loss does not depend on h0
+    return df, di, dh0
 
 
 def hgrn_gates_backward(zf: np.ndarray, zi: np.ndarray, df: np.ndarray,

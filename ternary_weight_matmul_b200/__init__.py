@@ -27,7 +27,7 @@ MMF_GEMM_AUTO, MMF_GEMM_TENSOR, MMF_GEMM_SIMT = range(3)
 EXPORTED = (
     "mmf_packed_row_words", "mmf_packed_words", "mmf_workspace_bytes", "mmf_pack_ternary",
     "mmf_bitlinear_fwd", "mmf_hgrn_scan", "mmf_block_fwd", "mmf_block_fwd_taps", "mmf_decode_step",
-    "mmf_embed_gather", "mmf_lm_head_argmax", "mmf_hgrn2_recurrence",
+    "mmf_embed_gather", "mmf_lm_head_argmax", "mmf_hgrn2_recurrence", "mmf_hgrn_scan_backward",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
     "mmf_bitlinear_fwd_noalloc",
@@ -93,6 +93,7 @@ def lib() -> ctypes.CDLL:
         "mmf_lm_head_argmax": (ctypes.c_int, [vp, ctypes.c_int, i32, i32, vp, ctypes.c_float, vp, ctypes.c_int, i32,
                                               vp, vp, vp, sz, st]),
         "mmf_hgrn2_recurrence": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, i32, i64, i32, i32, i32, vp, vp, vp, st]),
+        "mmf_hgrn_scan_backward": (ctypes.c_int, [vp, vp, vp, vp, ctypes.c_int, i32, i64, i32, vp, vp, vp, vp, st]),
         "mmf_stack_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, i32, i64, vp, i32,
                                          ctypes.c_int, vp, vp, vp, sz, st]),
         "mmf_sync_status": (ctypes.c_int, [st]),
@@ -278,6 +279,24 @@ def hgrn_scan(zf: torch.Tensor, zi: torch.Tensor, h0: torch.Tensor | None = None
                                h.data_ptr(), _dt(h_dtype), h_last.data_ptr(), ws.data_ptr(), ws.numel(),
                                _stream(zf.device)), "mmf_hgrn_scan")
     return h, h_last
+
+
+def hgrn_scan_backward(zf: torch.Tensor, zi: torch.Tensor, h: torch.Tensor, dh: torch.Tensor,
+                       h0: torch.Tensor | None = None):
+    """mmf_hgrn_scan_backward on [b, t, d] tensors of one dtype (contiguous): the gradients
+    (dzf, dzi [b, t, d], dh0 [b, d] float32) given the forward's states h and dL/dh."""
+    for a in (zf, zi, h, dh):
+        _dev(a)
+        if a.dtype != zf.dtype or tuple(a.shape) != tuple(zf.shape):
+            raise ValueError("zf, zi, h and dh need one dtype and one shape [b, t, d]")
+    b, t, d = zf.shape
+    dzf = torch.empty_like(zf)
+    dzi = torch.empty_like(zf)
+    dh0 = torch.empty(b, d, dtype=torch.float32, device=zf.device)
+    _check(lib().mmf_hgrn_scan_backward(zf.data_ptr(), zi.data_ptr(), h.data_ptr(), dh.data_ptr(), _dt(zf.dtype),
+                                        b, t, d, _ptr(h0), dzf.data_ptr(), dzi.data_ptr(), dh0.data_ptr(),
+                                        _stream(zf.device)), "mmf_hgrn_scan_backward")
+    return dzf, dzi, dh0
 
 
 def hgrn2_recurrence(q: torch.Tensor, f: torch.Tensor, i: torch.Tensor, s0: torch.Tensor | None = None,

@@ -19,6 +19,7 @@
 #include "gemm_tc.cuh"
 #include "head.cuh"
 #include "hgrn2.cuh"
+#include "backward.cuh"
 #include "kernels.cuh"
 
 using namespace mmf;
@@ -1221,6 +1222,31 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
   }
   g_launches.fetch_sub(1);  // the timing scope counted one launch itself
   return check_launch("head kernels");
+}
+
+// ---------------------------------------------------------------------------------------------
+// gradients of the HGRN scan with its gates
+// ---------------------------------------------------------------------------------------------
+mmf_status mmf_hgrn_scan_backward(const void* zf, const void* zi, const void* h, const void* dh, mmf_dtype dtype,
+                                  int32_t b, int64_t t, int32_t d, const float* h0, void* dzf, void* dzi,
+                                  float* dh0, mmf_stream_t stream) {
+  MMF_CHECK_ARG(b >= 0 && t >= 0 && d >= 0, "scan backward: negative size");
+  MMF_CHECK_ARG(valid_dtype(dtype), "scan backward: bad dtype");
+  if ((int64_t)b * d == 0) return MMF_OK;
+  MMF_CHECK_ARG(t == 0 || (zf && zi && h && dh && dzf && dzi), "scan backward: null pointer");
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  bwd::ScanBwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.zf = zf; a.zi = zi; a.h = h; a.dh = dh; a.dt = dtype; a.b = b; a.t = t; a.d = d;
+  a.h0 = h0; a.dzf = dzf; a.dzi = dzi; a.dh0 = dh0;
+  const int64_t threads = (int64_t)b * d;
+  const dim3 grid((unsigned)((threads + bwd::kThreads - 1) / bwd::kThreads));
+  LaunchScope ls(MMF_KERNEL_SCAN, (double)b * t * d * 6.0 * dsize(dtype), st);
+  if (dtype == MMF_F32) launch_k(bwd::scan_bwd_kernel<MMF_F32>, grid, dim3(bwd::kThreads), 0, st, a);
+  else launch_k(bwd::scan_bwd_kernel<MMF_BF16>, grid, dim3(bwd::kThreads), 0, st, a);
+  return check_launch("scan_bwd_kernel");
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -113,6 +113,15 @@ def test_hgrn2_arguments_on_host(L):
     assert h2(None, None, None, 0, 0, 4, 1, 8, 4, None, None, None, None) == mmf.MMF_OK          # b = 0
 
 
+def test_scan_backward_arguments_on_host(L):
+    # mmf_hgrn_scan_backward(zf, zi, h, dh, dtype, b, t, d, h0, dzf, dzi, dh0, stream)
+    sb = L.mmf_hgrn_scan_backward
+    assert sb(16, 16, 16, 16, 0, -1, 4, 8, None, 16, 16, None, None) == mmf.MMF_ERR_INVALID_ARG  # b < 0
+    assert sb(16, 16, 16, 16, 3, 1, 4, 8, None, 16, 16, None, None) == mmf.MMF_ERR_INVALID_ARG   # dtype
+    assert sb(16, 16, None, 16, 0, 1, 4, 8, None, 16, 16, None, None) == mmf.MMF_ERR_INVALID_ARG  # null h
+    assert sb(None, None, None, None, 0, 0, 4, 8, None, None, None, None, None) == mmf.MMF_OK     # b = 0
+
+
 def test_block_shape_mismatch_rejected(L):
     z = mmf.Ternary(256, 256, 64, 64)
     bw = mmf.BlockWeightsC(d=64, inner=32, eps=1e-8, i=z, f=z, g=z, o=z,

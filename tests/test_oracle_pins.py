@@ -516,6 +516,9 @@ def test_scan_backward_finite_differences():
     np.testing.assert_allclose(df, _fd(loss, f), rtol=1e-6, atol=1e-8)
     np.testing.assert_allclose(di, _fd(loss, i), rtol=1e-6, atol=1e-8)
     np.testing.assert_allclose(dh0, _fd(loss, h0), rtol=1e-6, atol=1e-8)
+    # an empty sequence: nothing depends on h0
+    df0, di0, dh00 = O.hgrn_scan_backward(f[:, :0], i[:, :0], c[:, :0], h0)
+    assert df0.shape == (B, 0, D) and di0.shape == (B, 0, D) and np.array_equal(dh00, np.zeros((B, D)))
 
 
 def test_gates_backward_finite_differences():
