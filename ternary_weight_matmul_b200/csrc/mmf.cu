@@ -1232,6 +1232,7 @@ mmf_status mmf_hgrn_scan_backward(const void* zf, const void* zi, const void* h,
                                   float* dh0, mmf_stream_t stream) {
   MMF_CHECK_ARG(b >= 0 && t >= 0 && d >= 0, "scan backward: negative size");
   MMF_CHECK_ARG(valid_dtype(dtype), "scan backward: bad dtype");
+  MMF_CHECK_ARG((int64_t)b * d < ((int64_t)1 << 38), "scan backward: b * d too large for one grid");
   if ((int64_t)b * d == 0) return MMF_OK;
   MMF_CHECK_ARG(t == 0 || (zf && zi && h && dh && dzf && dzi), "scan backward: null pointer");
   DevInfo* di;
