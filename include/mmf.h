@@ -236,6 +236,24 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
                               float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
                               int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
+/* Training gradients of FusedBitLinear with the straight-through estimator (nightvoyager.top,
+ * innovations table: weight_quant quantises in the forward pass and keeps the gradient in the
+ * backward pass; the activation quantiser is read the same way). With the forward's activation
+ * codes q and factors a/127 (mmf_bitlinear_fwd's q_dbg and deq_dbg), rq = q (a/127), Wq = t s:
+ *   dr = dy Wq;  u = dr norm_w;  rho = (mean(x^2) + eps)^(-1/2)
+ *   dx = rho u - rho^3 x mean(u x)                     [m][w->k] float32 out
+ *   dnorm_w[k] = sum_m dr[m][k] x[m][k] rho_m          [w->k] float32 out, or NULL
+ *   dW = dy^T rq (the latent float weight's gradient)  [w->n][w->k] float32 out, or NULL
+ *   x [m][w->k] x_dtype; norm_w [w->k] float32 or NULL (unit gain); q [m][w->k] int8;
+ *   deq [m] float32; dy [m][w->n] dy_dtype. w->n <= 65535.
+ *   ws >= 4 * m bytes, 256-byte aligned (mmf_workspace_bytes(MMF_OP_BITLINEAR, m, w->k, w->n, 0)
+ *   is always enough). m = 0 writes zero dnorm_w / dW.
+ * CUDA cores, float32 arithmetic. */
+mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, const float* norm_w, float eps,
+                                  const mmf_ternary* w, const int8_t* q, const float* deq, const void* dy,
+                                  mmf_dtype dy_dtype, float* dx, float* dnorm_w, float* dW, void* ws,
+                                  size_t ws_bytes, mmf_stream_t stream);
+
 /* Gradients of mmf_hgrn_scan for a training step (the recurrence and its gates are smooth, so
  * these are exact derivatives; nightvoyager.top, innovations table, names the training method):
  *   forward  f = sigmoid(zf), i = SiLU(zi) (1 - f), h_t = f_t h_{t-1} + i_t, h_{-1} = h0 or 0;

@@ -28,6 +28,7 @@ EXPORTED = (
     "mmf_packed_row_words", "mmf_packed_words", "mmf_workspace_bytes", "mmf_pack_ternary",
     "mmf_bitlinear_fwd", "mmf_hgrn_scan", "mmf_block_fwd", "mmf_block_fwd_taps", "mmf_decode_step",
     "mmf_embed_gather", "mmf_lm_head_argmax", "mmf_hgrn2_recurrence", "mmf_hgrn_scan_backward",
+    "mmf_bitlinear_backward",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
     "mmf_bitlinear_fwd_noalloc",
@@ -94,6 +95,8 @@ def lib() -> ctypes.CDLL:
                                               vp, vp, vp, sz, st]),
         "mmf_hgrn2_recurrence": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, i32, i64, i32, i32, i32, vp, vp, vp, st]),
         "mmf_hgrn_scan_backward": (ctypes.c_int, [vp, vp, vp, vp, ctypes.c_int, i32, i64, i32, vp, vp, vp, vp, st]),
+        "mmf_bitlinear_backward": (ctypes.c_int, [vp, ctypes.c_int, i64, vp, ctypes.c_float, ctypes.POINTER(Ternary),
+                                                  vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, sz, st]),
         "mmf_stack_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, i32, i64, vp, i32,
                                          ctypes.c_int, vp, vp, vp, sz, st]),
         "mmf_sync_status": (ctypes.c_int, [st]),
@@ -279,6 +282,28 @@ def hgrn_scan(zf: torch.Tensor, zi: torch.Tensor, h0: torch.Tensor | None = None
                                h.data_ptr(), _dt(h_dtype), h_last.data_ptr(), ws.data_ptr(), ws.numel(),
                                _stream(zf.device)), "mmf_hgrn_scan")
     return h, h_last
+
+
+def bitlinear_backward(x: torch.Tensor, norm_w: torch.Tensor | None, w: "PackedTernary", q: torch.Tensor,
+                       deq: torch.Tensor, dy: torch.Tensor, eps: float = 1e-8, want_dnorm_w: bool = True,
+                       want_dW: bool = True):
+    """mmf_bitlinear_backward: (dx [m, k], dnorm_w [k] or None, dW [n, k] or None), float32, from
+    x [m, k], the forward's codes q [m, k] int8 and factors deq [m] float32, and dy [m, n]."""
+    for a in (x, q, deq, dy):
+        _dev(a)
+    m, k = x.shape
+    if tuple(q.shape) != (m, k) or q.dtype != torch.int8 or tuple(deq.shape) != (m,) or tuple(dy.shape) != (m, w.n):
+        raise ValueError("shapes: x, q [m, k] (q int8), deq [m], dy [m, n]")
+    dx = torch.empty(m, k, dtype=torch.float32, device=x.device)
+    dnw = torch.empty(k, dtype=torch.float32, device=x.device) if want_dnorm_w else None
+    dW = torch.empty(w.n, k, dtype=torch.float32, device=x.device) if want_dW else None
+    ws = workspace(MMF_OP_BITLINEAR, m, k, w.n, 0, x.device)
+    tw = w.c()
+    _check(lib().mmf_bitlinear_backward(x.data_ptr(), _dt(x.dtype), m, _ptr(norm_w), eps, ctypes.byref(tw),
+                                        q.data_ptr(), deq.data_ptr(), dy.data_ptr(), _dt(dy.dtype), dx.data_ptr(),
+                                        _ptr(dnw), _ptr(dW), ws.data_ptr(), ws.numel(), _stream(x.device)),
+           "mmf_bitlinear_backward")
+    return dx, dnw, dW
 
 
 def hgrn_scan_backward(zf: torch.Tensor, zi: torch.Tensor, h: torch.Tensor, dh: torch.Tensor,

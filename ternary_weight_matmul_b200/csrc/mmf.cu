@@ -1251,6 +1251,48 @@ mmf_status mmf_hgrn_scan_backward(const void* zf, const void* zi, const void* h,
 }
 
 // ---------------------------------------------------------------------------------------------
+// BitLinear training gradients (straight-through estimator)
+// ---------------------------------------------------------------------------------------------
+mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, const float* norm_w, float eps,
+                                  const mmf_ternary* w, const int8_t* q, const float* deq, const void* dy,
+                                  mmf_dtype dy_dtype, float* dx, float* dnorm_w, float* dW, void* ws,
+                                  size_t ws_bytes, mmf_stream_t stream) {
+  MMF_CHECK_ARG(w != nullptr && w->codes && w->scale, "bitlinear backward: null weight");
+  MMF_CHECK_ARG(w->n > 0 && w->k > 0 && w->n <= 65535, "bitlinear backward: weight shape [%d][%d]", w->n, w->k);
+  MMF_CHECK_ARG(m >= 0 && m <= 0x7fffffff, "bitlinear backward: m = %lld", (long long)m);
+  MMF_CHECK_ARG(valid_dtype(x_dtype) && valid_dtype(dy_dtype), "bitlinear backward: bad dtype");
+  MMF_CHECK_ARG(m == 0 || (x && q && deq && dy && dx), "bitlinear backward: null pointer");
+  if (m > 0) MMF_TRY(check_ws(ws, ws_bytes, align256((size_t)m * 4)));
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  bwd::LinBwdArgs a;
+  memset(&a, 0, sizeof(a));
+  a.x = x; a.xdt = x_dtype; a.m = m; a.k = w->k; a.n = w->n; a.norm_w = norm_w; a.eps = eps;
+  a.codes = w->codes; a.kw = row_words(w->k); a.scale = w->scale; a.q = q; a.deq = deq;
+  a.dy = dy; a.dydt = dy_dtype; a.dx = dx; a.dnorm_w = dnorm_w; a.dW = dW;
+  a.rho = reinterpret_cast<float*>(ws);
+  const unsigned kcols = (unsigned)((w->k + bwd::kThreads - 1) / bwd::kThreads);
+  LaunchScope ls(MMF_KERNEL_OTHER, (double)m * (w->k * (dsize(x_dtype) + 1.0 + 8.0) + w->n * dsize(dy_dtype)) +
+                 (double)w->n * row_words(w->k) * 4.0, st);
+  int launches = 0;
+  if (m > 0) {
+    launch_k(bwd::lin_bwd_rho_kernel, dim3((unsigned)((m + bwd::kThreads / 32 - 1) / (bwd::kThreads / 32))),
+             dim3(bwd::kThreads), 0, st, a);
+    const unsigned words = (unsigned)((w->k + 15) / 16);
+    launch_k(bwd::lin_bwd_dr_kernel, dim3((unsigned)m, (words + bwd::kThreads - 1) / bwd::kThreads), dim3(bwd::kThreads),
+             0, st, a);
+    launches += 2;
+  }
+  if (dnorm_w) { launch_k(bwd::lin_bwd_dnw_kernel, dim3(kcols), dim3(bwd::kThreads), 0, st, a); ++launches; }
+  if (m > 0) { launch_k(bwd::lin_bwd_dx_kernel, dim3((unsigned)m), dim3(bwd::kThreads), 0, st, a); ++launches; }
+  if (dW) { launch_k(bwd::lin_bwd_dw_kernel, dim3(kcols, (unsigned)w->n), dim3(bwd::kThreads), 0, st, a); ++launches; }
+  if (launches > 0) g_launches.fetch_add(launches - 1);  // the timing scope counted one launch itself
+  else g_launches.fetch_sub(1);
+  return check_launch("bitlinear backward kernels");
+}
+
+// ---------------------------------------------------------------------------------------------
 // HGRN2 recurrence (state expansion)
 // ---------------------------------------------------------------------------------------------
 mmf_status mmf_hgrn2_recurrence(const void* q, const void* f, const void* i, mmf_dtype dtype, int32_t b, int64_t t,

@@ -122,6 +122,25 @@ def test_scan_backward_arguments_on_host(L):
     assert sb(None, None, None, None, 0, 0, 4, 8, None, None, None, None, None) == mmf.MMF_OK     # b = 0
 
 
+def test_bitlinear_backward_arguments_on_host(L):
+    # mmf_bitlinear_backward(x, x_dtype, m, norm_w, eps, w, q, deq, dy, dy_dtype, dx, dnorm_w, dW,
+    # ws, ws_bytes, stream)
+    bb = L.mmf_bitlinear_backward
+    ok_w = mmf.Ternary(16, 32, 8, 64)
+    assert bb(16, 0, 4, None, 1e-8, None, 16, 16, 16, 0, 16, None, None, 256, 1 << 20, None) == mmf.MMF_ERR_INVALID_ARG
+    big = mmf.Ternary(16, 32, 70000, 64)
+    assert bb(16, 0, 4, None, 1e-8, ctypes.byref(big), 16, 16, 16, 0, 16, None, None, 256, 1 << 20,
+              None) == mmf.MMF_ERR_INVALID_ARG                                                     # n > 65535
+    assert bb(16, 0, -1, None, 1e-8, ctypes.byref(ok_w), 16, 16, 16, 0, 16, None, None, 256, 1 << 20,
+              None) == mmf.MMF_ERR_INVALID_ARG                                                     # m < 0
+    assert bb(16, 4, 4, None, 1e-8, ctypes.byref(ok_w), 16, 16, 16, 0, 16, None, None, 256, 1 << 20,
+              None) == mmf.MMF_ERR_INVALID_ARG                                                     # dtype
+    assert bb(16, 0, 4, None, 1e-8, ctypes.byref(ok_w), None, 16, 16, 0, 16, None, None, 256, 1 << 20,
+              None) == mmf.MMF_ERR_INVALID_ARG                                                     # null q
+    assert bb(16, 0, 1000, None, 1e-8, ctypes.byref(ok_w), 16, 16, 16, 0, 16, None, None, 256, 1024,
+              None) == mmf.MMF_ERR_WORKSPACE                                                       # 4 KB needed
+
+
 def test_block_shape_mismatch_rejected(L):
     z = mmf.Ternary(256, 256, 64, 64)
     bw = mmf.BlockWeightsC(d=64, inner=32, eps=1e-8, i=z, f=z, g=z, o=z,

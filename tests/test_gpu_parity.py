@@ -617,3 +617,34 @@ def test_scan_backward_parity(mmf, dt, b, t, d, long_memory):
         np.testing.assert_allclose(_np(dzf), dzf_ref, rtol=tol, atol=tol * np.abs(dzf_ref).max())
         np.testing.assert_allclose(_np(dzi), dzi_ref, rtol=tol, atol=tol * np.abs(dzi_ref).max())
     np.testing.assert_allclose(dh0.cpu().numpy(), dh0_ref, rtol=tol, atol=tol * max(np.abs(dh0_ref).max(), 1e-30))
+
+
+# BitLinear gradients with the straight-through estimator against the oracle, on the forward's own
+# activation codes (the kernel backward takes them from mmf_bitlinear_fwd, whose codes the forward
+# parity tests check against the oracle's): dx and the gain's gradient against the oracle's RMSNorm
+# backward of dr = dy (t s), dW against dy^T (q a/127) with the forward's q and a/127. float32
+# accumulation over n (dr) or m (dW): within 1e-4 of the largest value.
+@pytest.mark.skip(reason="compiled for sm_100a, first GPU run pending")
+@pytest.mark.parametrize("xdt", ["f32", "bf16"])
+@pytest.mark.parametrize("m,n,k", [(5, 33, 200), (64, 128, 256), (0, 16, 64)])
+def test_bitlinear_backward_parity(mmf, xdt, m, n, k):
+    dts = {"f32": torch.float32, "bf16": torch.bfloat16}
+    x = _to(synth.activations(100, (m, k)), dts[xdt])
+    nw = synth.norm_weight(101, k, random=True)
+    Wl = synth.weight(102, n, k)
+    w = mmf.pack_ternary(_to(Wl))
+    dy = _to(synth.activations(103, (m, n)), dts[xdt])
+    _, q, deq, _ = mmf.bitlinear_fwd(x, _to(nw), w, y_dtype=torch.float32, debug=True)
+    dx, dnw, dW = mmf.bitlinear_backward(x, _to(nw), w, q, deq, dy)
+    _ok(mmf)
+    t, s = O.ternarize(Wl)
+    x64, dy64 = _np(x).astype(np.float64), _np(dy).astype(np.float64)
+    dr = dy64 @ (t.astype(np.float64) * float(s))
+    dx_ref, dnw_ref = O.rmsnorm_backward(x64, nw, dr)
+    dW_ref = dy64.T @ (q.cpu().numpy().astype(np.float64) * deq.cpu().numpy().astype(np.float64)[:, None])
+    if m:
+        np.testing.assert_allclose(dx.cpu().numpy(), dx_ref, rtol=1e-4, atol=1e-4 * np.abs(dx_ref).max())
+    scale_nw = max(np.abs(dnw_ref).max(), 1e-30)
+    np.testing.assert_allclose(dnw.cpu().numpy(), dnw_ref, rtol=1e-4, atol=1e-4 * scale_nw)
+    scale_w = max(np.abs(dW_ref).max(), 1e-30)
+    np.testing.assert_allclose(dW.cpu().numpy(), dW_ref, rtol=1e-4, atol=1e-4 * scale_w)
