@@ -154,3 +154,19 @@ def test_binding_refuses_cpu_tensors(L):
     import torch
     with pytest.raises(ValueError):
         mmf.pack_ternary(torch.zeros(4, 4))
+
+
+def test_new_bindings_refuse_cpu_tensors(L):
+    # the training-gradient and HGRN2 wrappers reject host tensors before any library call
+    import torch
+    z = torch.zeros(1, 4, 2, 8)
+    with pytest.raises(ValueError):
+        mmf.hgrn2_recurrence(z, z, z)
+    z3 = torch.zeros(1, 4, 8)
+    with pytest.raises(ValueError):
+        mmf.hgrn_scan_backward(z3, z3, z3, z3)
+    w = mmf.PackedTernary.__new__(mmf.PackedTernary)
+    w.n, w.k = 4, 8
+    with pytest.raises(ValueError):
+        mmf.bitlinear_backward(torch.zeros(2, 8), None, w, torch.zeros(2, 8, dtype=torch.int8),
+                               torch.zeros(2), torch.zeros(2, 4))
