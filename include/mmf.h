@@ -236,6 +236,12 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
                               float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
                               int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
+/* Integrity check of a packed ternary matrix (the format above): *bad (device) receives the number
+ * of 2-bit fields holding the unused pattern 10 plus the nonzero fields in each row's padding
+ * columns k .. 16 * mmf_packed_row_words(k) - 1; 0 means the codes are well formed. The count is
+ * reset and written on `stream` (read it after mmf_sync_status). Any shape. */
+mmf_status mmf_validate_packed(const mmf_ternary* w, unsigned long long* bad, mmf_stream_t stream);
+
 /* Training gradients of FusedBitLinear with the straight-through estimator (nightvoyager.top,
  * innovations table: weight_quant quantises in the forward pass and keeps the gradient in the
  * backward pass; the activation quantiser is read the same way). With the forward's activation

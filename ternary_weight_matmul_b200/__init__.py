@@ -28,7 +28,7 @@ EXPORTED = (
     "mmf_packed_row_words", "mmf_packed_words", "mmf_workspace_bytes", "mmf_pack_ternary",
     "mmf_bitlinear_fwd", "mmf_hgrn_scan", "mmf_block_fwd", "mmf_block_fwd_taps", "mmf_decode_step",
     "mmf_embed_gather", "mmf_lm_head_argmax", "mmf_hgrn2_recurrence", "mmf_hgrn_scan_backward",
-    "mmf_bitlinear_backward",
+    "mmf_bitlinear_backward", "mmf_validate_packed",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
     "mmf_bitlinear_fwd_noalloc",
@@ -95,6 +95,7 @@ def lib() -> ctypes.CDLL:
                                               vp, vp, vp, sz, st]),
         "mmf_hgrn2_recurrence": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, i32, i64, i32, i32, i32, vp, vp, vp, st]),
         "mmf_hgrn_scan_backward": (ctypes.c_int, [vp, vp, vp, vp, ctypes.c_int, i32, i64, i32, vp, vp, vp, vp, st]),
+        "mmf_validate_packed": (ctypes.c_int, [ctypes.POINTER(Ternary), vp, st]),
         "mmf_bitlinear_backward": (ctypes.c_int, [vp, ctypes.c_int, i64, vp, ctypes.c_float, ctypes.POINTER(Ternary),
                                                   vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, sz, st]),
         "mmf_stack_fwd": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, i32, i64, vp, i32,
@@ -282,6 +283,16 @@ def hgrn_scan(zf: torch.Tensor, zi: torch.Tensor, h0: torch.Tensor | None = None
                                h.data_ptr(), _dt(h_dtype), h_last.data_ptr(), ws.data_ptr(), ws.numel(),
                                _stream(zf.device)), "mmf_hgrn_scan")
     return h, h_last
+
+
+def validate_packed(w: "PackedTernary") -> int:
+    """mmf_validate_packed: the number of malformed 2-bit fields in w (0 when well formed)."""
+    _dev(w.codes)
+    bad = torch.empty(1, dtype=torch.int64, device=w.codes.device)
+    tw = w.c()
+    _check(lib().mmf_validate_packed(ctypes.byref(tw), bad.data_ptr(), _stream(w.codes.device)),
+           "mmf_validate_packed")
+    return int(bad.item())
 
 
 def bitlinear_backward(x: torch.Tensor, norm_w: torch.Tensor | None, w: "PackedTernary", q: torch.Tensor,

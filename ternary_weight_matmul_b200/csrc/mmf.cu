@@ -20,6 +20,7 @@
 #include "head.cuh"
 #include "hgrn2.cuh"
 #include "backward.cuh"
+#include "validate.cuh"
 #include "kernels.cuh"
 
 using namespace mmf;
@@ -1222,6 +1223,26 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
   }
   g_launches.fetch_sub(1);  // the timing scope counted one launch itself
   return check_launch("head kernels");
+}
+
+// ---------------------------------------------------------------------------------------------
+// packed-code integrity
+// ---------------------------------------------------------------------------------------------
+mmf_status mmf_validate_packed(const mmf_ternary* w, unsigned long long* bad, mmf_stream_t stream) {
+  MMF_CHECK_ARG(w != nullptr && w->codes != nullptr && bad != nullptr, "validate: null pointer");
+  MMF_CHECK_ARG(w->n >= 0 && w->k >= 0, "validate: negative shape");
+  DevInfo* di;
+  MMF_TRY(device_info(&di));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  MMF_CUDA(cudaMemsetAsync(bad, 0, sizeof(unsigned long long), st));
+  const int32_t kw = w->k > 0 ? row_words(w->k) : 0;
+  const int64_t total = (int64_t)w->n * kw;
+  if (total == 0) return MMF_OK;
+  const int64_t blocks = std::min<int64_t>((total + validate::kThreads - 1) / validate::kThreads, (int64_t)di->sms * 8);
+  LaunchScope ls(MMF_KERNEL_OTHER, (double)total * 4.0, st);
+  launch_k(validate::validate_packed_kernel, dim3((unsigned)blocks), dim3(validate::kThreads), 0, st, w->codes,
+           w->n, w->k, kw, bad);
+  return check_launch("validate_packed_kernel");
 }
 
 // ---------------------------------------------------------------------------------------------

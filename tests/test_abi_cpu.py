@@ -170,3 +170,11 @@ def test_new_bindings_refuse_cpu_tensors(L):
     with pytest.raises(ValueError):
         mmf.bitlinear_backward(torch.zeros(2, 8), None, w, torch.zeros(2, 8, dtype=torch.int8),
                                torch.zeros(2), torch.zeros(2, 4))
+
+
+def test_validate_packed_arguments_on_host(L):
+    assert L.mmf_validate_packed(None, 16, None) == mmf.MMF_ERR_INVALID_ARG
+    t = mmf.Ternary(16, 32, 4, 64)
+    assert L.mmf_validate_packed(ctypes.byref(t), None, None) == mmf.MMF_ERR_INVALID_ARG
+    neg = mmf.Ternary(16, 32, -1, 64)
+    assert L.mmf_validate_packed(ctypes.byref(neg), 16, None) == mmf.MMF_ERR_INVALID_ARG
