@@ -166,6 +166,24 @@ def unpack_codes(words: np.ndarray, k: int) -> np.ndarray:
     return t
 
 
+def count_malformed_fields(words: np.ndarray, k: int) -> int:
+    """Integrity of a packed matrix [N, KW] holding K real columns: the number of 2-bit fields
+    that ``pack_codes`` never writes -- a real column (col < k) holding the unused pattern 10, or
+    a padding column (k <= col < 16 * KW) holding anything but 00. Each field counts once.
+    Written as plain loops over the columns of the format."""
+    words = np.asarray(words, dtype=np.uint64)
+    n, kw = words.shape
+    bad = 0
+    for col in range(16 * kw):
+        w, j = divmod(col, 16)
+        f = (words[:, w] >> np.uint64(code_bit(j))) & np.uint64(3)
+        if col < k:
+            bad += int(np.count_nonzero(f == 2))
+        else:
+            bad += int(np.count_nonzero(f != 0))
+    return bad
+
+
 # ----------------------------------------------------------------------------------------------
 # BitLinear
 # ----------------------------------------------------------------------------------------------

@@ -260,6 +260,30 @@ def test_pack_roundtrip_ragged():
         O.unpack_codes(np.array([[0b10, 0, 0, 0]], dtype=np.uint32), 1)
 
 
+def test_count_malformed_fields():
+    # freshly packed codes (ragged k: the last word of a row holds padding fields) are well formed
+    g = np.random.default_rng(17)
+    t = g.integers(-1, 2, (5, 70)).astype(np.int8)
+    w = O.pack_codes(t)
+    assert O.count_malformed_fields(w, 70) == 0
+    # the hand-worked word: its sixteen fields are real columns at k = 16 and padding at k = 7
+    gd = _golden("packed_word_handworked.json")
+    hw = np.array([[int(gd["word_hex"], 16), 0, 0, 0]], dtype=np.uint32)
+    assert O.count_malformed_fields(hw, 16) == 0
+    assert O.count_malformed_fields(hw, 7) == sum(1 for c in gd["codes"][7:] if c != 0)  # 6 nonzero codes
+    # a 10 in a real column counts once; nonzero padding fields count once each, a 10 there too
+    bad = w.copy()
+    bad[1, 0] = (bad[1, 0] & ~np.uint32(3 << O.code_bit(5))) | np.uint32(2 << O.code_bit(5))
+    assert O.count_malformed_fields(bad, 70) == 1
+    bad[2, 4] |= np.uint32(1 << O.code_bit(75 - 64))   # column 75: padding, +1
+    bad[3, 4] |= np.uint32(2 << O.code_bit(77 - 64))   # column 77: padding, 10
+    assert O.count_malformed_fields(bad, 70) == 3
+    # a field pattern 11 in a real column is a valid -1
+    ok = w.copy()
+    ok[0, 0] |= np.uint32(3 << O.code_bit(2))
+    assert O.count_malformed_fields(ok, 70) == 0
+
+
 # ---------------------------------------------------------------------------------------------
 # block, decode and stack
 # ---------------------------------------------------------------------------------------------
