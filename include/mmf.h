@@ -209,6 +209,40 @@ mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, co
                            mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
                            size_t ws_bytes, mmf_stream_t stream);
 
+/* Debug taps of one decode step, one struct per layer; every non-NULL pointer receives that
+ * intermediate of the layer (b token rows, es = dtype):
+ *   q_ifg [3][b][d] int8, deq_ifg [3][b]: codes / a/127 of the i, f, g inputs
+ *   z [b][3d] float32 = [zi | zf | g]      h [b][d] float32: the h that g_norm reads
+ *   q_o [b][d], deq_o [b]                  x1 [b][d] dtype
+ *   q_gate [b][d], deq_gate [b]
+ *   v [b][I] dtype = SiLU(gate) * up, written when the step forms it (the fused decode, or the
+ *     block path with the GLU in gate_proj's epilogue); gu [b][2I] dtype = [gate | up] otherwise
+ *   q_down [b][I], deq_down [b]            y [b][d] dtype: the layer's output
+ * On the block path z and h are the stored dtype values widened to float32. */
+typedef struct {
+  int8_t* q_ifg;
+  float* deq_ifg;
+  float* z;
+  float* h;
+  int8_t* q_o;
+  float* deq_o;
+  void* x1;
+  int8_t* q_gate;
+  float* deq_gate;
+  void* gu;
+  void* v;
+  int8_t* q_down;
+  float* deq_down;
+  void* y;
+} mmf_decode_taps;
+
+/* mmf_decode_step with the intermediates of every layer copied into taps[0 .. n_layers) (HOST
+ * array): same kernels and workspace; for tests and debugging (the copies add traffic). */
+mmf_status mmf_decode_step_taps(const mmf_block_weights* layers, int32_t n_layers, const void* x,
+                                mmf_dtype dtype, int32_t b, float* state, void* y,
+                                const mmf_decode_taps* taps, void* ws, size_t ws_bytes,
+                                mmf_stream_t stream);
+
 /* Token embedding gather: out[r] = table[ids[r]] for r < m.
  *   ids [m] int32. Ids live on the device and are not checked on the host; an id outside
  *   [0, vocab) yields a zero row (never an out-of-bounds read).
@@ -236,10 +270,11 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
                               float eps, const void* table, mmf_dtype table_dtype, int32_t vocab,
                               int32_t* ids, float* logits, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
-/* Integrity check of a packed ternary matrix (the format above): *bad (device) receives the number
- * of 2-bit fields holding the unused pattern 10 plus the nonzero fields in each row's padding
- * columns k .. 16 * mmf_packed_row_words(k) - 1; 0 means the codes are well formed. The count is
- * reset and written on `stream` (read it after mmf_sync_status). Any shape. */
+/* Integrity check of a packed ternary matrix (the format above): *bad (device, 8-byte aligned)
+ * receives the number of malformed 2-bit fields: fields of real columns holding the unused
+ * pattern 10, plus nonzero fields in each row's padding columns k .. 16 * mmf_packed_row_words(k)
+ * - 1 (each field counts once); 0 means the codes are well formed. w->codes 16-byte aligned. The
+ * count is reset and written on `stream` (read it after mmf_sync_status). Any shape. */
 mmf_status mmf_validate_packed(const mmf_ternary* w, unsigned long long* bad, mmf_stream_t stream);
 
 /* Training gradients of FusedBitLinear with the straight-through estimator (nightvoyager.top,
@@ -313,7 +348,9 @@ mmf_status mmf_stack_fwd(const mmf_block_weights* layers, int32_t n_layers, cons
  *   process exits. A call needs mmf_workspace_bytes(MMF_OP_BITLINEAR, m, w->k, w->n, 0) bytes of
  *   it; larger requests return MMF_ERR_WORKSPACE before anything is enqueued.
  *   Set-up: the first call on each device looks up the array's device address on that device
- *   (the device must be current); make that first call before any stream capture begins.
+ *   (the device must be current); make that first call before any stream capture begins. The
+ *   address belongs to the device's context: after a cudaDeviceReset the next call looks it up
+ *   again (that call, too, should come before any stream capture).
  *   Sharing: every call on a device uses the same array and leaves its contents behind; the
  *   kernels overwrite every byte they read, so nothing needs clearing between calls. Calls whose
  *   execution overlaps on the GPU (other streams, other host threads) race on the array: order

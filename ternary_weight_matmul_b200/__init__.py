@@ -31,7 +31,7 @@ EXPORTED = (
     "mmf_bitlinear_backward", "mmf_validate_packed",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
-    "mmf_bitlinear_fwd_noalloc",
+    "mmf_bitlinear_fwd_noalloc", "mmf_decode_step_taps",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -58,6 +58,12 @@ class BlockTapsC(ctypes.Structure):
     _fields_ = [(name, ctypes.c_void_p) for name in (
         "q_ifg", "deq_ifg", "z", "h", "q_o", "deq_o", "x1", "q_gate", "deq_gate", "gu", "q_down", "deq_down",
         "v")]
+
+
+class DecodeTapsC(ctypes.Structure):
+    _fields_ = [(name, ctypes.c_void_p) for name in (
+        "q_ifg", "deq_ifg", "z", "h", "q_o", "deq_o", "x1", "q_gate", "deq_gate", "gu", "v", "q_down", "deq_down",
+        "y")]
 
 
 _lib = None
@@ -90,6 +96,8 @@ def lib() -> ctypes.CDLL:
                                               vp, ctypes.POINTER(BlockTapsC), vp, sz, st]),
         "mmf_decode_step": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, ctypes.c_int, i32, vp, vp,
                                            vp, sz, st]),
+        "mmf_decode_step_taps": (ctypes.c_int, [ctypes.POINTER(BlockWeightsC), i32, vp, ctypes.c_int, i32, vp, vp,
+                                                ctypes.POINTER(DecodeTapsC), vp, sz, st]),
         "mmf_embed_gather": (ctypes.c_int, [vp, i64, vp, ctypes.c_int, i32, i32, vp, st]),
         "mmf_lm_head_argmax": (ctypes.c_int, [vp, ctypes.c_int, i32, i32, vp, ctypes.c_float, vp, ctypes.c_int, i32,
                                               vp, vp, vp, sz, st]),
@@ -286,7 +294,9 @@ def hgrn_scan(zf: torch.Tensor, zi: torch.Tensor, h0: torch.Tensor | None = None
 
 
 def validate_packed(w: "PackedTernary") -> int:
-    """mmf_validate_packed: the number of malformed 2-bit fields in w (0 when well formed)."""
+    """mmf_validate_packed: the number of malformed 2-bit fields in w (0 when well formed): fields
+    of real columns holding the unused pattern 10 plus nonzero fields in the padding columns,
+    each malformed field counted once."""
     _dev(w.codes)
     bad = torch.empty(1, dtype=torch.int64, device=w.codes.device)
     tw = w.c()
@@ -415,6 +425,46 @@ def decode_step(blocks: list[Block], x: torch.Tensor, state: torch.Tensor, out: 
     _check(lib().mmf_decode_step(arr, len(blocks), x.data_ptr(), _dt(x.dtype), b, state.data_ptr(), y.data_ptr(),
                                  ws.data_ptr(), ws.numel(), _stream(x.device)), "mmf_decode_step")
     return y
+
+
+def decode_step_taps(blocks: list[Block], x: torch.Tensor, state: torch.Tensor):
+    """mmf_decode_step_taps: decode_step plus every layer's intermediates (see mmf_decode_taps).
+    Returns (y, taps) with taps a list (one dict of tensors per layer)."""
+    _dev(x)
+    _dev(state)
+    b, d = x.shape
+    inner, dev, dt = blocks[0].inner, x.device, x.dtype
+    y = torch.empty_like(x)
+    taps = []
+    for _ in blocks:
+        taps.append({
+            "q_ifg": torch.empty(3, b, d, dtype=torch.int8, device=dev),
+            "deq_ifg": torch.empty(3, b, dtype=torch.float32, device=dev),
+            "z": torch.empty(b, 3 * d, dtype=torch.float32, device=dev),
+            "h": torch.empty(b, d, dtype=torch.float32, device=dev),
+            "q_o": torch.empty(b, d, dtype=torch.int8, device=dev),
+            "deq_o": torch.empty(b, dtype=torch.float32, device=dev),
+            "x1": torch.empty(b, d, dtype=dt, device=dev),
+            "q_gate": torch.empty(b, d, dtype=torch.int8, device=dev),
+            "deq_gate": torch.empty(b, dtype=torch.float32, device=dev),
+            "gu": torch.full((b, 2 * inner), float("nan"), dtype=dt, device=dev),
+            "v": torch.full((b, inner), float("nan"), dtype=dt, device=dev),
+            "q_down": torch.empty(b, inner, dtype=torch.int8, device=dev),
+            "deq_down": torch.empty(b, dtype=torch.float32, device=dev),
+            "y": torch.empty(b, d, dtype=dt, device=dev),
+        })
+    arr_t = (DecodeTapsC * len(blocks))(*[DecodeTapsC(**{k: v.data_ptr() for k, v in t.items()}) for t in taps])
+    ws = workspace(MMF_OP_DECODE, b, blocks[0].d, inner, len(blocks), dev)
+    arr = _blocks_array(blocks)
+    _check(lib().mmf_decode_step_taps(arr, len(blocks), x.data_ptr(), _dt(dt), b, state.data_ptr(), y.data_ptr(),
+                                      arr_t, ws.data_ptr(), ws.numel(), _stream(dev)), "mmf_decode_step_taps")
+    return y, taps
+
+
+def decode_fused(b: int, d: int, inner: int) -> bool:
+    """Whether a decode step of b rows takes the fused four-launch path (engine choice as set)."""
+    tensor = _gemm_path == MMF_GEMM_TENSOR or (_gemm_path == MMF_GEMM_AUTO and b >= 8)
+    return b in (1, 2, 4, 8) and not tensor and d % 8 == 0 and inner % 8 == 0
 
 
 def embed_gather(ids: torch.Tensor, table: torch.Tensor) -> torch.Tensor:

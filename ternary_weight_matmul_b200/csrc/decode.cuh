@@ -61,6 +61,11 @@ struct Args {
   float* g_out;           // kIFG: g [b][nout] float32
   float* state;           // kIFG: recurrent state [b][nout] float32, read and overwritten
   uint32_t wait_limit_us;
+  // debug taps (null on the timed path): CTA 0 copies the codes it formed, [gain][row][k] int8,
+  // and the factors a/127, [gain][row]; kIFG also writes zi, zf and g as [row][3 * nout] float32
+  int8_t* q_tap;
+  float* deq_tap;
+  float* z_tap;
 };
 
 // Shared-memory layout of one CTA: weight rows, norm gains (ngain vectors of k floats; kO also
@@ -340,6 +345,16 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
     }
   }
   __syncthreads();
+  if (a.q_tap != nullptr && cta == 0) {
+    // the codes every CTA formed, unscrambled from the piece-major layout
+    for (int j = 0; j < ng; ++j)
+      for (int e = threadIdx.x; e < NB * a.k; e += kThreads) {
+        const int r = e / a.k, kk = e - r * a.k;
+        a.q_tap[((size_t)j * NB + r) * a.k + kk] =
+            qs[(size_t)(j * NB + r) * kq + ((kk & 63) >> 4) * (kq >> 2) + (kk >> 6) * 16 + (kk & 15)];
+      }
+    if (threadIdx.x < ng * NB) a.deq_tap[threadIdx.x] = deqs[(threadIdx.x / NB) * kMaxRows + threadIdx.x % NB];
+  }
 
   if (!wait_or_leave(B.bar_w, B.par_w)) return false;
 
@@ -430,6 +445,12 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
       a.state[o] = hv;
       reinterpret_cast<float*>(a.y)[o] = hv;
       a.g_out[o] = zg;
+      if (a.z_tap != nullptr) {
+        float* zt = a.z_tap + (int64_t)r * 3 * a.nout + c0 + cl;
+        zt[0] = zi;
+        zt[a.nout] = zf;
+        zt[2 * (int64_t)a.nout] = zg;
+      }
     } else if (a.mode == kGate) {
       store_from_float(a.y, o, a.ydt, siluf_(zof(0)) * zof(1));
     } else {

@@ -1003,4 +1003,15 @@ __global__ void __launch_bounds__(256) embed_gather_kernel(const int32_t* __rest
   }
 }
 
+// Debug taps: dst[r][c] = float(src[r][c]) for r < rows, c < cols (row strides in elements).
+__global__ void __launch_bounds__(256) tap_to_f32_kernel(const void* __restrict__ src, mmf_dtype sdt, int64_t rows,
+                                                         int32_t cols, int64_t src_ld, float* __restrict__ dst,
+                                                         int64_t dst_ld) {
+  const int64_t total = rows * cols;
+  for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total; e += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = e / cols, c = e - r * cols;
+    dst[r * dst_ld + c] = load_as_float(src, r * src_ld + c, sdt);
+  }
+}
+
 }  // namespace mmf

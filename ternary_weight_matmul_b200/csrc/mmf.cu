@@ -72,12 +72,41 @@ inline int64_t row_q(int32_t k) { return 16 * (int64_t)row_words(k); }  // int8 
 // ---------------------------------------------------------------------------------------------
 struct DevInfo {
   bool init = false;
+  unsigned long long ctx_id = 0;  // the context the kernel attributes below were set in
   int sms = 0;
   int major = 0, minor = 0;
   bool tc_ready = false;
 };
 DevInfo g_dev[64];
 std::mutex g_dev_mu;
+
+// Unique id of the calling thread's current CUDA context (never reused within a process), or 0
+// when the driver cannot tell. A device reset ends the context, so per-context state (kernel
+// attributes, symbol addresses) is set up again when this id changes.
+typedef CUresult (*PfnCtxGetCurrent)(CUcontext*);
+typedef CUresult (*PfnCtxGetId)(CUcontext, unsigned long long*);
+unsigned long long current_ctx_id() {
+  static PfnCtxGetCurrent get_current = nullptr;
+  static PfnCtxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PfnCtxGetCurrent>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PfnCtxGetId>(fn);
+  });
+  if (!get_current || !get_id) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
 
 template <mmf_dtype ZT, mmf_dtype HT>
 cudaError_t scan_tile_attrs() {
@@ -95,6 +124,21 @@ cudaError_t scan_tile_attrs() {
   return e;
 }
 
+template <mmf_dtype XT, mmf_dtype TT>
+cudaError_t head_attrs() {
+  const int smem = 200 * 1024;
+  cudaError_t e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
+}
+cudaError_t head_tc_attrs() {
+  return cudaFuncSetAttribute(head::head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              head::tc_smem_bytes(head::kTcRowsMax));
+}
+
+
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 std::once_flag g_encode_once;
 
@@ -102,9 +146,15 @@ mmf_status device_info(DevInfo** out) {
   int dev = 0;
   MMF_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(MMF_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> lk(g_dev_mu);
   DevInfo& di = g_dev[dev];
+  if (di.init && ctx != 0) {
+    if (di.ctx_id == 0) di.ctx_id = ctx;          // set up before the context was current
+    else if (ctx != di.ctx_id) di = DevInfo();    // a new context (after a reset): set up again
+  }
   if (!di.init) {
+    di.ctx_id = ctx;
     MMF_CUDA(cudaDeviceGetAttribute(&di.sms, cudaDevAttrMultiProcessorCount, dev));
     MMF_CUDA(cudaDeviceGetAttribute(&di.major, cudaDevAttrComputeCapabilityMajor, dev));
     MMF_CUDA(cudaDeviceGetAttribute(&di.minor, cudaDevAttrComputeCapabilityMinor, dev));
@@ -133,6 +183,11 @@ mmf_status device_info(DevInfo** out) {
       MMF_CUDA((scan_tile_attrs<MMF_F32, MMF_BF16>()));
       MMF_CUDA((scan_tile_attrs<MMF_BF16, MMF_F32>()));
       MMF_CUDA((scan_tile_attrs<MMF_BF16, MMF_BF16>()));
+      MMF_CUDA((head_attrs<MMF_F32, MMF_F32>()));
+      MMF_CUDA((head_attrs<MMF_F32, MMF_BF16>()));
+      MMF_CUDA((head_attrs<MMF_BF16, MMF_F32>()));
+      MMF_CUDA((head_attrs<MMF_BF16, MMF_BF16>()));
+      MMF_CUDA(head_tc_attrs());
       di.tc_ready = true;
     }
     di.init = true;
@@ -696,20 +751,27 @@ mmf_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 // Device-side storage; in host code `g_noalloc_scratch` only names the symbol, so its device
 // address is looked up once per device with cudaGetSymbolAddress and passed to the kernels.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[MMF_NOALLOC_SCRATCH_BYTES];
+// Looked up once per device and context: a device reset ends the context, and the address is
+// looked up again in the next one.
 void* g_noalloc_ptr[64] = {};
+unsigned long long g_noalloc_ctx[64] = {};
 std::mutex g_noalloc_mu;
 
 mmf_status noalloc_scratch(void** out) {
   int dev = 0;
   MMF_CUDA(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return fail(MMF_ERR_UNSUPPORTED, "device ordinal %d out of range", dev);
+  const unsigned long long ctx = current_ctx_id();
   std::lock_guard<std::mutex> lk(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  if (g_noalloc_ptr[dev] == nullptr || (ctx != 0 && g_noalloc_ctx[dev] != 0 && ctx != g_noalloc_ctx[dev])) {
     void* p = nullptr;
     cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
     if (e != cudaSuccess || p == nullptr)
       return fail(MMF_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
     g_noalloc_ptr[dev] = p;
+    g_noalloc_ctx[dev] = ctx;
+  } else if (g_noalloc_ctx[dev] == 0) {
+    g_noalloc_ctx[dev] = ctx;
   }
   *out = g_noalloc_ptr[dev];
   return MMF_OK;
@@ -769,20 +831,6 @@ mmf_status head_tc_pass(const void* x, mmf_dtype xdt, int nb, int d, const float
   launch_k(head::head_argmax_kernel, dim3((unsigned)((nb + head::kWarps - 1) / head::kWarps)), dim3(head::kThreads), 0, st,
            (const float*)pmax, (const int32_t*)pidx, tiles, (int)head::kTcRowsMax, nb, ids);
   return MMF_OK;
-}
-
-template <mmf_dtype XT, mmf_dtype TT>
-cudaError_t head_attrs() {
-  const int smem = 200 * 1024;
-  cudaError_t e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e == cudaSuccess) e = cudaFuncSetAttribute(head::head_logits_kernel<XT, TT, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  return e;
-}
-cudaError_t head_tc_attrs() {
-  return cudaFuncSetAttribute(head::head_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              head::tc_smem_bytes(head::kTcRowsMax));
 }
 
 }  // namespace
@@ -992,6 +1040,10 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
   return MMF_OK;
 }
 
+}  // extern "C"
+
+namespace {
+
 // ---------------------------------------------------------------------------------------------
 // fused decode (up to 8 token rows on the CUDA-core engine): four launches per block
 // ---------------------------------------------------------------------------------------------
@@ -1041,10 +1093,34 @@ mmf_status launch_dec(dec::Args& a, const DevInfo& di, cudaStream_t st) {
   return check_launch("dec_proj_kernel");
 }
 
+mmf_status tap_copy(void* dst, const void* src, size_t bytes, cudaStream_t st) {
+  if (!dst || bytes == 0) return MMF_OK;
+  cudaError_t e = cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "taps copy: %s", cudaGetErrorString(e));
+  return MMF_OK;
+}
+mmf_status tap_copy2d(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width, size_t rows,
+                      cudaStream_t st) {
+  if (!dst || width == 0 || rows == 0) return MMF_OK;
+  cudaError_t e = cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, rows, cudaMemcpyDeviceToDevice, st);
+  if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "taps copy: %s", cudaGetErrorString(e));
+  return MMF_OK;
+}
+// dst[r][c] = float(src[r][c]) (debug taps).
+mmf_status tap_to_f32(float* dst, int64_t dst_ld, const void* src, mmf_dtype sdt, int64_t src_ld, int64_t rows,
+                      int32_t cols, cudaStream_t st) {
+  if (!dst || rows * cols == 0) return MMF_OK;
+  const int64_t blocks = std::min<int64_t>((rows * cols + 255) / 256, 4096);
+  launch_k(tap_to_f32_kernel, dim3((unsigned)blocks), dim3(256), 0, st, src, sdt, rows, cols, src_ld, dst, dst_ld);
+  return check_launch("tap_to_f32_kernel");
+}
+
 // One block, one token per row: x [b][d] -> y [b][d], state [b][d] updated in place. Scratch:
-// h and g (float32, [b][d]), x1 [b][d] and v [b][inner] (dtype).
+// h and g (float32, [b][d]), x1 [b][d] and v [b][inner] (dtype). `tp` (nullable) receives the
+// step's intermediates.
 mmf_status run_block_decode(const mmf_block_weights* w, const void* x, mmf_dtype dt, int32_t b, float* state,
-                            void* y, uint8_t* scratch, const DevInfo& di, cudaStream_t st) {
+                            void* y, uint8_t* scratch, const DevInfo& di, cudaStream_t st,
+                            const mmf_decode_taps* tp = nullptr) {
   const int32_t d = w->d, inner = w->inner;
   float* h32 = reinterpret_cast<float*>(scratch);
   float* g32 = reinterpret_cast<float*>(scratch + align256((size_t)b * d * 4));
@@ -1059,14 +1135,18 @@ mmf_status run_block_decode(const mmf_block_weights* w, const void* x, mmf_dtype
   a.sw[0] = w->i.scale; a.sw[1] = w->f.scale; a.sw[2] = w->g.scale;
   a.gain[0] = w->nw_i; a.gain[1] = w->nw_f; a.gain[2] = w->nw_g;
   a.x = x; a.y = h32; a.g_out = g32; a.state = state;
+  if (tp) { a.q_tap = tp->q_ifg; a.deq_tap = tp->deq_ifg; a.z_tap = tp->z; }
   MMF_TRY(launch_dec(a, di, st));
+  if (tp) MMF_TRY(tap_copy(tp->h, h32, (size_t)b * d * 4, st));
   // g_norm + o_proj + residual
   memset(&a, 0, sizeof(a));
   a.b = b; a.eps = w->eps; a.xdt = dt; a.ydt = dt;
   a.mode = dec::kO; a.k = d; a.kw = row_words(d); a.nout = d; a.nmat = 1; a.ngain = 1;
   a.w[0] = w->o.codes; a.sw[0] = w->o.scale; a.gain[0] = w->nw_o;
   a.h = h32; a.gin = g32; a.gnorm_w = w->gnorm_w; a.res = x; a.y = x1;
+  if (tp) { a.q_tap = tp->q_o; a.deq_tap = tp->deq_o; }
   MMF_TRY(launch_dec(a, di, st));
+  if (tp) MMF_TRY(tap_copy(tp->x1, x1, (size_t)b * d * dsize(dt), st));
   // gate_proj: v = SiLU(gate) * up
   memset(&a, 0, sizeof(a));
   a.b = b; a.eps = w->eps; a.xdt = dt; a.ydt = dt;
@@ -1074,14 +1154,43 @@ mmf_status run_block_decode(const mmf_block_weights* w, const void* x, mmf_dtype
   a.w[0] = w->gate.codes; a.w[1] = w->gate.codes; a.row_off[1] = inner;
   a.sw[0] = w->gate.scale; a.sw[1] = w->gate.scale; a.gain[0] = w->nw_gate;
   a.x = x1; a.y = v;
+  if (tp) { a.q_tap = tp->q_gate; a.deq_tap = tp->deq_gate; }
   MMF_TRY(launch_dec(a, di, st));
+  if (tp) MMF_TRY(tap_copy(tp->v, v, (size_t)b * inner * dsize(dt), st));
   // down_proj + residual
   memset(&a, 0, sizeof(a));
   a.b = b; a.eps = w->eps; a.xdt = dt; a.ydt = dt;
   a.mode = dec::kDown; a.k = inner; a.kw = row_words(inner); a.nout = d; a.nmat = 1; a.ngain = 1;
   a.w[0] = w->down.codes; a.sw[0] = w->down.scale; a.gain[0] = w->nw_down;
   a.x = v; a.res = x1; a.y = y;
-  return launch_dec(a, di, st);
+  if (tp) { a.q_tap = tp->q_down; a.deq_tap = tp->deq_down; }
+  MMF_TRY(launch_dec(a, di, st));
+  if (tp) MMF_TRY(tap_copy(tp->y, y, (size_t)b * d * dsize(dt), st));
+  return MMF_OK;
+}
+
+// The intermediates of one block path step (run_block with t = 1) into decode taps.
+mmf_status block_decode_taps(const mmf_block_weights* w, int32_t b, mmf_dtype dt, const BlockWs& W, const void* y,
+                             const mmf_decode_taps* tp, cudaStream_t st) {
+  const int64_t m = b;
+  const int32_t d = w->d, inner = w->inner;
+  const size_t es = dsize(dt);
+  MMF_TRY(tap_copy2d(tp->q_ifg, d, W.q3, row_q(d), d, 3 * m, st));
+  MMF_TRY(tap_copy(tp->deq_ifg, W.deq, 3 * m * 4, st));
+  for (int p = 0; p < 3; ++p)
+    MMF_TRY(tap_to_f32(tp->z ? tp->z + p * d : nullptr, 3 * (int64_t)d,
+                       reinterpret_cast<const uint8_t*>(W.z) + p * (size_t)m * d * es, dt, d, m, d, st));
+  MMF_TRY(tap_to_f32(tp->h, d, W.h, dt, d, m, d, st));
+  MMF_TRY(tap_copy2d(tp->q_o, d, W.qo, row_q(d), d, m, st));
+  MMF_TRY(tap_copy(tp->deq_o, W.deq + 3 * m, m * 4, st));
+  MMF_TRY(tap_copy(tp->x1, W.x1, m * d * es, st));
+  MMF_TRY(tap_copy2d(tp->q_gate, d, W.qg, row_q(d), d, m, st));
+  MMF_TRY(tap_copy(tp->deq_gate, W.deq + 4 * m, m * 4, st));
+  if (glu_fused(m, inner)) MMF_TRY(tap_copy(tp->v, W.gu, m * inner * es, st));
+  else MMF_TRY(tap_copy(tp->gu, W.gu, m * 2 * inner * es, st));
+  MMF_TRY(tap_copy2d(tp->q_down, inner, W.qd, row_q(inner), inner, m, st));
+  MMF_TRY(tap_copy(tp->deq_down, W.deq + 5 * m, m * 4, st));
+  return tap_copy(tp->y, y, m * d * es, st);
 }
 
 // The fused decode paths bulk-copy the norm gains: every gain vector must start on 16 bytes.
@@ -1095,9 +1204,9 @@ bool gains_aligned(const mmf_block_weights* layers, int32_t n_layers) {
   return true;
 }
 
-mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
-                           mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
-                           size_t ws_bytes, mmf_stream_t stream) {
+mmf_status decode_impl(const mmf_block_weights* layers, int32_t n_layers, const void* x, mmf_dtype dtype, int32_t b,
+                       float* state, void* y, const mmf_decode_taps* taps, void* ws, size_t ws_bytes,
+                       mmf_stream_t stream) {
   MMF_CHECK_ARG(layers != nullptr && n_layers > 0, "decode: no layers");
   MMF_CHECK_ARG(valid_dtype(dtype), "decode: bad dtype");
   MMF_CHECK_ARG(b >= 0, "decode: negative batch");
@@ -1123,11 +1232,33 @@ mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, co
   for (int l = 0; l < n_layers; ++l) {
     void* out = (l == n_layers - 1) ? y : buf[l & 1];
     float* st_l = state + (int64_t)l * b * d;
-    if (fused) MMF_TRY(run_block_decode(&layers[l], cur, dtype, b, st_l, out, reinterpret_cast<uint8_t*>(ws), *di, st));
-    else MMF_TRY(run_block(&layers[l], cur, dtype, b, 1, st_l, out, st_l, W, *di, st));
+    const mmf_decode_taps* tp = taps ? &taps[l] : nullptr;
+    if (fused) {
+      MMF_TRY(run_block_decode(&layers[l], cur, dtype, b, st_l, out, reinterpret_cast<uint8_t*>(ws), *di, st, tp));
+    } else {
+      MMF_TRY(run_block(&layers[l], cur, dtype, b, 1, st_l, out, st_l, W, *di, st));
+      if (tp) MMF_TRY(block_decode_taps(&layers[l], b, dtype, W, out, tp, st));
+    }
     cur = out;
   }
   return MMF_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
+                           mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
+                           size_t ws_bytes, mmf_stream_t stream) {
+  return decode_impl(layers, n_layers, x, dtype, b, state, y, nullptr, ws, ws_bytes, stream);
+}
+
+mmf_status mmf_decode_step_taps(const mmf_block_weights* layers, int32_t n_layers, const void* x,
+                                mmf_dtype dtype, int32_t b, float* state, void* y, const mmf_decode_taps* taps,
+                                void* ws, size_t ws_bytes, mmf_stream_t stream) {
+  MMF_CHECK_ARG(taps != nullptr, "decode taps: null taps");
+  return decode_impl(layers, n_layers, x, dtype, b, state, y, taps, ws, ws_bytes, stream);
 }
 
 mmf_status mmf_embed_gather(const int32_t* ids, int64_t m, const void* table, mmf_dtype dtype,
@@ -1164,19 +1295,6 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
   DevInfo* di;
   MMF_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  {
-    static std::once_flag once;
-    static cudaError_t attr_err = cudaSuccess;
-    std::call_once(once, [] {
-      cudaError_t e = head_attrs<MMF_F32, MMF_F32>();
-      if (e == cudaSuccess) e = head_attrs<MMF_F32, MMF_BF16>();
-      if (e == cudaSuccess) e = head_attrs<MMF_BF16, MMF_F32>();
-      if (e == cudaSuccess) e = head_attrs<MMF_BF16, MMF_BF16>();
-      if (e == cudaSuccess) e = head_tc_attrs();
-      attr_err = e;
-    });
-    if (attr_err != cudaSuccess) return fail(MMF_ERR_CUDA, "head attributes: %s", cudaGetErrorString(attr_err));
-  }
   const size_t parr = head_parts_bytes(vocab);
   float* pmax = reinterpret_cast<float*>(ws);
   int32_t* pidx = reinterpret_cast<int32_t*>(reinterpret_cast<uint8_t*>(ws) + parr);
@@ -1231,6 +1349,8 @@ mmf_status mmf_lm_head_argmax(const void* x, mmf_dtype x_dtype, int32_t b, int32
 mmf_status mmf_validate_packed(const mmf_ternary* w, unsigned long long* bad, mmf_stream_t stream) {
   MMF_CHECK_ARG(w != nullptr && w->codes != nullptr && bad != nullptr, "validate: null pointer");
   MMF_CHECK_ARG(w->n >= 0 && w->k >= 0, "validate: negative shape");
+  MMF_CHECK_ARG(aligned16(w->codes), "validate: codes not 16-byte aligned");
+  MMF_CHECK_ARG((reinterpret_cast<uintptr_t>(bad) & 7u) == 0, "validate: bad counter not 8-byte aligned");
   DevInfo* di;
   MMF_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);

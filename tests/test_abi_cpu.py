@@ -178,3 +178,19 @@ def test_validate_packed_arguments_on_host(L):
     assert L.mmf_validate_packed(ctypes.byref(t), None, None) == mmf.MMF_ERR_INVALID_ARG
     neg = mmf.Ternary(16, 32, -1, 64)
     assert L.mmf_validate_packed(ctypes.byref(neg), 16, None) == mmf.MMF_ERR_INVALID_ARG
+
+
+def test_validate_packed_alignment_on_host(L):
+    # misaligned codes (not 16 bytes) or counter (not 8 bytes) are refused before any CUDA call
+    good = ctypes.c_void_p(4096)
+    t = mmf.Ternary(4096 + 4, 32, 4, 64)
+    assert L.mmf_validate_packed(ctypes.byref(t), good, None) == mmf.MMF_ERR_INVALID_ARG
+    t = mmf.Ternary(4096, 32, 4, 64)
+    assert L.mmf_validate_packed(ctypes.byref(t), ctypes.c_void_p(4096 + 4), None) == mmf.MMF_ERR_INVALID_ARG
+
+
+def test_decode_taps_arguments_on_host(L):
+    assert L.mmf_decode_step_taps(None, 1, None, 0, 1, None, None, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    bw = mmf.BlockWeightsC()
+    assert L.mmf_decode_step_taps(ctypes.byref(bw), 1, None, 0, 1, None, None, None, None, 0, None) == \
+        mmf.MMF_ERR_INVALID_ARG
