@@ -4,11 +4,19 @@ Workload (default): the 370M-shape stack, prefill forward, 24 HGRNBit blocks of 
 MLP gate_proj 1024->5632 and down_proj 2816->1024, vocabulary 32000 embedding, bf16 activations,
 token ids uniform in [0, 32000) for batch 8 x sequence 2048 per GPU. Weights are random N(0, 0.02)
 latent weights ternarised and 2-bit packed by the library. One step = one forward of the whole
-stack (embedding gather + 24 blocks) over one batch.
+stack (embedding gather + 24 blocks) over one batch; the tied head is not part of the prefill
+step (it runs in the decode measurement, where generation needs it).
 
-Prints one JSON line (rank 0). --impl reference times the CPU oracle on a bounded sample of the
-same workload instead. Multi-GPU runs are independent replicas (one batch per rank, no
-collective on the data path); timing is the max over ranks.
+Prints one JSON line (rank 0). On one GPU the line also carries, as extra keys: the 2.7B-shape
+greedy decode at batch 1 / 8 / 64 (every rank, as replicas), the 1.3B-shape prefill, the kernel
+sweeps (BitLinear over three (K, N) shapes and five row counts; the HGRN scan at d 2048 up to
+T 65536), the next-row kernels (HGRN2 recurrence, scan and BitLinear gradients) and two CPU
+baselines (the oracle as written, and an fp32-BLAS restatement on every host core).
+
+--impl reference times the CPU oracle on a bounded sample of the same workload instead.
+--case NAME runs one kernel case a few times and prints its device time (profiler captures).
+Multi-GPU runs are independent replicas (one batch per rank, no collective on the data path);
+timing is the max over ranks.
 """
 from __future__ import annotations
 
@@ -25,19 +33,25 @@ sys.path.insert(0, ROOT)
 
 METRIC = "HGRNBit block-stack tokens/s (prefill & decode, 1 B200); % HBM / INT8 roofline"
 INT8_OVER_BF16 = 2.0  # nominal dense ratio: 4.5 POPS int8/fp8 vs 2.25 PFLOP/s bf16
+# CUDA-core float32 FMA peak: 148 SMs x 128 FMA/clk x 2 flop x 1.965 GHz (the listed unit counts
+# and the maximum SM clock)
+FP32_FMA_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
 
 WORKLOADS = {
     "prefill-370M": dict(d=1024, inner=2816, layers=24, vocab=32000, batch=8, seq=2048),
     "prefill-1.3B": dict(d=2048, inner=5632, layers=24, vocab=32000, batch=16, seq=2048),
 }
-# Autoregressive decode of the 2.7B-shape stack: a 512-token prompt (prefill, untimed) then
-# decode steps with the recurrent state carried per layer, at three batch sizes.
 # DRAM traffic of one ternary_gemm_tc_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum,
 # averaged over the 96 GEMM launches of one step) from an ncu capture of this bench's own workload;
 # valid only while the kernel source is the one captured (SHA-256 prefix), else reported as null.
 GEMM_TRAFFIC = {"prefill-370M": dict(bytes=78.3e6, algorithmic=115.2e6, sha256="14a6d8df0242cadf",
                                      profile="profiles/ternary_gemm_tc_kernel_prefill-370M_traffic.md")}
+# Autoregressive decode of the 2.7B-shape stack: a 512-token prompt (prefill, untimed) then
+# decode steps with the recurrent state carried per layer, at three batch sizes.
 DECODE = dict(name="decode-2.7B", d=2560, inner=7040, layers=32, vocab=32000, prompt=512, batches=(1, 8, 64))
+# Kernel sweeps (the pages' 1.3B layer shapes): BitLinear (K, N) x M, and the HGRN scan
+SWEEP_BITLINEAR = dict(kn=((2048, 2048), (2048, 11264), (5632, 2048)), m=(1, 16, 256, 4096, 32768))
+SWEEP_SCAN = dict(b=4, d=2048, t=(1024, 8192, 65536))
 
 
 def parse():
@@ -50,8 +64,48 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--decode-steps", type=int, default=64)
+    ap.add_argument("--no-extra", action="store_true", help="skip the 1.3B prefill, sweeps and next-row kernels")
+    ap.add_argument("--decode-steps", type=int, default=256)
+    ap.add_argument("--case", default=None,
+                    choices=["gemm", "scan", "block", "norm", "decode", "head", "hgrn2", "scan_bwd", "lin_bwd"],
+                    help="run one kernel case and print its device time (for profiler captures)")
+    ap.add_argument("--m", type=int, default=16384)
+    ap.add_argument("--n", type=int, default=5632)
+    ap.add_argument("--k", type=int, default=1024)
+    ap.add_argument("--b", type=int, default=4)
+    ap.add_argument("--t", type=int, default=8192)
+    ap.add_argument("--d", type=int, default=1024)
+    ap.add_argument("--inner", type=int, default=2816)
+    ap.add_argument("--layers", type=int, default=4)
+    ap.add_argument("--vocab", type=int, default=32000)
+    ap.add_argument("--heads", type=int, default=8)
+    ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
+    ap.add_argument("--iters", type=int, default=5)
+    ap.add_argument("--engine", default="auto", choices=["auto", "tensor", "simt"])
     return ap.parse_args()
+
+
+def load_peaks() -> dict:
+    pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(pp):
+        with open(pp) as fh:
+            return json.load(fh)
+    return {}
+
+
+def int8_peak(peaks: dict) -> tuple[float, str]:
+    """The int8 tensor peak for a kernel timed inside a step of milliseconds: the measured burst
+    bf16 cuBLAS figure x the nominal int8/bf16 ratio (no int8 GEMM is measured on this machine)."""
+    if peaks.get("bf16_tflops"):
+        return (peaks["bf16_tflops"] * INT8_OVER_BF16,
+                "of measured: bf16 burst cuBLAS x nominal int8/bf16 ratio 2 (the step lasts milliseconds)")
+    return 1590.0 * INT8_OVER_BF16, "of fallback: 1.59 PFLOP/s bf16 burst x nominal ratio 2"
+
+
+def hbm_peak(peaks: dict) -> tuple[float, str]:
+    if peaks.get("hbm_gbs"):
+        return peaks["hbm_gbs"], "of measured: STREAM-style copy"
+    return 6650.0, "of fallback: 6.65 TB/s"
 
 
 def gemm_traffic(workload: str):
@@ -103,7 +157,7 @@ def dist_env():
 
 
 # ---------------------------------------------------------------------------------------------
-# CPU oracle timing (reference arm and cpu_baseline)
+# CPU baselines: the oracle (reference arm and cpu_baseline) and an fp32-BLAS restatement
 # ---------------------------------------------------------------------------------------------
 _ORACLE_LAYER = {}
 
@@ -145,6 +199,58 @@ def oracle_threads() -> int:
     return 1  # the integer product and the scan loop run on one core; BLAS is not used
 
 
+def cpu_fast_tokens_per_s(wl: dict, tokens: int, seed: int = 0) -> tuple[float, str, float, int]:
+    """A fast CPU baseline (timing only; never called by the library): the block forward
+    restated with torch CPU tensors in float32 on every host core. The integer product runs as an
+    fp32 BLAS product of the int8 codes and the ternary codes, which is exact: every partial sum
+    is an integer of magnitude <= 127 * K < 2^24. The recurrence is a loop over time, vectorised
+    over the channels. One layer on one sequence of `tokens` tokens, extrapolated linearly to the
+    stack. Returns (tokens/s, description, seconds, threads)."""
+    import torch
+
+    threads = os.cpu_count() or 1
+    torch.set_num_threads(threads)
+    g = torch.Generator().manual_seed(seed)
+    d, inner, eps = wl["d"], wl["inner"], 1e-8
+    shapes = {"i": (d, d), "f": (d, d), "g": (d, d), "o": (d, d), "gate": (2 * inner, d), "down": (d, inner)}
+    lay = {}
+    for p, (n, k) in shapes.items():
+        w = torch.randn(n, k, generator=g) * 0.02
+        s = w.abs().mean().clamp_min(1e-5)
+        lay[p] = ((w / s).round().clamp(-1, 1).t().contiguous(), float(s))  # [K, N] float32 codes
+    x = torch.randn(1, tokens, d, generator=g)
+
+    def bitlinear(v, tt, s):
+        r = v * torch.rsqrt((v * v).mean(-1, keepdim=True) + eps)
+        a = r.abs().amax(-1, keepdim=True).clamp_min(1e-5)
+        q = torch.round(r * (127.0 / a)).clamp(-127, 127)
+        return (q @ tt) * (a / 127.0) * s
+
+    def block(v):
+        zi, zf, gg = (bitlinear(v, *lay[p]) for p in ("i", "f", "g"))
+        f = torch.sigmoid(zf)
+        i = torch.nn.functional.silu(zi) * (1 - f)
+        h = torch.empty_like(i)
+        prev = torch.zeros(v.shape[0], d)
+        for t in range(v.shape[1]):
+            prev = f[:, t] * prev + i[:, t]
+            h[:, t] = prev
+        u = h * torch.rsqrt((h * h).mean(-1, keepdim=True) + eps) * torch.nn.functional.silu(gg)
+        x1 = v + bitlinear(u, *lay["o"])
+        gu = bitlinear(x1, *lay["gate"])
+        vv = torch.nn.functional.silu(gu[..., :inner]) * gu[..., inner:]
+        return x1 + bitlinear(vv, *lay["down"])
+
+    block(x[:, :64])  # warm-up (thread pool, BLAS)
+    t0 = time.perf_counter()
+    block(x)
+    dt = time.perf_counter() - t0
+    desc = (f"torch CPU float32 restatement (fp32 BLAS on the int8 x ternary codes, exact; recurrence "
+            f"vectorised over d) of 1 of {wl['layers']} layers on 1 sequence of {tokens} tokens, "
+            f"extrapolated linearly to {wl['layers']} layers")
+    return tokens / (dt * wl["layers"]), desc, dt, threads
+
+
 def run_reference(args, wl):
     rank, world, _ = dist_env()
     if rank != 0:
@@ -163,6 +269,8 @@ def run_reference(args, wl):
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": per_step_stack * 1e3,
+        "ms_per_step_kind": (f"extrapolated: each step times 1 of {wl['layers']} layers on {tokens} tokens "
+                             f"and scales by {wl['layers']}; the stack itself is never run"),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64 / int64 (oracle)", "data": "synthetic",
         "config": {"workload": args.workload, **{k: wl[k] for k in ("d", "inner", "layers", "vocab")},
@@ -253,7 +361,27 @@ def build_model(wl, device, seed=1234):
     return blocks, table
 
 
-def run_decode(args, device, hbm_peak, world=1):
+def kernel_classes(mmf) -> dict:
+    """Per kernel class: launches, device ms and algorithmic work recorded since the last read."""
+    out = {}
+    for cls in ("gemm_tc", "gemm_simt", "norm_quant", "scan", "other"):
+        n, kms, work = mmf.timing_read(cls)
+        out[cls] = {"launches": n, "ms": kms, "work": work}
+    return out
+
+
+def hbm_breakdown(kern: dict, total_ms: float, hbm: float) -> dict:
+    out = {}
+    for cls in ("norm_quant", "scan", "gemm_simt", "other"):
+        k = kern[cls]
+        if k["launches"]:
+            gbs = k["work"] / (k["ms"] / 1e3) / 1e9
+            out[cls] = {"launches": k["launches"], "ms_total": k["ms"], "GB/s": gbs, "frac_hbm": gbs / hbm,
+                        "share_of_step": k["ms"] / total_ms}
+    return out
+
+
+def run_decode(args, device, hbm, world=1):
     """Greedy autoregressive decode throughput of the 2.7B-shape stack for each batch size: prompt
     prefill through mmf_stack_fwd (untimed; gives every layer's recurrent state and, through the
     final norm and the tied head, the first generated token), then `--decode-steps` generated
@@ -261,9 +389,10 @@ def run_decode(args, device, hbm_peak, world=1):
     tied head and argmax (mmf_lm_head_argmax writes the next ids in place), replayed from a CUDA
     graph (captured after warm-up) and timed with CUDA events on the replay stream. HBM roofline:
     every step streams all packed weights and the bf16 head table (once per pass of the head: one
-    row on the CUDA cores, up to 128 rows on the tensor cores). With several ranks every rank is
-    a replica generating for its own sequences; the ranks meet at a barrier before each timed
-    region and the step time is the slowest rank's."""
+    row on the CUDA cores, up to 128 rows on the tensor cores). Then a few steps run eagerly with
+    the library's per-launch events on, which attribute the step time to the kernel classes. With
+    several ranks every rank is a replica generating for its own sequences; the ranks meet at a
+    barrier before each timed region and the step time is the slowest rank's."""
     import torch
     import torch.distributed as dist
 
@@ -325,10 +454,255 @@ def run_decode(args, device, hbm_peak, world=1):
         step_bytes = weight_bytes + head_bytes * ((B + 127) // 128)
         ids_end = cur.cpu()
         assert int(ids_end.min()) >= 0 and int(ids_end.max()) < dw["vocab"]
-        out["batches"][str(B)] = decode_entry(B, ms, step_bytes, device, world, hbm_peak)
+        entry = decode_entry(B, ms, step_bytes, device, world, hbm)
+        # per-class attribution from a few eager steps with the library's launch events
+        kernel_classes(mmf)  # clear
+        n_eager = 4
+        with torch.cuda.stream(s):
+            mmf.timing_enable(True)
+            for i in range(n_eager):
+                step()
+            torch.cuda.synchronize(device)
+            mmf.timing_enable(False)
+        kern = kernel_classes(mmf)
+        cls_ms = {c: v["ms"] / n_eager for c, v in kern.items() if v["launches"]}
+        dom = max(cls_ms, key=cls_ms.get)
+        names = {"gemm_tc": "ternary_gemm_tc_kernel", "gemm_simt": "dec_proj_kernel / simt_gemm_kernel",
+                 "norm_quant": "norm_quant_vec_kernel", "scan": "scan kernels", "other": "head / gather kernels"}
+        gemm_ms = sum(cls_ms.get(c, 0.0) for c in ("gemm_tc", "gemm_simt"))
+        gemm_gbs = weight_bytes / (gemm_ms / 1e3) / 1e9 if gemm_ms > 0 else None
+        entry["roofline"] = {
+            "bound": "hbm", "dominant": names[dom], "dominant_ms_per_step": cls_ms[dom],
+            "launches_per_step": {c: kern[c]["launches"] / n_eager for c in kern if kern[c]["launches"]},
+            "ms_per_step_by_class": cls_ms,
+            "weight_products_ms_per_step": gemm_ms,
+            "weight_products_GB/s": gemm_gbs, "weight_products_frac_hbm": gemm_gbs / hbm if gemm_gbs else None,
+            "note": "class times from eager steps with per-launch events (launch gaps excluded); "
+                    "the step time above is the graph replay"}
+        out["batches"][str(B)] = entry
         del graph
     del blocks, table
     torch.cuda.empty_cache()
+    return out
+
+
+def time_prefill(wl, device, steps, warmup, flush, clocks=None):
+    """Device time of the block-stack prefill step over one batch (seeded ids), L2 flushed between
+    steps; returns (ms per step list, kernel classes, launches, ids_host, blocks, table, y)."""
+    import torch
+
+    import ternary_weight_matmul_b200 as mmf
+
+    rank = dist_env()[0]
+    blocks, table = build_model(wl, device)
+    B, T, d = wl["batch"], wl["seq"], wl["d"]
+    g = torch.Generator(device="cpu")
+    g.manual_seed(4321 + rank)
+    ids_host = torch.randint(0, wl["vocab"], (B, T), generator=g, dtype=torch.int32).pin_memory()
+    ids = ids_host.to(device)
+    y = torch.empty(B, T, d, dtype=torch.bfloat16, device=device)
+
+    def step():
+        mmf.stack_fwd(blocks, ids, table, out=y)
+
+    for _ in range(max(warmup, 3)):
+        flush.zero_()
+        step()
+    st = mmf.sync_status(device)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+    stream = torch.cuda.current_stream(device)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    return blocks, table, ids_host, y, step, stream, starts, ends
+
+
+def gemm_roofline(kern: dict, total_ms: float, peak: float, peak_src: str, workload: str | None) -> dict:
+    tc = kern["gemm_tc"]
+    achieved = (tc["work"] / (tc["ms"] / 1e3) / 1e12) if tc["ms"] > 0 else 0.0
+    r = {"bound": "tensor", "kernel": "ternary_gemm_tc_kernel", "achieved": achieved, "peak": peak,
+         "unit": "TOPS (int8)", "frac": achieved / peak, "peak_source": peak_src,
+         "launches": tc["launches"], "avg_launch_us": tc["ms"] / max(tc["launches"], 1) * 1e3,
+         "share_of_step": tc["ms"] / total_ms}
+    if workload is not None:
+        r.update({"traffic": gemm_traffic(workload),
+                  "traffic_source": GEMM_TRAFFIC.get(workload, {}).get("profile"),
+                  "algorithmic_bytes_per_launch": GEMM_TRAFFIC.get(workload, {}).get("algorithmic")})
+    return r
+
+
+def run_prefill_extra(wl_name, device, flush, peaks) -> dict:
+    """A second prefill workload (the 1.3B shape), device time only, as an extra key."""
+    import torch
+
+    import ternary_weight_matmul_b200 as mmf
+
+    wl = WORKLOADS[wl_name]
+    blocks, table, ids_host, y, step, stream, starts, ends = time_prefill(wl, device, 5, 3, flush)
+    mmf.timing_enable(True)
+    for i in range(5):
+        flush.zero_()
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    mmf.timing_enable(False)
+    if mmf.sync_status(device) != 0:
+        raise RuntimeError(f"device status after {wl_name}")
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    ms = statistics.mean(step_ms)
+    kern = kernel_classes(mmf)
+    peak, src = int8_peak(peaks)
+    hbm, _ = hbm_peak(peaks)
+    tokens = wl["batch"] * wl["seq"]
+    out = {"workload": wl_name, "value": tokens / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+           "steps": 5, "config": wl, "roofline": gemm_roofline(kern, ms * 5, peak, src, None),
+           "hbm_kernels": hbm_breakdown(kern, ms * 5, hbm)}
+    del blocks, table, y
+    torch.cuda.empty_cache()
+    return out
+
+
+def run_sweeps(device, flush, peaks) -> dict:
+    """Kernel sweeps: each BitLinear call (norm-quant + product) and each scan timed alone with CUDA
+    events, L2 flushed before every repetition; the median of the repetitions is reported against
+    its roofline (HBM bytes below the ridge, int8 ops above it)."""
+    import torch
+
+    import ternary_weight_matmul_b200 as mmf
+
+    peak, _ = int8_peak(peaks)
+    hbm, _ = hbm_peak(peaks)
+    g = torch.Generator(device=device)
+    g.manual_seed(77)
+    stream = torch.cuda.current_stream(device)
+    reps = 8
+
+    def median_ms(fn, classes=False):
+        times, kern_total = [], None
+        for r in range(reps + 2):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            if classes and r >= 2:
+                mmf.timing_enable(True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(device)
+            mmf.timing_enable(False)
+            if r >= 2:
+                times.append(a.elapsed_time(b))
+        if classes:
+            kern_total = kernel_classes(mmf)
+        return statistics.median(times), kern_total
+
+    bl = []
+    for k, n in SWEEP_BITLINEAR["kn"]:
+        w = mmf.pack_ternary(torch.randn(n, k, generator=g, device=device) * 0.02)
+        for m in SWEEP_BITLINEAR["m"]:
+            x = torch.randn(m, k, generator=g, device=device).to(torch.bfloat16)
+            yb = torch.empty(m, n, dtype=torch.bfloat16, device=device)
+            ms, kern = median_ms(lambda: mmf.bitlinear_fwd(x, None, w, y_dtype=torch.bfloat16), classes=True)
+            ops = 2.0 * m * n * k
+            byts = n * (k // 4) + 2.0 * m * k + 2.0 * m * n
+            e = {"K": k, "N": n, "M": m, "call_ms": ms, "call_TOPS": ops / (ms / 1e3) / 1e12,
+                 "call_GB/s": byts / (ms / 1e3) / 1e9}
+            gk = "gemm_tc" if kern["gemm_tc"]["launches"] else "gemm_simt"
+            gms = kern[gk]["ms"] / reps
+            e["product_kernel"] = "ternary_gemm_tc_kernel" if gk == "gemm_tc" else "simt_gemm_kernel"
+            e["product_ms"] = gms
+            if m <= 16:
+                gbs = (n * (k // 4) + m * k + 2.0 * m * n) / (gms / 1e3) / 1e9
+                e.update({"bound": "hbm", "product_GB/s": gbs, "frac": gbs / hbm})
+            else:
+                tops = ops / (gms / 1e3) / 1e12
+                e.update({"bound": "tensor", "product_TOPS": tops, "frac": tops / peak})
+            bl.append(e)
+            del x, yb
+        del w
+    torch.cuda.empty_cache()
+    sc = []
+    b, d = SWEEP_SCAN["b"], SWEEP_SCAN["d"]
+    for t in SWEEP_SCAN["t"]:
+        zf = torch.randn(b, t, d, generator=g, device=device).add_(4.0)
+        zi = torch.randn(b, t, d, generator=g, device=device)
+        ms, _ = median_ms(lambda: mmf.hgrn_scan(zf, zi, None, h_dtype=torch.float32))
+        byts = 12.0 * b * t * d
+        gbs = byts / (ms / 1e3) / 1e9
+        sc.append({"B": b, "T": t, "d": d, "dtype": "f32 in / f32 out", "ms": ms, "GB/s": gbs, "frac_hbm": gbs / hbm,
+                   "bytes": byts})
+        del zf, zi
+    torch.cuda.empty_cache()
+    return {"bitlinear": bl, "scan": sc, "reps": reps, "l2": "flushed before every repetition",
+            "activations": "N(0,1) bf16 (BitLinear); scan gates zf ~ N(4,1), zi ~ N(0,1) float32"}
+
+
+def run_next_rows(device, flush, peaks) -> dict:
+    """The next-row kernels timed alone (median of a few calls, L2 flushed before each): the HGRN2
+    recurrence (step by step on the CUDA cores), the scan gradients and the BitLinear gradients
+    (straight-through estimator, CUDA cores)."""
+    import torch
+
+    import ternary_weight_matmul_b200 as mmf
+
+    hbm, _ = hbm_peak(peaks)
+    g = torch.Generator(device=device)
+    g.manual_seed(88)
+    stream = torch.cuda.current_stream(device)
+
+    def median_ms(fn, reps=5):
+        ts = []
+        for r in range(reps + 1):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(device)
+            if r:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    out = {}
+    # HGRN2: 8 sequences x 2048 steps, 8 heads of dk = dv = 128 (hidden 1024), bf16
+    B, T, H, dk = 8, 2048, 8, 128
+    q = torch.randn(B, T, H, dk, generator=g, device=device).to(torch.bfloat16)
+    f = torch.sigmoid(torch.randn(B, T, H, dk, generator=g, device=device) + 2).to(torch.bfloat16)
+    i = torch.randn(B, T, H, dk, generator=g, device=device).to(torch.bfloat16)
+    ms = median_ms(lambda: mmf.hgrn2_recurrence(q, f, i))
+    flops = 4.0 * B * T * H * dk * dk   # per (step, head): dk x dv decay-and-add FMAs + the dk x dv readout
+    byts = 2.0 * B * T * H * (3 * dk)   # q, f, i in and o out in bf16 (q, f shared across columns)
+    out["hgrn2_recurrence"] = {"shape": f"B {B} T {T} heads {H} dk {dk} dv {dk} bf16", "ms": ms,
+                               "TFLOP/s": flops / (ms / 1e3) / 1e12,
+                               "frac_fp32_fma_peak": flops / (ms / 1e3) / 1e12 / FP32_FMA_TFLOPS,
+                               "GB/s": byts / (ms / 1e3) / 1e9, "bound": "alu",
+                               "peak_source": "CUDA-core fp32 FMA peak from unit counts x 1.965 GHz"}
+    del q, f, i
+    # scan backward: 8 x 2048 x 1024 bf16 (the 370M prefill shape)
+    B, T, d = 8, 2048, 1024
+    zf = torch.randn(B, T, d, generator=g, device=device).add_(2).to(torch.bfloat16)
+    zi = torch.randn(B, T, d, generator=g, device=device).to(torch.bfloat16)
+    h, _ = mmf.hgrn_scan(zf, zi, None, h_dtype=torch.bfloat16)
+    dh = torch.randn(B, T, d, generator=g, device=device).to(torch.bfloat16)
+    ms = median_ms(lambda: mmf.hgrn_scan_backward(zf, zi, h, dh))
+    byts = 6.0 * 2 * B * T * d
+    out["hgrn_scan_backward"] = {"shape": f"B {B} T {T} d {d} bf16", "ms": ms, "GB/s": byts / (ms / 1e3) / 1e9,
+                                 "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm, "bound": "hbm"}
+    del zf, zi, h, dh
+    # BitLinear backward: 4096 rows, K = N = 1024, bf16 activations and gradients
+    m, k, n = 4096, 1024, 1024
+    w = mmf.pack_ternary(torch.randn(n, k, generator=g, device=device) * 0.02)
+    x = torch.randn(m, k, generator=g, device=device).to(torch.bfloat16)
+    nw = torch.ones(k, device=device)
+    _, qq, deq, _ = mmf.bitlinear_fwd(x, nw, w, y_dtype=torch.float32, debug=True)
+    dy = torch.randn(m, n, generator=g, device=device).to(torch.bfloat16)
+    ms = median_ms(lambda: mmf.bitlinear_backward(x, nw, w, qq, deq, dy))
+    flops = 2 * 2.0 * m * n * k   # dr and dW
+    out["bitlinear_backward"] = {"shape": f"M {m} K {k} N {n} bf16", "ms": ms, "TFLOP/s": flops / (ms / 1e3) / 1e12,
+                                 "frac_fp32_fma_peak": flops / (ms / 1e3) / 1e12 / FP32_FMA_TFLOPS,
+                                 "bound": "alu", "peak_source": "CUDA-core fp32 FMA peak from unit counts x 1.965 GHz"}
+    if mmf.sync_status(device) != 0:
+        raise RuntimeError("device status after the next-row kernels")
     return out
 
 
@@ -345,30 +719,13 @@ def run_gpu(args, wl):
         dist.init_process_group("nccl", device_id=device, timeout=__import__("datetime").timedelta(seconds=300))
 
     mmf.lib()
-    blocks, table = build_model(wl, device)
-    B, T, d = wl["batch"], wl["seq"], wl["d"]
-    g = torch.Generator(device="cpu")
-    g.manual_seed(4321 + rank)
-    ids_host = torch.randint(0, wl["vocab"], (B, T), generator=g, dtype=torch.int32).pin_memory()
-    ids = ids_host.to(device)
-    y = torch.empty(B, T, d, dtype=torch.bfloat16, device=device)
+    peaks = load_peaks()
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
     flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=device)
-
-    def step():
-        mmf.stack_fwd(blocks, ids, table, out=y)
-
-    for _ in range(max(args.warmup, 3)):
-        flush.zero_()
-        step()
-    st = mmf.sync_status(device)
-    if st != 0:
-        raise RuntimeError(f"device status {st} after warm-up")
+    blocks, table, ids_host, y, step, stream, starts, ends = time_prefill(wl, device, args.steps, args.warmup, flush)
+    B, T, d = wl["batch"], wl["seq"], wl["d"]
 
     # ---------------- timed region (device time, events on the launching stream)
-    stream = torch.cuda.current_stream(device)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     clocks = Clocks(local)
     if world > 1:
         dist.barrier()
@@ -394,15 +751,9 @@ def run_gpu(args, wl):
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     ms = sum(step_ms) / len(step_ms)
     ms_max = max_over_ranks(ms, device, world)
-    tokens = B * T * world
     value = replicas_throughput(B * T, world, ms_max)
-
-    kern = {}
-    for cls in ("gemm_tc", "gemm_simt", "norm_quant", "scan", "other"):
-        n, kms, work = mmf.timing_read(cls)
-        kern[cls] = {"launches": n, "ms": kms, "work": work}
-    # our kernels launched per step: timing scopes count launches (pack uses none here)
-    gpu_launches = int(launches)
+    kern = kernel_classes(mmf)
+    gpu_launches = int(launches)  # our kernels launched in the timed region (timing scopes count them)
 
     # ---------------- end to end through the public API with host buffers
     e2e = None
@@ -424,48 +775,33 @@ def run_gpu(args, wl):
         e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)) / args.steps
         e2e = {"value": replicas_throughput(B * T, world, max_over_ranks(e_ms, device, world)), "unit": "tokens/s",
                "h2d_bytes_per_step": ids_host.numel() * 4, "d2h_bytes_per_step": y_host.numel() * 2}
+    del blocks, table, y
+    torch.cuda.empty_cache()
 
+    hbm, hbm_src = hbm_peak(peaks)
     decode = None
     if not args.no_decode:  # every rank: decode replicas, timed as the slowest rank
-        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
-        hbm = json.load(open(pp)).get("hbm_gbs", 6650.0) if os.path.exists(pp) else 6650.0
         decode = run_decode(args, device, hbm, world)
+
+    extra = {}
+    if world == 1 and not args.no_extra:
+        extra["prefill-1.3B"] = run_prefill_extra("prefill-1.3B", device, flush, peaks)
+        extra["sweeps"] = run_sweeps(device, flush, peaks)
+        extra["next_rows"] = run_next_rows(device, flush, peaks)
 
     line = None
     if rank == 0:
-        peaks = {}
-        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
-        if os.path.exists(pp):
-            with open(pp) as fh:
-                peaks = json.load(fh)
-        if peaks.get("bf16_tflops_sustained"):
-            int8_peak = peaks["bf16_tflops_sustained"] * INT8_OVER_BF16
-            peak_src = "of measured: bf16 sustained cuBLAS x nominal int8/bf16 ratio 2"
-        else:
-            int8_peak = 1400.0 * INT8_OVER_BF16
-            peak_src = "of fallback: 1.4 PFLOP/s bf16 sustained x nominal ratio 2"
-        hbm_peak = peaks.get("hbm_gbs", 6650.0)
-        tc = kern["gemm_tc"]
-        achieved = (tc["work"] / (tc["ms"] / 1e3) / 1e12) if tc["ms"] > 0 else 0.0
-        roofline = {"bound": "tensor", "kernel": "ternary_gemm_tc_kernel", "achieved": achieved,
-                    "peak": int8_peak, "unit": "TOPS (int8)", "frac": achieved / int8_peak,
-                    "peak_source": peak_src, "traffic": gemm_traffic(args.workload),
-                    "traffic_source": GEMM_TRAFFIC.get(args.workload, {}).get("profile"),
-                    "algorithmic_bytes_per_launch": GEMM_TRAFFIC.get(args.workload, {}).get("algorithmic"),
-                    "launches": tc["launches"], "avg_launch_us": tc["ms"] / max(tc["launches"], 1) * 1e3,
-                    "share_of_step": tc["ms"] / (ms * args.steps)}
-        hbm_kernels = {}
-        for cls in ("norm_quant", "scan", "gemm_simt", "other"):
-            k = kern[cls]
-            if k["launches"]:
-                gbs = k["work"] / (k["ms"] / 1e3) / 1e9
-                hbm_kernels[cls] = {"launches": k["launches"], "ms_total": k["ms"], "GB/s": gbs,
-                                    "frac_hbm": gbs / hbm_peak, "share_of_step": k["ms"] / (ms * args.steps)}
-        cpu = None
+        peak, peak_src = int8_peak(peaks)
+        roofline = gemm_roofline(kern, ms * args.steps, peak, peak_src, args.workload)
+        hbm_kernels = hbm_breakdown(kern, ms * args.steps, hbm)
+        cpu = cpu_fast = None
         if not args.no_cpu_baseline and world == 1:
             v, desc, dt = oracle_sample_tokens_per_s(wl, 1024)
             cpu = {"value": v, "unit": "tokens/s", "cores": oracle_threads(), "kind": "oracle",
                    "sample": desc + f" ({dt:.1f} s)", "host_cpus": os.cpu_count()}
+            v, desc, dt, thr = cpu_fast_tokens_per_s(wl, 2048)
+            cpu_fast = {"value": v, "unit": "tokens/s", "cores": thr, "kind": "fp32 BLAS restatement (exact)",
+                        "sample": desc + f" ({dt:.2f} s)", "host_cpus": os.cpu_count()}
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_max, "higher_is_better": True, "scaling": "weak",
@@ -474,12 +810,13 @@ def run_gpu(args, wl):
             "config": {"workload": args.workload, "model": "HGRNBit stack (random init)",
                        "global_batch": B * world, "seq_len": T, "hidden": d, "inner": wl["inner"],
                        "layers": wl["layers"], "vocab": wl["vocab"], "parallelism": f"replicas x{world}",
+                       "head": "excluded (block stack only; the tied head runs in the decode measurement)",
                        "l2": "flushed between steps (write of a 2x-L2 buffer, untimed)"},
-            "roofline": roofline, "hbm_kernels": hbm_kernels, "hbm_peak_gbs": hbm_peak,
-            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": gpu_launches,
+            "roofline": roofline, "hbm_kernels": hbm_kernels, "hbm_peak_gbs": hbm, "hbm_peak_source": hbm_src,
+            "cpu_baseline": cpu, "cpu_baseline_fast": cpu_fast, "e2e": e2e, "gpu_launches": gpu_launches,
             "gpu_launches_per_step": gpu_launches / args.steps, "clocks": clk,
             "step_ms_all": [round(v, 4) for v in step_ms],
-            "decode": decode,
+            "decode": decode, **extra,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -488,8 +825,137 @@ def run_gpu(args, wl):
     return 0
 
 
+# ---------------------------------------------------------------------------------------------
+# one kernel case (profiler captures and quick timing)
+# ---------------------------------------------------------------------------------------------
+def run_case(a) -> int:
+    """Runs one kernel case `--iters` times after two warm-up calls and prints the mean device time
+    per call (CUDA events). Inputs are seeded and synthetic (weights N(0, 0.02), activations
+    N(0, 1)). Examples:
+        python bench.py --case gemm --m 16384 --n 5632 --k 1024
+        python bench.py --case scan --b 8 --t 2048 --d 1024
+        python bench.py --case block --m 16384 --d 1024 --inner 2816
+        python bench.py --case decode --b 1 --d 2560 --inner 7040 --layers 4
+        python bench.py --case head --b 8 --d 2560 --vocab 32000 --iters 1
+    """
+    import torch
+
+    import ternary_weight_matmul_b200 as mmf
+
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    dt = torch.bfloat16 if a.dtype == "bf16" else torch.float32
+    g = torch.Generator(device=dev)
+    g.manual_seed(0)
+    mmf.set_gemm_path({"auto": mmf.MMF_GEMM_AUTO, "tensor": mmf.MMF_GEMM_TENSOR, "simt": mmf.MMF_GEMM_SIMT}[a.engine])
+
+    def blocks_of(d, inner, layers):
+        shapes = {"i": (d, d), "f": (d, d), "g": (d, d), "o": (d, d), "gate": (2 * inner, d), "down": (d, inner)}
+        out = []
+        for _ in range(layers):
+            packed = {p: mmf.pack_ternary(torch.randn(n, k, generator=g, device=dev) * 0.02) for p, (n, k) in shapes.items()}
+            norms = {f"nw_{p}": torch.ones(k, device=dev) for p, (n, k) in shapes.items()}
+            norms["gnorm_w"] = torch.ones(d, device=dev)
+            out.append(mmf.Block(d, inner, packed, norms))
+        return out
+
+    if a.case == "gemm":
+        w = mmf.pack_ternary(torch.randn(a.n, a.k, generator=g, device=dev) * 0.02)
+        x = torch.randn(a.m, a.k, generator=g, device=dev).to(dt)
+
+        def run():
+            return mmf.bitlinear_fwd(x, None, w, y_dtype=dt)
+        work, unit = 2.0 * a.m * a.n * a.k, "TOPS"
+    elif a.case == "scan":
+        zf = torch.randn(a.b, a.t, a.d, generator=g, device=dev).add_(4.0).to(dt)
+        zi = torch.randn(a.b, a.t, a.d, generator=g, device=dev).to(dt)
+        es = 4 if dt == torch.float32 else 2
+
+        def run():
+            return mmf.hgrn_scan(zf, zi, None, h_dtype=dt)
+        work, unit = float(a.b * a.t * a.d * 3 * es), "GB/s"
+    elif a.case == "norm":
+        x = torch.randn(a.m, a.k, generator=g, device=dev).to(dt)
+        w = mmf.pack_ternary(torch.randn(64, a.k, generator=g, device=dev) * 0.02)
+
+        def run():
+            return mmf.bitlinear_fwd(x, None, w, y_dtype=dt)
+        work, unit = float(a.m * a.k * (x.element_size() + 1)), "GB/s (norm part only)"
+    elif a.case == "decode":
+        blocks = blocks_of(a.d, a.inner, a.layers)
+        x = torch.randn(a.b, a.d, generator=g, device=dev).to(dt)
+        state = torch.zeros(a.layers, a.b, a.d, device=dev)
+        y = torch.empty_like(x)
+
+        def run():
+            return mmf.decode_step(blocks, x, state, out=y)
+        wbytes = sum(p.codes.numel() * 4 for blk in blocks for p in blk.packed.values())
+        work, unit = float(wbytes), "GB/s (packed weights)"
+    elif a.case == "head":
+        table = (torch.randn(a.vocab, a.d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
+        nw = torch.ones(a.d, device=dev)
+        x = torch.randn(a.b, a.d, generator=g, device=dev).to(dt)
+        ids = torch.empty(a.b, dtype=torch.int32, device=dev)
+
+        def run():
+            return mmf.lm_head_argmax(x, nw, table, ids_out=ids)
+        work, unit = float(table.numel() * 2 * ((a.b + 127) // 128 if a.b >= 2 else 1)), "GB/s (table)"
+    elif a.case == "hgrn2":
+        dk = a.d // a.heads
+        q = torch.randn(a.b, a.t, a.heads, dk, generator=g, device=dev).to(dt)
+        f = torch.sigmoid(torch.randn(a.b, a.t, a.heads, dk, generator=g, device=dev) + 2).to(dt)
+        i = torch.randn(a.b, a.t, a.heads, dk, generator=g, device=dev).to(dt)
+
+        def run():
+            return mmf.hgrn2_recurrence(q, f, i)
+        work, unit = 4.0 * a.b * a.t * a.heads * dk * dk, "TFLOP/s (fp32 FMA)"
+    elif a.case == "scan_bwd":
+        zf = torch.randn(a.b, a.t, a.d, generator=g, device=dev).add_(2.0).to(dt)
+        zi = torch.randn(a.b, a.t, a.d, generator=g, device=dev).to(dt)
+        h, _ = mmf.hgrn_scan(zf, zi, None, h_dtype=dt)
+        dh = torch.randn(a.b, a.t, a.d, generator=g, device=dev).to(dt)
+
+        def run():
+            return mmf.hgrn_scan_backward(zf, zi, h, dh)
+        work, unit = float(6 * a.b * a.t * a.d * (4 if dt == torch.float32 else 2)), "GB/s"
+    elif a.case == "lin_bwd":
+        w = mmf.pack_ternary(torch.randn(a.n, a.k, generator=g, device=dev) * 0.02)
+        x = torch.randn(a.m, a.k, generator=g, device=dev).to(dt)
+        nw = torch.ones(a.k, device=dev)
+        _, qq, deq, _ = mmf.bitlinear_fwd(x, nw, w, y_dtype=torch.float32, debug=True)
+        dy = torch.randn(a.m, a.n, generator=g, device=dev).to(dt)
+
+        def run():
+            return mmf.bitlinear_backward(x, nw, w, qq, deq, dy)
+        work, unit = 4.0 * a.m * a.n * a.k, "TFLOP/s (dr + dW)"
+    else:  # block
+        blk = blocks_of(a.d, a.inner, 1)[0]
+        x = torch.randn(1, a.m, a.d, generator=g, device=dev).to(dt)
+
+        def run():
+            return mmf.block_fwd(blk, x)
+        work, unit = 2.0 * a.m * (4 * a.d * a.d + 3 * a.d * a.inner), "TOPS (GEMM ops / block time)"
+
+    for _ in range(2):
+        run()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(a.iters):
+        run()
+    e.record()
+    torch.cuda.synchronize()
+    st = mmf.sync_status(dev)
+    ms = s.elapsed_time(e) / a.iters
+    rate = work / (ms / 1e3) / (1e12 if "TOPS" in unit or "TFLOP" in unit else 1e9)
+    print(f"{a.case}: {ms:.4f} ms/iter, {rate:.1f} {unit}, status {st}")
+    return 0 if st == 0 else 1
+
+
 def main():
     args = parse()
+    if args.case:
+        return run_case(args)
     wl = WORKLOADS[args.workload]
     if args.impl == "reference":
         return run_reference(args, wl)
