@@ -82,6 +82,7 @@ def parse():
     ap.add_argument("--dtype", default="bf16", choices=["bf16", "f32"])
     ap.add_argument("--iters", type=int, default=5)
     ap.add_argument("--engine", default="auto", choices=["auto", "tensor", "simt"])
+    ap.add_argument("--decode-path", default="auto", choices=["auto", "fused", "skinny", "block"])
     return ap.parse_args()
 
 
@@ -467,10 +468,15 @@ def run_decode(args, device, hbm, world=1):
         kern = kernel_classes(mmf)
         cls_ms = {c: v["ms"] / n_eager for c, v in kern.items() if v["launches"]}
         dom = max(cls_ms, key=cls_ms.get)
-        names = {"gemm_tc": "ternary_gemm_tc_kernel", "gemm_simt": "dec_proj_kernel / simt_gemm_kernel",
-                 "norm_quant": "norm_quant_vec_kernel", "scan": "scan kernels", "other": "head / gather kernels"}
+        path = {mmf.MMF_DECODE_FUSED: "fused", mmf.MMF_DECODE_SKINNY: "skinny",
+                mmf.MMF_DECODE_BLOCK: "block"}.get(mmf.decode_path(B, dw["d"], dw["inner"]), "?")
+        names = {"gemm_tc": "ternary_gemm_skinny_kernel" if path == "skinny" else "ternary_gemm_tc_kernel",
+                 "gemm_simt": "dec_proj_kernel" if path == "fused" else "simt_gemm_kernel",
+                 "norm_quant": "row_stage_kernel" if path == "skinny" else "norm_quant_vec_kernel",
+                 "scan": "scan kernels", "other": "head / gather kernels"}
         gemm_ms = sum(cls_ms.get(c, 0.0) for c in ("gemm_tc", "gemm_simt"))
         gemm_gbs = weight_bytes / (gemm_ms / 1e3) / 1e9 if gemm_ms > 0 else None
+        entry["path"] = path
         entry["roofline"] = {
             "bound": "hbm", "dominant": names[dom], "dominant_ms_per_step": cls_ms[dom],
             "launches_per_step": {c: kern[c]["launches"] / n_eager for c in kern if kern[c]["launches"]},
@@ -848,6 +854,8 @@ def run_case(a) -> int:
     g = torch.Generator(device=dev)
     g.manual_seed(0)
     mmf.set_gemm_path({"auto": mmf.MMF_GEMM_AUTO, "tensor": mmf.MMF_GEMM_TENSOR, "simt": mmf.MMF_GEMM_SIMT}[a.engine])
+    mmf.set_decode_path({"auto": mmf.MMF_DECODE_AUTO, "fused": mmf.MMF_DECODE_FUSED, "skinny": mmf.MMF_DECODE_SKINNY,
+                         "block": mmf.MMF_DECODE_BLOCK}[a.decode_path])
 
     def blocks_of(d, inner, layers):
         shapes = {"i": (d, d), "f": (d, d), "g": (d, d), "o": (d, d), "gate": (2 * inner, d), "down": (d, inner)}
@@ -890,7 +898,7 @@ def run_case(a) -> int:
         def run():
             return mmf.decode_step(blocks, x, state, out=y)
         wbytes = sum(p.codes.numel() * 4 for blk in blocks for p in blk.packed.values())
-        work, unit = float(wbytes), "GB/s (packed weights)"
+        work, unit = float(wbytes), f"GB/s (packed weights; path {mmf.decode_path(a.b, a.d, a.inner)})"
     elif a.case == "head":
         table = (torch.randn(a.vocab, a.d, generator=g, device=dev) * 0.02).to(torch.bfloat16)
         nw = torch.ones(a.d, device=dev)
@@ -940,11 +948,26 @@ def run_case(a) -> int:
         run()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
-    for _ in range(a.iters):
-        run()
-    e.record()
-    torch.cuda.synchronize()
+    if a.case in ("decode", "head"):
+        # replayed from a CUDA graph, as the decode measurement runs it (no host launch costs)
+        cs = torch.cuda.Stream()
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=cs):
+            run()
+        with torch.cuda.stream(cs):
+            graph.replay()
+            torch.cuda.synchronize()
+            s.record(cs)
+            for _ in range(a.iters):
+                graph.replay()
+            e.record(cs)
+        torch.cuda.synchronize()
+    else:
+        s.record()
+        for _ in range(a.iters):
+            run()
+        e.record()
+        torch.cuda.synchronize()
     st = mmf.sync_status(dev)
     ms = s.elapsed_time(e) / a.iters
     rate = work / (ms / 1e3) / (1e12 if "TOPS" in unit or "TFLOP" in unit else 1e9)

@@ -200,11 +200,9 @@ mmf_status mmf_block_fwd_taps(const mmf_block_weights* w, const void* x, mmf_dty
  *   state   [n_layers][b][d] float32, read and overwritten in place.
  *   y       [b][d] dtype: hidden state leaving the last layer (may not alias x).
  *   ws >= mmf_workspace_bytes(MMF_OP_DECODE, b, d, inner, n_layers).
- * With b in {1, 2, 4} rows (CUDA-core engine or MMF_GEMM_AUTO) or 8 rows (CUDA-core engine
- * only; MMF_GEMM_AUTO gives 8 rows to the tensor-core engine), d and inner multiples of 8
- * and 16-byte aligned norm gains, each block runs as four fused launches (norm + quantisation
- * of the input inside each, the products, and the gates / recurrence step / residual / GLU in
- * their epilogues); otherwise as the block path with t = 1. Same arithmetic either way. */
+ * Which kernels run is set by mmf_set_decode_path (below): four fused CUDA-core launches per
+ * block, four skinny tensor-core products each followed by a row stage, or the block path with
+ * t = 1. Same arithmetic either way. */
 mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
                            mmf_dtype dtype, int32_t b, float* state, void* y, void* ws,
                            size_t ws_bytes, mmf_stream_t stream);
@@ -377,6 +375,27 @@ const char* mmf_last_error(void);
  * Both produce identical int32 accumulators; tests use this to check each on every shape. */
 typedef enum { MMF_GEMM_AUTO = 0, MMF_GEMM_TENSOR = 1, MMF_GEMM_SIMT = 2 } mmf_gemm_path;
 mmf_status mmf_set_gemm_path(mmf_gemm_path path);
+
+/* Which kernels a decode step (mmf_decode_step) runs (process-wide, not thread-safe):
+ *   MMF_DECODE_AUTO    the fused CUDA-core path for 1 or 2 rows, the skinny tensor-core path
+ *                      for 3 to 64 rows, the block path above (default); with the CUDA-core engine
+ *                      (mmf_set_gemm_path) the fused path for 1, 2, 4 or 8 rows and the block path
+ *                      otherwise; with the tensor-core engine the block path;
+ *   MMF_DECODE_FUSED   four fused CUDA-core launches per block (1, 2, 4 or 8 rows, d and inner
+ *                      multiples of 8; other counts take the block path);
+ *   MMF_DECODE_SKINNY  per block four skinny tensor-core products into exact int32 accumulators
+ *                      (narrow token tiles of 16 / 32 / 64, K split across a thread-block cluster
+ *                      and reduced through distributed shared memory), each followed by a row
+ *                      stage that applies the product's epilogue and quantises the next input
+ *                      (1 to 64 rows, d and inner multiples of 8 up to 8192, 16-byte aligned
+ *                      norm gains; otherwise the block path);
+ *   MMF_DECODE_BLOCK   the prefill block forward with t = 1 (norm-quant, GEMM, scan kernels).
+ * All paths compute the same arithmetic; tests use this to check each. */
+typedef enum { MMF_DECODE_AUTO = 0, MMF_DECODE_FUSED = 1, MMF_DECODE_SKINNY = 2, MMF_DECODE_BLOCK = 3 } mmf_decode_path;
+mmf_status mmf_set_decode_path(mmf_decode_path path);
+/* The path (MMF_DECODE_FUSED / SKINNY / BLOCK) a decode step of b rows takes under the current
+ * settings, or -1 for sizes that are not positive. */
+int32_t mmf_decode_path_for(int32_t b, int32_t d, int32_t inner);
 
 /* Wall-clock cap, in microseconds, of every bounded in-kernel wait (default 2,000,000 = 2 s;
  * 0 restores the default), measured on the GPU's global timer. Lowering it makes waits run out

@@ -23,6 +23,7 @@ MMF_OK, MMF_ERR_INVALID_ARG, MMF_ERR_UNSUPPORTED, MMF_ERR_WORKSPACE, MMF_ERR_CUD
 MMF_F32, MMF_BF16 = 0, 1
 MMF_OP_PACK, MMF_OP_BITLINEAR, MMF_OP_BLOCK, MMF_OP_DECODE, MMF_OP_STACK, MMF_OP_SCAN, MMF_OP_HEAD = range(7)
 MMF_GEMM_AUTO, MMF_GEMM_TENSOR, MMF_GEMM_SIMT = range(3)
+MMF_DECODE_AUTO, MMF_DECODE_FUSED, MMF_DECODE_SKINNY, MMF_DECODE_BLOCK = range(4)
 
 EXPORTED = (
     "mmf_packed_row_words", "mmf_packed_words", "mmf_workspace_bytes", "mmf_pack_ternary",
@@ -31,7 +32,7 @@ EXPORTED = (
     "mmf_bitlinear_backward", "mmf_validate_packed",
     "mmf_stack_fwd", "mmf_sync_status", "mmf_status_string", "mmf_last_error",
     "mmf_set_gemm_path", "mmf_set_wait_limit", "mmf_launch_count", "mmf_timing_enable", "mmf_timing_read",
-    "mmf_bitlinear_fwd_noalloc", "mmf_decode_step_taps",
+    "mmf_bitlinear_fwd_noalloc", "mmf_decode_step_taps", "mmf_set_decode_path", "mmf_decode_path_for",
 )
 NOALLOC_SCRATCH_BYTES = 8 << 20
 
@@ -112,6 +113,8 @@ def lib() -> ctypes.CDLL:
         "mmf_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         "mmf_last_error": (ctypes.c_char_p, []),
         "mmf_set_gemm_path": (ctypes.c_int, [ctypes.c_int]),
+        "mmf_set_decode_path": (ctypes.c_int, [ctypes.c_int]),
+        "mmf_decode_path_for": (i32, [i32, i32, i32]),
         "mmf_set_wait_limit": (ctypes.c_int, [ctypes.c_uint32]),
         "mmf_launch_count": (ctypes.c_uint64, []),
         "mmf_timing_enable": (ctypes.c_int, [ctypes.c_int]),
@@ -461,10 +464,20 @@ def decode_step_taps(blocks: list[Block], x: torch.Tensor, state: torch.Tensor):
     return y, taps
 
 
+def decode_path(b: int, d: int, inner: int) -> int:
+    """mmf_decode_path_for: the path (MMF_DECODE_FUSED / SKINNY / BLOCK) a decode step of b rows
+    takes under the current settings."""
+    return int(lib().mmf_decode_path_for(b, d, inner))
+
+
+def set_decode_path(path: int) -> None:
+    """mmf_set_decode_path: MMF_DECODE_AUTO, _FUSED, _SKINNY or _BLOCK (process-wide)."""
+    _check(lib().mmf_set_decode_path(path), "mmf_set_decode_path")
+
+
 def decode_fused(b: int, d: int, inner: int) -> bool:
-    """Whether a decode step of b rows takes the fused four-launch path (engine choice as set)."""
-    tensor = _gemm_path == MMF_GEMM_TENSOR or (_gemm_path == MMF_GEMM_AUTO and b >= 8)
-    return b in (1, 2, 4, 8) and not tensor and d % 8 == 0 and inner % 8 == 0
+    """Whether a decode step of b rows takes the fused four-launch CUDA-core path."""
+    return decode_path(b, d, inner) == MMF_DECODE_FUSED
 
 
 def embed_gather(ids: torch.Tensor, table: torch.Tensor) -> torch.Tensor:

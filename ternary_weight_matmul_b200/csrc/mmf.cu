@@ -16,6 +16,8 @@
 
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_rows.cuh"
+#include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "head.cuh"
 #include "hgrn2.cuh"
@@ -29,6 +31,7 @@ namespace {
 
 thread_local std::string g_last_error;
 std::atomic<int> g_gemm_path{MMF_GEMM_AUTO};
+std::atomic<int> g_decode_path{MMF_DECODE_AUTO};
 constexpr uint32_t kDefaultWaitLimit = 2000000u;  // microseconds
 std::atomic<uint32_t> g_wait_limit{kDefaultWaitLimit};
 
@@ -188,6 +191,12 @@ mmf_status device_info(DevInfo** out) {
       MMF_CUDA((head_attrs<MMF_BF16, MMF_F32>()));
       MMF_CUDA((head_attrs<MMF_BF16, MMF_BF16>()));
       MMF_CUDA(head_tc_attrs());
+      MMF_CUDA(cudaFuncSetAttribute(sk::ternary_gemm_skinny_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    sk::Layout<16>::SMEM));
+      MMF_CUDA(cudaFuncSetAttribute(sk::ternary_gemm_skinny_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    sk::Layout<32>::SMEM));
+      MMF_CUDA(cudaFuncSetAttribute(sk::ternary_gemm_skinny_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    sk::Layout<64>::SMEM));
       di.tc_ready = true;
     }
     di.init = true;
@@ -736,6 +745,132 @@ mmf_status run_block(const mmf_block_weights* w, const void* x, mmf_dtype dt, in
   return launch_gemm(g, di, st);
 }
 
+// Workspace carve-up of one decode step on the skinny tensor-core path (b <= 64 rows): the
+// integer products of the current group, the codes and factors of the four quantisations, x1 and v.
+struct SkWs {
+  int32_t* acc;  // [b][max(3d, 2I)]
+  int8_t* q3;    // [3][b][ldq_d]
+  int8_t* qo;    // [b][ldq_d]
+  int8_t* qg;    // [b][ldq_d]
+  int8_t* qd;    // [b][ldq_I]
+  float* deq;    // [6][b]
+  void* x1;      // [b][d]
+  void* v;       // [b][I]
+  size_t bytes;
+};
+SkWs sk_ws(void* base, int64_t m, int32_t d, int32_t inner) {
+  SkWs w;
+  uint8_t* p = reinterpret_cast<uint8_t*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    uint8_t* r = p ? p + off : nullptr;
+    off += align256(bytes);
+    return r;
+  };
+  w.acc = reinterpret_cast<int32_t*>(take((size_t)m * std::max(3 * d, 2 * inner) * 4));
+  w.q3 = reinterpret_cast<int8_t*>(take(3 * m * row_q(d)));
+  w.qo = reinterpret_cast<int8_t*>(take(m * row_q(d)));
+  w.qg = reinterpret_cast<int8_t*>(take(m * row_q(d)));
+  w.qd = reinterpret_cast<int8_t*>(take(m * row_q(inner)));
+  w.deq = reinterpret_cast<float*>(take(6 * m * sizeof(float)));
+  w.x1 = take((size_t)m * d * 4);
+  w.v = take((size_t)m * inner * 4);
+  w.bytes = off;
+  return w;
+}
+// Bytes of a decode step's workspace before its two layer-output buffers: the largest of the
+// block path's, the skinny path's (the fused path uses a prefix of either).
+size_t decode_ws_head(int64_t m, int32_t d, int32_t inner) {
+  return std::max(block_ws(nullptr, m, d, inner, MMF_F32).bytes, sk_ws(nullptr, m, d, inner).bytes);
+}
+
+struct SkSeg {
+  const int8_t* q;        // [m][ldq] codes
+  const uint32_t* codes;  // [n][kw] packed weights
+  int32_t n;
+  int32_t* acc;           // acc[row * ldacc + col]
+};
+
+// acc = q . t^T for m <= 64 rows on the skinny tensor-core kernel (one launch, up to three
+// segments sharing m, k and the accumulator stride).
+mmf_status launch_skinny(const SkSeg* segs, int nseg, int64_t m, int32_t k, int64_t ldq, int64_t ldacc,
+                         const DevInfo& di, cudaStream_t st) {
+  if (m == 0) return MMF_OK;
+  if (m > 64) return fail(MMF_ERR_UNSUPPORTED, "skinny product: %lld rows (at most 64)", (long long)m);
+  sk::Params P;
+  memset(&P, 0, sizeof(P));
+  const int bn = m <= 16 ? 16 : (m <= 32 ? 32 : 64);
+  const int32_t kw = row_words(k);
+  int32_t tiles = 0;
+  for (int s = 0; s < nseg; ++s) {
+    P.tile_start[s] = tiles;
+    tiles += (segs[s].n + sk::BM - 1) / sk::BM;
+    MMF_TRY(encode_2d(&P.act_map[s], CU_TENSOR_MAP_DATA_TYPE_UINT8, segs[s].q, (uint64_t)ldq, (uint64_t)m,
+                      (uint64_t)ldq, 128, (uint32_t)bn, CU_TENSOR_MAP_SWIZZLE_128B));
+    MMF_TRY(encode_2d(&P.w_map[s], CU_TENSOR_MAP_DATA_TYPE_UINT32, segs[s].codes, (uint64_t)kw, (uint64_t)segs[s].n,
+                      (uint64_t)kw * 4, sk::W_WORDS_PER_ROW, sk::BM, CU_TENSOR_MAP_SWIZZLE_64B));
+    P.acc[s] = segs[s].acc;
+    P.n[s] = segs[s].n;
+  }
+  P.tile_start[nseg] = tiles;
+  P.nseg = nseg;
+  P.m = (int32_t)m;
+  P.ldacc = ldacc;
+  P.num_kb = (int32_t)((ldq + sk::BK - 1) / sk::BK);
+  // the largest power-of-two split (<= 8) that keeps one CTA per SM and at least one k-block each
+  int splits = 1;
+  while (splits * 2 <= sk::MAX_SPLITS && tiles * splits * 2 <= di.sms && splits * 2 <= P.num_kb) splits *= 2;
+  P.splits = splits;
+  P.kb_per_split = (P.num_kb + splits - 1) / splits;
+  P.wait_limit_us = g_wait_limit.load();
+  double ops = 0;
+  for (int s = 0; s < nseg; ++s) ops += 2.0 * (double)m * segs[s].n * k;
+  LaunchScope ls(MMF_KERNEL_GEMM_TC, ops, st);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)(tiles * splits));
+  cfg.blockDim = dim3(sk::NUM_THREADS);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = splits > 1 ? 2 : 1;
+  if (bn == 16) {
+    cfg.dynamicSmemBytes = sk::Layout<16>::SMEM;
+    cudaLaunchKernelEx(&cfg, sk::ternary_gemm_skinny_kernel<16>, P);
+  } else if (bn == 32) {
+    cfg.dynamicSmemBytes = sk::Layout<32>::SMEM;
+    cudaLaunchKernelEx(&cfg, sk::ternary_gemm_skinny_kernel<32>, P);
+  } else {
+    cfg.dynamicSmemBytes = sk::Layout<64>::SMEM;
+    cudaLaunchKernelEx(&cfg, sk::ternary_gemm_skinny_kernel<64>, P);
+  }
+  return check_launch("ternary_gemm_skinny_kernel");
+}
+
+mmf_status launch_row_stage(const drow::Args& a, int64_t b, cudaStream_t st) {
+  const int kv = (a.mode == drow::kGate) ? a.inner : a.d;
+  const double es = a.dt == MMF_F32 ? 4.0 : 2.0;
+  LaunchScope ls(MMF_KERNEL_NORM_QUANT, (double)b * kv * (es + 4.0 + a.ngain), st);
+  cudaLaunchConfig_t cfg;
+  memset(&cfg, 0, sizeof(cfg));
+  cfg.gridDim = dim3((unsigned)b);
+  cfg.blockDim = dim3(drow::kThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, drow::row_stage_kernel, a);
+  return check_launch("row_stage_kernel");
+}
+
 mmf_status check_ws(void* ws, size_t ws_bytes, size_t need) {
   if (need == 0) return MMF_OK;
   if (ws == nullptr || ws_bytes < need)
@@ -861,6 +996,7 @@ size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32
     case MMF_OP_HEAD:
       return inner > 0 ? head_ws_bytes(inner, d) : 0;
     case MMF_OP_DECODE:
+      return decode_ws_head(m, d, inner) + 2 * align256((size_t)m * d * 4);
     case MMF_OP_STACK:
       return block_ws(nullptr, m, d, inner, MMF_F32).bytes + 2 * align256((size_t)m * d * 4);
   }
@@ -1193,6 +1329,112 @@ mmf_status block_decode_taps(const mmf_block_weights* w, int32_t b, mmf_dtype dt
   return tap_copy(tp->y, y, m * d * es, st);
 }
 
+// The quantisation of a decode step's input with layer w's three i / f / g gains (row stage).
+mmf_status sk_quant_in(const mmf_block_weights* w, const void* x, mmf_dtype dt, int32_t b, const SkWs& S,
+                       cudaStream_t st) {
+  drow::Args a;
+  memset(&a, 0, sizeof(a));
+  a.mode = drow::kQuantIn; a.d = w->d; a.inner = w->inner; a.eps = w->eps; a.dt = dt; a.x = x;
+  a.ngain = 3; a.ldq = row_q(w->d);
+  a.gain[0] = w->nw_i; a.gain[1] = w->nw_f; a.gain[2] = w->nw_g;
+  for (int j = 0; j < 3; ++j) { a.q[j] = S.q3 + (int64_t)j * b * a.ldq; a.deq[j] = S.deq + j * b; }
+  return launch_row_stage(a, b, st);
+}
+
+// One block of a decode step on the skinny tensor-core path: four products (each one launch of
+// the skinny kernel into exact int32 accumulators) and four row stages (the products' epilogues:
+// gates and the recurrence step, residuals, GLU; each quantising the next product's input). The
+// codes of x for this layer are in S.q3 / S.deq[0..3b) on entry; on exit they hold the codes of y
+// for `next` (the following layer, or none). `tp` (nullable) receives the intermediates.
+mmf_status run_block_decode_sk(const mmf_block_weights* w, const mmf_block_weights* next, const void* x,
+                               mmf_dtype dt, int32_t b, float* state, void* y, const SkWs& S, const DevInfo& di,
+                               cudaStream_t st, const mmf_decode_taps* tp) {
+  const int32_t d = w->d, inner = w->inner;
+  const int64_t ldq_d = row_q(d), ldq_i = row_q(inner);
+  const size_t es = dsize(dt);
+  if (tp) {
+    MMF_TRY(tap_copy2d(tp->q_ifg, d, S.q3, ldq_d, d, 3 * (size_t)b, st));
+    MMF_TRY(tap_copy(tp->deq_ifg, S.deq, 3 * (size_t)b * 4, st));
+  }
+  // i / f / g products: acc = [zi | zf | g] accumulators
+  SkSeg g3[3] = {{S.q3, w->i.codes, d, S.acc},
+                 {S.q3 + (int64_t)b * ldq_d, w->f.codes, d, S.acc + d},
+                 {S.q3 + 2 * (int64_t)b * ldq_d, w->g.codes, d, S.acc + 2 * d}};
+  MMF_TRY(launch_skinny(g3, 3, b, d, ldq_d, 3 * (int64_t)d, di, st));
+  drow::Args a;
+  memset(&a, 0, sizeof(a));
+  a.mode = drow::kIFG; a.d = d; a.inner = inner; a.eps = w->eps; a.dt = dt; a.acc = S.acc; a.ldacc = 3 * (int64_t)d;
+  a.deq_in[0] = S.deq; a.deq_in[1] = S.deq + b; a.deq_in[2] = S.deq + 2 * b;
+  a.sw[0] = w->i.scale; a.sw[1] = w->f.scale; a.sw[2] = w->g.scale;
+  a.state = state; a.gnorm_w = w->gnorm_w;
+  a.ngain = 1; a.gain[0] = w->nw_o; a.q[0] = S.qo; a.ldq = ldq_d; a.deq[0] = S.deq + 3 * b;
+  if (tp) { a.z_tap = tp->z; a.h_tap = tp->h; }
+  MMF_TRY(launch_row_stage(a, b, st));
+  if (tp) {
+    MMF_TRY(tap_copy2d(tp->q_o, d, S.qo, ldq_d, d, b, st));
+    MMF_TRY(tap_copy(tp->deq_o, S.deq + 3 * b, (size_t)b * 4, st));
+  }
+  // o_proj, then x1 = x + o and gate_proj's codes
+  SkSeg go = {S.qo, w->o.codes, d, S.acc};
+  MMF_TRY(launch_skinny(&go, 1, b, d, ldq_d, d, di, st));
+  memset(&a, 0, sizeof(a));
+  a.mode = drow::kO; a.d = d; a.inner = inner; a.eps = w->eps; a.dt = dt; a.acc = S.acc; a.ldacc = d;
+  a.deq_in[0] = S.deq + 3 * b; a.sw[0] = w->o.scale; a.res = x; a.out = S.x1;
+  a.ngain = 1; a.gain[0] = w->nw_gate; a.q[0] = S.qg; a.ldq = ldq_d; a.deq[0] = S.deq + 4 * b;
+  MMF_TRY(launch_row_stage(a, b, st));
+  if (tp) {
+    MMF_TRY(tap_copy(tp->x1, S.x1, (size_t)b * d * es, st));
+    MMF_TRY(tap_copy2d(tp->q_gate, d, S.qg, ldq_d, d, b, st));
+    MMF_TRY(tap_copy(tp->deq_gate, S.deq + 4 * b, (size_t)b * 4, st));
+  }
+  // gate_proj ([gate | up] accumulators), then v = SiLU(gate) * up and down_proj's codes
+  SkSeg gg = {S.qg, w->gate.codes, 2 * inner, S.acc};
+  MMF_TRY(launch_skinny(&gg, 1, b, d, ldq_d, 2 * (int64_t)inner, di, st));
+  memset(&a, 0, sizeof(a));
+  a.mode = drow::kGate; a.d = d; a.inner = inner; a.eps = w->eps; a.dt = dt; a.acc = S.acc; a.ldacc = 2 * (int64_t)inner;
+  a.deq_in[0] = S.deq + 4 * b; a.sw[0] = w->gate.scale; a.out = S.v;
+  a.ngain = 1; a.gain[0] = w->nw_down; a.q[0] = S.qd; a.ldq = ldq_i; a.deq[0] = S.deq + 5 * b;
+  MMF_TRY(launch_row_stage(a, b, st));
+  if (tp) {
+    MMF_TRY(tap_copy(tp->v, S.v, (size_t)b * inner * es, st));
+    MMF_TRY(tap_copy2d(tp->q_down, inner, S.qd, ldq_i, inner, b, st));
+    MMF_TRY(tap_copy(tp->deq_down, S.deq + 5 * b, (size_t)b * 4, st));
+  }
+  // down_proj, then y = x1 + down and the next layer's input codes
+  SkSeg gd = {S.qd, w->down.codes, d, S.acc};
+  MMF_TRY(launch_skinny(&gd, 1, b, inner, ldq_i, d, di, st));
+  memset(&a, 0, sizeof(a));
+  a.mode = drow::kDown; a.d = d; a.inner = inner; a.eps = w->eps; a.dt = dt; a.acc = S.acc; a.ldacc = d;
+  a.deq_in[0] = S.deq + 5 * b; a.sw[0] = w->down.scale; a.res = S.x1; a.out = y;
+  if (next) {
+    a.ngain = 3; a.ldq = ldq_d;
+    a.gain[0] = next->nw_i; a.gain[1] = next->nw_f; a.gain[2] = next->nw_g;
+    for (int j = 0; j < 3; ++j) { a.q[j] = S.q3 + (int64_t)j * b * ldq_d; a.deq[j] = S.deq + j * b; }
+  }
+  MMF_TRY(launch_row_stage(a, b, st));
+  if (tp) MMF_TRY(tap_copy(tp->y, y, (size_t)b * d * es, st));
+  return MMF_OK;
+}
+
+// Which decode path a step of b rows takes (the automatic choice and the forced ones).
+enum DecodePath { kDecFused = 0, kDecSkinny = 1, kDecBlock = 2 };
+int decode_path_for(int32_t b, int32_t d, int32_t inner) {
+  const int p = g_decode_path.load();
+  const bool sk_ok = b >= 1 && b <= 64 && d <= drow::kMaxK && inner <= drow::kMaxK && d % 8 == 0 && inner % 8 == 0;
+  if (p == MMF_DECODE_SKINNY) return sk_ok ? kDecSkinny : kDecBlock;
+  if (p == MMF_DECODE_BLOCK) return kDecBlock;
+  if (p == MMF_DECODE_FUSED) return (b == 1 || b == 2 || b == 4 || b == 8) && d % 8 == 0 && inner % 8 == 0 ? kDecFused
+                                                                                                              : kDecBlock;
+  // automatic: the engine setting first (the CUDA-core engine keeps the fused path, the
+  // tensor-core engine the block path), then the row count. Measured on the 2.7B shape (8 layers,
+  // graph replay): fused 0.244 ms at 1 row against 0.377 ms skinny; skinny 0.373 / 0.468 ms at
+  // 8 / 64 rows against 0.52 / 0.53 ms on the block path.
+  if (g_gemm_path.load() == MMF_GEMM_SIMT) return decode_fused(b, d, inner) ? kDecFused : kDecBlock;
+  if (g_gemm_path.load() == MMF_GEMM_TENSOR) return kDecBlock;
+  if ((b == 1 || b == 2) && d % 8 == 0 && inner % 8 == 0) return kDecFused;
+  return sk_ok ? kDecSkinny : kDecBlock;
+}
+
 // The fused decode paths bulk-copy the norm gains: every gain vector must start on 16 bytes.
 bool gains_aligned(const mmf_block_weights* layers, int32_t n_layers) {
   for (int l = 0; l < n_layers; ++l) {
@@ -1224,16 +1466,22 @@ mmf_status decode_impl(const mmf_block_weights* layers, int32_t n_layers, const 
   MMF_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const BlockWs W = block_ws(ws, b, d, inner, dtype);
-  uint8_t* pp = reinterpret_cast<uint8_t*>(ws) + W.bytes;
+  const SkWs S = sk_ws(ws, b, d, inner);
+  uint8_t* pp = reinterpret_cast<uint8_t*>(ws) + decode_ws_head(b, d, inner);
   void* buf[2] = {pp, pp + align256((size_t)b * d * 4)};
   const void* cur = x;
-  // the input rows and the gains are bulk-copied
-  const bool fused = decode_fused(b, d, inner) && al16(x) && gains_aligned(layers, n_layers);
+  int path = decode_path_for(b, d, inner);
+  // the fused path bulk-copies the input rows and the gains; the row stages read gains as float4
+  if ((path == kDecFused || path == kDecSkinny) && !(al16(x) && gains_aligned(layers, n_layers))) path = kDecBlock;
+  if (path == kDecSkinny) MMF_TRY(sk_quant_in(&layers[0], x, dtype, b, S, st));
   for (int l = 0; l < n_layers; ++l) {
     void* out = (l == n_layers - 1) ? y : buf[l & 1];
     float* st_l = state + (int64_t)l * b * d;
     const mmf_decode_taps* tp = taps ? &taps[l] : nullptr;
-    if (fused) {
+    if (path == kDecSkinny) {
+      MMF_TRY(run_block_decode_sk(&layers[l], l + 1 < n_layers ? &layers[l + 1] : nullptr, cur, dtype, b, st_l, out,
+                                  S, *di, st, tp));
+    } else if (path == kDecFused) {
       MMF_TRY(run_block_decode(&layers[l], cur, dtype, b, st_l, out, reinterpret_cast<uint8_t*>(ws), *di, st, tp));
     } else {
       MMF_TRY(run_block(&layers[l], cur, dtype, b, 1, st_l, out, st_l, W, *di, st));
@@ -1537,6 +1785,19 @@ const char* mmf_status_string(mmf_status s) {
 }
 
 const char* mmf_last_error(void) { return g_last_error.c_str(); }
+
+mmf_status mmf_set_decode_path(mmf_decode_path path) {
+  if (path != MMF_DECODE_AUTO && path != MMF_DECODE_FUSED && path != MMF_DECODE_SKINNY && path != MMF_DECODE_BLOCK)
+    return fail(MMF_ERR_INVALID_ARG, "bad decode path %d", (int)path);
+  g_decode_path.store(path);
+  return MMF_OK;
+}
+
+int32_t mmf_decode_path_for(int32_t b, int32_t d, int32_t inner) {
+  if (b <= 0 || d <= 0 || inner <= 0) return -1;
+  return decode_path_for(b, d, inner) == kDecFused ? MMF_DECODE_FUSED
+         : decode_path_for(b, d, inner) == kDecSkinny ? MMF_DECODE_SKINNY : MMF_DECODE_BLOCK;
+}
 
 mmf_status mmf_set_gemm_path(mmf_gemm_path path) {
   if (path != MMF_GEMM_AUTO && path != MMF_GEMM_TENSOR && path != MMF_GEMM_SIMT)

@@ -1,8 +1,9 @@
 """GPU parity at the model widths the measurements run (the pages' model table: 370M d 1024 /
 I 2816, 1.3B d 2048 / I 5632, 2.7B d 2560 / I 7040), through the C ABI.
 
-* Decode: two layers of the 2.7B width at batch 1, 2, 4 (the fused four-launch path) and 8, 64
-  (the block path), float32 and bf16: every stage of every layer against the oracle's definition
+* Decode: two layers of the 2.7B width at batch 1 to 64 on each decode path (the fused CUDA-core
+  launches, the skinny tensor-core products with their row stages, the block path), float32 and
+  bf16: every stage of every layer against the oracle's definition
   applied to the kernel's own inputs to that stage (mmf_decode_step_taps), the second layer fed
   the first layer's output as the kernels produced it; then the whole step against the oracle's
   own two-layer step.
@@ -67,9 +68,14 @@ def _layers(mmf, d, inner, n, seed):
     return _LAYERS[key]
 
 
-@pytest.mark.parametrize("b,dtype", [(1, "f32"), (1, "bf16"), (2, "f32"), (4, "bf16"), (8, "f32"), (8, "bf16"),
-                                     (64, "bf16"), (64, "f32")])
-def test_decode_step_full_width_stages(mmf, b, dtype):
+PATHS = {"auto": 0, "fused": 1, "skinny": 2, "block": 3}
+DECODE_CASES = [(1, "f32", "auto"), (1, "bf16", "auto"), (2, "f32", "auto"), (4, "bf16", "auto"), (8, "f32", "auto"),
+                (64, "f32", "auto"), (1, "f32", "skinny"), (3, "bf16", "skinny"), (17, "f32", "skinny"),
+                (33, "bf16", "skinny"), (8, "bf16", "block"), (64, "f32", "block")]
+
+
+@pytest.mark.parametrize("b,dtype,path", DECODE_CASES)
+def test_decode_step_full_width_stages(mmf, b, dtype, path):
     d, inner = 2560, 7040
     bf16 = dtype == "bf16"
     tdt = torch.bfloat16 if bf16 else torch.float32
@@ -78,22 +84,31 @@ def test_decode_step_full_width_stages(mmf, b, dtype):
     if bf16:
         x = _bf16_round(x)
     state0 = synth.activations(511 + b, (2, b, d)) * 0.5
-    st = _to(state0)
-    y, taps = mmf.decode_step_taps([c[1] for c in layers], _to(x, tdt), st)
-    _ok(mmf)
-    fused = mmf.decode_fused(b, d, inner)
-    assert fused == (b in (1, 2, 4))
+    mmf.set_decode_path(PATHS[path])
+    try:
+        taken = mmf.decode_path(b, d, inner)
+        st = _to(state0)
+        y, taps = mmf.decode_step_taps([c[1] for c in layers], _to(x, tdt), st)
+        _ok(mmf)
+        # the step without taps runs the same kernels: bit-identical output and state
+        st2 = _to(state0)
+        y2 = mmf.decode_step([c[1] for c in layers], _to(x, tdt), st2)
+        _ok(mmf)
+    finally:
+        mmf.set_decode_path(mmf.MMF_DECODE_AUTO)
+    if path == "auto":
+        assert taken == (mmf.MMF_DECODE_FUSED if b in (1, 2) else mmf.MMF_DECODE_SKINNY)
+    else:
+        assert taken == PATHS[path]
+    assert torch.equal(y, y2) and torch.equal(st, st2)
     st_g = st.cpu().numpy()
     x_in = x.astype(np.float64)
     for l, (qp, _) in enumerate(layers):
-        y_l = check_decode_layer(x_in, state0[l], st_g[l], qp, taps[l], bf16, z_rounded=bf16 and not fused)
+        # the block path stores z and h in the activation dtype; the others keep them in float32
+        y_l = check_decode_layer(x_in, state0[l], st_g[l], qp, taps[l], bf16,
+                                 z_rounded=bf16 and taken == mmf.MMF_DECODE_BLOCK)
         x_in = y_l
     assert np.array_equal(_np(taps[-1]["y"]), _np(y))
-    # the step without taps runs the same kernels: bit-identical output and state
-    st2 = _to(state0)
-    y2 = mmf.decode_step([c[1] for c in layers], _to(x, tdt), st2)
-    _ok(mmf)
-    assert torch.equal(y, y2) and torch.equal(st, st2)
     # end to end against the oracle's own two-layer step. float32: rows whose code decisions all
     # match the oracle's elementwise (output and both states), every other row's first differing
     # code a near-tie. bf16: the kernels store every intermediate in bf16 and the oracle none, so
@@ -106,7 +121,7 @@ def test_decode_step_full_width_stages(mmf, b, dtype):
     else:
         rel, frac = check_chain_end_to_end(x[:, None, :], [c[0] for c in layers], taps, _np(y), st_g,
                                            h0s=state0.astype(np.float64))
-    print(f"decode full width b={b} {dtype} fused={fused}: rel L2 y {rel:.3e}, clean rows {frac:.2f}")
+    print(f"decode full width b={b} {dtype} path={taken}: rel L2 y {rel:.3e}, clean rows {frac:.2f}")
 
 
 @pytest.mark.parametrize("d,inner,b,t,dtype", [(1024, 2816, 2, 96, "f32"), (1024, 2816, 2, 96, "bf16"),

@@ -462,6 +462,37 @@ def test_head_wait_cap_ends_and_recovers(mmf):
     np.testing.assert_allclose(logits.cpu().numpy(), ref, rtol=1e-4, atol=1e-4 * scale)
 
 
+def test_decode_skinny_wait_cap_ends_and_recovers(mmf):
+    # the skinny tensor-core decode (8 rows: cluster split-K products and row stages) under a 1 us
+    # cap on every in-kernel wait: every launch ends (an abandoned CTA still joins its cluster's
+    # barriers), the step reports MMF_ERR_TIMEOUT or is right, and the next step at the default
+    # cap is right
+    layers = [_block_case(mmf, 75 + l, 256, 704) for l in range(2)]
+    blocks = [c[2] for c in layers]
+    x = _to(synth.activations(76, (8, 256)))
+    state0 = _to(synth.activations(77, (2, 8, 256)) * 0.5)
+    y_ref, st_ref = O.decode_step(_np(x).astype(np.float64), [c[1] for c in layers], _np(state0).astype(np.float64))
+    mmf.set_decode_path(mmf.MMF_DECODE_SKINNY)
+    try:
+        st = state0.clone()
+        mmf.set_wait_limit(1)
+        try:
+            y = mmf.decode_step(blocks, x, st)
+            status = mmf.sync_status(DEV)
+        finally:
+            mmf.set_wait_limit(0)
+        assert status in (mmf.MMF_OK, mmf.MMF_ERR_TIMEOUT)
+        if status == mmf.MMF_OK:
+            assert np.linalg.norm(_np(y) - y_ref) / np.linalg.norm(y_ref) < 1e-3
+        st = state0.clone()
+        y = mmf.decode_step(blocks, x, st)
+        _ok(mmf)
+    finally:
+        mmf.set_decode_path(mmf.MMF_DECODE_AUTO)
+    assert np.linalg.norm(_np(y) - y_ref) / np.linalg.norm(y_ref) < 1e-3
+    np.testing.assert_allclose(_np(st)[0], st_ref[0], rtol=RTOL32, atol=ATOL32)
+
+
 # CUDA-core form: float32 table, or one row; tensor-core form: bf16 table and b >= 2 (ragged d and
 # vocabulary tails, two passes at b = 130)
 @pytest.mark.parametrize("b,d,vocab,xdt,tdt", [(1, 256, 1000, "f32", "f32"), (5, 264, 900, "bf16", "f32"),
