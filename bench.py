@@ -42,9 +42,9 @@ WORKLOADS = {
     "prefill-1.3B": dict(d=2048, inner=5632, layers=24, vocab=32000, batch=16, seq=2048),
 }
 # DRAM traffic of one ternary_gemm_tc_kernel launch (dram__bytes_read.sum + dram__bytes_write.sum,
-# averaged over the 96 GEMM launches of one step) from an ncu capture of this bench's own workload;
-# valid only while the kernel source is the one captured (SHA-256 prefix), else reported as null.
-GEMM_TRAFFIC = {"prefill-370M": dict(bytes=78.3e6, algorithmic=115.2e6, sha256="14a6d8df0242cadf",
+# averaged over the four GEMM launches of one block at this workload's per-launch shapes) from an ncu
+# capture; valid only while the kernel source is the one captured (SHA-256 prefix), else null.
+GEMM_TRAFFIC = {"prefill-370M": dict(bytes=79.1e6, algorithmic=115.2e6, sha256="14a6d8df0242cadf",
                                      profile="profiles/ternary_gemm_tc_kernel_prefill-370M_traffic.md")}
 # Autoregressive decode of the 2.7B-shape stack: a 512-token prompt (prefill, untimed) then
 # decode steps with the recurrent state carried per layer, at three batch sizes.
