@@ -300,10 +300,16 @@ mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, c
  *   dzf = (df - di SiLU(zi)) f (1 - f);  dzi = di (1 - f) SiLU'(zi);  dh0 = f_0 G_0.
  *   zf, zi, h (the forward's states), dh (dL/dh) [b][t][d] dtype, contiguous.
  *   h0 [b][d] float32 or NULL.   dzf, dzi [b][t][d] dtype out.   dh0 [b][d] float32 out or NULL.
- * CUDA cores, float32 arithmetic: one thread per (sequence, channel), steps in reverse. */
+ *   ws >= mmf_workspace_bytes(MMF_OP_SCAN, b*t, d, 0, 0) when t > 32 (unused otherwise), 256-byte
+ *   aligned, caller-owned, not retained; a smaller or misaligned ws is MMF_ERR_WORKSPACE.
+ *   t = 0 writes dh0 = 0. b * ceil(t / chunk) * ceil(d / 256) CTAs must fit one grid (< 2^31).
+ * CUDA cores, float32 arithmetic, chunked like the forward scan with time reversed: G is affine
+ * in the carry from the later steps, so chunks fold to (A, B), a reverse walk over the chunks
+ * gives each its carry, and each chunk is replayed from it. The chunk sums associate differently
+ * from one sequential reverse walk (float32 rounding order only). */
 mmf_status mmf_hgrn_scan_backward(const void* zf, const void* zi, const void* h, const void* dh, mmf_dtype dtype,
                                   int32_t b, int64_t t, int32_t d, const float* h0, void* dzf, void* dzi,
-                                  float* dh0, mmf_stream_t stream);
+                                  float* dh0, void* ws, size_t ws_bytes, mmf_stream_t stream);
 
 /* HGRN2 recurrence with state expansion, per sequence and head (nightvoyager.top, innovations
  * table, names HGRN2 and its fused-recurrent and chunked kernels; the recurrence is HGRN2's

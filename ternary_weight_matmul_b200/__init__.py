@@ -103,7 +103,8 @@ def lib() -> ctypes.CDLL:
         "mmf_lm_head_argmax": (ctypes.c_int, [vp, ctypes.c_int, i32, i32, vp, ctypes.c_float, vp, ctypes.c_int, i32,
                                               vp, vp, vp, sz, st]),
         "mmf_hgrn2_recurrence": (ctypes.c_int, [vp, vp, vp, ctypes.c_int, i32, i64, i32, i32, i32, vp, vp, vp, st]),
-        "mmf_hgrn_scan_backward": (ctypes.c_int, [vp, vp, vp, vp, ctypes.c_int, i32, i64, i32, vp, vp, vp, vp, st]),
+        "mmf_hgrn_scan_backward": (ctypes.c_int, [vp, vp, vp, vp, ctypes.c_int, i32, i64, i32, vp, vp, vp, vp, vp,
+                                                   ctypes.c_size_t, st]),
         "mmf_validate_packed": (ctypes.c_int, [ctypes.POINTER(Ternary), vp, st]),
         "mmf_bitlinear_backward": (ctypes.c_int, [vp, ctypes.c_int, i64, vp, ctypes.c_float, ctypes.POINTER(Ternary),
                                                   vp, vp, vp, ctypes.c_int, vp, vp, vp, vp, sz, st]),
@@ -342,9 +343,10 @@ def hgrn_scan_backward(zf: torch.Tensor, zi: torch.Tensor, h: torch.Tensor, dh: 
     dzf = torch.empty_like(zf)
     dzi = torch.empty_like(zf)
     dh0 = torch.empty(b, d, dtype=torch.float32, device=zf.device)
+    ws = workspace(MMF_OP_SCAN, b * t, d, 0, 0, zf.device)
     _check(lib().mmf_hgrn_scan_backward(zf.data_ptr(), zi.data_ptr(), h.data_ptr(), dh.data_ptr(), _dt(zf.dtype),
                                         b, t, d, _ptr(h0), dzf.data_ptr(), dzi.data_ptr(), dh0.data_ptr(),
-                                        _stream(zf.device)), "mmf_hgrn_scan_backward")
+                                        ws.data_ptr(), ws.numel(), _stream(zf.device)), "mmf_hgrn_scan_backward")
     return dzf, dzi, dh0
 
 

@@ -8,11 +8,17 @@
 // (nightvoyager.top, innovations table) names the straight-through estimator for training; the
 // recurrence and its gates are smooth, so these are their exact derivatives.
 //
-// One thread per (sequence, channel) walks the steps in reverse, reading zf, zi, dh and the
-// forward's h_{t-1} and writing dzf, dzi: consecutive threads take consecutive channels, so every
-// access is coalesced across the warp. f_{t+1} is carried in a register from the previous
-// (later) step.
-//
+// G obeys the affine recurrence G_t = f_{t+1} G_{t+1} + dh_t backwards in time, so it is chunked
+// like the forward scan with the time axis reversed. With `carry` = f_{t1} G_{t1}, what enters
+// chunk [t0, t1) from the later steps (0 for the last chunk), the chunk passes f_{t0} G_{t0} =
+// A carry + B on to the earlier steps, A the product of its forget gates and B the value at
+// carry 0. Phase 1 folds every (sequence, chunk, channel) into (A, B) reading zf and dh; phase 2
+// walks the chunks of each channel from the last to the first and records every chunk's carry
+// (the final one is dh0); phase 3 replays each chunk from its carry, reading zf, zi, dh and
+// h_{t-1} and writing dzf and dzi. Sequences no longer than one chunk take phase 3 alone. Each
+// thread owns VEC adjacent channels (paired loads when rows allow), lanes cover consecutive
+// channels, so every access is a coalesced row segment; steps are loaded ahead into registers
+// before the dependent chain runs over them.
 // FusedBitLinear with the straight-through estimator (the report: weight_quant quantises in the
 // forward pass and keeps the gradient in the backward pass; the activation quantiser is taken the
 // same way): with the forward's codes q and factors a/127, the dequantised operands are
@@ -25,6 +31,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "kernels.cuh"
 
 namespace mmf {
 namespace bwd {
@@ -44,37 +51,158 @@ struct ScanBwdArgs {
   void* dzf;          // [b][t][d] out
   void* dzi;          // [b][t][d] out
   float* dh0;         // [b][d] out, or null
+  int32_t chunk;      // steps per chunk
+  int32_t nchunk;
+  int32_t gx;         // CTAs across the channels of one (sequence, chunk)
+  float* agg_a;       // [b][nchunk][d] product of the chunk's forget gates
+  float* agg_b;       // [b][nchunk][d] f_{t0} G_{t0} of the chunk at carry 0
+  float* cin;         // [b][nchunk][d] carry entering each chunk from the later steps
 };
+constexpr int kScanBwdThreads = 128;
+constexpr int kScanBwdFold = 16;    // steps loaded ahead in phase 1 (two arrays)
+constexpr int kScanBwdReplay = 8;   // steps loaded ahead in phase 3 (four arrays)
 
-template <mmf_dtype DT>
-__global__ void __launch_bounds__(kThreads) scan_bwd_kernel(const ScanBwdArgs a) {
-  using T = typename Elem<DT>::T;
-  const int64_t gid = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-  if (gid >= (int64_t)a.b * a.d) return;
-  const int bi = (int)(gid / a.d), c = (int)(gid - (int64_t)bi * a.d);
-  const int64_t base = (int64_t)bi * a.t * a.d + c;
-  const T* zf = reinterpret_cast<const T*>(a.zf);
-  const T* zi = reinterpret_cast<const T*>(a.zi);
-  const T* h = reinterpret_cast<const T*>(a.h);
-  const T* dh = reinterpret_cast<const T*>(a.dh);
-  T* dzf = reinterpret_cast<T*>(a.dzf);
-  T* dzi = reinterpret_cast<T*>(a.dzi);
-  const float h_init = a.h0 ? a.h0[(int64_t)bi * a.d + c] : 0.0f;
-  float G = 0.0f, f_next = 0.0f;
-  for (int64_t s = a.t - 1; s >= 0; --s) {
-    const int64_t idx = base + s * a.d;
-    G = fmaf(f_next, G, Elem<DT>::load(dh + idx));
-    const float hp = s > 0 ? Elem<DT>::load(h + idx - a.d) : h_init;
-    float f, omf;
-    hgrn_forget(Elem<DT>::load(zf + idx), f, omf);
-    const float z = Elem<DT>::load(zi + idx);
-    const float sz = sigmoidf_(z);
-    const float df = G * hp;
-    Elem<DT>::store(dzf + idx, (df - G * (z * sz)) * f * omf);
-    Elem<DT>::store(dzi + idx, G * omf * sz * fmaf(z, 1.0f - sz, 1.0f));
-    f_next = f;
+// blockIdx.x runs over (sequence, chunk, channel block) with the channel block fastest, so the
+// grid has no per-dimension limit on b or the chunk count.
+__device__ __forceinline__ void scan_bwd_block(const ScanBwdArgs& a, int& cx, int& c, int& bi) {
+  const int64_t id = blockIdx.x;
+  const int64_t rest = id / a.gx;
+  cx = (int)(id - rest * a.gx);
+  bi = (int)(rest / a.nchunk);
+  c = (int)(rest - (int64_t)bi * a.nchunk);
+}
+
+// Phase 1: (A, B) of every (sequence, chunk, channel).
+template <mmf_dtype DT, int VEC>
+__global__ void __launch_bounds__(kScanBwdThreads) scan_bwd_fold_kernel(const ScanBwdArgs a) {
+  int cx, c, bi;
+  scan_bwd_block(a, cx, c, bi);
+  const int64_t ch = ((int64_t)cx * kScanBwdThreads + threadIdx.x) * VEC;
+  if (ch >= a.d) return;
+  const int64_t t0 = (int64_t)c * a.chunk;
+  const int64_t t1 = t0 + a.chunk < a.t ? t0 + a.chunk : a.t;
+  const int64_t base = (int64_t)bi * a.t * a.d + ch;
+  float A[VEC], B[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) { A[v] = 1.0f; B[v] = 0.0f; }
+  for (int64_t te = t1; te > t0; te -= kScanBwdFold) {
+    float zf[kScanBwdFold][VEC], dh[kScanBwdFold][VEC];
+#pragma unroll
+    for (int u = 0; u < kScanBwdFold; ++u) {
+      if (te - 1 - u >= t0) {
+        load_vec<DT, VEC>(a.zf, base + (te - 1 - u) * a.d, zf[u]);
+        load_vec<DT, VEC>(a.dh, base + (te - 1 - u) * a.d, dh[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kScanBwdFold; ++u) {
+      if (te - 1 - u >= t0) {
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          float f, omf;
+          hgrn_forget(zf[u][v], f, omf);
+          B[v] = f * (dh[u][v] + B[v]);
+          A[v] = f * A[v];
+        }
+      }
+    }
   }
-  if (a.dh0) a.dh0[(int64_t)bi * a.d + c] = f_next * G;
+  const int64_t o = ((int64_t)bi * a.nchunk + c) * a.d + ch;
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    a.agg_a[o + v] = A[v];
+    a.agg_b[o + v] = B[v];
+  }
+}
+
+// Phase 2: one thread per (sequence, channel) walks the chunks from the last to the first.
+__global__ void __launch_bounds__(kScanBwdThreads) scan_bwd_carry_kernel(const ScanBwdArgs a) {
+  const int64_t gid = (int64_t)blockIdx.x * kScanBwdThreads + threadIdx.x;
+  if (gid >= (int64_t)a.b * a.d) return;
+  const int bi = (int)(gid / a.d);
+  const int64_t ch = gid - (int64_t)bi * a.d;
+  const int64_t base = (int64_t)bi * a.nchunk * a.d + ch;
+  float carry = 0.0f;
+  constexpr int PF = 32;
+  for (int c1 = a.nchunk; c1 > 0; c1 -= PF) {
+    float av[PF], bv[PF];
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      if (c1 - 1 - u >= 0) {
+        av[u] = a.agg_a[base + (int64_t)(c1 - 1 - u) * a.d];
+        bv[u] = a.agg_b[base + (int64_t)(c1 - 1 - u) * a.d];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      if (c1 - 1 - u >= 0) {
+        a.cin[base + (int64_t)(c1 - 1 - u) * a.d] = carry;
+        carry = fmaf(av[u], carry, bv[u]);
+      }
+    }
+  }
+  if (a.dh0) a.dh0[gid] = carry;
+}
+
+// Phase 3: replays chunk c from its carry and writes dzf, dzi; with SINGLE the sequence is one
+// chunk entered with carry 0, and its f_0 G_0 is dh0.
+template <mmf_dtype DT, int VEC, bool SINGLE>
+__global__ void __launch_bounds__(kScanBwdThreads) scan_bwd_replay_kernel(const ScanBwdArgs a) {
+  int cx, c, bi;
+  scan_bwd_block(a, cx, c, bi);
+  const int64_t ch = ((int64_t)cx * kScanBwdThreads + threadIdx.x) * VEC;
+  if (ch >= a.d) return;
+  const int64_t t0 = (int64_t)c * a.chunk;
+  const int64_t t1 = t0 + a.chunk < a.t ? t0 + a.chunk : a.t;
+  const int64_t base = (int64_t)bi * a.t * a.d + ch;
+  float cterm[VEC], hinit[VEC];
+#pragma unroll
+  for (int v = 0; v < VEC; ++v) {
+    cterm[v] = SINGLE ? 0.0f : a.cin[((int64_t)bi * a.nchunk + c) * a.d + ch + v];
+    hinit[v] = a.h0 ? a.h0[(int64_t)bi * a.d + ch + v] : 0.0f;
+  }
+  for (int64_t te = t1; te > t0; te -= kScanBwdReplay) {
+    float zf[kScanBwdReplay][VEC], zi[kScanBwdReplay][VEC], dh[kScanBwdReplay][VEC], hp[kScanBwdReplay][VEC];
+#pragma unroll
+    for (int u = 0; u < kScanBwdReplay; ++u) {
+      const int64_t t = te - 1 - u;
+      if (t >= t0) {
+        load_vec<DT, VEC>(a.zf, base + t * a.d, zf[u]);
+        load_vec<DT, VEC>(a.zi, base + t * a.d, zi[u]);
+        load_vec<DT, VEC>(a.dh, base + t * a.d, dh[u]);
+        if (t > 0) {
+          load_vec<DT, VEC>(a.h, base + (t - 1) * a.d, hp[u]);
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) hp[u][v] = hinit[v];
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kScanBwdReplay; ++u) {
+      const int64_t t = te - 1 - u;
+      if (t >= t0) {
+        float gzf[VEC], gzi[VEC];
+#pragma unroll
+        for (int v = 0; v < VEC; ++v) {
+          const float G = dh[u][v] + cterm[v];
+          float f, omf;
+          hgrn_forget(zf[u][v], f, omf);
+          const float z = zi[u][v];
+          const float sz = sigmoidf_(z);
+          gzf[v] = (G * hp[u][v] - G * (z * sz)) * f * omf;
+          gzi[v] = G * omf * sz * fmaf(z, 1.0f - sz, 1.0f);
+          cterm[v] = f * G;
+        }
+        store_vec<DT, VEC>(a.dzf, base + t * a.d, gzf);
+        store_vec<DT, VEC>(a.dzi, base + t * a.d, gzi);
+      }
+    }
+  }
+  if (SINGLE && a.dh0) {
+#pragma unroll
+    for (int v = 0; v < VEC; ++v) a.dh0[(int64_t)bi * a.d + ch + v] = cterm[v];
+  }
 }
 
 

@@ -5,12 +5,14 @@
 //
 // HGRN2 is named by the MatMul-Free LLM report (nightvoyager.top, innovations table: gated
 // linear recurrence with fused-recurrent and chunked kernels); the recurrence is HGRN2's
-// published one. Column v of the state sees only i_t[v], so the dv columns evolve independently:
-// one thread owns one column, keeps its dk state values in registers for the whole sequence and
-// forms o_t[v] as the dot product of q_t with them, with no exchange between threads. A CTA
-// serves 128 columns of one (sequence, head); per tile of kTS steps it stages q_t and f_t (dk
-// values each, shared by every column) in shared memory as float32. Rows past dk are padded with
-// q = 0 and f = 1 (key 0), so they stay zero and never contribute.
+// published one. Column v of the state sees only i_t[v], so the dv columns evolve independently,
+// and within a column every state row k evolves on its own (S[k][v] = f[k] S[k][v] + (1 - f[k])
+// i[v]); only the readout o_t[v] = q_t . S_t[:, v] sums over k. Four adjacent threads share one
+// column, each keeping dk / 4 state rows in registers for the whole sequence, and combine their
+// partial readouts with two shuffles per step; the partial readout runs as four independent FMA
+// chains. A CTA serves 32 columns of one (sequence, head); per tile of kTS steps it stages q_t and
+// f_t (dk values each, shared by every column) in shared memory as float32. Rows past dk are
+// padded with q = 0 and f = 1 (key 0), so they stay zero and never contribute.
 #pragma once
 
 #include "common.cuh"
@@ -18,7 +20,9 @@
 namespace mmf {
 namespace hgrn2 {
 
-constexpr int kThreads = 128;   // value columns per CTA
+constexpr int kThreads = 128;   // threads per CTA
+constexpr int kSplit = 4;       // threads per value column (each owns dk / kSplit state rows)
+constexpr int kCols = kThreads / kSplit;  // value columns per CTA
 constexpr int kTS = 16;         // steps per staged tile
 
 struct Args {
@@ -39,9 +43,12 @@ struct Args {
 template <mmf_dtype DT, int DK>
 __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a) {
   using T = typename Elem<DT>::T;
+  constexpr int KR = DK / kSplit;  // state rows per thread
   __shared__ __align__(16) float qs[kTS][DK];
   __shared__ __align__(16) float fs[kTS][DK];
-  const int v = blockIdx.x * kThreads + threadIdx.x;
+  const int sub = threadIdx.x & (kSplit - 1);
+  const int k0 = sub * KR;
+  const int v = blockIdx.x * kCols + (threadIdx.x >> 2);
   const int h = blockIdx.y, bi = blockIdx.z;
   const bool active = v < a.dv;
   const int64_t qk_step = (int64_t)a.heads * a.dk;   // elements of q / f per step
@@ -52,9 +59,10 @@ __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a)
   T* o = reinterpret_cast<T*>(a.o) + (int64_t)bi * a.t * iv_step + (int64_t)h * a.dv;
   const int64_t s_base = ((int64_t)bi * a.heads + h) * a.dk * a.dv;
 
-  float S[DK];
+  float S[KR];
 #pragma unroll
-  for (int k = 0; k < DK; ++k) S[k] = (a.s0 && active && k < a.dk) ? a.s0[s_base + (int64_t)k * a.dv + v] : 0.0f;
+  for (int j = 0; j < KR; ++j)
+    S[j] = (a.s0 && active && k0 + j < a.dk) ? a.s0[s_base + (int64_t)(k0 + j) * a.dv + v] : 0.0f;
 
   for (int64_t t0 = 0; t0 < a.t; t0 += kTS) {
     const int ns = (int)(a.t - t0 < kTS ? a.t - t0 : kTS);
@@ -70,31 +78,33 @@ __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a)
       fs[s][k] = fv;
     }
     __syncthreads();
-    if (active) {
-      for (int s = 0; s < ns; ++s) {
-        const float iv = Elem<DT>::load(in + (t0 + s) * iv_step + v);
-        float acc = 0.0f;
+    // (inactive columns take part in the shuffles with zero contributions)
+    for (int s = 0; s < ns; ++s) {
+      const float iv = active ? Elem<DT>::load(in + (t0 + s) * iv_step + v) : 0.0f;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-        for (int k = 0; k < DK; k += 4) {
-          const float4 f4 = *reinterpret_cast<const float4*>(&fs[s][k]);
-          const float4 q4 = *reinterpret_cast<const float4*>(&qs[s][k]);
-          S[k] = fmaf(f4.x, S[k], (1.0f - f4.x) * iv);
-          S[k + 1] = fmaf(f4.y, S[k + 1], (1.0f - f4.y) * iv);
-          S[k + 2] = fmaf(f4.z, S[k + 2], (1.0f - f4.z) * iv);
-          S[k + 3] = fmaf(f4.w, S[k + 3], (1.0f - f4.w) * iv);
-          acc = fmaf(q4.x, S[k], acc);
-          acc = fmaf(q4.y, S[k + 1], acc);
-          acc = fmaf(q4.z, S[k + 2], acc);
-          acc = fmaf(q4.w, S[k + 3], acc);
-        }
-        Elem<DT>::store(o + (t0 + s) * iv_step + v, acc);
+      for (int j = 0; j < KR; j += 4) {
+        const float4 f4 = *reinterpret_cast<const float4*>(&fs[s][k0 + j]);
+        const float4 q4 = *reinterpret_cast<const float4*>(&qs[s][k0 + j]);
+        S[j] = fmaf(f4.x, S[j], (1.0f - f4.x) * iv);
+        S[j + 1] = fmaf(f4.y, S[j + 1], (1.0f - f4.y) * iv);
+        S[j + 2] = fmaf(f4.z, S[j + 2], (1.0f - f4.z) * iv);
+        S[j + 3] = fmaf(f4.w, S[j + 3], (1.0f - f4.w) * iv);
+        acc[0] = fmaf(q4.x, S[j], acc[0]);
+        acc[1] = fmaf(q4.y, S[j + 1], acc[1]);
+        acc[2] = fmaf(q4.z, S[j + 2], acc[2]);
+        acc[3] = fmaf(q4.w, S[j + 3], acc[3]);
       }
+      float part = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+      part += __shfl_xor_sync(0xffffffffu, part, 1);
+      part += __shfl_xor_sync(0xffffffffu, part, 2);
+      if (active && sub == 0) Elem<DT>::store(o + (t0 + s) * iv_step + v, part);
     }
   }
   if (active && a.s_out) {
 #pragma unroll
-    for (int k = 0; k < DK; ++k)
-      if (k < a.dk) a.s_out[s_base + (int64_t)k * a.dv + v] = S[k];
+    for (int j = 0; j < KR; ++j)
+      if (k0 + j < a.dk) a.s_out[s_base + (int64_t)(k0 + j) * a.dv + v] = S[j];
   }
 }
 

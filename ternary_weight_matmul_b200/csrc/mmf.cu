@@ -1494,6 +1494,29 @@ mmf_status decode_impl(const mmf_block_weights* layers, int32_t n_layers, const 
 
 }  // namespace
 
+// Steps per chunk of the chunked scan backward: the whole sequence up to 32 steps, 32 up to 4096
+// steps, then a multiple of 16 giving at most 128 chunks; so b * nchunk <= ceil(b t / 8) and the
+// forward scan's scratch size bounds the three [b][nchunk][d] arrays.
+inline int32_t scan_bwd_chunk(int64_t t) {
+  if (t <= 32) return (int32_t)t;
+  if (t <= 4096) return 32;
+  const int64_t c = (t + 127) / 128;
+  return (int32_t)((c + 15) / 16 * 16);
+}
+
+template <mmf_dtype DT, int VEC>
+void scan_bwd_launch(const bwd::ScanBwdArgs& a, cudaStream_t st) {
+  const unsigned blocks = (unsigned)((int64_t)a.gx * a.nchunk * a.b);
+  if (a.nchunk == 1) {
+    launch_k(bwd::scan_bwd_replay_kernel<DT, VEC, true>, dim3(blocks), dim3(bwd::kScanBwdThreads), 0, st, a);
+    return;
+  }
+  launch_k(bwd::scan_bwd_fold_kernel<DT, VEC>, dim3(blocks), dim3(bwd::kScanBwdThreads), 0, st, a);
+  const unsigned cb = (unsigned)(((int64_t)a.b * a.d + bwd::kScanBwdThreads - 1) / bwd::kScanBwdThreads);
+  launch_k(bwd::scan_bwd_carry_kernel, dim3(cb), dim3(bwd::kScanBwdThreads), 0, st, a);
+  launch_k(bwd::scan_bwd_replay_kernel<DT, VEC, false>, dim3(blocks), dim3(bwd::kScanBwdThreads), 0, st, a);
+}
+
 extern "C" {
 
 mmf_status mmf_decode_step(const mmf_block_weights* layers, int32_t n_layers, const void* x,
@@ -1618,25 +1641,55 @@ mmf_status mmf_validate_packed(const mmf_ternary* w, unsigned long long* bad, mm
 // ---------------------------------------------------------------------------------------------
 mmf_status mmf_hgrn_scan_backward(const void* zf, const void* zi, const void* h, const void* dh, mmf_dtype dtype,
                                   int32_t b, int64_t t, int32_t d, const float* h0, void* dzf, void* dzi,
-                                  float* dh0, mmf_stream_t stream) {
+                                  float* dh0, void* ws, size_t ws_bytes, mmf_stream_t stream) {
   MMF_CHECK_ARG(b >= 0 && t >= 0 && d >= 0, "scan backward: negative size");
   MMF_CHECK_ARG(valid_dtype(dtype), "scan backward: bad dtype");
-  MMF_CHECK_ARG((int64_t)b * d < ((int64_t)1 << 38), "scan backward: b * d too large for one grid");
   if ((int64_t)b * d == 0) return MMF_OK;
   MMF_CHECK_ARG(t == 0 || (zf && zi && h && dh && dzf && dzi), "scan backward: null pointer");
+  const int32_t chunk = t > 0 ? scan_bwd_chunk(t) : 1;
+  const int32_t nchunk = (int32_t)((t + chunk - 1) / chunk);
+  if (nchunk > 1) MMF_TRY(check_ws(ws, ws_bytes, scan_ws_bytes((int64_t)b * t, d)));
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   DevInfo* di;
   MMF_TRY(device_info(&di));
-  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (t == 0) {
+    // no steps: nothing reaches h0
+    if (dh0) {
+      cudaError_t e = cudaMemsetAsync(dh0, 0, (size_t)b * d * sizeof(float), st);
+      if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    }
+    return MMF_OK;
+  }
   bwd::ScanBwdArgs a;
   memset(&a, 0, sizeof(a));
   a.zf = zf; a.zi = zi; a.h = h; a.dh = dh; a.dt = dtype; a.b = b; a.t = t; a.d = d;
   a.h0 = h0; a.dzf = dzf; a.dzi = dzi; a.dh0 = dh0;
-  const int64_t threads = (int64_t)b * d;
-  const dim3 grid((unsigned)((threads + bwd::kThreads - 1) / bwd::kThreads));
-  LaunchScope ls(MMF_KERNEL_SCAN, (double)b * t * d * 6.0 * dsize(dtype), st);
-  if (dtype == MMF_F32) launch_k(bwd::scan_bwd_kernel<MMF_F32>, grid, dim3(bwd::kThreads), 0, st, a);
-  else launch_k(bwd::scan_bwd_kernel<MMF_BF16>, grid, dim3(bwd::kThreads), 0, st, a);
-  return check_launch("scan_bwd_kernel");
+  a.chunk = chunk;
+  a.nchunk = nchunk;
+  if (nchunk > 1) {
+    const size_t arr = align256((size_t)d * 4 * (size_t)(((int64_t)b * t + 7) / 8));
+    uint8_t* p = reinterpret_cast<uint8_t*>(ws);
+    a.agg_a = reinterpret_cast<float*>(p);
+    a.agg_b = reinterpret_cast<float*>(p + arr);
+    a.cin = reinterpret_cast<float*>(p + 2 * arr);
+  }
+  const size_t es = dsize(dtype);
+  const auto aligned = [&](const void* q) { return q == nullptr || (reinterpret_cast<uintptr_t>(q) % (2 * es)) == 0; };
+  const bool pair = d % 2 == 0 && aligned(zf) && aligned(zi) && aligned(h) && aligned(dh) && aligned(dzf) &&
+                    aligned(dzi);
+  const int vec = pair ? 2 : 1;
+  a.gx = (int32_t)((d / vec + bwd::kScanBwdThreads - 1) / bwd::kScanBwdThreads);
+  MMF_CHECK_ARG((int64_t)a.gx * a.nchunk * b < ((int64_t)1 << 31), "scan backward: b * t * d too large for one grid");
+  LaunchScope ls(MMF_KERNEL_SCAN, (double)b * t * d * 6.0 * es, st);
+  if (a.nchunk > 1) g_launches.fetch_add(2);  // three kernels under one timing scope
+  if (dtype == MMF_F32) {
+    if (pair) scan_bwd_launch<MMF_F32, 2>(a, st);
+    else scan_bwd_launch<MMF_F32, 1>(a, st);
+  } else {
+    if (pair) scan_bwd_launch<MMF_BF16, 2>(a, st);
+    else scan_bwd_launch<MMF_BF16, 1>(a, st);
+  }
+  return check_launch("scan backward");
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1700,7 +1753,7 @@ mmf_status mmf_hgrn2_recurrence(const void* q, const void* f, const void* i, mmf
   memset(&a, 0, sizeof(a));
   a.q = q; a.f = f; a.i = i; a.dt = dtype; a.b = b; a.t = t; a.heads = heads; a.dk = dk; a.dv = dv;
   a.s0 = s0; a.s_out = s_out; a.o = o;
-  const dim3 grid((unsigned)((dv + hgrn2::kThreads - 1) / hgrn2::kThreads), (unsigned)heads, (unsigned)b);
+  const dim3 grid((unsigned)((dv + hgrn2::kCols - 1) / hgrn2::kCols), (unsigned)heads, (unsigned)b);
   const double es = (double)dsize(dtype);
   LaunchScope ls(MMF_KERNEL_OTHER, (double)b * t * heads * (2.0 * dk + 2.0 * dv) * es, st);
 #define MMF_HGRN2(DT_, DK_) launch_k(hgrn2::hgrn2_recurrent_kernel<DT_, DK_>, grid, dim3(hgrn2::kThreads), 0, st, a)

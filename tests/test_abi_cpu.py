@@ -114,12 +114,18 @@ def test_hgrn2_arguments_on_host(L):
 
 
 def test_scan_backward_arguments_on_host(L):
-    # mmf_hgrn_scan_backward(zf, zi, h, dh, dtype, b, t, d, h0, dzf, dzi, dh0, stream)
+    # mmf_hgrn_scan_backward(zf, zi, h, dh, dtype, b, t, d, h0, dzf, dzi, dh0, ws, ws_bytes, stream)
     sb = L.mmf_hgrn_scan_backward
-    assert sb(16, 16, 16, 16, 0, -1, 4, 8, None, 16, 16, None, None) == mmf.MMF_ERR_INVALID_ARG  # b < 0
-    assert sb(16, 16, 16, 16, 3, 1, 4, 8, None, 16, 16, None, None) == mmf.MMF_ERR_INVALID_ARG   # dtype
-    assert sb(16, 16, None, 16, 0, 1, 4, 8, None, 16, 16, None, None) == mmf.MMF_ERR_INVALID_ARG  # null h
-    assert sb(None, None, None, None, 0, 0, 4, 8, None, None, None, None, None) == mmf.MMF_OK     # b = 0
+    assert sb(16, 16, 16, 16, 0, -1, 4, 8, None, 16, 16, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG  # b < 0
+    assert sb(16, 16, 16, 16, 3, 1, 4, 8, None, 16, 16, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG   # dtype
+    assert sb(16, 16, None, 16, 0, 1, 4, 8, None, 16, 16, None, None, 0, None) == mmf.MMF_ERR_INVALID_ARG  # null h
+    assert sb(None, None, None, None, 0, 0, 4, 8, None, None, None, None, None, 0, None) == mmf.MMF_OK     # b = 0
+    # past 32 steps the chunked backward needs the scan's workspace, 256-byte aligned
+    need = mmf.workspace_bytes(mmf.MMF_OP_SCAN, 2 * 64, 8, 0, 0)
+    assert need > 0
+    assert sb(16, 16, 16, 16, 0, 2, 64, 8, None, 16, 16, None, None, 0, None) == mmf.MMF_ERR_WORKSPACE
+    assert sb(16, 16, 16, 16, 0, 2, 64, 8, None, 16, 16, None, 256, need - 1, None) == mmf.MMF_ERR_WORKSPACE
+    assert sb(16, 16, 16, 16, 0, 2, 64, 8, None, 16, 16, None, 272, need, None) == mmf.MMF_ERR_WORKSPACE
 
 
 def test_bitlinear_backward_arguments_on_host(L):

@@ -595,11 +595,14 @@ def test_hgrn2_recurrence_parity(mmf, dt, b, t, heads, dk, dv):
 
 
 # Gradients of the scan with its gates against the oracle's chain (gates -> scan backward -> gate
-# backward) on the oracle's own forward states, rounded to the kernel's dtype; ragged d, a carried
-# initial state, long memory, an empty sequence. float32 within 1e-4 of the largest gradient
-# (float32 accumulation over up to 700 steps of G); bf16 inputs, states and outputs within 2e-2.
+# backward) on the oracle's own forward states, rounded to the kernel's dtype; one chunk (up to 32
+# steps), two chunks with a ragged last one, many chunks (700 steps, and 5000 steps in chunks of
+# 48), odd d (one channel per thread) and even d (channel pairs), a carried initial state, long
+# memory, an empty sequence. float32 within 1e-4 of the largest gradient (float32 accumulation
+# over up to 5000 steps of G); bf16 inputs, states and outputs within 2e-2.
 @pytest.mark.parametrize("dt", ["f32", "bf16"])
-@pytest.mark.parametrize("b,t,d,long_memory", [(2, 37, 100, False), (1, 700, 64, True), (2, 0, 16, False)])
+@pytest.mark.parametrize("b,t,d,long_memory", [(2, 37, 100, False), (1, 700, 64, True), (2, 0, 16, False),
+                                               (3, 20, 6, False), (3, 33, 7, True), (1, 5000, 10, True)])
 def test_scan_backward_parity(mmf, dt, b, t, d, long_memory):
     dts = {"f32": torch.float32, "bf16": torch.bfloat16}
     zf, zi = synth.scan_inputs(95, b, t, d, long_memory)
