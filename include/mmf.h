@@ -75,7 +75,8 @@ typedef enum {
   MMF_OP_DECODE = 3,    /* mmf_decode_step: m = b, d, inner                       */
   MMF_OP_STACK = 4,     /* mmf_stack_fwd: m = b*t tokens, d, inner, n_layers      */
   MMF_OP_SCAN = 5,      /* mmf_hgrn_scan: m = b*t tokens, d channels              */
-  MMF_OP_HEAD = 6       /* mmf_lm_head_argmax: inner = vocabulary size            */
+  MMF_OP_HEAD = 6,      /* mmf_lm_head_argmax: inner = vocabulary size            */
+  MMF_OP_BITLINEAR_BWD = 7 /* mmf_bitlinear_backward: m rows, d = K, inner = N     */
 } mmf_op;
 
 /* A packed ternary weight (device pointers). */
@@ -285,9 +286,14 @@ mmf_status mmf_validate_packed(const mmf_ternary* w, unsigned long long* bad, mm
  *   dW = dy^T rq (the latent float weight's gradient)  [w->n][w->k] float32 out, or NULL
  *   x [m][w->k] x_dtype; norm_w [w->k] float32 or NULL (unit gain); q [m][w->k] int8;
  *   deq [m] float32; dy [m][w->n] dy_dtype. w->n <= 65535.
- *   ws >= 4 * m bytes, 256-byte aligned (mmf_workspace_bytes(MMF_OP_BITLINEAR, m, w->k, w->n, 0)
- *   is always enough). m = 0 writes zero dnorm_w / dW.
- * CUDA cores, float32 arithmetic. */
+ *   ws >= mmf_workspace_bytes(MMF_OP_BITLINEAR_BWD, m, w->k, w->n, 0), 256-byte aligned,
+ *   caller-owned. m = 0 writes zero dnorm_w / dW.
+ * dr and dW run on the bf16 tensor cores (tcgen05.mma.kind::f16, float32 accumulation): dy (and
+ * dy (a/127) for dW) enters as bf16 hi / lo pairs, the ternary and int8 codes are exact in bf16,
+ * so both products are float32-accurate (about 2^-17 relative per term); the operands are first
+ * laid out K-major in the workspace (transposes of t, q and dy). mmf_set_gemm_path(MMF_GEMM_SIMT)
+ * selects CUDA-core kernels with float32 arithmetic instead. rho, the gain's gradient and dx are
+ * CUDA-core kernels either way. */
 mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, const float* norm_w, float eps,
                                   const mmf_ternary* w, const int8_t* q, const float* deq, const void* dy,
                                   mmf_dtype dy_dtype, float* dx, float* dnorm_w, float* dW, void* ws,

@@ -21,7 +21,8 @@ LIB_PATH = os.path.join(_HERE, "libmmf.so")
 
 MMF_OK, MMF_ERR_INVALID_ARG, MMF_ERR_UNSUPPORTED, MMF_ERR_WORKSPACE, MMF_ERR_CUDA, MMF_ERR_TIMEOUT = range(6)
 MMF_F32, MMF_BF16 = 0, 1
-MMF_OP_PACK, MMF_OP_BITLINEAR, MMF_OP_BLOCK, MMF_OP_DECODE, MMF_OP_STACK, MMF_OP_SCAN, MMF_OP_HEAD = range(7)
+(MMF_OP_PACK, MMF_OP_BITLINEAR, MMF_OP_BLOCK, MMF_OP_DECODE, MMF_OP_STACK, MMF_OP_SCAN, MMF_OP_HEAD,
+ MMF_OP_BITLINEAR_BWD) = range(8)
 MMF_GEMM_AUTO, MMF_GEMM_TENSOR, MMF_GEMM_SIMT = range(3)
 MMF_DECODE_AUTO, MMF_DECODE_FUSED, MMF_DECODE_SKINNY, MMF_DECODE_BLOCK = range(4)
 
@@ -313,16 +314,19 @@ def bitlinear_backward(x: torch.Tensor, norm_w: torch.Tensor | None, w: "PackedT
                        deq: torch.Tensor, dy: torch.Tensor, eps: float = 1e-8, want_dnorm_w: bool = True,
                        want_dW: bool = True):
     """mmf_bitlinear_backward: (dx [m, k], dnorm_w [k] or None, dW [n, k] or None), float32, from
-    x [m, k], the forward's codes q [m, k] int8 and factors deq [m] float32, and dy [m, n]."""
+    x [m, k], the forward's codes q [m, k] int8 and factors deq [m] float32, and dy [m, n]
+    (contiguous)."""
     for a in (x, q, deq, dy):
         _dev(a)
+        if not a.is_contiguous():
+            raise ValueError("x, q, deq and dy need contiguous storage")
     m, k = x.shape
     if tuple(q.shape) != (m, k) or q.dtype != torch.int8 or tuple(deq.shape) != (m,) or tuple(dy.shape) != (m, w.n):
         raise ValueError("shapes: x, q [m, k] (q int8), deq [m], dy [m, n]")
     dx = torch.empty(m, k, dtype=torch.float32, device=x.device)
     dnw = torch.empty(k, dtype=torch.float32, device=x.device) if want_dnorm_w else None
     dW = torch.empty(w.n, k, dtype=torch.float32, device=x.device) if want_dW else None
-    ws = workspace(MMF_OP_BITLINEAR, m, k, w.n, 0, x.device)
+    ws = workspace(MMF_OP_BITLINEAR_BWD, m, k, w.n, 0, x.device)
     tw = w.c()
     _check(lib().mmf_bitlinear_backward(x.data_ptr(), _dt(x.dtype), m, _ptr(norm_w), eps, ctypes.byref(tw),
                                         q.data_ptr(), deq.data_ptr(), dy.data_ptr(), _dt(dy.dtype), dx.data_ptr(),

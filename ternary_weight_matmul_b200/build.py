@@ -9,7 +9,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "mmf.cu")
-DEPS = [os.path.join(HERE, "csrc", f) for f in ("mmf.cu", "common.cuh", "kernels.cuh", "gemm_tc.cuh", "decode.cuh", "head.cuh", "hgrn2.cuh", "backward.cuh", "validate.cuh", "decode_rows.cuh", "gemm_skinny.cuh")] + [
+DEPS = [os.path.join(HERE, "csrc", f) for f in ("mmf.cu", "common.cuh", "kernels.cuh", "gemm_tc.cuh", "decode.cuh", "head.cuh", "hgrn2.cuh", "backward.cuh", "validate.cuh", "decode_rows.cuh", "gemm_skinny.cuh", "gemm_bf16.cuh")] + [
     os.path.join(ROOT, "include", "mmf.h")]
 OUT = os.path.join(HERE, "libmmf.so")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]

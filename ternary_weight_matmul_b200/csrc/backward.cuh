@@ -30,6 +30,8 @@
 // over dr; dW per (weight row, column).
 #pragma once
 
+#include <type_traits>
+
 #include "common.cuh"
 #include "kernels.cuh"
 
@@ -59,8 +61,41 @@ struct ScanBwdArgs {
   float* cin;         // [b][nchunk][d] carry entering each chunk from the later steps
 };
 constexpr int kScanBwdThreads = 128;
-constexpr int kScanBwdFold = 16;    // steps loaded ahead in phase 1 (two arrays)
-constexpr int kScanBwdReplay = 8;   // steps loaded ahead in phase 3 (four arrays)
+constexpr int kScanBwdFold = 8;     // steps loaded ahead in phase 1 (two arrays)
+constexpr int kScanBwdReplay = 4;   // steps loaded ahead in phase 3 (four arrays)
+
+// Steps are loaded ahead as raw words (a bf16 pair in one register) and widened to float32 only
+// when used, which keeps the prefetch to one register per bf16 value pair.
+template <mmf_dtype DT, int VEC>
+struct RawV {
+  using T = typename std::conditional<DT == MMF_F32 && VEC == 2, uint2, uint32_t>::type;
+};
+template <mmf_dtype DT, int VEC>
+__device__ __forceinline__ typename RawV<DT, VEC>::T raw_load(const void* base, int64_t idx) {
+  if constexpr (DT == MMF_F32 && VEC == 2) {
+    return *reinterpret_cast<const uint2*>(reinterpret_cast<const float*>(base) + idx);
+  } else if constexpr (DT == MMF_F32) {
+    return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const float*>(base) + idx);
+  } else if constexpr (VEC == 2) {
+    return *reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+  } else {
+    return (uint32_t)*reinterpret_cast<const unsigned short*>(reinterpret_cast<const __nv_bfloat16*>(base) + idx);
+  }
+}
+template <mmf_dtype DT, int VEC>
+__device__ __forceinline__ void raw_unpack(const typename RawV<DT, VEC>::T& r, float (&o)[VEC]) {
+  if constexpr (DT == MMF_F32 && VEC == 2) {
+    o[0] = __uint_as_float(r.x);
+    o[VEC - 1] = __uint_as_float(r.y);
+  } else if constexpr (DT == MMF_F32) {
+    o[0] = __uint_as_float(r);
+  } else if constexpr (VEC == 2) {
+    o[0] = __uint_as_float(r << 16);
+    o[VEC - 1] = __uint_as_float(r & 0xffff0000u);
+  } else {
+    o[0] = __uint_as_float(r << 16);
+  }
+}
 
 // blockIdx.x runs over (sequence, chunk, channel block) with the channel block fastest, so the
 // grid has no per-dimension limit on b or the chunk count.
@@ -85,23 +120,27 @@ __global__ void __launch_bounds__(kScanBwdThreads) scan_bwd_fold_kernel(const Sc
   float A[VEC], B[VEC];
 #pragma unroll
   for (int v = 0; v < VEC; ++v) { A[v] = 1.0f; B[v] = 0.0f; }
+  using R = typename RawV<DT, VEC>::T;
   for (int64_t te = t1; te > t0; te -= kScanBwdFold) {
-    float zf[kScanBwdFold][VEC], dh[kScanBwdFold][VEC];
+    R rzf[kScanBwdFold], rdh[kScanBwdFold];
 #pragma unroll
     for (int u = 0; u < kScanBwdFold; ++u) {
       if (te - 1 - u >= t0) {
-        load_vec<DT, VEC>(a.zf, base + (te - 1 - u) * a.d, zf[u]);
-        load_vec<DT, VEC>(a.dh, base + (te - 1 - u) * a.d, dh[u]);
+        rzf[u] = raw_load<DT, VEC>(a.zf, base + (te - 1 - u) * a.d);
+        rdh[u] = raw_load<DT, VEC>(a.dh, base + (te - 1 - u) * a.d);
       }
     }
 #pragma unroll
     for (int u = 0; u < kScanBwdFold; ++u) {
       if (te - 1 - u >= t0) {
+        float zf[VEC], dh[VEC];
+        raw_unpack<DT, VEC>(rzf[u], zf);
+        raw_unpack<DT, VEC>(rdh[u], dh);
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
           float f, omf;
-          hgrn_forget(zf[u][v], f, omf);
-          B[v] = f * (dh[u][v] + B[v]);
+          hgrn_forget(zf[v], f, omf);
+          B[v] = f * (dh[v] + B[v]);
           A[v] = f * A[v];
         }
       }
@@ -161,36 +200,42 @@ __global__ void __launch_bounds__(kScanBwdThreads) scan_bwd_replay_kernel(const 
     cterm[v] = SINGLE ? 0.0f : a.cin[((int64_t)bi * a.nchunk + c) * a.d + ch + v];
     hinit[v] = a.h0 ? a.h0[(int64_t)bi * a.d + ch + v] : 0.0f;
   }
+  using R = typename RawV<DT, VEC>::T;
   for (int64_t te = t1; te > t0; te -= kScanBwdReplay) {
-    float zf[kScanBwdReplay][VEC], zi[kScanBwdReplay][VEC], dh[kScanBwdReplay][VEC], hp[kScanBwdReplay][VEC];
+    R rzf[kScanBwdReplay], rzi[kScanBwdReplay], rdh[kScanBwdReplay], rhp[kScanBwdReplay];
 #pragma unroll
     for (int u = 0; u < kScanBwdReplay; ++u) {
       const int64_t t = te - 1 - u;
       if (t >= t0) {
-        load_vec<DT, VEC>(a.zf, base + t * a.d, zf[u]);
-        load_vec<DT, VEC>(a.zi, base + t * a.d, zi[u]);
-        load_vec<DT, VEC>(a.dh, base + t * a.d, dh[u]);
-        if (t > 0) {
-          load_vec<DT, VEC>(a.h, base + (t - 1) * a.d, hp[u]);
-        } else {
-#pragma unroll
-          for (int v = 0; v < VEC; ++v) hp[u][v] = hinit[v];
-        }
+        rzf[u] = raw_load<DT, VEC>(a.zf, base + t * a.d);
+        rzi[u] = raw_load<DT, VEC>(a.zi, base + t * a.d);
+        rdh[u] = raw_load<DT, VEC>(a.dh, base + t * a.d);
+        if (t > 0) rhp[u] = raw_load<DT, VEC>(a.h, base + (t - 1) * a.d);
       }
     }
 #pragma unroll
     for (int u = 0; u < kScanBwdReplay; ++u) {
       const int64_t t = te - 1 - u;
       if (t >= t0) {
+        float zf[VEC], zi[VEC], dh[VEC], hp[VEC];
+        raw_unpack<DT, VEC>(rzf[u], zf);
+        raw_unpack<DT, VEC>(rzi[u], zi);
+        raw_unpack<DT, VEC>(rdh[u], dh);
+        if (t > 0) {
+          raw_unpack<DT, VEC>(rhp[u], hp);
+        } else {
+#pragma unroll
+          for (int v = 0; v < VEC; ++v) hp[v] = hinit[v];
+        }
         float gzf[VEC], gzi[VEC];
 #pragma unroll
         for (int v = 0; v < VEC; ++v) {
-          const float G = dh[u][v] + cterm[v];
+          const float G = dh[v] + cterm[v];
           float f, omf;
-          hgrn_forget(zf[u][v], f, omf);
-          const float z = zi[u][v];
+          hgrn_forget(zf[v], f, omf);
+          const float z = zi[v];
           const float sz = sigmoidf_(z);
-          gzf[v] = (G * hp[u][v] - G * (z * sz)) * f * omf;
+          gzf[v] = (G * hp[v] - G * (z * sz)) * f * omf;
           gzi[v] = G * omf * sz * fmaf(z, 1.0f - sz, 1.0f);
           cterm[v] = f * G;
         }
@@ -266,15 +311,34 @@ __global__ void __launch_bounds__(kThreads) lin_bwd_dr_kernel(const LinBwdArgs a
     if (16 * w + j < a.k) a.dx[row * a.k + 16 * w + j] = acc[j] * s;
 }
 
-// dw[c] = sum_m dr[m][c] x[m][c] rho_m, one thread per column (coalesced across columns); m = 0
-// gives zeros.
-__global__ void __launch_bounds__(kThreads) lin_bwd_dnw_kernel(const LinBwdArgs a) {
+// dw[c] = sum_m dr[m][c] x[m][c] rho_m in two passes: blocks of 32 columns x 8 row lanes each add a
+// slice of rows_per rows into part[split][c] (blockIdx.y = split), then one thread per column
+// adds the splits in order (deterministic). Coalesced across columns throughout.
+__global__ void __launch_bounds__(256) lin_bwd_dnw_part_kernel(const LinBwdArgs a, float* part, int rows_per) {
+  __shared__ float red[8][33];
+  const int c = blockIdx.x * 32 + threadIdx.x;
+  const int64_t r0 = (int64_t)blockIdx.y * rows_per;
+  const int64_t r1 = r0 + rows_per < a.m ? r0 + rows_per : a.m;
+  float acc = 0.0f;
+  if (c < a.k)
+    for (int64_t row = r0 + threadIdx.y; row < r1; row += 8)
+      acc = fmaf(a.dx[row * a.k + c] * load_as_float(a.x, row * a.k + c, a.xdt), a.rho[row], acc);
+  red[threadIdx.y][threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.y == 0 && c < a.k) {
+    float t = 0.0f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) t += red[j][threadIdx.x];
+    part[(int64_t)blockIdx.y * a.k + c] = t;
+  }
+}
+__global__ void __launch_bounds__(kThreads) lin_bwd_dnw_reduce_kernel(const LinBwdArgs a, const float* part,
+                                                                      int splits) {
   const int c = blockIdx.x * kThreads + threadIdx.x;
   if (c >= a.k) return;
-  float acc = 0.0f;
-  for (int64_t row = 0; row < a.m; ++row)
-    acc = fmaf(a.dx[row * a.k + c] * load_as_float(a.x, row * a.k + c, a.xdt), a.rho[row], acc);
-  a.dnorm_w[c] = acc;
+  float t = 0.0f;
+  for (int z = 0; z < splits; ++z) t += part[(int64_t)z * a.k + c];
+  a.dnorm_w[c] = t;
 }
 
 // dx = rho u - rho^3 x mean(u x) with u = dr w, one CTA per row, in place over dr.
@@ -306,6 +370,67 @@ __global__ void __launch_bounds__(kThreads) lin_bwd_dw_kernel(const LinBwdArgs a
   for (int64_t row = 0; row < a.m; ++row)
     acc = fmaf(load_as_float(a.dy, row * a.n + nn, a.dydt) * a.deq[row], (float)a.q[row * a.k + c], acc);
   a.dW[(int64_t)nn * a.k + c] = acc;
+}
+
+// Operands of the tensor-core form of dr and dW (bf16_gemm_kernel): bf16 arrays, K-major, row
+// pitch ld (a multiple of 8 elements). A float32 value v enters as hi = bf16(v) and
+// lo = bf16(v - hi); the codes are exact in bf16.
+__device__ __forceinline__ void split_bf16(float v, __nv_bfloat16* hi, __nv_bfloat16* lo, int64_t idx) {
+  const __nv_bfloat16 h = __float2bfloat16_rn(v);
+  hi[idx] = h;
+  if (lo) lo[idx] = __float2bfloat16_rn(v - __bfloat162float(h));
+}
+
+// dr's A operand: dy [m][n] as hi / lo rows [m][ld].
+__global__ void __launch_bounds__(kThreads) lin_bwd_split_kernel(const LinBwdArgs a, __nv_bfloat16* hi,
+                                                                 __nv_bfloat16* lo, int64_t ld) {
+  const int64_t total = a.m * a.n;
+  for (int64_t e = (int64_t)blockIdx.x * kThreads + threadIdx.x; e < total; e += (int64_t)gridDim.x * kThreads) {
+    const int64_t r = e / a.n, c = e - r * a.n;
+    split_bf16(load_as_float(a.dy, e, a.dydt), hi, lo, r * ld + c);
+  }
+}
+
+// Transposed operands, dst[c][r] = value(r, c), through 32 x 32 shared-memory tiles (block 32 x 8;
+// blockIdx.x over rows r, blockIdx.y over columns c):
+//   kTrDyScaled  dW's A:  r = token, c = output feature: dy[r][c] * (a/127)_r as hi / lo   [n][ld]
+//   kTrCodes     dW's B:  r = token, c = input feature:  q[r][c]                            [k][ld]
+//   kTrTernary   dr's B:  r = weight row, c = input feature: t[r][c] from the packed words   [k][ld]
+enum TrMode : int { kTrDyScaled = 0, kTrCodes = 1, kTrTernary = 2 };
+
+template <int MODE>
+__global__ void __launch_bounds__(256) lin_bwd_transpose_kernel(const LinBwdArgs a, __nv_bfloat16* hi,
+                                                                __nv_bfloat16* lo, int64_t ld) {
+  __shared__ float tile[32][33];
+  const int64_t rows = MODE == kTrTernary ? (int64_t)a.n : a.m;
+  const int cols = MODE == kTrDyScaled ? a.n : a.k;
+  const int64_t r0 = (int64_t)blockIdx.x * 32;
+  const int c0 = blockIdx.y * 32;
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  for (int j = ty; j < 32; j += 8) {
+    const int64_t r = r0 + j;
+    const int c = c0 + tx;
+    float v = 0.0f;
+    if (r < rows && c < cols) {
+      if (MODE == kTrDyScaled) {
+        v = load_as_float(a.dy, r * a.n + c, a.dydt) * a.deq[r];
+      } else if (MODE == kTrCodes) {
+        v = (float)a.q[r * a.k + c];
+      } else {
+        const uint32_t word = a.codes[r * a.kw + (c >> 4)];
+        const int jj = c & 15, quad = jj >> 2, ln = jj & 3;
+        const uint32_t f = (word >> (16 * (quad >> 1) + 2 * (quad & 1) + 4 * ln)) & 3u;
+        v = f == 1u ? 1.0f : (f == 3u ? -1.0f : 0.0f);
+      }
+    }
+    tile[j][tx] = v;
+  }
+  __syncthreads();
+  for (int j = ty; j < 32; j += 8) {
+    const int c = c0 + j;
+    const int64_t r = r0 + tx;
+    if (c < cols && r < rows) split_bf16(tile[tx][j], hi, MODE == kTrDyScaled ? lo : nullptr, (int64_t)c * ld + r);
+  }
 }
 
 }  // namespace bwd

@@ -25,11 +25,13 @@ __device__ __forceinline__ void raise_device_error(unsigned code) { atomicOr(&g_
 template <mmf_dtype DT> struct Elem;
 template <> struct Elem<MMF_F32> {
   using T = float;
+  static __device__ __forceinline__ float to_float(T v) { return v; }
   static __device__ __forceinline__ float load(const T* p) { return *p; }
   static __device__ __forceinline__ void store(T* p, float v) { *p = v; }
 };
 template <> struct Elem<MMF_BF16> {
   using T = __nv_bfloat16;
+  static __device__ __forceinline__ float to_float(T v) { return __bfloat162float(v); }
   static __device__ __forceinline__ float load(const T* p) { return __bfloat162float(*p); }
   static __device__ __forceinline__ void store(T* p, float v) { *p = __float2bfloat16_rn(v); }
 };

@@ -64,23 +64,49 @@ __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a)
   for (int j = 0; j < KR; ++j)
     S[j] = (a.s0 && active && k0 + j < a.dk) ? a.s0[s_base + (int64_t)(k0 + j) * a.dv + v] : 0.0f;
 
+  // The next tile's q, f (kTS x DK values spread over the CTA) and this column's i (kTS values)
+  // are loaded into registers while the current tile runs, so no step waits on global memory.
+  constexpr int PER = kTS * DK / kThreads;
+  static_assert(PER * kThreads == kTS * DK, "tile split");
+  T rq[PER], rf[PER], ri[kTS];
+  auto load_tile = [&](int64_t tt) {
+    const int nn = (int)(a.t - tt < kTS ? a.t - tt : kTS);
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      const int e = threadIdx.x + r * kThreads;
+      const int st = e / DK, k = e - st * DK;
+      if (st < nn && k < a.dk) {
+        rq[r] = q[(tt + st) * qk_step + k];
+        rf[r] = f[(tt + st) * qk_step + k];
+      }
+    }
+#pragma unroll
+    for (int st = 0; st < kTS; ++st)
+      if (active && st < nn) ri[st] = in[(tt + st) * iv_step + v];
+  };
+  if (a.t > 0) load_tile(0);
   for (int64_t t0 = 0; t0 < a.t; t0 += kTS) {
     const int ns = (int)(a.t - t0 < kTS ? a.t - t0 : kTS);
     __syncthreads();  // every column is done with the previous tile
-    for (int e = threadIdx.x; e < kTS * DK; e += kThreads) {
-      const int s = e / DK, k = e - s * DK;
-      float qv = 0.0f, fv = 1.0f;
-      if (s < ns && k < a.dk) {
-        qv = Elem<DT>::load(q + (t0 + s) * qk_step + k);
-        fv = Elem<DT>::load(f + (t0 + s) * qk_step + k);
-      }
-      qs[s][k] = qv;
-      fs[s][k] = fv;
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      const int e = threadIdx.x + r * kThreads;
+      const int st = e / DK, k = e - st * DK;
+      const bool live = st < ns && k < a.dk;
+      qs[st][k] = live ? Elem<DT>::to_float(rq[r]) : 0.0f;
+      fs[st][k] = live ? Elem<DT>::to_float(rf[r]) : 1.0f;
     }
+    float ivs[kTS];
+#pragma unroll
+    for (int st = 0; st < kTS; ++st) ivs[st] = active && st < ns ? Elem<DT>::to_float(ri[st]) : 0.0f;
     __syncthreads();
+    if (t0 + kTS < a.t) load_tile(t0 + kTS);
     // (inactive columns take part in the shuffles with zero contributions)
+#pragma unroll 1
     for (int s = 0; s < ns; ++s) {
-      const float iv = active ? Elem<DT>::load(in + (t0 + s) * iv_step + v) : 0.0f;
+      float iv = ivs[0];
+#pragma unroll
+      for (int st = 1; st < kTS; ++st) iv = s == st ? ivs[st] : iv;
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int j = 0; j < KR; j += 4) {

@@ -17,6 +17,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "decode_rows.cuh"
+#include "gemm_bf16.cuh"
 #include "gemm_skinny.cuh"
 #include "gemm_tc.cuh"
 #include "head.cuh"
@@ -191,6 +192,7 @@ mmf_status device_info(DevInfo** out) {
       MMF_CUDA((head_attrs<MMF_BF16, MMF_F32>()));
       MMF_CUDA((head_attrs<MMF_BF16, MMF_BF16>()));
       MMF_CUDA(head_tc_attrs());
+      MMF_CUDA(cudaFuncSetAttribute(gb::bf16_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gb::SMEM_BYTES));
       MMF_CUDA(cudaFuncSetAttribute(sk::ternary_gemm_skinny_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     sk::Layout<16>::SMEM));
       MMF_CUDA(cudaFuncSetAttribute(sk::ternary_gemm_skinny_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -973,6 +975,57 @@ mmf_status head_tc_pass(const void* x, mmf_dtype xdt, int nb, int d, const float
 // =============================================================================================
 // exported C ABI
 // =============================================================================================
+// Tensor-core form of mmf_bitlinear_backward: the bf16 operand arrays (row pitch rounded up to 8
+// elements) and the K split of both products, from (m, k, n) alone so that the workspace query
+// and the launch agree. dr's arrays and dW's share the space after rho (the products run in
+// turn on one stream).
+struct LinBwdPlan {
+  int64_t ld_n, ld_m;
+  size_t rho, dr_hi, dr_lo, tt, dr_part, dw_hi, dw_lo, qt, dw_part, dnw_part, bytes;
+  int dr_split, dr_kbc, dw_split, dw_kbc, dnw_split, dnw_rows;
+};
+// Splits of K so that an M x N product with few tiles still covers the SMs: floor(148 / tiles),
+// at most 16 and at most the k-block count; every split gets at least one k-block.
+inline void gb_split(int64_t M, int64_t N, int64_t K, int& splits, int& kbc) {
+  const int64_t tiles = ((M + gb::BM - 1) / gb::BM) * ((N + gb::BN - 1) / gb::BN);
+  const int64_t nkb = std::max<int64_t>((K + gb::BK - 1) / gb::BK, 1);
+  int64_t sp = std::max<int64_t>(148 / std::max<int64_t>(tiles, 1), 1);
+  sp = std::min<int64_t>(sp, std::min<int64_t>(nkb, 16));
+  kbc = (int)((nkb + sp - 1) / sp);
+  splits = (int)((nkb + kbc - 1) / kbc);
+}
+inline LinBwdPlan lin_bwd_plan(int64_t m, int32_t k, int32_t n) {
+  LinBwdPlan P;
+  memset(&P, 0, sizeof(P));
+  P.ld_n = ((int64_t)n + 7) / 8 * 8;
+  P.ld_m = (m + 7) / 8 * 8;
+  P.rho = 0;
+  const size_t base = align256((size_t)m * 4);
+  size_t o = base;
+  P.dr_hi = o; o += align256((size_t)m * P.ld_n * 2);
+  P.dr_lo = o; o += align256((size_t)m * P.ld_n * 2);
+  P.tt = o; o += align256((size_t)k * P.ld_n * 2);
+  gb_split(m, k, n, P.dr_split, P.dr_kbc);
+  P.dr_part = o;
+  if (P.dr_split > 1) o += align256((size_t)P.dr_split * m * k * 4);
+  const size_t end_dr = o;
+  o = base;
+  P.dw_hi = o; o += align256((size_t)n * P.ld_m * 2);
+  P.dw_lo = o; o += align256((size_t)n * P.ld_m * 2);
+  P.qt = o; o += align256((size_t)k * P.ld_m * 2);
+  gb_split(n, k, m, P.dw_split, P.dw_kbc);
+  P.dw_part = o;
+  if (P.dw_split > 1) o += align256((size_t)P.dw_split * n * k * 4);
+  // the gain's gradient: row slices of at least 32 rows, at most 128 slices (between the two
+  // products, so it reuses the same space)
+  P.dnw_split = (int)std::max<int64_t>(std::min<int64_t>((m + 31) / 32, 128), 1);
+  P.dnw_rows = (int)std::max<int64_t>((m + P.dnw_split - 1) / P.dnw_split, 1);
+  P.dnw_part = base;
+  const size_t end_dnw = base + align256((size_t)P.dnw_split * k * 4);
+  P.bytes = std::max(std::max(end_dr, o), end_dnw);
+  return P;
+}
+
 extern "C" {
 
 int32_t mmf_packed_row_words(int32_t k) { return k <= 0 ? 0 : row_words(k); }
@@ -995,6 +1048,8 @@ size_t mmf_workspace_bytes(mmf_op op, int64_t m, int32_t d, int32_t inner, int32
       return d > 0 ? scan_ws_bytes(m, d) : 0;
     case MMF_OP_HEAD:
       return inner > 0 ? head_ws_bytes(inner, d) : 0;
+    case MMF_OP_BITLINEAR_BWD:
+      return d > 0 && inner > 0 ? lin_bwd_plan(m, d, inner).bytes : 0;
     case MMF_OP_DECODE:
       return decode_ws_head(m, d, inner) + 2 * align256((size_t)m * d * 4);
     case MMF_OP_STACK:
@@ -1494,6 +1549,42 @@ mmf_status decode_impl(const mmf_block_weights* layers, int32_t n_layers, const 
 
 }  // namespace
 
+// D [M][N] (row pitch ldd) = alpha * (Ahi + Alo) . B^T on the bf16 tensor cores; A [M][K] and
+// B [N][K] bf16 with row pitches lda, ldb (multiples of 8). Returns the number of launches.
+mmf_status launch_bf16_gemm(const void* a_hi, const void* a_lo, int64_t lda, const void* b, int64_t ldb,
+                            int64_t M, int64_t N, int64_t K, const float* alpha, float* d, int64_t ldd, int splits,
+                            int kbc, float* part, cudaStream_t st, int* launches) {
+  gb::Params P;
+  memset(&P, 0, sizeof(P));
+  MMF_TRY(encode_2d(&P.a_hi, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_hi, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2,
+                    gb::BK, gb::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  if (a_lo)
+    MMF_TRY(encode_2d(&P.a_lo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a_lo, (uint64_t)K, (uint64_t)M, (uint64_t)lda * 2,
+                      gb::BK, gb::BM, CU_TENSOR_MAP_SWIZZLE_128B));
+  MMF_TRY(encode_2d(&P.b, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, b, (uint64_t)K, (uint64_t)N, (uint64_t)ldb * 2, gb::BK,
+                    gb::BN, CU_TENSOR_MAP_SWIZZLE_128B));
+  P.m = (int32_t)M;
+  P.n = (int32_t)N;
+  P.num_kb = (int32_t)std::max<int64_t>((K + gb::BK - 1) / gb::BK, 1);
+  P.kb_per_cta = kbc;
+  P.has_lo = a_lo ? 1 : 0;
+  P.alpha = alpha;
+  P.d = d;
+  P.ldd = ldd;
+  P.part = splits > 1 ? part : nullptr;
+  P.wait_limit_us = g_wait_limit.load();
+  const dim3 grid((unsigned)((N + gb::BN - 1) / gb::BN), (unsigned)((M + gb::BM - 1) / gb::BM), (unsigned)splits);
+  launch_k(gb::bf16_gemm_kernel, grid, dim3(gb::THREADS), gb::SMEM_BYTES, st, P);
+  ++*launches;
+  if (splits > 1) {
+    const int64_t total = M * N;
+    launch_k(gb::bf16_gemm_reduce_kernel, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st, part, splits,
+             (int32_t)M, (int32_t)N, alpha, d, ldd);
+    ++*launches;
+  }
+  return MMF_OK;
+}
+
 // Steps per chunk of the chunked scan backward: the whole sequence up to 32 steps, 32 up to 4096
 // steps, then a multiple of 16 giving at most 128 chunks; so b * nchunk <= ceil(b t / 8) and the
 // forward scan's scratch size bounds the three [b][nchunk][d] arrays.
@@ -1704,7 +1795,8 @@ mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, c
   MMF_CHECK_ARG(m >= 0 && m <= 0x7fffffff, "bitlinear backward: m = %lld", (long long)m);
   MMF_CHECK_ARG(valid_dtype(x_dtype) && valid_dtype(dy_dtype), "bitlinear backward: bad dtype");
   MMF_CHECK_ARG(m == 0 || (x && q && deq && dy && dx), "bitlinear backward: null pointer");
-  if (m > 0) MMF_TRY(check_ws(ws, ws_bytes, align256((size_t)m * 4)));
+  const LinBwdPlan plan = lin_bwd_plan(m, w->k, w->n);
+  if (m > 0) MMF_TRY(check_ws(ws, ws_bytes, plan.bytes));
   DevInfo* di;
   MMF_TRY(device_info(&di));
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -1713,7 +1805,10 @@ mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, c
   a.x = x; a.xdt = x_dtype; a.m = m; a.k = w->k; a.n = w->n; a.norm_w = norm_w; a.eps = eps;
   a.codes = w->codes; a.kw = row_words(w->k); a.scale = w->scale; a.q = q; a.deq = deq;
   a.dy = dy; a.dydt = dy_dtype; a.dx = dx; a.dnorm_w = dnorm_w; a.dW = dW;
-  a.rho = reinterpret_cast<float*>(ws);
+  uint8_t* wsb = reinterpret_cast<uint8_t*>(ws);
+  a.rho = reinterpret_cast<float*>(wsb + plan.rho);
+  // dr and dW on the tensor cores unless the CUDA-core engine is forced (mmf_set_gemm_path)
+  const bool tc = g_gemm_path.load() != MMF_GEMM_SIMT && di->tc_ready;
   const unsigned kcols = (unsigned)((w->k + bwd::kThreads - 1) / bwd::kThreads);
   LaunchScope ls(MMF_KERNEL_OTHER, (double)m * (w->k * (dsize(x_dtype) + 1.0 + 8.0) + w->n * dsize(dy_dtype)) +
                  (double)w->n * row_words(w->k) * 4.0, st);
@@ -1721,14 +1816,65 @@ mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, c
   if (m > 0) {
     launch_k(bwd::lin_bwd_rho_kernel, dim3((unsigned)((m + bwd::kThreads / 32 - 1) / (bwd::kThreads / 32))),
              dim3(bwd::kThreads), 0, st, a);
-    const unsigned words = (unsigned)((w->k + 15) / 16);
-    launch_k(bwd::lin_bwd_dr_kernel, dim3((unsigned)m, (words + bwd::kThreads - 1) / bwd::kThreads), dim3(bwd::kThreads),
-             0, st, a);
-    launches += 2;
+    ++launches;
+    if (tc) {
+      // dr [m][k] = s * dy [m][n] . t [n][k]: A = dy (bf16 as given, else hi / lo rows),
+      // B = t transposed to [k][n]
+      const bool direct = dy_dtype == MMF_BF16 && w->n % 8 == 0 && aligned16(dy);
+      __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(wsb + plan.dr_hi);
+      __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(wsb + plan.dr_lo);
+      __nv_bfloat16* tt = reinterpret_cast<__nv_bfloat16*>(wsb + plan.tt);
+      if (!direct) {
+        const int64_t total = m * w->n;
+        const unsigned blocks = (unsigned)std::min<int64_t>((total + bwd::kThreads - 1) / bwd::kThreads, (int64_t)di->sms * 16);
+        launch_k(bwd::lin_bwd_split_kernel, dim3(blocks), dim3(bwd::kThreads), 0, st, a, hi,
+                 dy_dtype == MMF_BF16 ? nullptr : lo, plan.ld_n);
+        ++launches;
+      }
+      launch_k(bwd::lin_bwd_transpose_kernel<bwd::kTrTernary>, dim3((unsigned)((w->n + 31) / 32), (unsigned)((w->k + 31) / 32)),
+               dim3(32, 8), 0, st, a, tt, nullptr, plan.ld_n);
+      ++launches;
+      MMF_TRY(launch_bf16_gemm(direct ? dy : hi, direct || dy_dtype == MMF_BF16 ? nullptr : lo,
+                               direct ? (int64_t)w->n : plan.ld_n, tt, plan.ld_n, m, w->k, w->n, w->scale, dx, w->k,
+                               plan.dr_split, plan.dr_kbc, reinterpret_cast<float*>(wsb + plan.dr_part), st, &launches));
+    } else {
+      const unsigned words = (unsigned)((w->k + 15) / 16);
+      launch_k(bwd::lin_bwd_dr_kernel, dim3((unsigned)m, (words + bwd::kThreads - 1) / bwd::kThreads), dim3(bwd::kThreads),
+               0, st, a);
+      ++launches;
+    }
   }
-  if (dnorm_w) { launch_k(bwd::lin_bwd_dnw_kernel, dim3(kcols), dim3(bwd::kThreads), 0, st, a); ++launches; }
+  if (dnorm_w) {
+    if (m > 0) {
+      float* part = reinterpret_cast<float*>(wsb + plan.dnw_part);
+      launch_k(bwd::lin_bwd_dnw_part_kernel, dim3((unsigned)((w->k + 31) / 32), (unsigned)plan.dnw_split), dim3(32, 8), 0,
+               st, a, part, plan.dnw_rows);
+      launch_k(bwd::lin_bwd_dnw_reduce_kernel, dim3(kcols), dim3(bwd::kThreads), 0, st, a, part, plan.dnw_split);
+      launches += 2;
+    } else {
+      cudaError_t e = cudaMemsetAsync(dnorm_w, 0, (size_t)w->k * sizeof(float), st);
+      if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+    }
+  }
   if (m > 0) { launch_k(bwd::lin_bwd_dx_kernel, dim3((unsigned)m), dim3(bwd::kThreads), 0, st, a); ++launches; }
-  if (dW) { launch_k(bwd::lin_bwd_dw_kernel, dim3(kcols, (unsigned)w->n), dim3(bwd::kThreads), 0, st, a); ++launches; }
+  if (dW && tc && m > 0) {
+    // dW [n][k] = (dy (a/127))^T [n][m] . q [m][k]: A = dy scaled and transposed (hi / lo),
+    // B = q transposed to [k][m]
+    __nv_bfloat16* hi = reinterpret_cast<__nv_bfloat16*>(wsb + plan.dw_hi);
+    __nv_bfloat16* lo = reinterpret_cast<__nv_bfloat16*>(wsb + plan.dw_lo);
+    __nv_bfloat16* qt = reinterpret_cast<__nv_bfloat16*>(wsb + plan.qt);
+    const unsigned rt = (unsigned)((m + 31) / 32);
+    launch_k(bwd::lin_bwd_transpose_kernel<bwd::kTrDyScaled>, dim3(rt, (unsigned)((w->n + 31) / 32)), dim3(32, 8), 0, st,
+             a, hi, lo, plan.ld_m);
+    launch_k(bwd::lin_bwd_transpose_kernel<bwd::kTrCodes>, dim3(rt, (unsigned)((w->k + 31) / 32)), dim3(32, 8), 0, st,
+             a, qt, nullptr, plan.ld_m);
+    launches += 2;
+    MMF_TRY(launch_bf16_gemm(hi, lo, plan.ld_m, qt, plan.ld_m, w->n, w->k, m, nullptr, dW, w->k, plan.dw_split,
+                             plan.dw_kbc, reinterpret_cast<float*>(wsb + plan.dw_part), st, &launches));
+  } else if (dW) {
+    launch_k(bwd::lin_bwd_dw_kernel, dim3(kcols, (unsigned)w->n), dim3(bwd::kThreads), 0, st, a);
+    ++launches;
+  }
   if (launches > 0) g_launches.fetch_add(launches - 1);  // the timing scope counted one launch itself
   else g_launches.fetch_sub(1);
   return check_launch("bitlinear backward kernels");

@@ -145,6 +145,14 @@ def test_bitlinear_backward_arguments_on_host(L):
               None) == mmf.MMF_ERR_INVALID_ARG                                                     # null q
     assert bb(16, 0, 1000, None, 1e-8, ctypes.byref(ok_w), 16, 16, 16, 0, 16, None, None, 256, 1024,
               None) == mmf.MMF_ERR_WORKSPACE                                                       # 4 KB needed
+    # the workspace holds rho and the bf16 operands of the tensor-core products (dr's dy hi / lo
+    # [m][n] and t^T [k][n]; dW's scaled dy^T hi / lo [n][m] and q^T [k][m], sharing the space)
+    m, k, n = 1000, 64, 8
+    need = mmf.workspace_bytes(mmf.MMF_OP_BITLINEAR_BWD, m, k, n, 0)
+    assert need >= 4 * m + max(2 * m * n * 2 + k * n * 2, 2 * n * m * 2 + k * m * 2)
+    assert bb(16, 0, m, None, 1e-8, ctypes.byref(ok_w), 16, 16, 16, 0, 16, None, None, 256, need - 1,
+              None) == mmf.MMF_ERR_WORKSPACE
+    assert mmf.workspace_bytes(mmf.MMF_OP_BITLINEAR_BWD, 0, k, n, 0) == 0 or m > 0
 
 
 def test_block_shape_mismatch_rejected(L):

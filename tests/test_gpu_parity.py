@@ -627,11 +627,16 @@ def test_scan_backward_parity(mmf, dt, b, t, d, long_memory):
 # BitLinear gradients with the straight-through estimator against the oracle, on the forward's own
 # activation codes (the kernel backward takes them from mmf_bitlinear_fwd, whose codes the forward
 # parity tests check against the oracle's): dx and the gain's gradient against the oracle's RMSNorm
-# backward of dr = dy (t s), dW against dy^T (q a/127) with the forward's q and a/127. float32
-# accumulation over n (dr) or m (dW): within 1e-4 of the largest value.
+# backward of dr = dy (t s), dW against dy^T (q a/127) with the forward's q and a/127. On the
+# tensor cores dy enters as bf16 hi / lo pairs (about 2^-17 relative per term) and the codes are
+# exact; on the CUDA cores everything is float32. float32 accumulation over n (dr) or m (dW):
+# within 1e-4 of the largest value either way. Shapes: ragged n and k (scalar epilogue stores,
+# split dy rows), n a multiple of 8 (bf16 dy used in place), m large enough for a K split of dW
+# (the partials added by the reduction kernel), m = 0.
+@pytest.mark.parametrize("engine", ["tensor", "simt"])
 @pytest.mark.parametrize("xdt", ["f32", "bf16"])
-@pytest.mark.parametrize("m,n,k", [(5, 33, 200), (64, 128, 256), (0, 16, 64)])
-def test_bitlinear_backward_parity(mmf, xdt, m, n, k):
+@pytest.mark.parametrize("m,n,k", [(5, 33, 200), (64, 128, 256), (0, 16, 64), (300, 640, 1024), (2000, 72, 88)])
+def test_bitlinear_backward_parity(mmf, engine, xdt, m, n, k):
     dts = {"f32": torch.float32, "bf16": torch.bfloat16}
     x = _to(synth.activations(100, (m, k)), dts[xdt])
     nw = synth.norm_weight(101, k, random=True)
@@ -639,8 +644,12 @@ def test_bitlinear_backward_parity(mmf, xdt, m, n, k):
     w = mmf.pack_ternary(_to(Wl))
     dy = _to(synth.activations(103, (m, n)), dts[xdt])
     _, q, deq, _ = mmf.bitlinear_fwd(x, _to(nw), w, y_dtype=torch.float32, debug=True)
-    dx, dnw, dW = mmf.bitlinear_backward(x, _to(nw), w, q, deq, dy)
-    _ok(mmf)
+    mmf.set_gemm_path(mmf.MMF_GEMM_SIMT if engine == "simt" else mmf.MMF_GEMM_TENSOR)
+    try:
+        dx, dnw, dW = mmf.bitlinear_backward(x, _to(nw), w, q, deq, dy)
+        _ok(mmf)
+    finally:
+        mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
     t, s = O.ternarize(Wl)
     x64, dy64 = _np(x).astype(np.float64), _np(dy).astype(np.float64)
     dr = dy64 @ (t.astype(np.float64) * float(s))
