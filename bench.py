@@ -103,6 +103,13 @@ def int8_peak(peaks: dict) -> tuple[float, str]:
     return 1590.0 * INT8_OVER_BF16, "of fallback: 1.59 PFLOP/s bf16 burst x nominal ratio 2"
 
 
+def bf16_peak(peaks: dict) -> tuple[float, str]:
+    """The measured burst bf16 cuBLAS figure (for a kernel timed alone)."""
+    if peaks.get("bf16_tflops"):
+        return peaks["bf16_tflops"], "of measured: bf16 burst cuBLAS"
+    return 1590.0, "of fallback: 1.59 PFLOP/s bf16 burst"
+
+
 def hbm_peak(peaks: dict) -> tuple[float, str]:
     if peaks.get("hbm_gbs"):
         return peaks["hbm_gbs"], "of measured: STREAM-style copy"
@@ -646,7 +653,7 @@ def run_sweeps(device, flush, peaks) -> dict:
 def run_next_rows(device, flush, peaks) -> dict:
     """The next-row kernels timed alone (median of a few calls, L2 flushed before each): the HGRN2
     recurrence (step by step on the CUDA cores), the scan gradients and the BitLinear gradients
-    (straight-through estimator, CUDA cores)."""
+    (straight-through estimator; dr and dW on the bf16 tensor cores)."""
     import torch
 
     import ternary_weight_matmul_b200 as mmf
@@ -695,18 +702,23 @@ def run_next_rows(device, flush, peaks) -> dict:
     out["hgrn_scan_backward"] = {"shape": f"B {B} T {T} d {d} bf16", "ms": ms, "GB/s": byts / (ms / 1e3) / 1e9,
                                  "frac_hbm": byts / (ms / 1e3) / 1e9 / hbm, "bound": "hbm"}
     del zf, zi, h, dh
-    # BitLinear backward: 4096 rows, K = N = 1024, bf16 activations and gradients
-    m, k, n = 4096, 1024, 1024
-    w = mmf.pack_ternary(torch.randn(n, k, generator=g, device=device) * 0.02)
-    x = torch.randn(m, k, generator=g, device=device).to(torch.bfloat16)
-    nw = torch.ones(k, device=device)
-    _, qq, deq, _ = mmf.bitlinear_fwd(x, nw, w, y_dtype=torch.float32, debug=True)
-    dy = torch.randn(m, n, generator=g, device=device).to(torch.bfloat16)
-    ms = median_ms(lambda: mmf.bitlinear_backward(x, nw, w, qq, deq, dy))
-    flops = 2 * 2.0 * m * n * k   # dr and dW
-    out["bitlinear_backward"] = {"shape": f"M {m} K {k} N {n} bf16", "ms": ms, "TFLOP/s": flops / (ms / 1e3) / 1e12,
-                                 "frac_fp32_fma_peak": flops / (ms / 1e3) / 1e12 / FP32_FMA_TFLOPS,
-                                 "bound": "alu", "peak_source": "CUDA-core fp32 FMA peak from unit counts x 1.965 GHz"}
+    # BitLinear backward, bf16 activations and gradients: 4096 rows with K = N = 1024, and the
+    # 370M prefill's gate_proj (16384 rows, K 1024, N 2816). The whole call (operand layout, the
+    # two tensor-core products, rho, the gain's gradient, dx) against the bf16 tensor peak for
+    # dr + dW's algorithmic 4 m n k flops (the hi / lo pairs issue twice that on the MMA)
+    bpk, bsrc = bf16_peak(peaks)
+    for key, (m, k, n) in (("bitlinear_backward", (4096, 1024, 1024)),
+                           ("bitlinear_backward_370M_gate", (16384, 1024, 2816))):
+        w = mmf.pack_ternary(torch.randn(n, k, generator=g, device=device) * 0.02)
+        x = torch.randn(m, k, generator=g, device=device).to(torch.bfloat16)
+        nw = torch.ones(k, device=device)
+        _, qq, deq, _ = mmf.bitlinear_fwd(x, nw, w, y_dtype=torch.float32, debug=True)
+        dy = torch.randn(m, n, generator=g, device=device).to(torch.bfloat16)
+        ms = median_ms(lambda: mmf.bitlinear_backward(x, nw, w, qq, deq, dy))
+        flops = 2 * 2.0 * m * n * k   # dr and dW
+        out[key] = {"shape": f"M {m} K {k} N {n} bf16", "ms": ms, "TFLOP/s": flops / (ms / 1e3) / 1e12,
+                    "frac_bf16_peak": flops / (ms / 1e3) / 1e12 / bpk, "bound": "tensor", "peak_source": bsrc}
+        del w, x, qq, deq, dy
     if mmf.sync_status(device) != 0:
         raise RuntimeError("device status after the next-row kernels")
     return out

@@ -186,16 +186,17 @@ __global__ void __launch_bounds__(THREADS) bf16_gemm_kernel(const __grid_constan
 }
 
 // d[i][j] = alpha * sum_z part[z][i][j] (alpha = 1 when alpha_p is null), the partials added in
-// split order (deterministic).
+// split order (deterministic); blockIdx.x = row i, 256 columns per block.
 __global__ void __launch_bounds__(256) bf16_gemm_reduce_kernel(const float* __restrict__ part, int splits,
                                                                int32_t m, int32_t n, const float* alpha_p,
                                                                float* __restrict__ d, int64_t ldd) {
-  const int64_t idx = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  const int64_t i = blockIdx.x;
+  const int j = blockIdx.y * 256 + threadIdx.x;
+  if (j >= n) return;
   const int64_t total = (int64_t)m * n;
-  if (idx >= total) return;
-  const int64_t i = idx / n, j = idx - i * n;
+  const float* p = part + i * n + j;
   float s = 0.0f;
-  for (int z = 0; z < splits; ++z) s += part[(int64_t)z * total + idx];
+  for (int z = 0; z < splits; ++z) s += p[(int64_t)z * total];
   d[i * ldd + j] = alpha_p ? s * *alpha_p : s;
 }
 

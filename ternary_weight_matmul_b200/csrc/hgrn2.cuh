@@ -10,7 +10,8 @@
 // i[v]); only the readout o_t[v] = q_t . S_t[:, v] sums over k. Four adjacent threads share one
 // column, each keeping dk / 4 state rows in registers for the whole sequence, and combine their
 // partial readouts with two shuffles per step; the partial readout runs as four independent FMA
-// chains. A CTA serves 32 columns of one (sequence, head); per tile of kTS steps it stages q_t and
+// chains. Thread `sub` of a column owns the rows 16 g + 4 sub + (0..3) for g = 0, 1, ..., so the
+// four threads' 16-byte reads of q_t and f_t at one g are adjacent (no bank conflict). A CTA serves 32 columns of one (sequence, head); per tile of kTS steps it stages q_t and
 // f_t (dk values each, shared by every column) in shared memory as float32. Rows past dk are
 // padded with q = 0 and f = 1 (key 0), so they stay zero and never contribute.
 #pragma once
@@ -47,7 +48,8 @@ __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a)
   __shared__ __align__(16) float qs[kTS][DK];
   __shared__ __align__(16) float fs[kTS][DK];
   const int sub = threadIdx.x & (kSplit - 1);
-  const int k0 = sub * KR;
+  // state row of register j: 16 (j / 4) + 4 sub + j % 4
+  auto krow = [&](int j) { return 16 * (j >> 2) + 4 * sub + (j & 3); };
   const int v = blockIdx.x * kCols + (threadIdx.x >> 2);
   const int h = blockIdx.y, bi = blockIdx.z;
   const bool active = v < a.dv;
@@ -62,7 +64,7 @@ __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a)
   float S[KR];
 #pragma unroll
   for (int j = 0; j < KR; ++j)
-    S[j] = (a.s0 && active && k0 + j < a.dk) ? a.s0[s_base + (int64_t)(k0 + j) * a.dv + v] : 0.0f;
+    S[j] = (a.s0 && active && krow(j) < a.dk) ? a.s0[s_base + (int64_t)krow(j) * a.dv + v] : 0.0f;
 
   // The next tile's q, f (kTS x DK values spread over the CTA) and this column's i (kTS values)
   // are loaded into registers while the current tile runs, so no step waits on global memory.
@@ -110,8 +112,8 @@ __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a)
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int j = 0; j < KR; j += 4) {
-        const float4 f4 = *reinterpret_cast<const float4*>(&fs[s][k0 + j]);
-        const float4 q4 = *reinterpret_cast<const float4*>(&qs[s][k0 + j]);
+        const float4 f4 = *reinterpret_cast<const float4*>(&fs[s][krow(j)]);
+        const float4 q4 = *reinterpret_cast<const float4*>(&qs[s][krow(j)]);
         S[j] = fmaf(f4.x, S[j], (1.0f - f4.x) * iv);
         S[j + 1] = fmaf(f4.y, S[j + 1], (1.0f - f4.y) * iv);
         S[j + 2] = fmaf(f4.z, S[j + 2], (1.0f - f4.z) * iv);
@@ -130,7 +132,7 @@ __global__ void __launch_bounds__(kThreads) hgrn2_recurrent_kernel(const Args a)
   if (active && a.s_out) {
 #pragma unroll
     for (int j = 0; j < KR; ++j)
-      if (k0 + j < a.dk) a.s_out[s_base + (int64_t)(k0 + j) * a.dv + v] = S[j];
+      if (krow(j) < a.dk) a.s_out[s_base + (int64_t)krow(j) * a.dv + v] = S[j];
   }
 }
 

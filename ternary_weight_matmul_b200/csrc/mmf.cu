@@ -1016,9 +1016,9 @@ inline LinBwdPlan lin_bwd_plan(int64_t m, int32_t k, int32_t n) {
   gb_split(n, k, m, P.dw_split, P.dw_kbc);
   P.dw_part = o;
   if (P.dw_split > 1) o += align256((size_t)P.dw_split * n * k * 4);
-  // the gain's gradient: row slices of at least 32 rows, at most 128 slices (between the two
+  // the gain's gradient: row slices of at least 128 rows, at most 64 slices (between the two
   // products, so it reuses the same space)
-  P.dnw_split = (int)std::max<int64_t>(std::min<int64_t>((m + 31) / 32, 128), 1);
+  P.dnw_split = (int)std::max<int64_t>(std::min<int64_t>((m + 127) / 128, 64), 1);
   P.dnw_rows = (int)std::max<int64_t>((m + P.dnw_split - 1) / P.dnw_split, 1);
   P.dnw_part = base;
   const size_t end_dnw = base + align256((size_t)P.dnw_split * k * 4);
@@ -1577,9 +1577,8 @@ mmf_status launch_bf16_gemm(const void* a_hi, const void* a_lo, int64_t lda, con
   launch_k(gb::bf16_gemm_kernel, grid, dim3(gb::THREADS), gb::SMEM_BYTES, st, P);
   ++*launches;
   if (splits > 1) {
-    const int64_t total = M * N;
-    launch_k(gb::bf16_gemm_reduce_kernel, dim3((unsigned)((total + 255) / 256)), dim3(256), 0, st, part, splits,
-             (int32_t)M, (int32_t)N, alpha, d, ldd);
+    launch_k(gb::bf16_gemm_reduce_kernel, dim3((unsigned)M, (unsigned)((N + 255) / 256)), dim3(256), 0, st, part,
+             splits, (int32_t)M, (int32_t)N, alpha, d, ldd);
     ++*launches;
   }
   return MMF_OK;
