@@ -50,15 +50,16 @@ constexpr uint32_t A_COLS = BK / 4;      // TMEM columns of one expanded A stage
 constexpr uint32_t A_COL = 2 * BN;       // A stages at 256 + 64 * s
 static_assert(A_COL + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
 
-// Epilogue staging: the raw int32 accumulators of a 32-token chunk, [32 tokens][128 rows],
-// double-buffered (2 x 16 KB). Within a token's 512-byte row the 16-byte chunk c sits at
+// Epilogue staging: the raw int32 accumulators of a 64-token chunk, [64 tokens][128 rows], one
+// 32 KB buffer (two chunks per tile; fewer, larger rounds measured faster than four 32-token
+// rounds on two buffers). Within a token's 512-byte row the 16-byte chunk c sits at
 // c ^ ((c >> 3) & 1), which keeps both the row-wise writes and the 32-byte piece reads free of
 // bank conflicts.
-constexpr int EPI_CHUNK = 32;
+constexpr int EPI_CHUNK = 64;
 constexpr int EPI_BUF_BYTES = EPI_CHUNK * BM * 4;
 constexpr int SMEM_W_OFF = STAGES * ACT_BYTES;
 constexpr int SMEM_EPI_OFF = SMEM_W_OFF + STAGES * W_BYTES;
-constexpr int SMEM_DQ_OFF = SMEM_EPI_OFF + 2 * EPI_BUF_BYTES;  // per-token (a/127)*s, 2 x BN floats
+constexpr int SMEM_DQ_OFF = SMEM_EPI_OFF + EPI_BUF_BYTES;  // per-token (a/127)*s, 2 x BN floats
 // residual tile (bf16 outputs), prefetched by the epilogue threads with cp.async before they wait
 // for the tile's accumulators: [chunk][piece][8 values], each thread reading back what it copied
 constexpr int RES_BYTES = BN * BM * 2;
@@ -332,21 +333,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
     }
   } else {
     // ------------------------------------------------------------------ epilogue
-    // Two phases per 32-token chunk. Phase 1: each warp loads its sub-partition's 32 weight rows
-    // x 16 tokens (its half of the chunk) of int32 accumulators from TMEM (thread = row) and
-    // stores them to shared memory transposed, as [token][row] (one conflict-free 32-bit store
-    // per element). Phase 2: the 256 epilogue threads walk the chunk token-major in pieces of
+    // Two phases per 64-token chunk. Phase 1: each warp loads its sub-partition's 32 weight rows
+    // x 32 tokens (its half of the chunk, 16 at a time) of int32 accumulators from TMEM (thread =
+    // row) and stores them to shared memory transposed, as [token][row] (one conflict-free 32-bit
+    // store per element); the second chunk waits for the first one's reads of the single staging
+    // buffer (a barrier). Phase 2: the 256 epilogue threads walk the chunk token-major in pieces of
     // 8 output columns, rescale by (a/127) * s of the token, add the residual (or, for a GLU
     // tile, form SiLU(gate) * up from rows r and 64 + r) and write 16- or 32-byte vectors, so
     // every global access covers whole row segments of the output.
     const uint32_t sub = (uint32_t)(warp & 3);
-    const int half = (warp - 6) >> 2;        // which 16 tokens of a chunk this warp loads
+    const int half = (warp - 6) >> 2;        // which 32 tokens of a chunk this warp loads
     const int row = (int)sub * 32 + lane;
     const int srow = epi_word(row);
     const uint32_t lane_addr = (sub * 32u) << 16;
     const int etid = threadIdx.x - 6 * 32;  // 0..255
     const bool small_acc = P.small_acc != 0;
-    uint32_t tl = 0, chunk_ctr = 0;
+    uint32_t tl = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++tl) {
       const uint32_t b = tl & 1u;
       int seg, nt, mt;
@@ -362,10 +364,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
 #pragma unroll
           for (int ci = 0; ci < BN / EPI_CHUNK; ++ci) {
 #pragma unroll
-            for (int itp = 0; itp < 2; ++itp) {
+            for (int itp = 0; itp < 4; ++itp) {
               const int pidx = etid + itp * EPI_THREADS;
               const int64_t m = (int64_t)mt * BN + ci * EPI_CHUNK + (pidx >> 4);
-              if (m < P.g.m) cp_async16(res_s + (ci * 2 * EPI_THREADS + pidx) * 8, rsrc + m * S->ldres + (pidx & 15) * 8);
+              if (m < P.g.m) cp_async16(res_s + (ci * 4 * EPI_THREADS + pidx) * 8, rsrc + m * S->ldres + (pidx & 15) * 8);
             }
             cp_async_commit();
           }
@@ -403,26 +405,33 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
           (!res || ((reinterpret_cast<uintptr_t>(res) | (uintptr_t)(ldres * sizeof(OutT))) & 15u) == 0) &&
           (!accp || ((reinterpret_cast<uintptr_t>(accp) | (uintptr_t)(ldacc * 4)) & 15u) == 0);
       const bool res_pf = res_prefetch<YT>(S, nt);  // the residual is in shared memory
-      for (int c0 = 0; c0 < BN; c0 += EPI_CHUNK, ++chunk_ctr) {
-        int32_t* buf = epi_s + (chunk_ctr & 1u) * (EPI_CHUNK * BM);
-        uint32_t v[16];
-        tmem_ld_32x32b_x16(tmem_base + lane_addr + ACC_COL + b * BN + c0 + 16 * half, v);
-        tmem_wait_ld();
-        if (c0 + EPI_CHUNK >= BN) {
-          // the accumulator buffer is drained: hand it back to the MMA issuer
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&accempty[b]);
-        }
+      for (int c0 = 0; c0 < BN; c0 += EPI_CHUNK) {
+        int32_t* buf = epi_s;
+        if (c0 > 0) asm volatile("bar.sync 1, 256;" ::: "memory");  // the first round has read buf
 #pragma unroll
-        for (int j = 0; j < 16; ++j) buf[(16 * half + j) * BM + srow] = (int32_t)v[j];
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t v[16];
+          tmem_ld_32x32b_x16(tmem_base + lane_addr + ACC_COL + b * BN + c0 + 32 * half + 16 * hh, v);
+          tmem_wait_ld();
+          if (hh == 1 && c0 + EPI_CHUNK >= BN) {
+            // the accumulator buffer is drained: hand it back to the MMA issuer
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&accempty[b]);
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) buf[(32 * half + 16 * hh + j) * BM + srow] = (int32_t)v[j];
+        }
         asm volatile("bar.sync 1, 256;" ::: "memory");
         const int64_t m0 = (int64_t)mt * BN + c0;
         const int64_t rem = P.g.m - m0;
         const int jmax = rem < EPI_CHUNK ? (int)rem : EPI_CHUNK;
         if (vec_ok && glu) {
-          // 32 tokens x 8 pieces of 8 output columns = 256 pieces, one per thread
-          const int j = etid >> 3, r8 = (etid & 7) * 8;
+          // 64 tokens x 8 pieces of 8 output columns = 512 pieces, two per thread
+#pragma unroll
+          for (int itp = 0; itp < 2; ++itp) {
+          const int pidx = etid + itp * EPI_THREADS;
+          const int j = pidx >> 3, r8 = (pidx & 7) * 8;
           if (j < jmax) {
             const int32_t* bj = buf + j * BM;
             const int4 g0 = *reinterpret_cast<const int4*>(bj + epi_word(r8));
@@ -439,11 +448,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
             for (int e = 0; e < 8; ++e) z[e] = siluf_(gv[e]) * z[e];
             store8<YT>(y + (m0 + j) * ldy + r8, z);
           }
+          }
         } else if (vec_ok) {
-          // 32 tokens x 16 pieces of 8 rows = 512 pieces, 2 per thread; a warp writes two whole
-          // 128-row segments (256 B in bf16, 512 B in fp32)
+          // 64 tokens x 16 pieces of 8 rows = 1024 pieces, 4 per thread; a warp writes two whole
+          // 128-row segments at a time (256 B in bf16, 512 B in fp32)
 #pragma unroll
-          for (int itp = 0; itp < 2; ++itp) {
+          for (int itp = 0; itp < 4; ++itp) {
             const int pidx = etid + itp * EPI_THREADS;
             const int j = pidx >> 4, r8 = (pidx & 15) * 8;
             if (j < jmax) {
@@ -462,11 +472,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1) ternary_gemm_tc_kernel(const _
               if (res_pf) {
                 // this chunk's cp.async group (and the earlier ones) have landed
                 const int ci = c0 / EPI_CHUNK;
-                if (ci == 0) cp_async_wait<3>();
-                else if (ci == 1) cp_async_wait<2>();
-                else if (ci == 2) cp_async_wait<1>();
+                if (ci == 0) cp_async_wait<1>();
                 else cp_async_wait<0>();
-                add8<YT>(res_s + (ci * 2 * EPI_THREADS + pidx) * 8, z);
+                add8<YT>(res_s + (ci * 4 * EPI_THREADS + pidx) * 8, z);
               } else if (res) {
                 add8<YT>(res + m * ldres + r8, z);
               }
