@@ -597,20 +597,26 @@ def run_sweeps(device, flush, peaks) -> dict:
     reps = 8
 
     def median_ms(fn, classes=False):
+        # the call times carry no per-launch events; with `classes`, the same number of calls
+        # again with the library's launch events gives the product kernel's own time
         times, kern_total = [], None
         for r in range(reps + 2):
             flush.zero_()
             a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            if classes and r >= 2:
-                mmf.timing_enable(True)
             a.record(stream)
             fn()
             b.record(stream)
             torch.cuda.synchronize(device)
-            mmf.timing_enable(False)
             if r >= 2:
                 times.append(a.elapsed_time(b))
         if classes:
+            kernel_classes(mmf)  # clear
+            for _ in range(reps):
+                flush.zero_()
+                mmf.timing_enable(True)
+                fn()
+                torch.cuda.synchronize(device)
+                mmf.timing_enable(False)
             kern_total = kernel_classes(mmf)
         return statistics.median(times), kern_total
 

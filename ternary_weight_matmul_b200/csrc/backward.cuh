@@ -25,9 +25,10 @@
 // rq = q (a/127) and Wq = t s, and
 //   dr = dy Wq;  u = dr w;  rho = (mean(x^2) + eps)^(-1/2);  dx = rho u - rho^3 x mean(u x);
 //   dw[k] = sum_m dr[m][k] x[m][k] rho_m;  dW = dy^T rq  (the latent weight's gradient).
-// Five small CUDA-core kernels, in this order: rho per row; dr per (row, 16-column word of the
-// packed codes), written into dx's buffer; the gain's gradient per column; dx per row, in place
-// over dr; dW per (weight row, column).
+// dr and dW are products: on the tensor cores (bf16_gemm_kernel, with the operand layout kernels
+// below) or, on the CUDA-core engine, one thread per (row, 16-column word of the packed codes)
+// for dr and per (weight row, column) for dW. dr is written into dx's buffer; one row-block
+// kernel then forms rho, the gain's gradient partials and dx in place over dr.
 #pragma once
 
 #include <type_traits>
@@ -272,20 +273,6 @@ struct LinBwdArgs {
   float* rho;           // [m] scratch
 };
 
-// rho_m = (mean(x_m^2) + eps)^(-1/2), one warp per row.
-__global__ void __launch_bounds__(kThreads) lin_bwd_rho_kernel(const LinBwdArgs a) {
-  const int64_t row = (int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (row >= a.m) return;
-  float ss = 0.0f;
-  for (int c = lane; c < a.k; c += 32) {
-    const float v = load_as_float(a.x, row * a.k + c, a.xdt);
-    ss = fmaf(v, v, ss);
-  }
-  ss = warp_sum(ss);
-  if (lane == 0) a.rho[row] = rsqrtf(ss / (float)a.k + a.eps);
-}
-
 // dr[m][16 w + j] = s sum_n dy[m][n] t[n][16 w + j]: one thread per (row, packed word column w),
 // the 16 codes of word (n, w) expanded to int8 lanes (quad q = columns 4q..4q+3, lowest column in
 // byte 0).
@@ -311,52 +298,73 @@ __global__ void __launch_bounds__(kThreads) lin_bwd_dr_kernel(const LinBwdArgs a
     if (16 * w + j < a.k) a.dx[row * a.k + 16 * w + j] = acc[j] * s;
 }
 
-// dw[c] = sum_m dr[m][c] x[m][c] rho_m in two passes: blocks of 32 columns x 8 row lanes each add a
-// slice of rows_per rows into part[split][c] (blockIdx.y = split), then one thread per column
-// adds the splits in order (deterministic). Coalesced across columns throughout.
-__global__ void __launch_bounds__(256) lin_bwd_dnw_part_kernel(const LinBwdArgs a, float* part, int rows_per) {
+// rho, the gain's gradient and dx for a block of rows_per rows (blockIdx.x), in one kernel:
+// phase A, one warp per row: rho_r = (mean(x^2) + eps)^(-1/2) and mean(u x) with u = dr w (into
+// rho[] and mux[]); phase B, threads over columns walking the block's rows in order:
+// part[block][c] = sum_r dr x rho (before dx replaces dr), then dx = rho u - rho^3 x mean(u x) in
+// place over dr. The partials are added per column by lin_bwd_dnw_reduce_kernel.
+__global__ void __launch_bounds__(kThreads) lin_bwd_rows_kernel(const LinBwdArgs a, float* mux, float* part,
+                                                                int rows_per) {
+  const int64_t r0 = (int64_t)blockIdx.x * rows_per;
+  const int64_t r1 = r0 + rows_per < a.m ? r0 + rows_per : a.m;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int64_t r = r0 + warp; r < r1; r += kThreads / 32) {
+    float ss = 0.0f, ux = 0.0f;
+    for (int c = lane; c < a.k; c += 32) {
+      const float xv = load_as_float(a.x, r * a.k + c, a.xdt);
+      const float u = a.dx[r * a.k + c] * (a.norm_w ? a.norm_w[c] : 1.0f);
+      ss = fmaf(xv, xv, ss);
+      ux = fmaf(u, xv, ux);
+    }
+    ss = warp_sum(ss);
+    ux = warp_sum(ux);
+    if (lane == 0) {
+      a.rho[r] = rsqrtf(ss / (float)a.k + a.eps);
+      mux[r] = ux / (float)a.k;
+    }
+  }
+  __syncthreads();
+  for (int c = threadIdx.x; c < a.k; c += kThreads) {
+    const float w = a.norm_w ? a.norm_w[c] : 1.0f;
+    float acc = 0.0f;
+    for (int64_t rb = r0; rb < r1; rb += 4) {
+      // four rows' loads in flight before the (ordered) arithmetic
+      float d[4], xv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (rb + u < r1) {
+          d[u] = a.dx[(rb + u) * a.k + c];
+          xv[u] = load_as_float(a.x, (rb + u) * a.k + c, a.xdt);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (rb + u < r1) {
+          const int64_t r = rb + u;
+          const float rho = a.rho[r];
+          acc = fmaf(d[u] * xv[u], rho, acc);
+          a.dx[r * a.k + c] = rho * (d[u] * w) - rho * rho * rho * xv[u] * mux[r];
+        }
+      }
+    }
+    if (part) part[(int64_t)blockIdx.x * a.k + c] = acc;
+  }
+}
+// dw[c] = sum over blocks of part[block][c], in block order; 32 columns x 8 lanes per CTA, each
+// lane adding every 8th block, then the 8 lane sums in order.
+__global__ void __launch_bounds__(256) lin_bwd_dnw_reduce_kernel(const LinBwdArgs a, const float* part, int splits) {
   __shared__ float red[8][33];
   const int c = blockIdx.x * 32 + threadIdx.x;
-  const int64_t r0 = (int64_t)blockIdx.y * rows_per;
-  const int64_t r1 = r0 + rows_per < a.m ? r0 + rows_per : a.m;
-  float acc = 0.0f;
+  float t = 0.0f;
   if (c < a.k)
-    for (int64_t row = r0 + threadIdx.y; row < r1; row += 8)
-      acc = fmaf(a.dx[row * a.k + c] * load_as_float(a.x, row * a.k + c, a.xdt), a.rho[row], acc);
-  red[threadIdx.y][threadIdx.x] = acc;
+    for (int z = threadIdx.y; z < splits; z += 8) t += part[(int64_t)z * a.k + c];
+  red[threadIdx.y][threadIdx.x] = t;
   __syncthreads();
   if (threadIdx.y == 0 && c < a.k) {
-    float t = 0.0f;
+    float s = 0.0f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) t += red[j][threadIdx.x];
-    part[(int64_t)blockIdx.y * a.k + c] = t;
-  }
-}
-__global__ void __launch_bounds__(kThreads) lin_bwd_dnw_reduce_kernel(const LinBwdArgs a, const float* part,
-                                                                      int splits) {
-  const int c = blockIdx.x * kThreads + threadIdx.x;
-  if (c >= a.k) return;
-  float t = 0.0f;
-  for (int z = 0; z < splits; ++z) t += part[(int64_t)z * a.k + c];
-  a.dnorm_w[c] = t;
-}
-
-// dx = rho u - rho^3 x mean(u x) with u = dr w, one CTA per row, in place over dr.
-__global__ void __launch_bounds__(kThreads) lin_bwd_dx_kernel(const LinBwdArgs a) {
-  __shared__ float red[32];
-  const int64_t row = blockIdx.x;
-  float* d = a.dx + row * a.k;
-  float ux = 0.0f;
-  for (int c = threadIdx.x; c < a.k; c += kThreads) {
-    const float u = d[c] * (a.norm_w ? a.norm_w[c] : 1.0f);
-    ux = fmaf(u, load_as_float(a.x, row * a.k + c, a.xdt), ux);
-  }
-  const float mean_ux = block_sum(ux, red) / (float)a.k;
-  const float r = a.rho[row];
-  const float r3 = r * r * r;
-  for (int c = threadIdx.x; c < a.k; c += kThreads) {
-    const float u = d[c] * (a.norm_w ? a.norm_w[c] : 1.0f);
-    d[c] = r * u - r3 * load_as_float(a.x, row * a.k + c, a.xdt) * mean_ux;
+    for (int j = 0; j < 8; ++j) s += red[j][threadIdx.x];
+    a.dnorm_w[c] = s;
   }
 }
 

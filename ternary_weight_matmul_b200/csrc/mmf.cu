@@ -981,7 +981,7 @@ mmf_status head_tc_pass(const void* x, mmf_dtype xdt, int nb, int d, const float
 // turn on one stream).
 struct LinBwdPlan {
   int64_t ld_n, ld_m;
-  size_t rho, dr_hi, dr_lo, tt, dr_part, dw_hi, dw_lo, qt, dw_part, dnw_part, bytes;
+  size_t rho, mux, dr_hi, dr_lo, tt, dr_part, dw_hi, dw_lo, qt, dw_part, dnw_part, bytes;
   int dr_split, dr_kbc, dw_split, dw_kbc, dnw_split, dnw_rows;
 };
 // Splits of K so that an M x N product with few tiles still covers the SMs: floor(148 / tiles),
@@ -1000,7 +1000,8 @@ inline LinBwdPlan lin_bwd_plan(int64_t m, int32_t k, int32_t n) {
   P.ld_n = ((int64_t)n + 7) / 8 * 8;
   P.ld_m = (m + 7) / 8 * 8;
   P.rho = 0;
-  const size_t base = align256((size_t)m * 4);
+  P.mux = align256((size_t)m * 4);
+  const size_t base = 2 * align256((size_t)m * 4);
   size_t o = base;
   P.dr_hi = o; o += align256((size_t)m * P.ld_n * 2);
   P.dr_lo = o; o += align256((size_t)m * P.ld_n * 2);
@@ -1016,9 +1017,10 @@ inline LinBwdPlan lin_bwd_plan(int64_t m, int32_t k, int32_t n) {
   gb_split(n, k, m, P.dw_split, P.dw_kbc);
   P.dw_part = o;
   if (P.dw_split > 1) o += align256((size_t)P.dw_split * n * k * 4);
-  // the gain's gradient: row slices of at least 128 rows, at most 64 slices (between the two
-  // products, so it reuses the same space)
-  P.dnw_split = (int)std::max<int64_t>(std::min<int64_t>((m + 127) / 128, 64), 1);
+  // rho, the gain's gradient and dx: row blocks of at least 16 rows, at most 2048 blocks, each
+  // leaving one partial row of the gain's gradient (between the two products, so it reuses the
+  // same space)
+  P.dnw_split = (int)std::max<int64_t>(std::min<int64_t>((m + 15) / 16, 2048), 1);
   P.dnw_rows = (int)std::max<int64_t>((m + P.dnw_split - 1) / P.dnw_split, 1);
   P.dnw_part = base;
   const size_t end_dnw = base + align256((size_t)P.dnw_split * k * 4);
@@ -1813,9 +1815,6 @@ mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, c
                  (double)w->n * row_words(w->k) * 4.0, st);
   int launches = 0;
   if (m > 0) {
-    launch_k(bwd::lin_bwd_rho_kernel, dim3((unsigned)((m + bwd::kThreads / 32 - 1) / (bwd::kThreads / 32))),
-             dim3(bwd::kThreads), 0, st, a);
-    ++launches;
     if (tc) {
       // dr [m][k] = s * dy [m][n] . t [n][k]: A = dy (bf16 as given, else hi / lo rows),
       // B = t transposed to [k][n]
@@ -1843,19 +1842,21 @@ mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, c
       ++launches;
     }
   }
-  if (dnorm_w) {
-    if (m > 0) {
-      float* part = reinterpret_cast<float*>(wsb + plan.dnw_part);
-      launch_k(bwd::lin_bwd_dnw_part_kernel, dim3((unsigned)((w->k + 31) / 32), (unsigned)plan.dnw_split), dim3(32, 8), 0,
-               st, a, part, plan.dnw_rows);
-      launch_k(bwd::lin_bwd_dnw_reduce_kernel, dim3(kcols), dim3(bwd::kThreads), 0, st, a, part, plan.dnw_split);
-      launches += 2;
-    } else {
-      cudaError_t e = cudaMemsetAsync(dnorm_w, 0, (size_t)w->k * sizeof(float), st);
-      if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
+  if (m > 0) {
+    // rho, the gain's gradient partials and dx (in place over dr), one row block per CTA
+    float* part = dnorm_w ? reinterpret_cast<float*>(wsb + plan.dnw_part) : nullptr;
+    launch_k(bwd::lin_bwd_rows_kernel, dim3((unsigned)plan.dnw_split), dim3(bwd::kThreads), 0, st, a,
+             reinterpret_cast<float*>(wsb + plan.mux), part, plan.dnw_rows);
+    ++launches;
+    if (dnorm_w) {
+      launch_k(bwd::lin_bwd_dnw_reduce_kernel, dim3((unsigned)((w->k + 31) / 32)), dim3(32, 8), 0, st, a, part,
+               plan.dnw_split);
+      ++launches;
     }
+  } else if (dnorm_w) {
+    cudaError_t e = cudaMemsetAsync(dnorm_w, 0, (size_t)w->k * sizeof(float), st);
+    if (e != cudaSuccess) return fail(MMF_ERR_CUDA, "cudaMemsetAsync: %s", cudaGetErrorString(e));
   }
-  if (m > 0) { launch_k(bwd::lin_bwd_dx_kernel, dim3((unsigned)m), dim3(bwd::kThreads), 0, st, a); ++launches; }
   if (dW && tc && m > 0) {
     // dW [n][k] = (dy (a/127))^T [n][m] . q [m][k]: A = dy scaled and transposed (hi / lo),
     // B = q transposed to [k][m]

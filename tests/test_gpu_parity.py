@@ -440,6 +440,38 @@ def test_gemm_wait_cap_ends_and_recovers(mmf):
     assert np.array_equal(acc.cpu().numpy().astype(np.int64), O.int_matmul(q.cpu().numpy(), t))
 
 
+def test_backward_products_wait_cap_ends_and_recovers(mmf):
+    # the BitLinear backward's bf16 tensor-core products under a 1 us cap on every in-kernel wait:
+    # the launches must end (each CTA drains its TMA copies and MMAs, releases its tensor memory and
+    # leaves), report MMF_ERR_TIMEOUT (or, if no wait ran out, be right), and the next call at the
+    # default cap must be right
+    m, n, k = 512, 512, 1024
+    x = _to(synth.activations(140, (m, k)))
+    Wl = synth.weight(141, n, k)
+    w = mmf.pack_ternary(_to(Wl))
+    dy = _to(synth.activations(142, (m, n)))
+    _, q, deq, _ = mmf.bitlinear_fwd(x, None, w, y_dtype=torch.float32, debug=True)
+    _ok(mmf)
+    dW_ref = _np(dy).astype(np.float64).T @ (q.cpu().numpy().astype(np.float64) * deq.cpu().numpy()[:, None])
+    scale = np.abs(dW_ref).max()
+    mmf.set_gemm_path(mmf.MMF_GEMM_TENSOR)
+    try:
+        mmf.set_wait_limit(1)
+        try:
+            dx, dnw, dW = mmf.bitlinear_backward(x, None, w, q, deq, dy)
+            status = mmf.sync_status(DEV)
+        finally:
+            mmf.set_wait_limit(0)
+        assert status in (mmf.MMF_OK, mmf.MMF_ERR_TIMEOUT)
+        if status == mmf.MMF_OK:
+            np.testing.assert_allclose(dW.cpu().numpy(), dW_ref, rtol=1e-4, atol=1e-4 * scale)
+        dx, dnw, dW = mmf.bitlinear_backward(x, None, w, q, deq, dy)
+        _ok(mmf)
+    finally:
+        mmf.set_gemm_path(mmf.MMF_GEMM_AUTO)
+    np.testing.assert_allclose(dW.cpu().numpy(), dW_ref, rtol=1e-4, atol=1e-4 * scale)
+
+
 def test_head_wait_cap_ends_and_recovers(mmf):
     # the tensor-core head under a 1 us cap: ends, reports MMF_ERR_TIMEOUT or is right, and the
     # next call at the default cap is right
