@@ -11,7 +11,7 @@
 //          v = SiLU(gate) * up (epilogue);
 //   kDown  down_proj's RMSNorm + quantisation of v, down_proj and y = x1 + down (epilogue).
 // Each CTA owns a contiguous range of output channels. Its first thread starts bulk copies of
-// the input rows and their norm gains, and of the CTA's packed weight rows, into shared memory
+// the input rows and their norm gains, then of the CTA's packed weight rows, into shared memory
 // (two barriers);
 // while the weights stream in, the CTA quantises the input rows itself -- every CTA computes the
 // same codes, in the arithmetic of norm_quant_vec_kernel -- and each warp then forms whole
@@ -160,8 +160,9 @@ __device__ __forceinline__ void dec_issue_weights(const Args& a, uint32_t* wsm, 
                 (uint32_t)nc * row_bytes, bar_w);
 }
 
-// One projection group on one CTA (its weight rows already requested on B.bar_w): input rows and
-// gains into shared memory, the codes of every input row, the products and the fused epilogue.
+// One projection group on one CTA: input rows and gains into shared memory, then the weight rows
+// (all requested by thread 0 at the start), the codes of every input row, the products and the
+// fused epilogue.
 // Returns false when a bounded wait gave up (the copies in flight are drained first).
 template <mmf_dtype XT, int NB>
 __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta) {
@@ -200,6 +201,9 @@ __device__ __forceinline__ bool dec_phase(const Args& a, const Bufs& B, int cta)
     for (int j = 0; j < ng; ++j)
       if (a.gain[j]) bulk_load(gains + (size_t)j * a.k, a.gain[j], gbytes, B.bar_in);
     if (has_gw) bulk_load(gains + (size_t)ng * a.k, a.gnorm_w, gbytes, B.bar_in);
+    // the weight rows after the inputs: the prologue waits only for the inputs, and copies
+    // requested first arrive first (requesting the weights first cost 5-7% of a decode step)
+    dec_issue_weights(a, B.wsm, B.bar_w, cta);
   }
   for (int j = 0; j < ng + (a.mode == kO ? 1 : 0); ++j) {
     const bool absent = j < ng ? a.gain[j] == nullptr : !has_gw;
@@ -485,7 +489,6 @@ __global__ void __launch_bounds__(kThreads) dec_proj_kernel(const __grid_constan
     mbar_init(&bar[0], 1);
     mbar_init(&bar[1], 1);
     mbar_fence_init();
-    dec_issue_weights(a, B.wsm, B.bar_w, blockIdx.x);
   }
   __syncthreads();
   dec_phase<XT, NB>(a, B, blockIdx.x);
