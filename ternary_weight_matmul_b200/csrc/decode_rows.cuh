@@ -15,6 +15,8 @@
 // One CTA of 512 threads per token row; a thread owns NI quads of four consecutive columns
 // (quad tid + 512 i) and keeps their values in registers, with every global load of the row
 // issued before the first use (the stage is bound by the latency of its loads, not their bytes).
+// The norm gains (constant weights) of the thread's quads are copied into shared memory before the
+// wait for the preceding product, so no gain load sits between the reductions.
 // The quantisation is norm_quant's: r = (v * (1/rms)) * gain in float32, a = max|r|,
 // code = rint(r * (127/a)), factor a/127. Requires the vector lengths to be multiples of 4 and
 // at most 4 * 512 * NI = 8192.
@@ -76,20 +78,39 @@ __device__ __forceinline__ void st4(void* base, int64_t idx, mmf_dtype dt, const
         make_uint2(*reinterpret_cast<const uint32_t*>(&a), *reinterpret_cast<const uint32_t*>(&b));
   }
 }
-__device__ __forceinline__ float4 gain4(const float* g, int c) {
-  return g ? *reinterpret_cast<const float4*>(g + c) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+// Shared-memory gain slots: slot j < ngain holds gain[j], slot ngain the g_norm gain (kIFG), each
+// k floats (only the slots of present gains are filled; absent ones read as ones).
+__host__ __device__ inline size_t row_stage_smem(int mode, int d, int inner, int ngain) {
+  const int k = mode == kGate ? inner : d;
+  return (size_t)(ngain + (mode == kIFG ? 1 : 0)) * (size_t)k * sizeof(float);
 }
 
 __global__ void __launch_bounds__(kThreads) row_stage_kernel(const Args a) {
   __shared__ float red[32];
-  // programmatic dependent launch: wait for the preceding product, then let the next product
-  // start streaming its weights while this stage runs
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  extern __shared__ __align__(16) float gsm[];     // gain slots (row_stage_smem)
   const int64_t r = blockIdx.x;
   const int tid = threadIdx.x;
   const int k = a.mode == kGate ? a.inner : a.d;  // length of the vector to quantise
   const int nq = k >> 2;                           // quads
+  // this thread's quads of every present gain (constant weights: copied before the wait)
+  for (int j = 0; j <= a.ngain; ++j) {
+    const float* src = j < a.ngain ? a.gain[j] : (a.mode == kIFG ? a.gnorm_w : nullptr);
+    if (src == nullptr) continue;
+#pragma unroll
+    for (int i = 0; i < kNI; ++i) {
+      const int qd = tid + i * kThreads;
+      if (qd < nq) cp_async16(gsm + (size_t)j * k + 4 * qd, src + 4 * qd);
+    }
+  }
+  cp_async_commit();
+  // programmatic dependent launch: wait for the preceding product, then let the next product
+  // start streaming its weights while this stage runs
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // a gain quad of this thread: from its own copy in shared memory (ones when absent)
+  auto sg4 = [&](int j, const float* present, int c) {
+    return present ? *reinterpret_cast<const float4*>(gsm + (size_t)j * k + c) : make_float4(1.0f, 1.0f, 1.0f, 1.0f);
+  };
   const int32_t* acc = a.acc ? a.acc + r * a.ldacc : nullptr;
   float v[kNI][4];
   float ss = 0.0f;
@@ -141,13 +162,14 @@ __global__ void __launch_bounds__(kThreads) row_stage_kernel(const Args a) {
         }
       }
     }
+    cp_async_wait<0>();  // this thread's gain copies have landed
     const float rh = nq_rinv(block_sum(sh, red), d, a.eps);
     // g_norm: u = (h * (1/rms(h))) * gnorm_w * SiLU(g)
 #pragma unroll
     for (int i = 0; i < kNI; ++i) {
       const int qd = tid + i * kThreads;
       if (qd < nq) {
-        const float4 w4 = gain4(a.gnorm_w, 4 * qd);
+        const float4 w4 = sg4(a.ngain, a.gnorm_w, 4 * qd);
         const float w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -198,6 +220,7 @@ __global__ void __launch_bounds__(kThreads) row_stage_kernel(const Args a) {
     }
   }
   if (a.ngain == 0) return;
+  cp_async_wait<0>();  // this thread's gain copies have landed
   const float rf = nq_rinv(block_sum(ss, red), k, a.eps);
   for (int j = 0; j < a.ngain; ++j) {
     const float* gn = a.gain[j];
@@ -206,7 +229,7 @@ __global__ void __launch_bounds__(kThreads) row_stage_kernel(const Args a) {
     for (int i = 0; i < kNI; ++i) {
       const int qd = tid + i * kThreads;
       if (qd < nq) {
-        const float4 w4 = gain4(gn, 4 * qd);
+        const float4 w4 = sg4(j, gn, 4 * qd);
         const float w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) am = fmaxf(am, fabsf(__fmul_rn(__fmul_rn(v[i][e], rf), w[e])));
@@ -219,7 +242,7 @@ __global__ void __launch_bounds__(kThreads) row_stage_kernel(const Args a) {
     for (int i = 0; i < kNI; ++i) {
       const int qd = tid + i * kThreads;
       if (qd < nq) {
-        const float4 w4 = gain4(gn, 4 * qd);
+        const float4 w4 = sg4(j, gn, 4 * qd);
         const float w[4] = {w4.x, w4.y, w4.z, w4.w};
         uint32_t qb[4];
 #pragma unroll

@@ -193,6 +193,8 @@ mmf_status device_info(DevInfo** out) {
       MMF_CUDA((head_attrs<MMF_BF16, MMF_BF16>()));
       MMF_CUDA(head_tc_attrs());
       MMF_CUDA(cudaFuncSetAttribute(gb::bf16_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gb::SMEM_BYTES));
+      MMF_CUDA(cudaFuncSetAttribute(drow::row_stage_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)(3 * drow::kMaxK * sizeof(float))));
       MMF_CUDA(cudaFuncSetAttribute(sk::ternary_gemm_skinny_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                     sk::Layout<16>::SMEM));
       MMF_CUDA(cudaFuncSetAttribute(sk::ternary_gemm_skinny_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -863,6 +865,7 @@ mmf_status launch_row_stage(const drow::Args& a, int64_t b, cudaStream_t st) {
   memset(&cfg, 0, sizeof(cfg));
   cfg.gridDim = dim3((unsigned)b);
   cfg.blockDim = dim3(drow::kThreads);
+  cfg.dynamicSmemBytes = drow::row_stage_smem(a.mode, a.d, a.inner, a.ngain);
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
