@@ -84,3 +84,26 @@ def test_gemm_traffic_tracks_kernel_source(monkeypatch):
     monkeypatch.setitem(bench.GEMM_TRAFFIC, "prefill-370M", dict(entry, sha256="0" * 16))
     assert bench.gemm_traffic("prefill-370M") is None
     assert bench.gemm_traffic("prefill-1.3B") is None
+
+
+def test_roofline_and_hbm_shares_from_kernel_classes():
+    """The roofline of the dominant GEMM and the HBM-kernel figures come from the library's
+    per-class launch records: achieved = algorithmic work / device time of the class, frac =
+    achieved / peak, share = class time / step time of the attribution pass."""
+    import bench
+
+    kern = {"gemm_tc": {"launches": 96, "ms": 8.0, "work": 16.0e12},
+            "gemm_simt": {"launches": 0, "ms": 0.0, "work": 0.0},
+            "norm_quant": {"launches": 96, "ms": 2.5, "work": 8.0e9},
+            "scan": {"launches": 24, "ms": 1.0, "work": 2.0e9},
+            "other": {"launches": 1, "ms": 0.01, "work": 3.0e7}}
+    r = bench.gemm_roofline(kern, 12.0, 3318.0, "test peak", None)
+    assert r["achieved"] == pytest.approx(16.0e12 / 8.0e-3 / 1e12)   # 2000 TOPS
+    assert r["frac"] == pytest.approx(2000.0 / 3318.0)
+    assert r["avg_launch_us"] == pytest.approx(8.0 / 96 * 1e3)
+    assert r["share_of_step"] == pytest.approx(8.0 / 12.0)
+    h = bench.hbm_breakdown(kern, 12.0, 6525.0)
+    assert set(h) == {"norm_quant", "scan", "other"}          # classes with no launch are left out
+    assert h["norm_quant"]["GB/s"] == pytest.approx(8.0e9 / 2.5e-3 / 1e9)
+    assert h["scan"]["frac_hbm"] == pytest.approx(2.0e9 / 1.0e-3 / 1e9 / 6525.0)
+    assert h["scan"]["share_of_step"] == pytest.approx(1.0 / 12.0)
