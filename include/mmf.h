@@ -326,8 +326,8 @@ mmf_status mmf_hgrn_scan_backward(const void* zf, const void* zi, const void* h,
  *         the caller).   i [b][t][heads][dv] dtype.   o [b][t][heads][dv] dtype out.
  *   s0    [b][heads][dk][dv] float32 or NULL (zeros).   s_out same shape float32 out, or NULL.
  *   1 <= dk <= 128; b, heads <= 65535. t = 0 writes only s_out.
- * CUDA cores, float32 state and accumulation: one thread per (sequence, head, value column),
- * steps in order. No workspace. */
+ * CUDA cores, float32 state and accumulation: four threads per (sequence, head, value column),
+ * each holding a quarter of the column's state rows, steps in order. No workspace. */
 mmf_status mmf_hgrn2_recurrence(const void* q, const void* f, const void* i, mmf_dtype dtype, int32_t b, int64_t t,
                                 int32_t heads, int32_t dk, int32_t dv, const float* s0, float* s_out, void* o,
                                 mmf_stream_t stream);
