@@ -59,7 +59,7 @@ typedef struct CUstream_st* mmf_stream_t; /* a cudaStream_t */
 typedef enum {
   MMF_OK = 0,
   MMF_ERR_INVALID_ARG = 1, /* null / misaligned pointer, bad size or dtype */
-  MMF_ERR_UNSUPPORTED = 2, /* valid request this build cannot serve (e.g. no sm_100a device) */
+  MMF_ERR_UNSUPPORTED = 2, /* valid request the library cannot serve (e.g. no sm_100a device) */
   MMF_ERR_WORKSPACE = 3,   /* ws smaller than mmf_workspace_bytes() or misaligned */
   MMF_ERR_CUDA = 4,        /* a CUDA runtime call or launch failed */
   MMF_ERR_TIMEOUT = 5      /* a bounded in-kernel wait ran out (reported by mmf_sync_status) */
