@@ -308,7 +308,8 @@ mmf_status mmf_bitlinear_backward(const void* x, mmf_dtype x_dtype, int64_t m, c
  *   h0 [b][d] float32 or NULL.   dzf, dzi [b][t][d] dtype out.   dh0 [b][d] float32 out or NULL.
  *   ws >= mmf_workspace_bytes(MMF_OP_SCAN, b*t, d, 0, 0) when t > 32 (unused otherwise), 256-byte
  *   aligned, caller-owned, not retained; a smaller or misaligned ws is MMF_ERR_WORKSPACE.
- *   t = 0 writes dh0 = 0. b * ceil(t / chunk) * ceil(d / 256) CTAs must fit one grid (< 2^31).
+ *   t = 0 writes dh0 = 0. Chunks of 32 steps up to t = 4096, else at most 128 chunks; b x chunks x
+ *   ceil(d / 256) CTAs (ceil(d / 128) for odd d or rows not 2-element aligned) must be < 2^31.
  * CUDA cores, float32 arithmetic, chunked like the forward scan with time reversed: G is affine
  * in the carry from the later steps, so chunks fold to (A, B), a reverse walk over the chunks
  * gives each its carry, and each chunk is replayed from it. The chunk sums associate differently
