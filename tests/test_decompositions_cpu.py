@@ -8,6 +8,10 @@ each restates a kernel's decomposition in numpy and compares it with the oracle'
 * The bf16 hi / lo pair of the tensor-core products: hi = bf16(a), lo = bf16(a - hi) carries a
   float32 value to within 2^-17 of its magnitude, and a product with an operand bf16 holds exactly
   (ternary or int8 codes) is then the float32 product up to that bound.
+* The chunked form a tensor-core HGRN2 kernel would evaluate (not built: the recurrence kernel is
+  the path): the factored chunk form overflows float32 for small gates, while sub-chunks of 16
+  steps with every decay taken relative to the sub-chunk (exponents <= 0) reproduce the oracle's
+  recurrence in float32 for gates down to 1e-6.
 """
 import numpy as np
 import pytest
@@ -96,3 +100,68 @@ def test_hi_lo_products_with_exact_codes_stay_float32_accurate():
     approx_w = hi.T @ q + lo.T @ q
     bound_w = 2.0 ** -17 * (np.abs(dy.astype(np.float64)).T @ np.abs(q))
     assert np.all(np.abs(approx_w - exact_w) <= bound_w + 1e-300)
+
+
+# ---------------------------------------------------------------------------------------------
+# HGRN2: the chunked form for a tensor-core kernel (plan; the recurrence kernel is the built path)
+# ---------------------------------------------------------------------------------------------
+def _hgrn2_inputs(seed, b, t, h, dk, dv, fmin):
+    g = np.random.default_rng(seed)
+    q = g.standard_normal((b, t, h, dk))
+    f = np.exp(g.uniform(np.log(fmin), 0.0, (b, t, h, dk)))   # forget gates down to fmin
+    i = g.standard_normal((b, t, h, dv))
+    s0 = g.standard_normal((b, h, dk, dv))
+    return q, f, i, s0
+
+
+def test_hgrn2_factored_chunk_form_overflows_float32_for_small_gates():
+    # the factored chunk form needs 1 / prod(f) over the chunk: with gates near 1e-3 it leaves
+    # float32 within 16 steps, so a kernel cannot use it as it stands
+    f = np.full(16, 1e-3, dtype=np.float32)
+    with np.errstate(over="ignore", divide="ignore"):
+        inv = np.float32(1.0) / np.cumprod(f)
+    assert not np.all(np.isfinite(inv))
+
+
+def _hgrn2_subchunk(q, f, i, s0, L, dt):
+    """The two-level form in precision dt: sub-chunks of L steps in order, the state passed
+    between them; inside a sub-chunk every decay is exp(G_t - G_s) <= 1 with G the running sum of
+    log f from the sub-chunk's start, so nothing overflows whatever the gates. Per (sequence,
+    head), with the state's dv columns as the rows of the products (O^T = S^T Q~^T and
+    S^T <- S^T diag(e^G_last) + I^T K~: 128-row operands when dv = 128):
+      o_t   = (q_t * e^{G_t}) S_b + sum_{s<=t} [sum_k q_t[k] (1 - f_s[k]) e^{G_t[k] - G_s[k]}] i_s
+      S_e   = diag(e^{G_last}) S_b + sum_s ((1 - f_s) * e^{G_last - G_s})^T i_s"""
+    q, f, i = q.astype(dt), f.astype(dt), i.astype(dt)
+    b, t, h, dk = f.shape
+    dv = i.shape[-1]
+    S = s0.astype(dt).copy()
+    o = np.zeros((b, t, h, dv), dtype=dt)
+    for b0 in range(0, t, L):
+        e0 = min(b0 + L, t)
+        lf = np.log(f[:, b0:e0])                          # [B, l, H, dk], <= 0
+        G = np.cumsum(lf, axis=1)                         # inclusive running log-decay
+        key = (dt(1) - f[:, b0:e0])
+        qc, ic = q[:, b0:e0], i[:, b0:e0]
+        inter = np.einsum("bthk,bhkv->bthv", qc * np.exp(G), S)
+        diff = G[:, :, None] - G[:, None, :]              # [B, t, s, H, dk] = G_t - G_s
+        mask = np.tril(np.ones((e0 - b0, e0 - b0), dtype=bool))[None, :, :, None, None]
+        dec = np.where(mask, np.exp(np.where(mask, diff, dt(0))), dt(0))
+        P = np.einsum("bthk,bshk,btshk->bhts", qc, key, dec)
+        o[:, b0:e0] = inter + np.einsum("bhts,bshv->bthv", P, ic)
+        Gl = G[:, -1]                                     # [B, H, dk]
+        S = np.exp(Gl)[..., :, None] * S + np.einsum("bshk,bshv->bhkv", key * np.exp(Gl[:, None] - G), ic)
+    return o, S
+
+
+@pytest.mark.parametrize("fmin", [0.5, 1e-3, 1e-6])
+def test_hgrn2_subchunk_form_matches_the_recurrence(fmin):
+    q, f, i, s0 = _hgrn2_inputs(170, 2, 70, 2, 16, 8, fmin)
+    o_ref, S_ref = O.hgrn2_recurrence(q, f, i, s0)
+    o64, S64 = _hgrn2_subchunk(q, f, i, s0, 16, np.float64)
+    np.testing.assert_allclose(o64, o_ref, rtol=1e-10, atol=1e-10 * np.abs(o_ref).max())
+    np.testing.assert_allclose(S64, S_ref, rtol=1e-10, atol=1e-10 * np.abs(S_ref).max())
+    # in float32 every intermediate stays finite and the result is float32-accurate
+    with np.errstate(over="raise", invalid="raise"):
+        o32, S32 = _hgrn2_subchunk(q, f, i, s0, 16, np.float32)
+    np.testing.assert_allclose(o32, o_ref, rtol=1e-4, atol=1e-5 * np.abs(o_ref).max())
+    np.testing.assert_allclose(S32, S_ref, rtol=1e-4, atol=1e-5 * np.abs(S_ref).max())
