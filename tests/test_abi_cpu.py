@@ -208,3 +208,40 @@ def test_decode_taps_arguments_on_host(L):
     bw = mmf.BlockWeightsC()
     assert L.mmf_decode_step_taps(ctypes.byref(bw), 1, None, 0, 1, None, None, None, None, 0, None) == \
         mmf.MMF_ERR_INVALID_ARG
+
+
+def test_header_is_plain_c_and_links_from_c(tmp_path):
+    # the boundary is a C ABI: the header compiles as C99, and a C program linked against the
+    # library calls its host-only entry points (sizes, status strings) with no C++ or torch
+    import shutil
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include <string.h>
+#include "mmf.h"
+int main(void) {
+  if (mmf_packed_row_words(65) != 8) return 1;
+  if (mmf_packed_words(3, 65) != 24) return 2;
+  if (mmf_workspace_bytes(MMF_OP_SCAN, 8 * 2048, 1024, 0, 0) < (size_t)3 * 1024 * 4 * 8 * 128) return 3;
+  if (mmf_workspace_bytes(MMF_OP_BITLINEAR_BWD, 1000, 64, 8, 0) == 0) return 4;
+  if (strlen(mmf_status_string(MMF_ERR_WORKSPACE)) == 0) return 5;
+  /* argument validation happens on the host before any device work */
+  if (mmf_hgrn_scan_backward(NULL, NULL, NULL, NULL, MMF_F32, -1, 4, 8, NULL, NULL, NULL, NULL, NULL, 0, NULL)
+      != MMF_ERR_INVALID_ARG) return 6;
+  printf("ok\n");
+  return 0;
+}
+''')
+    exe = tmp_path / "abi"
+    lib_dir = os.path.dirname(mbuild.OUT)
+    res = subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(root, "include"),
+                          str(src), "-L", lib_dir, "-lmmf", "-Wl,-rpath," + lib_dir, "-o", str(exe)],
+                         capture_output=True, text=True)
+    assert res.returncode == 0, res.stderr
+    run = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
