@@ -245,3 +245,64 @@ int main(void) {
     assert res.returncode == 0, res.stderr
     run = subprocess.run([str(exe)], capture_output=True, text=True)
     assert run.returncode == 0 and run.stdout.strip() == "ok", (run.returncode, run.stdout, run.stderr)
+
+
+def test_decode_path_choice_on_host(L):
+    # the automatic choice (fused CUDA-core launches for 1 or 2 rows, skinny tensor-core products
+    # for 3 to 64 rows, the block path beyond), the engine setting's precedence and the forced
+    # paths that fall back to the block path where their kernel cannot serve the shape
+    F, S, B = mmf.MMF_DECODE_FUSED, mmf.MMF_DECODE_SKINNY, mmf.MMF_DECODE_BLOCK
+    pf = L.mmf_decode_path_for
+    try:
+        assert L.mmf_set_decode_path(7) == mmf.MMF_ERR_INVALID_ARG
+        assert L.mmf_set_decode_path(mmf.MMF_DECODE_AUTO) == mmf.MMF_OK
+        assert pf(0, 2560, 7040) == -1 and pf(1, 0, 7040) == -1 and pf(1, 2560, -1) == -1
+        assert [pf(b, 2560, 7040) for b in (1, 2, 3, 4, 8, 17, 64, 65, 256)] == [F, F, S, S, S, S, S, B, B]
+        assert pf(1, 2564, 7040) == B                               # d % 8 != 0: neither fused nor skinny
+        assert pf(8, 8200, 7040) == B                               # a row stage holds K <= 8192
+        assert L.mmf_set_gemm_path(mmf.MMF_GEMM_SIMT) == mmf.MMF_OK
+        assert [pf(b, 2560, 7040) for b in (1, 2, 3, 4, 8, 16)] == [F, F, B, F, F, B]
+        assert L.mmf_set_gemm_path(mmf.MMF_GEMM_TENSOR) == mmf.MMF_OK
+        assert [pf(b, 2560, 7040) for b in (1, 8, 64)] == [B, B, B]
+        assert L.mmf_set_gemm_path(mmf.MMF_GEMM_AUTO) == mmf.MMF_OK
+        assert L.mmf_set_decode_path(mmf.MMF_DECODE_FUSED) == mmf.MMF_OK
+        assert [pf(b, 2560, 7040) for b in (1, 2, 3, 4, 8, 9)] == [F, F, B, F, F, B]
+        assert L.mmf_set_decode_path(mmf.MMF_DECODE_SKINNY) == mmf.MMF_OK
+        assert [pf(b, 2560, 7040) for b in (1, 64, 65)] == [S, S, B]
+        assert L.mmf_set_decode_path(mmf.MMF_DECODE_BLOCK) == mmf.MMF_OK
+        assert [pf(b, 2560, 7040) for b in (1, 8, 64)] == [B, B, B]
+    finally:
+        L.mmf_set_decode_path(mmf.MMF_DECODE_AUTO)
+        L.mmf_set_gemm_path(mmf.MMF_GEMM_AUTO)
+
+
+def test_noalloc_and_taps_arguments_on_host(L):
+    # the allocation-free BitLinear refuses, before any CUDA call, a request whose scratch exceeds
+    # its static array; the block taps refuse a null taps struct
+    w = mmf.Ternary(4096, 32, 2048, 2048)
+    # the codes (m x K bytes) plus per-row factors and padding: 4088 rows fit at K = 2048, 4096 not
+    assert L.mmf_workspace_bytes(mmf.MMF_OP_BITLINEAR, 4088, 2048, 2048, 0) <= 8 << 20
+    assert L.mmf_workspace_bytes(mmf.MMF_OP_BITLINEAR, 4096, 2048, 2048, 0) > 8 << 20
+    m_big = 4096
+    assert L.mmf_bitlinear_fwd_noalloc(16, 0, m_big, None, ctypes.byref(w), 16, 0, None) == mmf.MMF_ERR_WORKSPACE
+    assert b"static array" in L.mmf_last_error()
+    assert L.mmf_bitlinear_fwd_noalloc(16, 0, -1, None, ctypes.byref(w), 16, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_bitlinear_fwd_noalloc(16, 0, 4, None, None, 16, 0, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_bitlinear_fwd_noalloc(16, 0, 0, None, ctypes.byref(w), 16, 0, None) == mmf.MMF_OK  # nothing to do
+    bw = mmf.BlockWeightsC()
+    assert L.mmf_block_fwd_taps(ctypes.byref(bw), None, 0, 1, 1, None, None, None, None, None, 0,
+                                None) == mmf.MMF_ERR_INVALID_ARG
+    assert b"taps" in L.mmf_last_error()
+
+
+def test_instrumentation_on_host(L):
+    # the launch counter and the per-class timing records need no device while nothing launches
+    n0 = L.mmf_launch_count()
+    assert L.mmf_timing_enable(1) == mmf.MMF_OK
+    assert L.mmf_timing_enable(0) == mmf.MMF_OK
+    launches, ms, work = ctypes.c_int64(-1), ctypes.c_double(-1.0), ctypes.c_double(-1.0)
+    assert L.mmf_timing_read(0, ctypes.byref(launches), ctypes.byref(ms), ctypes.byref(work)) == mmf.MMF_OK
+    assert (launches.value, ms.value, work.value) == (0, 0.0, 0.0)
+    assert L.mmf_timing_read(-1, None, None, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_timing_read(99, None, None, None) == mmf.MMF_ERR_INVALID_ARG
+    assert L.mmf_launch_count() == n0
