@@ -126,8 +126,9 @@ mmf_status mmf_pack_ternary(const void* w, mmf_dtype w_dtype, int32_t n, int32_t
  *   a = max(max|r|, 1e-5);  q = clamp(rint(r * (127/a)), -127, 127)   (int8, float32 decision)
  *   acc[m][n] = sum_k q[m][k] * t[n][k]                 (exact int32)
  *   y[m][n] = acc * (a/127) * s
- *   x       [m][w->k] x_dtype.    norm_w [w->k] float32, or NULL for a unit gain.
- *   y       [m][w->n] y_dtype.
+ *   x       [m][w->k] x_dtype, 16-byte aligned.    norm_w [w->k] float32, or NULL for a unit gain.
+ *   y       [m][w->n] y_dtype, 16-byte aligned.
+ *   w       1 <= w->k <= 32768, w->n >= 1; codes 16-byte aligned, codes and scale non-NULL.
  *   q_dbg   optional [m][w->k] int8: the activation codes.
  *   deq_dbg optional [m] float32: a/127 per row.
  *   acc_dbg optional [m][w->n] int32: the integer accumulators.

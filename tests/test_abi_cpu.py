@@ -306,3 +306,25 @@ def test_instrumentation_on_host(L):
     assert L.mmf_timing_read(-1, None, None, None) == mmf.MMF_ERR_INVALID_ARG
     assert L.mmf_timing_read(99, None, None, None) == mmf.MMF_ERR_INVALID_ARG
     assert L.mmf_launch_count() == n0
+
+
+def test_bitlinear_limits_on_host(L):
+    # the documented limits of mmf_bitlinear_fwd: K in [1, 32768], codes 16-byte aligned, codes and
+    # scale present, x and y 16-byte aligned; each refused before any CUDA call
+    ws = 1 << 30
+
+    def call(w, x=16, y=16, m=4):
+        return L.mmf_bitlinear_fwd(x, 0, m, None, ctypes.byref(w), y, 0, None, None, None, 256, ws, None)
+
+    assert call(mmf.Ternary(16, 32, 8, 32769)) == mmf.MMF_ERR_INVALID_ARG
+    assert call(mmf.Ternary(16, 32, 0, 64)) == mmf.MMF_ERR_INVALID_ARG
+    assert call(mmf.Ternary(16, None, 8, 64)) == mmf.MMF_ERR_INVALID_ARG
+    assert call(mmf.Ternary(16, 32, 8, 64), x=24) == mmf.MMF_ERR_INVALID_ARG
+    assert call(mmf.Ternary(16, 32, 8, 64), y=None) == mmf.MMF_ERR_INVALID_ARG
+    assert call(mmf.Ternary(16, 32, 8, 64), m=-1) == mmf.MMF_ERR_INVALID_ARG
+    assert call(mmf.Ternary(16, 32, 8, 64), m=0) == mmf.MMF_OK
+    # a workspace one byte short is refused, naming the size it needs
+    need = L.mmf_workspace_bytes(mmf.MMF_OP_BITLINEAR, 4, 64, 8, 0)
+    w = mmf.Ternary(16, 32, 8, 64)
+    assert L.mmf_bitlinear_fwd(16, 0, 4, None, ctypes.byref(w), 16, 0, None, None, None, 256, need - 1,
+                               None) == mmf.MMF_ERR_WORKSPACE
