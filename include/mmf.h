@@ -91,9 +91,9 @@ typedef struct {
  * nw_i/f/g/o/gate have d entries, nw_down has `inner`, gnorm_w has d. The GLU reading:
  * gate_proj rows [0, inner) are the SiLU gate, rows [inner, 2*inner) the linear "up" half. */
 typedef struct {
-  int32_t d;     /* hidden size */
-  int32_t inner; /* MLP inner size I; gate_proj is [2I][d], down_proj is [d][I] */
-  float eps;     /* RMSNorm eps of every norm in the block (1e-8) */
+  int32_t d;     /* hidden size, 1 to 32768 */
+  int32_t inner; /* MLP inner size I, 1 to 32768; gate_proj is [2I][d], down_proj is [d][I] */
+  float eps;     /* RMSNorm eps of every norm in the block (1e-8), >= 0 */
   const float *nw_i, *nw_f, *nw_g, *nw_o, *nw_gate, *nw_down, *gnorm_w;
   mmf_ternary i, f, g, o, gate, down;
 } mmf_block_weights;
@@ -286,7 +286,7 @@ mmf_status mmf_validate_packed(const mmf_ternary* w, unsigned long long* bad, mm
  *   dnorm_w[k] = sum_m dr[m][k] x[m][k] rho_m          [w->k] float32 out, or NULL
  *   dW = dy^T rq (the latent float weight's gradient)  [w->n][w->k] float32 out, or NULL
  *   x [m][w->k] x_dtype; norm_w [w->k] float32 or NULL (unit gain); q [m][w->k] int8;
- *   deq [m] float32; dy [m][w->n] dy_dtype. w->n <= 65535.
+ *   deq [m] float32; dy [m][w->n] dy_dtype. w->n <= 65535; 0 <= m <= 2^31 - 1.
  *   ws >= mmf_workspace_bytes(MMF_OP_BITLINEAR_BWD, m, w->k, w->n, 0), 256-byte aligned,
  *   caller-owned. m = 0 writes zero dnorm_w / dW.
  * dr and dW run on the bf16 tensor cores (tcgen05.mma.kind::f16, float32 accumulation): dy (and

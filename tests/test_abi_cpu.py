@@ -328,3 +328,14 @@ def test_bitlinear_limits_on_host(L):
     w = mmf.Ternary(16, 32, 8, 64)
     assert L.mmf_bitlinear_fwd(16, 0, 4, None, ctypes.byref(w), 16, 0, None, None, None, 256, need - 1,
                                None) == mmf.MMF_ERR_WORKSPACE
+
+
+def test_block_and_backward_limits_on_host(L):
+    # block sizes are 1 to 32768 with eps >= 0; the backward takes at most 2^31 - 1 rows
+    for d, inner, eps in ((32776, 64, 1e-8), (64, 32776, 1e-8), (64, 64, -1.0)):
+        bw = mmf.BlockWeightsC(d=d, inner=inner, eps=eps)
+        assert L.mmf_block_fwd(ctypes.byref(bw), None, 0, 1, 1, None, None, None, None, 0,
+                               None) == mmf.MMF_ERR_INVALID_ARG
+    w = mmf.Ternary(16, 32, 8, 64)
+    assert L.mmf_bitlinear_backward(16, 0, 1 << 31, None, 1e-8, ctypes.byref(w), 16, 16, 16, 0, 16, None,
+                                    None, 256, 1 << 40, None) == mmf.MMF_ERR_INVALID_ARG
