@@ -157,6 +157,29 @@ def _dev(t: torch.Tensor) -> torch.Tensor:
     return t
 
 
+def _cuda(t: torch.Tensor, name: str) -> torch.Tensor:
+    """A CUDA tensor of any strides (strided views the library reads through a row stride)."""
+    if not t.is_cuda:
+        raise ValueError(f"{name}: expected a CUDA tensor")
+    return t
+
+
+def _f32(t: torch.Tensor | None, shape: tuple[int, ...], name: str) -> torch.Tensor | None:
+    """An optional contiguous float32 CUDA tensor of the given shape (norm gains, states): the
+    library reads exactly that many float32 values from its pointer."""
+    if t is None:
+        return None
+    if t.dtype != torch.float32 or tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: expected float32 of shape {tuple(shape)}, got {t.dtype} {tuple(t.shape)}")
+    return _dev(t)
+
+
+def _i32(t: torch.Tensor, name: str) -> torch.Tensor:
+    if t.dtype != torch.int32:
+        raise ValueError(f"{name}: expected int32 token ids, got {t.dtype}")
+    return _dev(t)
+
+
 def _stream(device: torch.device) -> int:
     return torch.cuda.current_stream(device).cuda_stream
 
@@ -262,6 +285,9 @@ def _blocks_array(blocks: list[Block]):
 def bitlinear_fwd(x: torch.Tensor, norm_w: torch.Tensor | None, w: PackedTernary,
                   y_dtype: torch.dtype | None = None, debug: bool = False):
     """mmf_bitlinear_fwd on x [..., k]. Returns y, or (y, q, deq, acc) with debug=True."""
+    if x.dim() < 1 or x.shape[-1] != w.k:
+        raise ValueError(f"x: last dimension {tuple(x.shape)[-1:]} is not the weight's k = {w.k}")
+    _f32(norm_w, (w.k,), "norm_w")
     _dev(x)
     lead = x.shape[:-1]
     m = int(x.numel() // w.k) if w.k else 0
@@ -284,6 +310,11 @@ def hgrn_scan(zf: torch.Tensor, zi: torch.Tensor, h0: torch.Tensor | None = None
     """mmf_hgrn_scan on [b, t, d] gate pre-activations (rows may be strided views with unit
     inner stride). Returns (h [b, t, d], h_last [b, d] float32)."""
     b, t, d = zf.shape
+    _cuda(zf, "zf")
+    _cuda(zi, "zi")
+    if tuple(zi.shape) != (b, t, d):
+        raise ValueError("zf and zi need one shape [b, t, d]")
+    _f32(h0, (b, d), "h0")
     if zf.stride(2) != 1 or zi.stride() != zf.stride() or zf.dtype != zi.dtype:
         raise ValueError("zf and zi need the same dtype and strides, unit inner stride")
     if t > 1 and zf.stride(0) != t * zf.stride(1):
@@ -321,6 +352,9 @@ def bitlinear_backward(x: torch.Tensor, norm_w: torch.Tensor | None, w: "PackedT
         if not a.is_contiguous():
             raise ValueError("x, q, deq and dy need contiguous storage")
     m, k = x.shape
+    if k != w.k:
+        raise ValueError(f"x: {k} columns, the weight has k = {w.k}")
+    _f32(norm_w, (k,), "norm_w")
     if tuple(q.shape) != (m, k) or q.dtype != torch.int8 or tuple(deq.shape) != (m,) or tuple(dy.shape) != (m, w.n):
         raise ValueError("shapes: x, q [m, k] (q int8), deq [m], dy [m, n]")
     dx = torch.empty(m, k, dtype=torch.float32, device=x.device)
@@ -344,6 +378,7 @@ def hgrn_scan_backward(zf: torch.Tensor, zi: torch.Tensor, h: torch.Tensor, dh: 
         if a.dtype != zf.dtype or tuple(a.shape) != tuple(zf.shape):
             raise ValueError("zf, zi, h and dh need one dtype and one shape [b, t, d]")
     b, t, d = zf.shape
+    _f32(h0, (b, d), "h0")
     dzf = torch.empty_like(zf)
     dzi = torch.empty_like(zf)
     dh0 = torch.empty(b, d, dtype=torch.float32, device=zf.device)
@@ -382,6 +417,9 @@ def block_fwd(block: Block, x: torch.Tensor, h0: torch.Tensor | None = None):
     """mmf_block_fwd on x [b, t, d]. Returns (y, h_last [b, d] float32)."""
     _dev(x)
     b, t, d = x.shape
+    if d != block.d:
+        raise ValueError(f"x: hidden size {d}, the block's is {block.d}")
+    _f32(h0, (b, d), "h0")
     y = torch.empty_like(x)
     h_last = torch.empty(b, d, dtype=torch.float32, device=x.device)
     ws = workspace(MMF_OP_BLOCK, b * t, block.d, block.inner, 1, x.device)
@@ -396,6 +434,9 @@ def block_fwd_taps(block: Block, x: torch.Tensor, h0: torch.Tensor | None = None
     Returns (y, h_last, taps) with taps a dict of tensors."""
     _dev(x)
     b, t, d = x.shape
+    if d != block.d:
+        raise ValueError(f"x: hidden size {d}, the block's is {block.d}")
+    _f32(h0, (b, d), "h0")
     m, inner, dev, dt = b * t, block.inner, x.device, x.dtype
     y = torch.empty_like(x)
     h_last = torch.empty(b, d, dtype=torch.float32, device=dev)
@@ -423,12 +464,22 @@ def block_fwd_taps(block: Block, x: torch.Tensor, h0: torch.Tensor | None = None
     return y, h_last, taps
 
 
+def _decode_shapes(blocks: list[Block], d: int, b: int, state: torch.Tensor) -> None:
+    if not blocks:
+        raise ValueError("no blocks")
+    if d != blocks[0].d:
+        raise ValueError(f"x: hidden size {d}, the blocks' is {blocks[0].d}")
+    _f32(state, (len(blocks), b, d), "state")
+
+
 def decode_step(blocks: list[Block], x: torch.Tensor, state: torch.Tensor, out: torch.Tensor | None = None):
     """mmf_decode_step: x [b, d] through every block with state [L, b, d] float32 updated in place."""
     _dev(x)
-    _dev(state)
     b, d = x.shape
-    y = out if out is not None else torch.empty_like(x)
+    _decode_shapes(blocks, d, b, state)
+    if out is not None and (tuple(out.shape) != (b, d) or out.dtype != x.dtype or out is x):
+        raise ValueError("out: needs x's shape and dtype and may not be x")
+    y = _dev(out) if out is not None else torch.empty_like(x)
     ws = workspace(MMF_OP_DECODE, b, blocks[0].d, blocks[0].inner, len(blocks), x.device)
     arr = _blocks_array(blocks)
     _check(lib().mmf_decode_step(arr, len(blocks), x.data_ptr(), _dt(x.dtype), b, state.data_ptr(), y.data_ptr(),
@@ -440,8 +491,8 @@ def decode_step_taps(blocks: list[Block], x: torch.Tensor, state: torch.Tensor):
     """mmf_decode_step_taps: decode_step plus every layer's intermediates (see mmf_decode_taps).
     Returns (y, taps) with taps a list (one dict of tensors per layer)."""
     _dev(x)
-    _dev(state)
     b, d = x.shape
+    _decode_shapes(blocks, d, b, state)
     inner, dev, dt = blocks[0].inner, x.device, x.dtype
     y = torch.empty_like(x)
     taps = []
@@ -488,7 +539,7 @@ def decode_fused(b: int, d: int, inner: int) -> bool:
 
 def embed_gather(ids: torch.Tensor, table: torch.Tensor) -> torch.Tensor:
     """mmf_embed_gather: rows of table [vocab, d] for int32 ids."""
-    _dev(ids)
+    _i32(ids, "ids")
     _dev(table)
     out = torch.empty(*ids.shape, table.shape[1], dtype=table.dtype, device=table.device)
     _check(lib().mmf_embed_gather(ids.data_ptr(), ids.numel(), table.data_ptr(), _dt(table.dtype), table.shape[0],
@@ -503,6 +554,11 @@ def lm_head_argmax(x: torch.Tensor, norm_w: torch.Tensor | None, table: torch.Te
     _dev(x)
     _dev(table)
     b, d = x.shape
+    if table.dim() != 2 or table.shape[1] != d:
+        raise ValueError(f"table: expected [vocab, {d}], got {tuple(table.shape)}")
+    _f32(norm_w, (d,), "norm_w")
+    if ids_out is not None and (_i32(ids_out, "ids_out").numel() != b):
+        raise ValueError(f"ids_out: expected {b} int32 entries")
     vocab = table.shape[0]
     ids = ids_out if ids_out is not None else torch.empty(b, dtype=torch.int32, device=x.device)
     logits = torch.empty(b, vocab, dtype=torch.float32, device=x.device) if want_logits else None
@@ -517,11 +573,15 @@ def lm_head_argmax(x: torch.Tensor, norm_w: torch.Tensor | None, table: torch.Te
 def stack_fwd(blocks: list[Block], ids: torch.Tensor, table: torch.Tensor, want_state: bool = False,
               out: torch.Tensor | None = None):
     """mmf_stack_fwd: embedding gather + every block on ids [b, t] int32. Returns (y, h_last or None)."""
-    _dev(ids)
+    _i32(ids, "ids")
     _dev(table)
     b, t = ids.shape
     d = table.shape[1]
-    y = out if out is not None else torch.empty(b, t, d, dtype=table.dtype, device=table.device)
+    if not blocks or blocks[0].d != d:
+        raise ValueError(f"table: hidden size {d} does not match the blocks")
+    if out is not None and (tuple(out.shape) != (b, t, d) or out.dtype != table.dtype):
+        raise ValueError(f"out: expected {table.dtype} of shape {(b, t, d)}")
+    y = _dev(out) if out is not None else torch.empty(b, t, d, dtype=table.dtype, device=table.device)
     h_last = torch.empty(len(blocks), b, d, dtype=torch.float32, device=table.device) if want_state else None
     ws = workspace(MMF_OP_STACK, b * t, blocks[0].d, blocks[0].inner, len(blocks), table.device)
     arr = _blocks_array(blocks)
@@ -572,5 +632,6 @@ def timing_read(cls: str) -> tuple[int, float, float]:
     return n.value, ms.value, wk.value
 
 
-def set_wait_limit(polls: int) -> None:
-    _check(lib().mmf_set_wait_limit(polls), "mmf_set_wait_limit")
+def set_wait_limit(microseconds: int) -> None:
+    """mmf_set_wait_limit: the cap of every bounded in-kernel wait (0 restores the default)."""
+    _check(lib().mmf_set_wait_limit(microseconds), "mmf_set_wait_limit")
