@@ -12,6 +12,8 @@ each restates a kernel's decomposition in numpy and compares it with the oracle'
   the path): the factored chunk form overflows float32 for small gates, while sub-chunks of 16
   steps with every decay taken relative to the sub-chunk (exponents <= 0) reproduce the oracle's
   recurrence in float32 for gates down to 1e-6.
+* The packed format's byte-permute expansion: four byte permutes of one constant turn a word of
+  16 two-bit codes into four int8 quads, and reproduce the oracle's packed codes column by column.
 """
 import numpy as np
 import pytest
@@ -165,3 +167,46 @@ def test_hgrn2_subchunk_form_matches_the_recurrence(fmin):
         o32, S32 = _hgrn2_subchunk(q, f, i, s0, 16, np.float32)
     np.testing.assert_allclose(o32, o_ref, rtol=1e-4, atol=1e-5 * np.abs(o_ref).max())
     np.testing.assert_allclose(S32, S_ref, rtol=1e-4, atol=1e-5 * np.abs(S_ref).max())
+
+
+# ---------------------------------------------------------------------------------------------
+# The packed format's byte-permute expansion (the device helper that turns one 32-bit word of
+# 16 codes into four int8 quads), restated with the byte-permute instruction's definition: each
+# 4-bit selector picks one byte of the 8-byte pair {y, x} (x = bytes 0-3); result byte i takes
+# the byte that selector nibble i names.
+# ---------------------------------------------------------------------------------------------
+def _byte_perm(x: int, y: int, s: int) -> int:
+    pair = (y << 32) | x
+    out = 0
+    for i in range(4):
+        sel = (s >> (4 * i)) & 7
+        out |= ((pair >> (8 * sel)) & 0xFF) << (8 * i)
+    return out
+
+
+def _expand_word(w: int) -> list[int]:
+    lo = w & 0x33333333
+    hi = (w >> 2) & 0x33333333
+    table = 0xFF000100                      # bytes 0x00, 0x01, 0x00, 0xFF for fields 00, 01, 10, 11
+    quads = [_byte_perm(table, 0, lo & 0xFFFF), _byte_perm(table, 0, hi & 0xFFFF),
+             _byte_perm(table, 0, lo >> 16), _byte_perm(table, 0, hi >> 16)]
+    codes = []
+    for q in quads:                         # lowest column in byte 0, int8 lanes
+        codes += [((q >> (8 * b)) & 0xFF) - 256 * (((q >> (8 * b)) & 0xFF) >= 128) for b in range(4)]
+    return codes
+
+
+@pytest.mark.parametrize("n,k", [(3, 16), (5, 65), (2, 200), (4, 1024)])
+def test_byte_permute_expansion_recovers_the_oracles_packed_codes(n, k):
+    rng = np.random.default_rng(180 + k)
+    t = rng.integers(-1, 2, (n, k)).astype(np.int8)
+    words = O.pack_codes(t).astype(np.uint32)
+    kw = O.packed_row_words(k)
+    assert words.shape == (n, kw)
+    for r in range(n):
+        got = [c for w in words[r] for c in _expand_word(int(w))]
+        assert got[:k] == t[r].tolist()
+        assert not any(got[k:])             # padding columns expand to zero codes
+    # the unused pattern 10 expands to 0 (a malformed field reads as a zero weight)
+    assert _expand_word(0xAAAAAAAA) == [0] * 16
+    assert _expand_word(0x55555555) == [1] * 16 and _expand_word(0xFFFFFFFF) == [-1] * 16
