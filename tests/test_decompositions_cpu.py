@@ -14,6 +14,8 @@ each restates a kernel's decomposition in numpy and compares it with the oracle'
   recurrence in float32 for gates down to 1e-6.
 * The packed format's byte-permute expansion: four byte permutes of one constant turn a word of
   16 two-bit codes into four int8 quads, and reproduce the oracle's packed codes column by column.
+* The GEMM epilogue's int32 -> float32 step through the mantissa of 1.5 * 2^23: exact for every
+  accumulator the library can produce (K <= 32768), checked exhaustively.
 """
 import numpy as np
 import pytest
@@ -210,3 +212,25 @@ def test_byte_permute_expansion_recovers_the_oracles_packed_codes(n, k):
     # the unused pattern 10 expands to 0 (a malformed field reads as a zero weight)
     assert _expand_word(0xAAAAAAAA) == [0] * 16
     assert _expand_word(0x55555555) == [1] * 16 and _expand_word(0xFFFFFFFF) == [-1] * 16
+
+
+# ---------------------------------------------------------------------------------------------
+# The GEMM epilogue's int32 -> float32 step without a conversion instruction: the bit pattern
+# a + 0x4B400000 is the float 1.5 * 2^23 + a (mantissa spacing 1 there), and subtracting 1.5 * 2^23
+# is exact, so the result is float(a) exactly for every |a| <= 2^22 -- which covers every
+# accumulator of K <= 32768 int8 x ternary products (|acc| <= 127 K < 2^22).
+# ---------------------------------------------------------------------------------------------
+def _acc_to_float(a: np.ndarray) -> np.ndarray:
+    bits = (a.astype(np.int64) + 0x4B400000).astype(np.uint32)
+    return bits.view(np.float32) - np.float32(12582912.0)
+
+
+def test_mantissa_int_to_float_is_exact_over_the_accumulator_range():
+    a = np.arange(-(1 << 22), (1 << 22) + 1, dtype=np.int32)       # every value, exhaustively
+    got = _acc_to_float(a)
+    assert got.dtype == np.float32
+    assert np.array_equal(got, a.astype(np.float32))
+    assert 127 * 32768 < (1 << 22)                                    # the library's largest K
+    # one step outside the range the identity no longer holds: the guard on K is needed
+    out = np.array([(1 << 22) + 1, -(1 << 22) - 1], dtype=np.int32)
+    assert not np.any(_acc_to_float(out) == out.astype(np.float32))
