@@ -16,6 +16,8 @@ each restates a kernel's decomposition in numpy and compares it with the oracle'
   16 two-bit codes into four int8 quads, and reproduce the oracle's packed codes column by column.
 * The GEMM epilogue's int32 -> float32 step through the mantissa of 1.5 * 2^23: exact for every
   accumulator the library can produce (K <= 32768), checked exhaustively.
+* The scan's gates with one reciprocal per channel and exponent arguments clamped at -40: float32-
+  accurate against sigmoid and SiLU (1 - f) over saturated arguments, never inf or NaN.
 """
 import numpy as np
 import pytest
@@ -234,3 +236,45 @@ def test_mantissa_int_to_float_is_exact_over_the_accumulator_range():
     # one step outside the range the identity no longer holds: the guard on K is needed
     out = np.array([(1 << 22) + 1, -(1 << 22) - 1], dtype=np.int32)
     assert not np.any(_acc_to_float(out) == out.astype(np.float32))
+
+
+# ---------------------------------------------------------------------------------------------
+# The scan's gate arithmetic with one reciprocal per channel: ef = e^-zf and ez = e^-zi with both
+# exponent arguments clamped at -40, r = 1 / ((1 + ef)(1 + ez)), f = (1 + ez) r, i = zi ef r.
+# Restated in float32 (exact exponentials and reciprocal; the device's approximate ones add a few
+# ulp) against the oracle's sigmoid and SiLU (1 - f) in float64, over saturated arguments too.
+# ---------------------------------------------------------------------------------------------
+def _gates_one_reciprocal(zf: np.ndarray, zi: np.ndarray):
+    f32 = np.float32
+    zf, zi = zf.astype(f32), zi.astype(f32)
+    nl = f32(-1.4426950408889634)
+    ef = np.exp2(np.maximum(zf, f32(-40.0)) * nl, dtype=f32)
+    ez = np.exp2(np.maximum(zi, f32(-40.0)) * nl, dtype=f32)
+    pz = ez + f32(1.0)
+    r = f32(1.0) / ((ef + f32(1.0)) * pz)
+    return pz * r, (zi * ef) * r
+
+
+def test_one_reciprocal_gates_match_sigmoid_and_silu():
+    g = np.linspace(-200.0, 200.0, 801)
+    zf, zi = np.meshgrid(g, g, indexing="ij")
+    rng = np.random.default_rng(190)
+    zf = np.concatenate([zf.ravel(), rng.normal(0, 3, 20000), rng.normal(4, 1, 20000)])
+    zi = np.concatenate([zi.ravel(), rng.normal(0, 3, 20000), rng.normal(0, 1, 20000)])
+    zf = zf.astype(np.float32).astype(np.float64)
+    zi = zi.astype(np.float32).astype(np.float64)
+    # the definitions in float64 with 1 - f taken as sigmoid(-zf) (no cancellation as f -> 1);
+    # they agree with the oracle's f and SiLU(zi) (1 - f) to its own float64 rounding of 1 - f
+    with np.errstate(over="ignore"):
+        f_ref = 1.0 / (1.0 + np.exp(-zf))
+        i_ref = zi / (1.0 + np.exp(-zi)) / (1.0 + np.exp(zf))
+    f_o, i_o = O.hgrn_gates(zf, zi)
+    assert np.all(np.abs(f_o - f_ref) <= 1e-15)
+    assert np.all(np.abs(i_o - i_ref) <= 1e-12 * np.abs(i_ref) + 2.3e-16 * np.abs(zi) / (1.0 + np.exp(-zi)))
+    with np.errstate(over="raise", invalid="raise"):
+        f, i = _gates_one_reciprocal(zf, zi)
+    assert np.all(np.isfinite(f)) and np.all(np.isfinite(i))
+    # float32 rounding (the exponent argument's rounding dominates near the clamp), and the clamp
+    # itself: sigmoid(-40) < 5e-18 bounds what it moves
+    np.testing.assert_array_less(np.abs(f - f_ref), 5e-6 * np.abs(f_ref) + 5e-18)
+    np.testing.assert_array_less(np.abs(i - i_ref), 5e-6 * np.abs(i_ref) + 5e-18 * np.abs(zi) + 1e-38)
