@@ -254,7 +254,7 @@ __device__ __forceinline__ void load8(const void* base, int64_t idx, float (&o)[
     o[4] = b.x; o[5] = b.y; o[6] = b.z; o[7] = b.w;
   }
 }
-// Bits of x + 1.5 * 2^23 for |x| <= 127.5: the addition (where the float32 spacing is exactly 1)
+// Bits of x + 1.5 * 2^23 for |x| < 127.5: the addition (where the float32 spacing is exactly 1)
 // rounds half to even, and the low byte of the result is the int8 code rint(x) itself
 // (0x4B400000 has a zero low byte). No clamp is needed: x = r * fl(127 / a) with a the maximum of
 // the very |r| values, so |x| <= 127 (1 + 2^-24)^2 < 127.5 and the code lies in [-127, 127].

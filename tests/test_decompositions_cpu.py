@@ -18,6 +18,8 @@ each restates a kernel's decomposition in numpy and compares it with the oracle'
   accumulator the library can produce (K <= 32768), checked exhaustively.
 * The scan's gates with one reciprocal per channel and exponent arguments clamped at -40: float32-
   accurate against sigmoid and SiLU (1 - f) over saturated arguments, never inf or NaN.
+* The activation code with no clamp: a row's maximum maps to exactly 127 (a whole binade of a
+  checked), and the low byte of x + 1.5 * 2^23 is rint(x), ties to even.
 """
 import numpy as np
 import pytest
@@ -278,3 +280,34 @@ def test_one_reciprocal_gates_match_sigmoid_and_silu():
     # itself: sigmoid(-40) < 5e-18 bounds what it moves
     np.testing.assert_array_less(np.abs(f - f_ref), 5e-6 * np.abs(f_ref) + 5e-18)
     np.testing.assert_array_less(np.abs(i - i_ref), 5e-6 * np.abs(i_ref) + 5e-18 * np.abs(zi) + 1e-38)
+
+
+# ---------------------------------------------------------------------------------------------
+# The activation code without a clamp or a conversion instruction: x = r * fl(127 / a) is at most
+# fl(a * fl(127 / a)) in magnitude (a = max |r| of the row), which rounds to exactly 127; and the
+# low byte of the float32 bits of x + 1.5 * 2^23 is rint(x) (ties to even) for |x| < 127.5 (at
+# x = +127.5 the code would be 128, which the bound above keeps out of reach).
+# ---------------------------------------------------------------------------------------------
+def test_row_maximum_maps_to_code_127_without_a_clamp():
+    f32 = np.float32
+    one_binade = (np.arange(1 << 23, dtype=np.uint32) | np.uint32(0x3F800000)).view(np.float32)  # [1, 2)
+    rng = np.random.default_rng(200)
+    spread = np.exp(rng.uniform(np.log(1e-5), np.log(1e30), 2_000_000)).astype(f32)
+    for a in (one_binade, spread):
+        x = a * (f32(127.0) / a)             # float32 product of float32 operands, each rounded
+        assert x.dtype == f32
+        assert np.all(np.abs(x - 127.0) <= 2 * np.spacing(f32(127.0)))
+        assert np.all(np.rint(x) == 127.0)
+
+
+def test_code_byte_from_the_rounding_add_is_rint_ties_to_even():
+    f32 = np.float32
+    halves = np.arange(-127.5, 128.0, 1.0, dtype=f32)
+    near = np.concatenate([halves, np.nextafter(halves, f32(-200)), np.nextafter(halves, f32(200)),
+                           np.arange(-127, 128, dtype=f32)])
+    rng = np.random.default_rng(201)
+    x = np.concatenate([near, rng.uniform(-127.5, 127.5, 2_000_000).astype(f32)])
+    x = x[np.abs(x) < 127.5]
+    bits = (x + f32(12582912.0)).astype(f32).view(np.uint32)
+    code = (bits & 0xFF).astype(np.uint8).view(np.int8)
+    assert np.array_equal(code.astype(np.int64), np.rint(x).astype(np.int64))
