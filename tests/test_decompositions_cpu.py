@@ -298,6 +298,11 @@ def test_row_maximum_maps_to_code_127_without_a_clamp():
         assert x.dtype == f32
         assert np.all(np.abs(x - 127.0) <= 2 * np.spacing(f32(127.0)))
         assert np.all(np.rint(x) == 127.0)
+    # the dequantisation factor a * fl(1/127) is within 1.5 ulp of a / 127 (scaling by powers of
+    # two is exact, so one binade covers every a in the normal range)
+    d = one_binade * (f32(1.0) / f32(127.0))
+    err = np.abs(d.astype(np.float64) - one_binade.astype(np.float64) / 127.0)
+    assert np.all(err <= 1.5 * np.spacing(d).astype(np.float64))
 
 
 def test_code_byte_from_the_rounding_add_is_rint_ties_to_even():
