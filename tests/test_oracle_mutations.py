@@ -1,7 +1,8 @@
 """The oracle's pins catch plausible mistakes: each test here plants one mistake in a copy of an
-oracle function (on the CPU, in this process only), runs the pins of that function against the
-planted copy, and requires that they fail. A pin set that passed a planted mistake would not be
-pinning the function."""
+oracle function (on the CPU, in this process only), runs the pins against the planted copy, and
+requires that they fail -- for HGRN2, the backward functions and every function of the forward
+(recurrence, gates, RMSNorm, both quantisers, BitLinear, the block's wiring, the packed layout and
+the head). A pin set that passed a planted mistake would not be pinning the function."""
 import numpy as np
 import pytest
 
@@ -149,3 +150,178 @@ def test_backward_pins_pass_on_the_oracle():
 def test_backward_pins_catch_planted_mistakes(monkeypatch, name, mutant):
     monkeypatch.setattr(O, name, mutant)
     assert _failures(BACKWARD_PINS) >= 1
+
+
+# ---------------------------------------------------------------------------------------------
+# the forward: every oracle function the block uses, each with plausible mistakes planted in the
+# package and in the module (so the oracle's internal calls see the planted copy too); the whole
+# pin set runs against each and at least one pin must fail
+# ---------------------------------------------------------------------------------------------
+def _expand(fn):
+    marks = [m for m in getattr(fn, "pytestmark", []) if m.name == "parametrize"]
+    if not marks:
+        return [fn]
+    names = [n.strip() for n in marks[0].args[0].split(",")]
+    out = []
+    for vals in marks[0].args[1]:
+        vals = vals if len(names) > 1 else (vals,)
+        out.append(lambda fn=fn, kw=dict(zip(names, vals)): fn(**kw))
+    return out
+
+
+ALL_PINS = [p for name in sorted(dir(P)) if name.startswith("test_") for p in _expand(getattr(P, name))]
+
+
+def _plant(monkeypatch, name, fn):
+    monkeypatch.setattr(O, name, fn)
+    monkeypatch.setattr(O.mmf_oracle, name, fn)
+
+
+def _scan_mutant(kind):
+    def run(f, i, h0=None):
+        f = np.asarray(f, dtype=np.float64)
+        i = np.asarray(i, dtype=np.float64)
+        b, t, d = f.shape
+        h = np.zeros((b, t, d))
+        prev = np.zeros((b, d)) if (h0 is None or kind == "h0_ignored") else np.asarray(h0, dtype=np.float64).copy()
+        for s in range(t):
+            if kind == "previous_input":
+                prev = f[:, s] * prev + (i[:, s - 1] if s else 0.0)
+            elif kind == "input_decayed":
+                prev = f[:, s] * (prev + i[:, s])
+            else:
+                prev = f[:, s] * prev + i[:, s]
+            h[:, s] = prev
+        return h
+    return run
+
+
+def _gates_mutant(kind):
+    def run(zf, zi):
+        f = O.sigmoid(-np.asarray(zf) if kind == "sign" else zf)
+        if kind == "complement_dropped":
+            return f, O.silu(zi)
+        if kind == "forget_as_input_gate":
+            return f, O.silu(zi) * f
+        return f, O.silu(zi) * (1.0 - f)
+    return run
+
+
+def _rmsnorm_mutant(kind):
+    def run(x, w, eps=O.EPS_NORM):
+        x = np.asarray(x, dtype=np.float64)
+        ms = np.sum(x * x, axis=-1, keepdims=True) if kind == "sum_not_mean" else np.mean(x * x, axis=-1, keepdims=True)
+        r = x / (np.sqrt(ms) + eps) if kind == "eps_outside" else x / np.sqrt(ms + eps)
+        if w is not None and kind != "gain_ignored":
+            r = r * np.asarray(w, dtype=np.float64)
+        return r
+    return run
+
+
+def _ternarize_mutant(kind):
+    def run(W):
+        W32 = np.asarray(W, dtype=np.float32)
+        if kind == "absmax_scale":
+            s = np.float32(max(float(np.max(np.abs(W32))) if W32.size else 0.0, O.EPS_QUANT))
+        else:
+            s = O.weight_scale(W32)
+        v = W32 / s
+        t = np.trunc(v) if kind == "truncate" else np.rint(v)
+        return np.clip(t, -1, 1).astype(np.int8), s
+    return run
+
+
+def _act_quant_mutant(kind):
+    def run(r):
+        r32 = np.asarray(r, dtype=np.float64).astype(np.float32)
+        red = np.mean if kind == "absmean" else np.max
+        a = red(np.abs(r32), axis=-1, keepdims=True) if r32.shape[-1] else np.zeros(r32.shape[:-1] + (1,), np.float32)
+        a = np.maximum(a, np.float32(O.EPS_QUANT)).astype(np.float32)
+        v = (r32 * (np.float32(127.0) / a).astype(np.float32)).astype(np.float32)
+        q = np.clip(np.rint(v), -127, 127).astype(np.int8)
+        deq = a[..., 0].astype(np.float64) / (128.0 if kind == "deq_128" else 127.0)
+        return q, deq, v
+    return run
+
+
+def _bitlinear_mutant(kind):
+    def run(x, norm_w, t, s_w, eps=O.EPS_NORM):
+        x = np.asarray(x, dtype=np.float64)
+        lead, k = x.shape[:-1], x.shape[-1]
+        x2 = x.reshape(-1, k)
+        r = O.rmsnorm(x2, norm_w, eps)
+        q, deq, v = O.act_quant(r)
+        acc = O.int_matmul(q, t)
+        y = acc.astype(np.float64) * (1.0 if kind == "no_deq" else deq[:, None]) * (1.0 if kind == "no_scale" else float(s_w))
+        if kind == "norm_skipped":
+            q2, deq2, _ = O.act_quant(x2)
+            y = O.int_matmul(q2, t) * deq2[:, None] * float(s_w)
+            q, deq, acc = q2, deq2, O.int_matmul(q2, t)
+        return y.reshape(lead + (t.shape[0],)), {"r": r, "q": q, "deq": deq, "v": v, "acc": acc}
+    return run
+
+
+def _block_mutant(kind):
+    def run(x, qp, h0=None, eps=O.EPS_NORM):
+        x = np.asarray(x, dtype=np.float64)
+        zi, _ = O.bitlinear(x, qp["nw_i"], qp["t_i"], qp["s_i"], eps)
+        zf, _ = O.bitlinear(x, qp["nw_f"], qp["t_f"], qp["s_f"], eps)
+        g, _ = O.bitlinear(x, qp["nw_g"], qp["t_g"], qp["s_g"], eps)
+        f, i = O.hgrn_gates(zf, zi)
+        h = O.hgrn_scan(f, i, h0)
+        u = O.rmsnorm(h, qp["gnorm_w"], eps) * (g if kind == "gate_without_silu" else O.silu(g))
+        o, _ = O.bitlinear(u, qp["nw_o"], qp["t_o"], qp["s_o"], eps)
+        x1 = o if kind == "no_first_residual" else x + o
+        gu, _ = O.bitlinear(x1, qp["nw_gate"], qp["t_gate"], qp["s_gate"], eps)
+        inner = gu.shape[-1] // 2
+        a, b = gu[..., :inner], gu[..., inner:]
+        v = O.silu(b) * a if kind == "glu_halves_swapped" else O.silu(a) * b
+        dn, _ = O.bitlinear(v, qp["nw_down"], qp["t_down"], qp["s_down"], eps)
+        y = x1 + dn
+        inter = {"zi": zi, "zf": zf, "g": g, "f": f, "i": i, "h": h, "u": u, "x1": x1, "v": v}
+        return y, h[:, -1, :].copy(), inter
+    return run
+
+
+def _code_bit_mutant(j):
+    return 2 * j                                   # plain sequential fields, not the quad layout
+
+
+def _lm_head_mutant(x, norm_w, table, eps=O.EPS_NORM):
+    return np.asarray(x, dtype=np.float64) @ np.asarray(table, dtype=np.float64).T   # final norm dropped
+
+
+FORWARD_MUTANTS = [
+    ("hgrn_scan", _scan_mutant("previous_input"), "scan:i_{t-1}"),
+    ("hgrn_scan", _scan_mutant("input_decayed"), "scan:f(h+i)"),
+    ("hgrn_scan", _scan_mutant("h0_ignored"), "scan:h0"),
+    ("hgrn_gates", _gates_mutant("sign"), "gates:sign"),
+    ("hgrn_gates", _gates_mutant("complement_dropped"), "gates:no_1-f"),
+    ("hgrn_gates", _gates_mutant("forget_as_input_gate"), "gates:f_for_1-f"),
+    ("rmsnorm", _rmsnorm_mutant("sum_not_mean"), "rmsnorm:sum"),
+    ("rmsnorm", _rmsnorm_mutant("eps_outside"), "rmsnorm:eps"),
+    ("rmsnorm", _rmsnorm_mutant("gain_ignored"), "rmsnorm:gain"),
+    ("ternarize", _ternarize_mutant("absmax_scale"), "ternarize:absmax"),
+    ("ternarize", _ternarize_mutant("truncate"), "ternarize:trunc"),
+    ("act_quant", _act_quant_mutant("absmean"), "act_quant:absmean"),
+    ("act_quant", _act_quant_mutant("deq_128"), "act_quant:deq/128"),
+    ("bitlinear", _bitlinear_mutant("no_deq"), "bitlinear:no_a/127"),
+    ("bitlinear", _bitlinear_mutant("no_scale"), "bitlinear:no_s"),
+    ("bitlinear", _bitlinear_mutant("norm_skipped"), "bitlinear:no_norm"),
+    ("block_forward", _block_mutant("gate_without_silu"), "block:g_no_silu"),
+    ("block_forward", _block_mutant("no_first_residual"), "block:no_residual"),
+    ("block_forward", _block_mutant("glu_halves_swapped"), "block:glu_swapped"),
+    ("code_bit", _code_bit_mutant, "pack:code_bit"),
+    ("lm_head_logits", _lm_head_mutant, "head:no_norm"),
+]
+
+
+def test_all_pins_pass_on_the_oracle():
+    assert len(ALL_PINS) >= 40
+    assert _failures(ALL_PINS) == 0
+
+
+@pytest.mark.parametrize("name,mutant", [(n, m) for n, m, _ in FORWARD_MUTANTS], ids=[i for _, _, i in FORWARD_MUTANTS])
+def test_forward_pins_catch_planted_mistakes(monkeypatch, name, mutant):
+    _plant(monkeypatch, name, mutant)
+    assert _failures(ALL_PINS) >= 1
