@@ -291,6 +291,37 @@ def _lm_head_mutant(x, norm_w, table, eps=O.EPS_NORM):
     return np.asarray(x, dtype=np.float64) @ np.asarray(table, dtype=np.float64).T   # final norm dropped
 
 
+_REAL_DECODE = O.decode_step
+
+
+def _decode_mutant(x, layers, state, eps=O.EPS_NORM):
+    # the carried state is not read: every step starts from h_prev = 0
+    return _REAL_DECODE(x, layers, np.zeros_like(np.asarray(state, dtype=np.float64)), eps)
+
+
+def _count_mutant(words, k):
+    # a 10 field in a padding column counted twice (once as 10, once as nonzero padding)
+    words = np.asarray(words, dtype=np.uint64)
+    bad = 0
+    for col in range(16 * words.shape[1]):
+        w, j = divmod(col, 16)
+        f = (words[:, w] >> np.uint64(O.code_bit(j))) & np.uint64(3)
+        bad += int(np.count_nonzero(f == 2))
+        if col >= k:
+            bad += int(np.count_nonzero(f != 0))
+    return bad
+
+
+def _greedy_mutant(logits):
+    lg = np.asarray(logits)
+    return (lg.shape[-1] - 1 - np.argmax(lg[..., ::-1], axis=-1)).astype(np.int64)   # last index on ties
+
+
+def _embed_mutant(ids, table):
+    t = np.asarray(table, dtype=np.float64)
+    return t[(np.asarray(ids, dtype=np.int64) + 1) % t.shape[0]]                    # off by one row
+
+
 FORWARD_MUTANTS = [
     ("hgrn_scan", _scan_mutant("previous_input"), "scan:i_{t-1}"),
     ("hgrn_scan", _scan_mutant("input_decayed"), "scan:f(h+i)"),
@@ -313,6 +344,10 @@ FORWARD_MUTANTS = [
     ("block_forward", _block_mutant("glu_halves_swapped"), "block:glu_swapped"),
     ("code_bit", _code_bit_mutant, "pack:code_bit"),
     ("lm_head_logits", _lm_head_mutant, "head:no_norm"),
+    ("decode_step", _decode_mutant, "decode:state_dropped"),
+    ("count_malformed_fields", _count_mutant, "integrity:double_count"),
+    ("greedy_next", _greedy_mutant, "greedy:last_on_ties"),
+    ("embed", _embed_mutant, "embed:off_by_one"),
 ]
 
 
