@@ -20,6 +20,8 @@ each restates a kernel's decomposition in numpy and compares it with the oracle'
   accurate against sigmoid and SiLU (1 - f) over saturated arguments, never inf or NaN.
 * The activation code with no clamp: a row's maximum maps to exactly 127 (a whole binade of a
   checked), and the low byte of x + 1.5 * 2^23 is rint(x), ties to even.
+* The integrity check's word-level bit count equals the oracle's field-by-field definition on
+  packed codes, planted faults and random words.
 """
 import numpy as np
 import pytest
@@ -316,3 +318,48 @@ def test_code_byte_from_the_rounding_add_is_rint_ties_to_even():
     bits = (x + f32(12582912.0)).astype(f32).view(np.uint32)
     code = (bits & 0xFF).astype(np.uint8).view(np.int8)
     assert np.array_equal(code.astype(np.int64), np.rint(x).astype(np.int64))
+
+
+# ---------------------------------------------------------------------------------------------
+# The integrity check's word-level count: with lo / hi the low / high bits of the 16 fields of a
+# word and pad the low bits of its padding fields, a word holds popc(hi & ~lo & ~pad) real-column
+# 10 fields and popc((lo | hi) & pad) nonzero padding fields (a padding 10 counted once).
+# Restated with the field offsets of the oracle's code_bit, against the oracle's definition.
+# ---------------------------------------------------------------------------------------------
+def _fields_from(jmin: int) -> int:
+    m = 0
+    for j in range(jmin, 16):
+        m |= 1 << O.code_bit(j)
+    return m
+
+
+def _word_level_count(words: np.ndarray, k: int) -> int:
+    n, kw = words.shape
+    total = 0
+    for r in range(n):
+        for e in range(kw):
+            w = int(words[r, e])
+            col0 = e * 16
+            lo, hi = w & 0x55555555, (w >> 1) & 0x55555555
+            pad = _fields_from(max(k - col0, 0)) if col0 + 16 > k else 0
+            total += bin(hi & ~lo & ~pad & 0xFFFFFFFF).count("1") + bin((lo | hi) & pad).count("1")
+    return total
+
+
+@pytest.mark.parametrize("k", [1, 16, 70, 130, 256])
+def test_integrity_word_count_equals_the_oracles_definition(k):
+    rng = np.random.default_rng(210 + k)
+    t = rng.integers(-1, 2, (6, k)).astype(np.int8)
+    words = O.pack_codes(t)
+    assert _word_level_count(words, k) == O.count_malformed_fields(words, k) == 0
+    kw = words.shape[1]
+    bad = words.copy()
+    bad[1, 0] = (int(bad[1, 0]) & ~(3 << O.code_bit(0))) | (2 << O.code_bit(0))      # real column: 10
+    if 16 * kw > k:                                                                  # padding fields
+        col = k
+        bad[2, col // 16] = int(bad[2, col // 16]) | (1 << O.code_bit(col % 16))      # +1
+        col = 16 * kw - 1
+        bad[3, col // 16] = int(bad[3, col // 16]) | (2 << O.code_bit(col % 16))      # 10, counted once
+    assert _word_level_count(bad, k) == O.count_malformed_fields(bad, k) >= 1
+    garbage = rng.integers(0, 1 << 32, (4, kw), dtype=np.uint64).astype(np.uint32)
+    assert _word_level_count(garbage, k) == O.count_malformed_fields(garbage, k)
