@@ -138,3 +138,27 @@ def test_oracle_chain_groups_follow_the_block(case):
     assert [len(g) for g in groups] == [3, 1, 1, 1]
     q_i, _ = groups[0][0]
     assert np.array_equal(q_i, taps["q_ifg"][0].numpy())
+
+
+def test_chain_checker_over_two_layers():
+    from parity_checks import check_chain_end_to_end
+
+    sh = synth.BlockShape("t", 32, 64, 1)
+    qps = [O.quantize_block(synth.block_params(310 + l, sh, random_norms=True)) for l in range(2)]
+    x = synth.activations(312, (2, 5, 32))
+    taps, states, cur = [], [], x.astype(np.float64)
+    for qp in qps:
+        t, y, hl = _oracle_taps(cur, qp)
+        taps.append(t)
+        states.append(hl)
+        cur = y
+    rel, clean = check_chain_end_to_end(x, qps, taps, cur, states_g=states)
+    assert rel < 1e-12 and clean == 1.0
+    bad = cur.copy()
+    bad[0, 2, 5] += 1e-2 * (1 + abs(bad[0, 2, 5]))
+    with pytest.raises(AssertionError):
+        check_chain_end_to_end(x, qps, taps, bad, states_g=states)
+    bad_states = [s.copy() for s in states]
+    bad_states[1][1, 3] += 1e-2
+    with pytest.raises(AssertionError):
+        check_chain_end_to_end(x, qps, taps, cur, states_g=bad_states)
