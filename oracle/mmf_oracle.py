@@ -24,7 +24,7 @@ section):
 The pages leave several steps open; the readings taken (absmax-to-127 activation codes, a
 per-tensor absmean weight scale with floor 1e-5, ties to even, f = sigmoid(zf),
 i = SiLU(zi) * (1 - f), residuals around the token mixer and the MLP, no bias, h_0 = 0,
-gate half first in the GLU split) are listed with the workload recipe in the design notes.
+gate half first in the GLU split) are each restated in the function that takes it.
 
 Where floating point decides an integer code, this oracle takes the decision in float32, the
 precision of the CUDA path: the weight code is rint(float32(W) / float32(s)) and the activation

@@ -3,8 +3,8 @@
 Each stage of a kernel path is compared with the oracle's definition of that stage applied to the
 kernel's own inputs to it (the debug taps), so every stage is checked element by element whatever
 happened upstream: integer accumulations exactly, activation codes exactly except by one step where
-the oracle's float32 value lies within a margin of a half-integer (reading 4 of the design notes:
-both sides decide in float32, so a code can flip only at such a near-tie), floats within the
+the oracle's float32 value lies within a margin of a half-integer (both sides decide in float32,
+so a code can flip only at such a near-tie), floats within the
 stated tolerances (float32: 1e-3 relative + 1e-5 absolute; bfloat16: 2e-2 relative).
 """
 import numpy as np
@@ -99,7 +99,7 @@ def check_block_stages(x, qp, taps, y_g, hl_g, h0, bf16, glu_fused=False):
 def chain_clean_rows(kernel_groups, oracle_groups, B, T, scan_groups, margins):
     """Follows every chained code decision of the forward in order and returns the rows that saw no
     code differing from the oracle's own chain, asserting that in every other row the FIRST
-    difference sits at a near-tie of the oracle's float32 value (reading 4: both sides decide in
+    difference sits at a near-tie of the oracle's float32 value (both sides decide in
     float32, so only a value within rounding of a half-integer can round the other way; after it,
     the row's later inputs differ and its later codes may differ anywhere).
 

@@ -11,10 +11,11 @@ I 2816, 1.3B d 2048 / I 5632, 2.7B d 2560 / I 7040), through the C ABI.
   then end to end.
 
 End to end, the oracle's own chain differs from the kernels' only where a float32 code decision
-sits at a near-tie (reading 4 of the design notes); after such a flip the row's later
+sits at a near-tie (both sides decide in float32, so only a value within rounding of a
+half-integer can round the other way); after such a flip the row's later
 quantisations see different inputs and differ in numbers. In float32 the end-to-end check follows
 every row's chain of code decisions: the first difference must be a near-tie, and rows without one
-match elementwise. In bf16 the kernels store every intermediate in bf16 (reading 9) and the oracle
+match elementwise. In bf16 the kernels store every intermediate in bf16 and the oracle
 none, so end to end only a sanity bound holds; the stage checks carry the elementwise claim.
 """
 import numpy as np

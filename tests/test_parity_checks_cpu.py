@@ -1,6 +1,6 @@
 """The GPU parity checkers themselves, on the CPU: fed the oracle's own stage values as if a kernel
 had produced them, they pass; fed a corrupted stage, a code off by one away from a near-tie, or a
-wrong residual, they fail; and the near-tie rule of reading 4 (both sides decide in float32) marks
+wrong residual, they fail; and the near-tie rule (both sides decide in float32) marks
 exactly the rows it should. A checker that accepted anything would make every GPU parity test
 vacuous."""
 import numpy as np

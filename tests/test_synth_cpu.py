@@ -1,6 +1,7 @@
-"""The seeded input generators produce the recipe the design notes state (distributions, shapes,
-dtypes, determinism), and hold none of the method's arithmetic (checked by what they import and
-return: raw draws only)."""
+"""The seeded input generators produce the input recipe of the tests and the benchmark -- latent
+weights N(0, 0.02^2), activations N(0, 1), forget pre-activations N(4, 1) (long memory) or N(0, 1),
+input pre-activations N(0, 1), token ids uniform in [0, 32000), gains ones or N(1, 0.1^2), the model
+table's shapes -- reproducibly from their seeds, and hold none of the method's arithmetic."""
 import numpy as np
 import pytest
 
