@@ -14,9 +14,10 @@
 // the input rows and their norm gains, then of the CTA's packed weight rows, into shared memory
 // (two barriers);
 // while the weights stream in, the CTA quantises the input rows itself -- every CTA computes the
-// same codes, in the arithmetic of norm_quant_vec_kernel -- and each warp then forms whole
-// output channels: lanes stride over 64-code chunks of the weight row (expanded with byte
-// permutes), dp4a against the codes, and a warp reduction per (matrix, row).
+// same codes, in the arithmetic of norm_quant_vec_kernel -- and each half-warp then forms whole
+// output channels (one at a time, four from four token rows on): its 16 lanes stride over 32-code
+// (8-byte) pieces of the weight rows (expanded with byte permutes), dp4a them against the codes,
+// and reduce per (matrix, channel, row) with shuffles inside the half-warp.
 #pragma once
 
 #include "common.cuh"
