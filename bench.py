@@ -735,6 +735,19 @@ def run_next_rows(device, flush, peaks) -> dict:
     return out
 
 
+def guarded(fn, *args):
+    """One extra measurement of the JSON line: a failure there is reported in its entry (and its
+    traceback on stderr) instead of losing the headline line. Used on one GPU only, where no other
+    rank waits in a collective."""
+    try:
+        return fn(*args)
+    except Exception as e:  # noqa: BLE001 -- any failure of an extra is reported, not raised
+        import traceback
+
+        traceback.print_exc(file=sys.stderr)
+        return {"error": f"{type(e).__name__}: {e}"}
+
+
 def run_gpu(args, wl):
     import torch
     import torch.distributed as dist
@@ -845,13 +858,13 @@ def run_gpu(args, wl):
     hbm, hbm_src = hbm_peak(peaks)
     decode = None
     if not args.no_decode:  # every rank: decode replicas, timed as the slowest rank
-        decode = run_decode(args, device, hbm, world)
+        decode = run_decode(args, device, hbm, world) if world > 1 else guarded(run_decode, args, device, hbm, world)
 
     extra = {}
     if world == 1 and not args.no_extra:
-        extra["prefill-1.3B"] = run_prefill_extra("prefill-1.3B", device, flush, peaks)
-        extra["sweeps"] = run_sweeps(device, flush, peaks)
-        extra["next_rows"] = run_next_rows(device, flush, peaks)
+        extra["prefill-1.3B"] = guarded(run_prefill_extra, "prefill-1.3B", device, flush, peaks)
+        extra["sweeps"] = guarded(run_sweeps, device, flush, peaks)
+        extra["next_rows"] = guarded(run_next_rows, device, flush, peaks)
 
     line = None
     if rank == 0:

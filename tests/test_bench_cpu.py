@@ -77,3 +77,10 @@ def test_reference_arm_other_ranks_do_no_work(monkeypatch):
     with redirect_stdout(buf):
         assert bench.run_reference(args, bench.WORKLOADS["prefill-370M"]) == 0
     assert buf.getvalue() == ""
+
+
+def test_an_extra_measurement_failure_is_reported_not_raised(capsys):
+    assert bench.guarded(lambda a, b: a * b, 3, 4) == 12
+    out = bench.guarded(lambda: [][1])
+    assert out == {"error": "IndexError: list index out of range"}
+    assert "IndexError" in capsys.readouterr().err
